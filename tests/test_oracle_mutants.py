@@ -1,0 +1,69 @@
+"""The pins must catch plausible mistakes in the oracle.
+
+Each case copies the oracle's C source, plants one mistake (a flipped sign, a
+dropped term, a wrong exponent, a wrong index or tie rule ...), builds the
+mutant on the CPU and runs the pin suite against it in a subprocess.  Every
+mutant must make the pin suite fail.  The real oracle is never modified.
+"""
+import concurrent.futures as cf
+import os
+import shutil
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "hqq_oracle.c")
+
+# (name, text in the source, replacement, expected number of occurrences)
+MUTANTS = [
+    ("z-update-sign", "float t = q[i] - (w[i] - we) * s;", "float t = q[i] + (w[i] - we) * s;", 1),
+    ("z-update-drops-We", "float t = q[i] - (w[i] - we) * s;", "float t = q[i] - (w[i] - 0.0f * we) * s;", 1),
+    ("shrink-exponent", "powf(a, p - 1.0f) / beta", "powf(a, p) / beta", 1),
+    ("shrink-beta-inverted", "powf(a, p - 1.0f) / beta", "powf(a, p - 1.0f) * beta", 1),
+    ("reconstruction-sign", "float wr = (qi - z) / s;", "float wr = (qi + z) / s;", 1),
+    ("l1-instead-of-lp", "acc += (double)powf(fabsf(d[i]), p);", "acc += (double)fabsf(d[i]);", 1),
+    ("tie-continues", "        if (e < best) {\n            best = e;\n            zbest = z;",
+     "        if (e <= best) {\n            best = e;\n            zbest = z;", 1),
+    ("keeps-last-z", "    res->zbest = zbest;", "    res->zbest = z;", 1),
+    ("beta-divides", "beta = beta * kappa;", "beta = beta / kappa;", 2),
+    ("z0-from-max", "*z_out = -mn * s;", "*z_out = -mx * s;", 1),
+    ("scale-uses-2^b", "s = (float)L / (mx - mn);", "s = (float)(L + 1) / (mx - mn);", 1),
+    ("floor-instead-of-round", "float q = nearbyintf(v);", "float q = floorf(v);", 1),
+    ("tensor-stop-first-group", "double e = G ? total / (double)(G * g) : 0.0;",
+     "double e = G ? gerr[0] / (double)g : 0.0;", 1),
+    ("zero8-scale", "sz = 255.0f / (zmx - zmn);", "sz = 254.0f / (zmx - zmn);", 1),
+    ("dequant-sign", "float v = (q - z) * from_f16(scale[j]);", "float v = (q + z) * from_f16(scale[j]);", 1),
+    ("pack-msb-first", "unsigned v = level << off; /* at most 8 + 7 bits */",
+     "unsigned v = (off + b <= 8 ? level << (8 - b - off) : level << off);", 1),
+]
+
+
+def _run_mutant(tmp, name, old, new, count):
+    src = open(SRC).read()
+    assert src.count(old) == count, f"{name}: pattern found {src.count(old)} times"
+    csrc = os.path.join(tmp, f"{name}.c")
+    lib = os.path.join(tmp, f"lib{name}.so")
+    open(csrc, "w").write(src.replace(old, new))
+    subprocess.run(["gcc", "-std=gnu11", "-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", "-w",
+                    csrc, "-o", lib, "-lm"], check=True)
+    env = dict(os.environ, HQQ_ORACLE_LIB=lib, OMP_NUM_THREADS="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return name, r.returncode, r.stdout[-400:]
+
+
+def test_every_mutant_is_caught():
+    tmp = tempfile.mkdtemp(prefix="hqq_mutants_")
+    try:
+        with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+            results = list(ex.map(lambda m: _run_mutant(tmp, *m), MUTANTS))
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
+    survivors = [(n, out) for n, rc, out in results if rc == 0]
+    assert not survivors, f"mutants not caught by the pins: {survivors}"
+    for n, rc, out in results:
+        assert rc == 1, f"{n}: pin run ended with code {rc} (expected test failures, not an error): {out}"

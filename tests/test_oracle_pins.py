@@ -1,0 +1,473 @@
+"""Pins of the CPU oracle to facts fixed outside the oracle itself.
+
+Each test checks the oracle against a hand value, a closed form, an
+invariant, a special case that reduces to a textbook rule, or brute force on
+a tiny input -- chosen so that a dropped term, a flipped sign, a wrong index
+or a transposed operand in the oracle fails at least one of them.
+
+Method source: techreport.ngo, "Weight-only quantization without the
+calibration tax" (Half-Quadratic Quantization of Large Machine Learning
+Models), sections "Outlier-aware optimization without gradients" and
+"Benchmark results" / "Llama-2".
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+NBITS = [1, 2, 3, 4, 8]
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _synth_f16(rows, cols, seed, std=0.02):
+    r = _rng(seed)
+    w = r.standard_normal((rows, cols)) * std
+    m = r.random((rows, cols)) < 1e-2
+    w = np.where(m, w * 10, w)
+    return w.astype(np.float16)
+
+
+def _lp_err(w, q, s, z, p):
+    """mean |w - (q - z)/s|^p in fp64 (the error measure the stop rule uses)."""
+    w = np.asarray(w, np.float64)
+    wr = (np.asarray(q, np.float64) - float(z)) / float(s)
+    return float(np.mean(np.abs(w - wr) ** p))
+
+
+# ---------------------------------------------------------------- shrink ----
+
+def _shrink_rows():
+    rows = []
+    with open(os.path.join(GOLDEN, "shrink_hand_values.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                x, p, b, ex = (float(t) for t in line.split())
+                rows.append((x, p, b, ex))
+    return rows
+
+
+@pytest.mark.parametrize("x,p,beta,expected", _shrink_rows())
+def test_shrink_hand_values(orc, x, p, beta, expected):
+    got = orc.shrink(x, p, beta)
+    assert got == pytest.approx(expected, rel=2e-6, abs=1e-7)
+
+
+def test_shrink_p1_is_soft_threshold(orc):
+    xs = _rng(1).standard_normal(2000) * 3
+    for beta in (0.5, 1.0, 2.0, 7.0):
+        for x in xs:
+            x = float(np.float32(x))
+            expect = math.copysign(max(abs(x) - 1.0 / beta, 0.0), x)
+            assert orc.shrink(x, 1.0, beta) == pytest.approx(expect, abs=2e-6)
+
+
+@pytest.mark.parametrize("p", [0.3, 0.7, 1.0, 1.4])
+@pytest.mark.parametrize("beta", [0.5, 1.0, 1.01 ** 19, 4.0])
+def test_shrink_zero_iff_below_threshold(orc, p, beta):
+    thr = beta ** (-1.0 / (2.0 - p))
+    for a in np.concatenate([np.linspace(0, 3 * thr, 301), thr * (1 + np.array([-1e-3, 1e-3]))]):
+        a = float(a)
+        for x in (a, -a):
+            got = orc.shrink(x, p, beta)
+            if a < thr * (1 - 1e-4):
+                assert got == 0.0
+            elif a > thr * (1 + 1e-4):
+                assert got != 0.0 and math.copysign(1, got) == math.copysign(1, x) and abs(got) < a
+
+
+def test_shrink_zero_input_is_zero_even_without_threshold(orc):
+    # |0|^(p-1) is infinite for p < 1 and 1/beta can be 0: shrink(0) must stay 0 (no NaN).
+    assert orc.shrink(0.0, 0.7, 1e30) == 0.0
+    assert orc.shrink(-0.0, 0.7, 1.0) == 0.0
+
+
+# ------------------------------------------------------------ worked groups --
+
+def _worked_rows():
+    rows = []
+    with open(os.path.join(GOLDEN, "worked_groups.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            cols = [c.strip() for c in line.split("|")]
+            rid = cols[0]
+            nb, p, beta, kappa = cols[1].split()
+            vals = np.array([float(t) for t in cols[2].split()], np.float32)
+            ev = lambda s: float(eval(s, {"__builtins__": {}}))  # closed-form expressions
+            rows.append(dict(id=rid, nbits=int(nb), p=float(p), beta=float(beta), kappa=float(kappa), w=vals,
+                             s=ev(cols[3]), z0=ev(cols[4]), codes=[int(t) for t in cols[5].split()],
+                             e0=ev(cols[6]), z1=ev(cols[7]), e1=ev(cols[8]), best_iter=int(cols[9]),
+                             zbest=ev(cols[10])))
+    return rows
+
+
+@pytest.mark.parametrize("row", _worked_rows(), ids=lambda r: r["id"])
+def test_worked_groups(orc, row):
+    s, z, e, b = orc.trace_group(row["w"], row["nbits"], row["p"], row["beta"], row["kappa"], iters=4)
+    assert s == row["s"]
+    assert z[0] == row["z0"]
+    assert list(orc.group_codes(row["w"], row["nbits"], s, z[0])) == row["codes"]
+    assert e[0] == pytest.approx(row["e0"], rel=1e-6, abs=1e-12)
+    assert z[1] == pytest.approx(row["z1"], rel=1e-7, abs=1e-9)
+    assert e[1] == pytest.approx(row["e1"], rel=1e-6, abs=1e-12)
+    # group mode through the full quantiser: kept iterate and zero-point
+    W = row["w"].astype(np.float16).reshape(1, -1)
+    assert np.array_equal(W.astype(np.float32), row["w"].reshape(1, -1))
+    out = orc.quantize(W, row["nbits"], W.shape[1], axis=1, p=row["p"], beta=row["beta"], kappa=row["kappa"],
+                       iters=20)
+    assert out["best_iter"][0] == row["best_iter"]
+    assert out["zero_f32"][0] == pytest.approx(row["zbest"], abs=1e-9)
+
+
+# ------------------------------------------------------------------ packing --
+
+@pytest.mark.parametrize("nbits", NBITS)
+@pytest.mark.parametrize("axis", [0, 1])
+def test_pack_roundtrip_exhaustive(orc, nbits, axis):
+    """Every level at every bit phase survives pack -> unpack; the byte layout is
+    the documented LSB-first stream (checked with numpy's own bit unpacking)."""
+    L = (1 << nbits) - 1
+    rows, cols = 8 * 3, 2 * (L + 1) if axis == 1 else 8
+    if axis == 0:
+        rows, cols = 8 * (L + 1), 3
+    r = _rng(nbits * 10 + axis)
+    levels = r.integers(0, L + 1, (rows, cols)).astype(np.uint8)
+    # make sure every level appears at every position modulo 8 along the stream
+    along = levels.reshape(-1) if axis == 1 else levels.T.reshape(-1)
+    along[: 8 * (L + 1)] = np.repeat(np.arange(L + 1), 8)[: along[: 8 * (L + 1)].size]
+    levels = along.reshape(rows, cols) if axis == 1 else along.reshape(cols, rows).T.copy()
+    packed = orc.pack_levels(levels, nbits, axis)
+    assert packed.size == rows * cols * nbits // 8
+    assert np.array_equal(orc.unpack_levels(packed, rows, cols, nbits, axis), levels)
+    # independent bit reader: numpy unpackbits, little bit order
+    if axis == 1:
+        bits = np.unpackbits(packed, bitorder="little").reshape(-1, nbits)
+        got = (bits * (1 << np.arange(nbits))).sum(1).reshape(rows, cols)
+    else:
+        colstreams = packed.reshape(rows * nbits // 8, cols).T  # [cols, bytes]
+        bits = np.unpackbits(np.ascontiguousarray(colstreams), axis=1, bitorder="little")
+        got = (bits.reshape(cols, rows, nbits) * (1 << np.arange(nbits))).sum(2).T
+    assert np.array_equal(got, levels)
+
+
+# ---------------------------------------------------- init / RTN properties --
+
+@pytest.mark.parametrize("nbits", NBITS)
+@pytest.mark.parametrize("g", [8, 64])
+def test_rtn_properties(orc, nbits, g):
+    """iters = 0 is plain min/max round-to-nearest: each group's min maps to code
+    0, its max to L, and every element is reconstructed within half a step."""
+    W = _synth_f16(16, 256, seed=nbits + g)
+    out = orc.quantize(W, nbits, g, axis=1, iters=0)
+    L = (1 << nbits) - 1
+    levels = orc.unpack_levels(out["packed"], 16, 256, nbits, 1).reshape(-1, g)
+    wg = W.astype(np.float64).reshape(-1, g)
+    for j in range(wg.shape[0]):
+        lo, hi = wg[j].argmin(), wg[j].argmax()
+        assert levels[j, lo] == 0
+        if L / (wg[j, hi] - wg[j, lo]) < 2e4 * (1 - 1e-6):  # scale cap (R1) not active
+            assert levels[j, hi] == L
+        else:
+            assert levels[j, hi] == round(float(np.float32(wg[j, hi] - wg[j, lo]) * np.float32(2e4)))
+    deq = orc.dequantize(out["packed"], out["scale"], out["zero"], None, 16, 256, nbits, g).astype(np.float64)
+    scale = out["scale"].astype(np.float64)[:, None]
+    z = out["zero"].astype(np.float64)[:, None]
+    err = np.abs(deq.reshape(-1, g) - wg)
+    # half a quantisation step, plus fp16 storage of scale, zero and the output
+    bound = scale * (0.5 + 1e-3 * (np.abs(z) + L)) + np.abs(wg) * 2.0 ** -10 + 1e-7
+    assert np.all(err <= bound)
+
+
+@pytest.mark.parametrize("nbits", NBITS)
+def test_one_iteration_equals_rtn(orc, nbits):
+    W = _synth_f16(32, 128, seed=7 + nbits)
+    a = orc.quantize(W, nbits, 32, iters=0)
+    b = orc.quantize(W, nbits, 32, iters=1)
+    for k in ("packed", "scale", "zero", "zero_f32"):
+        assert np.array_equal(a[k], b[k]), k
+    assert np.all(b["best_iter"] == 0)
+
+
+@pytest.mark.parametrize("nbits", [2, 4])
+def test_huge_beta_keeps_z0(orc, nbits):
+    """beta -> inf makes W_e = W - W_r, so z = mean(W_q - W_r*s) = z: z stays at
+    z0 (within fp32 rounding) and the codes equal round-to-nearest."""
+    W = _synth_f16(16, 256, seed=11)
+    rtn = orc.quantize(W, nbits, 64, iters=0)
+    out = orc.quantize(W, nbits, 64, beta=1e30, iters=20, stop_mode=orc.STOP_NONE)
+    z0, zb = rtn["zero_f32"], out["zero_f32"]
+    assert np.all(np.abs(zb - z0) <= 1e-5 * np.maximum(np.abs(z0), 1))
+    la = orc.unpack_levels(rtn["packed"], 16, 256, nbits, 1)
+    lb = orc.unpack_levels(out["packed"], 16, 256, nbits, 1)
+    assert np.mean(la != lb) <= 1e-3
+
+
+@pytest.mark.parametrize("c", [0.0, 0.015625, -0.75, 1e-4])
+@pytest.mark.parametrize("nbits", [1, 4, 8])
+def test_constant_group_fixed_point(orc, c, nbits):
+    """A constant group: codes 0, z = -c*s, zero error, and the second evaluation
+    repeats the first so the solver stops with best_iter 0."""
+    W = np.full((2, 64), c, np.float16)
+    out = orc.quantize(W, nbits, 64, iters=20)
+    cf = float(np.float16(c))
+    assert np.all(orc.unpack_levels(out["packed"], 2, 64, nbits, 1) == 0)
+    s = np.float32(2e4)
+    assert np.all(out["zero_f32"] == np.float32(-np.float32(cf) * s))
+    assert np.all(out["best_iter"] == 0)
+    assert np.all(out["best_err"] <= 1e-6)
+
+
+# ------------------------------------------------- the stop rule and best z --
+
+@pytest.mark.parametrize("nbits,g", [(1, 8), (2, 8), (2, 16), (3, 8), (4, 16)])
+def test_kept_error_between_optimum_and_rtn(orc, nbits, g):
+    """Brute force on tiny groups: the kept zero-point's lp error is no worse than
+    round-to-nearest (iterate 0) and no better than the best z on a fine scan."""
+    r = _rng(100 + nbits * g)
+    for t in range(40):
+        w = (r.standard_normal(g) * 0.02).astype(np.float16)
+        if t % 4 == 0:
+            w[r.integers(g)] *= 10  # an outlier
+        W = w.reshape(1, g)
+        out = orc.quantize(W, nbits, g, iters=20)
+        rtn = orc.quantize(W, nbits, g, iters=0)
+        w32 = w.astype(np.float32)
+        s, z, e, _ = orc.trace_group(w32, nbits, iters=1)
+        lv = orc.unpack_levels(out["packed"], 1, g, nbits, 1)[0]
+        lv0 = orc.unpack_levels(rtn["packed"], 1, g, nbits, 1)[0]
+        e_kept = _lp_err(w32, lv, s, out["zero_f32"][0], 0.7)
+        e_rtn = _lp_err(w32, lv0, s, rtn["zero_f32"][0], 0.7)
+        assert e_kept <= e_rtn * (1 + 1e-9) + 1e-15
+        # Exact global minimum over z: between code changes each term |.|^p is
+        # concave in z, so the minimum sits at a kink (some d_i = 0, z = k - w_i s)
+        # or next to a code change (z = k + 1/2 - w_i s); evaluate all of them.
+        L = (1 << nbits) - 1
+        ws = w32.astype(np.float64) * s
+        k = np.arange(L + 1, dtype=np.float64)
+        kinks = (k[:, None] - ws[None, :]).ravel()
+        brk = (k[:, None] + 0.5 - ws[None, :]).ravel()
+        zs = np.concatenate([kinks, brk - 1e-9, brk + 1e-9, np.linspace(-L - 1, 2 * L + 1, 2001)])
+        q = np.clip(np.rint(ws[None, :] + zs[:, None]), 0, L)
+        e_scan = np.mean(np.abs(w32[None, :] - (q - zs[:, None]) / s) ** 0.7, axis=1).min()
+        assert e_kept >= e_scan * (1 - 1e-6)
+
+
+def test_group_mode_stops_at_first_rise(orc):
+    """The kept iterate is the last one before the first non-improvement."""
+    W = _synth_f16(64, 256, seed=5)
+    out = orc.quantize(W, 4, 64, iters=20)
+    wg = W.astype(np.float32).reshape(-1, 64)
+    for j in range(wg.shape[0]):
+        s, z, e, _ = orc.trace_group(wg[j], 4, iters=20)
+        k = 0
+        while k + 1 < 20 and e[k + 1] < e[k]:
+            k += 1
+        assert out["best_iter"][j] == k
+        assert out["zero_f32"][j] == z[k]
+        assert out["best_err"][j] == np.float32(e[k])
+
+
+def test_no_stop_mode_keeps_global_best(orc):
+    W = _synth_f16(32, 128, seed=6)
+    out = orc.quantize(W, 3, 64, iters=20, stop_mode=orc.STOP_NONE)
+    grp = orc.quantize(W, 3, 64, iters=20)
+    wg = W.astype(np.float32).reshape(-1, 64)
+    for j in range(wg.shape[0]):
+        s, z, e, _ = orc.trace_group(wg[j], 3, iters=20)
+        k = int(np.argmin(e))  # first occurrence of the minimum
+        assert out["best_iter"][j] == k and out["zero_f32"][j] == z[k]
+        assert out["best_err"][j] <= grp["best_err"][j]
+
+
+def test_beta_schedule(orc):
+    w = _synth_f16(1, 64, seed=9).astype(np.float32)[0]
+    _, _, _, b = orc.trace_group(w, 4, beta=1.0, kappa=1.01, iters=20)
+    assert b[0] == 1.0
+    assert np.allclose(b, 1.01 ** np.arange(20), rtol=1e-6)
+    _, _, _, b2 = orc.trace_group(w, 4, beta=2.0, kappa=1.0, iters=5)
+    assert np.all(b2 == 2.0)
+
+
+def test_beta_schedule_changes_shrink_path(orc):
+    """Wide groups (|W - W_r| > 1) make the shrink active, so kappa matters."""
+    w = (_rng(3).standard_normal(64) * 40).astype(np.float32)
+    _, za, _, _ = orc.trace_group(w, 1, kappa=1.0, iters=6)
+    _, zb, _, _ = orc.trace_group(w, 1, kappa=1.5, iters=6)
+    assert za[1] == zb[1]  # first update uses beta0 in both
+    assert not np.allclose(za[2:], zb[2:])
+
+
+# ------------------------------------------------------ the z update (LS) --
+
+@pytest.mark.parametrize("beta", [1.0, 50.0])
+def test_z_update_is_least_squares_minimiser(orc, beta):
+    """Sub-problem 2: the average minimises sum (W_q - (W - W_e)*s - z)^2."""
+    r = _rng(21)
+    for _ in range(20):
+        w = (r.standard_normal(32) * 3).astype(np.float32)
+        s = np.float32(1.5)
+        q = np.clip(np.rint(w * s + 4), 0, 15).astype(np.float32)
+        d = (w - (q - 4) / s).astype(np.float32)
+        z = orc.update_zero(w, q, d, s, 0.7, beta)
+        we = np.array([orc.shrink(float(x), 0.7, beta) for x in d], np.float64)
+        t = q.astype(np.float64) - (w.astype(np.float64) - we) * float(s)
+        zs = np.linspace(t.min(), t.max(), 200001)
+        obj = ((t[None, :] - zs[:, None]) ** 2).sum(1)
+        zbf = zs[obj.argmin()]
+        assert abs(z - zbf) <= (t.max() - t.min()) / 200000 + 1e-5
+        if beta > 1:  # threshold beta^(-1/(2-p)) < 0.05 here: the shrink is active and must move z
+            assert abs(z - np.mean(q - w * s)) > 1e-3
+
+
+# ------------------------------------------------------------- invariances --
+
+def test_translation_equivariance(orc):
+    """Adding c to a group leaves the codes and the error unchanged and shifts z
+    by -c*s (exactly representable shifts; fp32 rounding only)."""
+    r = _rng(31)
+    base = np.round(r.standard_normal((8, 64)) * 64) / 1024  # multiples of 2^-10
+    for c in (0.25, -0.5, 0.125):
+        W0, W1 = base.astype(np.float16), (base + c).astype(np.float16)
+        assert np.array_equal(W1.astype(np.float64) - W0.astype(np.float64), np.full(base.shape, c))
+        a, b = orc.quantize(W0, 4, 64), orc.quantize(W1, 4, 64)
+        la = orc.unpack_levels(a["packed"], 8, 64, 4, 1)
+        lb = orc.unpack_levels(b["packed"], 8, 64, 4, 1)
+        assert np.mean(la != lb) <= 2 / la.size
+        s = 1.0 / a["scale"].astype(np.float64)
+        assert np.allclose(b["zero_f32"], a["zero_f32"] - c * s, rtol=2e-3, atol=2e-3)
+        assert np.allclose(a["best_err"], b["best_err"], rtol=1e-3)
+
+
+def test_permutation_within_group(orc):
+    W = _synth_f16(4, 64, seed=41)
+    perm = _rng(4).permutation(64)
+    a, b = orc.quantize(W, 3, 64), orc.quantize(W[:, perm], 3, 64)
+    la = orc.unpack_levels(a["packed"], 4, 64, 3, 1)
+    lb = orc.unpack_levels(b["packed"], 4, 64, 3, 1)
+    assert np.array_equal(la[:, perm], lb)
+    assert np.array_equal(a["best_iter"], b["best_iter"])
+    assert np.allclose(a["zero_f32"], b["zero_f32"], rtol=1e-6)
+
+
+def test_groups_are_independent(orc):
+    W = _synth_f16(16, 128, seed=42)
+    perm = _rng(5).permutation(16)
+    a, b = orc.quantize(W, 2, 32), orc.quantize(W[perm], 2, 32)
+    ga = a["zero_f32"].reshape(16, 4)[perm]
+    assert np.array_equal(ga, b["zero_f32"].reshape(16, 4))
+    la = orc.unpack_levels(a["packed"], 16, 128, 2, 1)[perm]
+    assert np.array_equal(la, orc.unpack_levels(b["packed"], 16, 128, 2, 1))
+
+
+@pytest.mark.parametrize("nbits", [3, 4])
+def test_axis0_is_axis1_of_transpose(orc, nbits):
+    W = _synth_f16(128, 48, seed=43)
+    a = orc.quantize(W, nbits, 32, axis=0)
+    b = orc.quantize(np.ascontiguousarray(W.T), nbits, 32, axis=1)
+    # scale/zero: axis 0 is [rows/g, cols]; axis 1 of W^T is [cols, rows/g]
+    assert np.array_equal(a["zero_f32"].reshape(4, 48), b["zero_f32"].reshape(48, 4).T)
+    assert np.array_equal(a["scale"].reshape(4, 48), b["scale"].reshape(48, 4).T)
+    la = orc.unpack_levels(a["packed"], 128, 48, nbits, 0)
+    lb = orc.unpack_levels(b["packed"], 48, 128, nbits, 1)
+    assert np.array_equal(la, lb.T)
+    # packed axis-0 bytes are the transpose of the axis-1 bytes of W^T
+    assert np.array_equal(a["packed"].reshape(128 * nbits // 8, 48), b["packed"].reshape(48, 128 * nbits // 8).T)
+
+
+def test_bf16_and_f16_agree_on_shared_values(orc):
+    r = _rng(44)
+    vals = np.clip(np.round(r.standard_normal((8, 64)) * 64), -255, 255) / 4096  # <= 8 significant bits: exact in both
+    f16 = vals.astype(np.float16)
+    bf = (vals.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(f16.astype(np.float32), (bf.astype(np.uint32) << 16).view(np.float32))
+    a = orc.quantize(f16, 4, 64)
+    b = orc.quantize(bf, 4, 64, dtype=orc.BF16)
+    for k in ("packed", "scale", "zero", "zero_f32", "best_iter"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+# ------------------------------------------------------------- tensor mode --
+
+def test_tensor_mode_single_group_equals_group_mode(orc):
+    for seed in range(6):
+        W = _synth_f16(1, 64, seed=50 + seed)
+        a = orc.quantize(W, 3, 64, stop_mode=orc.STOP_GROUP)
+        b = orc.quantize(W, 3, 64, stop_mode=orc.STOP_TENSOR)
+        for k in ("packed", "zero_f32", "best_iter"):
+            assert np.array_equal(a[k], b[k]), k
+
+
+def test_tensor_mode_identical_groups_equals_group_mode(orc):
+    row = _synth_f16(1, 64, seed=60)
+    W = np.repeat(row, 8, axis=0)
+    a = orc.quantize(W, 4, 64, stop_mode=orc.STOP_GROUP)
+    b = orc.quantize(W, 4, 64, stop_mode=orc.STOP_TENSOR)
+    assert np.array_equal(a["zero_f32"], b["zero_f32"])
+    assert np.array_equal(a["best_iter"], b["best_iter"])
+
+
+def test_tensor_mode_uses_tensor_mean(orc):
+    """The tensor stop follows the mean of all per-group errors."""
+    W = _synth_f16(16, 256, seed=61)
+    out = orc.quantize(W, 2, 16, stop_mode=orc.STOP_TENSOR, iters=20)
+    wg = W.astype(np.float32).reshape(-1, 16)
+    traces = [orc.trace_group(wg[j], 2, iters=20) for j in range(wg.shape[0])]
+    E = np.mean([t[2] for t in traces], axis=0)
+    k = 0
+    while k + 1 < 20 and E[k + 1] < E[k]:
+        k += 1
+    assert np.all(out["best_iter"] == k)
+    assert np.array_equal(out["zero_f32"], np.array([t[1][k] for t in traces], np.float32))
+
+
+# ------------------------------------------------------------- zero 8-bit --
+
+@pytest.mark.parametrize("nbits", [2, 4])
+def test_zero_8bit_roundtrip(orc, nbits):
+    W = _synth_f16(64, 256, seed=70)
+    out = orc.quantize(W, nbits, 64, zero_nbits=8)
+    z = out["zero_f32"].astype(np.float64)
+    inv_sz, zz = out["zero_meta"].astype(np.float64)
+    zdeq = (out["zero"].astype(np.float64) - zz) * inv_sz
+    span = z.max() - z.min()
+    assert out["zero"].min() == 0 and out["zero"].max() == 255
+    assert np.all(np.abs(zdeq - z) <= span / 510 * (1 + 1e-5) + 1e-6 * np.abs(z).max())
+    # the codes are those of the fp32 zero-point (zero quantisation does not re-solve W_q)
+    ref = orc.quantize(W, nbits, 64, zero_nbits=16)
+    assert np.array_equal(ref["packed"], out["packed"])
+
+
+def test_zero_8bit_all_equal(orc):
+    W = np.repeat(_synth_f16(1, 64, seed=71), 4, axis=0)
+    out = orc.quantize(W, 4, 64, zero_nbits=8)
+    inv_sz, zz = out["zero_meta"].astype(np.float64)
+    zdeq = (out["zero"].astype(np.float64) - zz) * inv_sz
+    assert np.all(out["zero"] == 0)
+    assert np.allclose(zdeq, out["zero_f32"], rtol=1e-6)
+
+
+def test_dequant_with_8bit_zero_close_to_16bit(orc):
+    W = _synth_f16(32, 256, seed=72)
+    a = orc.quantize(W, 4, 64, zero_nbits=16)
+    b = orc.quantize(W, 4, 64, zero_nbits=8)
+    da = orc.dequantize(a["packed"], a["scale"], a["zero"], None, 32, 256, 4, 64).astype(np.float64)
+    db = orc.dequantize(b["packed"], b["scale"], b["zero"], b["zero_meta"], 32, 256, 4, 64,
+                        zero_nbits=8).astype(np.float64)
+    span = a["zero_f32"].max() - a["zero_f32"].min()
+    step = np.repeat(a["scale"].astype(np.float64), 64).reshape(32, 256)
+    assert np.all(np.abs(da - db) <= step * (span / 510 + 0.01) + 1e-6)
+
+
+def test_dequant_bf16_output(orc):
+    W = _synth_f16(8, 64, seed=73)
+    a = orc.quantize(W, 4, 64)
+    h = orc.dequantize(a["packed"], a["scale"], a["zero"], None, 8, 64, 4, 64, out_dtype=orc.F16)
+    b = orc.dequantize(a["packed"], a["scale"], a["zero"], None, 8, 64, 4, 64, out_dtype=orc.BF16)
+    bf = (b.astype(np.uint32) << 16).view(np.float32)
+    assert np.allclose(bf, h.astype(np.float32), rtol=2 ** -8, atol=1e-6)
