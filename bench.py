@@ -1,0 +1,361 @@
+"""Benchmark: HQQ quantisation throughput on Llama-2-7B MLP shapes.
+
+One step = the whole quantiser over one batch: the MLP weights of one decoder
+layer (gate/up 11008x4096, down 4096x11008, bf16, synthetic Llama-2 weight
+statistics) quantised at every (nbits, group_size) of the sweep
+(8/128, 4/64, 3/64, 2/16, 1/16), each with stop_mode=group and
+stop_mode=tensor: 30 hqq_quantize calls, 1.353 G weights.
+
+value     = weights quantised / device time (CUDA events), inputs resident in HBM.
+e2e       = the same through the C ABI with host buffers: every step copies the
+            step's inputs from pinned host memory and reads all outputs back.
+roofline  = the dominant kernel (solve_tensor): bound by the MUFU pipe that
+            evaluates |r|^p (two ops per element and iteration).
+cpu_baseline / --impl reference = the CPU oracle on a bounded sample.
+
+Multi-GPU (torchrun): each rank quantises its own layer's MLP (weak scaling,
+no data-path collective); time = max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from calibration_free_weight_b200 import synth  # noqa: E402
+
+METRIC = "HQQ quantize Gweights/s and achieved HBM GB/s (% of B200 roofline) vs CPU oracle"
+UNIT = "Gweights/s"
+SWEEP = [(8, 128), (4, 64), (3, 64), (2, 16), (1, 16)]
+MODES = [0, 1]  # stop_mode group, tensor
+MATS = [("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008)]
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+SMS = 148
+MUFU_PER_CLK_PER_SM = 16
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("sm_max_mhz", 1965.0)), "measured"
+    except Exception:
+        return 6650.0, 1965.0, "fallback"
+
+
+def algorithmic_bytes(rows, cols, nbits, g, zero_nbits=16):
+    """One read of W (2 B/weight) + packed codes + fp16 scale + zero."""
+    n = rows * cols
+    G = n // g
+    return 2 * n + n * nbits // 8 + 2 * G + (2 if zero_nbits == 16 else 1) * G
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def make_inputs(layer):
+    return {name: synth.weight(r, c, seed=synth.seed_for(layer, name), dtype=torch.bfloat16)
+            for name, r, c in MATS}
+
+
+def plan():
+    """The 30 calls of one step, ordered so consecutive calls use different matrices."""
+    calls = []
+    for nbits, g in SWEEP:
+        for mode in MODES:
+            for name, r, c in MATS:
+                calls.append((name, r, c, nbits, g, mode))
+    return calls
+
+
+# ----------------------------------------------------------------- oracle ---
+
+def oracle_sample_rate(layer, budget_s=12.0, nthreads=0):
+    """Time the CPU oracle, as it stands, on a bounded sample of the step's work:
+    the first `rows` output rows of every matrix at every setting and mode.
+    Returns (weights/s, threads used, sample description)."""
+    import oracle
+    oracle.lib()
+    nth = nthreads or (os.cpu_count() or 1)
+    ins = make_inputs(layer)
+    rows = 16
+    while True:
+        t0 = time.perf_counter()
+        n = 0
+        for name, r, c, nbits, g, mode in plan():
+            W = ins[name][:rows if name != "down" else max(1, rows * 4096 // 11008)].contiguous()
+            Wb = W.view(torch.int16).numpy().view(np.uint16)
+            oracle.quantize(Wb, nbits, g, 1, 0.7, 1.0, 1.01, 20, mode, 16, dtype=oracle.BF16, nthreads=nth)
+            n += W.numel()
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 4 or rows >= 2048:
+            break
+        rows *= 4
+    desc = (f"first {rows} rows of gate/up (and the same element count of down) at all 10 settings/modes, "
+            f"{n / 1e6:.2f} M weights per pass, bf16, OpenMP over groups")
+    return n / dt, nth, desc, n, dt
+
+
+# ------------------------------------------------------------------- main ---
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    per_step = []
+    desc, nth, total_n = "", 0, 0
+    for i in range(args.warmup + args.steps):
+        rate, nth, desc, n, dt = oracle_sample_rate(0, budget_s=args.ref_budget)
+        if i >= args.warmup:
+            per_step.append((n, dt))
+    n = sum(a for a, _ in per_step)
+    t = sum(b for _, b in per_step)
+    value = n / t / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": config_dict(world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nth, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def config_dict(world):
+    return {"workload": "llama2-7b-mlp-sweep", "model": "Llama-2-7B MLP shapes (synthetic weights)",
+            "matrices": "gate 11008x4096, up 11008x4096, down 4096x11008 (out x in), bf16",
+            "settings": "nbits/group 8/128 4/64 3/64 2/16 1/16, axis 1, p 0.7, beta 1, kappa 1.01, 20 iters",
+            "stop_modes": ["group", "tensor"], "zero": "fp16", "calls_per_step": len(plan()),
+            "weights_per_step": sum(r * c for _, r, c, _, _, _ in plan()),
+            "global_batch": world, "seq_len": None, "parallelism": f"replicas{world}",
+            "l2": "inputs 270 MB > 126 MB L2; consecutive calls use different matrices"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--ref-budget", type=float, default=8.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    if args.impl == "reference":
+        # CPU oracle only: rank 0 times it, other ranks exit without work
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup()
+
+    from calibration_free_weight_b200 import hqq
+    hbm_peak, sm_max, peak_kind = peaks()
+    layer = rank
+    ins_cpu = make_inputs(layer)
+    ins = {k: v.cuda() for k, v in ins_cpu.items()}
+    calls = plan()
+    stream = torch.cuda.current_stream()
+    outs = {}
+    for name, r, c, nbits, g, mode in calls:
+        outs[(name, nbits, g, mode)] = hqq.alloc_outputs(r, c, nbits, g, 1, mode, 16)
+
+    # algorithmic work per call: element-evaluations from the kept iterates (untimed pass)
+    evals = {}
+    for name, r, c, nbits, g, mode in calls:
+        q = hqq.quantize(ins[name], nbits, g, stop_mode=mode, debug=True)
+        bi = q["best_iter"].to(torch.int64)
+        e = torch.where(bi >= 19, torch.full_like(bi, 20), bi + 2) if mode == 0 else \
+            torch.full_like(bi, min(int(bi[0]) + 2, 20))
+        evals[(name, nbits, g, mode)] = int(e.sum().item()) * g
+        del q
+    torch.cuda.synchronize()
+
+    def one_step(record=None):
+        for name, r, c, nbits, g, mode in calls:
+            o = outs[(name, nbits, g, mode)]
+            if record is not None:
+                record.append((mode, torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                               (name, nbits, g, mode)))
+                record[-1][1].record(stream)
+            rc = hqq.hqq_quantize(ins[name], r, c, hqq.HQQ_BF16, nbits, g, 1, 0.7, 1.0, 1.01, 20, mode, 16,
+                                  o["packed"], o["scale"], o["zero"], None, o["workspace"], o["workspace"].numel())
+            if rc != hqq.HQQ_OK:
+                raise RuntimeError(hqq.hqq_status_string(rc))
+            if record is not None:
+                record[-1][2].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    barrier(world)
+    rec = []
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        barrier(world)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            one_step(rec)
+        ev1.record(stream)
+        barrier(world)
+    for o in outs.values():
+        st = hqq.hqq_get_status(o["workspace"])
+        if st != hqq.HQQ_OK:
+            raise RuntimeError(hqq.hqq_status_string(st))
+    dev_ms = ev0.elapsed_time(ev1)
+    dev_ms = max_over_ranks(dev_ms, world)
+    w_step = sum(r * c for _, r, c, _, _, _ in calls)
+    value = world * w_step * args.steps / (dev_ms / 1e3) / 1e9
+
+    # per-launch durations by kernel family
+    fam = {0: [], 1: []}
+    for mode, a, b, key in rec:
+        fam[mode].append((a.elapsed_time(b), key))
+    tot = {m: sum(t for t, _ in v) for m, v in fam.items()}
+    dom = max(tot, key=tot.get)
+    dom_name = "solve_tensor_kernel" if dom == 1 else "solve_group_kernel"
+    n_l = len(fam[dom])
+    avg_ms = tot[dom] / n_l
+    mufu_ops = sum(2 * evals[key] for _, key in fam[dom]) / n_l  # per launch
+    mufu_peak = SMS * MUFU_PER_CLK_PER_SM * sm_max * 1e6 / 1e9  # Gop/s
+    achieved = mufu_ops / (avg_ms / 1e3) / 1e9
+    # HBM view of the same launches (the metric's second half)
+    bytes_dom = sum(algorithmic_bytes(*[(r, c) for n_, r, c in MATS if n_ == key[0]][0], key[1], key[2])
+                    for _, key in fam[dom]) / n_l
+    gb_dom = bytes_dom / (avg_ms / 1e3) / 1e9
+    bytes_step = sum(algorithmic_bytes(r, c, nb, g) for _, r, c, nb, g, _ in calls)
+    hbm_step = bytes_step * args.steps / (dev_ms / 1e3) / 1e9 * world
+    grp = fam[0]
+    g_ms = sum(t for t, _ in grp) / max(1, len(grp))
+    g_bytes = sum(algorithmic_bytes(*[(r, c) for n_, r, c in MATS if n_ == key[0]][0], key[1], key[2])
+                  for _, key in grp) / max(1, len(grp))
+    g_w = sum([(r * c) for _, key in grp for n_, r, c in MATS if n_ == key[0]]) / max(1, len(grp))
+
+    # end to end through the C ABI with host buffers
+    pinned = {k: v.pin_memory() for k, v in ins_cpu.items()}
+    host_out = {key: {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in o.items()
+                      if k in ("packed", "scale", "zero")} for key, o in outs.items()}
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = sum(v.numel() * v.element_size() for o in host_out.values() for v in o.values())
+
+    def e2e_step():
+        for k, v in pinned.items():
+            ins[k].copy_(v, non_blocking=True)
+        one_step()
+        for key, o in outs.items():
+            for k, v in host_out[key].items():
+                v.copy_(o[k], non_blocking=True)
+
+    e2e_step()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * w_step * args.steps / (e2e_ms / 1e3) / 1e9
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dev_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_dict(world),
+            "roofline": {"bound": "alu", "kernel": dom_name, "achieved": achieved, "peak": mufu_peak,
+                         "unit": "Gop/s (MUFU lg2+ex2)", "frac": achieved / mufu_peak, "traffic": None,
+                         "peak_basis": f"{SMS} SMs x {MUFU_PER_CLK_PER_SM} MUFU/clk x {sm_max:.0f} MHz",
+                         "avg_launch_ms": avg_ms, "hbm_gbs": gb_dom, "hbm_frac": gb_dom / hbm_peak},
+            "hbm": {"achieved_gbs_step": hbm_step, "peak_gbs": hbm_peak, "peak_kind": peak_kind,
+                    "frac_step": hbm_step / hbm_peak,
+                    "group_mode": {"avg_launch_ms": g_ms, "gbs": g_bytes / (g_ms / 1e3) / 1e9,
+                                   "frac": g_bytes / (g_ms / 1e3) / 1e9 / hbm_peak,
+                                   "gweights_s": g_w / (g_ms / 1e3) / 1e9}},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": len(calls) * args.steps,
+            "clocks": clk.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, nth, desc, _, _ = oracle_sample_rate(0, budget_s=args.ref_budget)
+        line["cpu_baseline"] = {"value": rate / 1e9, "unit": UNIT, "cores": nth, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

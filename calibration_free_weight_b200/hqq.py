@@ -1,0 +1,167 @@
+"""Thin ctypes binding of libhqq_b200.so (include/hqq.h), same names as the C ABI.
+
+Argument marshalling only: every step of the quantiser runs in the library's
+CUDA kernels.  torch provides device memory and streams.  If the library is
+missing the import fails loudly; there is no CPU fallback.
+"""
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhqq_b200.so")
+
+HQQ_OK, HQQ_ERR_INVALID_ARG, HQQ_ERR_SHAPE, HQQ_ERR_DTYPE, HQQ_ERR_ALIGN = 0, 1, 2, 3, 4
+HQQ_ERR_CUDA, HQQ_ERR_TIMEOUT, HQQ_ERR_COOP_UNSUPPORTED, HQQ_ERR_WORKSPACE = 5, 6, 7, 8
+HQQ_F16, HQQ_BF16 = 0, 1
+HQQ_STOP_GROUP, HQQ_STOP_TENSOR, HQQ_STOP_NONE = 0, 1, 2
+
+EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_quantize", "hqq_dequantize",
+            "hqq_get_status", "hqq_status_string", "hqq_debug_set_barrier")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with calibration_free_weight_b200/build.py "
+                          "(there is no CPU fallback)")
+    L = C.CDLL(LIB_PATH)
+    P, i64, i32, f32, sz = C.c_void_p, C.c_int64, C.c_int, C.c_float, C.c_size_t
+    L.hqq_packed_bytes.restype = sz
+    L.hqq_packed_bytes.argtypes = [i64, i64, i32, i32, i32]
+    L.hqq_num_groups.restype = i64
+    L.hqq_num_groups.argtypes = [i64, i64, i32, i32]
+    L.hqq_workspace_bytes.restype = sz
+    L.hqq_workspace_bytes.argtypes = [i64, i64, i32, i32, i32, i32]
+    L.hqq_quantize.restype = i32
+    L.hqq_quantize.argtypes = [P, i64, i64, i32, i32, i32, i32, f32, f32, f32, i32, i32, i32,
+                               P, P, P, P, P, sz, P, P, P, P]
+    L.hqq_dequantize.restype = i32
+    L.hqq_dequantize.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, i32, i32, P, P]
+    L.hqq_get_status.restype = i32
+    L.hqq_get_status.argtypes = [P, P]
+    L.hqq_status_string.restype = C.c_char_p
+    L.hqq_status_string.argtypes = [i32]
+    L.hqq_debug_set_barrier.restype = None
+    L.hqq_debug_set_barrier.argtypes = [i32, C.c_uint64]
+    return L
+
+
+lib = _load()
+
+
+class HQQError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {hqq_status_string(code)} (code {code})")
+        self.code = code
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+# -------------------------------------------------------- C ABI, same names --
+
+def hqq_packed_bytes(rows, cols, nbits, group_size, axis=1):
+    return lib.hqq_packed_bytes(rows, cols, nbits, group_size, axis)
+
+
+def hqq_num_groups(rows, cols, group_size, axis=1):
+    return lib.hqq_num_groups(rows, cols, group_size, axis)
+
+
+def hqq_workspace_bytes(rows, cols, group_size, axis=1, stop_mode=HQQ_STOP_GROUP, zero_nbits=16):
+    return lib.hqq_workspace_bytes(rows, cols, group_size, axis, stop_mode, zero_nbits)
+
+
+def hqq_quantize(W, rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode, zero_nbits,
+                 W_q_packed, scale, zero, zero_meta, workspace, workspace_bytes, debug_best_iter=None,
+                 debug_best_err=None, debug_zero_f32=None, stream=None):
+    """Raw call: tensors are passed by device address; returns the status code."""
+    return lib.hqq_quantize(_ptr(W), rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
+                            zero_nbits, _ptr(W_q_packed), _ptr(scale), _ptr(zero), _ptr(zero_meta), _ptr(workspace),
+                            workspace_bytes, _ptr(debug_best_iter), _ptr(debug_best_err), _ptr(debug_zero_f32),
+                            _stream(stream))
+
+
+def hqq_dequantize(W_q_packed, scale, zero, zero_meta, rows, cols, nbits, group_size, axis, zero_nbits, out_dtype,
+                   W_out, stream=None):
+    return lib.hqq_dequantize(_ptr(W_q_packed), _ptr(scale), _ptr(zero), _ptr(zero_meta), rows, cols, nbits,
+                              group_size, axis, zero_nbits, out_dtype, _ptr(W_out), _stream(stream))
+
+
+def hqq_get_status(workspace, stream=None):
+    return lib.hqq_get_status(_ptr(workspace), _stream(stream))
+
+
+def hqq_status_string(code):
+    return lib.hqq_status_string(code).decode()
+
+
+def hqq_debug_set_barrier(skip_block=-1, timeout_ns=0):
+    lib.hqq_debug_set_barrier(skip_block, timeout_ns)
+
+
+# ------------------------------------------------------ allocating helpers --
+
+_DT = {torch.float16: HQQ_F16, torch.bfloat16: HQQ_BF16}
+
+
+def alloc_outputs(rows, cols, nbits, group_size, axis=1, stop_mode=HQQ_STOP_GROUP, zero_nbits=16, debug=False,
+                  device="cuda"):
+    """torch-allocated output and workspace buffers for one hqq_quantize call."""
+    G = hqq_num_groups(rows, cols, group_size, axis)
+    if G < 0:
+        raise HQQError(HQQ_ERR_SHAPE, "hqq_num_groups")
+    nb = hqq_packed_bytes(rows, cols, nbits, group_size, axis)
+    wsb = hqq_workspace_bytes(rows, cols, group_size, axis, stop_mode, zero_nbits)
+    u8 = torch.uint8
+    out = dict(
+        packed=torch.empty(max(nb, 16), dtype=u8, device=device)[:nb],
+        scale=torch.empty(G, dtype=torch.float16, device=device),
+        zero=torch.empty(G, dtype=torch.float16 if zero_nbits == 16 else u8, device=device),
+        zero_meta=torch.empty(2, dtype=torch.float32, device=device) if zero_nbits == 8 else None,
+        workspace=torch.empty(wsb, dtype=u8, device=device),
+    )
+    if debug:
+        out.update(best_iter=torch.empty(G, dtype=torch.int32, device=device),
+                   best_err=torch.empty(G, dtype=torch.float32, device=device),
+                   zero_f32=torch.empty(G, dtype=torch.float32, device=device))
+    return out
+
+
+def quantize(W, nbits=4, group_size=64, axis=1, p=0.7, beta=1.0, kappa=1.01, iters=20, stop_mode=HQQ_STOP_GROUP,
+             zero_nbits=16, debug=False, out=None, stream=None):
+    """Quantise a CUDA fp16/bf16 [rows, cols] tensor; returns the output dict."""
+    if W.dtype not in _DT or not W.is_cuda or W.dim() != 2 or not W.is_contiguous():
+        raise HQQError(HQQ_ERR_INVALID_ARG, "quantize expects a contiguous 2-D CUDA fp16/bf16 tensor")
+    rows, cols = W.shape
+    if out is None:
+        out = alloc_outputs(rows, cols, nbits, group_size, axis, stop_mode, zero_nbits, debug, W.device)
+    rc = hqq_quantize(W, rows, cols, _DT[W.dtype], nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
+                      zero_nbits, out["packed"], out["scale"], out["zero"], out["zero_meta"], out["workspace"],
+                      out["workspace"].numel(), out.get("best_iter"), out.get("best_err"), out.get("zero_f32"),
+                      stream)
+    if rc != HQQ_OK:
+        raise HQQError(rc, "hqq_quantize")
+    return out
+
+
+def dequantize(q, rows, cols, nbits, group_size, axis=1, zero_nbits=16, out_dtype=torch.float16, out=None,
+               stream=None):
+    """Dequantise the outputs of quantize() into a [rows, cols] tensor."""
+    if out is None:
+        out = torch.empty(rows, cols, dtype=out_dtype, device=q["scale"].device)
+    rc = hqq_dequantize(q["packed"], q["scale"], q["zero"], q["zero_meta"], rows, cols, nbits, group_size, axis,
+                        zero_nbits, _DT[out_dtype], out, stream)
+    if rc != HQQ_OK:
+        raise HQQError(rc, "hqq_dequantize")
+    return out

@@ -1,0 +1,161 @@
+/*
+ * hqq.h -- C ABI of the B200 (sm_100a) Half-Quadratic Quantization library.
+ *
+ * The library quantises an fp16/bf16 weight matrix to 8/4/3/2/1-bit codes with
+ * the HQQ zero-point solver, with no calibration data.  Method: techreport.ngo,
+ * "Weight-only quantization without the calibration tax" (Half-Quadratic
+ * Quantization of Large Machine Learning Models):
+ *   - section "Outlier-aware optimization without gradients": lp loss with
+ *     p < 1, half-quadratic split with an auxiliary variable W_e, scale s fixed,
+ *     zero-point z optimised; sub-problem 1 = generalised soft-thresholding,
+ *     sub-problem 2 = average over the quantisation group axis; ~20 closed-form
+ *     iterations;
+ *   - section "Benchmark results" / "Llama-2": p = 0.7, beta = 1,
+ *     kappa = 1.01, 20 iterations, early stopping, zero-point quantised to 8
+ *     bit without extra grouping.
+ * The interface nouns (nbits, group_size, axis -> W_q, scale, zero, and a
+ * dequantize() for inspection) follow "HQQ - Half-Quadratic Quantization"
+ * (skill4agent.com), section "Core concepts" ("Quantization configuration",
+ * "HQQLinear layer").
+ *
+ * Per group of g weights w (L = 2^nbits - 1), all arithmetic in fp32:
+ *   s  = min(L / (max w - min w), 2e4)   (2e4 when max == min)
+ *   z0 = -min(w) * s
+ *   iteration k (k = 0 .. iters-1), beta_0 = beta, beta_{k+1} = kappa * beta_k:
+ *     W_q = clamp(round_half_even(w*s + z_k), 0, L);  W_r = (W_q - z_k) / s
+ *     e_k = mean |w - W_r|^p
+ *     stop rule (below); then
+ *     W_e = sign(w - W_r) * max(|w - W_r| - |w - W_r|^(p-1) / beta_k, 0)
+ *     z_{k+1} = mean(W_q - (w - W_e) * s)
+ *   stop rule: keep going while e_k is strictly below every earlier error; the
+ *   kept zero-point z* is the iterate with the lowest error so far.
+ *     HQQ_STOP_GROUP : each group stops at its own first non-improvement;
+ *     HQQ_STOP_TENSOR: all groups stop together at the first non-improvement of
+ *                      the tensor-wide mean error (summed in fp64);
+ *     HQQ_STOP_NONE  : all `iters` iterations, z* = lowest-error iterate.
+ *   Output codes: clamp(round(w*s + z*), 0, L).  scale = fp16(1/s).
+ *   iters = 0 gives plain min/max round-to-nearest (z* = z0).
+ *
+ * Layout.  W is row-major [rows, cols] (rows = output features).
+ *   axis = 1: group j = the g contiguous elements [j*g, (j+1)*g) of the
+ *             flattened matrix (g must divide cols); scale/zero are
+ *             [rows, cols/g] row-major.
+ *   axis = 0: group (rb, c) = rows rb*g .. rb*g+g-1 of column c (g must divide
+ *             rows); scale/zero are [rows/g, cols] row-major.
+ *   Packed codes (LSB-first bit streams, nbits bits per code):
+ *   axis = 1: one stream over the flattened matrix; element e occupies bits
+ *             e*nbits .. e*nbits+nbits-1, bit k of byte B is stream bit 8B+k.
+ *             Size rows*cols*nbits/8 bytes (3-bit: 8 codes per 3 bytes).
+ *   axis = 0: one stream per column running down the rows; byte R of column c
+ *             is stored at R*cols + c (packed shape [rows*nbits/8, cols]).
+ *   This layout is this library's own; it is not claimed compatible with any
+ *   other HQQ format.
+ *
+ * Conventions for every call:
+ *   - All buffers are caller-owned device memory (cudaMalloc, torch, ...).
+ *     The library never allocates or frees.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = legacy default stream).  Argument errors are detected on the host
+ *     and returned before anything is launched; no output is touched then.
+ *   - Inputs must be finite.
+ */
+#ifndef HQQ_B200_H
+#define HQQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HQQ_OK = 0,
+    HQQ_ERR_INVALID_ARG = 1,      /* bad nbits/p/beta/kappa/iters/mode, NULL pointer, host pointer */
+    HQQ_ERR_SHAPE = 2,            /* group_size not a power of two in [8,1024] or not dividing the group axis */
+    HQQ_ERR_DTYPE = 3,            /* dtype not HQQ_F16 / HQQ_BF16 */
+    HQQ_ERR_ALIGN = 4,            /* a buffer is not aligned as documented */
+    HQQ_ERR_CUDA = 5,             /* a CUDA runtime call failed (launch, attribute query) */
+    HQQ_ERR_TIMEOUT = 6,          /* device-side: a bounded wait gave up (tensor-mode grid barrier) */
+    HQQ_ERR_COOP_UNSUPPORTED = 7, /* device cannot run the cooperative tensor-mode kernel */
+    HQQ_ERR_WORKSPACE = 8         /* workspace missing or smaller than hqq_workspace_bytes() */
+} hqq_status;
+
+typedef enum { HQQ_F16 = 0, HQQ_BF16 = 1 } hqq_dtype;
+
+typedef enum { HQQ_STOP_GROUP = 0, HQQ_STOP_TENSOR = 1, HQQ_STOP_NONE = 2 } hqq_stop_mode;
+
+/* Bytes of the packed code buffer: rows*cols*nbits/8.  0 for invalid args. */
+size_t hqq_packed_bytes(int64_t rows, int64_t cols, int nbits, int group_size, int axis);
+
+/* Number of groups G = rows*cols/group_size.  -1 for invalid args. */
+int64_t hqq_num_groups(int64_t rows, int64_t cols, int group_size, int axis);
+
+/* Bytes of device workspace hqq_quantize needs for this problem (always > 0;
+ * holds the device status word, the tensor-mode state and the fp32 zeros of
+ * the 8-bit zero path).  0 for invalid args. */
+size_t hqq_workspace_bytes(int64_t rows, int64_t cols, int group_size, int axis, int stop_mode, int zero_nbits);
+
+/*
+ * Quantise W.
+ *   W            device, dtype [rows, cols] row-major, 16-byte aligned.
+ *   p, beta, kappa, iters
+ *                0 < p < 2, beta > 0, kappa >= 1, 0 <= iters <= 1000.
+ *   stop_mode    hqq_stop_mode.
+ *   zero_nbits   16: zero is fp16[G];  8: zero is uint8[G] and zero_meta is
+ *                fp32[2] = (1/sz, zz), one round-to-nearest quantiser for the
+ *                whole tensor: sz = min(255/(max z* - min z*), 2e4) (2e4 when
+ *                all equal), zz = -min(z*)*sz, zq = clamp(round(z*sz + zz), 0,
+ *                255); the dequantised zero is (zq - zz) * (1/sz).  The codes
+ *                W_q use the unquantised fp32 z*.
+ *   W_q_packed   device uint8[hqq_packed_bytes], 16-byte aligned.
+ *   scale        device fp16[G] (= 1/s), 2-byte aligned.
+ *   zero         device fp16[G] or uint8[G], see zero_nbits.
+ *   zero_meta    device fp32[2] when zero_nbits == 8, else ignored (may be NULL).
+ *   workspace    device, >= hqq_workspace_bytes(...), 256-byte aligned;
+ *                contents need no initialisation and are overwritten.
+ *   debug_best_iter  optional device int32[G]: index k of the kept iterate.
+ *   debug_best_err   optional device fp32[G]: mean |w - W_r|^p of the kept
+ *                    zero-point (lg2/ex2 hardware approximations, ~1e-6 rel).
+ *   debug_zero_f32   optional device fp32[G]: z* before storage.
+ *   stream       cudaStream_t as void*.
+ * Returns HQQ_OK or an error code; device-side errors (HQQ_ERR_TIMEOUT) are
+ * reported by hqq_get_status on the same workspace.  Calls that share a
+ * workspace must not run concurrently.
+ */
+int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis,
+                 float p, float beta, float kappa, int iters, int stop_mode, int zero_nbits,
+                 void* W_q_packed, void* scale, void* zero, void* zero_meta,
+                 void* workspace, size_t workspace_bytes,
+                 int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32,
+                 void* stream);
+
+/*
+ * Dequantise for inspection: W_out = (W_q - zero) * scale computed in fp32 and
+ * rounded (to nearest even) to out_dtype; with zero_nbits == 8 the zero is
+ * first rebuilt as (zq - zz) * (1/sz) from zero_meta.  Buffers as in
+ * hqq_quantize; W_out is device out_dtype [rows, cols], 16-byte aligned.
+ */
+int hqq_dequantize(const void* W_q_packed, const void* scale, const void* zero, const void* zero_meta,
+                   int64_t rows, int64_t cols, int nbits, int group_size, int axis, int zero_nbits,
+                   int out_dtype, void* W_out, void* stream);
+
+/* Synchronise `stream` and return the device status word held in `workspace`
+ * by the last hqq_quantize on it (HQQ_OK or HQQ_ERR_TIMEOUT), or
+ * HQQ_ERR_CUDA if the synchronisation or copy fails. */
+int hqq_get_status(const void* workspace, void* stream);
+
+/* Static English description of a status code. */
+const char* hqq_status_string(int status);
+
+/* Test hook: the next tensor-mode launches use `timeout_ns` for their grid
+ * barrier wait (0 restores the default of 4 s) and, when skip_block >= 0, that
+ * block does not arrive at the first barrier, so the others give up after the
+ * timeout and report HQQ_ERR_TIMEOUT.  Never hangs: every wait is bounded. */
+void hqq_debug_set_barrier(int skip_block, uint64_t timeout_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQQ_B200_H */

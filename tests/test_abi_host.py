@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+function include/hqq.h declares, answers the size queries, and rejects bad
+arguments on the host before anything is launched."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def hq():
+    from calibration_free_weight_b200 import build
+    build.build()
+    from calibration_free_weight_b200 import hqq
+    return hqq
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "hqq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hqq_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(hq):
+    names = _declared()
+    assert "hqq_quantize" in names and "hqq_dequantize" in names
+    for n in names:
+        assert hasattr(hq.lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", hq.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (hqq_\w+)", out))
+    assert set(names) <= exported
+    assert set(hq.EXPORTED) == set(names)
+
+
+@pytest.mark.parametrize("rows,cols,nbits,g,axis", [(4096, 4096, 4, 64, 1), (11008, 4096, 3, 64, 1),
+                                                    (128, 48, 2, 16, 0), (8, 24, 1, 8, 1), (0, 64, 4, 64, 1)])
+def test_size_queries(hq, rows, cols, nbits, g, axis):
+    assert hq.hqq_packed_bytes(rows, cols, nbits, g, axis) == rows * cols * nbits // 8
+    assert hq.hqq_num_groups(rows, cols, g, axis) == rows * cols // g
+    for stop in (0, 1, 2):
+        for zb in (8, 16):
+            ws = hq.hqq_workspace_bytes(rows, cols, g, axis, stop, zb)
+            G = rows * cols // g
+            assert ws >= 256
+            if zb == 8:
+                assert ws >= 4 * G
+            if stop == 1:
+                assert ws >= 40 * G
+
+
+@pytest.mark.parametrize("args", [(64, 100, 4, 64, 1), (100, 64, 4, 64, 0), (64, 64, 4, 48, 1), (64, 64, 4, 4, 1),
+                                  (64, 64, 4, 2048, 1), (-1, 64, 4, 64, 1), (64, 64, 4, 64, 2)])
+def test_size_queries_reject_bad_shapes(hq, args):
+    rows, cols, nbits, g, axis = args
+    assert hq.hqq_packed_bytes(rows, cols, nbits, g, axis) == 0
+    assert hq.hqq_num_groups(rows, cols, g, axis) == -1
+
+
+def test_bad_nbits_rejected(hq):
+    for b in (0, 5, 6, 7, 9, 16):
+        assert hq.hqq_packed_bytes(64, 64, b, 64, 1) == 0
+
+
+def _call(hq, **kw):
+    a = dict(W=None, rows=64, cols=64, dtype=0, nbits=4, g=64, axis=1, p=0.7, beta=1.0, kappa=1.01, iters=20,
+             stop=0, zb=16, ws_bytes=0)
+    a.update(kw)
+    return hq.lib.hqq_quantize(None, a["rows"], a["cols"], a["dtype"], a["nbits"], a["g"], a["axis"], a["p"],
+                               a["beta"], a["kappa"], a["iters"], a["stop"], a["zb"], None, None, None, None, None,
+                               a["ws_bytes"], None, None, None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=2), 3), (dict(nbits=5), 1), (dict(g=48), 2), (dict(cols=96), 2), (dict(axis=0, rows=96), 2),
+    (dict(axis=3), 1), (dict(p=0.0), 1), (dict(p=2.0), 1), (dict(p=float("nan")), 1), (dict(beta=0.0), 1),
+    (dict(beta=float("inf")), 1), (dict(kappa=0.99), 1), (dict(iters=-1), 1), (dict(iters=1001), 1),
+    (dict(stop=3), 1), (dict(zb=4), 1), (dict(), 8),
+])
+def test_quantize_rejects_on_host(hq, kw, code):
+    assert _call(hq, **kw) == code
+
+
+def test_dequantize_rejects_on_host(hq):
+    L = hq.lib
+    assert L.hqq_dequantize(None, None, None, None, 64, 64, 4, 64, 1, 16, 7, None, None) == 3
+    assert L.hqq_dequantize(None, None, None, None, 64, 64, 5, 64, 1, 16, 0, None, None) == 1
+    assert L.hqq_dequantize(None, None, None, None, 64, 96, 4, 64, 1, 16, 0, None, None) == 2
+    assert L.hqq_dequantize(None, None, None, None, 64, 64, 4, 64, 1, 12, 0, None, None) == 1
+    assert L.hqq_dequantize(None, None, None, None, 0, 64, 4, 64, 1, 16, 0, None, None) == 0
+
+
+def test_status_strings(hq):
+    for code in range(9):
+        s = hq.hqq_status_string(code)
+        assert s and s != "unknown status"
+    assert hq.hqq_status_string(99) == "unknown status"
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    """Importing the binding with the library missing raises; nothing falls back to the CPU."""
+    import shutil
+    import sys
+    pkg = tmp_path / "calibration_free_weight_b200"
+    shutil.copytree(os.path.join(ROOT, "calibration_free_weight_b200"), pkg,
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    code = "import calibration_free_weight_b200.hqq"
+    r = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True)
+    assert r.returncode != 0 and "missing" in r.stderr

@@ -1,0 +1,244 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Inputs are seeded synthetic weights with the pages' weight statistics
+(0.02 * N(0,1), 0.1% outliers x10) plus degenerate cases.  Small shapes span
+several tiles and a ragged tail; full Llama-2 shapes are checked on sampled
+groups in the launch configuration the benchmark uses.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from calibration_free_weight_b200 import synth
+
+from . import parity_check as pc
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from calibration_free_weight_b200 import hqq
+    return hqq
+
+
+def _params(nbits, g, axis=1, p=0.7, beta=1.0, kappa=1.01, iters=20, stop=0, zb=16):
+    return dict(nbits=nbits, group_size=g, axis=axis, p=p, beta=beta, kappa=kappa, iters=iters, stop_mode=stop,
+                zero_nbits=zb)
+
+
+def _run(hq, W_cpu, prm, check_recon=True):
+    W = W_cpu.cuda()
+    out = hq.quantize(W, prm["nbits"], prm["group_size"], prm["axis"], prm["p"], prm["beta"], prm["kappa"],
+                      prm["iters"], prm["stop_mode"], prm["zero_nbits"], debug=True)
+    torch.cuda.synchronize()
+    st = hq.hqq_get_status(out["workspace"])
+    assert st == hq.HQQ_OK, hq.hqq_status_string(st)
+    gpu = pc.gpu_to_numpy(out)
+    Wo, dt = pc.w_for_oracle(W_cpu)
+    orc = oracle.quantize(Wo, prm["nbits"], prm["group_size"], prm["axis"], prm["p"], prm["beta"], prm["kappa"],
+                          prm["iters"], prm["stop_mode"], prm["zero_nbits"], dtype=dt)
+    rep = pc.check(W_cpu, prm, gpu, orc)
+    if prm["zero_nbits"] == 8:
+        pc.check_zero8(gpu, orc)
+    if check_recon:
+        rows, cols = W_cpu.shape
+        for out_dt in (torch.float16, torch.bfloat16):
+            deq = hq.dequantize(out, rows, cols, prm["nbits"], prm["group_size"], prm["axis"], prm["zero_nbits"],
+                                out_dt)
+            d = deq.cpu()
+            d = d.numpy() if out_dt == torch.float16 else d.view(torch.int16).numpy().view(np.uint16)
+            pc.check_reconstruction(W_cpu, prm, gpu, d, orc)
+    return rep, gpu, orc
+
+
+# ------------------------------------------------------------- group mode --
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("g", [8, 16, 32, 64, 128, 256, 512, 1024])
+def test_group_mode_axis1(hq, dtype, nbits, g):
+    rows = max(8, 40960 // 512)  # several tiles for small g, ragged tails for large g
+    W = synth.weight(rows + 3, 1024, seed=nbits * 100 + g, dtype=dtype)
+    _run(hq, W, _params(nbits, g), check_recon=(g in (16, 64)))
+
+
+@pytest.mark.parametrize("rows,cols,g", [(37, 192, 64), (1000, 320, 64), (777, 64, 16), (5, 1024, 1024),
+                                         (301, 1536, 512), (2049, 40, 8)])
+def test_ragged_tiles(hq, rows, cols, g):
+    W = synth.weight(rows, cols, seed=rows + cols, dtype=torch.float16)
+    _run(hq, W, _params(4, g))
+
+
+@pytest.mark.parametrize("rows,cols,g", [(256, 200, 64), (128, 37, 32), (1024, 520, 16), (2048, 24, 1024),
+                                         (64, 1000, 8)])
+@pytest.mark.parametrize("nbits", [3, 4])
+def test_axis0(hq, rows, cols, g, nbits):
+    W = synth.weight(rows, cols, seed=7 * rows + cols, dtype=torch.bfloat16)
+    _run(hq, W, _params(nbits, g, axis=0))
+
+
+@pytest.mark.parametrize("iters", [0, 1, 2, 5, 50])
+@pytest.mark.parametrize("stop", [0, 1, 2])
+def test_iteration_counts_and_modes(hq, iters, stop):
+    W = synth.weight(300, 512, seed=iters * 3 + stop, dtype=torch.float16)
+    _run(hq, W, _params(2, 32, iters=iters, stop=stop))
+
+
+@pytest.mark.parametrize("p,beta,kappa", [(0.5, 1.0, 1.01), (1.2, 1.0, 1.01), (0.7, 10.0, 1.05), (0.7, 1.0, 1.0)])
+def test_solver_parameters(hq, p, beta, kappa):
+    W = synth.weight(256, 512, seed=int(p * 100), dtype=torch.float16)
+    for stop in (0, 1):
+        _run(hq, W, _params(4, 64, p=p, beta=beta, kappa=kappa, stop=stop), check_recon=False)
+
+
+@pytest.mark.parametrize("stop", [0, 1, 2])
+def test_shrink_active(hq, stop):
+    """Large weights make |W - W_r| exceed the shrink threshold: W_e != 0 path."""
+    W = (synth.weight(128, 256, seed=5, dtype=torch.float32) * 200.0).to(torch.float16)
+    for nbits in (1, 2):
+        _run(hq, W, _params(nbits, 64, beta=4.0, stop=stop), check_recon=False)
+
+
+def test_constant_and_zero_groups(hq):
+    W = synth.weight(64, 512, seed=9, dtype=torch.float16)
+    W[0:8] = 0.0
+    W[8:16, :] = 0.015625
+    W[16, :256] = -0.5
+    for zb in (16, 8):
+        _run(hq, W, _params(4, 64, zb=zb))
+
+
+@pytest.mark.parametrize("stop", [0, 1])
+@pytest.mark.parametrize("nbits,g", [(4, 128), (2, 16)])
+def test_zero_8bit(hq, stop, nbits, g):
+    W = synth.weight(512, 1024, seed=11, dtype=torch.float16)
+    _run(hq, W, _params(nbits, g, stop=stop, zb=8))
+
+
+def test_empty_input(hq):
+    W = torch.empty(0, 64, dtype=torch.float16, device="cuda")
+    out = hq.quantize(W, 4, 64, zero_nbits=8)
+    torch.cuda.synchronize()
+    meta = out["zero_meta"].cpu().numpy()
+    assert meta[0] == np.float32(1.0 / np.float32(2e4)) and meta[1] == 0.0
+    out = hq.quantize(W, 4, 64, zero_nbits=16)
+    torch.cuda.synchronize()
+    assert hq.hqq_get_status(out["workspace"]) == hq.HQQ_OK
+
+
+def test_repeated_calls_reuse_outputs(hq):
+    """The same buffers and workspace serve consecutive calls (workspace needs no
+    initialisation by the caller)."""
+    W = synth.weight(512, 512, seed=12, dtype=torch.float16)
+    prm = _params(4, 64, stop=1, zb=8)
+    out = hq.quantize(W.cuda(), 4, 64, stop_mode=1, zero_nbits=8, debug=True)
+    first = pc.gpu_to_numpy(out)
+    out = hq.quantize(W.cuda(), 4, 64, stop_mode=1, zero_nbits=8, debug=True, out=out)
+    second = pc.gpu_to_numpy(out)
+    for k in ("packed", "scale", "zero", "zero_meta", "best_iter", "zero_f32"):
+        assert np.array_equal(first[k], second[k]), k
+    pc.check(W, prm, second)
+
+
+# ---------------------------------------------------------- error paths ----
+
+def test_host_pointer_rejected(hq):
+    W = synth.weight(64, 64, seed=1, dtype=torch.float16)  # CPU tensor
+    out = hq.alloc_outputs(64, 64, 4, 64)
+    rc = hq.hqq_quantize(W, 64, 64, hq.HQQ_F16, 4, 64, 1, 0.7, 1.0, 1.01, 20, 0, 16, out["packed"], out["scale"],
+                         out["zero"], None, out["workspace"], out["workspace"].numel())
+    assert rc == hq.HQQ_ERR_INVALID_ARG
+
+
+def test_small_workspace_rejected(hq):
+    W = synth.weight(64, 64, seed=1, dtype=torch.float16).cuda()
+    out = hq.alloc_outputs(64, 64, 4, 64, stop_mode=1)
+    rc = hq.hqq_quantize(W, 64, 64, hq.HQQ_F16, 4, 64, 1, 0.7, 1.0, 1.01, 20, 1, 16, out["packed"], out["scale"],
+                         out["zero"], None, out["workspace"], out["workspace"].numel() - 1)
+    assert rc == hq.HQQ_ERR_WORKSPACE
+
+
+def test_misaligned_input_rejected(hq):
+    W = synth.weight(64, 72, seed=1, dtype=torch.float16).cuda().reshape(-1)[8:8 + 64 * 64].view(64, 64)
+    base = synth.weight(64, 65, seed=1, dtype=torch.float16).cuda().reshape(-1)[1:1 + 64 * 64].view(64, 64)
+    out = hq.alloc_outputs(64, 64, 4, 64)
+    rc = hq.hqq_quantize(base, 64, 64, hq.HQQ_F16, 4, 64, 1, 0.7, 1.0, 1.01, 20, 0, 16, out["packed"], out["scale"],
+                         out["zero"], None, out["workspace"], out["workspace"].numel())
+    assert rc == hq.HQQ_ERR_ALIGN
+    rc = hq.hqq_quantize(W, 64, 64, hq.HQQ_F16, 4, 64, 1, 0.7, 1.0, 1.01, 20, 0, 16, out["packed"], out["scale"],
+                         out["zero"], None, out["workspace"], out["workspace"].numel())
+    assert rc == hq.HQQ_OK
+
+
+def test_tensor_barrier_timeout_is_reported(hq):
+    """A block that never arrives at the grid barrier: the other blocks give up
+    after the (short) bounded wait, the status word says so, and the context
+    stays usable."""
+    W = synth.weight(4096, 1024, seed=3, dtype=torch.float16).cuda()
+    try:
+        hq.hqq_debug_set_barrier(skip_block=0, timeout_ns=200_000_000)
+        out = hq.quantize(W, 4, 64, stop_mode=hq.HQQ_STOP_TENSOR)
+        assert hq.hqq_get_status(out["workspace"]) == hq.HQQ_ERR_TIMEOUT
+    finally:
+        hq.hqq_debug_set_barrier(-1, 0)
+    out = hq.quantize(W, 4, 64, stop_mode=hq.HQQ_STOP_TENSOR)
+    assert hq.hqq_get_status(out["workspace"]) == hq.HQQ_OK
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------- full sizes, sampled -----
+
+def _sampled(hq, W_cpu, prm, n=6000, seed=0):
+    rows, cols = W_cpu.shape
+    G = rows * cols // prm["group_size"]
+    W = W_cpu.cuda()
+    out = hq.quantize(W, prm["nbits"], prm["group_size"], prm["axis"], prm["p"], prm["beta"], prm["kappa"],
+                      prm["iters"], prm["stop_mode"], prm["zero_nbits"], debug=True)
+    torch.cuda.synchronize()
+    assert hq.hqq_get_status(out["workspace"]) == hq.HQQ_OK
+    gpu = pc.gpu_to_numpy(out)
+    ids = np.sort(np.random.default_rng(seed).choice(G, size=min(n, G), replace=False))
+    ids[0], ids[-1] = 0, G - 1  # first and last group always
+    rep = pc.check(W_cpu, prm, gpu, sample=np.unique(ids))
+    return rep, gpu
+
+
+def test_llama_square_4096_fp16_b4_g64(hq):
+    W = synth.weight(4096, 4096, seed=0, dtype=torch.float16)
+    rep, gpu = _sampled(hq, W, _params(4, 64), n=20000)
+    assert rep["tie_groups"] <= 3
+
+
+@pytest.mark.parametrize("nbits,g", [(8, 128), (4, 64), (3, 64), (2, 16), (1, 16)])
+@pytest.mark.parametrize("shape", [(11008, 4096), (4096, 11008)])
+def test_llama_mlp_group_mode_sampled(hq, nbits, g, shape):
+    W = synth.weight(*shape, seed=1000 * 0 + (4 if shape[0] == 11008 else 6), dtype=torch.bfloat16)
+    _sampled(hq, W, _params(nbits, g), n=4000, seed=nbits)
+
+
+@pytest.mark.parametrize("nbits,g", [(8, 128), (4, 64), (3, 64), (2, 16), (1, 16)])
+def test_llama_mlp_tensor_mode_groups_follow_kept_iterate(hq, nbits, g):
+    """Full-size tensor mode: every sampled group's z* and codes are the oracle's
+    iterate at the GPU's tensor-wide index."""
+    W_cpu = synth.weight(11008, 4096, seed=4, dtype=torch.bfloat16)
+    prm = _params(nbits, g, stop=1)
+    out = hq.quantize(W_cpu.cuda(), nbits, g, stop_mode=1, debug=True)
+    torch.cuda.synchronize()
+    assert hq.hqq_get_status(out["workspace"]) == hq.HQQ_OK
+    gpu = pc.gpu_to_numpy(out)
+    G = W_cpu.numel() // g
+    bi = gpu["best_iter"]
+    assert np.all(bi == bi[0])
+    k = int(bi[0])
+    Wf = pc.w_float(W_cpu)
+    gl = oracle.unpack_levels(gpu["packed"], *W_cpu.shape, nbits, 1)
+    for j in np.random.default_rng(1).choice(G, 500, replace=False):
+        w = pc.group_values(Wf, j, g, 1)
+        s, zt, et, _ = oracle.trace_group(w, nbits, iters=20)
+        assert abs(gpu["zero_f32"][j] - zt[k]) <= pc.Z_TOL * max(abs(zt[k]), 1)
+        lv = oracle.group_codes(w, nbits, s, zt[k])
+        assert np.count_nonzero(pc.group_levels(gl, j, g, 1).astype(int) - lv) <= 1
