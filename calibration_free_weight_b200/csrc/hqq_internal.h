@@ -24,9 +24,9 @@ constexpr uint32_t kStatusTimeout = 6;
 //   partial min/max          float2[kMaxPartials]
 //   tensor error partials    double[2][kMaxPartials]
 //   zbest                    float[G]            (zero_nbits == 8)
-//   tensor state             s f32[G], z0 f32[G], sws f64[G], Z f32[3][G], E f32[3][G]
+//   tensor state             s f32[G], 1/s f32[G], z0 f32[G], sws f64[G], Z f32[3][G], E f32[3][G]
 struct WorkspaceLayout {
-    size_t header, minmax, tparts, zbest, t_s, t_z0, t_sws, t_z, t_e, total;
+    size_t header, minmax, tparts, zbest, t_s, t_is, t_z0, t_sws, t_z, t_e, total;
 };
 WorkspaceLayout workspace_layout(int64_t G, int stop_mode, int zero_nbits);
 

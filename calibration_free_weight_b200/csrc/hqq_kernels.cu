@@ -145,6 +145,7 @@ struct KParams {
     double* tparts;
     float* zbest_ws;
     float* t_s;
+    float* t_is;
     float* t_z0;
     double* t_sws;
     float* t_z;
@@ -265,19 +266,20 @@ __device__ __forceinline__ void init_item(const KParams& k, const uint16_t* sg, 
 }
 
 struct Eval {
-    float err;    // sum over the group of |w*s + z - W_q|^p  (= s^p * sum |w - W_r|^p)
-    float sq;     // sum of W_q (exact: integers < 2^24)
-    float sterm;  // sum of W_q - (w - W_e)*s, only when the shrink may be active
-    bool sp;      // the shrink may be active for this group
+    float err;     // sum over the group of |w - W_r|^p
+    float sq;      // sum of W_q (exact: integers < 2^24)
+    double sws_e;  // sum of fl((w - W_e)*s), only when the shrink may be active
+    bool sp;       // the shrink may be active for this group
 };
 
 // Evaluate zero-point z on the item's pieces and reduce over the group's lanes.
-// Whole warps only.  The shrink W_e is exactly zero unless some |w - W_r|
-// exceeds beta^(-1/(2-p)) (= thr); |w - W_r|*s <= max(0.5, |z - z0|) up to
-// rounding, so groups below the bound skip the per-element proximal step.
+// Whole warps only.  W_r = (W_q - z) * (1/s) in fp32, the dequantiser's form.
+// The shrink W_e is exactly zero unless some |w - W_r| exceeds
+// beta^(-1/(2-p)) (= thr); |w - W_r|*s <= max(0.5, |z - z0|) up to rounding,
+// so groups below that bound skip the per-element proximal step.
 template <int DT>
-__device__ __forceinline__ Eval eval_item(const KParams& k, const uint16_t* sg, int part, bool valid, float s, float z,
-                                          float z0, float beta, float thr) {
+__device__ __forceinline__ Eval eval_item(const KParams& k, const uint16_t* sg, int part, bool valid, float s,
+                                          float inv_s, float z, float z0, float beta, float thr) {
     Eval e;
     float err = 0.0f, sq = 0.0f;
     const bool sp = valid && (fmaxf(0.5f, fabsf(z - z0)) + 1e-3f * (1.0f + k.Lf + fabsf(z)) >= 0.99f * thr * s);
@@ -289,18 +291,18 @@ __device__ __forceinline__ Eval eval_item(const KParams& k, const uint16_t* sg, 
             for (int i = 0; i < 8; ++i) {
                 float v;
                 const float q = quant(w[i], s, z, k.Lf, &v);
-                const float r = __fsub_rn(v, q);
-                err += pow_pos(fabsf(r), k.p);
+                const float d = __fsub_rn(w[i], __fmul_rn(__fsub_rn(q, z), inv_s));
+                err += pow_pos(fabsf(d), k.p);
                 sq += q;
             }
         }
     }
     e.err = seg_sum(err, k.P);
     e.sq = seg_sum(sq, k.P);
-    e.sterm = 0.0f;
+    e.sws_e = 0.0;
     e.sp = sp;
     if (__any_sync(kFull, sp)) {
-        float st = 0.0f;
+        double st = 0.0;
         if (sp) {
             for (int n = 0; n < k.NP; ++n) {
                 float w[8];
@@ -309,25 +311,27 @@ __device__ __forceinline__ Eval eval_item(const KParams& k, const uint16_t* sg, 
                 for (int i = 0; i < 8; ++i) {
                     float v;
                     const float q = quant(w[i], s, z, k.Lf, &v);
-                    const float d = __fsub_rn(w[i], __fdiv_rn(__fsub_rn(q, z), s));
+                    const float d = __fsub_rn(w[i], __fmul_rn(__fsub_rn(q, z), inv_s));
                     const float a = fabsf(d);
                     float we = 0.0f;
                     if (a != 0.0f) {
                         const float t = __fsub_rn(a, __fdiv_rn(pow_pos(a, k.p - 1.0f), beta));
                         if (t > 0.0f) we = copysignf(t, d);
                     }
-                    st += __fsub_rn(q, __fmul_rn(__fsub_rn(w[i], we), s));
+                    st += static_cast<double>(__fmul_rn(__fsub_rn(w[i], we), s));
                 }
             }
         }
-        e.sterm = seg_sum(st, k.P);
+        e.sws_e = seg_sum_d(st, k.P);
     }
     return e;
 }
 
+// z_{k+1} = (sum W_q - sum fl((w - W_e)*s)) / g with fp64 sums; sws is the
+// precomputed sum of fl(w*s) used when W_e is zero for the whole group.
 __device__ __forceinline__ float next_zero(const Eval& e, double sws, int g) {
-    if (e.sp) return __fmul_rn(e.sterm, 1.0f / static_cast<float>(g));  // g is a power of two: exact scaling
-    return static_cast<float>((static_cast<double>(e.sq) - sws) / static_cast<double>(g));
+    const double t = e.sp ? e.sws_e : sws;
+    return static_cast<float>((static_cast<double>(e.sq) - t) / static_cast<double>(g));
 }
 
 // beta^(-1/(2-p)): below this |w - W_r| the proximal step returns exactly 0.
@@ -466,7 +470,7 @@ __device__ __forceinline__ int compact(const uint8_t* active, uint16_t* list, in
 
 struct GroupSmem {
     uint16_t* data;
-    float *s, *z, *zb, *z0, *be;
+    float *s, *is, *z, *zb, *z0, *be;
     double* sws;
     int* bi;
     uint8_t* active;
@@ -482,6 +486,8 @@ __device__ __forceinline__ GroupSmem carve_group_smem(unsigned char* base, const
     m.sws = reinterpret_cast<double*>(base + off);
     off += TG * 8;
     m.s = reinterpret_cast<float*>(base + off);
+    off += TG * 4;
+    m.is = reinterpret_cast<float*>(base + off);
     off += TG * 4;
     m.z = reinterpret_cast<float*>(base + off);
     off += TG * 4;
@@ -526,6 +532,7 @@ __global__ void __launch_bounds__(kThreads) solve_group_kernel(const KParams k) 
             init_item<DT>(k, m.data + lt * k.g, part, valid, &s, &z0, &sws);
             if (valid && part == 0) {
                 m.s[lt] = s;
+                m.is[lt] = __fdiv_rn(1.0f, s);
                 m.z0[lt] = z0;
                 m.z[lt] = z0;
                 m.zb[lt] = z0;
@@ -549,8 +556,8 @@ __global__ void __launch_bounds__(kThreads) solve_group_kernel(const KParams k) 
                 const bool valid = item < items;
                 const int lt = valid ? m.list[item >> k.logP] : 0;
                 const int part = item & (k.P - 1);
-                const float s = m.s[lt], z = m.z[lt], z0 = m.z0[lt];
-                const Eval e = eval_item<DT>(k, m.data + lt * k.g, part, valid, s, z, z0, beta, thr);
+                const float s = m.s[lt], is = m.is[lt], z = m.z[lt], z0 = m.z0[lt];
+                const Eval e = eval_item<DT>(k, m.data + lt * k.g, part, valid, s, is, z, z0, beta, thr);
                 if (valid && part == 0) {
                     bool alive = true;
                     if (e.err < m.be[lt]) {
@@ -574,9 +581,8 @@ __global__ void __launch_bounds__(kThreads) solve_group_kernel(const KParams k) 
         // final codes and group outputs
         pack_tile<DT, AXIS>(k, t, m.data, m.s, m.zb);
         for (int lt = tid; lt < t.ntg; lt += kThreads) {
-            const float s = m.s[lt];
-            const float err_mean = m.be[lt] * pow_pos(s, -k.p) / static_cast<float>(k.g);
-            store_group(k, group_index<AXIS>(k, t, lt), s, m.zb[lt], m.bi[lt], err_mean, &zmin, &zmax);
+            const float err_mean = m.be[lt] / static_cast<float>(k.g);
+            store_group(k, group_index<AXIS>(k, t, lt), m.s[lt], m.zb[lt], m.bi[lt], err_mean, &zmin, &zmax);
         }
         __syncthreads();
     }
@@ -665,6 +671,7 @@ __global__ void __launch_bounds__(kThreads) solve_tensor_kernel(const KParams k)
             if (valid && part == 0) {
                 const int64_t j = group_index<AXIS>(k, t, lt);
                 k.t_s[j] = s;
+                k.t_is[j] = __fdiv_rn(1.0f, s);
                 k.t_z0[j] = z0;
                 k.t_sws[j] = sws;
                 Z0[j] = z0;
@@ -696,12 +703,12 @@ __global__ void __launch_bounds__(kThreads) solve_tensor_kernel(const KParams k)
                 const int part = item & (k.P - 1);
                 const int64_t j = group_index<AXIS>(k, t, valid ? lt : 0);
                 const float s = valid ? k.t_s[j] : 1.0f;
+                const float is = valid ? k.t_is[j] : 1.0f;
                 const float z = valid ? Zc[j] : 0.0f;
                 const float z0 = valid ? k.t_z0[j] : 0.0f;
-                const Eval e = eval_item<DT>(k, sdata + lt * k.g, part, valid, s, z, z0, beta, thr);
+                const Eval e = eval_item<DT>(k, sdata + lt * k.g, part, valid, s, is, z, z0, beta, thr);
                 if (valid && part == 0) {
-                    const float spow = pow_pos(s, -k.p);
-                    const float gerr = e.err * spow;  // sum over the group of |w - W_r|^p
+                    const float gerr = e.err;  // sum over the group of |w - W_r|^p
                     acc += static_cast<double>(gerr);
                     Zn[j] = next_zero(e, k.t_sws[j], k.g);
                     if (Ec) Ec[j] = gerr / static_cast<float>(k.g);
@@ -902,7 +909,7 @@ DevInfo device_info() {
 }
 
 size_t group_smem_bytes(const Geometry& geo) {
-    return static_cast<size_t>(geo.tile_elems) * 2 + static_cast<size_t>(geo.tile_groups) * (8 + 4 * 6 + 2 + 1);
+    return static_cast<size_t>(geo.tile_elems) * 2 + static_cast<size_t>(geo.tile_groups) * (8 + 4 * 7 + 2 + 1);
 }
 
 size_t tensor_smem_bytes(const Geometry& geo) {
@@ -978,9 +985,11 @@ WorkspaceLayout workspace_layout(int64_t G, int stop_mode, int zero_nbits) {
     const size_t Gs = static_cast<size_t>(G > 0 ? G : 0);
     l.zbest = off;
     if (zero_nbits == 8) off = up(off + 4 * Gs);
-    l.t_s = l.t_z0 = l.t_sws = l.t_z = l.t_e = off;
+    l.t_s = l.t_is = l.t_z0 = l.t_sws = l.t_z = l.t_e = off;
     if (stop_mode == 1) {
         l.t_s = off;
+        off = up(off + 4 * Gs);
+        l.t_is = off;
         off = up(off + 4 * Gs);
         l.t_z0 = off;
         off = up(off + 4 * Gs);
@@ -1047,6 +1056,7 @@ cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream, int* coop_unsu
     k.zbest_ws = a.zero_nbits == 8 ? reinterpret_cast<float*>(a.ws + L.zbest) : nullptr;
     if (a.stop_mode == 1) {
         k.t_s = reinterpret_cast<float*>(a.ws + L.t_s);
+        k.t_is = reinterpret_cast<float*>(a.ws + L.t_is);
         k.t_z0 = reinterpret_cast<float*>(a.ws + L.t_z0);
         k.t_sws = reinterpret_cast<double*>(a.ws + L.t_sws);
         k.t_z = reinterpret_cast<float*>(a.ws + L.t_z);

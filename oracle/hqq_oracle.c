@@ -42,6 +42,10 @@
  *   R8  packing: LSB-first bitstream along the group axis (layout below).
  *   R9  scale (= 1/s) and a 16-bit zero are stored as IEEE fp16.
  *   R10 element-wise arithmetic in fp32; every sum is accumulated in fp64.
+ *   R13 W_r = (W_q - z)/s is evaluated as (W_q - z) * (1/s) with the fp32
+ *       scale 1/s, the form the dequantiser uses.
+ *   R14 the group mean of W_q - (W - W_e)*s is evaluated as
+ *       (sum W_q - sum fl((W - W_e)*s)) / g, both sums in fp64.
  *
  * Layout.  W is row-major [rows, cols].  axis = 1: group j holds the g
  * contiguous elements [j*g, (j+1)*g) of the flattened tensor (g | cols);
@@ -139,13 +143,16 @@ static float quantize_elem(float w, float s, float z, int L)
 }
 
 /* Quantise the group with zero-point z, reconstruct W_r = (W_q - z)/s and
- * return the sum of |W - W_r|^p (R3).  q and d receive W_q and W - W_r. */
+ * return the sum of |W - W_r|^p (R3).  The reconstruction multiplies by the
+ * fp32 scale 1/s, the form the dequantiser uses (R13).  q and d receive W_q
+ * and W - W_r. */
 static double evaluate(const float *w, int g, int L, float s, float z, float p, float *q, float *d)
 {
+    const float inv_s = 1.0f / s;
     double acc = 0.0;
     for (int i = 0; i < g; ++i) {
         float qi = quantize_elem(w[i], s, z, L);
-        float wr = (qi - z) / s;
+        float wr = (qi - z) * inv_s;
         q[i] = qi;
         d[i] = w[i] - wr;
         acc += (double)powf(fabsf(d[i]), p);
@@ -153,16 +160,18 @@ static double evaluate(const float *w, int g, int L, float s, float z, float p, 
     return acc;
 }
 
-/* Sub-problem 2: W_e = shrink(W - W_r), then z = mean(W_q - (W - W_e)*s). */
+/* Sub-problem 2: W_e = shrink(W - W_r), then z = mean(W_q - (W - W_e)*s),
+ * evaluated as mean(W_q) - mean((W - W_e)*s) with both sums in fp64 (R14). */
 static float update_zero(const float *w, const float *q, const float *d, int g, float s, float p, float beta)
 {
-    double acc = 0.0;
+    double sq = 0.0, sws = 0.0;
     for (int i = 0; i < g; ++i) {
         float we = oracle_shrink(d[i], p, beta);
-        float t = q[i] - (w[i] - we) * s;
-        acc += (double)t;
+        float ws = (w[i] - we) * s;
+        sq += (double)q[i];
+        sws += (double)ws;
     }
-    return (float)(acc / (double)g);
+    return (float)((sq - sws) / (double)g);
 }
 
 /* ---- one group, group-wise (or no) early stopping ------------------------ */

@@ -2,8 +2,8 @@
 
 Inputs are seeded synthetic weights with the pages' weight statistics
 (0.02 * N(0,1), 0.1% outliers x10) plus degenerate cases.  Small shapes span
-several tiles and a ragged tail; full Llama-2 shapes are checked on sampled
-groups in the launch configuration the benchmark uses.
+several tiles and a ragged tail; the Llama-2 shapes the benchmark quantises
+are checked in full, in the same launch configuration.
 """
 import numpy as np
 import pytest
@@ -208,37 +208,26 @@ def _sampled(hq, W_cpu, prm, n=6000, seed=0):
 
 
 def test_llama_square_4096_fp16_b4_g64(hq):
+    """Single 4096x4096 fp16 weight, b4 g64, group stop, fp16 zero: full tensor."""
     W = synth.weight(4096, 4096, seed=0, dtype=torch.float16)
-    rep, gpu = _sampled(hq, W, _params(4, 64), n=20000)
+    rep, _, _ = _run(hq, W, _params(4, 64))
     assert rep["tie_groups"] <= 3
 
 
-@pytest.mark.parametrize("nbits,g", [(8, 128), (4, 64), (3, 64), (2, 16), (1, 16)])
+SWEEP = [(8, 128), (4, 64), (3, 64), (2, 16), (1, 16)]
+
+
+@pytest.mark.parametrize("nbits,g", SWEEP)
 @pytest.mark.parametrize("shape", [(11008, 4096), (4096, 11008)])
-def test_llama_mlp_group_mode_sampled(hq, nbits, g, shape):
-    W = synth.weight(*shape, seed=1000 * 0 + (4 if shape[0] == 11008 else 6), dtype=torch.bfloat16)
-    _sampled(hq, W, _params(nbits, g), n=4000, seed=nbits)
+def test_llama_mlp_group_mode(hq, nbits, g, shape):
+    """Llama-2-7B MLP shapes (gate/up and down), bf16, group stop: full tensors."""
+    W = synth.weight(*shape, seed=4 if shape[0] == 11008 else 6, dtype=torch.bfloat16)
+    _run(hq, W, _params(nbits, g), check_recon=(nbits == 4))
 
 
-@pytest.mark.parametrize("nbits,g", [(8, 128), (4, 64), (3, 64), (2, 16), (1, 16)])
-def test_llama_mlp_tensor_mode_groups_follow_kept_iterate(hq, nbits, g):
-    """Full-size tensor mode: every sampled group's z* and codes are the oracle's
-    iterate at the GPU's tensor-wide index."""
-    W_cpu = synth.weight(11008, 4096, seed=4, dtype=torch.bfloat16)
-    prm = _params(nbits, g, stop=1)
-    out = hq.quantize(W_cpu.cuda(), nbits, g, stop_mode=1, debug=True)
-    torch.cuda.synchronize()
-    assert hq.hqq_get_status(out["workspace"]) == hq.HQQ_OK
-    gpu = pc.gpu_to_numpy(out)
-    G = W_cpu.numel() // g
-    bi = gpu["best_iter"]
-    assert np.all(bi == bi[0])
-    k = int(bi[0])
-    Wf = pc.w_float(W_cpu)
-    gl = oracle.unpack_levels(gpu["packed"], *W_cpu.shape, nbits, 1)
-    for j in np.random.default_rng(1).choice(G, 500, replace=False):
-        w = pc.group_values(Wf, j, g, 1)
-        s, zt, et, _ = oracle.trace_group(w, nbits, iters=20)
-        assert abs(gpu["zero_f32"][j] - zt[k]) <= pc.Z_TOL * max(abs(zt[k]), 1)
-        lv = oracle.group_codes(w, nbits, s, zt[k])
-        assert np.count_nonzero(pc.group_levels(gl, j, g, 1).astype(int) - lv) <= 1
+@pytest.mark.parametrize("nbits,g", SWEEP)
+def test_llama_mlp_tensor_mode(hq, nbits, g):
+    """Llama-2-7B gate shape, bf16, tensor stop: full tensor against the full oracle."""
+    W = synth.weight(11008, 4096, seed=4, dtype=torch.bfloat16)
+    rep, gpu, orc = _run(hq, W, _params(nbits, g, stop=1), check_recon=(nbits == 2))
+    assert np.all(gpu["best_iter"] == orc["best_iter"][0])

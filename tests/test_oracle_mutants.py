@@ -19,11 +19,11 @@ SRC = os.path.join(ROOT, "oracle", "hqq_oracle.c")
 
 # (name, text in the source, replacement, expected number of occurrences)
 MUTANTS = [
-    ("z-update-sign", "float t = q[i] - (w[i] - we) * s;", "float t = q[i] + (w[i] - we) * s;", 1),
-    ("z-update-drops-We", "float t = q[i] - (w[i] - we) * s;", "float t = q[i] - (w[i] - 0.0f * we) * s;", 1),
+    ("z-update-sign", "return (float)((sq - sws) / (double)g);", "return (float)((sq + sws) / (double)g);", 1),
+    ("z-update-drops-We", "float ws = (w[i] - we) * s;", "float ws = (w[i] - 0.0f * we) * s;", 1),
     ("shrink-exponent", "powf(a, p - 1.0f) / beta", "powf(a, p) / beta", 1),
     ("shrink-beta-inverted", "powf(a, p - 1.0f) / beta", "powf(a, p - 1.0f) * beta", 1),
-    ("reconstruction-sign", "float wr = (qi - z) / s;", "float wr = (qi + z) / s;", 1),
+    ("reconstruction-sign", "float wr = (qi - z) * inv_s;", "float wr = (qi + z) * inv_s;", 1),
     ("l1-instead-of-lp", "acc += (double)powf(fabsf(d[i]), p);", "acc += (double)fabsf(d[i]);", 1),
     ("tie-continues", "        if (e < best) {\n            best = e;\n            zbest = z;",
      "        if (e <= best) {\n            best = e;\n            zbest = z;", 1),
