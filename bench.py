@@ -210,6 +210,30 @@ def config_dict(world):
             "l2": "inputs 270 MB > 126 MB L2; consecutive calls use different matrices"}
 
 
+def run_case(spec):
+    """Time hqq_quantize on one synthetic bf16 matrix (used for kernel profiles)."""
+    from calibration_free_weight_b200 import hqq
+    v = [int(x) for x in spec.split(",")]
+    mode, rows, cols, nbits, g = v[:5]
+    reps = v[5] if len(v) > 5 else 3
+    torch.cuda.set_device(0)
+    W = synth.weight(rows, cols, seed=4, dtype=torch.bfloat16).cuda()
+    out = hqq.alloc_outputs(rows, cols, nbits, g, 1, mode, 16)
+    ev = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        hqq.quantize(W, nbits, g, stop_mode=mode, out=out)
+        b.record()
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    st = hqq.hqq_get_status(out["workspace"])
+    if st != hqq.HQQ_OK:
+        raise RuntimeError(hqq.hqq_status_string(st))
+    ms = [a.elapsed_time(b) for a, b in ev]
+    print(json.dumps({"case": spec, "ms_per_call": ms, "gweights_s_last": rows * cols / (ms[-1] / 1e3) / 1e9}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -218,7 +242,12 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--ref-budget", type=float, default=8.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None,
+                    help="single-matrix timing instead of the sweep: stop_mode,rows,cols,nbits,group_size[,reps]")
     args = ap.parse_args()
+    if args.case:
+        run_case(args.case)
+        return
 
     if args.impl == "reference":
         # CPU oracle only: rank 0 times it, other ranks exit without work
