@@ -18,7 +18,8 @@ HQQ_F16, HQQ_BF16 = 0, 1
 HQQ_STOP_GROUP, HQQ_STOP_TENSOR, HQQ_STOP_NONE = 0, 1, 2
 
 EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_quantize", "hqq_dequantize",
-            "hqq_get_status", "hqq_status_string", "hqq_debug_set_barrier")
+            "hqq_get_status", "hqq_status_string", "hqq_debug_set_barrier", "hqq_quantize_noalloc")
+HQQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def _load():
@@ -44,6 +45,9 @@ def _load():
     L.hqq_status_string.argtypes = [i32]
     L.hqq_debug_set_barrier.restype = None
     L.hqq_debug_set_barrier.argtypes = [i32, C.c_uint64]
+    L.hqq_quantize_noalloc.restype = i32
+    L.hqq_quantize_noalloc.argtypes = [P, i64, i64, i32, i32, i32, i32, f32, f32, f32, i32, i32, i32,
+                                       P, P, P, P, P, P, P, P]
     return L
 
 
@@ -90,6 +94,17 @@ def hqq_quantize(W, rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, 
                             zero_nbits, _ptr(W_q_packed), _ptr(scale), _ptr(zero), _ptr(zero_meta), _ptr(workspace),
                             workspace_bytes, _ptr(debug_best_iter), _ptr(debug_best_err), _ptr(debug_zero_f32),
                             _stream(stream))
+
+
+def hqq_quantize_noalloc(W, rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
+                         zero_nbits, W_q_packed, scale, zero, zero_meta, debug_best_iter=None, debug_best_err=None,
+                         debug_zero_f32=None, stream=None):
+    """hqq_quantize without a workspace argument: the library's own static
+    device scratch is used (for callers that cannot allocate)."""
+    return lib.hqq_quantize_noalloc(_ptr(W), rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters,
+                                    stop_mode, zero_nbits, _ptr(W_q_packed), _ptr(scale), _ptr(zero), _ptr(zero_meta),
+                                    _ptr(debug_best_iter), _ptr(debug_best_err), _ptr(debug_zero_f32),
+                                    _stream(stream))
 
 
 def hqq_dequantize(W_q_packed, scale, zero, zero_meta, rows, cols, nbits, group_size, axis, zero_nbits, out_dtype,

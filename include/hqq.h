@@ -154,6 +154,39 @@ const char* hqq_status_string(int status);
  * timeout and report HQQ_ERR_TIMEOUT.  Never hangs: every wait is bounded. */
 void hqq_debug_set_barrier(int skip_block, uint64_t timeout_ns);
 
+/* Size of the library-owned scratch buffer used by hqq_quantize_noalloc. */
+#define HQQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * hqq_quantize_noalloc -- hqq_quantize for callers that cannot allocate
+ * device memory, such as a plugin inside a host runtime that owns every device
+ * allocation, or a latency-critical loop that must not pay for cudaMalloc and
+ * the device synchronisation it can cause.  The HQQ pages have no counterpart:
+ * this is an interface convenience of this library.
+ *
+ * Same arguments and results as hqq_quantize minus workspace/workspace_bytes.
+ * The caller still passes (and owns) W and every output buffer.  stop_mode must
+ * be HQQ_STOP_GROUP or HQQ_STOP_NONE; HQQ_STOP_TENSOR returns
+ * HQQ_ERR_INVALID_ARG (use hqq_quantize for it).
+ * Scratch: one buffer of HQQ_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory per
+ * GPU, held by the library from load until the process exits.  A problem whose
+ * hqq_workspace_bytes() exceeds it returns HQQ_ERR_WORKSPACE before anything is
+ * launched: with zero_nbits = 8 that means more than 4,169,664 groups (4 bytes
+ * per group plus 98,560 fixed bytes); with zero_nbits = 16 every size fits.
+ * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine).  The first call on each device looks up the buffer's device
+ * address (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call on a device shares the buffer, which
+ * keeps the last call's contents (each call clears what must start at zero);
+ * calls whose work overlaps on the GPU race on it, so keep them ordered, e.g.
+ * on one stream.
+ */
+int hqq_quantize_noalloc(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis,
+                         float p, float beta, float kappa, int iters, int stop_mode, int zero_nbits,
+                         void* W_q_packed, void* scale, void* zero, void* zero_meta,
+                         int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32,
+                         void* stream);
+
 #ifdef __cplusplus
 }
 #endif
