@@ -64,7 +64,7 @@ int64_t hqq_num_groups(int64_t rows, int64_t cols, int group_size, int axis) {
 size_t hqq_workspace_bytes(int64_t rows, int64_t cols, int group_size, int axis, int stop_mode, int zero_nbits) {
     if (check_shape(rows, cols, group_size, axis) != HQQ_OK) return 0;
     if (stop_mode < 0 || stop_mode > 2 || (zero_nbits != 8 && zero_nbits != 16)) return 0;
-    return hqq::workspace_layout(rows * cols / group_size, stop_mode, zero_nbits).total;
+    return hqq::workspace_layout(rows * cols / group_size, stop_mode, zero_nbits, hqq::kMaxIters).total;
 }
 
 int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p,
@@ -78,11 +78,11 @@ int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits
     if (!(p > 0.0f && p < 2.0f) || !(beta > 0.0f) || !std::isfinite(beta) || !(kappa >= 1.0f) ||
         !std::isfinite(kappa))
         return HQQ_ERR_INVALID_ARG;
-    if (iters < 0 || iters > 1000) return HQQ_ERR_INVALID_ARG;
+    if (iters < 0 || iters > hqq::kMaxIters) return HQQ_ERR_INVALID_ARG;
     if (stop_mode < 0 || stop_mode > 2) return HQQ_ERR_INVALID_ARG;
     if (zero_nbits != 8 && zero_nbits != 16) return HQQ_ERR_INVALID_ARG;
     const int64_t G = rows * cols / group_size;
-    const size_t need = hqq::workspace_layout(G, stop_mode, zero_nbits).total;
+    const size_t need = hqq::workspace_layout(G, stop_mode, zero_nbits, hqq::kMaxIters).total;
     if (workspace == nullptr || workspace_bytes < need) return HQQ_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return HQQ_ERR_ALIGN;
     if (!is_device_ptr(workspace)) return HQQ_ERR_INVALID_ARG;
@@ -126,10 +126,7 @@ int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits
     a.dbg_iter = debug_best_iter;
     a.dbg_err = debug_best_err;
     a.dbg_zero = debug_zero_f32;
-    a.vec_ok = axis == 1 || (cols % 8 == 0);
-    int coop_unsupported = 0;
-    const cudaError_t err = hqq::launch_solve(a, static_cast<cudaStream_t>(stream), &coop_unsupported);
-    if (coop_unsupported) return HQQ_ERR_COOP_UNSUPPORTED;
+    const cudaError_t err = hqq::launch_solve(a, static_cast<cudaStream_t>(stream));
     if (err != cudaSuccess) {
         cudaGetLastError();
         return HQQ_ERR_CUDA;
@@ -193,13 +190,11 @@ const char* hqq_status_string(int status) {
         case HQQ_ERR_DTYPE: return "unsupported dtype";
         case HQQ_ERR_ALIGN: return "misaligned buffer";
         case HQQ_ERR_CUDA: return "CUDA runtime error";
-        case HQQ_ERR_TIMEOUT: return "device wait timed out";
-        case HQQ_ERR_COOP_UNSUPPORTED: return "cooperative launch unsupported";
+        case HQQ_ERR_TIMEOUT: return "device wait timed out (reserved; not produced)";
+        case HQQ_ERR_COOP_UNSUPPORTED: return "cooperative launch unsupported (reserved; not produced)";
         case HQQ_ERR_WORKSPACE: return "workspace missing or too small";
         default: return "unknown status";
     }
 }
-
-void hqq_debug_set_barrier(int skip_block, uint64_t timeout_ns) { hqq::set_barrier_debug(skip_block, timeout_ns); }
 
 }  // extern "C"

@@ -1,0 +1,209 @@
+// hqq_device.cuh -- device-side building blocks shared by the solver kernels.
+//
+// Method: techreport.ngo, "Weight-only quantization without the calibration
+// tax" (Half-Quadratic Quantization of Large Machine Learning Models), section
+// "Outlier-aware optimization without gradients".  Per element, with
+// ws = fl(w*s) and v = fl(ws + z):
+//   W_q = clamp(round_half_even(v), 0, L)
+//   r   = v - W_q                      (exact in fp32)
+//   W - W_r = W - (W_q - z)/s = r/s    so |W - W_r|^p = |r|^p * s^-p
+// The group sums are sum |r|^p (MUFU lg2/ex2), sum W_q (exact: integers) and,
+// precomputed once per group, sum fl(w*s) in fp64; the zero update is
+// z' = (sum W_q - sum fl((w - W_e)*s)) / g, which equals sum W_q - sum ws when
+// the proximal step W_e is zero for the whole group.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include <cfloat>
+#include <cstdint>
+
+#include "hqq_internal.h"
+
+namespace hqq {
+namespace dev {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23: adding it rounds to an integer
+constexpr uint32_t kMagicBits = 0x4B400000u;  // bit pattern of kMagic
+
+// ------------------------------------------------------------ math ------
+
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// a^e for a >= 0 through the hardware base-2 log and exponential (0^e = 0, e > 0).
+__device__ __forceinline__ float pow_pos(float a, float e) { return ex2_approx(e * lg2_approx(a)); }
+
+// beta^(-1/(2-p)): |d| at or below it gives a proximal step of exactly 0.
+__device__ __forceinline__ float shrink_threshold(float beta, float p) {
+    return ex2_approx(-lg2_approx(beta) / (2.0f - p));
+}
+
+// round_half_even(clamp(v, 0, L)) == clamp(round_half_even(v), 0, L) for
+// integer bounds; adding 1.5*2^23 rounds to nearest-even exactly for
+// |x| < 2^22, and the integer code is read from the sum's low mantissa bits.
+__device__ __forceinline__ float round_clamp(float v, float Lf, uint32_t* code) {
+    const float t = __fadd_rn(fminf(fmaxf(v, 0.0f), Lf), kMagic);
+    *code = __float_as_uint(t) - kMagicBits;
+    return __fsub_rn(t, kMagic);
+}
+
+// One element of one evaluation: ws = fl(w*s) precomputed.
+struct ElemEval {
+    float v, q, r;
+    uint32_t code;
+};
+__device__ __forceinline__ ElemEval eval_elem(float ws, float z, float Lf) {
+    ElemEval e;
+    e.v = __fadd_rn(ws, z);
+    e.q = round_clamp(e.v, Lf, &e.code);
+    e.r = __fsub_rn(e.v, e.q);
+    return e;
+}
+
+// Proximal step of the lp term for one element: d = r/s, W_e = shrink(d).
+__device__ __forceinline__ float shrink_elem(float r, float s, float p, float beta) {
+    const float d = __fdiv_rn(r, s);
+    const float a = fabsf(d);
+    if (a == 0.0f) return 0.0f;
+    const float t = __fsub_rn(a, __fdiv_rn(pow_pos(a, p - 1.0f), beta));
+    return t > 0.0f ? copysignf(t, d) : 0.0f;
+}
+
+// |w - W_r| * s <= max(0.5, |z - z0|) + rounding for every element of a
+// group (v spans [z - z0, L + z - z0] up to rounding), so the proximal step
+// is zero for the whole group unless this bound reaches thr * s.
+__device__ __forceinline__ bool shrink_possible(float s, float z, float z0, float thr, float Lf) {
+    return fmaxf(0.5f, fabsf(z - z0)) + 1e-3f * (1.0f + Lf + fabsf(z)) >= 0.99f * thr * s;
+}
+
+__device__ __forceinline__ float zero_from_sums(float sq, double sws, int g) {
+    return static_cast<float>((static_cast<double>(sq) - sws) / static_cast<double>(g));
+}
+
+// ------------------------------------------------------ reductions -------
+
+// Over P consecutive lanes (P a power of two <= 32); all lanes of the segment
+// get the same value.
+__device__ __forceinline__ float seg_sum(float x, int P) {
+    for (int o = 1; o < P; o <<= 1) x += __shfl_xor_sync(kFull, x, o);
+    return x;
+}
+__device__ __forceinline__ double seg_sum_d(double x, int P) {
+    for (int o = 1; o < P; o <<= 1) x += __shfl_xor_sync(kFull, x, o);
+    return x;
+}
+__device__ __forceinline__ float seg_min(float x, int P) {
+    for (int o = 1; o < P; o <<= 1) x = fminf(x, __shfl_xor_sync(kFull, x, o));
+    return x;
+}
+__device__ __forceinline__ float seg_max(float x, int P) {
+    for (int o = 1; o < P; o <<= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
+    return x;
+}
+
+// --------------------------------------------------------- elements ------
+
+template <int DT>
+__device__ __forceinline__ float bits_to_float(uint32_t b16) {
+    if (DT == 0) return __half2float(__ushort_as_half(static_cast<unsigned short>(b16)));
+    return __uint_as_float(b16 << 16);
+}
+
+// Eight 16-bit elements held in a uint4 -> fp32.
+template <int DT>
+__device__ __forceinline__ void unpack8(const uint4 u, float* w) {
+    const uint32_t x[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (DT == 0) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&x[i]));
+            w[2 * i] = f.x;
+            w[2 * i + 1] = f.y;
+        } else {
+            w[2 * i] = __uint_as_float(x[i] << 16);
+            w[2 * i + 1] = __uint_as_float(x[i] & 0xffff0000u);
+        }
+    }
+}
+
+// ----------------------------------------------------------- packing -----
+
+// Eight codes, LSB first, nbits each.
+__device__ __forceinline__ uint64_t pack8(const uint32_t* c, int nbits) {
+    uint64_t v = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v |= static_cast<uint64_t>(c[i]) << (i * nbits);
+    return v;
+}
+
+// Store the nbits bytes of one packed 8-element piece (dst aligned to nbits
+// bytes for nbits in {1,2,4,8}; byte stores for 3).
+__device__ __forceinline__ void store_piece(uint8_t* dst, uint64_t v, int nbits) {
+    switch (nbits) {
+        case 1: *dst = static_cast<uint8_t>(v); break;
+        case 2: *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(v); break;
+        case 4: *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(v); break;
+        case 8: *reinterpret_cast<uint64_t*>(dst) = v; break;
+        default:
+            dst[0] = static_cast<uint8_t>(v);
+            dst[1] = static_cast<uint8_t>(v >> 8);
+            dst[2] = static_cast<uint8_t>(v >> 16);
+            break;
+    }
+}
+
+__device__ __forceinline__ uint16_t half_bits(float x) { return __half_as_ushort(__float2half_rn(x)); }
+
+// --------------------------------------------------------- async copy ----
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+}  // namespace dev
+
+// Kernel parameters shared by the solver kernels (passed by value).
+struct KParams {
+    const uint16_t* W;
+    int64_t rows, cols, G;
+    int g, P, logP, E, nbits, iters, iters_eff, stop_mode, zero_nbits, axis;
+    float p, beta, kappa, Lf;
+    int64_t n;  // rows * cols
+    uint8_t* packed;
+    uint16_t* scale;
+    void* zero;
+    int32_t* dbg_iter;
+    float* dbg_err;
+    float* dbg_zero;
+    // workspace
+    uint32_t* counters;  // [0] status, [1] work counter, [2] CTA ticket
+    float2* minmax;      // per-CTA zero min/max
+    double* tparts;      // per-iteration per-CTA tensor error partials [iters][kMaxPartials]
+    double* etot;        // per-iteration tensor mean error [iters]
+    float* zbest_ws;     // fp32 kept zero (8-bit zero path)
+    float* t_s;          // tensor state: s, z0, sum ws, chunk-start zeros (ring of 3)
+    float* t_z0;
+    double* t_sws;
+    float* t_zs;
+    // pool kernel geometry
+    int NC;              // cells per warp
+    int pool_warp_bytes;
+};
+
+}  // namespace hqq

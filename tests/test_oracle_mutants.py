@@ -23,7 +23,8 @@ MUTANTS = [
     ("z-update-drops-We", "float ws = (w[i] - we) * s;", "float ws = (w[i] - 0.0f * we) * s;", 1),
     ("shrink-exponent", "powf(a, p - 1.0f) / beta", "powf(a, p) / beta", 1),
     ("shrink-beta-inverted", "powf(a, p - 1.0f) / beta", "powf(a, p - 1.0f) * beta", 1),
-    ("reconstruction-sign", "float wr = (qi - z) * inv_s;", "float wr = (qi + z) * inv_s;", 1),
+    ("residual-sign", "float r = v - qi;", "float r = qi - v + 2.0f * (qi - v) * (qi > 0.0f);", 1),
+    ("residual-unscaled", "d[i] = r / s;", "d[i] = r;", 1),
     ("l1-instead-of-lp", "acc += (double)powf(fabsf(d[i]), p);", "acc += (double)fabsf(d[i]);", 1),
     ("tie-continues", "        if (e < best) {\n            best = e;\n            zbest = z;",
      "        if (e <= best) {\n            best = e;\n            zbest = z;", 1),
