@@ -72,6 +72,34 @@ __device__ __forceinline__ ElemEval eval_elem(float ws, float z, float Lf) {
     return e;
 }
 
+// Same without the clamp: exact when every v of the group lies in
+// [-0.5, L + 0.5), where round-half-even(v) is already in [0, L].
+__device__ __forceinline__ ElemEval eval_elem_nc(float ws, float z) {
+    ElemEval e;
+    e.v = __fadd_rn(ws, z);
+    const float t = __fadd_rn(e.v, kMagic);
+    e.code = __float_as_uint(t) - kMagicBits;
+    e.q = __fsub_rn(t, kMagic);
+    e.r = __fsub_rn(e.v, e.q);
+    return e;
+}
+
+// True when no v = fl(ws + z) of a set with ws in [wsmin, wsmax] needs the
+// clamp (fl(. + z) is monotone, so the extremes decide).
+__device__ __forceinline__ bool clamp_free(float wsmin, float wsmax, float z, float Lf) {
+    return __fadd_rn(wsmin, z) >= -0.5f && __fadd_rn(wsmax, z) < Lf + 0.5f;
+}
+
+// Compensated (TwoSum) fp32 accumulation: hi + lo carries the running sum of
+// fp32 terms to ~2^-48 relative, so no per-term conversion to fp64 is needed.
+__device__ __forceinline__ void two_sum_acc(float& hi, float& lo, float x) {
+    const float s = __fadd_rn(hi, x);
+    const float bp = __fsub_rn(s, hi);
+    const float e = __fadd_rn(__fsub_rn(hi, __fsub_rn(s, bp)), __fsub_rn(x, bp));
+    hi = s;
+    lo = __fadd_rn(lo, e);
+}
+
 // Proximal step of the lp term for one element: d = r/s, W_e = shrink(d).
 __device__ __forceinline__ float shrink_elem(float r, float s, float p, float beta) {
     const float d = __fdiv_rn(r, s);
@@ -90,6 +118,28 @@ __device__ __forceinline__ bool shrink_possible(float s, float z, float z0, floa
 
 __device__ __forceinline__ float zero_from_sums(float sq, double sws, int g) {
     return static_cast<float>((static_cast<double>(sq) - sws) / static_cast<double>(g));
+}
+
+// A double split into two floats, hi = fl32(x), lo = fl32(x - hi).
+struct F2 {
+    float hi, lo;
+};
+__device__ __forceinline__ F2 split_f2(double x) {
+    F2 r;
+    r.hi = static_cast<float>(x);
+    r.lo = static_cast<float>(x - static_cast<double>(r.hi));
+    return r;
+}
+
+// zero_from_sums in fp32 only: (sq - hi) is formed exactly by TwoSum, the
+// small remainder (e - lo) is added once, and the single rounding of that sum
+// gives fl32(sq - sws) (ties aside), which is exact after scaling by 1/g (a
+// power of two).  Short dependency chain: no fp64 conversions.
+__device__ __forceinline__ float zero_from_sums_f2(float sq, F2 sws, float inv_g) {
+    const float d = __fsub_rn(sq, sws.hi);
+    const float bp = __fsub_rn(d, sq);
+    const float e = __fadd_rn(__fsub_rn(sq, __fsub_rn(d, bp)), __fsub_rn(-sws.hi, bp));
+    return __fmul_rn(__fadd_rn(d, __fsub_rn(e, sws.lo)), inv_g);
 }
 
 // ------------------------------------------------------ reductions -------

@@ -93,10 +93,10 @@ __device__ __forceinline__ void write_minmax(const KParams& k, float zmin, float
 // the cell by cp.async; initialisation overwrites the cell with fp32 w*s.
 struct Pool {
     float* data;
-    float4* zs4;  // (z, s, z0, thr): what every lane of a group reads per evaluation
-    double* sws;
+    float4* zs4;  // (z, s, z0, flags): what every lane of a group reads per evaluation
+    float2* sws;  // sum of w*s as a float pair (hi, lo)
     int64_t* gidx;
-    float *be, *zb, *beta;
+    float *be, *zb, *beta, *wsmax;
     int *kk, *bi, *issued;
     uint8_t *st, *list;
 };
@@ -104,7 +104,7 @@ struct Pool {
 __host__ __device__ inline int pool_cell_floats(int g) { return g + 4; }
 
 __host__ __device__ inline int pool_warp_bytes(int NC, int g) {
-    const int b = NC * (4 * pool_cell_floats(g) + 16 + 8 + 8 + 3 * 4 + 3 * 4 + 2);
+    const int b = NC * (4 * pool_cell_floats(g) + 16 + 8 + 8 + 4 * 4 + 3 * 4 + 2);
     return (b + 15) & ~15;
 }
 
@@ -115,7 +115,7 @@ __device__ __forceinline__ Pool carve_pool(unsigned char* base, int NC, int g) {
     off += static_cast<size_t>(NC) * pool_cell_floats(g) * 4;
     m.zs4 = reinterpret_cast<float4*>(base + off);
     off += NC * 16;
-    m.sws = reinterpret_cast<double*>(base + off);
+    m.sws = reinterpret_cast<float2*>(base + off);
     off += NC * 8;
     m.gidx = reinterpret_cast<int64_t*>(base + off);
     off += NC * 8;
@@ -123,7 +123,8 @@ __device__ __forceinline__ Pool carve_pool(unsigned char* base, int NC, int g) {
     m.be = f;
     m.zb = f + NC;
     m.beta = f + 2 * NC;
-    off += NC * 3 * 4;
+    m.wsmax = f + 3 * NC;
+    off += NC * 4 * 4;
     int* iv = reinterpret_cast<int*>(base + off);
     m.kk = iv;
     m.bi = iv + NC;
@@ -187,8 +188,21 @@ __device__ __forceinline__ void store_piece_t(uint8_t* dst, const uint32_t* c) {
     }
 }
 
-// Group-level decision after evaluating zero-point z (one lane per group).
-// Returns the new state (kActive or kDone) and updates the cell.
+constexpr unsigned kFlagShrink = 1u;  // the proximal step may be non-zero
+constexpr unsigned kFlagClamp = 2u;   // some v may leave [-0.5, L + 0.5)
+
+// Flags of the next evaluation of a group at zero-point z (v = fl(ws + z) with
+// ws in [-z0, wsmax]: fl(min w * s) = -z0 exactly).
+__device__ __forceinline__ float eval_flags(float s, float z, float z0, float wsmax, float thr, float Lf) {
+    unsigned f = 0;
+    if (shrink_possible(s, z, z0, thr, Lf)) f |= kFlagShrink;
+    if (!clamp_free(-z0, wsmax, z, Lf)) f |= kFlagClamp;
+    return __uint_as_float(f);
+}
+
+// Group-level decision after evaluating zero-point z (one lane per group):
+// keep the best iterate, apply the stop rule, compute the next zero-point and
+// the flags of its evaluation.
 __device__ __forceinline__ void decide(const KParams& k, const Pool& m, int c, bool stop_group, float err, float sq,
                                        bool sp, double swe, float z, float s, float z0, float beta, int kk) {
     const bool improved = err < m.be[c];
@@ -199,12 +213,14 @@ __device__ __forceinline__ void decide(const KParams& k, const Pool& m, int c, b
     }
     bool stop = (stop_group && !improved) || kk >= k.iters_eff - 1;
     if (!stop) {
-        const float zn = zero_from_sums(sq, sp ? swe : m.sws[c], k.g);
+        const float2 f = m.sws[c];
+        const float zn = sp ? zero_from_sums(sq, swe, k.g)
+                            : zero_from_sums_f2(sq, F2{f.x, f.y}, 1.0f / static_cast<float>(k.g));
         if (stop_group && zn == z) {
             stop = true;  // fixed point: the next error would equal this one
         } else {
             const float nbeta = __fmul_rn(beta, k.kappa);
-            m.zs4[c] = make_float4(zn, s, z0, shrink_threshold(nbeta, k.p));
+            m.zs4[c] = make_float4(zn, s, z0, eval_flags(s, zn, z0, m.wsmax[c], shrink_threshold(nbeta, k.p), k.Lf));
             m.kk[c] = kk + 1;
             m.beta[c] = nbeta;
         }
@@ -351,17 +367,19 @@ __global__ void __launch_bounds__(kPoolThreads, 6) solve_pool_kernel(const KPara
                 float s = kScaleCap;
                 if (mx > mn) s = fminf(__fdiv_rn(Lf, __fsub_rn(mx, mn)), kScaleCap);
                 const float z0 = __fmul_rn(-mn, s);
-                double acc = 0.0;
+                float hi = 0.0f, lo = 0.0f;
                 float ws[E];
                 float err = 0.0f, sq = 0.0f;
 #pragma unroll
                 for (int i = 0; i < E; ++i) {
                     ws[i] = __fmul_rn(w[i], s);
-                    acc += static_cast<double>(ws[i]);
-                    const ElemEval ee = eval_elem(ws[i], z0, Lf);
+                    two_sum_acc(hi, lo, ws[i]);
+                    // at z0 every v lies in [0, L]: fl(min w * s) + z0 = 0, fl(max w * s) + z0 <= L
+                    const ElemEval ee = eval_elem_nc(ws[i], z0);
                     err += pow_pos(fabsf(ee.r), k.p);
                     sq += ee.q;
                 }
+                double acc = static_cast<double>(hi) + static_cast<double>(lo);
                 if (!valid) err = sq = 0.0f, acc = 0.0;
                 acc = seg_sum_d(acc, P);
                 err = seg_sum(err, P);
@@ -393,10 +411,12 @@ __global__ void __launch_bounds__(kPoolThreads, 6) solve_pool_kernel(const KPara
                         dst[1] = make_float4(ws[t * 8 + 4], ws[t * 8 + 5], ws[t * 8 + 6], ws[t * 8 + 7]);
                     }
                     if (part == 0) {
-                        m.sws[c] = acc;
+                        const F2 f = split_f2(acc);
+                        m.sws[c] = make_float2(f.hi, f.lo);
                         m.zb[c] = z0;
                         m.bi[c] = 0;
-                        m.zs4[c] = make_float4(z0, s, z0, thr0);
+                        m.wsmax[c] = __fmul_rn(mx, s);
+                        m.zs4[c] = make_float4(z0, s, z0, 0.0f);
                         if (k.iters_eff == 0) {
                             m.be[c] = INFINITY;
                             m.st[c] = kDone;
@@ -420,11 +440,26 @@ __global__ void __launch_bounds__(kPoolThreads, 6) solve_pool_kernel(const KPara
                 const int c = valid ? m.list[it >> logP] : 0;
                 const int part = it & (P - 1);
                 const float4 st4 = m.zs4[c];
-                const float z = st4.x, s = st4.y, z0 = st4.z, thr = st4.w;
-                const bool sp = valid && shrink_possible(s, z, z0, thr, Lf);
+                const float z = st4.x, s = st4.y, z0 = st4.z;
+                const unsigned flags = valid ? __float_as_uint(st4.w) : 0u;
+                const bool sp = (flags & kFlagShrink) != 0;
                 const float* cell = cell_ptr(m, c, g);
                 float err = 0.0f, sq = 0.0f;
-                if (valid) {
+                if (__all_sync(kFull, (flags & kFlagClamp) == 0)) {
+                    if (valid) {
+#pragma unroll
+                        for (int t = 0; t < NPL; ++t) {
+                            float ws[8];
+                            load_ws8(cell, part + t * P, ws);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const ElemEval ee = eval_elem_nc(ws[i], z);
+                                err += pow_pos(fabsf(ee.r), k.p);
+                                sq += ee.q;
+                            }
+                        }
+                    }
+                } else if (valid) {
 #pragma unroll
                     for (int t = 0; t < NPL; ++t) {
                         float ws[8];
@@ -561,30 +596,34 @@ __device__ __forceinline__ void store_lane_codes(const KParams& k, const WarpTil
 }
 
 // min/max -> s, z0; fp32 w*s; fp64 sum of w*s (over the group's P lanes).
+// Also returns this lane's range of w*s (for the clamp-free test).
 template <int E>
 __device__ __forceinline__ void init_lane(const KParams& k, const WarpTile& w, const float* x, float* ws, float* s_out,
-                                          float* z0_out, double* sws_out) {
-    float mn = FLT_MAX, mx = -FLT_MAX;
+                                          float* z0_out, double* sws_out, float* lmin_out, float* lmax_out) {
+    float lmn = FLT_MAX, lmx = -FLT_MAX;
     if (w.valid) {
 #pragma unroll
         for (int i = 0; i < E; ++i) {
-            mn = fminf(mn, x[i]);
-            mx = fmaxf(mx, x[i]);
+            lmn = fminf(lmn, x[i]);
+            lmx = fmaxf(lmx, x[i]);
         }
     }
-    mn = seg_min(mn, k.P);
-    mx = seg_max(mx, k.P);
+    const float mn = seg_min(lmn, k.P);
+    const float mx = seg_max(lmx, k.P);
     float s = kScaleCap;
     if (mx > mn) s = fminf(__fdiv_rn(k.Lf, __fsub_rn(mx, mn)), kScaleCap);
-    double acc = 0.0;
+    float hi = 0.0f, lo = 0.0f;
 #pragma unroll
     for (int i = 0; i < E; ++i) {
         ws[i] = __fmul_rn(x[i], s);
-        if (w.valid) acc += static_cast<double>(ws[i]);
+        two_sum_acc(hi, lo, ws[i]);
     }
+    const double acc = w.valid ? static_cast<double>(hi) + static_cast<double>(lo) : 0.0;
     *s_out = s;
     *z0_out = __fmul_rn(-mn, s);
     *sws_out = seg_sum_d(acc, k.P);
+    *lmin_out = w.valid ? __fmul_rn(lmn, s) : 0.0f;
+    *lmax_out = w.valid ? __fmul_rn(lmx, s) : 0.0f;
 }
 
 // One evaluation of zero-point z: group sums of |r|^p and W_q, and (only when
@@ -621,14 +660,30 @@ __device__ __forceinline__ void eval_lane(const KParams& k, bool active, const f
     *swe_out = swe;
 }
 
+// beta_k = kappa^k * beta as the sequential fp32 product.
+__device__ __forceinline__ float beta_at(const KParams& k, int it) {
+    float b = k.beta;
+    for (int i = 0; i < it; ++i) b = __fmul_rn(b, k.kappa);
+    return b;
+}
+
 // eval_lane without the raw values in registers: the rare shrink path reloads them.
 template <int DT, int AXIS, int E>
-__device__ __forceinline__ void eval_lane_reload(const KParams& k, const WarpTile& w, const float* ws, float s,
-                                                 float z, float z0, float beta, float thr, float* err_out,
-                                                 float* sq_out, bool* sp_out, double* swe_out) {
+__device__ __forceinline__ void eval_lane_reload(const KParams& k, const WarpTile& w, const float* ws, float lmin,
+                                                 float lmax, float s, float z, float z0, int it, float thr,
+                                                 float* err_out, float* sq_out, bool* sp_out, double* swe_out) {
     float err = 0.0f, sq = 0.0f;
     const bool sp = w.valid && shrink_possible(s, z, z0, thr, k.Lf);
-    if (w.valid) {
+    if (__all_sync(kFull, !w.valid || clamp_free(lmin, lmax, z, k.Lf))) {
+        if (w.valid) {
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const ElemEval ee = eval_elem_nc(ws[i], z);
+                err += pow_pos(fabsf(ee.r), k.p);
+                sq += ee.q;
+            }
+        }
+    } else if (w.valid) {
 #pragma unroll
         for (int i = 0; i < E; ++i) {
             const ElemEval ee = eval_elem(ws[i], z, k.Lf);
@@ -641,6 +696,7 @@ __device__ __forceinline__ void eval_lane_reload(const KParams& k, const WarpTil
     double swe = 0.0;
     if (__any_sync(kFull, sp)) {
         if (sp) {
+            const float beta = beta_at(k, it);
             float x[E];
             load_lane<DT, AXIS, E>(k, w, x);
 #pragma unroll
@@ -687,7 +743,7 @@ __device__ __forceinline__ float step_lane(const KParams& k, bool valid, const f
         }
         swe = seg_sum_d(swe, k.P);
     }
-    return zero_from_sums(sq, sp ? swe : sws, k.g);
+    return sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, split_f2(sws), 1.0f / static_cast<float>(k.g));
 }
 
 __device__ __forceinline__ double warp_sum_d(double x) {
@@ -695,15 +751,9 @@ __device__ __forceinline__ double warp_sum_d(double x) {
     return x;
 }
 
-// beta_k = kappa^k * beta as the sequential fp32 product.
-__device__ __forceinline__ float beta_at(const KParams& k, int it) {
-    float b = k.beta;
-    for (int i = 0; i < it; ++i) b = __fmul_rn(b, k.kappa);
-    return b;
-}
-
 template <int DT, int AXIS, int E, int MODE>
-__global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2) solve_reg_kernel(const KParams k, int chunk) {
+__global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2)
+    solve_reg_kernel(const KParams k, int chunk) {
     __shared__ float2 sred[kRegWarps];
     __shared__ double sacc[kChunkMax][kRegWarps];
     __shared__ int sflag;
@@ -711,6 +761,7 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2) s
     const int64_t ntiles = num_warp_tiles<AXIS>(k);
     const int64_t wstride = static_cast<int64_t>(gridDim.x) * kRegWarps;
     const int64_t G = k.G;
+    const float inv_g = 1.0f / static_cast<float>(k.g);
     float zmin = FLT_MAX, zmax = -FLT_MAX;
 
     if (MODE == MODE_LOCAL) {
@@ -719,9 +770,10 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2) s
             const WarpTile w = warp_tile<AXIS>(k, t);
             float x[E], ws[E];
             load_lane<DT, AXIS, E>(k, w, x);
-            float s, z0;
+            float s, z0, lmin, lmax;
             double sws;
-            init_lane<E>(k, w, x, ws, &s, &z0, &sws);
+            init_lane<E>(k, w, x, ws, &s, &z0, &sws, &lmin, &lmax);
+            const F2 sws2 = split_f2(sws);
             float z = z0, zb = z0, be = INFINITY, beta = k.beta;
             int bi = 0;
             bool active = w.valid && k.iters_eff > 0;
@@ -740,7 +792,7 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2) s
                     }
                     bool stop = (stop_group && !improved) || it >= k.iters_eff - 1;
                     if (!stop) {
-                        const float zn = zero_from_sums(sq, sp ? swe : sws, k.g);
+                        const float zn = sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, sws2, inv_g);
                         if (stop_group && zn == z) stop = true;
                         else z = zn;
                     }
@@ -796,9 +848,9 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2) s
             const WarpTile w = warp_tile<AXIS>(k, t);
             float x[E], ws[E];
             load_lane<DT, AXIS, E>(k, w, x);
-            float s, z0;
+            float s, z0, lmin, lmax;
             double sws;
-            init_lane<E>(k, w, x, ws, &s, &z0, &sws);
+            init_lane<E>(k, w, x, ws, &s, &z0, &sws, &lmin, &lmax);
             float z = (iters == 0 || cb == 0) ? z0 : (w.valid ? Zc[w.j] : 0.0f);
             float beta = beta_at(k, b0);
             for (int it = b0; it < kb; ++it) {
@@ -826,23 +878,23 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2) s
     float* const Zin = (chunk % 3 == 0) ? Zs0 : (chunk % 3 == 1 ? Zs1 : Zs2);
     float* const Zout = ((chunk + 1) % 3 == 0) ? Zs0 : ((chunk + 1) % 3 == 1 ? Zs1 : Zs2);
     double acc[kChunkMax] = {0.0, 0.0, 0.0, 0.0};
-    float betaq[kChunkMax], thrq[kChunkMax];  // beta_k and its shrink threshold, same for every group
+    float thrq[kChunkMax];  // shrink threshold of beta_k, the same for every group
     {
         float b = beta_at(k, k0);
 #pragma unroll
         for (int q = 0; q < kChunkMax; ++q) {
-            betaq[q] = b;
             thrq[q] = shrink_threshold(b, k.p);
             b = __fmul_rn(b, k.kappa);
         }
     }
+    constexpr bool kPrefetch = AXIS == 1 && E <= 16;
     int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp;
-    uint4 raw[E / kPiece];
-    if (AXIS == 1 && t < ntiles) load_raw1<E>(k, warp_tile<AXIS>(k, t), raw);
+    uint4 raw[kPrefetch ? E / kPiece : 1];
+    if (kPrefetch && t < ntiles) load_raw1<E>(k, warp_tile<AXIS>(k, t), raw);
     for (; t < ntiles; t += wstride) {
         const WarpTile w = warp_tile<AXIS>(k, t);
         float x[E], ws[E];
-        if (AXIS == 1) {
+        if (kPrefetch) {
 #pragma unroll
             for (int q = 0; q < E / kPiece; ++q) unpack8<DT>(raw[q], x + q * kPiece);
             if (t + wstride < ntiles) load_raw1<E>(k, warp_tile<AXIS>(k, t + wstride), raw);  // prefetch
@@ -853,10 +905,10 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2) s
         } else {
             load_lane<DT, AXIS, E>(k, w, x);
         }
-        float s, z0, z;
+        float s, z0, z, lmin, lmax;
         double sws;
         if (k0 == 0) {
-            init_lane<E>(k, w, x, ws, &s, &z0, &sws);
+            init_lane<E>(k, w, x, ws, &s, &z0, &sws, &lmin, &lmax);
             if (w.valid && w.part == 0) {
                 k.t_s[w.j] = s;
                 k.t_z0[w.j] = z0;
@@ -868,19 +920,28 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2) s
             z0 = w.valid ? k.t_z0[w.j] : 0.0f;
             sws = w.valid ? k.t_sws[w.j] : 0.0;
             z = w.valid ? Zin[w.j] : 0.0f;
+            float xmn = FLT_MAX, xmx = -FLT_MAX;
 #pragma unroll
-            for (int i = 0; i < E; ++i) ws[i] = __fmul_rn(x[i], s);
+            for (int i = 0; i < E; ++i) {
+                ws[i] = __fmul_rn(x[i], s);
+                xmn = fminf(xmn, x[i]);
+                xmx = fmaxf(xmx, x[i]);
+            }
+            lmin = w.valid ? __fmul_rn(xmn, s) : 0.0f;
+            lmax = w.valid ? __fmul_rn(xmx, s) : 0.0f;
         }
         const float spow = pow_pos(s, -k.p);
+        const F2 sws2 = split_f2(sws);
 #pragma unroll
         for (int q = 0; q < kChunkMax; ++q) {
             if (q < nk) {
                 float err, sq;
                 bool sp;
                 double swe;
-                eval_lane_reload<DT, AXIS, E>(k, w, ws, s, z, z0, betaq[q], thrq[q], &err, &sq, &sp, &swe);
+                eval_lane_reload<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z, z0, k0 + q, thrq[q], &err, &sq, &sp,
+                                              &swe);
                 if (w.valid && w.part == 0) acc[q] += static_cast<double>(err * spow);
-                z = zero_from_sums(sq, sp ? swe : sws, k.g);
+                z = sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, sws2, inv_g);
             }
         }
         if (w.valid && w.part == 0) Zout[w.j] = z;
@@ -1129,8 +1190,15 @@ cudaError_t launch_reg(KParams& k, cudaStream_t stream, int* grid) {
     return cudaSuccess;
 }
 
+// The register kernel holds a whole group per thread up to g = 32 (E = g,
+// P = 1): every lane then has E independent elements per iteration and the
+// group sums need no shuffles; larger groups spread over P = g/32 lanes.
 template <int DT, int AXIS>
 cudaError_t launch_reg_e(KParams& k, cudaStream_t stream, int* grid) {
+    k.E = k.g < 32 ? k.g : 32;
+    k.P = k.g / k.E;
+    k.logP = 0;
+    while ((1 << k.logP) < k.P) ++k.logP;
     if (k.E == 8) return launch_reg<DT, AXIS, 8>(k, stream, grid);
     if (k.E == 16) return launch_reg<DT, AXIS, 16>(k, stream, grid);
     return launch_reg<DT, AXIS, 32>(k, stream, grid);
