@@ -667,47 +667,60 @@ __device__ __forceinline__ float beta_at(const KParams& k, int it) {
     return b;
 }
 
-// eval_lane without the raw values in registers: the rare shrink path reloads them.
+// Slow path of one evaluation for one lane: a group that needs the clamp or
+// may have a non-zero proximal step (rare).  The lane's raw values are reloaded and ws = fl(w*s) recomputed (the
+// same product as at init); returns the lane's partial sums of |r|^p, W_q and
+// (when sp) fl((w - W_e)*s).
+template <int DT, int AXIS, int E>
+__device__ __forceinline__ float3 eval_lane_slow(const KParams k, const WarpTile w, float s, float z, int it, bool sp,
+                                              double* swe_out) {
+    float x[E];
+    load_lane<DT, AXIS, E>(k, w, x);
+    float err = 0.0f, sq = 0.0f;
+    double swe = 0.0;
+    const float beta = beta_at(k, it);
+#pragma unroll 4
+    for (int i = 0; i < E; ++i) {
+        const ElemEval ee = eval_elem(__fmul_rn(x[i], s), z, k.Lf);
+        err += pow_pos(fabsf(ee.r), k.p);
+        sq += ee.q;
+        if (sp) {
+            const float we = shrink_elem(ee.r, s, k.p, beta);
+            swe += static_cast<double>(__fmul_rn(__fsub_rn(x[i], we), s));
+        }
+    }
+    *swe_out = swe;
+    return make_float3(err, sq, 0.0f);
+}
+
+// One evaluation of zero-point z for a warp tile whose raw values are not kept
+// in registers.  Fast path (warp-uniform): every group clamp-free and no
+// proximal step possible -- then only v, round, r, |r|^p and W_q per element.
 template <int DT, int AXIS, int E>
 __device__ __forceinline__ void eval_lane_reload(const KParams& k, const WarpTile& w, const float* ws, float lmin,
                                                  float lmax, float s, float z, float z0, int it, float thr,
                                                  float* err_out, float* sq_out, bool* sp_out, double* swe_out) {
-    float err = 0.0f, sq = 0.0f;
     const bool sp = w.valid && shrink_possible(s, z, z0, thr, k.Lf);
-    if (__all_sync(kFull, !w.valid || clamp_free(lmin, lmax, z, k.Lf))) {
+    const bool fast = __all_sync(kFull, !w.valid || (!sp && clamp_free(lmin, lmax, z, k.Lf)));
+    float err = 0.0f, sq = 0.0f;
+    double swe = 0.0;
+    if (fast) {
         if (w.valid) {
 #pragma unroll
             for (int i = 0; i < E; ++i) {
-                const ElemEval ee = eval_elem_nc(ws[i], z);
-                err += pow_pos(fabsf(ee.r), k.p);
-                sq += ee.q;
+                const ElemEval e = eval_elem_nc(ws[i], z);
+                err += pow_pos(fabsf(e.r), k.p);
+                sq += e.q;
             }
         }
     } else if (w.valid) {
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-            const ElemEval ee = eval_elem(ws[i], z, k.Lf);
-            err += pow_pos(fabsf(ee.r), k.p);
-            sq += ee.q;
-        }
+        const float3 r = eval_lane_slow<DT, AXIS, E>(k, w, s, z, it, sp, &swe);
+        err = r.x;
+        sq = r.y;
     }
     *err_out = seg_sum(err, k.P);
     *sq_out = seg_sum(sq, k.P);
-    double swe = 0.0;
-    if (__any_sync(kFull, sp)) {
-        if (sp) {
-            const float beta = beta_at(k, it);
-            float x[E];
-            load_lane<DT, AXIS, E>(k, w, x);
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                const ElemEval ee = eval_elem(ws[i], z, k.Lf);
-                const float we = shrink_elem(ee.r, s, k.p, beta);
-                swe += static_cast<double>(__fmul_rn(__fsub_rn(x[i], we), s));
-            }
-        }
-        swe = seg_sum_d(swe, k.P);
-    }
+    if (__any_sync(kFull, sp)) swe = seg_sum_d(swe, k.P);
     *sp_out = sp;
     *swe_out = swe;
 }
@@ -746,6 +759,20 @@ __device__ __forceinline__ float step_lane(const KParams& k, bool valid, const f
     return sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, split_f2(sws), 1.0f / static_cast<float>(k.g));
 }
 
+// One tensor-mode iteration of a warp tile: evaluate z, add this group's
+// error term to its per-thread partial, step z.
+template <int DT, int AXIS, int E>
+__device__ __forceinline__ void tensor_iteration(const KParams& k, const WarpTile& w, const float* ws, float lmin,
+                                                 float lmax, float s, float z0, int it, float thr, float spow,
+                                                 F2 sws2, float inv_g, double& acc, float& z) {
+    float err, sq;
+    bool sp;
+    double swe;
+    eval_lane_reload<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z, z0, it, thr, &err, &sq, &sp, &swe);
+    if (w.valid && w.part == 0) acc += static_cast<double>(err * spow);
+    z = sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, sws2, inv_g);
+}
+
 __device__ __forceinline__ double warp_sum_d(double x) {
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
     return x;
@@ -755,7 +782,8 @@ template <int DT, int AXIS, int E, int MODE>
 __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2)
     solve_reg_kernel(const KParams k, int chunk) {
     __shared__ float2 sred[kRegWarps];
-    __shared__ double sacc[kChunkMax][kRegWarps];
+    __shared__ double sacc[kChunkMax][kRegThreads];  // per-thread tensor error partials
+    __shared__ float sthr[kChunkMax];                 // shrink threshold of each iteration of the chunk
     __shared__ int sflag;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t ntiles = num_warp_tiles<AXIS>(k);
@@ -877,16 +905,11 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2)
     const int nk = k1 - k0;
     float* const Zin = (chunk % 3 == 0) ? Zs0 : (chunk % 3 == 1 ? Zs1 : Zs2);
     float* const Zout = ((chunk + 1) % 3 == 0) ? Zs0 : ((chunk + 1) % 3 == 1 ? Zs1 : Zs2);
-    double acc[kChunkMax] = {0.0, 0.0, 0.0, 0.0};
-    float thrq[kChunkMax];  // shrink threshold of beta_k, the same for every group
-    {
-        float b = beta_at(k, k0);
-#pragma unroll
-        for (int q = 0; q < kChunkMax; ++q) {
-            thrq[q] = shrink_threshold(b, k.p);
-            b = __fmul_rn(b, k.kappa);
-        }
-    }
+    // per-thread tensor error partials: registers for small tiles, else shared
+    double accr[kChunkMax] = {0.0, 0.0, 0.0, 0.0};
+    for (int q = 0; q < kChunkMax; ++q) sacc[q][threadIdx.x] = 0.0;
+    if (threadIdx.x < kChunkMax) sthr[threadIdx.x] = shrink_threshold(beta_at(k, k0 + threadIdx.x), k.p);
+    __syncthreads();
     constexpr bool kPrefetch = AXIS == 1 && E <= 16;
     int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp;
     uint4 raw[kPrefetch ? E / kPiece : 1];
@@ -932,31 +955,32 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2)
         }
         const float spow = pow_pos(s, -k.p);
         const F2 sws2 = split_f2(sws);
+        // small tiles: unrolled over the chunk's iterations (more independent
+        // work in flight); large tiles: a loop, to keep the code cache-resident
+        if constexpr (E <= 16) {
 #pragma unroll
-        for (int q = 0; q < kChunkMax; ++q) {
-            if (q < nk) {
-                float err, sq;
-                bool sp;
-                double swe;
-                eval_lane_reload<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z, z0, k0 + q, thrq[q], &err, &sq, &sp,
-                                              &swe);
-                if (w.valid && w.part == 0) acc[q] += static_cast<double>(err * spow);
-                z = sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, sws2, inv_g);
-            }
+            for (int q = 0; q < kChunkMax; ++q)
+                if (q < nk) tensor_iteration<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z0, k0 + q, sthr[q], spow, sws2,
+                                                          inv_g, accr[q], z);
+        } else {
+#pragma unroll 1
+            for (int q = 0; q < nk; ++q)
+                tensor_iteration<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z0, k0 + q, sthr[q], spow, sws2, inv_g,
+                                              sacc[q][threadIdx.x], z);
         }
         if (w.valid && w.part == 0) Zout[w.j] = z;
     }
-    // per-CTA partials, then the last CTA sums them in a fixed order
+    // per-CTA partials (fixed order), then the last CTA sums them in a fixed order
+    if constexpr (E <= 16) {
 #pragma unroll
-    for (int q = 0; q < kChunkMax; ++q) {
-        const double v = warp_sum_d(acc[q]);
-        if (lane == 0) sacc[q][warp] = v;
+        for (int q = 0; q < kChunkMax; ++q) sacc[q][threadIdx.x] = accr[q];
     }
     __syncthreads();
-    if (threadIdx.x < nk) {
+    for (int q = warp; q < nk; q += kRegWarps) {
         double v = 0.0;
-        for (int w = 0; w < kRegWarps; ++w) v += sacc[threadIdx.x][w];
-        k.tparts[static_cast<size_t>(threadIdx.x) * kMaxPartials + blockIdx.x] = v;
+        for (int i = lane; i < kRegThreads; i += 32) v += sacc[q][i];
+        v = warp_sum_d(v);
+        if (lane == 0) k.tparts[static_cast<size_t>(q) * kMaxPartials + blockIdx.x] = v;
     }
     __threadfence();
     __syncthreads();
