@@ -49,28 +49,12 @@ bool is_device_ptr(const void* p) {
 
 }  // namespace
 
-extern "C" {
+namespace hqq {
 
-size_t hqq_packed_bytes(int64_t rows, int64_t cols, int nbits, int group_size, int axis) {
-    if (!valid_nbits(nbits) || check_shape(rows, cols, group_size, axis) != HQQ_OK) return 0;
-    return static_cast<size_t>(rows * cols * nbits / 8);
-}
-
-int64_t hqq_num_groups(int64_t rows, int64_t cols, int group_size, int axis) {
-    if (check_shape(rows, cols, group_size, axis) != HQQ_OK) return -1;
-    return rows * cols / group_size;
-}
-
-size_t hqq_workspace_bytes(int64_t rows, int64_t cols, int group_size, int axis, int stop_mode, int zero_nbits) {
-    if (check_shape(rows, cols, group_size, axis) != HQQ_OK) return 0;
-    if (stop_mode < 0 || stop_mode > 2 || (zero_nbits != 8 && zero_nbits != 16)) return 0;
-    return hqq::workspace_layout(rows * cols / group_size, stop_mode, zero_nbits, hqq::kMaxIters).total;
-}
-
-int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p,
-                 float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* W_q_packed, void* scale,
-                 void* zero, void* zero_meta, void* workspace, size_t workspace_bytes, int32_t* debug_best_iter,
-                 float* debug_best_err, float* debug_zero_f32, void* stream) {
+int quantize_entry(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p,
+                   float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* W_q_packed, void* scale,
+                   void* zero, void* zero_meta, void* workspace, size_t workspace_bytes, bool allow_slices,
+                   int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32, void* stream) {
     if (dtype != HQQ_F16 && dtype != HQQ_BF16) return HQQ_ERR_DTYPE;
     if (!valid_nbits(nbits)) return HQQ_ERR_INVALID_ARG;
     const int sh = check_shape(rows, cols, group_size, axis);
@@ -82,8 +66,10 @@ int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits
     if (stop_mode < 0 || stop_mode > 2) return HQQ_ERR_INVALID_ARG;
     if (zero_nbits != 8 && zero_nbits != 16) return HQQ_ERR_INVALID_ARG;
     const int64_t G = rows * cols / group_size;
-    const size_t need = hqq::workspace_layout(G, stop_mode, zero_nbits, hqq::kMaxIters).total;
-    if (workspace == nullptr || workspace_bytes < need) return HQQ_ERR_WORKSPACE;
+    const int64_t slice =
+        hqq::fit_slice(rows, cols, group_size, axis, stop_mode, zero_nbits, workspace == nullptr ? 0 : workspace_bytes);
+    const size_t need = hqq::workspace_layout(rows, cols, group_size, axis, stop_mode, zero_nbits, 0).total;
+    if (workspace == nullptr || (!allow_slices && workspace_bytes < need) || slice <= 0) return HQQ_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return HQQ_ERR_ALIGN;
     if (!is_device_ptr(workspace)) return HQQ_ERR_INVALID_ARG;
     if (zero_nbits == 8) {
@@ -123,6 +109,7 @@ int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits
     a.zero = zero;
     a.zero_meta = static_cast<float*>(zero_meta);
     a.ws = static_cast<uint8_t*>(workspace);
+    a.slice = slice;
     a.dbg_iter = debug_best_iter;
     a.dbg_err = debug_best_err;
     a.dbg_zero = debug_zero_f32;
@@ -132,6 +119,35 @@ int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits
         return HQQ_ERR_CUDA;
     }
     return HQQ_OK;
+}
+
+}  // namespace hqq
+
+extern "C" {
+
+size_t hqq_packed_bytes(int64_t rows, int64_t cols, int nbits, int group_size, int axis) {
+    if (!valid_nbits(nbits) || check_shape(rows, cols, group_size, axis) != HQQ_OK) return 0;
+    return static_cast<size_t>(rows * cols * nbits / 8);
+}
+
+int64_t hqq_num_groups(int64_t rows, int64_t cols, int group_size, int axis) {
+    if (check_shape(rows, cols, group_size, axis) != HQQ_OK) return -1;
+    return rows * cols / group_size;
+}
+
+size_t hqq_workspace_bytes(int64_t rows, int64_t cols, int group_size, int axis, int stop_mode, int zero_nbits) {
+    if (check_shape(rows, cols, group_size, axis) != HQQ_OK) return 0;
+    if (stop_mode < 0 || stop_mode > 2 || (zero_nbits != 8 && zero_nbits != 16)) return 0;
+    return hqq::workspace_layout(rows, cols, group_size, axis, stop_mode, zero_nbits, 0).total;
+}
+
+int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p,
+                 float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* W_q_packed, void* scale,
+                 void* zero, void* zero_meta, void* workspace, size_t workspace_bytes, int32_t* debug_best_iter,
+                 float* debug_best_err, float* debug_zero_f32, void* stream) {
+    return hqq::quantize_entry(W, rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
+                               zero_nbits, W_q_packed, scale, zero, zero_meta, workspace, workspace_bytes, false,
+                               debug_best_iter, debug_best_err, debug_zero_f32, stream);
 }
 
 int hqq_dequantize(const void* W_q_packed, const void* scale, const void* zero, const void* zero_meta, int64_t rows,

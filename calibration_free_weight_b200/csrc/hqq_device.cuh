@@ -90,8 +90,12 @@ __device__ __forceinline__ bool clamp_free(float wsmin, float wsmax, float z, fl
     return __fadd_rn(wsmin, z) >= -0.5f && __fadd_rn(wsmax, z) < Lf + 0.5f;
 }
 
-// Compensated (TwoSum) fp32 accumulation: hi + lo carries the running sum of
-// fp32 terms to ~2^-48 relative, so no per-term conversion to fp64 is needed.
+// Compensated (TwoSum) fp32 accumulation: every rounding error of the running
+// sum is formed exactly and collected in lo, so hi + lo carries the sum of the
+// fp32 terms to ~n^2 * 2^-48 of it (Kahan's compensation is not enough here: it
+// leaves an error of order 2^-23 of the sum of magnitudes, which can move z by
+// an ulp, flip a code and change the whole trajectory).  No per-term
+// conversion to fp64 (an XU-pipe op on this GPU) is needed.
 __device__ __forceinline__ void two_sum_acc(float& hi, float& lo, float x) {
     const float s = __fadd_rn(hi, x);
     const float bp = __fsub_rn(s, hi);
@@ -188,32 +192,6 @@ __device__ __forceinline__ void unpack8(const uint4 u, float* w) {
     }
 }
 
-// ----------------------------------------------------------- packing -----
-
-// Eight codes, LSB first, nbits each.
-__device__ __forceinline__ uint64_t pack8(const uint32_t* c, int nbits) {
-    uint64_t v = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v |= static_cast<uint64_t>(c[i]) << (i * nbits);
-    return v;
-}
-
-// Store the nbits bytes of one packed 8-element piece (dst aligned to nbits
-// bytes for nbits in {1,2,4,8}; byte stores for 3).
-__device__ __forceinline__ void store_piece(uint8_t* dst, uint64_t v, int nbits) {
-    switch (nbits) {
-        case 1: *dst = static_cast<uint8_t>(v); break;
-        case 2: *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(v); break;
-        case 4: *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(v); break;
-        case 8: *reinterpret_cast<uint64_t*>(dst) = v; break;
-        default:
-            dst[0] = static_cast<uint8_t>(v);
-            dst[1] = static_cast<uint8_t>(v >> 8);
-            dst[2] = static_cast<uint8_t>(v >> 16);
-            break;
-    }
-}
-
 __device__ __forceinline__ uint16_t half_bits(float x) { return __half_as_ushort(__float2half_rn(x)); }
 
 // --------------------------------------------------------- async copy ----
@@ -234,6 +212,7 @@ struct KParams {
     int64_t rows, cols, G;
     int g, P, logP, E, nbits, iters, iters_eff, stop_mode, zero_nbits, axis;
     float p, beta, kappa, Lf;
+    float beta_last;     // beta of the last iteration (sequential fp32 products)
     int64_t n;  // rows * cols
     uint8_t* packed;
     uint16_t* scale;
@@ -242,8 +221,7 @@ struct KParams {
     float* dbg_err;
     float* dbg_zero;
     // workspace
-    uint32_t* counters;  // [0] status, [1] work counter, [2] CTA ticket
-    float2* minmax;      // per-CTA zero min/max
+    uint32_t* counters;  // workspace header words (status, CTA ticket, zero range, pass counts)
     double* tparts;      // per-iteration per-CTA tensor error partials [iters][kMaxPartials]
     double* etot;        // per-iteration tensor mean error [iters]
     float* zbest_ws;     // fp32 kept zero (8-bit zero path)
@@ -251,9 +229,6 @@ struct KParams {
     float* t_z0;
     double* t_sws;
     float* t_zs;
-    // pool kernel geometry
-    int NC;              // cells per warp
-    int pool_warp_bytes;
 };
 
 }  // namespace hqq

@@ -9,27 +9,38 @@
 namespace hqq {
 
 constexpr int kPiece = 8;            // elements per 16-byte piece of 16-bit data
-constexpr int kMaxPartials = 4096;   // per-CTA partial slots in the workspace
+constexpr int kMaxPartials = 4096;   // per-CTA partial slots in the workspace (tensor mode)
+constexpr int64_t kMinSlice = 4096;  // smallest group-mode slice (entries) a workspace may be cut into
 constexpr int kMaxIters = 1000;      // upper bound on iters (argument check)
 constexpr float kScaleCap = 2.0e4f;  // cap on s (and on the 8-bit zero quantiser's scale)
 
 // Workspace layout (offsets 256-byte aligned):
-//   header      256 B: status word, CTA ticket, 64-bit work counter
-//   minmax      float2[kMaxPartials]   per-CTA min/max of the kept zeros
+//   header      256 B: status word, CTA ticket, kept-zero range, pass counts
 //   zbest       float[G]               kept zeros (8-bit zero path)
+//   group / no stop, per slice of S entries (a warp-tile slot each; S = all
+//   entries unless the workspace is smaller):
+//                state float4[2][S], state_it int[S], survivor lists u32[2][S]
 //   tensor mode: tparts double[4][kMaxPartials], etot double[kMaxIters],
 //                s f32[G], z0 f32[G], sum w*s f64[G], chunk-start zeros f32[3][G]
 struct WorkspaceLayout {
-    size_t header, minmax, zbest, tparts, etot, t_s, t_z0, t_sws, t_zs, total;
+    size_t header, zbest, state, state_it, list0, list1, tparts, etot, t_s, t_z0, t_sws, t_zs, total;
+    int64_t slice;  // group mode: entries per slice
 };
-WorkspaceLayout workspace_layout(int64_t G, int stop_mode, int zero_nbits, int iters);
+// slice <= 0: one slice holding every entry.
+WorkspaceLayout workspace_layout(int64_t rows, int64_t cols, int g, int axis, int stop_mode, int zero_nbits,
+                                 int64_t slice);
+// Group mode: the largest slice whose layout fits in `bytes` (0 if none of at
+// least kMinSlice entries does); every entry if the full layout fits.
+int64_t fit_slice(int64_t rows, int64_t cols, int g, int axis, int stop_mode, int zero_nbits, size_t bytes);
 
 struct Geometry {
-    int g;  // group size
-    int E;  // elements per lane
-    int P;  // lanes per group (g / E, <= 32)
+    int g;     // group size
+    int E;     // elements per lane: min(g, 32)
+    int P;     // lanes per group: g / E
+    int logP;
 };
 Geometry make_geometry(int g);
+int64_t group_entries(int64_t rows, int64_t cols, int g, int axis);  // warp-tile slots over all groups
 
 struct SolveArgs {
     const void* W;
@@ -41,6 +52,7 @@ struct SolveArgs {
     void* zero;        // fp16 bits or uint8
     float* zero_meta;  // fp32[2] or null
     uint8_t* ws;       // workspace base
+    int64_t slice;     // group mode: entries per slice (from the workspace layout)
     int32_t* dbg_iter;
     float* dbg_err;
     float* dbg_zero;
@@ -59,5 +71,12 @@ struct DequantArgs {
 // Launchers: return cudaSuccess or the launch error.
 cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream);
 cudaError_t launch_dequant(const DequantArgs& a, cudaStream_t stream);
+
+// hqq_quantize with an option to cut group-mode work into slices that fit a
+// smaller workspace (used by hqq_quantize_noalloc).
+int quantize_entry(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p,
+                   float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* W_q_packed, void* scale,
+                   void* zero, void* zero_meta, void* workspace, size_t workspace_bytes, bool allow_slices,
+                   int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32, void* stream);
 
 }  // namespace hqq

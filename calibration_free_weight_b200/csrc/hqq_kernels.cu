@@ -9,28 +9,29 @@
 // the per-element evaluation is in hqq_device.cuh.
 //
 // The path has no dense contraction: no tensor cores.  Each element and
-// iteration costs ~8 FP32-pipe instructions and two MUFU ops (|r|^p through
+// evaluation costs ~7 FP32-pipe instructions and two MUFU ops (|r|^p through
 // lg2/ex2), so the MUFU pipe, not HBM, bounds the solver.
 //
-// solve_pool_kernel (group / no stop, axis 1): every warp owns a pool of
-//   "cells" in shared memory, one group each.  Per round it (A) packs and
-//   stores the groups that finished, (B) refills free cells with the next
-//   groups of a global work counter by cp.async (16-byte copies straight into
-//   shared memory), (C) waits for the copies issued one round earlier,
-//   (D) initialises those groups (min/max -> s, z0; w*s stored as fp32; sum
-//   of w*s in fp64) and (E) evaluates every active group once, mapping each
-//   onto P = g/E consecutive lanes after a ballot compaction.  Early-stopped
-//   groups free their lanes at once; warps never wait on each other.
-// solve_reg_kernel: a warp holds 32/P whole groups in registers.
-//   MODE_LOCAL (group / no stop, any axis): iterates until every group of the
-//   warp tile has stopped (used for axis 0).
-//   MODE_TENSOR: runs iterations [k0, k1) of every group, accumulates the
-//   per-iteration tensor error in fp64 per CTA, and the last CTA to finish
-//   (atomic ticket) sums the partials in a fixed order.  The next launch
-//   reads those sums, applies the stop rule, and either runs the next chunk
-//   or writes the final codes with the kept iterate (recomputed from the
-//   stored chunk-start zero with the cheap part of the iteration).  No CTA
-//   ever waits for another.
+// Both solver kernels hold a warp tile of 32/P groups in registers, E = g/P
+// elements per lane (E = min(g, 32)), and re-read W from HBM rather than keep
+// a second copy on chip; no CTA ever waits for another.
+//
+// solve_group_kernel (group / no stop, both axes): a sequence of passes.  Pass
+//   0 initialises every group (min/max -> s, z0; fp32 w*s; sum of w*s) and runs
+//   up to m_0 evaluations; a group that stops is packed and stored at once, a
+//   group still running leaves its state (z, best error, kept zero, s, z0,
+//   max w*s, sum of w*s) in the workspace and its index in a survivor list
+//   (warp-aggregated atomic append).  Pass p runs the survivors of pass p-1
+//   for m_p more evaluations.  Every group in a pass has done the same number
+//   of iterations, so the iteration index and beta are warp-uniform, and the
+//   lanes of a warp stay busy: a tile only runs as long as its slowest group
+//   within one pass.
+// solve_tensor_kernel (tensor stop): runs iterations [k0, k1) of every group,
+//   accumulates the per-iteration tensor error in fp64 per CTA, and the last
+//   CTA to finish (atomic ticket) sums the partials in a fixed order.  The next
+//   launch reads those sums, applies the stop rule, and either runs the next
+//   chunk or writes the final codes with the kept iterate (recomputed from the
+//   stored chunk-start zero with the cheap part of the iteration).
 
 #include "hqq_device.cuh"
 
@@ -40,13 +41,16 @@ namespace {
 
 using namespace dev;
 
-constexpr int kPoolWarps = 4;
-constexpr int kPoolThreads = kPoolWarps * 32;
 constexpr int kRegThreads = 256;
 constexpr int kRegWarps = kRegThreads / 32;
 constexpr int kChunkMax = 4;  // iterations per tensor-mode launch (after the first, which has 2)
 
-enum : uint8_t { kEmpty = 0, kLoading = 1, kActive = 2, kDone = 3 };
+// Header words of the workspace (uint32 index); word 0 is the status word.
+constexpr int kWordTicket = 1;
+constexpr int kWordZmin = 2;   // ~key(min kept zero), by atomicMax
+constexpr int kWordZmax = 3;   // key(max kept zero), by atomicMax
+constexpr int kWordPass = 8;   // survivor count of group pass p at kWordPass + p
+constexpr int kMaxPasses = 16;
 
 // ------------------------------------------------------- group outputs ----
 
@@ -65,9 +69,20 @@ __device__ __forceinline__ void store_group(const KParams& k, int64_t j, float s
     if (k.dbg_zero) k.dbg_zero[j] = zb;
 }
 
-// Block-wide min/max of the kept zeros -> one partial per CTA.
+// Order-preserving key of a float (x < y <=> key(x) < key(y) as unsigned).
+__device__ __forceinline__ uint32_t order_key(float x) {
+    const uint32_t b = __float_as_uint(x);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+// Block-wide min/max of the kept zeros, merged into the workspace header by
+// two atomics per CTA (exact and order-independent, so launches and slices
+// can all contribute).  The header starts at zero: the neutral element of both.
 template <int NW>
-__device__ __forceinline__ void write_minmax(const KParams& k, float zmin, float zmax, float2* sred) {
+__device__ __forceinline__ void merge_zero_range(const KParams& k, float zmin, float zmax, float2* sred) {
     for (int o = 16; o > 0; o >>= 1) {
         zmin = fminf(zmin, __shfl_xor_sync(kFull, zmin, o));
         zmax = fmaxf(zmax, __shfl_xor_sync(kFull, zmax, o));
@@ -81,436 +96,14 @@ __device__ __forceinline__ void write_minmax(const KParams& k, float zmin, float
             r.x = fminf(r.x, sred[w].x);
             r.y = fmaxf(r.y, sred[w].y);
         }
-        k.minmax[blockIdx.x] = r;
-    }
-}
-
-// ============================================================ pool kernel ==
-
-// Per-warp pool layout (NC cells).  A cell holds one group: CS = g + 4 floats
-// (the 16-byte pad staggers consecutive cells across shared-memory banks).
-// Before initialisation the raw 16-bit group is staged in the top 2g bytes of
-// the cell by cp.async; initialisation overwrites the cell with fp32 w*s.
-struct Pool {
-    float* data;
-    float4* zs4;  // (z, s, z0, flags): what every lane of a group reads per evaluation
-    float2* sws;  // sum of w*s as a float pair (hi, lo)
-    int64_t* gidx;
-    float *be, *zb, *beta, *wsmax;
-    int *kk, *bi, *issued;
-    uint8_t *st, *list;
-};
-
-__host__ __device__ inline int pool_cell_floats(int g) { return g + 4; }
-
-__host__ __device__ inline int pool_warp_bytes(int NC, int g) {
-    const int b = NC * (4 * pool_cell_floats(g) + 16 + 8 + 8 + 4 * 4 + 3 * 4 + 2);
-    return (b + 15) & ~15;
-}
-
-__device__ __forceinline__ Pool carve_pool(unsigned char* base, int NC, int g) {
-    Pool m;
-    size_t off = 0;
-    m.data = reinterpret_cast<float*>(base + off);
-    off += static_cast<size_t>(NC) * pool_cell_floats(g) * 4;
-    m.zs4 = reinterpret_cast<float4*>(base + off);
-    off += NC * 16;
-    m.sws = reinterpret_cast<float2*>(base + off);
-    off += NC * 8;
-    m.gidx = reinterpret_cast<int64_t*>(base + off);
-    off += NC * 8;
-    float* f = reinterpret_cast<float*>(base + off);
-    m.be = f;
-    m.zb = f + NC;
-    m.beta = f + 2 * NC;
-    m.wsmax = f + 3 * NC;
-    off += NC * 4 * 4;
-    int* iv = reinterpret_cast<int*>(base + off);
-    m.kk = iv;
-    m.bi = iv + NC;
-    m.issued = iv + 2 * NC;
-    off += NC * 3 * 4;
-    m.st = base + off;
-    m.list = base + off + NC;
-    return m;
-}
-
-// Ordered list of the cells whose predicate holds (a: cell lane, b: cell lane+32).
-__device__ __forceinline__ int make_list(bool a, bool b, uint8_t* list) {
-    const int lane = threadIdx.x & 31;
-    const unsigned lo = __ballot_sync(kFull, a), hi = __ballot_sync(kFull, b);
-    const unsigned below = (1u << lane) - 1u;
-    const int nlo = __popc(lo);
-    if (a) list[__popc(lo & below)] = static_cast<uint8_t>(lane);
-    if (b) list[nlo + __popc(hi & below)] = static_cast<uint8_t>(lane + 32);
-    __syncwarp();
-    return nlo + __popc(hi);
-}
-
-__device__ __forceinline__ float* cell_ptr(const Pool& m, int c, int g) {
-    return m.data + static_cast<size_t>(c) * pool_cell_floats(g);
-}
-
-// The 8 fp32 values of piece pc of cell c.
-__device__ __forceinline__ void load_ws8(const float* cell, int pc, float* ws) {
-    const float4* p = reinterpret_cast<const float4*>(cell + pc * kPiece);
-    const float4 a = p[0], b = p[1];
-    ws[0] = a.x;
-    ws[1] = a.y;
-    ws[2] = a.z;
-    ws[3] = a.w;
-    ws[4] = b.x;
-    ws[5] = b.y;
-    ws[6] = b.z;
-    ws[7] = b.w;
-}
-
-// Eight codes, LSB first, NBITS each (32-bit arithmetic when they fit).
-template <int NBITS>
-__device__ __forceinline__ void store_piece_t(uint8_t* dst, const uint32_t* c) {
-    if (NBITS == 8) {
-        uint2 v;
-        v.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-        v.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-        *reinterpret_cast<uint2*>(dst) = v;
-    } else {
-        uint32_t v = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v |= c[i] << (i * NBITS);
-        if (NBITS == 4) *reinterpret_cast<uint32_t*>(dst) = v;
-        else if (NBITS == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(v);
-        else if (NBITS == 1) *dst = static_cast<uint8_t>(v);
-        else {
-            dst[0] = static_cast<uint8_t>(v);
-            dst[1] = static_cast<uint8_t>(v >> 8);
-            dst[2] = static_cast<uint8_t>(v >> 16);
+        if (r.x <= r.y) {  // this CTA stored at least one zero
+            atomicMax(k.counters + kWordZmin, ~order_key(r.x));
+            atomicMax(k.counters + kWordZmax, order_key(r.y));
         }
     }
 }
 
-constexpr unsigned kFlagShrink = 1u;  // the proximal step may be non-zero
-constexpr unsigned kFlagClamp = 2u;   // some v may leave [-0.5, L + 0.5)
-
-// Flags of the next evaluation of a group at zero-point z (v = fl(ws + z) with
-// ws in [-z0, wsmax]: fl(min w * s) = -z0 exactly).
-__device__ __forceinline__ float eval_flags(float s, float z, float z0, float wsmax, float thr, float Lf) {
-    unsigned f = 0;
-    if (shrink_possible(s, z, z0, thr, Lf)) f |= kFlagShrink;
-    if (!clamp_free(-z0, wsmax, z, Lf)) f |= kFlagClamp;
-    return __uint_as_float(f);
-}
-
-// Group-level decision after evaluating zero-point z (one lane per group):
-// keep the best iterate, apply the stop rule, compute the next zero-point and
-// the flags of its evaluation.
-__device__ __forceinline__ void decide(const KParams& k, const Pool& m, int c, bool stop_group, float err, float sq,
-                                       bool sp, double swe, float z, float s, float z0, float beta, int kk) {
-    const bool improved = err < m.be[c];
-    if (improved) {
-        m.be[c] = err;
-        m.zb[c] = z;
-        m.bi[c] = kk;
-    }
-    bool stop = (stop_group && !improved) || kk >= k.iters_eff - 1;
-    if (!stop) {
-        const float2 f = m.sws[c];
-        const float zn = sp ? zero_from_sums(sq, swe, k.g)
-                            : zero_from_sums_f2(sq, F2{f.x, f.y}, 1.0f / static_cast<float>(k.g));
-        if (stop_group && zn == z) {
-            stop = true;  // fixed point: the next error would equal this one
-        } else {
-            const float nbeta = __fmul_rn(beta, k.kappa);
-            m.zs4[c] = make_float4(zn, s, z0, eval_flags(s, zn, z0, m.wsmax[c], shrink_threshold(nbeta, k.p), k.Lf));
-            m.kk[c] = kk + 1;
-            m.beta[c] = nbeta;
-        }
-    }
-    m.st[c] = stop ? kDone : kActive;
-}
-
-template <int DT, int E, int NBITS>
-__global__ void __launch_bounds__(kPoolThreads, 6) solve_pool_kernel(const KParams k) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    __shared__ float2 sred[kPoolWarps];
-    constexpr int NPL = E / kPiece;  // pieces per lane
-    constexpr float Lf = static_cast<float>((1 << NBITS) - 1);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int NC = k.NC, g = k.g, P = k.P, logP = k.logP;
-    const int ppg = g / kPiece;  // pieces (16-byte raw copies) per group
-    const Pool m = carve_pool(smem_raw + static_cast<size_t>(warp) * k.pool_warp_bytes, NC, g);
-    const bool stop_group = k.stop_mode == 0;
-    const float thr0 = shrink_threshold(k.beta, k.p);
-    unsigned long long* work = reinterpret_cast<unsigned long long*>(k.counters + 2);
-    float zmin = FLT_MAX, zmax = -FLT_MAX;
-    int64_t qn = 0, qe = 0;
-    bool exhausted = false;
-
-    if (lane < NC) m.st[lane] = kEmpty;
-    if (lane + 32 < NC) m.st[lane + 32] = kEmpty;
-    __syncwarp();
-
-    for (int round = 0;; ++round) {
-        // (A) pack and store the groups that finished
-        {
-            const bool a = lane < NC && m.st[lane] == kDone;
-            const bool b = lane + 32 < NC && m.st[lane + 32] == kDone;
-            const int items = make_list(a, b, m.list) << logP;
-            for (int it = lane; it < items; it += 32) {
-                const int c = m.list[it >> logP], part = it & (P - 1);
-                const int64_t j = m.gidx[c];
-                const float zb = m.zb[c];
-                const float* cell = cell_ptr(m, c, g);
-#pragma unroll
-                for (int t = 0; t < NPL; ++t) {
-                    const int pc = part + t * P;
-                    float ws[8];
-                    uint32_t code[8];
-                    load_ws8(cell, pc, ws);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) round_clamp(__fadd_rn(ws[i], zb), Lf, &code[i]);
-                    store_piece_t<NBITS>(k.packed + (j * ppg + pc) * NBITS, code);
-                }
-                if (part == 0) {
-                    const float s = m.zs4[c].y;
-                    const float err = m.be[c] * pow_pos(s, -k.p) / static_cast<float>(g);
-                    store_group(k, j, s, zb, m.bi[c], err, &zmin, &zmax);
-                }
-            }
-            __syncwarp();
-            if (a) m.st[lane] = kEmpty;
-            if (b) m.st[lane + 32] = kEmpty;
-            __syncwarp();
-        }
-        // (B) refill free cells from the work counter and start their copies
-        {
-            const bool a = lane < NC && m.st[lane] == kEmpty;
-            const bool b = lane + 32 < NC && m.st[lane + 32] == kEmpty;
-            const unsigned lo = __ballot_sync(kFull, a), hi = __ballot_sync(kFull, b);
-            const int nf = __popc(lo) + __popc(hi);
-            const int avail = static_cast<int>(qe - qn);
-            int64_t q2 = 0;
-            int avail2 = 0;
-            if (nf > avail && !exhausted) {
-                unsigned long long base = 0;
-                if (lane == 0) base = atomicAdd(work, static_cast<unsigned long long>(NC));
-                base = __shfl_sync(kFull, base, 0);
-                if (static_cast<int64_t>(base) >= k.G) {
-                    exhausted = true;
-                } else {
-                    q2 = static_cast<int64_t>(base);
-                    const int64_t left = k.G - q2;
-                    avail2 = left < NC ? static_cast<int>(left) : NC;
-                }
-            }
-            const unsigned below = (1u << lane) - 1u;
-            const int ra = __popc(lo & below), rb = __popc(lo) + __popc(hi & below);
-            bool la = false, lb = false;
-            if (a && ra < avail + avail2) {
-                m.gidx[lane] = ra < avail ? qn + ra : q2 + (ra - avail);
-                m.st[lane] = kLoading;
-                m.issued[lane] = round;
-                la = true;
-            }
-            if (b && rb < avail + avail2) {
-                m.gidx[lane + 32] = rb < avail ? qn + rb : q2 + (rb - avail);
-                m.st[lane + 32] = kLoading;
-                m.issued[lane + 32] = round;
-                lb = true;
-            }
-            const int used = nf < avail + avail2 ? nf : avail + avail2;
-            if (used <= avail) {
-                qn += used;
-            } else {
-                qn = q2 + (used - avail);
-                qe = q2 + avail2;
-            }
-            const int copies = make_list(la, lb, m.list) * ppg;
-            for (int it = lane; it < copies; it += 32) {
-                const int c = m.list[it / ppg], pc = it % ppg;
-                const uint16_t* src = k.W + m.gidx[c] * g + pc * kPiece;
-                unsigned char* dst = reinterpret_cast<unsigned char*>(cell_ptr(m, c, g)) + 2 * g + 16 + pc * 16;
-                cp_async16(dst, src);
-            }
-        }
-        cp_async_commit();
-        // (C) copies issued one round earlier have landed
-        cp_async_wait_prev();
-        __syncwarp();
-        // (D) initialise those groups and evaluate their first zero-point z0
-        {
-            const bool a = lane < NC && m.st[lane] == kLoading && m.issued[lane] < round;
-            const bool b = lane + 32 < NC && m.st[lane + 32] == kLoading && m.issued[lane + 32] < round;
-            const int items = make_list(a, b, m.list) << logP;
-            for (int base = 0; base < items; base += 32) {
-                const int it = base + lane;
-                const bool valid = it < items;
-                const int c = valid ? m.list[it >> logP] : 0;
-                const int part = it & (P - 1);
-                float* cell = cell_ptr(m, c, g);
-                const unsigned char* stage = reinterpret_cast<const unsigned char*>(cell) + 2 * g + 16;
-                float w[E];
-                float mn = FLT_MAX, mx = -FLT_MAX;
-#pragma unroll
-                for (int i = 0; i < E; ++i) w[i] = 0.0f;
-                if (valid) {
-#pragma unroll
-                    for (int t = 0; t < NPL; ++t)
-                        unpack8<DT>(*reinterpret_cast<const uint4*>(stage + (part + t * P) * 16), w + t * kPiece);
-#pragma unroll
-                    for (int i = 0; i < E; ++i) {
-                        mn = fminf(mn, w[i]);
-                        mx = fmaxf(mx, w[i]);
-                    }
-                }
-                mn = seg_min(mn, P);
-                mx = seg_max(mx, P);
-                float s = kScaleCap;
-                if (mx > mn) s = fminf(__fdiv_rn(Lf, __fsub_rn(mx, mn)), kScaleCap);
-                const float z0 = __fmul_rn(-mn, s);
-                float hi = 0.0f, lo = 0.0f;
-                float ws[E];
-                float err = 0.0f, sq = 0.0f;
-#pragma unroll
-                for (int i = 0; i < E; ++i) {
-                    ws[i] = __fmul_rn(w[i], s);
-                    two_sum_acc(hi, lo, ws[i]);
-                    // at z0 every v lies in [0, L]: fl(min w * s) + z0 = 0, fl(max w * s) + z0 <= L
-                    const ElemEval ee = eval_elem_nc(ws[i], z0);
-                    err += pow_pos(fabsf(ee.r), k.p);
-                    sq += ee.q;
-                }
-                double acc = static_cast<double>(hi) + static_cast<double>(lo);
-                if (!valid) err = sq = 0.0f, acc = 0.0;
-                acc = seg_sum_d(acc, P);
-                err = seg_sum(err, P);
-                sq = seg_sum(sq, P);
-                const bool sp = valid && k.iters_eff > 1 && shrink_possible(s, z0, z0, thr0, Lf);
-                double swe = 0.0;
-                if (__any_sync(kFull, sp)) {  // rare: re-read the staged raw values (still intact here)
-                    if (sp) {
-#pragma unroll
-                        for (int t = 0; t < NPL; ++t) {
-                            float x[8];
-                            unpack8<DT>(*reinterpret_cast<const uint4*>(stage + (part + t * P) * 16), x);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const ElemEval ee = eval_elem(ws[t * 8 + i], z0, Lf);
-                                const float we = shrink_elem(ee.r, s, k.p, k.beta);
-                                swe += static_cast<double>(__fmul_rn(__fsub_rn(x[i], we), s));
-                            }
-                        }
-                    }
-                    swe = seg_sum_d(swe, P);
-                }
-                __syncwarp();  // every lane has read its raw data before any fp32 write below
-                if (valid) {
-#pragma unroll
-                    for (int t = 0; t < NPL; ++t) {
-                        float4* dst = reinterpret_cast<float4*>(cell + (part + t * P) * kPiece);
-                        dst[0] = make_float4(ws[t * 8 + 0], ws[t * 8 + 1], ws[t * 8 + 2], ws[t * 8 + 3]);
-                        dst[1] = make_float4(ws[t * 8 + 4], ws[t * 8 + 5], ws[t * 8 + 6], ws[t * 8 + 7]);
-                    }
-                    if (part == 0) {
-                        const F2 f = split_f2(acc);
-                        m.sws[c] = make_float2(f.hi, f.lo);
-                        m.zb[c] = z0;
-                        m.bi[c] = 0;
-                        m.wsmax[c] = __fmul_rn(mx, s);
-                        m.zs4[c] = make_float4(z0, s, z0, 0.0f);
-                        if (k.iters_eff == 0) {
-                            m.be[c] = INFINITY;
-                            m.st[c] = kDone;
-                        } else {
-                            m.be[c] = INFINITY;
-                            decide(k, m, c, stop_group, err, sq, sp, swe, z0, s, z0, k.beta, 0);
-                        }
-                    }
-                }
-                __syncwarp();
-            }
-        }
-        // (E) one evaluation of every active group
-        {
-            const bool a = lane < NC && m.st[lane] == kActive;
-            const bool b = lane + 32 < NC && m.st[lane + 32] == kActive;
-            const int items = make_list(a, b, m.list) << logP;
-            for (int base = 0; base < items; base += 32) {
-                const int it = base + lane;
-                const bool valid = it < items;
-                const int c = valid ? m.list[it >> logP] : 0;
-                const int part = it & (P - 1);
-                const float4 st4 = m.zs4[c];
-                const float z = st4.x, s = st4.y, z0 = st4.z;
-                const unsigned flags = valid ? __float_as_uint(st4.w) : 0u;
-                const bool sp = (flags & kFlagShrink) != 0;
-                const float* cell = cell_ptr(m, c, g);
-                float err = 0.0f, sq = 0.0f;
-                if (__all_sync(kFull, (flags & kFlagClamp) == 0)) {
-                    if (valid) {
-#pragma unroll
-                        for (int t = 0; t < NPL; ++t) {
-                            float ws[8];
-                            load_ws8(cell, part + t * P, ws);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const ElemEval ee = eval_elem_nc(ws[i], z);
-                                err += pow_pos(fabsf(ee.r), k.p);
-                                sq += ee.q;
-                            }
-                        }
-                    }
-                } else if (valid) {
-#pragma unroll
-                    for (int t = 0; t < NPL; ++t) {
-                        float ws[8];
-                        load_ws8(cell, part + t * P, ws);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const ElemEval ee = eval_elem(ws[i], z, Lf);
-                            err += pow_pos(fabsf(ee.r), k.p);
-                            sq += ee.q;
-                        }
-                    }
-                }
-                err = seg_sum(err, P);
-                sq = seg_sum(sq, P);
-                double swe = 0.0;
-                float beta = 0.0f;
-                if (__any_sync(kFull, sp)) {  // rare: the proximal step may be non-zero
-                    beta = m.beta[c];
-                    if (sp) {
-                        const int64_t j = m.gidx[c];
-#pragma unroll
-                        for (int t = 0; t < NPL; ++t) {
-                            const int pc = part + t * P;
-                            float ws[8], w[8];
-                            load_ws8(cell, pc, ws);
-                            unpack8<DT>(__ldg(reinterpret_cast<const uint4*>(k.W + j * g + pc * kPiece)), w);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const ElemEval ee = eval_elem(ws[i], z, Lf);
-                                const float we = shrink_elem(ee.r, s, k.p, beta);
-                                swe += static_cast<double>(__fmul_rn(__fsub_rn(w[i], we), s));
-                            }
-                        }
-                    }
-                    swe = seg_sum_d(swe, P);
-                }
-                if (valid && part == 0) decide(k, m, c, stop_group, err, sq, sp, swe, z, s, z0, m.beta[c], m.kk[c]);
-            }
-            __syncwarp();
-        }
-        const bool live = (lane < NC && m.st[lane] != kEmpty) || (lane + 32 < NC && m.st[lane + 32] != kEmpty);
-        if (exhausted && !__any_sync(kFull, live)) break;
-    }
-    cp_async_wait_all();
-    if (k.zero_nbits == 8) write_minmax<kPoolWarps>(k, zmin, zmax, sred);
-}
-
-// ======================================================== register kernel ==
-
-constexpr int MODE_LOCAL = 0;
-constexpr int MODE_TENSOR = 1;
+// ====================================================== register tiles ==
 
 // Chunk schedule of tensor mode: chunk 0 = iterations [0, 2), chunk c >= 1 =
 // [4c - 2, 4c + 2) (clipped to iters).
@@ -573,25 +166,61 @@ __device__ __forceinline__ void load_lane(const KParams& k, const WarpTile& w, f
     }
 }
 
-// Packed codes of this lane's E elements with zero-point z.
-template <int AXIS, int E>
-__device__ __forceinline__ void store_lane_codes(const KParams& k, const WarpTile& w, const float* ws, float z) {
-    if (!w.valid) return;
+// Eight codes, LSB first, NBITS each, as the NBITS bytes of one piece.
+template <int NBITS>
+__device__ __forceinline__ uint64_t pack8_t(const uint32_t* c) {
+    if (NBITS == 8) {
+        const uint32_t lo = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+        const uint32_t hi = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+        return static_cast<uint64_t>(lo) | (static_cast<uint64_t>(hi) << 32);
+    }
+    uint32_t v = 0;  // 8 * NBITS <= 32
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v |= c[i] << (i * NBITS);
+    return v;
+}
+
+template <int AXIS, int E, int NBITS>
+__device__ __forceinline__ void store_lane_codes_t(const KParams& k, const WarpTile& w, const float* ws, float z) {
+    constexpr float Lf = static_cast<float>((1 << NBITS) - 1);
 #pragma unroll
     for (int t = 0; t < E / kPiece; ++t) {
         uint32_t code[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) code[i] = eval_elem(ws[t * 8 + i], z, k.Lf).code;
-        const uint64_t v = pack8(code, k.nbits);
+        for (int i = 0; i < 8; ++i) round_clamp(__fadd_rn(ws[t * 8 + i], z), Lf, &code[i]);
+        const uint64_t v = pack8_t<NBITS>(code);
         const int pc = (w.part * E) / kPiece + t;  // piece index within the group
         if (AXIS == 1) {
-            store_piece(k.packed + (w.j * (k.g / kPiece) + pc) * k.nbits, v, k.nbits);
+            uint8_t* dst = k.packed + (w.j * (k.g / kPiece) + pc) * NBITS;
+            if (NBITS == 8) *reinterpret_cast<uint64_t*>(dst) = v;
+            else if (NBITS == 4) *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(v);
+            else if (NBITS == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(v);
+            else if (NBITS == 1) *dst = static_cast<uint8_t>(v);
+            else {
+                dst[0] = static_cast<uint8_t>(v);
+                dst[1] = static_cast<uint8_t>(v >> 8);
+                dst[2] = static_cast<uint8_t>(v >> 16);
+            }
         } else {
             const int64_t rb = w.j / k.cols, c = w.j % k.cols;
-            uint8_t* dst =
-                k.packed + ((rb * k.g) / kPiece * k.nbits + static_cast<int64_t>(pc) * k.nbits) * k.cols + c;
-            for (int b = 0; b < k.nbits; ++b) dst[b * k.cols] = static_cast<uint8_t>(v >> (8 * b));
+            uint8_t* dst = k.packed + ((rb * k.g) / kPiece * NBITS + static_cast<int64_t>(pc) * NBITS) * k.cols + c;
+#pragma unroll
+            for (int b = 0; b < NBITS; ++b) dst[b * k.cols] = static_cast<uint8_t>(v >> (8 * b));
         }
+    }
+}
+
+// Packed codes of this lane's E elements with zero-point z (bit width chosen
+// by a warp-uniform switch, so the packing is compiled per width).
+template <int AXIS, int E>
+__device__ __forceinline__ void store_lane_codes(const KParams& k, const WarpTile& w, const float* ws, float z) {
+    if (!w.valid) return;
+    switch (k.nbits) {
+        case 1: store_lane_codes_t<AXIS, E, 1>(k, w, ws, z); break;
+        case 2: store_lane_codes_t<AXIS, E, 2>(k, w, ws, z); break;
+        case 3: store_lane_codes_t<AXIS, E, 3>(k, w, ws, z); break;
+        case 4: store_lane_codes_t<AXIS, E, 4>(k, w, ws, z); break;
+        default: store_lane_codes_t<AXIS, E, 8>(k, w, ws, z); break;
     }
 }
 
@@ -673,20 +302,30 @@ __device__ __forceinline__ float beta_at(const KParams& k, int it) {
 // (when sp) fl((w - W_e)*s).
 template <int DT, int AXIS, int E>
 __device__ __forceinline__ float3 eval_lane_slow(const KParams k, const WarpTile w, float s, float z, int it, bool sp,
-                                              double* swe_out) {
-    float x[E];
-    load_lane<DT, AXIS, E>(k, w, x);
+                                                 double* swe_out) {
     float err = 0.0f, sq = 0.0f;
     double swe = 0.0;
     const float beta = beta_at(k, it);
-#pragma unroll 4
-    for (int i = 0; i < E; ++i) {
-        const ElemEval ee = eval_elem(__fmul_rn(x[i], s), z, k.Lf);
-        err += pow_pos(fabsf(ee.r), k.p);
-        sq += ee.q;
-        if (sp) {
-            const float we = shrink_elem(ee.r, s, k.p, beta);
-            swe += static_cast<double>(__fmul_rn(__fsub_rn(x[i], we), s));
+    const int64_t rb = AXIS == 1 ? 0 : w.j / k.cols, c = AXIS == 1 ? 0 : w.j % k.cols;
+#pragma unroll 1
+    for (int t = 0; t < E / kPiece; ++t) {  // one 8-element piece at a time: few live registers
+        float x[kPiece];
+        if (AXIS == 1) {
+            unpack8<DT>(__ldg(reinterpret_cast<const uint4*>(k.W + w.j * k.g + w.part * E) + t), x);
+        } else {
+            const uint16_t* src = k.W + (rb * k.g + w.part * E + t * kPiece) * k.cols + c;
+#pragma unroll
+            for (int i = 0; i < kPiece; ++i) x[i] = bits_to_float<DT>(__ldg(src + i * k.cols));
+        }
+#pragma unroll
+        for (int i = 0; i < kPiece; ++i) {
+            const ElemEval ee = eval_elem(__fmul_rn(x[i], s), z, k.Lf);
+            err += pow_pos(fabsf(ee.r), k.p);
+            sq += ee.q;
+            if (sp) {
+                const float we = shrink_elem(ee.r, s, k.p, beta);
+                swe += static_cast<double>(__fmul_rn(__fsub_rn(x[i], we), s));
+            }
         }
     }
     *swe_out = swe;
@@ -778,9 +417,10 @@ __device__ __forceinline__ double warp_sum_d(double x) {
     return x;
 }
 
-template <int DT, int AXIS, int E, int MODE>
-__global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2)
-    solve_reg_kernel(const KParams k, int chunk) {
+// ============================================================ tensor stop ==
+
+template <int DT, int AXIS, int E>
+__global__ void __launch_bounds__(kRegThreads, E <= 16 ? 3 : 2) solve_tensor_kernel(const KParams k, int chunk) {
     __shared__ float2 sred[kRegWarps];
     __shared__ double sacc[kChunkMax][kRegThreads];  // per-thread tensor error partials
     __shared__ float sthr[kChunkMax];                 // shrink threshold of each iteration of the chunk
@@ -792,51 +432,6 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2)
     const float inv_g = 1.0f / static_cast<float>(k.g);
     float zmin = FLT_MAX, zmax = -FLT_MAX;
 
-    if (MODE == MODE_LOCAL) {
-        const bool stop_group = k.stop_mode == 0;
-        for (int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp; t < ntiles; t += wstride) {
-            const WarpTile w = warp_tile<AXIS>(k, t);
-            float x[E], ws[E];
-            load_lane<DT, AXIS, E>(k, w, x);
-            float s, z0, lmin, lmax;
-            double sws;
-            init_lane<E>(k, w, x, ws, &s, &z0, &sws, &lmin, &lmax);
-            const F2 sws2 = split_f2(sws);
-            float z = z0, zb = z0, be = INFINITY, beta = k.beta;
-            int bi = 0;
-            bool active = w.valid && k.iters_eff > 0;
-            for (int it = 0; it < k.iters_eff && __any_sync(kFull, active); ++it) {
-                const float thr = shrink_threshold(beta, k.p);
-                float err, sq;
-                bool sp;
-                double swe;
-                eval_lane<E>(k, active, x, ws, s, z, z0, beta, thr, &err, &sq, &sp, &swe);
-                if (active) {
-                    const bool improved = err < be;
-                    if (improved) {
-                        be = err;
-                        zb = z;
-                        bi = it;
-                    }
-                    bool stop = (stop_group && !improved) || it >= k.iters_eff - 1;
-                    if (!stop) {
-                        const float zn = sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, sws2, inv_g);
-                        if (stop_group && zn == z) stop = true;
-                        else z = zn;
-                    }
-                    if (stop) active = false;
-                }
-                beta = __fmul_rn(beta, k.kappa);
-            }
-            store_lane_codes<AXIS, E>(k, w, ws, zb);
-            if (w.valid && w.part == 0)
-                store_group(k, w.j, s, zb, bi, be * pow_pos(s, -k.p) / static_cast<float>(k.g), &zmin, &zmax);
-        }
-        if (k.zero_nbits == 8) write_minmax<kRegWarps>(k, zmin, zmax, sred);
-        return;
-    }
-
-    // ---------------------------------------------------- tensor mode ----
     const int iters = k.iters_eff;
     const int nch = num_chunks(iters);
     // Stop rule on the tensor errors of iterations [0, k0) (same decision in every CTA).
@@ -896,7 +491,7 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2)
             }
             if (w.valid && w.part == 0) store_group(k, w.j, s, z, kb, err_mean, &zmin, &zmax);
         }
-        if (k.zero_nbits == 8) write_minmax<kRegWarps>(k, zmin, zmax, sred);
+        if (k.zero_nbits == 8) merge_zero_range<kRegWarps>(k, zmin, zmax, sred);
         return;
     }
 
@@ -985,7 +580,7 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2)
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
-        const unsigned prev = atomicAdd(k.counters + 1, 1u);
+        const unsigned prev = atomicAdd(k.counters + kWordTicket, 1u);
         sflag = prev == gridDim.x - 1;
     }
     __syncthreads();
@@ -998,33 +593,167 @@ __global__ void __launch_bounds__(kRegThreads, (MODE == 1 && E <= 16) ? 3 : 2)
         v = warp_sum_d(v);
         if (lane == 0) k.etot[k0 + q] = v / static_cast<double>(k.n);
     }
-    if (threadIdx.x == 0) k.counters[1] = 0;
+    if (threadIdx.x == 0) k.counters[kWordTicket] = 0;
+}
+
+// ============================================================= group stop ==
+
+// One pass of the group-stop solver (see the file comment).  Entries are warp
+// tile slots: axis 1, entry e is group e; axis 0, entry e is lane group
+// e % gpw of warp tile e / gpw (32/P neighbouring columns of one row block).
+// State and survivor lists are indexed by the entry's offset in the slice.
+struct PassArgs {
+    const uint32_t* in;         // entries of this pass (nullptr: every entry of the slice, in order)
+    const uint32_t* in_count;   // number of entries in `in`
+    uint32_t* out;              // entries still running after the pass (nullptr: the last pass)
+    uint32_t* out_count;
+    float4* state;              // [2 * slice]: (z, best error, kept zero, s), (z0, max w*s, sum w*s hi, lo)
+    int* state_it;              // [slice]: iteration of the kept zero
+    int64_t e0;                 // first entry of the slice
+    int64_t n;                  // entries in the slice
+    int k0;                     // iterations every group of this pass has done
+    int evals;                  // evaluations in this pass
+};
+
+template <int AXIS>
+__device__ __forceinline__ bool entry_group(const KParams& k, int64_t e, int64_t* j) {
+    if (AXIS == 1) {
+        *j = e;
+        return e < k.G;
+    }
+    const int gpw = 32 >> k.logP;
+    const int64_t t = e >> (5 - k.logP);
+    const int64_t ncb = (k.cols + gpw - 1) / gpw;
+    const int64_t rb = t / ncb, c = (t % ncb) * gpw + (e & (gpw - 1));
+    *j = rb * k.cols + c;
+    return c < k.cols;
+}
+
+__host__ __device__ inline int64_t num_entries(int64_t rows, int64_t cols, int64_t G, int g, int axis, int logP) {
+    const int gpw = 32 >> logP;
+    if (axis == 1) return G;
+    return (rows / g) * ((cols + gpw - 1) / gpw) * gpw;
+}
+
+// Three CTAs per SM (80 registers): occupancy beats the few spilled bytes.
+template <int DT, int AXIS, int E>
+__global__ void __launch_bounds__(kRegThreads, 3) solve_group_kernel(const KParams k, const PassArgs pa) {
+    __shared__ float2 sred[kRegWarps];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gpw = 32 >> k.logP;
+    const int part = lane & (k.P - 1);
+    const int64_t count = pa.in ? static_cast<int64_t>(__ldcg(pa.in_count)) : pa.n;
+    const int64_t ntiles = (count + gpw - 1) / gpw;
+    const bool stop_group = k.stop_mode == 0;
+    const float inv_g = 1.0f / static_cast<float>(k.g);
+    // smallest shrink threshold of the run (beta only grows): a conservative gate
+    const float thr = shrink_threshold(k.beta_last, k.p);
+    float zmin = FLT_MAX, zmax = -FLT_MAX;
+
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp; t < ntiles;
+         t += static_cast<int64_t>(gridDim.x) * kRegWarps) {
+        const int64_t slot = t * gpw + (lane >> k.logP);
+        int64_t el = -1;  // entry offset in the slice
+        if (slot < count) el = pa.in ? static_cast<int64_t>(pa.in[slot]) : slot;
+        WarpTile w;
+        w.part = part;
+        w.j = 0;
+        w.valid = el >= 0 && entry_group<AXIS>(k, pa.e0 + el, &w.j);
+        float x[E], ws[E];
+        load_lane<DT, AXIS, E>(k, w, x);
+        float s, z0, z, be, zb, lmin, lmax, wsmax;
+        F2 sws2;
+        int bi;
+        if (pa.k0 == 0) {
+            double sws;
+            init_lane<E>(k, w, x, ws, &s, &z0, &sws, &lmin, &lmax);
+            sws2 = split_f2(sws);
+            wsmax = seg_max(w.valid ? lmax : -FLT_MAX, k.P);
+            z = zb = z0;
+            be = INFINITY;
+            bi = 0;
+        } else {
+            float4 a = make_float4(0.0f, INFINITY, 0.0f, 1.0f), b = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            bi = 0;
+            if (w.valid) {
+                a = __ldcg(pa.state + 2 * el);
+                b = __ldcg(pa.state + 2 * el + 1);
+                bi = __ldcg(pa.state_it + el);
+            }
+            z = a.x;
+            be = a.y;
+            zb = a.z;
+            s = a.w;
+            z0 = b.x;
+            wsmax = b.y;
+            sws2 = F2{b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < E; ++i) ws[i] = __fmul_rn(x[i], s);
+            lmin = -z0;  // fl(min w * s) = -fl(-min w * s) = -z0
+            lmax = wsmax;
+        }
+        bool active = w.valid && pa.k0 < k.iters_eff;
+        for (int e = 0; e < pa.evals && __any_sync(kFull, active); ++e) {
+            const int it = pa.k0 + e;
+            WarpTile wa = w;
+            wa.valid = active;
+            float err, sq;
+            bool sp;
+            double swe;
+            eval_lane_reload<DT, AXIS, E>(k, wa, ws, lmin, lmax, s, z, z0, it, thr, &err, &sq, &sp, &swe);
+            if (active) {
+                const bool improved = err < be;
+                if (improved) {
+                    be = err;
+                    zb = z;
+                    bi = it;
+                }
+                bool stop = (stop_group && !improved) || it >= k.iters_eff - 1;
+                if (!stop) {
+                    const float zn = sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, sws2, inv_g);
+                    if (stop_group && zn == z) stop = true;  // fixed point: the next error equals this one
+                    else z = zn;
+                }
+                if (stop) active = false;
+            }
+        }
+        if (!pa.out) active = false;  // the last pass: evals reach iters_eff - 1, every group has stopped
+        if (active) {
+            // still running: leave the state for the next pass
+            if (part == 0) {
+                pa.state[2 * el] = make_float4(z, be, zb, s);
+                pa.state[2 * el + 1] = make_float4(z0, wsmax, sws2.hi, sws2.lo);
+                pa.state_it[el] = bi;
+            }
+        } else if (w.valid) {
+            store_lane_codes<AXIS, E>(k, w, ws, zb);
+            if (part == 0) {
+                const float err_mean = k.dbg_err ? be * pow_pos(s, -k.p) / static_cast<float>(k.g) : 0.0f;
+                store_group(k, w.j, s, zb, bi, err_mean, &zmin, &zmax);
+            }
+        }
+        const unsigned run = __ballot_sync(kFull, active && part == 0);
+        if (run) {
+            uint32_t base = 0;
+            if (lane == 0) base = atomicAdd(pa.out_count, static_cast<uint32_t>(__popc(run)));
+            base = __shfl_sync(kFull, base, 0);
+            if (active && part == 0) pa.out[base + __popc(run & ((1u << lane) - 1u))] = static_cast<uint32_t>(el);
+        }
+    }
+    if (k.zero_nbits == 8) merge_zero_range<kRegWarps>(k, zmin, zmax, sred);
 }
 
 // ------------------------------------------------------- 8-bit zero ------
 
-__global__ void __launch_bounds__(256) zero_q8_kernel(const float* zbest, int64_t G, const float2* minmax, int nparts,
+// One RTN quantiser for all kept zeros of the tensor, from their min/max
+// (merged into the workspace header by the solver kernels).
+__global__ void __launch_bounds__(256) zero_q8_kernel(const float* zbest, int64_t G, const uint32_t* counters,
                                                        uint8_t* zq, float* meta) {
-    __shared__ float2 sred[8];
-    float mn = FLT_MAX, mx = -FLT_MAX;
-    for (int i = threadIdx.x; i < nparts; i += 256) {
-        const float2 v = minmax[i];
-        mn = fminf(mn, v.x);
-        mx = fmaxf(mx, v.y);
+    float mn = 0.0f, mx = 0.0f;
+    if (G > 0) {
+        mn = key_value(~__ldcg(counters + kWordZmin));
+        mx = key_value(__ldcg(counters + kWordZmax));
     }
-    for (int o = 16; o > 0; o >>= 1) {
-        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-    }
-    if ((threadIdx.x & 31) == 0) sred[threadIdx.x >> 5] = make_float2(mn, mx);
-    __syncthreads();
-    mn = sred[0].x;
-    mx = sred[0].y;
-    for (int w = 1; w < 8; ++w) {
-        mn = fminf(mn, sred[w].x);
-        mx = fmaxf(mx, sred[w].y);
-    }
-    if (G == 0) mn = mx = 0.0f;
     float sz = kScaleCap;
     if (mx > mn) sz = fminf(__fdiv_rn(255.0f, __fsub_rn(mx, mn)), kScaleCap);
     const float zz = __fmul_rn(-mn, sz);
@@ -1156,113 +885,130 @@ cudaError_t persistent_grid(K kernel, int threads, size_t smem, int64_t work_uni
     return cudaSuccess;
 }
 
-// Cells per warp of the pool kernel: ~6 KB of fp32 data, at least one full
-// pass of lanes, at most 64 cells.
-int pool_cells(int g, int P) {
-    int nc = 6144 / (4 * pool_cell_floats(g));
-    if (nc * P < 32) nc = 32 / P;
-    if (nc > 64) nc = 64;
-    if (nc < 1) nc = 1;
-    return nc;
-}
-
-template <int DT, int E, int NBITS>
-cudaError_t launch_pool(KParams& k, cudaStream_t stream, int* grid) {
-    k.NC = pool_cells(k.g, k.P);
-    k.pool_warp_bytes = pool_warp_bytes(k.NC, k.g);
-    const size_t smem = static_cast<size_t>(k.pool_warp_bytes) * kPoolWarps;
-    auto kern = solve_pool_kernel<DT, E, NBITS>;
-    const int64_t warps_needed = (k.G + k.NC - 1) / k.NC;
-    cudaError_t err = persistent_grid(kern, kPoolThreads, smem, (warps_needed + kPoolWarps - 1) / kPoolWarps, grid);
-    if (err != cudaSuccess) return err;
-    kern<<<*grid, kPoolThreads, smem, stream>>>(k);
-    return cudaGetLastError();
-}
-
-template <int DT, int E>
-cudaError_t launch_pool_b(KParams& k, cudaStream_t stream, int* grid) {
-    switch (k.nbits) {
-        case 1: return launch_pool<DT, E, 1>(k, stream, grid);
-        case 2: return launch_pool<DT, E, 2>(k, stream, grid);
-        case 3: return launch_pool<DT, E, 3>(k, stream, grid);
-        case 4: return launch_pool<DT, E, 4>(k, stream, grid);
-        default: return launch_pool<DT, E, 8>(k, stream, grid);
+// Evaluations per group-mode pass: short passes first (most groups stop after
+// two or three evaluations), longer ones for the tail, then the rest.
+int pass_schedule(int iters_eff, int stop_mode, int* m) {
+    if (stop_mode != 0 || iters_eff <= 2) {  // no early stop: one pass runs everything
+        m[0] = iters_eff;
+        return 1;
     }
+    static const int sched[] = {2, 3};
+    int n = 0, done = 0;
+    for (int v : sched) {
+        if (done + v >= iters_eff) break;
+        m[n++] = v;
+        done += v;
+    }
+    m[n++] = iters_eff - done;
+    return n;
 }
 
 template <int DT, int AXIS, int E>
-cudaError_t launch_reg(KParams& k, cudaStream_t stream, int* grid) {
+cudaError_t launch_group(KParams& k, const WorkspaceLayout& L, uint8_t* ws, cudaStream_t stream) {
+    auto kern = solve_group_kernel<DT, AXIS, E>;
+    const int64_t n_all = num_entries(k.rows, k.cols, k.G, k.g, AXIS, k.logP);
+    const int64_t slice = L.slice < n_all ? L.slice : n_all;
+    const int gpw = 32 >> k.logP;
+    int grid = 0;
+    cudaError_t err = persistent_grid(kern, kRegThreads, 0, ((slice + gpw - 1) / gpw + kRegWarps - 1) / kRegWarps, &grid);
+    if (err != cudaSuccess) return err;
+    int m[kMaxPasses];
+    const int np = pass_schedule(k.iters_eff, k.stop_mode, m);
+    uint32_t* const list[2] = {reinterpret_cast<uint32_t*>(ws + L.list0), reinterpret_cast<uint32_t*>(ws + L.list1)};
+    for (int64_t e0 = 0; e0 < n_all; e0 += slice) {
+        if (e0 > 0) {  // pass counts of the previous slice
+            err = cudaMemsetAsync(k.counters + kWordPass, 0, sizeof(uint32_t) * kMaxPasses, stream);
+            if (err != cudaSuccess) return err;
+        }
+        PassArgs pa{};
+        pa.state = reinterpret_cast<float4*>(ws + L.state);
+        pa.state_it = reinterpret_cast<int*>(ws + L.state_it);
+        pa.e0 = e0;
+        pa.n = n_all - e0 < slice ? n_all - e0 : slice;
+        int k0 = 0;
+        for (int q = 0; q < np; ++q) {
+            pa.in = q == 0 ? nullptr : list[(q - 1) & 1];
+            pa.in_count = q == 0 ? nullptr : k.counters + kWordPass + q - 1;
+            pa.out = q + 1 < np ? list[q & 1] : nullptr;
+            pa.out_count = k.counters + kWordPass + q;
+            pa.k0 = k0;
+            pa.evals = m[q];
+            kern<<<grid, kRegThreads, 0, stream>>>(k, pa);
+            err = cudaGetLastError();
+            if (err != cudaSuccess) return err;
+            k0 += m[q];
+        }
+    }
+    return cudaSuccess;
+}
+
+template <int DT, int AXIS, int E>
+cudaError_t launch_tensor(KParams& k, cudaStream_t stream) {
     const int gpw = 32 >> k.logP;
     const int64_t tiles = AXIS == 1 ? (k.G + gpw - 1) / gpw : (k.rows / k.g) * ((k.cols + gpw - 1) / gpw);
-    const int64_t ctas = (tiles + kRegWarps - 1) / kRegWarps;
-    if (k.stop_mode != 1) {
-        auto kern = solve_reg_kernel<DT, AXIS, E, MODE_LOCAL>;
-        cudaError_t err = persistent_grid(kern, kRegThreads, 0, ctas, grid);
-        if (err != cudaSuccess) return err;
-        kern<<<*grid, kRegThreads, 0, stream>>>(k, 0);
-        return cudaGetLastError();
-    }
-    auto kern = solve_reg_kernel<DT, AXIS, E, MODE_TENSOR>;
-    cudaError_t err = persistent_grid(kern, kRegThreads, 0, ctas, grid);
+    auto kern = solve_tensor_kernel<DT, AXIS, E>;
+    int grid = 0;
+    cudaError_t err = persistent_grid(kern, kRegThreads, 0, (tiles + kRegWarps - 1) / kRegWarps, &grid);
     if (err != cudaSuccess) return err;
     const int nch = num_chunks(k.iters_eff);
     for (int c = 0; c <= nch; ++c) {  // nch chunks, then the launch that writes the outputs
-        kern<<<*grid, kRegThreads, 0, stream>>>(k, c);
+        kern<<<grid, kRegThreads, 0, stream>>>(k, c);
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }
     return cudaSuccess;
 }
 
-// The register kernel holds a whole group per thread up to g = 32 (E = g,
-// P = 1): every lane then has E independent elements per iteration and the
-// group sums need no shuffles; larger groups spread over P = g/32 lanes.
-template <int DT, int AXIS>
-cudaError_t launch_reg_e(KParams& k, cudaStream_t stream, int* grid) {
-    k.E = k.g < 32 ? k.g : 32;
-    k.P = k.g / k.E;
-    k.logP = 0;
-    while ((1 << k.logP) < k.P) ++k.logP;
-    if (k.E == 8) return launch_reg<DT, AXIS, 8>(k, stream, grid);
-    if (k.E == 16) return launch_reg<DT, AXIS, 16>(k, stream, grid);
-    return launch_reg<DT, AXIS, 32>(k, stream, grid);
+template <int DT, int AXIS, int E>
+cudaError_t launch_solver(KParams& k, const WorkspaceLayout& L, uint8_t* ws, cudaStream_t stream) {
+    if (k.stop_mode == 1) return launch_tensor<DT, AXIS, E>(k, stream);
+    return launch_group<DT, AXIS, E>(k, L, ws, stream);
 }
 
-template <int DT>
-cudaError_t launch_pool_e(KParams& k, cudaStream_t stream, int* grid) {
-    if (k.E == 8) return launch_pool_b<DT, 8>(k, stream, grid);
-    if (k.E == 16) return launch_pool_b<DT, 16>(k, stream, grid);
-    return launch_pool_b<DT, 32>(k, stream, grid);
+template <int DT, int AXIS>
+cudaError_t launch_solver_e(KParams& k, const WorkspaceLayout& L, uint8_t* ws, cudaStream_t stream) {
+    if (k.E == 8) return launch_solver<DT, AXIS, 8>(k, L, ws, stream);
+    if (k.E == 16) return launch_solver<DT, AXIS, 16>(k, L, ws, stream);
+    return launch_solver<DT, AXIS, 32>(k, L, ws, stream);
 }
 
 }  // namespace
 
+// A whole group per lane up to g = 32 (E = g, P = 1): every lane has E
+// independent elements per evaluation and the group sums need no shuffles;
+// larger groups spread over P = g/32 lanes.
 Geometry make_geometry(int g) {
     Geometry geo;
     geo.g = g;
-    geo.E = g <= 8 ? 8 : (g <= 512 ? 16 : 32);
+    geo.E = g < 32 ? g : 32;
     geo.P = g / geo.E;
+    geo.logP = 0;
+    while ((1 << geo.logP) < geo.P) ++geo.logP;
     return geo;
 }
 
-WorkspaceLayout workspace_layout(int64_t G, int stop_mode, int zero_nbits, int iters) {
+int64_t group_entries(int64_t rows, int64_t cols, int g, int axis) {
+    return num_entries(rows, cols, rows * cols / g, g, axis, make_geometry(g).logP);
+}
+
+WorkspaceLayout workspace_layout(int64_t rows, int64_t cols, int g, int axis, int stop_mode, int zero_nbits,
+                                 int64_t slice) {
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    const int64_t G = rows * cols / g;
+    const size_t Gs = static_cast<size_t>(G > 0 ? G : 0);
     WorkspaceLayout l{};
     size_t off = 0;
     l.header = off;
     off += 256;
-    l.minmax = off;
-    off = up(off + sizeof(float) * 2 * kMaxPartials);
-    const size_t Gs = static_cast<size_t>(G > 0 ? G : 0);
     l.zbest = off;
     if (zero_nbits == 8) off = up(off + 4 * Gs);
+    l.state = l.state_it = l.list0 = l.list1 = off;
     l.tparts = l.etot = l.t_s = l.t_z0 = l.t_sws = l.t_zs = off;
     if (stop_mode == 1) {
-        const size_t it = static_cast<size_t>(iters > 0 ? iters : 1);
         l.tparts = off;
         off = up(off + sizeof(double) * kChunkMax * kMaxPartials);
         l.etot = off;
-        off = up(off + sizeof(double) * it);
+        off = up(off + sizeof(double) * kMaxIters);
         l.t_s = off;
         off = up(off + 4 * Gs);
         l.t_z0 = off;
@@ -1271,14 +1017,39 @@ WorkspaceLayout workspace_layout(int64_t G, int stop_mode, int zero_nbits, int i
         off = up(off + 8 * Gs);
         l.t_zs = off;
         off = up(off + 12 * Gs);
+    } else {
+        const int64_t n = group_entries(rows, cols, g, axis);
+        l.slice = (slice > 0 && slice < n) ? slice : n;
+        const size_t S = static_cast<size_t>(l.slice > 0 ? l.slice : 0);
+        l.state = off;
+        off = up(off + 32 * S);
+        l.state_it = off;
+        off = up(off + 4 * S);
+        l.list0 = off;
+        off = up(off + 4 * S);
+        l.list1 = off;
+        off = up(off + 4 * S);
     }
     l.total = off;
     return l;
 }
 
+int64_t fit_slice(int64_t rows, int64_t cols, int g, int axis, int stop_mode, int zero_nbits, size_t bytes) {
+    const WorkspaceLayout full = workspace_layout(rows, cols, g, axis, stop_mode, zero_nbits, 0);
+    if (full.total <= bytes) return full.slice > 0 ? full.slice : 1;
+    if (stop_mode == 1) return 0;
+    const WorkspaceLayout base = workspace_layout(rows, cols, g, axis, stop_mode, zero_nbits, 1);
+    const size_t fixed = base.state;  // header and kept zeros
+    const size_t per = 44, pad = 4 * 256;
+    if (bytes < fixed + pad) return 0;
+    int64_t s = static_cast<int64_t>((bytes - fixed - pad) / per) & ~static_cast<int64_t>(31);
+    while (s >= kMinSlice && workspace_layout(rows, cols, g, axis, stop_mode, zero_nbits, s).total > bytes) s -= 32;
+    return s >= kMinSlice ? s : 0;
+}
+
 cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream) {
     const Geometry geo = make_geometry(a.g);
-    const WorkspaceLayout L = workspace_layout(a.G, a.stop_mode, a.zero_nbits, kMaxIters);
+    const WorkspaceLayout L = workspace_layout(a.rows, a.cols, a.g, a.axis, a.stop_mode, a.zero_nbits, a.slice);
     KParams k{};
     k.W = static_cast<const uint16_t*>(a.W);
     k.rows = a.rows;
@@ -1288,8 +1059,7 @@ cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream) {
     k.g = a.g;
     k.E = geo.E;
     k.P = geo.P;
-    k.logP = 0;
-    while ((1 << k.logP) < geo.P) ++k.logP;
+    k.logP = geo.logP;
     k.nbits = a.nbits;
     k.iters = a.iters;
     k.iters_eff = a.iters > 0 ? a.iters : (a.dbg_err ? 1 : 0);  // iters 0 == 1: z* = z0 either way
@@ -1299,6 +1069,9 @@ cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream) {
     k.p = a.p;
     k.beta = a.beta;
     k.kappa = a.kappa;
+    float bl = a.beta;
+    for (int i = 1; i < k.iters_eff; ++i) bl *= a.kappa;  // the same sequential fp32 products as the device
+    k.beta_last = bl;
     k.Lf = static_cast<float>((1 << a.nbits) - 1);
     k.packed = a.packed;
     k.scale = a.scale;
@@ -1307,7 +1080,6 @@ cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream) {
     k.dbg_err = a.dbg_err;
     k.dbg_zero = a.dbg_zero;
     k.counters = reinterpret_cast<uint32_t*>(a.ws + L.header);
-    k.minmax = reinterpret_cast<float2*>(a.ws + L.minmax);
     k.zbest_ws = a.zero_nbits == 8 ? reinterpret_cast<float*>(a.ws + L.zbest) : nullptr;
     if (a.stop_mode == 1) {
         k.tparts = reinterpret_cast<double*>(a.ws + L.tparts);
@@ -1320,14 +1092,11 @@ cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream) {
 
     cudaError_t err = cudaMemsetAsync(a.ws + L.header, 0, 256, stream);
     if (err != cudaSuccess) return err;
-    int grid = 0;
     if (a.G > 0) {
-        const bool pool = a.axis == 1 && a.stop_mode != 1;
-        if (pool) err = a.dtype == 0 ? launch_pool_e<0>(k, stream, &grid) : launch_pool_e<1>(k, stream, &grid);
-        else if (a.dtype == 0 && a.axis == 1) err = launch_reg_e<0, 1>(k, stream, &grid);
-        else if (a.dtype == 0) err = launch_reg_e<0, 0>(k, stream, &grid);
-        else if (a.axis == 1) err = launch_reg_e<1, 1>(k, stream, &grid);
-        else err = launch_reg_e<1, 0>(k, stream, &grid);
+        if (a.dtype == 0 && a.axis == 1) err = launch_solver_e<0, 1>(k, L, a.ws, stream);
+        else if (a.dtype == 0) err = launch_solver_e<0, 0>(k, L, a.ws, stream);
+        else if (a.axis == 1) err = launch_solver_e<1, 1>(k, L, a.ws, stream);
+        else err = launch_solver_e<1, 0>(k, L, a.ws, stream);
         if (err != cudaSuccess) return err;
     }
     if (a.zero_nbits == 8) {
@@ -1335,7 +1104,7 @@ cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream) {
         const int64_t cap = static_cast<int64_t>(device_info().sms) * 8;
         if (blocks > cap) blocks = cap;
         if (blocks < 1) blocks = 1;
-        zero_q8_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(k.zbest_ws, a.G, k.minmax, grid,
+        zero_q8_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(k.zbest_ws, a.G, k.counters,
                                                                     static_cast<uint8_t*>(a.zero), a.zero_meta);
         err = cudaGetLastError();
     }

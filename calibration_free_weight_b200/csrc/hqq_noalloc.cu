@@ -24,6 +24,7 @@
 #include <mutex>
 
 #include "../../include/hqq.h"
+#include "hqq_internal.h"
 
 namespace {
 
@@ -61,15 +62,17 @@ extern "C" int hqq_quantize_noalloc(const void* W, int64_t rows, int64_t cols, i
                                     void* stream) {
     if (stop_mode == HQQ_STOP_TENSOR) return HQQ_ERR_INVALID_ARG;
     const size_t need = hqq_workspace_bytes(rows, cols, group_size, axis, stop_mode, zero_nbits);
-    if (need > kScratchBytes) return HQQ_ERR_WORKSPACE;
     void* ws = nullptr;
-    if (need > 0) {  // need == 0: invalid arguments, reported by hqq_quantize below
+    if (need > 0) {  // need == 0: invalid arguments, reported by quantize_entry below
+        if (hqq::fit_slice(rows, cols, group_size, axis, stop_mode, zero_nbits, kScratchBytes) <= 0)
+            return HQQ_ERR_WORKSPACE;
         if (scratch_for_current_device(&ws) != cudaSuccess) {
             cudaGetLastError();
             return HQQ_ERR_CUDA;
         }
     }
-    return hqq_quantize(W, rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode, zero_nbits,
-                        W_q_packed, scale, zero, zero_meta, ws, ws ? kScratchBytes : 0, debug_best_iter,
-                        debug_best_err, debug_zero_f32, stream);
+    // a problem whose full workspace exceeds the scratch runs in slices of groups
+    return hqq::quantize_entry(W, rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
+                               zero_nbits, W_q_packed, scale, zero, zero_meta, ws, ws ? kScratchBytes : 0, true,
+                               debug_best_iter, debug_best_err, debug_zero_f32, stream);
 }

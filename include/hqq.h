@@ -166,9 +166,12 @@ const char* hqq_status_string(int status);
  * HQQ_ERR_INVALID_ARG (use hqq_quantize for it).
  * Scratch: one buffer of HQQ_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory per
  * GPU, held by the library from load until the process exits.  A problem whose
- * hqq_workspace_bytes() exceeds it returns HQQ_ERR_WORKSPACE before anything is
- * launched: with zero_nbits = 8 that means more than 4,186,048 groups (4 bytes
- * per group plus 33,024 fixed bytes); with zero_nbits = 16 every size fits.
+ * hqq_workspace_bytes() exceeds it runs in slices of groups, one after another
+ * on `stream` (same results); each slice needs 44 bytes per group and at least
+ * 4,096 groups.  With zero_nbits = 8 the kept zeros of all groups (4 bytes each)
+ * must fit beside one slice: more than 4,149,184 groups (4 bytes per group plus
+ * 180,480 fixed bytes) returns HQQ_ERR_WORKSPACE before anything is launched.
+ * With zero_nbits = 16 every size fits.
  * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
  * routine).  The first call on each device looks up the buffer's device
  * address (cudaGetSymbolAddress) with that device current; make that first call

@@ -74,6 +74,8 @@ def test_noalloc_matches_workspace_entry_point_twice(hq):
     cases = [  # second call: other shape, dtype, group size and stop rule on the same scratch
         (synth.weight(4096, 4096, seed=0, dtype=torch.float16), 4, 64, hq.HQQ_STOP_GROUP, 8),
         (synth.weight(11008, 4096, seed=4, dtype=torch.bfloat16), 2, 16, hq.HQQ_STOP_NONE, 8),
+        # full workspace 31 MB > scratch: runs in slices of groups
+        (synth.weight(11008, 4096, seed=5, dtype=torch.bfloat16), 4, 64, hq.HQQ_STOP_GROUP, 16),
     ]
     for W_cpu, nbits, g, stop, zb in cases:
         W = W_cpu.cuda()
@@ -84,7 +86,7 @@ def test_noalloc_matches_workspace_entry_point_twice(hq):
 
 
 def test_noalloc_rejects_what_does_not_fit(hq):
-    W = torch.empty(8192, 8192, dtype=torch.float16, device="cuda")  # 4.19 M groups at g16: above the limit
+    W = torch.empty(8192, 8192, dtype=torch.float16, device="cuda")  # 4.19 M groups at g16: above 4,149,184
     G = W.numel() // 16
     assert hq.hqq_workspace_bytes(8192, 8192, 16, 1, 0, 8) > hq.HQQ_NOALLOC_SCRATCH_BYTES
     out = [torch.empty(W.numel() * 2 // 8, dtype=torch.uint8, device="cuda"),
