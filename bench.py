@@ -9,8 +9,12 @@ stop_mode=tensor: 30 hqq_quantize calls, 1.353 G weights.
 value     = weights quantised / device time (CUDA events), inputs resident in HBM.
 e2e       = the same through the C ABI with host buffers: every step copies the
             step's inputs from pinned host memory and reads all outputs back.
-roofline  = the dominant kernel (solve_tensor): bound by the MUFU pipe that
-            evaluates |r|^p (two ops per element and iteration).
+roofline  = the dominant kernel family (solve_tensor_kernel: the tensor-stop
+            calls), bound by the MUFU pipe that evaluates |r|^p (two ops per
+            element and evaluated iterate); timed per hqq_quantize call (its
+            launch sequence) with CUDA events on the launching stream.
+            traffic = DRAM bytes per call from the ncu launch list in
+            profiles/, reported only while the kernel sources are unchanged.
 cpu_baseline / --impl reference = the CPU oracle on a bounded sample.
 
 Multi-GPU (torchrun): each rank quantises its own layer's MLP (weak scaling,
@@ -40,6 +44,40 @@ MATS = [("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008)]
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 SMS = 148
 MUFU_PER_CLK_PER_SM = 16
+KERNEL_SOURCES = ["calibration_free_weight_b200/csrc/hqq_kernels.cu", "calibration_free_weight_b200/csrc/hqq_device.cuh"]
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernel per hqq_quantize call, averaged over the timed step's tensor-stop calls,
+# from the ncu launch list summarised in profiles/ (taken on the kernel sources
+# whose sha256 is recorded here; None until a capture exists).
+TRAFFIC = {"src_sha256": "14447d5a6c5caa9de19e382558cc4b7a6534e641ecfe016f71e486b942affa22",
+           "bytes_per_call": 568482492, "summary": "profiles/launches_llama2-7b-mlp-sweep.md"}
+
+
+def kernel_sources_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def solver_launches(mode, iters=20):
+    """Kernel launches of one hqq_quantize call (fp16 zero), as the library
+    schedules them: group stop runs passes of 2 and 3 evaluations and then the
+    rest (no stop: one pass); tensor stop runs chunks of iterations [0,2),
+    [2,6), [6,10), ... and one launch that writes the outputs."""
+    if mode == 1:
+        last = iters - 1
+        return (0 if iters <= 0 else (0 if last < 2 else (last + 2) // 4) + 1) + 1
+    if mode == 2 or iters <= 2:
+        return 1
+    n, done = 0, 0
+    for v in (2, 3):
+        if done + v >= iters:
+            break
+        n, done = n + 1, done + v
+    return n + 1
 
 
 def peaks():
@@ -321,7 +359,7 @@ def main():
     dom_name = "solve_tensor_kernel" if dom == 1 else "solve_group_kernel"
     n_l = len(fam[dom])
     avg_ms = tot[dom] / n_l
-    mufu_ops = sum(2 * evals[key] for _, key in fam[dom]) / n_l  # per launch
+    mufu_ops = sum(2 * evals[key] for _, key in fam[dom]) / n_l  # per call
     mufu_peak = SMS * MUFU_PER_CLK_PER_SM * sm_max * 1e6 / 1e9  # Gop/s
     achieved = mufu_ops / (avg_ms / 1e3) / 1e9
     # HBM view of the same launches (the metric's second half)
@@ -335,6 +373,8 @@ def main():
     g_bytes = sum(algorithmic_bytes(*[(r, c) for n_, r, c in MATS if n_ == key[0]][0], key[1], key[2])
                   for _, key in grp) / max(1, len(grp))
     g_w = sum([(r * c) for _, key in grp for n_, r, c in MATS if n_ == key[0]]) / max(1, len(grp))
+
+    traffic = TRAFFIC["bytes_per_call"] if TRAFFIC["src_sha256"] == kernel_sources_sha() else None
 
     # end to end through the C ABI with host buffers
     pinned = {k: v.pin_memory() for k, v in ins_cpu.items()}
@@ -366,8 +406,10 @@ def main():
             "warmup": args.warmup, "ms_per_step": dev_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config_dict(world),
             "roofline": {"bound": "alu", "kernel": dom_name, "achieved": achieved, "peak": mufu_peak,
-                         "unit": "Gop/s (MUFU lg2+ex2)", "frac": achieved / mufu_peak, "traffic": None,
+                         "unit": "Gop/s (MUFU lg2+ex2)", "frac": achieved / mufu_peak, "traffic": traffic,
+                         "traffic_unit": "bytes per call", "algorithmic_bytes_per_call": bytes_dom,
                          "peak_basis": f"{SMS} SMs x {MUFU_PER_CLK_PER_SM} MUFU/clk x {sm_max:.0f} MHz",
+                         "timed_unit": f"one hqq_quantize call = {solver_launches(dom)} launches of {dom_name}",
                          "avg_launch_ms": avg_ms, "hbm_gbs": gb_dom, "hbm_frac": gb_dom / hbm_peak},
             "hbm": {"achieved_gbs_step": hbm_step, "peak_gbs": hbm_peak, "peak_kind": peak_kind,
                     "frac_step": hbm_step / hbm_peak,
@@ -375,7 +417,7 @@ def main():
                                    "frac": g_bytes / (g_ms / 1e3) / 1e9 / hbm_peak,
                                    "gweights_s": g_w / (g_ms / 1e3) / 1e9}},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": len(calls) * args.steps,
+            "gpu_launches": sum(solver_launches(mode) for *_, mode in calls) * args.steps,
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, nth, desc, _, _ = oracle_sample_rate(0, budget_s=args.ref_budget)
