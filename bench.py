@@ -97,24 +97,33 @@ def algorithmic_bytes(rows, cols, nbits, g, zero_nbits=16):
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    """nvidia-smi sampling of SM clock and throttle reasons; only the samples
+    taken between mark_start() and mark_end() (the timed region) count."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.5)  # let the sampler start before the timed region
         except Exception:
             self.proc = None
         return self
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def __exit__(self, *a):
         self.lines = []
@@ -128,11 +137,15 @@ class Clocks:
             self.lines = [l for l in out.splitlines() if l.strip()]
 
     def summary(self):
+        import datetime
         sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for l in getattr(self, "lines", []):
             f = [x.strip() for x in l.split(",")]
             try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if self.t0 is not None and not (self.t0 <= ts <= self.t1):
+                    continue
                 sm.append(float(f[1]))
                 mx = max(mx, float(f[2]))
             except (ValueError, IndexError):
@@ -189,16 +202,22 @@ def oracle_sample_rate(layer, budget_s=12.0, nthreads=0):
 
 # ------------------------------------------------------------------- main ---
 
-def dist_setup():
+def dist_setup(backend="nccl"):
+    """One process per GPU from the torchrun environment (RANK, LOCAL_RANK,
+    WORLD_SIZE, MASTER_ADDR/PORT).  NCCL carries only the barrier and the max
+    over ranks; the gloo backend serves the CPU tests of this path."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
-    else:
+        timeout = datetime.timedelta(seconds=120)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group(backend, timeout=timeout)
+    elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -206,7 +225,8 @@ def dist_setup():
 def max_over_ranks(x, world):
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -214,7 +234,14 @@ def max_over_ranks(x, world):
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def throughput(world, weights_per_step, steps, ms):
+    """Whole-job G weights/s: every rank quantises weights_per_step per step
+    (weak scaling), ms = the max over ranks of the timed region."""
+    return world * weights_per_step * steps / (ms / 1e3) / 1e9
 
 
 def run_reference(args, world, rank):
@@ -275,7 +302,7 @@ def run_case(spec):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--ref-budget", type=float, default=8.0)
@@ -336,11 +363,13 @@ def main():
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with Clocks(local) as clk:
         barrier(world)
+        clk.mark_start()
         ev0.record(stream)
         for _ in range(args.steps):
             one_step(rec)
         ev1.record(stream)
         barrier(world)
+        clk.mark_end()
     for o in outs.values():
         st = hqq.hqq_get_status(o["workspace"])
         if st != hqq.HQQ_OK:
@@ -348,7 +377,7 @@ def main():
     dev_ms = ev0.elapsed_time(ev1)
     dev_ms = max_over_ranks(dev_ms, world)
     w_step = sum(r * c for _, r, c, _, _, _ in calls)
-    value = world * w_step * args.steps / (dev_ms / 1e3) / 1e9
+    value = throughput(world, w_step, args.steps, dev_ms)
 
     # per-launch durations by kernel family
     fam = {0: [], 1: []}
@@ -400,7 +429,7 @@ def main():
     e1.record(stream)
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * w_step * args.steps / (e2e_ms / 1e3) / 1e9
+    e2e_value = throughput(world, w_step, args.steps, e2e_ms)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dev_ms / args.steps, "higher_is_better": True, "scaling": "weak",

@@ -1,0 +1,46 @@
+"""Host-side logic of bench.py that needs no GPU: the launch count it claims,
+the clock-sample filter, the step plan and the algorithmic byte count."""
+import datetime
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_solver_launches_follow_the_schedules():
+    # group stop: passes of 2 and 3 evaluations, then the rest
+    assert bench.solver_launches(0, 20) == 3
+    assert bench.solver_launches(0, 5) == 2 and bench.solver_launches(0, 6) == 3
+    assert bench.solver_launches(0, 2) == 1 and bench.solver_launches(0, 1) == 1
+    # no stop: one pass
+    assert bench.solver_launches(2, 20) == 1
+    # tensor stop: chunks [0,2) [2,6) [6,10) [10,14) [14,18) [18,20) + the writing launch
+    assert bench.solver_launches(1, 20) == 7
+    assert bench.solver_launches(1, 2) == 2 and bench.solver_launches(1, 3) == 3 and bench.solver_launches(1, 6) == 3
+    assert bench.solver_launches(1, 7) == 4
+
+
+def test_clock_samples_outside_the_timed_region_are_dropped():
+    c = bench.Clocks(0)
+    c.lines = ["2026/12/02 12:30:51.900, 1000, 1965, 100.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+               "2026/12/02 12:30:52.123, 1965, 1965, 500.0, 0x0, Not Active, Not Active, Not Active, Active",
+               "2026/12/02 12:30:52.800, 1905, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+               "2026/12/02 12:30:53.500, 1200, 1965, 900.0, 0x8, Active, Not Active, Not Active, Not Active"]
+    c.t0 = datetime.datetime(2026, 12, 2, 12, 30, 52).timestamp()
+    c.t1 = datetime.datetime(2026, 12, 2, 12, 30, 53).timestamp()
+    s = c.summary()
+    assert s["samples"] == 2 and s["sm_mhz"] == (1965 + 1905) / 2
+    assert s["reasons"] == ["sw_power_cap"]  # the hw_slowdown sample lies after the region
+
+
+def test_plan_and_bytes():
+    calls = bench.plan()
+    assert len(calls) == 30
+    assert sum(r * c for _, r, c, *_ in calls) == 1352663040
+    # b4 g64 on 4096x4096: 2 B read + 0.5 B codes + 4/64 B scale/zero per weight
+    assert bench.algorithmic_bytes(4096, 4096, 4, 64) == 4096 * 4096 * 2.5625
+    # consecutive calls never reuse the previous call's matrix
+    assert all(a[0] != b[0] for a, b in zip(calls, calls[1:]))
