@@ -174,30 +174,44 @@ def plan():
 
 # ----------------------------------------------------------------- oracle ---
 
+def oracle_pass(ins, rows, nth):
+    """One pass of the CPU oracle, as it stands, over a bounded sample of the
+    step's work: the first `rows` output rows of every matrix at every setting
+    and mode.  Returns (weights, seconds)."""
+    import oracle
+    t0 = time.perf_counter()
+    n = 0
+    for name, r, c, nbits, g, mode in plan():
+        W = ins[name][:rows if name != "down" else max(1, rows * 4096 // 11008)].contiguous()
+        Wb = W.view(torch.int16).numpy().view(np.uint16)
+        oracle.quantize(Wb, nbits, g, 1, 0.7, 1.0, 1.01, 20, mode, 16, dtype=oracle.BF16, nthreads=nth)
+        n += W.numel()
+    return n, time.perf_counter() - t0
+
+
+def oracle_calibrate(ins, pass_s, nth):
+    """Rows per oracle pass so that one pass takes about pass_s seconds."""
+    rows = 16
+    while True:
+        n, dt = oracle_pass(ins, rows, nth)
+        if dt >= pass_s / 4 or rows >= 4096:
+            return rows, n, dt
+        rows *= 4
+
+
+def oracle_desc(rows, n):
+    return (f"first {rows} rows of gate/up (and the same element count of down) at all 10 settings/modes, "
+            f"{n / 1e6:.2f} M weights per pass, bf16, OpenMP over groups")
+
+
 def oracle_sample_rate(layer, budget_s=12.0, nthreads=0):
-    """Time the CPU oracle, as it stands, on a bounded sample of the step's work:
-    the first `rows` output rows of every matrix at every setting and mode.
-    Returns (weights/s, threads used, sample description)."""
+    """Weights/s of the CPU oracle on a sample of about budget_s / 4 to budget_s
+    seconds.  Returns (weights/s, threads used, sample description, n, s)."""
     import oracle
     oracle.lib()
     nth = nthreads or (os.cpu_count() or 1)
-    ins = make_inputs(layer)
-    rows = 16
-    while True:
-        t0 = time.perf_counter()
-        n = 0
-        for name, r, c, nbits, g, mode in plan():
-            W = ins[name][:rows if name != "down" else max(1, rows * 4096 // 11008)].contiguous()
-            Wb = W.view(torch.int16).numpy().view(np.uint16)
-            oracle.quantize(Wb, nbits, g, 1, 0.7, 1.0, 1.01, 20, mode, 16, dtype=oracle.BF16, nthreads=nth)
-            n += W.numel()
-        dt = time.perf_counter() - t0
-        if dt >= budget_s / 4 or rows >= 2048:
-            break
-        rows *= 4
-    desc = (f"first {rows} rows of gate/up (and the same element count of down) at all 10 settings/modes, "
-            f"{n / 1e6:.2f} M weights per pass, bf16, OpenMP over groups")
-    return n / dt, nth, desc, n, dt
+    rows, n, dt = oracle_calibrate(make_inputs(layer), budget_s, nth)
+    return n / dt, nth, oracle_desc(rows, n), n, dt
 
 
 # ------------------------------------------------------------------- main ---
@@ -245,14 +259,21 @@ def throughput(world, weights_per_step, steps, ms):
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle timed on the host cores, one bounded
+    sample (about --ref-step seconds) per step.  Rank 0 only."""
     if rank != 0:
         return
+    import oracle
+    oracle.lib()
+    nth = os.cpu_count() or 1
+    ins = make_inputs(0)
+    rows, _, _ = oracle_calibrate(ins, args.ref_step, nth)
     per_step = []
-    desc, nth, total_n = "", 0, 0
     for i in range(args.warmup + args.steps):
-        rate, nth, desc, n, dt = oracle_sample_rate(0, budget_s=args.ref_budget)
+        n, dt = oracle_pass(ins, rows, nth)
         if i >= args.warmup:
             per_step.append((n, dt))
+    desc = oracle_desc(rows, per_step[0][0] if per_step else 0)
     n = sum(a for a, _ in per_step)
     t = sum(b for _, b in per_step)
     value = n / t / 1e9
@@ -305,7 +326,8 @@ def main():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--ref-budget", type=float, default=8.0)
+    ap.add_argument("--ref-budget", type=float, default=8.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-step", type=float, default=1.0, help="seconds of oracle work per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
                     help="single-matrix timing instead of the sweep: stop_mode,rows,cols,nbits,group_size[,reps]")

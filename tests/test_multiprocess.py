@@ -46,7 +46,7 @@ def _worker(rank, world, port, out_dir):
     buf = io.StringIO()
     if rank != 0:
         class A:
-            gpus, steps, warmup, ref_budget = world, 1, 0, 0.1
+            gpus, steps, warmup, ref_budget, ref_step = world, 1, 0, 0.1, 0.1
         with contextlib.redirect_stdout(buf):
             bench.run_reference(A, w, r)
     cfg = bench.config_dict(w)
