@@ -39,6 +39,10 @@ def _bind(L):
                                   P, P, P, P, P, P, P, i32]
     L.oracle_dequantize.restype = i32
     L.oracle_dequantize.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, i32, i32, P]
+    L.oracle_dequantize_s8.restype = i32
+    L.oracle_dequantize_s8.argtypes = [P, P, P, i32, P, P, i64, i64, i32, i32, i32, i32, i32, P]
+    L.oracle_quantize_scale8.restype = i32
+    L.oracle_quantize_scale8.argtypes = [P, i64, i32, P, P]
     L.oracle_trace_group.restype = i32
     L.oracle_trace_group.argtypes = [P, i32, i32, f32, f32, f32, i32, P, P, P, P]
     L.oracle_pack_levels.restype = None
@@ -108,6 +112,33 @@ def dequantize(packed, scale, zero, zero_meta, rows, cols, nbits, group_size, ax
                              zero_nbits, out_dtype, _p(out))
     if rc != 0:
         raise ValueError(f"oracle_dequantize failed with code {rc}")
+    return out.view(np.float16) if out_dtype == F16 else out
+
+
+def quantize_scale8(scale, scale_group=128, L=None):
+    """8-bit quantisation of fp16 scales in runs of scale_group (reading R15).
+    Returns (codes uint8[G], meta fp32[ceil(G/scale_group), 2] = (1/sc, zc))."""
+    L = L or lib()
+    scale = np.ascontiguousarray(scale, np.float16)
+    G = scale.size
+    codes = np.zeros(G, np.uint8)
+    meta = np.zeros((max(1, -(-G // scale_group)), 2), np.float32)
+    if L.oracle_quantize_scale8(_p(scale), G, scale_group, _p(codes), _p(meta)) != 0:
+        raise ValueError("oracle_quantize_scale8 failed")
+    return codes, meta
+
+
+def dequantize_s8(packed, scale_q, scale_meta, scale_group, zero, zero_meta, rows, cols, nbits, group_size, axis=1,
+                  zero_nbits=16, out_dtype=F16, L=None):
+    """dequantize() with 8-bit scales (codes + per-run meta from quantize_scale8)."""
+    L = L or lib()
+    out = np.zeros((rows, cols), np.uint16)
+    rc = L.oracle_dequantize_s8(_p(np.ascontiguousarray(packed)), _p(np.ascontiguousarray(scale_q)),
+                                _p(np.ascontiguousarray(scale_meta, np.float32)), scale_group,
+                                _p(np.ascontiguousarray(zero)), _p(zero_meta), rows, cols, nbits, group_size, axis,
+                                zero_nbits, out_dtype, _p(out))
+    if rc != 0:
+        raise ValueError(f"oracle_dequantize_s8 failed with code {rc}")
     return out.view(np.float16) if out_dtype == F16 else out
 
 

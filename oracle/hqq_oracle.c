@@ -441,11 +441,18 @@ int oracle_quantize(const uint16_t *W, int64_t rows, int64_t cols, int dtype, in
  * Dequantise: W_r = (W_q - zero) * scale in fp32, cast to out_dtype.  With
  * zero_nbits = 8 the zero is first rebuilt as (zq - zz) * (1/sz).
  */
-int oracle_dequantize(const uint8_t *W_q_packed, const uint16_t *scale, const void *zero, const float *zero_meta,
-                      int64_t rows, int64_t cols, int nbits, int group_size, int axis, int zero_nbits, int out_dtype,
-                      uint16_t *W_out)
+/*
+ * Dequantise: W_r = (W_q - zero) * scale per element, in fp32, then rounded to
+ * the output dtype.  The scale of group j is either the stored fp16 value
+ * (scale_meta == NULL) or, for the "_s*" variant, rebuilt from its 8-bit code:
+ * (code - zc) * (1/sc) with the pair of its scale group j / scale_group.
+ */
+static int dequantize_impl(const uint8_t *W_q_packed, const void *scale, const float *scale_meta, int scale_group,
+                           const void *zero, const float *zero_meta, int64_t rows, int64_t cols, int nbits,
+                           int group_size, int axis, int zero_nbits, int out_dtype, uint16_t *W_out)
 {
     if (!valid_args(rows, cols, out_dtype, nbits, group_size, axis, 0, zero_nbits)) return 1;
+    if (scale_meta && scale_group < 1) return 1;
     const int g = group_size;
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t c = 0; c < cols; ++c) {
@@ -454,9 +461,70 @@ int oracle_dequantize(const uint8_t *W_q_packed, const uint16_t *scale, const vo
             float z;
             if (zero_nbits == 16) z = from_f16(((const uint16_t *)zero)[j]);
             else z = ((float)((const uint8_t *)zero)[j] - zero_meta[1]) * zero_meta[0];
-            float v = (q - z) * from_f16(scale[j]);
+            float sc;
+            if (scale_meta == NULL) {
+                sc = from_f16(((const uint16_t *)scale)[j]);
+            } else {
+                const float *m = scale_meta + 2 * (j / scale_group);
+                sc = ((float)((const uint8_t *)scale)[j] - m[1]) * m[0];
+            }
+            float v = (q - z) * sc;
             W_out[r * cols + c] = out_dtype == ORACLE_BF16 ? to_bf16(v) : to_f16(v);
         }
+    }
+    return 0;
+}
+
+int oracle_dequantize(const uint8_t *W_q_packed, const uint16_t *scale, const void *zero, const float *zero_meta,
+                      int64_t rows, int64_t cols, int nbits, int group_size, int axis, int zero_nbits, int out_dtype,
+                      uint16_t *W_out)
+{
+    return dequantize_impl(W_q_packed, scale, NULL, 0, zero, zero_meta, rows, cols, nbits, group_size, axis,
+                           zero_nbits, out_dtype, W_out);
+}
+
+int oracle_dequantize_s8(const uint8_t *W_q_packed, const uint8_t *scale_q, const float *scale_meta, int scale_group,
+                         const void *zero, const float *zero_meta, int64_t rows, int64_t cols, int nbits,
+                         int group_size, int axis, int zero_nbits, int out_dtype, uint16_t *W_out)
+{
+    if (scale_meta == NULL) return 1;
+    return dequantize_impl(W_q_packed, scale_q, scale_meta, scale_group, zero, zero_meta, rows, cols, nbits,
+                           group_size, axis, zero_nbits, out_dtype, W_out);
+}
+
+/*
+ * The "_s*" variant of the Llama-2 table ("Benchmark results"/"Llama-2",
+ * footnote of the table): the scale is also quantised to 8 bit, with a group
+ * size of 128.  Reading R15: the quantity quantised is the stored fp16 scale
+ * (the dequantisation multiplier 1/s); its G values, in group order, are cut
+ * into runs of scale_group consecutive values (the last run may be shorter);
+ * each run gets one round-to-nearest quantiser from its min and max:
+ *   sc = 255 / (max - min)  (1 when max == min),  zc = -min * sc,
+ *   code = clamp(round_half_even(scale * sc + zc), 0, 255),
+ *   stored meta per run: (1/sc, zc) in fp32, and the scale is rebuilt as
+ *   (code - zc) * (1/sc).
+ * No cap on sc is needed: two distinct fp16 values differ by at least 2^-24.
+ */
+int oracle_quantize_scale8(const uint16_t *scale, int64_t G, int scale_group, uint8_t *codes, float *meta)
+{
+    if (G < 0 || scale_group < 1) return 1;
+    for (int64_t k0 = 0; k0 < G; k0 += scale_group) {
+        const int64_t k1 = k0 + scale_group < G ? k0 + scale_group : G;
+        float mn = from_f16(scale[k0]), mx = mn;
+        for (int64_t i = k0 + 1; i < k1; ++i) {
+            const float v = from_f16(scale[i]);
+            if (v < mn) mn = v;
+            if (v > mx) mx = v;
+        }
+        const float sc = mx > mn ? 255.0f / (mx - mn) : 1.0f;
+        const float zc = -mn * sc;
+        for (int64_t i = k0; i < k1; ++i) {
+            float c = nearbyintf(from_f16(scale[i]) * sc + zc);
+            c = c < 0.0f ? 0.0f : (c > 255.0f ? 255.0f : c);
+            codes[i] = (uint8_t)c;
+        }
+        meta[2 * (k0 / scale_group)] = 1.0f / sc;
+        meta[2 * (k0 / scale_group) + 1] = zc;
     }
     return 0;
 }

@@ -36,7 +36,15 @@ MUTANTS = [
     ("tensor-stop-first-group", "double e = G ? total / (double)(G * g) : 0.0;",
      "double e = G ? gerr[0] / (double)g : 0.0;", 1),
     ("zero8-scale", "sz = 255.0f / (zmx - zmn);", "sz = 254.0f / (zmx - zmn);", 1),
-    ("dequant-sign", "float v = (q - z) * from_f16(scale[j]);", "float v = (q + z) * from_f16(scale[j]);", 1),
+    ("dequant-sign", "float v = (q - z) * sc;", "float v = (q + z) * sc;", 1),
+    ("scale8-zc-sign", "const float zc = -mn * sc;", "const float zc = mn * sc;", 1),
+    ("scale8-254-levels", "? 255.0f / (mx - mn) : 1.0f;", "? 254.0f / (mx - mn) : 1.0f;", 1),
+    ("scale8-truncates", "float c = nearbyintf(from_f16(scale[i]) * sc + zc);",
+     "float c = truncf(from_f16(scale[i]) * sc + zc);", 1),
+    ("scale8-one-run", "const int64_t k1 = k0 + scale_group < G ? k0 + scale_group : G;",
+     "const int64_t k1 = G;", 1),
+    ("dequant-s8-first-run-meta", "const float *m = scale_meta + 2 * (j / scale_group);",
+     "const float *m = scale_meta;", 1),
     ("pack-msb-first", "unsigned v = level << off; /* at most 8 + 7 bits */",
      "unsigned v = (off + b <= 8 ? level << (8 - b - off) : level << off);", 1),
 ]

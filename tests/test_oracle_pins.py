@@ -471,3 +471,74 @@ def test_dequant_bf16_output(orc):
     b = orc.dequantize(a["packed"], a["scale"], a["zero"], None, 8, 64, 4, 64, out_dtype=orc.BF16)
     bf = (b.astype(np.uint32) << 16).view(np.float32)
     assert np.allclose(bf, h.astype(np.float32), rtol=2 ** -8, atol=1e-6)
+
+
+# ------------------------------------------- 8-bit scales ("_s*" variant) ---
+
+def _scale8_rows():
+    rows = []
+    for line in open(os.path.join(GOLDEN, "scale8_hand_values.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        S, scales, codes, meta = [f.strip() for f in line.split("|")]
+        rows.append((int(S), [float(x) for x in scales.split()], [int(x) for x in codes.split()],
+                     [tuple(float(v) for v in m.split(",")) for m in meta.split(";")]))
+    return rows
+
+
+@pytest.mark.parametrize("row", _scale8_rows())
+def test_scale8_hand_values(orc, row):
+    S, scales, codes, meta = row
+    c, m = orc.quantize_scale8(np.array(scales, np.float16), S)
+    assert c.tolist() == codes
+    assert np.allclose(m, np.array(meta, np.float32), rtol=1e-7, atol=0)
+
+
+@pytest.mark.parametrize("G,S", [(1000, 128), (128, 128), (129, 128), (5, 128), (300, 7)])
+def test_scale8_roundtrip_bound_and_extremes(orc, G, S):
+    rng = np.random.default_rng(G + S)
+    sc = (np.abs(rng.normal(0.004, 0.002, G)) + 1e-4).astype(np.float16)
+    c, m = orc.quantize_scale8(sc, S)
+    assert m.shape == (-(-G // S), 2)
+    v = sc.astype(np.float32)
+    for k in range(m.shape[0]):
+        run = slice(k * S, min(G, (k + 1) * S))
+        x, q = v[run], c[run]
+        rebuilt = (q.astype(np.float32) - m[k, 1]) * m[k, 0]
+        span = float(x.max() - x.min())
+        # round to nearest: within half a step of 255 levels over the run's range
+        assert np.all(np.abs(rebuilt - x) <= span / 510 * (1 + 1e-5) + 1e-9)
+        if span > 0:
+            assert q[np.argmin(x)] == 0 and q[np.argmax(x)] == 255
+        else:
+            assert np.all(q == 0) and np.all(rebuilt == x)
+
+
+def test_scale8_runs_are_independent(orc):
+    rng = np.random.default_rng(3)
+    sc = (np.abs(rng.normal(0.004, 0.002, 512)) + 1e-4).astype(np.float16)
+    c0, m0 = orc.quantize_scale8(sc, 128)
+    sc2 = sc.copy()
+    sc2[128:256] *= np.float16(3)  # only run 1 changes
+    c1, m1 = orc.quantize_scale8(sc2, 128)
+    for k in (0, 2, 3):
+        assert np.array_equal(c0[k * 128:(k + 1) * 128], c1[k * 128:(k + 1) * 128]) and np.array_equal(m0[k], m1[k])
+    assert not np.array_equal(m0[1], m1[1])
+
+
+def test_dequant_with_8bit_scale(orc):
+    """dequantize_s8 rebuilds each group's scale from its code and run pair, and
+    otherwise equals dequantize with those rebuilt scales stored in fp16
+    wherever the rebuilt scale is exact in fp16."""
+    W = (np.random.default_rng(4).normal(0, 0.02, (64, 256))).astype(np.float16)
+    o = orc.quantize(W, 4, 32, 1, 0.7, 1.0, 1.01, 20, orc.STOP_GROUP, 16)
+    c, m = orc.quantize_scale8(o["scale"], 16)
+    d8 = orc.dequantize_s8(o["packed"], c, m, 16, o["zero"], None, 64, 256, 4, 32)
+    rebuilt = np.array([(np.float32(c[j]) - m[j // 16, 1]) * m[j // 16, 0] for j in range(c.size)], np.float32)
+    # a worked element: group 0, element 0
+    q = orc.unpack_levels(o["packed"], 64, 256, 4, 1).reshape(64, 256)
+    v = np.float32(np.float32(q[0, 0]) - np.float32(o["zero"][0])) * rebuilt[0]
+    assert d8[0, 0] == np.float16(v)
+    # close to the fp16-scale dequantisation: the scale moved by at most half a step of its run
+    d16 = orc.dequantize(o["packed"], o["scale"], o["zero"], None, 64, 256, 4, 32).astype(np.float32)
+    assert np.max(np.abs(d8.astype(np.float32) - d16)) < 0.02 * np.abs(d16).max()
