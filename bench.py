@@ -296,8 +296,44 @@ def config_dict(world):
             "l2": "inputs 270 MB > 126 MB L2; consecutive calls use different matrices"}
 
 
+def run_scale8_case(spec):
+    """Time hqq_quantize_scale8 (8-bit scales in runs of S) on G synthetic fp16
+    scales: "scale8,G[,S[,reps]]".  HBM-bound: 2 B read + 1 B written per scale
+    and 8 B per run."""
+    from calibration_free_weight_b200 import hqq
+    v = spec.split(",")[1:]
+    G = int(v[0])
+    S = int(v[1]) if len(v) > 1 else 128
+    reps = int(v[2]) if len(v) > 2 else 20
+    torch.cuda.set_device(0)
+    q = {"scale": synth.scales(G, seed=G).cuda()}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # 256 MB > L2: each call starts cold
+    hqq.quantize_scale8(q, S)
+    ev = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        rc = hqq.hqq_quantize_scale8(q["scale"], G, S, q["scale_q"], q["scale_meta"])
+        b.record()
+        if rc != hqq.HQQ_OK:
+            raise RuntimeError(hqq.hqq_status_string(rc))
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    ms = sorted(a.elapsed_time(b) for a, b in ev)
+    med = ms[len(ms) // 2]
+    nbytes = 3 * G + 8 * (-(-G // S))
+    hbm, _, kind = peaks()
+    print(json.dumps({"case": spec, "ms_median": med, "ms_min": ms[0], "bytes": nbytes,
+                      "gbs": nbytes / (med / 1e3) / 1e9, "hbm_peak_gbs": hbm, "peak_kind": kind,
+                      "frac": nbytes / (med / 1e3) / 1e9 / hbm, "l2": "flushed before every call"}))
+
+
 def run_case(spec):
     """Time hqq_quantize on one synthetic bf16 matrix (used for kernel profiles)."""
+    if spec.startswith("scale8"):
+        run_scale8_case(spec)
+        return
     from calibration_free_weight_b200 import hqq
     v = [int(x) for x in spec.split(",")]
     mode, rows, cols, nbits, g = v[:5]
@@ -330,7 +366,8 @@ def main():
     ap.add_argument("--ref-step", type=float, default=1.0, help="seconds of oracle work per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
-                    help="single-matrix timing instead of the sweep: stop_mode,rows,cols,nbits,group_size[,reps]")
+                    help="single-matrix timing instead of the sweep: stop_mode,rows,cols,nbits,group_size[,reps]; "
+                         "or scale8,G[,S[,reps]] for the 8-bit scale quantiser")
     args = ap.parse_args()
     if args.case:
         run_case(args.case)

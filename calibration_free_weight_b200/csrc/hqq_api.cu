@@ -150,25 +150,38 @@ int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits
                                debug_best_iter, debug_best_err, debug_zero_f32, stream);
 }
 
-int hqq_dequantize(const void* W_q_packed, const void* scale, const void* zero, const void* zero_meta, int64_t rows,
-                   int64_t cols, int nbits, int group_size, int axis, int zero_nbits, int out_dtype, void* W_out,
-                   void* stream) {
+}  // extern "C"
+
+namespace {
+
+// hqq_dequantize and hqq_dequantize_s8: scale8 == true reads 8-bit scale codes
+// and their per-run meta instead of fp16 scales.
+int dequantize_entry(const void* W_q_packed, const void* scale, const void* scale_meta, int scale_group, bool scale8,
+                     const void* zero, const void* zero_meta, int64_t rows, int64_t cols, int nbits, int group_size,
+                     int axis, int zero_nbits, int out_dtype, void* W_out, void* stream) {
     if (out_dtype != HQQ_F16 && out_dtype != HQQ_BF16) return HQQ_ERR_DTYPE;
     if (!valid_nbits(nbits)) return HQQ_ERR_INVALID_ARG;
     const int sh = check_shape(rows, cols, group_size, axis);
     if (sh != HQQ_OK) return sh;
     if (zero_nbits != 8 && zero_nbits != 16) return HQQ_ERR_INVALID_ARG;
+    if (scale8 && scale_group < 1) return HQQ_ERR_INVALID_ARG;
     if (rows * cols == 0) return HQQ_OK;
     if (!is_device_ptr(W_q_packed) || !is_device_ptr(scale) || !is_device_ptr(zero) || !is_device_ptr(W_out))
         return HQQ_ERR_INVALID_ARG;
     if (zero_nbits == 8 && !is_device_ptr(zero_meta)) return HQQ_ERR_INVALID_ARG;
-    if (!aligned(W_q_packed, 16) || !aligned(scale, 2) || !aligned(W_out, 16)) return HQQ_ERR_ALIGN;
+    if (scale8 && !is_device_ptr(scale_meta)) return HQQ_ERR_INVALID_ARG;
+    if (!aligned(W_q_packed, 16) || !aligned(W_out, 16)) return HQQ_ERR_ALIGN;
+    if (!scale8 && !aligned(scale, 2)) return HQQ_ERR_ALIGN;
+    if (scale8 && !aligned(scale_meta, 4)) return HQQ_ERR_ALIGN;
     if (zero_nbits == 16 && !aligned(zero, 2)) return HQQ_ERR_ALIGN;
     if (zero_nbits == 8 && !aligned(zero_meta, 4)) return HQQ_ERR_ALIGN;
     if (axis == 1 && cols % 8 != 0) return HQQ_ERR_SHAPE;  // implied by g | cols, kept explicit
     hqq::DequantArgs a{};
     a.packed = static_cast<const uint8_t*>(W_q_packed);
-    a.scale = static_cast<const uint16_t*>(scale);
+    a.scale = scale8 ? nullptr : static_cast<const uint16_t*>(scale);
+    a.scale_q = scale8 ? static_cast<const uint8_t*>(scale) : nullptr;
+    a.scale_meta = scale8 ? static_cast<const float*>(scale_meta) : nullptr;
+    a.scale_group = scale8 ? scale_group : 1;
     a.zero = zero;
     a.zero_meta = static_cast<const float*>(zero_meta);
     a.rows = rows;
@@ -180,6 +193,39 @@ int hqq_dequantize(const void* W_q_packed, const void* scale, const void* zero, 
     a.out_dtype = out_dtype;
     a.out = W_out;
     if (hqq::launch_dequant(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return HQQ_ERR_CUDA;
+    }
+    return HQQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hqq_dequantize(const void* W_q_packed, const void* scale, const void* zero, const void* zero_meta, int64_t rows,
+                   int64_t cols, int nbits, int group_size, int axis, int zero_nbits, int out_dtype, void* W_out,
+                   void* stream) {
+    return dequantize_entry(W_q_packed, scale, nullptr, 0, false, zero, zero_meta, rows, cols, nbits, group_size, axis,
+                            zero_nbits, out_dtype, W_out, stream);
+}
+
+int hqq_dequantize_s8(const void* W_q_packed, const void* scale_q, const void* scale_meta, int scale_group,
+                      const void* zero, const void* zero_meta, int64_t rows, int64_t cols, int nbits, int group_size,
+                      int axis, int zero_nbits, int out_dtype, void* W_out, void* stream) {
+    return dequantize_entry(W_q_packed, scale_q, scale_meta, scale_group, true, zero, zero_meta, rows, cols, nbits,
+                            group_size, axis, zero_nbits, out_dtype, W_out, stream);
+}
+
+int hqq_quantize_scale8(const void* scale, int64_t num_groups, int scale_group, void* scale_q, void* scale_meta,
+                        void* stream) {
+    if (num_groups < 0 || scale_group < 1) return HQQ_ERR_INVALID_ARG;
+    if (num_groups == 0) return HQQ_OK;
+    if (!is_device_ptr(scale) || !is_device_ptr(scale_q) || !is_device_ptr(scale_meta)) return HQQ_ERR_INVALID_ARG;
+    if (!aligned(scale, 2) || !aligned(scale_meta, 4)) return HQQ_ERR_ALIGN;
+    if (hqq::launch_scale8(static_cast<const uint16_t*>(scale), num_groups, scale_group,
+                           static_cast<uint8_t*>(scale_q), static_cast<float*>(scale_meta),
+                           static_cast<cudaStream_t>(stream)) != cudaSuccess) {
         cudaGetLastError();
         return HQQ_ERR_CUDA;
     }

@@ -60,7 +60,10 @@ struct SolveArgs {
 
 struct DequantArgs {
     const uint8_t* packed;
-    const uint16_t* scale;
+    const uint16_t* scale;      // fp16 scales (scale_meta == null), else
+    const uint8_t* scale_q;     // 8-bit codes and
+    const float* scale_meta;    // (1/sc, zc) per run of scale_group
+    int scale_group;
     const void* zero;
     const float* zero_meta;
     int64_t rows, cols;
@@ -71,6 +74,7 @@ struct DequantArgs {
 // Launchers: return cudaSuccess or the launch error.
 cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream);
 cudaError_t launch_dequant(const DequantArgs& a, cudaStream_t stream);
+cudaError_t launch_scale8(const uint16_t* scale, int64_t G, int S, uint8_t* codes, float* meta, cudaStream_t stream);
 
 // hqq_quantize with an option to cut group-mode work into slices that fit a
 // smaller workspace (used by hqq_quantize_noalloc).

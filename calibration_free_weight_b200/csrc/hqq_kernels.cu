@@ -769,6 +769,96 @@ __global__ void __launch_bounds__(256) zero_q8_kernel(const float* zbest, int64_
     }
 }
 
+// ------------------------------------------------------ 8-bit scales -----
+
+// The "_s*" variant (table footnote of "Benchmark results"/"Llama-2"): one
+// round-to-nearest 8-bit quantiser per run of S consecutive fp16 scales, from
+// the run's min and max (sc = 255/(max-min), 1 for a constant run; zc =
+// -min*sc; meta (1/sc, zc)).  HBM-bound: 2 bytes read, 1 written per scale.
+__device__ __forceinline__ float2 scale8_pair(float mn, float mx) {
+    const float sc = mx > mn ? __fdiv_rn(255.0f, __fsub_rn(mx, mn)) : 1.0f;
+    return make_float2(sc, __fmul_rn(-mn, sc));
+}
+
+__device__ __forceinline__ uint32_t scale8_code(float v, float2 p) {
+    uint32_t code;
+    round_clamp(__fadd_rn(__fmul_rn(v, p.x), p.y), 255.0f, &code);
+    return code;
+}
+
+// Any S: one warp per run, lanes stride over the run.
+__device__ __forceinline__ void scale8_run(const uint16_t* scale, int64_t G, int S, int64_t r, uint8_t* codes,
+                                           float* meta) {
+    const int lane = threadIdx.x & 31;
+    const int64_t k0 = r * S;
+    const int len = static_cast<int>(G - k0 < S ? G - k0 : S);
+    float mn = FLT_MAX, mx = -FLT_MAX;
+    for (int i = lane; i < len; i += 32) {
+        const float v = __half2float(__ushort_as_half(__ldg(scale + k0 + i)));
+        mn = fminf(mn, v);
+        mx = fmaxf(mx, v);
+    }
+    mn = seg_min(mn, 32);
+    mx = seg_max(mx, 32);
+    const float2 p = scale8_pair(mn, mx);
+    for (int i = lane; i < len; i += 32)
+        codes[k0 + i] = static_cast<uint8_t>(scale8_code(__half2float(__ushort_as_half(__ldg(scale + k0 + i))), p));
+    if (lane == 0) {
+        meta[2 * r] = __fdiv_rn(1.0f, p.x);
+        meta[2 * r + 1] = p.y;
+    }
+}
+
+__global__ void __launch_bounds__(256) scale8_kernel(const uint16_t* scale, int64_t G, int S, uint8_t* codes,
+                                                      float* meta) {
+    const int64_t nruns = (G + S - 1) / S;
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); r < nruns;
+         r += static_cast<int64_t>(gridDim.x) * 8)
+        scale8_run(scale, G, S, r, codes, meta);
+}
+
+// S == 128, 16-byte aligned scales and codes: a warp takes 4 runs, 8 lanes
+// per run, 16 consecutive scales per lane (two 16-byte loads, one 16-byte
+// store of codes); a warp whose runs are not all full uses scale8_run.
+__global__ void __launch_bounds__(256) scale8_kernel_128(const uint16_t* scale, int64_t G, uint8_t* codes,
+                                                          float* meta) {
+    const int lane = threadIdx.x & 31, part = lane & 7;
+    const int64_t nruns = (G + 127) / 128;
+    for (int64_t w = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); w * 4 < nruns;
+         w += static_cast<int64_t>(gridDim.x) * 8) {
+        if ((w + 1) * 4 * 128 > G) {  // the tail: a partial run or fewer than 4 runs
+            for (int64_t r = w * 4; r < nruns && r < (w + 1) * 4; ++r) scale8_run(scale, G, 128, r, codes, meta);
+            continue;
+        }
+        const int64_t r = w * 4 + (lane >> 3);
+        const int64_t e0 = r * 128 + part * 16;
+        const uint4* src = reinterpret_cast<const uint4*>(scale + e0);
+        const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+        float v[16];
+        unpack8<0>(u0, v);
+        unpack8<0>(u1, v + 8);
+        float mn = v[0], mx = v[0];
+#pragma unroll
+        for (int i = 1; i < 16; ++i) {
+            mn = fminf(mn, v[i]);
+            mx = fmaxf(mx, v[i]);
+        }
+        mn = seg_min(mn, 8);
+        mx = seg_max(mx, 8);
+        const float2 p = scale8_pair(mn, mx);
+        uint32_t c[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+            c[t] = scale8_code(v[4 * t], p) | (scale8_code(v[4 * t + 1], p) << 8) |
+                   (scale8_code(v[4 * t + 2], p) << 16) | (scale8_code(v[4 * t + 3], p) << 24);
+        *reinterpret_cast<uint4*>(codes + e0) = make_uint4(c[0], c[1], c[2], c[3]);
+        if (part == 0) {
+            meta[2 * r] = __fdiv_rn(1.0f, p.x);
+            meta[2 * r + 1] = p.y;
+        }
+    }
+}
+
 // -------------------------------------------------------- dequantise -----
 
 template <int OUT_DT>
@@ -791,13 +881,22 @@ __device__ __forceinline__ uint64_t load_piece(const uint8_t* src, int nbits) {
 
 struct DqParams {
     const uint8_t* packed;
-    const uint16_t* scale;
+    const uint16_t* scale;     // fp16 scales, or
+    const uint8_t* scale_q;    // 8-bit scale codes with
+    const float* scale_meta;   // (1/sc, zc) per run of scale_group (null: fp16 scales)
+    int scale_group;
     const void* zero;
     const float* meta;
     int64_t rows, cols;
     int nbits, g, zero_nbits;
     uint16_t* out;
 };
+
+__device__ __forceinline__ float dq_scale(const DqParams& d, int64_t j) {
+    if (!d.scale_meta) return __half2float(__ushort_as_half(d.scale[j]));
+    const float* m = d.scale_meta + 2 * (j / d.scale_group);
+    return __fmul_rn(__fsub_rn(static_cast<float>(d.scale_q[j]), m[1]), m[0]);
+}
 
 __device__ __forceinline__ float dq_zero(const DqParams& d, int64_t j) {
     if (d.zero_nbits == 16) return __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(d.zero)[j]));
@@ -815,7 +914,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const DqParams d) {
             const uint64_t v = load_piece(d.packed + pc * d.nbits, d.nbits);
             const int64_t j = pc * kPiece / d.g;
             const float z = dq_zero(d, j);
-            const float sc = __half2float(__ushort_as_half(d.scale[j]));
+            const float sc = dq_scale(d, j);
             uint32_t o[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -836,7 +935,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const DqParams d) {
                 v |= static_cast<uint64_t>(d.packed[(m * d.nbits + b) * d.cols + c]) << (8 * b);
             const int64_t j = (m * kPiece / d.g) * d.cols + c;
             const float z = dq_zero(d, j);
-            const float sc = __half2float(__ushort_as_half(d.scale[j]));
+            const float sc = dq_scale(d, j);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float q = static_cast<float>(static_cast<uint32_t>(v >> (i * d.nbits)) & mask);
@@ -1111,10 +1210,28 @@ cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream) {
     return err;
 }
 
+cudaError_t launch_scale8(const uint16_t* scale, int64_t G, int S, uint8_t* codes, float* meta,
+                          cudaStream_t stream) {
+    const int64_t runs = (G + S - 1) / S;
+    if (runs == 0) return cudaSuccess;
+    const bool vec = S == 128 && (reinterpret_cast<uintptr_t>(scale) & 15) == 0 &&
+                     (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
+    const int64_t warps = vec ? (runs + 3) / 4 : runs;
+    int64_t blocks = (warps + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(device_info().sms) * 64;
+    if (blocks > cap) blocks = cap;
+    if (vec) scale8_kernel_128<<<static_cast<int>(blocks), 256, 0, stream>>>(scale, G, codes, meta);
+    else scale8_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(scale, G, S, codes, meta);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_dequant(const DequantArgs& a, cudaStream_t stream) {
     DqParams d;
     d.packed = a.packed;
     d.scale = a.scale;
+    d.scale_q = a.scale_q;
+    d.scale_meta = a.scale_meta;
+    d.scale_group = a.scale_group;
     d.zero = a.zero;
     d.meta = a.zero_meta;
     d.rows = a.rows;

@@ -18,7 +18,8 @@ HQQ_F16, HQQ_BF16 = 0, 1
 HQQ_STOP_GROUP, HQQ_STOP_TENSOR, HQQ_STOP_NONE = 0, 1, 2
 
 EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_quantize", "hqq_dequantize",
-            "hqq_get_status", "hqq_status_string", "hqq_quantize_noalloc")
+            "hqq_get_status", "hqq_status_string", "hqq_quantize_noalloc", "hqq_quantize_scale8",
+            "hqq_dequantize_s8")
 HQQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -43,6 +44,10 @@ def _load():
     L.hqq_get_status.argtypes = [P, P]
     L.hqq_status_string.restype = C.c_char_p
     L.hqq_status_string.argtypes = [i32]
+    L.hqq_quantize_scale8.restype = i32
+    L.hqq_quantize_scale8.argtypes = [P, i64, i32, P, P, P]
+    L.hqq_dequantize_s8.restype = i32
+    L.hqq_dequantize_s8.argtypes = [P, P, P, i32, P, P, i64, i64, i32, i32, i32, i32, i32, P, P]
     L.hqq_quantize_noalloc.restype = i32
     L.hqq_quantize_noalloc.argtypes = [P, i64, i64, i32, i32, i32, i32, f32, f32, f32, i32, i32, i32,
                                        P, P, P, P, P, P, P, P]
@@ -111,6 +116,18 @@ def hqq_dequantize(W_q_packed, scale, zero, zero_meta, rows, cols, nbits, group_
                               group_size, axis, zero_nbits, out_dtype, _ptr(W_out), _stream(stream))
 
 
+def hqq_quantize_scale8(scale, num_groups, scale_group, scale_q, scale_meta, stream=None):
+    return lib.hqq_quantize_scale8(_ptr(scale), num_groups, scale_group, _ptr(scale_q), _ptr(scale_meta),
+                                   _stream(stream))
+
+
+def hqq_dequantize_s8(W_q_packed, scale_q, scale_meta, scale_group, zero, zero_meta, rows, cols, nbits, group_size,
+                      axis, zero_nbits, out_dtype, W_out, stream=None):
+    return lib.hqq_dequantize_s8(_ptr(W_q_packed), _ptr(scale_q), _ptr(scale_meta), scale_group, _ptr(zero),
+                                 _ptr(zero_meta), rows, cols, nbits, group_size, axis, zero_nbits, out_dtype,
+                                 _ptr(W_out), _stream(stream))
+
+
 def hqq_get_status(workspace, stream=None):
     return lib.hqq_get_status(_ptr(workspace), _stream(stream))
 
@@ -161,6 +178,32 @@ def quantize(W, nbits=4, group_size=64, axis=1, p=0.7, beta=1.0, kappa=1.01, ite
                       stream)
     if rc != HQQ_OK:
         raise HQQError(rc, "hqq_quantize")
+    return out
+
+
+def quantize_scale8(q, scale_group=128, stream=None):
+    """8-bit scales (the "_s*" variant) for the outputs of quantize(): adds
+    q["scale_q"] (uint8[G]) and q["scale_meta"] (fp32[ceil(G/S), 2])."""
+    G = q["scale"].numel()
+    dev = q["scale"].device
+    q["scale_q"] = torch.empty(G, dtype=torch.uint8, device=dev)
+    q["scale_meta"] = torch.empty(max(1, -(-G // scale_group)), 2, dtype=torch.float32, device=dev)
+    q["scale_group"] = scale_group
+    rc = hqq_quantize_scale8(q["scale"], G, scale_group, q["scale_q"], q["scale_meta"], stream)
+    if rc != HQQ_OK:
+        raise HQQError(rc, "hqq_quantize_scale8")
+    return q
+
+
+def dequantize_s8(q, rows, cols, nbits, group_size, axis=1, zero_nbits=16, out_dtype=torch.float16, out=None,
+                  stream=None):
+    """dequantize() with the 8-bit scales of quantize_scale8()."""
+    if out is None:
+        out = torch.empty(rows, cols, dtype=out_dtype, device=q["scale"].device)
+    rc = hqq_dequantize_s8(q["packed"], q["scale_q"], q["scale_meta"], q["scale_group"], q["zero"], q["zero_meta"],
+                           rows, cols, nbits, group_size, axis, zero_nbits, _DT[out_dtype], out, stream)
+    if rc != HQQ_OK:
+        raise HQQError(rc, "hqq_dequantize_s8")
     return out
 
 

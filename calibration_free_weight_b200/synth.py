@@ -56,3 +56,15 @@ class ModelShape:
 LLAMA2_7B = ModelShape("llama-2-7b", 32, 4096, 11008, 4096)
 LLAMA2_13B = ModelShape("llama-2-13b", 40, 5120, 13824, 5120)
 LLAMA2_70B = ModelShape("llama-2-70b", 80, 8192, 28672, 1024)
+
+
+def scales(G: int, seed: int) -> torch.Tensor:
+    """Seeded synthetic per-group scales (fp16, positive, spread like the
+    dequantisation multipliers of 0.02-std weights at 2-4 bits), with a few
+    constant runs: 0.004 * |N(1, 0.5)| + 1e-4, and every 977th block of 128
+    set to one value."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    v = 0.004 * torch.randn(G, generator=gen, dtype=torch.float32).mul(0.5).add(1.0).abs() + 1e-4
+    for b in range(0, G // 128, 977):
+        v[b * 128:(b + 1) * 128] = v[b * 128]
+    return v.to(torch.float16)

@@ -142,6 +142,40 @@ int hqq_dequantize(const void* W_q_packed, const void* scale, const void* zero, 
                    int64_t rows, int64_t cols, int nbits, int group_size, int axis, int zero_nbits,
                    int out_dtype, void* W_out, void* stream);
 
+/*
+ * hqq_quantize_scale8 -- the "_s*" variant of the Llama-2 table
+ * (techreport.ngo, "Weight-only quantization without the calibration tax",
+ * section "Benchmark results" / "Llama-2", table footnote: the scale is also
+ * quantised to 8 bit with a group size of 128).  The pages give no formula;
+ * this library reads it as one round-to-nearest 8-bit quantiser per run of
+ * scale_group consecutive scales (in group order; the last run may be shorter):
+ *   sc = 255 / (max - min) over the run (1 when max == min), zc = -min * sc,
+ *   code = clamp(round_half_even(scale * sc + zc), 0, 255),
+ * all in fp32 from the fp16 scales, stored meta per run (1/sc, zc) in fp32.
+ * The codes W_q are not recomputed; hqq_dequantize_s8 rebuilds each scale as
+ * (code - zc) * (1/sc).
+ *   scale        device fp16[G] from hqq_quantize, 2-byte aligned (read only).
+ *   num_groups   G >= 0.
+ *   scale_group  run length S >= 1 (128 in the pages).
+ *   scale_q      device uint8[G] (output).
+ *   scale_meta   device fp32[2 * ceil(G / S)] (output), 4-byte aligned.
+ *   stream       cudaStream_t as void*.
+ * Returns HQQ_OK, HQQ_ERR_INVALID_ARG (bad pointer or S < 1, G < 0),
+ * HQQ_ERR_ALIGN or HQQ_ERR_CUDA.  Allocates nothing.
+ */
+int hqq_quantize_scale8(const void* scale, int64_t num_groups, int scale_group, void* scale_q, void* scale_meta,
+                        void* stream);
+
+/*
+ * hqq_dequantize with 8-bit scales: as hqq_dequantize, but the scale of
+ * group j is (scale_q[j] - zc) * (1/sc) with the (1/sc, zc) pair of run
+ * j / scale_group from hqq_quantize_scale8.  scale_q is device uint8[G],
+ * scale_meta device fp32[2 * ceil(G / scale_group)] (4-byte aligned).
+ */
+int hqq_dequantize_s8(const void* W_q_packed, const void* scale_q, const void* scale_meta, int scale_group,
+                      const void* zero, const void* zero_meta, int64_t rows, int64_t cols, int nbits,
+                      int group_size, int axis, int zero_nbits, int out_dtype, void* W_out, void* stream);
+
 /* Synchronise `stream` and return the device status word held in `workspace`
  * by the last hqq_quantize on it (HQQ_OK), or HQQ_ERR_CUDA if the
  * synchronisation or copy fails. */

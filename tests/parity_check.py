@@ -176,17 +176,42 @@ def check(W_cpu, params, gpu, orc=None, sample=None, report=None):
     return rep
 
 
-def check_reconstruction(W_cpu, params, gpu, gpu_deq, orc):
-    """Tensor lp error of the GPU's and the oracle's dequantised weights; the GPU
-    dequantiser against the oracle's dequantisation of the GPU's own codes."""
+def gpu_dequantizer(hq):
+    """A function running the GPU dequantiser (through the C ABI) on given
+    numpy arrays -- used with the oracle's own outputs, so that no oracle input
+    comes from the CUDA path."""
+    import torch
+
+    def run(q, rows, cols, nbits, g, axis, zero_nbits, out_code, scale8=None):
+        dev = {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in q.items() if v is not None}
+        out_dt = torch.float16 if out_code == oracle.F16 else torch.bfloat16
+        out = torch.empty(rows, cols, dtype=out_dt, device="cuda")
+        if scale8 is None:
+            rc = hq.hqq_dequantize(dev["packed"], dev["scale"], dev["zero"], dev.get("zero_meta"), rows, cols, nbits,
+                                   g, axis, zero_nbits, hq.HQQ_F16 if out_code == oracle.F16 else hq.HQQ_BF16, out)
+        else:
+            rc = hq.hqq_dequantize_s8(dev["packed"], dev["scale_q"], dev["scale_meta"], scale8, dev["zero"],
+                                      dev.get("zero_meta"), rows, cols, nbits, g, axis, zero_nbits,
+                                      hq.HQQ_F16 if out_code == oracle.F16 else hq.HQQ_BF16, out)
+        assert rc == hq.HQQ_OK, hq.hqq_status_string(rc)
+        torch.cuda.synchronize()
+        o = out.cpu()
+        return (o.numpy() if out_dt == torch.float16 else o.view(torch.int16).numpy()).view(np.uint16)
+    return run
+
+
+def check_reconstruction(W_cpu, params, gpu_deq, orc, gpu_dequant):
+    """The GPU dequantiser bit-exact against the oracle's dequantisation, both
+    run on the oracle's outputs; and the tensor lp error of the GPU's
+    dequantised weights (its own codes) against the oracle's."""
     nb, g, axis, zb, p = params["nbits"], params["group_size"], params["axis"], params["zero_nbits"], params["p"]
     rows, cols = W_cpu.shape
     out_dt = oracle.F16 if gpu_deq.dtype == np.float16 else oracle.BF16
-    meta = gpu.get("zero_meta")
-    ref = oracle.dequantize(gpu["packed"], gpu["scale"], gpu["zero"], meta, rows, cols, nb, g, axis, zb, out_dt)
-    assert np.array_equal(ref.view(np.uint16), gpu_deq.view(np.uint16)), "dequantiser differs from the oracle's"
     od = oracle.dequantize(orc["packed"], orc["scale"], orc["zero"], orc["zero_meta"], rows, cols, nb, g, axis, zb,
                            out_dt)
+    got = gpu_dequant(dict(packed=orc["packed"], scale=orc["scale"], zero=orc["zero"], zero_meta=orc["zero_meta"]),
+                      rows, cols, nb, g, axis, zb, out_dt)
+    assert np.array_equal(od.view(np.uint16), got), "dequantiser differs from the oracle's"
     Wf = w_float(W_cpu).astype(np.float64)
 
     def tofloat(a):

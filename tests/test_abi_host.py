@@ -93,6 +93,25 @@ def test_dequantize_rejects_on_host(hq):
     assert L.hqq_dequantize(None, None, None, None, 0, 64, 4, 64, 1, 16, 0, None, None) == 0
 
 
+def test_scale8_entry_points_reject_on_host(hq):
+    L = hq.lib
+    # run length below 1, negative count: rejected before any pointer is looked at
+    assert L.hqq_quantize_scale8(None, 10, 0, None, None, None) == hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_quantize_scale8(None, -1, 128, None, None, None) == hq.HQQ_ERR_INVALID_ARG
+    # nothing to do
+    assert L.hqq_quantize_scale8(None, 0, 128, None, None, None) == hq.HQQ_OK
+    # host (non-device) pointers
+    buf = C.create_string_buffer(64)
+    p = C.cast(buf, C.c_void_p).value
+    assert L.hqq_quantize_scale8(p, 8, 128, p, p, None) == hq.HQQ_ERR_INVALID_ARG
+    # dequantize with 8-bit scales: bad run length, bad dtype, bad shape, empty
+    args = (None, None, None)
+    assert L.hqq_dequantize_s8(*args, 0, None, None, 64, 64, 4, 64, 1, 16, 0, None, None) == hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_dequantize_s8(*args, 128, None, None, 64, 64, 4, 64, 1, 16, 7, None, None) == hq.HQQ_ERR_DTYPE
+    assert L.hqq_dequantize_s8(*args, 128, None, None, 64, 96, 4, 64, 1, 16, 0, None, None) == hq.HQQ_ERR_SHAPE
+    assert L.hqq_dequantize_s8(*args, 128, None, None, 0, 64, 4, 64, 1, 16, 0, None, None) == hq.HQQ_OK
+
+
 def test_status_strings(hq):
     for code in range(9):
         s = hq.hqq_status_string(code)

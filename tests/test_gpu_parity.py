@@ -51,7 +51,7 @@ def _run(hq, W_cpu, prm, check_recon=True):
                                 out_dt)
             d = deq.cpu()
             d = d.numpy() if out_dt == torch.float16 else d.view(torch.int16).numpy().view(np.uint16)
-            pc.check_reconstruction(W_cpu, prm, gpu, d, orc)
+            pc.check_reconstruction(W_cpu, prm, d, orc, pc.gpu_dequantizer(hq))
     return rep, gpu, orc
 
 
