@@ -329,6 +329,63 @@ def run_scale8_case(spec):
                       "frac": nbytes / (med / 1e3) / 1e9 / hbm, "l2": "flushed before every call"}))
 
 
+LLAMA70B = [("q", 8192, 8192), ("k", 1024, 8192), ("v", 1024, 8192), ("o", 8192, 8192),
+            ("gate", 28672, 8192), ("up", 28672, 8192), ("down", 8192, 28672)]
+
+
+def run_stream(args):
+    """Llama-2-70B-shaped model (80 layers x q, k, v, o, gate, up, down; fp16)
+    streamed layer by layer from pinned host memory through hqq_quantize_stream
+    at b2 g16 and b4 g128, 8-bit zero, group stop.  One layer of synthetic
+    weights (layer 0's seeds) is generated and pinned, and every layer streams
+    those buffers: each layer's copy-in, solve and copy-out is real, only the
+    values repeat (137 GB of distinct synthetic weights would take minutes to
+    generate).  Reports the end-to-end wall time of the blocking call and, for
+    the same matrices resident on the device, the solver's throughput."""
+    from calibration_free_weight_b200 import hqq
+    torch.cuda.set_device(0)
+    layers = args.layers
+    Ws = [synth.weight(r, c, seed=synth.seed_for(0, n), dtype=torch.float16).pin_memory() for n, r, c in LLAMA70B]
+    w_layer = sum(r * c for _, r, c in LLAMA70B)
+    res = []
+    for nbits, g in ((2, 16), (4, 128)):
+        outs = [hqq.host_outputs(r, c, nbits, g, zero_nbits=8) for _, r, c in LLAMA70B]
+        buf = hqq.quantize_stream(Ws, outs, nbits, g, zero_nbits=8)  # warm-up: one layer
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        hqq.quantize_stream(Ws * layers, outs * layers, nbits, g, zero_nbits=8, device_buffer=buf)
+        wall = time.perf_counter() - t0
+        del buf
+        # the same matrices resident on the device: solver time per layer (CUDA events)
+        dev = [w.cuda() for w in Ws]
+        q = [hqq.alloc_outputs(r, c, nbits, g, 1, 0, 8) for _, r, c in LLAMA70B]
+        for _ in range(2):
+            for w, o in zip(dev, q):
+                hqq.quantize(w, nbits, g, zero_nbits=8, out=o)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for w, o in zip(dev, q):
+            hqq.quantize(w, nbits, g, zero_nbits=8, out=o)
+        b.record()
+        torch.cuda.synchronize()
+        layer_ms = a.elapsed_time(b)
+        alg = sum(algorithmic_bytes(r, c, nbits, g, 8) for _, r, c in LLAMA70B)
+        hbm, _, kind = peaks()
+        h2d = 2 * w_layer * layers
+        d2h = sum(o["packed"].numel() + o["scale"].numel() * 2 + o["zero"].numel() + 8 for o in outs) * layers
+        res.append({"nbits": nbits, "group_size": g, "e2e_s": wall, "e2e_gweights_s": w_layer * layers / wall / 1e9,
+                    "h2d_bytes": h2d, "d2h_bytes": d2h, "h2d_gbs_effective": h2d / wall / 1e9,
+                    "device_resident": {"ms_per_layer": layer_ms, "gweights_s": w_layer / (layer_ms / 1e3) / 1e9,
+                                        "algorithmic_gbs": alg / (layer_ms / 1e3) / 1e9,
+                                        "hbm_frac": alg / (layer_ms / 1e3) / 1e9 / hbm, "peak_kind": kind,
+                                        "solve_s_all_layers": layer_ms / 1e3 * layers}})
+        del dev, q
+        torch.cuda.empty_cache()
+    print(json.dumps({"workload": "llama2-70b-stream", "layers": layers, "weights": w_layer * layers,
+                      "dtype_in": "fp16", "zero": "8-bit", "stop_mode": "group", "host": "pinned",
+                      "data": "synthetic; one layer's buffers streamed for every layer", "results": res}))
+
+
 def run_case(spec):
     """Time hqq_quantize on one synthetic bf16 matrix (used for kernel profiles)."""
     if spec.startswith("scale8"):
@@ -368,7 +425,12 @@ def main():
     ap.add_argument("--case", default=None,
                     help="single-matrix timing instead of the sweep: stop_mode,rows,cols,nbits,group_size[,reps]; "
                          "or scale8,G[,S[,reps]] for the 8-bit scale quantiser")
+    ap.add_argument("--workload", default="llama2-7b-mlp-sweep", choices=["llama2-7b-mlp-sweep", "llama2-70b-stream"])
+    ap.add_argument("--layers", type=int, default=80, help="layers of the llama2-70b-stream workload")
     args = ap.parse_args()
+    if args.workload == "llama2-70b-stream":
+        run_stream(args)
+        return
     if args.case:
         run_case(args.case)
         return

@@ -19,7 +19,13 @@ HQQ_STOP_GROUP, HQQ_STOP_TENSOR, HQQ_STOP_NONE = 0, 1, 2
 
 EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_quantize", "hqq_dequantize",
             "hqq_get_status", "hqq_status_string", "hqq_quantize_noalloc", "hqq_quantize_scale8",
-            "hqq_dequantize_s8")
+            "hqq_dequantize_s8", "hqq_stream_device_bytes", "hqq_quantize_stream")
+
+
+class hqq_host_matrix(C.Structure):
+    """struct hqq_host_matrix of include/hqq.h (host pointers)."""
+    _fields_ = [("W", C.c_void_p), ("rows", C.c_int64), ("cols", C.c_int64), ("W_q_packed", C.c_void_p),
+                ("scale", C.c_void_p), ("zero", C.c_void_p), ("zero_meta", C.c_void_p)]
 HQQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -48,6 +54,11 @@ def _load():
     L.hqq_quantize_scale8.argtypes = [P, i64, i32, P, P, P]
     L.hqq_dequantize_s8.restype = i32
     L.hqq_dequantize_s8.argtypes = [P, P, P, i32, P, P, i64, i64, i32, i32, i32, i32, i32, P, P]
+    HM = C.POINTER(hqq_host_matrix)
+    L.hqq_stream_device_bytes.restype = sz
+    L.hqq_stream_device_bytes.argtypes = [HM, i32, i32, i32, i32, i32, i32]
+    L.hqq_quantize_stream.restype = i32
+    L.hqq_quantize_stream.argtypes = [HM, i32, i32, i32, i32, i32, f32, f32, f32, i32, i32, i32, P, sz, P]
     L.hqq_quantize_noalloc.restype = i32
     L.hqq_quantize_noalloc.argtypes = [P, i64, i64, i32, i32, i32, i32, f32, f32, f32, i32, i32, i32,
                                        P, P, P, P, P, P, P, P]
@@ -128,6 +139,16 @@ def hqq_dequantize_s8(W_q_packed, scale_q, scale_meta, scale_group, zero, zero_m
                                  _ptr(W_out), _stream(stream))
 
 
+def hqq_stream_device_bytes(mats, n, nbits, group_size, axis=1, stop_mode=HQQ_STOP_GROUP, zero_nbits=16):
+    return lib.hqq_stream_device_bytes(mats, n, nbits, group_size, axis, stop_mode, zero_nbits)
+
+
+def hqq_quantize_stream(mats, n, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode, zero_nbits,
+                        device_buffer, device_bytes, stream=None):
+    return lib.hqq_quantize_stream(mats, n, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
+                                   zero_nbits, _ptr(device_buffer), device_bytes, _stream(stream))
+
+
 def hqq_get_status(workspace, stream=None):
     return lib.hqq_get_status(_ptr(workspace), _stream(stream))
 
@@ -179,6 +200,43 @@ def quantize(W, nbits=4, group_size=64, axis=1, p=0.7, beta=1.0, kappa=1.01, ite
     if rc != HQQ_OK:
         raise HQQError(rc, "hqq_quantize")
     return out
+
+
+def host_outputs(rows, cols, nbits, group_size, axis=1, zero_nbits=16, pin=True):
+    """Pinned host output buffers for one matrix of quantize_stream()."""
+    G = hqq_num_groups(rows, cols, group_size, axis)
+    nb = hqq_packed_bytes(rows, cols, nbits, group_size, axis)
+    mk = (lambda t: t.pin_memory()) if pin else (lambda t: t)
+    return dict(packed=mk(torch.empty(nb, dtype=torch.uint8)), scale=mk(torch.empty(G, dtype=torch.float16)),
+                zero=mk(torch.empty(G, dtype=torch.float16 if zero_nbits == 16 else torch.uint8)),
+                zero_meta=mk(torch.empty(2, dtype=torch.float32)) if zero_nbits == 8 else None)
+
+
+def quantize_stream(Ws, outs, nbits=4, group_size=64, axis=1, p=0.7, beta=1.0, kappa=1.01, iters=20,
+                    stop_mode=HQQ_STOP_GROUP, zero_nbits=16, device_buffer=None, stream=None):
+    """Quantise host fp16/bf16 matrices (pinned for overlap) into host output
+    dicts (host_outputs()), streaming them through the GPU.  Returns the
+    device buffer used (reusable for another call with the same sizes)."""
+    if not Ws or len(Ws) != len(outs):
+        raise HQQError(HQQ_ERR_INVALID_ARG, "quantize_stream needs one output dict per matrix")
+    dt = Ws[0].dtype
+    if dt not in _DT or any(w.dtype != dt or w.is_cuda or w.dim() != 2 or not w.is_contiguous() for w in Ws):
+        raise HQQError(HQQ_ERR_INVALID_ARG, "quantize_stream expects contiguous 2-D host tensors of one dtype")
+    arr = (hqq_host_matrix * len(Ws))()
+    for a, w, o in zip(arr, Ws, outs):
+        a.W, a.rows, a.cols = w.data_ptr(), w.shape[0], w.shape[1]
+        a.W_q_packed, a.scale, a.zero = o["packed"].data_ptr(), o["scale"].data_ptr(), o["zero"].data_ptr()
+        a.zero_meta = o["zero_meta"].data_ptr() if o.get("zero_meta") is not None else None
+    need = hqq_stream_device_bytes(arr, len(Ws), nbits, group_size, axis, stop_mode, zero_nbits)
+    if need == 0:
+        raise HQQError(HQQ_ERR_INVALID_ARG, "hqq_stream_device_bytes")
+    if device_buffer is None or device_buffer.numel() < need:
+        device_buffer = torch.empty(need, dtype=torch.uint8, device="cuda")
+    rc = hqq_quantize_stream(arr, len(Ws), _DT[dt], nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
+                             zero_nbits, device_buffer, device_buffer.numel(), stream)
+    if rc != HQQ_OK:
+        raise HQQError(rc, "hqq_quantize_stream")
+    return device_buffer
 
 
 def quantize_scale8(q, scale_group=128, stream=None):

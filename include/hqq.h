@@ -176,6 +176,47 @@ int hqq_dequantize_s8(const void* W_q_packed, const void* scale_q, const void* s
                       const void* zero, const void* zero_meta, int64_t rows, int64_t cols, int nbits,
                       int group_size, int axis, int zero_nbits, int out_dtype, void* W_out, void* stream);
 
+/*
+ * Streaming a list of host-resident matrices through one GPU (a model
+ * quantised layer by layer; the pages run the solver on the GPU and move the
+ * data once, techreport.ngo, "Weight-only quantization without the
+ * calibration tax", section "Speed: from hours to minutes").
+ *
+ * hqq_host_matrix: one matrix and its outputs, all in HOST memory (pinned
+ * for the copies to overlap the solver):
+ *   W            [rows, cols] fp16/bf16 (dtype of the call), read.
+ *   W_q_packed   uint8[hqq_packed_bytes], scale fp16[G], zero fp16[G] or
+ *                uint8[G], zero_meta fp32[2] (zero_nbits == 8): written.
+ */
+typedef struct hqq_host_matrix {
+    const void* W;
+    int64_t rows, cols;
+    void* W_q_packed;
+    void* scale;
+    void* zero;
+    void* zero_meta;
+} hqq_host_matrix;
+
+/* Device bytes hqq_quantize_stream needs for this list: two slots, each
+ * sized for the largest matrix (W, outputs and solver workspace).  0 on
+ * invalid arguments. */
+size_t hqq_stream_device_bytes(const hqq_host_matrix* mats, int n, int nbits, int group_size, int axis,
+                               int stop_mode, int zero_nbits);
+
+/*
+ * hqq_quantize_stream -- hqq_quantize on each of the n matrices, with the
+ * copy of matrix i+1 to the GPU and of matrix i-1's outputs back to the host
+ * overlapping the solver on matrix i (two device slots; copies on two
+ * streams the call creates; the solver on `stream`).  Solver arguments as in
+ * hqq_quantize, the same for every matrix.  device_buffer: device memory of
+ * at least hqq_stream_device_bytes(...), 256-byte aligned, owned by the
+ * caller.  Blocks until every output is in host memory.  Returns HQQ_OK or
+ * the first error (HQQ_ERR_WORKSPACE if device_bytes is too small).
+ */
+int hqq_quantize_stream(const hqq_host_matrix* mats, int n, int dtype, int nbits, int group_size, int axis, float p,
+                        float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* device_buffer,
+                        size_t device_bytes, void* stream);
+
 /* Synchronise `stream` and return the device status word held in `workspace`
  * by the last hqq_quantize on it (HQQ_OK), or HQQ_ERR_CUDA if the
  * synchronisation or copy fails. */

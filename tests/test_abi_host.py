@@ -112,6 +112,25 @@ def test_scale8_entry_points_reject_on_host(hq):
     assert L.hqq_dequantize_s8(*args, 128, None, None, 0, 64, 4, 64, 1, 16, 0, None, None) == hq.HQQ_OK
 
 
+def test_stream_size_query_and_rejections(hq):
+    L = hq.lib
+    arr = (hq.hqq_host_matrix * 3)()
+    for a, (r, c) in zip(arr, [(4096, 1024), (256, 2048), (1024, 512)]):
+        a.rows, a.cols = r, c
+    one = hq.hqq_stream_device_bytes(arr, 1, 4, 64)
+    three = hq.hqq_stream_device_bytes(arr, 3, 4, 64)
+    assert one > 2 * 4096 * 1024 * 2 and three == one  # two slots sized by the largest matrix
+    arr[2].cols = 100  # not a multiple of the group size
+    assert hq.hqq_stream_device_bytes(arr, 3, 4, 64) == 0
+    assert hq.hqq_stream_device_bytes(arr, 0, 4, 64) == 0
+    assert L.hqq_quantize_stream(None, 1, 0, 4, 64, 1, 0.7, 1.0, 1.01, 20, 0, 16, None, 0, None) == \
+        hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_quantize_stream(arr, 0, 0, 4, 64, 1, 0.7, 1.0, 1.01, 20, 0, 16, None, 0, None) == hq.HQQ_OK
+    arr[2].cols = 512  # host buffers missing
+    assert L.hqq_quantize_stream(arr, 3, 0, 4, 64, 1, 0.7, 1.0, 1.01, 20, 0, 16, None, 0, None) == \
+        hq.HQQ_ERR_INVALID_ARG
+
+
 def test_status_strings(hq):
     for code in range(9):
         s = hq.hqq_status_string(code)
