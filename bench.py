@@ -62,14 +62,16 @@ def kernel_sources_sha():
     return h.hexdigest()
 
 
-def solver_launches(mode, iters=20):
+def solver_launches(mode, iters=20, g=64):
     """Kernel launches of one hqq_quantize call (fp16 zero), as the library
     schedules them: group stop runs passes of 2 and 3 evaluations and then the
-    rest (no stop: one pass); tensor stop runs chunks of iterations [0,2),
-    [2,6), [6,10), ... and one launch that writes the outputs."""
+    rest (no stop: one pass); tensor stop runs chunks of iterations [0,2) and
+    then C at a time (C = 8 for g >= 32, 4 for g <= 16), and one launch that
+    writes the outputs."""
     if mode == 1:
+        C = 4 if g <= 16 else 8
         last = iters - 1
-        return (0 if iters <= 0 else (0 if last < 2 else (last + 2) // 4) + 1) + 1
+        return (0 if iters <= 0 else (0 if last < 2 else (last - 2) // C + 1) + 1) + 1
     if mode == 2 or iters <= 2:
         return 1
     n, done = 0, 0
@@ -559,7 +561,8 @@ def main():
                          "unit": "Gop/s (MUFU lg2+ex2)", "frac": achieved / mufu_peak, "traffic": traffic,
                          "traffic_unit": "bytes per call", "algorithmic_bytes_per_call": bytes_dom,
                          "peak_basis": f"{SMS} SMs x {MUFU_PER_CLK_PER_SM} MUFU/clk x {sm_max:.0f} MHz",
-                         "timed_unit": f"one hqq_quantize call = {solver_launches(dom)} launches of {dom_name}",
+                         "timed_unit": f"one hqq_quantize call = {solver_launches(dom, 20, 64)} (g >= 32) or "
+                                       f"{solver_launches(dom, 20, 16)} (g <= 16) launches of {dom_name}",
                          "avg_launch_ms": avg_ms, "hbm_gbs": gb_dom, "hbm_frac": gb_dom / hbm_peak},
             "hbm": {"achieved_gbs_step": hbm_step, "peak_gbs": hbm_peak, "peak_kind": peak_kind,
                     "frac_step": hbm_step / hbm_peak,
@@ -567,7 +570,7 @@ def main():
                                    "frac": g_bytes / (g_ms / 1e3) / 1e9 / hbm_peak,
                                    "gweights_s": g_w / (g_ms / 1e3) / 1e9}},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": sum(solver_launches(mode) for *_, mode in calls) * args.steps,
+            "gpu_launches": sum(solver_launches(mode, 20, g) for _, _, _, _, g, mode in calls) * args.steps,
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, nth, desc, _, _ = oracle_sample_rate(0, budget_s=args.ref_budget)

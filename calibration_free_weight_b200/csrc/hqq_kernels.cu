@@ -43,7 +43,12 @@ using namespace dev;
 
 constexpr int kRegThreads = 256;
 constexpr int kRegWarps = kRegThreads / 32;
-constexpr int kChunkMax = 4;  // iterations per tensor-mode launch (after the first, which has 2)
+constexpr int kChunkMax = 8;  // most iterations of one tensor-mode launch (after the first, which has 2)
+
+// Iterations per tensor-mode launch: 8 for tiles of 32 elements per lane (the
+// per-tile reload and set-up amortised over more iterations), 4 for smaller
+// tiles (their iteration loop is unrolled and their partials held in registers).
+__host__ __device__ constexpr int chunk_len(int E) { return E <= 16 ? 4 : 8; }
 
 // Header words of the workspace (uint32 index); word 0 is the status word.
 constexpr int kWordTicket = 1;
@@ -105,14 +110,14 @@ __device__ __forceinline__ void merge_zero_range(const KParams& k, float zmin, f
 
 // ====================================================== register tiles ==
 
-// Chunk schedule of tensor mode: chunk 0 = iterations [0, 2), chunk c >= 1 =
-// [4c - 2, 4c + 2) (clipped to iters).
-__host__ __device__ inline int chunk_begin(int c, int iters) {
-    const int b = c == 0 ? 0 : 4 * c - 2;
+// Chunk schedule of tensor mode with chunk length C: chunk 0 = iterations
+// [0, 2), chunk c >= 1 = [C(c-1) + 2, Cc + 2) (clipped to iters).
+__host__ __device__ inline int chunk_begin(int c, int iters, int C) {
+    const int b = c == 0 ? 0 : C * (c - 1) + 2;
     return b < iters ? b : iters;
 }
-__host__ __device__ inline int chunk_of(int k) { return k < 2 ? 0 : (k + 2) / 4; }
-__host__ __device__ inline int num_chunks(int iters) { return iters <= 0 ? 0 : chunk_of(iters - 1) + 1; }
+__host__ __device__ inline int chunk_of(int k, int C) { return k < 2 ? 0 : (k - 2) / C + 1; }
+__host__ __device__ inline int num_chunks(int iters, int C) { return iters <= 0 ? 0 : chunk_of(iters - 1, C) + 1; }
 
 struct WarpTile {
     bool valid;  // this lane's group exists
@@ -433,9 +438,10 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 3 : 2) solve_tensor_ker
     float zmin = FLT_MAX, zmax = -FLT_MAX;
 
     const int iters = k.iters_eff;
-    const int nch = num_chunks(iters);
+    constexpr int C = chunk_len(E);
+    const int nch = num_chunks(iters, C);
     // Stop rule on the tensor errors of iterations [0, k0) (same decision in every CTA).
-    const int k0 = chunk_begin(chunk, iters);
+    const int k0 = chunk_begin(chunk, iters, C);
     int best_it = -1, stop_at = -1;
     {
         double best = INFINITY;
@@ -450,7 +456,7 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 3 : 2) solve_tensor_ker
             }
         }
     }
-    const int prev_begin = chunk > 0 ? chunk_begin(chunk - 1, iters) : 0;
+    const int prev_begin = chunk > 0 ? chunk_begin(chunk - 1, iters, C) : 0;
     bool finalize;
     if (stop_at >= 0) {
         if (stop_at < prev_begin) return;  // an earlier launch already wrote the outputs
@@ -465,7 +471,7 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 3 : 2) solve_tensor_ker
 
     if (finalize) {
         const int kb = best_it < 0 ? 0 : best_it;  // iters == 0: z* = z0
-        const int cb = chunk_of(kb), b0 = chunk_begin(cb, iters);
+        const int cb = chunk_of(kb, C), b0 = chunk_begin(cb, iters, C);
         const float* Zc = (cb % 3 == 0) ? Zs0 : (cb % 3 == 1 ? Zs1 : Zs2);
         for (int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp; t < ntiles; t += wstride) {
             const WarpTile w = warp_tile<AXIS>(k, t);
@@ -496,14 +502,14 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 3 : 2) solve_tensor_ker
     }
 
     // run iterations [k0, k1)
-    const int k1 = chunk_begin(chunk + 1, iters);
+    const int k1 = chunk_begin(chunk + 1, iters, C);
     const int nk = k1 - k0;
     float* const Zin = (chunk % 3 == 0) ? Zs0 : (chunk % 3 == 1 ? Zs1 : Zs2);
     float* const Zout = ((chunk + 1) % 3 == 0) ? Zs0 : ((chunk + 1) % 3 == 1 ? Zs1 : Zs2);
     // per-thread tensor error partials: registers for small tiles, else shared
-    double accr[kChunkMax] = {0.0, 0.0, 0.0, 0.0};
-    for (int q = 0; q < kChunkMax; ++q) sacc[q][threadIdx.x] = 0.0;
-    if (threadIdx.x < kChunkMax) sthr[threadIdx.x] = shrink_threshold(beta_at(k, k0 + threadIdx.x), k.p);
+    double accr[C] = {};
+    for (int q = 0; q < C; ++q) sacc[q][threadIdx.x] = 0.0;
+    if (threadIdx.x < C) sthr[threadIdx.x] = shrink_threshold(beta_at(k, k0 + threadIdx.x), k.p);
     __syncthreads();
     constexpr bool kPrefetch = AXIS == 1 && E <= 16;
     int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp;
@@ -554,7 +560,7 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 3 : 2) solve_tensor_ker
         // work in flight); large tiles: a loop, to keep the code cache-resident
         if constexpr (E <= 16) {
 #pragma unroll
-            for (int q = 0; q < kChunkMax; ++q)
+            for (int q = 0; q < C; ++q)
                 if (q < nk) tensor_iteration<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z0, k0 + q, sthr[q], spow, sws2,
                                                           inv_g, accr[q], z);
         } else {
@@ -568,7 +574,7 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 3 : 2) solve_tensor_ker
     // per-CTA partials (fixed order), then the last CTA sums them in a fixed order
     if constexpr (E <= 16) {
 #pragma unroll
-        for (int q = 0; q < kChunkMax; ++q) sacc[q][threadIdx.x] = accr[q];
+        for (int q = 0; q < C; ++q) sacc[q][threadIdx.x] = accr[q];
     }
     __syncthreads();
     for (int q = warp; q < nk; q += kRegWarps) {
@@ -1049,7 +1055,7 @@ cudaError_t launch_tensor(KParams& k, cudaStream_t stream) {
     int grid = 0;
     cudaError_t err = persistent_grid(kern, kRegThreads, 0, (tiles + kRegWarps - 1) / kRegWarps, &grid);
     if (err != cudaSuccess) return err;
-    const int nch = num_chunks(k.iters_eff);
+    const int nch = num_chunks(k.iters_eff, chunk_len(E));
     for (int c = 0; c <= nch; ++c) {  // nch chunks, then the launch that writes the outputs
         kern<<<grid, kRegThreads, 0, stream>>>(k, c);
         err = cudaGetLastError();
