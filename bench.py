@@ -66,12 +66,20 @@ def solver_launches(mode, iters=20, g=64):
     """Kernel launches of one hqq_quantize call (fp16 zero), as the library
     schedules them: group stop runs passes of 2 and 3 evaluations and then the
     rest (no stop: one pass); tensor stop runs chunks of iterations [0,2) and
-    then C at a time (C = 8 for g >= 32, 4 for g <= 16), and one launch that
-    writes the outputs."""
+    then C at a time (C = 8 for g >= 32, with a last chunk shorter than 4
+    merged into the one before; C = 4 for g <= 16), and one launch that writes
+    the outputs."""
     if mode == 1:
         C = 4 if g <= 16 else 8
-        last = iters - 1
-        return (0 if iters <= 0 else (0 if last < 2 else (last - 2) // C + 1) + 1) + 1
+        if iters <= 0:
+            n = 0
+        elif iters <= 2:
+            n = 1
+        else:
+            n = 1 + -(-(iters - 2) // C)
+            if C >= 8 and n > 2 and (iters - 2) - (n - 2) * C < C // 2:
+                n -= 1
+        return n + 1
     if mode == 2 or iters <= 2:
         return 1
     n, done = 0, 0

@@ -20,8 +20,9 @@ constexpr float kScaleCap = 2.0e4f;  // cap on s (and on the 8-bit zero quantise
 //   group / no stop, per slice of S entries (a warp-tile slot each; S = all
 //   entries unless the workspace is smaller):
 //                state float4[2][S], state_it int[S], survivor lists u32[2][S]
-//   tensor mode: tparts double[4][kMaxPartials], etot double[kMaxIters],
-//                s f32[G], z0 f32[G], sum w*s f64[G], chunk-start zeros f32[3][G]
+//   tensor mode: tparts double[12][kMaxPartials], etot double[kMaxIters],
+//                s f32[G], z0 f32[G], sum w*s f64[G], zeros of every iteration of
+//                two chunks f32[2][slots][G] (slots = 6 for g <= 16, 12 above)
 struct WorkspaceLayout {
     size_t header, zbest, state, state_it, list0, list1, tparts, etot, t_s, t_z0, t_sws, t_zs, total;
     int64_t slice;  // group mode: entries per slice

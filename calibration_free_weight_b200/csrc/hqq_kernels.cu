@@ -43,12 +43,14 @@ using namespace dev;
 
 constexpr int kRegThreads = 256;
 constexpr int kRegWarps = kRegThreads / 32;
-constexpr int kChunkMax = 8;  // most iterations of one tensor-mode launch (after the first, which has 2)
+constexpr int kChunkMax = 12;  // most iterations of one tensor-mode launch
 
 // Iterations per tensor-mode launch: 8 for tiles of 32 elements per lane (the
 // per-tile reload and set-up amortised over more iterations), 4 for smaller
 // tiles (their iteration loop is unrolled and their partials held in registers).
 __host__ __device__ constexpr int chunk_len(int E) { return E <= 16 ? 4 : 8; }
+// Longest chunk: with C >= 8 a short last chunk is merged into the one before.
+__host__ __device__ constexpr int chunk_max(int C) { return C >= 8 ? C + C / 2 - 1 : C; }
 
 // Header words of the workspace (uint32 index); word 0 is the status word.
 constexpr int kWordTicket = 1;
@@ -111,13 +113,28 @@ __device__ __forceinline__ void merge_zero_range(const KParams& k, float zmin, f
 // ====================================================== register tiles ==
 
 // Chunk schedule of tensor mode with chunk length C: chunk 0 = iterations
-// [0, 2), chunk c >= 1 = [C(c-1) + 2, Cc + 2) (clipped to iters).
+// [0, 2), chunk c >= 1 = [C(c-1) + 2, Cc + 2), clipped to iters; with C >= 8
+// a last chunk shorter than C/2 is merged into the one before it.
+__host__ __device__ inline int num_chunks(int iters, int C) {
+    if (iters <= 0) return 0;
+    if (iters <= 2) return 1;
+    int n = 1 + (iters - 2 + C - 1) / C;
+    const int last = (iters - 2) - (n - 2) * C;
+    if (C >= 8 && n > 2 && last < C / 2) --n;
+    return n;
+}
+// First iteration of chunk c (iters for c >= num_chunks: the end of the last chunk).
 __host__ __device__ inline int chunk_begin(int c, int iters, int C) {
-    const int b = c == 0 ? 0 : C * (c - 1) + 2;
+    if (c == 0) return 0;
+    if (c >= num_chunks(iters, C)) return iters;
+    const int b = C * (c - 1) + 2;
     return b < iters ? b : iters;
 }
-__host__ __device__ inline int chunk_of(int k, int C) { return k < 2 ? 0 : (k - 2) / C + 1; }
-__host__ __device__ inline int num_chunks(int iters, int C) { return iters <= 0 ? 0 : chunk_of(iters - 1, C) + 1; }
+__host__ __device__ inline int chunk_of(int k, int C, int iters) {
+    if (k < 2) return 0;
+    const int c = (k - 2) / C + 1, n = num_chunks(iters, C);
+    return c < n ? c : n - 1;
+}
 
 struct WarpTile {
     bool valid;  // this lane's group exists
@@ -231,7 +248,7 @@ __device__ __forceinline__ void store_lane_codes(const KParams& k, const WarpTil
 
 // min/max -> s, z0; fp32 w*s; fp64 sum of w*s (over the group's P lanes).
 // Also returns this lane's range of w*s (for the clamp-free test).
-template <int E>
+template <int E, bool SUM = true>
 __device__ __forceinline__ void init_lane(const KParams& k, const WarpTile& w, const float* x, float* ws, float* s_out,
                                           float* z0_out, double* sws_out, float* lmin_out, float* lmax_out) {
     float lmn = FLT_MAX, lmx = -FLT_MAX;
@@ -250,12 +267,12 @@ __device__ __forceinline__ void init_lane(const KParams& k, const WarpTile& w, c
 #pragma unroll
     for (int i = 0; i < E; ++i) {
         ws[i] = __fmul_rn(x[i], s);
-        two_sum_acc(hi, lo, ws[i]);
+        if (SUM) two_sum_acc(hi, lo, ws[i]);
     }
-    const double acc = w.valid ? static_cast<double>(hi) + static_cast<double>(lo) : 0.0;
+    const double acc = (SUM && w.valid) ? static_cast<double>(hi) + static_cast<double>(lo) : 0.0;
     *s_out = s;
     *z0_out = __fmul_rn(-mn, s);
-    *sws_out = seg_sum_d(acc, k.P);
+    *sws_out = SUM ? seg_sum_d(acc, k.P) : 0.0;
     *lmin_out = w.valid ? __fmul_rn(lmn, s) : 0.0f;
     *lmax_out = w.valid ? __fmul_rn(lmx, s) : 0.0f;
 }
@@ -377,32 +394,6 @@ __device__ __forceinline__ void load_raw1(const KParams& k, const WarpTile& w, u
     for (int t = 0; t < E / kPiece; ++t) raw[t] = w.valid ? __ldg(src + t) : make_uint4(0, 0, 0, 0);
 }
 
-// The cheap part of one iteration (no |r|^p): the next zero-point.
-template <int E>
-__device__ __forceinline__ float step_lane(const KParams& k, bool valid, const float* x, const float* ws, float s,
-                                           float z, float z0, float beta, float thr, double sws) {
-    float sq = 0.0f;
-    const bool sp = valid && shrink_possible(s, z, z0, thr, k.Lf);
-    if (valid) {
-#pragma unroll
-        for (int i = 0; i < E; ++i) sq += eval_elem(ws[i], z, k.Lf).q;
-    }
-    sq = seg_sum(sq, k.P);
-    double swe = 0.0;
-    if (__any_sync(kFull, sp)) {
-        if (sp) {
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                const ElemEval ee = eval_elem(ws[i], z, k.Lf);
-                const float we = shrink_elem(ee.r, s, k.p, beta);
-                swe += static_cast<double>(__fmul_rn(__fsub_rn(x[i], we), s));
-            }
-        }
-        swe = seg_sum_d(swe, k.P);
-    }
-    return sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, split_f2(sws), 1.0f / static_cast<float>(k.g));
-}
-
 // One tensor-mode iteration of a warp tile: evaluate z, add this group's
 // error term to its per-thread partial, step z.
 template <int DT, int AXIS, int E>
@@ -465,33 +456,31 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 3 : 2) solve_tensor_ker
         finalize = chunk >= nch;
         if (finalize) best_it = iters - 1;
     }
-    float* const Zs0 = k.t_zs;
-    float* const Zs1 = k.t_zs + G;
-    float* const Zs2 = k.t_zs + 2 * G;
+    // z of every iteration of a chunk, two slots by chunk parity:
+    // slot(c)[q][j] = z of iteration chunk_begin(c) + q, q = nk: the next chunk's start
+    constexpr int kSlots = chunk_max(C) + 1;
+    auto zslot = [&](int c, int q) { return k.t_zs + (static_cast<int64_t>(c & 1) * kSlots + q) * G; };
 
     if (finalize) {
+        // the kept iterate lies in the last chunk run or the one before it: both slots intact
         const int kb = best_it < 0 ? 0 : best_it;  // iters == 0: z* = z0
-        const int cb = chunk_of(kb, C), b0 = chunk_begin(cb, iters, C);
-        const float* Zc = (cb % 3 == 0) ? Zs0 : (cb % 3 == 1 ? Zs1 : Zs2);
+        const int cb = chunk_of(kb, C, iters), b0 = chunk_begin(cb, iters, C);
+        const float* Zc = zslot(cb, kb - b0);
         for (int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp; t < ntiles; t += wstride) {
             const WarpTile w = warp_tile<AXIS>(k, t);
             float x[E], ws[E];
             load_lane<DT, AXIS, E>(k, w, x);
             float s, z0, lmin, lmax;
             double sws;
-            init_lane<E>(k, w, x, ws, &s, &z0, &sws, &lmin, &lmax);
-            float z = (iters == 0 || cb == 0) ? z0 : (w.valid ? Zc[w.j] : 0.0f);
-            float beta = beta_at(k, b0);
-            for (int it = b0; it < kb; ++it) {
-                z = step_lane<E>(k, w.valid, x, ws, s, z, z0, beta, shrink_threshold(beta, k.p), sws);
-                beta = __fmul_rn(beta, k.kappa);
-            }
+            init_lane<E, false>(k, w, x, ws, &s, &z0, &sws, &lmin, &lmax);
+            const float z = iters == 0 ? z0 : (w.valid ? Zc[w.j] : 0.0f);
             store_lane_codes<AXIS, E>(k, w, ws, z);
             float err_mean = 0.0f;
             if (k.dbg_err) {
                 float err, sq;
                 bool sp;
                 double swe;
+                const float beta = beta_at(k, kb);
                 eval_lane<E>(k, w.valid, x, ws, s, z, z0, beta, shrink_threshold(beta, k.p), &err, &sq, &sp, &swe);
                 err_mean = err * pow_pos(s, -k.p) / static_cast<float>(k.g);
             }
@@ -504,12 +493,13 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 3 : 2) solve_tensor_ker
     // run iterations [k0, k1)
     const int k1 = chunk_begin(chunk + 1, iters, C);
     const int nk = k1 - k0;
-    float* const Zin = (chunk % 3 == 0) ? Zs0 : (chunk % 3 == 1 ? Zs1 : Zs2);
-    float* const Zout = ((chunk + 1) % 3 == 0) ? Zs0 : ((chunk + 1) % 3 == 1 ? Zs1 : Zs2);
+    const float* const Zin = chunk > 0 ? zslot(chunk - 1, k0 - prev_begin) : nullptr;
+    float* const Zcur = zslot(chunk, 0);
     // per-thread tensor error partials: registers for small tiles, else shared
-    double accr[C] = {};
-    for (int q = 0; q < C; ++q) sacc[q][threadIdx.x] = 0.0;
-    if (threadIdx.x < C) sthr[threadIdx.x] = shrink_threshold(beta_at(k, k0 + threadIdx.x), k.p);
+    constexpr int CM = chunk_max(C);
+    double accr[CM] = {};
+    for (int q = 0; q < CM; ++q) sacc[q][threadIdx.x] = 0.0;
+    if (threadIdx.x < CM) sthr[threadIdx.x] = shrink_threshold(beta_at(k, k0 + threadIdx.x), k.p);
     __syncthreads();
     constexpr bool kPrefetch = AXIS == 1 && E <= 16;
     int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp;
@@ -558,23 +548,29 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 3 : 2) solve_tensor_ker
         const F2 sws2 = split_f2(sws);
         // small tiles: unrolled over the chunk's iterations (more independent
         // work in flight); large tiles: a loop, to keep the code cache-resident
+        float* const zrow = (w.valid && w.part == 0) ? Zcur + w.j : nullptr;
         if constexpr (E <= 16) {
 #pragma unroll
-            for (int q = 0; q < C; ++q)
-                if (q < nk) tensor_iteration<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z0, k0 + q, sthr[q], spow, sws2,
-                                                          inv_g, accr[q], z);
+            for (int q = 0; q < CM; ++q)
+                if (q < nk) {
+                    if (zrow) zrow[q * G] = z;
+                    tensor_iteration<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z0, k0 + q, sthr[q], spow, sws2, inv_g,
+                                                  accr[q], z);
+                }
         } else {
 #pragma unroll 1
-            for (int q = 0; q < nk; ++q)
+            for (int q = 0; q < nk; ++q) {
+                if (zrow) zrow[q * G] = z;
                 tensor_iteration<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z0, k0 + q, sthr[q], spow, sws2, inv_g,
                                               sacc[q][threadIdx.x], z);
+            }
         }
-        if (w.valid && w.part == 0) Zout[w.j] = z;
+        if (zrow) zrow[nk * G] = z;  // the next chunk's first zero-point
     }
     // per-CTA partials (fixed order), then the last CTA sums them in a fixed order
     if constexpr (E <= 16) {
 #pragma unroll
-        for (int q = 0; q < C; ++q) sacc[q][threadIdx.x] = accr[q];
+        for (int q = 0; q < CM; ++q) sacc[q][threadIdx.x] = accr[q];
     }
     __syncthreads();
     for (int q = warp; q < nk; q += kRegWarps) {
@@ -1120,8 +1116,9 @@ WorkspaceLayout workspace_layout(int64_t rows, int64_t cols, int g, int axis, in
         off = up(off + 4 * Gs);
         l.t_sws = off;
         off = up(off + 8 * Gs);
-        l.t_zs = off;
-        off = up(off + 12 * Gs);
+        l.t_zs = off;  // z of every iteration of two chunks
+        const size_t slots = static_cast<size_t>(chunk_max(chunk_len(g < 32 ? g : 32)) + 1);
+        off = up(off + 4 * 2 * slots * Gs);
     } else {
         const int64_t n = group_entries(rows, cols, g, axis);
         l.slice = (slice > 0 && slice < n) ? slice : n;

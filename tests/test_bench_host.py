@@ -21,9 +21,10 @@ def test_solver_launches_follow_the_schedules():
     assert bench.solver_launches(1, 20, 16) == 7
     assert bench.solver_launches(1, 2, 16) == 2 and bench.solver_launches(1, 3, 16) == 3
     assert bench.solver_launches(1, 6, 16) == 3 and bench.solver_launches(1, 7, 16) == 4
-    # g >= 32: chunks [0,2) [2,10) [10,18) [18,20) + the writing launch
-    assert bench.solver_launches(1, 20, 64) == 5 and bench.solver_launches(1, 20, 32) == 5
-    assert bench.solver_launches(1, 10, 128) == 3 and bench.solver_launches(1, 11, 128) == 4
+    # g >= 32: chunks [0,2) [2,10) [10,20) (a last chunk shorter than 4 merged) + the writing launch
+    assert bench.solver_launches(1, 20, 64) == 4 and bench.solver_launches(1, 20, 32) == 4
+    assert bench.solver_launches(1, 10, 128) == 3 and bench.solver_launches(1, 11, 128) == 3
+    assert bench.solver_launches(1, 14, 128) == 4 and bench.solver_launches(1, 13, 128) == 3
 
 
 def test_clock_samples_outside_the_timed_region_are_dropped():

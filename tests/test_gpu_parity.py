@@ -81,7 +81,7 @@ def test_axis0(hq, rows, cols, g, nbits):
     _run(hq, W, _params(nbits, g, axis=0))
 
 
-@pytest.mark.parametrize("iters", [0, 1, 2, 5, 50])
+@pytest.mark.parametrize("iters", [0, 1, 2, 5, 11, 20, 50])  # 11, 20: tensor-stop tail chunks merged (g = 32)
 @pytest.mark.parametrize("stop", [0, 1, 2])
 def test_iteration_counts_and_modes(hq, iters, stop):
     W = synth.weight(300, 512, seed=iters * 3 + stop, dtype=torch.float16)
