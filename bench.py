@@ -49,8 +49,8 @@ KERNEL_SOURCES = ["calibration_free_weight_b200/csrc/hqq_kernels.cu", "calibrati
 # kernel per hqq_quantize call, averaged over the timed step's tensor-stop calls,
 # from the ncu launch list summarised in profiles/ (taken on the kernel sources
 # whose sha256 is recorded here; None until a capture exists).
-TRAFFIC = {"src_sha256": "14447d5a6c5caa9de19e382558cc4b7a6534e641ecfe016f71e486b942affa22",
-           "bytes_per_call": 568482492, "summary": "profiles/launches_llama2-7b-mlp-sweep.md"}
+TRAFFIC = {"src_sha256": "9a60d8380ce04766634a59571142b28e6f3b5be0eb786da03639d9a971725bb4",
+           "bytes_per_call": 410190592, "summary": "profiles/launches_llama2-7b-mlp-sweep.md"}
 
 
 def kernel_sources_sha():
