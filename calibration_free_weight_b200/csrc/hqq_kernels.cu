@@ -394,18 +394,39 @@ __device__ __forceinline__ void load_raw1(const KParams& k, const WarpTile& w, u
     for (int t = 0; t < E / kPiece; ++t) raw[t] = w.valid ? __ldg(src + t) : make_uint4(0, 0, 0, 0);
 }
 
-// One tensor-mode iteration of a warp tile: evaluate z, add this group's
-// error term to its per-thread partial, step z.
+// One tensor-mode iteration of a warp tile: evaluate z, add this lane's share
+// of the group's error to its per-thread partial (tensor mode needs only the
+// sum over all groups, so the error is not reduced over the group's lanes),
+// step z.  Fast path: one vote, one reduction (of the sum of W_q).
 template <int DT, int AXIS, int E>
 __device__ __forceinline__ void tensor_iteration(const KParams& k, const WarpTile& w, const float* ws, float lmin,
                                                  float lmax, float s, float z0, int it, float thr, float spow,
                                                  F2 sws2, float inv_g, double& acc, float& z) {
-    float err, sq;
-    bool sp;
-    double swe;
-    eval_lane_reload<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z, z0, it, thr, &err, &sq, &sp, &swe);
-    if (w.valid && w.part == 0) acc += static_cast<double>(err * spow);
-    z = sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, sws2, inv_g);
+    const bool sp = w.valid && shrink_possible(s, z, z0, thr, k.Lf);
+    float err = 0.0f, sq = 0.0f;
+    if (__all_sync(kFull, !w.valid || (!sp && clamp_free(lmin, lmax, z, k.Lf)))) {
+        if (w.valid) {
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const ElemEval e = eval_elem_nc(ws[i], z);
+                err += pow_pos(fabsf(e.r), k.p);
+                sq += e.q;
+            }
+        }
+        sq = seg_sum(sq, k.P);
+        z = zero_from_sums_f2(sq, sws2, inv_g);
+    } else {
+        double swe = 0.0;
+        if (w.valid) {
+            const float3 r = eval_lane_slow<DT, AXIS, E>(k, w, s, z, it, sp, &swe);
+            err = r.x;
+            sq = r.y;
+        }
+        sq = seg_sum(sq, k.P);
+        if (__any_sync(kFull, sp)) swe = seg_sum_d(swe, k.P);
+        z = sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, sws2, inv_g);
+    }
+    if (w.valid) acc += static_cast<double>(err * spow);
 }
 
 __device__ __forceinline__ double warp_sum_d(double x) {
@@ -415,8 +436,10 @@ __device__ __forceinline__ double warp_sum_d(double x) {
 
 // ============================================================ tensor stop ==
 
+// Resident CTAs per SM: 2 for 32 elements per lane (128 registers), 4 below
+// (64 registers; the few spilled bytes cost less than the lost occupancy).
 template <int DT, int AXIS, int E>
-__global__ void __launch_bounds__(kRegThreads, E <= 16 ? 3 : 2) solve_tensor_kernel(const KParams k, int chunk) {
+__global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2) solve_tensor_kernel(const KParams k, int chunk) {
     __shared__ float2 sred[kRegWarps];
     __shared__ double sacc[kChunkMax][kRegThreads];  // per-thread tensor error partials
     __shared__ float sthr[kChunkMax];                 // shrink threshold of each iteration of the chunk
@@ -637,9 +660,10 @@ __host__ __device__ inline int64_t num_entries(int64_t rows, int64_t cols, int64
     return (rows / g) * ((cols + gpw - 1) / gpw) * gpw;
 }
 
-// Three CTAs per SM (80 registers): occupancy beats the few spilled bytes.
+// Three CTAs per SM (80 registers) for 32 elements per lane, four (64) below:
+// occupancy beats the few spilled bytes.
 template <int DT, int AXIS, int E>
-__global__ void __launch_bounds__(kRegThreads, 3) solve_group_kernel(const KParams k, const PassArgs pa) {
+__global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 3) solve_group_kernel(const KParams k, const PassArgs pa) {
     __shared__ float2 sred[kRegWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gpw = 32 >> k.logP;
