@@ -398,10 +398,10 @@ __device__ __forceinline__ void load_raw1(const KParams& k, const WarpTile& w, u
 // of the group's error to its per-thread partial (tensor mode needs only the
 // sum over all groups, so the error is not reduced over the group's lanes),
 // step z.  Fast path: one vote, one reduction (of the sum of W_q).
-template <int DT, int AXIS, int E>
+template <int DT, int AXIS, int E, typename Acc>
 __device__ __forceinline__ void tensor_iteration(const KParams& k, const WarpTile& w, const float* ws, float lmin,
                                                  float lmax, float s, float z0, int it, float thr, float spow,
-                                                 F2 sws2, float inv_g, double& acc, float& z) {
+                                                 F2 sws2, float inv_g, Acc& acc, float& z) {
     const bool sp = w.valid && shrink_possible(s, z, z0, thr, k.Lf);
     float err = 0.0f, sq = 0.0f;
     if (__all_sync(kFull, !w.valid || (!sp && clamp_free(lmin, lmax, z, k.Lf)))) {
@@ -426,7 +426,7 @@ __device__ __forceinline__ void tensor_iteration(const KParams& k, const WarpTil
         if (__any_sync(kFull, sp)) swe = seg_sum_d(swe, k.P);
         z = sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, sws2, inv_g);
     }
-    if (w.valid) acc += static_cast<double>(err * spow);
+    if (w.valid) acc += static_cast<Acc>(err * spow);
 }
 
 __device__ __forceinline__ double warp_sum_d(double x) {
@@ -442,6 +442,7 @@ template <int DT, int AXIS, int E>
 __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2) solve_tensor_kernel(const KParams k, int chunk) {
     __shared__ float2 sred[kRegWarps];
     __shared__ double sacc[kChunkMax][kRegThreads];  // per-thread tensor error partials
+    __shared__ float saccf[E <= 16 ? 1 : kChunkMax][kRegThreads];  // fp32 running partials (32-element tiles)
     __shared__ float sthr[kChunkMax];                 // shrink threshold of each iteration of the chunk
     __shared__ int sflag;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -522,6 +523,8 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2) solve_tensor_ker
     constexpr int CM = chunk_max(C);
     double accr[CM] = {};
     for (int q = 0; q < CM; ++q) sacc[q][threadIdx.x] = 0.0;
+    if constexpr (E > 16)
+        for (int q = 0; q < CM; ++q) saccf[q][threadIdx.x] = 0.0f;
     if (threadIdx.x < CM) sthr[threadIdx.x] = shrink_threshold(beta_at(k, k0 + threadIdx.x), k.p);
     __syncthreads();
     constexpr bool kPrefetch = AXIS == 1 && E <= 16;
@@ -585,7 +588,7 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2) solve_tensor_ker
             for (int q = 0; q < nk; ++q) {
                 if (zrow) zrow[q * G] = z;
                 tensor_iteration<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z0, k0 + q, sthr[q], spow, sws2, inv_g,
-                                              sacc[q][threadIdx.x], z);
+                                              saccf[q][threadIdx.x], z);
             }
         }
         if (zrow) zrow[nk * G] = z;  // the next chunk's first zero-point
@@ -594,6 +597,9 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2) solve_tensor_ker
     if constexpr (E <= 16) {
 #pragma unroll
         for (int q = 0; q < CM; ++q) sacc[q][threadIdx.x] = accr[q];
+    } else {
+        // fp32 running sums of at most ~20 tiles per thread (relative error ~1e-6), then fp64
+        for (int q = 0; q < CM; ++q) sacc[q][threadIdx.x] = static_cast<double>(saccf[q][threadIdx.x]);
     }
     __syncthreads();
     for (int q = warp; q < nk; q += kRegWarps) {
