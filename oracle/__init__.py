@@ -41,6 +41,8 @@ def _bind(L):
     L.oracle_dequantize.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, i32, i32, P]
     L.oracle_dequantize_s8.restype = i32
     L.oracle_dequantize_s8.argtypes = [P, P, P, i32, P, P, i64, i64, i32, i32, i32, i32, i32, P]
+    L.oracle_gemv.restype = i32
+    L.oracle_gemv.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, i32, i32, P]
     L.oracle_quantize_scale8.restype = i32
     L.oracle_quantize_scale8.argtypes = [P, i64, i32, P, P]
     L.oracle_trace_group.restype = i32
@@ -140,6 +142,21 @@ def dequantize_s8(packed, scale_q, scale_meta, scale_group, zero, zero_meta, row
     if rc != 0:
         raise ValueError(f"oracle_dequantize_s8 failed with code {rc}")
     return out.view(np.float16) if out_dtype == F16 else out
+
+
+def gemv(packed, scale, zero, zero_meta, rows, cols, nbits, group_size, zero_nbits, x, x_dtype=F16, L=None):
+    """y[b] = W_r @ x[b] in fp64 with W_r = (W_q - zero) * scale in fp32 (axis 1).
+    x: [batch, cols] float16 array (x_dtype F16) or uint16 bf16 bits (BF16)."""
+    L = L or lib()
+    x = np.ascontiguousarray(x)
+    x2 = x.reshape(-1, cols)
+    y = np.zeros((x2.shape[0], rows), np.float64)
+    rc = L.oracle_gemv(_p(np.ascontiguousarray(packed)), _p(np.ascontiguousarray(scale)),
+                       _p(np.ascontiguousarray(zero)), _p(zero_meta), rows, cols, nbits, group_size, zero_nbits,
+                       _p(x2.view(np.uint16)), x_dtype, x2.shape[0], _p(y))
+    if rc != 0:
+        raise ValueError(f"oracle_gemv failed with code {rc}")
+    return y
 
 
 def shrink(x, p, beta, L=None):

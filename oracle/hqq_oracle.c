@@ -493,6 +493,37 @@ int oracle_dequantize_s8(const uint8_t *W_q_packed, const uint8_t *scale_q, cons
 }
 
 /*
+ * Fused consumer of the packed layout (the step after quantisation: the
+ * inference backends of "Weight-only quantization without the calibration
+ * tax" dequantise W_q and multiply): y[b][r] = sum_c W_r[r][c] * x[b][c] for a
+ * batch of activation vectors, with W_r = (W_q - zero) * scale rebuilt per
+ * element exactly as oracle_dequantize does before its final rounding (fp32),
+ * and every product and sum in fp64.  Groups along the input dimension
+ * (axis 1).  x: [batch][cols] fp16/bf16 bits; y: [batch][rows] fp64.
+ */
+int oracle_gemv(const uint8_t *W_q_packed, const uint16_t *scale, const void *zero, const float *zero_meta,
+                int64_t rows, int64_t cols, int nbits, int group_size, int zero_nbits, const uint16_t *x,
+                int x_dtype, int batch, double *y)
+{
+    if (!valid_args(rows, cols, x_dtype, nbits, group_size, 1, 0, zero_nbits) || batch < 1) return 1;
+    const int g = group_size;
+    for (int b = 0; b < batch; ++b)
+        for (int64_t r = 0; r < rows; ++r) y[b * rows + r] = 0.0;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t c = 0; c < cols; ++c) {
+            const int64_t j = (r * cols + c) / g;
+            const float q = (float)unpack_elem(W_q_packed, r, c, cols, nbits, 1);
+            float z;
+            if (zero_nbits == 16) z = from_f16(((const uint16_t *)zero)[j]);
+            else z = ((float)((const uint8_t *)zero)[j] - zero_meta[1]) * zero_meta[0];
+            const float w = (q - z) * from_f16(scale[j]);
+            for (int b = 0; b < batch; ++b) y[b * rows + r] += (double)w * (double)load_elem(x + b * cols, x_dtype, c);
+        }
+    }
+    return 0;
+}
+
+/*
  * The "_s*" variant of the Llama-2 table ("Benchmark results"/"Llama-2",
  * footnote of the table): the scale is also quantised to 8 bit, with a group
  * size of 128.  Reading R15: the quantity quantised is the stored fp16 scale

@@ -45,6 +45,11 @@ MUTANTS = [
      "const int64_t k1 = G;", 1),
     ("dequant-s8-first-run-meta", "const float *m = scale_meta + 2 * (j / scale_group);",
      "const float *m = scale_meta;", 1),
+    ("gemv-drops-zero", "const float w = (q - z) * from_f16(scale[j]);", "const float w = q * from_f16(scale[j]);",
+     1),
+    ("gemv-group-index", "const int64_t j = (r * cols + c) / g;", "const int64_t j = (r * cols + c) / (2 * g);", 1),
+    ("gemv-skips-last-column", "        for (int64_t c = 0; c < cols; ++c) {\n            const int64_t j = (r * cols + c) / g;",
+     "        for (int64_t c = 0; c < cols - 1; ++c) {\n            const int64_t j = (r * cols + c) / g;", 1),
     ("pack-msb-first", "unsigned v = level << off; /* at most 8 + 7 bits */",
      "unsigned v = (off + b <= 8 ? level << (8 - b - off) : level << off);", 1),
 ]

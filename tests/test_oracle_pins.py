@@ -542,3 +542,60 @@ def test_dequant_with_8bit_scale(orc):
     # close to the fp16-scale dequantisation: the scale moved by at most half a step of its run
     d16 = orc.dequantize(o["packed"], o["scale"], o["zero"], None, 64, 256, 4, 32).astype(np.float32)
     assert np.max(np.abs(d8.astype(np.float32) - d16)) < 0.02 * np.abs(d16).max()
+
+
+# ------------------------------------- fused dequantise + matrix-vector ---
+
+def _gemv_case():
+    d = {}
+    for line in open(os.path.join(GOLDEN, "gemv_hand_values.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        k, *v = line.split()
+        d[k] = v
+    return d
+
+
+def test_gemv_hand_values(orc):
+    d = _gemv_case()
+    rows, cols, nb, g = (int(d[k][0]) for k in ("rows", "cols", "nbits", "group"))
+    lv = np.array([int(v) for v in d["levels"]], np.uint8).reshape(rows, cols)
+    packed = np.zeros(rows * cols * nb // 8, np.uint8)
+    orc.lib().oracle_pack_levels(lv.ctypes.data, rows, cols, nb, 1, packed.ctypes.data)
+    sc = np.array([float(v) for v in d["scale"]], np.float16)
+    z = np.array([float(v) for v in d["zero"]], np.float16)
+    x = np.array([float(v) for v in d["x"]], np.float16)
+    y = orc.gemv(packed, sc, z, None, rows, cols, nb, g, 16, x)
+    assert y[0].tolist() == [float(v) for v in d["y"]]
+
+
+@pytest.mark.parametrize("nbits,g,zb", [(4, 64, 16), (2, 16, 8), (3, 32, 16), (8, 128, 8), (1, 8, 16)])
+def test_gemv_unit_vectors_give_dequantised_columns(orc, nbits, g, zb):
+    W = _synth_f16(24, 256, seed=nbits + g)
+    o = orc.quantize(W, nbits, g, 1, 0.7, 1.0, 1.01, 20, orc.STOP_GROUP, zb)
+    deq = orc.dequantize(o["packed"], o["scale"], o["zero"], o["zero_meta"], 24, 256, nbits, g, 1, zb)
+    cols = [0, 1, g - 1, g, 255]
+    X = np.zeros((len(cols), 256), np.float16)
+    for i, c in enumerate(cols):
+        X[i, c] = 1.0
+    Y = orc.gemv(o["packed"], o["scale"], o["zero"], o["zero_meta"], 24, 256, nbits, g, zb, X)
+    for i, c in enumerate(cols):
+        # the fp32 W_r of column c, rounded to fp16, is the dequantiser's output
+        assert np.array_equal(Y[i].astype(np.float32).astype(np.float16), deq[:, c])
+
+
+def test_gemv_is_linear_and_batched(orc):
+    W = _synth_f16(40, 512, seed=11)
+    o = orc.quantize(W, 4, 64, 1, 0.7, 1.0, 1.01, 20, orc.STOP_GROUP, 16)
+    r = np.random.default_rng(5)
+    # multiples of 1/8 below 2: sums exact in fp16, values exact in bf16
+    x1 = (r.integers(-8, 8, 512) / 8).astype(np.float16)
+    x2 = (r.integers(-8, 8, 512) / 8).astype(np.float16)
+    args = (o["packed"], o["scale"], o["zero"], None, 40, 512, 4, 64, 16)
+    y1, y2 = orc.gemv(*args, x1)[0], orc.gemv(*args, x2)[0]
+    y12 = orc.gemv(*args, (x1 + x2).astype(np.float16))[0]
+    assert np.allclose(y12, y1 + y2, rtol=1e-12, atol=1e-12)
+    Y = orc.gemv(*args, np.stack([x1, x2, x1]))
+    assert np.array_equal(Y[0], y1) and np.array_equal(Y[1], y2) and np.array_equal(Y[2], y1)
+    xb = (x1.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(orc.gemv(*args, xb, x_dtype=orc.BF16)[0], y1)
