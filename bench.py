@@ -396,10 +396,51 @@ def run_stream(args):
                       "data": "synthetic; one layer's buffers streamed for every layer", "results": res}))
 
 
+def run_gemv_case(spec):
+    """Time hqq_gemv (fused dequantisation + matrix-vector product) on one
+    quantised synthetic fp16 matrix: "gemv,rows,cols,nbits,g[,batch[,reps]]".
+    HBM-bound: codes b/8 B + fp16 scale and 8-bit zero 3/g B per weight, plus
+    the activations and outputs; L2 flushed before every call."""
+    from calibration_free_weight_b200 import hqq
+    v = [int(x) for x in spec.split(",")[1:]]
+    rows, cols, nbits, g = v[:4]
+    batch = v[4] if len(v) > 4 else 1
+    reps = v[5] if len(v) > 5 else 20
+    torch.cuda.set_device(0)
+    W = synth.weight(rows, cols, seed=7, dtype=torch.float16).cuda()
+    q = hqq.quantize(W, nbits, g, zero_nbits=8)
+    del W
+    x = (synth.weight(batch, cols, seed=8, dtype=torch.float32) * 50).to(torch.float16).cuda()
+    y = torch.empty(batch, rows, dtype=torch.float32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    hqq.gemv(q, x, rows, cols, nbits, g, zero_nbits=8, out=y)
+    ev = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        hqq.gemv(q, x, rows, cols, nbits, g, zero_nbits=8, out=y)
+        b.record()
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    ms = sorted(a.elapsed_time(b) for a, b in ev)
+    med = ms[len(ms) // 2]
+    G = rows * cols // g
+    nbytes = rows * cols * nbits // 8 + 2 * G + G + 8 + batch * cols * 2 + batch * rows * 4
+    hbm, _, kind = peaks()
+    print(json.dumps({"case": spec, "ms_median": med, "ms_min": ms[0], "bytes": nbytes,
+                      "gbs": nbytes / (med / 1e3) / 1e9, "hbm_peak_gbs": hbm, "peak_kind": kind,
+                      "frac": nbytes / (med / 1e3) / 1e9 / hbm,
+                      "gweights_s": rows * cols / (med / 1e3) / 1e9, "l2": "flushed before every call"}))
+
+
 def run_case(spec):
     """Time hqq_quantize on one synthetic bf16 matrix (used for kernel profiles)."""
     if spec.startswith("scale8"):
         run_scale8_case(spec)
+        return
+    if spec.startswith("gemv"):
+        run_gemv_case(spec)
         return
     from calibration_free_weight_b200 import hqq
     v = [int(x) for x in spec.split(",")]
@@ -434,7 +475,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
                     help="single-matrix timing instead of the sweep: stop_mode,rows,cols,nbits,group_size[,reps]; "
-                         "or scale8,G[,S[,reps]] for the 8-bit scale quantiser")
+                         "or scale8,G[,S[,reps]] for the 8-bit scale quantiser, "
+                         "or gemv,rows,cols,nbits,g[,batch[,reps]] for the fused dequantise + matrix-vector product")
     ap.add_argument("--workload", default="llama2-7b-mlp-sweep", choices=["llama2-7b-mlp-sweep", "llama2-70b-stream"])
     ap.add_argument("--layers", type=int, default=80, help="layers of the llama2-70b-stream workload")
     args = ap.parse_args()

@@ -72,6 +72,19 @@ struct DequantArgs {
     void* out;
 };
 
+struct GemvArgs {
+    const uint8_t* packed;
+    const uint16_t* scale;
+    const void* zero;
+    const float* zero_meta;
+    int64_t rows, cols;
+    int nbits, g, zero_nbits;
+    const void* x;  // [batch][cols] fp16/bf16
+    int x_dtype, batch;
+    float* y;       // [batch][rows]
+};
+cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t stream);
+
 // Launchers: return cudaSuccess or the launch error.
 cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream);
 cudaError_t launch_dequant(const DequantArgs& a, cudaStream_t stream);

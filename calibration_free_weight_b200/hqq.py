@@ -19,7 +19,7 @@ HQQ_STOP_GROUP, HQQ_STOP_TENSOR, HQQ_STOP_NONE = 0, 1, 2
 
 EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_quantize", "hqq_dequantize",
             "hqq_get_status", "hqq_status_string", "hqq_quantize_noalloc", "hqq_quantize_scale8",
-            "hqq_dequantize_s8", "hqq_stream_device_bytes", "hqq_quantize_stream")
+            "hqq_dequantize_s8", "hqq_stream_device_bytes", "hqq_quantize_stream", "hqq_gemv")
 
 
 class hqq_host_matrix(C.Structure):
@@ -54,6 +54,8 @@ def _load():
     L.hqq_quantize_scale8.argtypes = [P, i64, i32, P, P, P]
     L.hqq_dequantize_s8.restype = i32
     L.hqq_dequantize_s8.argtypes = [P, P, P, i32, P, P, i64, i64, i32, i32, i32, i32, i32, P, P]
+    L.hqq_gemv.restype = i32
+    L.hqq_gemv.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, i32, i32, P, P]
     HM = C.POINTER(hqq_host_matrix)
     L.hqq_stream_device_bytes.restype = sz
     L.hqq_stream_device_bytes.argtypes = [HM, i32, i32, i32, i32, i32, i32]
@@ -149,6 +151,12 @@ def hqq_quantize_stream(mats, n, dtype, nbits, group_size, axis, p, beta, kappa,
                                    zero_nbits, _ptr(device_buffer), device_bytes, _stream(stream))
 
 
+def hqq_gemv(W_q_packed, scale, zero, zero_meta, rows, cols, nbits, group_size, zero_nbits, x, x_dtype, batch, y,
+             stream=None):
+    return lib.hqq_gemv(_ptr(W_q_packed), _ptr(scale), _ptr(zero), _ptr(zero_meta), rows, cols, nbits, group_size,
+                        zero_nbits, _ptr(x), x_dtype, batch, _ptr(y), _stream(stream))
+
+
 def hqq_get_status(workspace, stream=None):
     return lib.hqq_get_status(_ptr(workspace), _stream(stream))
 
@@ -237,6 +245,20 @@ def quantize_stream(Ws, outs, nbits=4, group_size=64, axis=1, p=0.7, beta=1.0, k
     if rc != HQQ_OK:
         raise HQQError(rc, "hqq_quantize_stream")
     return device_buffer
+
+
+def gemv(q, x, rows, cols, nbits, group_size, zero_nbits=16, out=None, stream=None):
+    """y = dequant(W) @ x.T for the outputs of quantize() (axis 1) and a CUDA
+    [batch, cols] fp16/bf16 tensor x (batch <= 8); returns fp32 [batch, rows]."""
+    if x.dtype not in _DT or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
+        raise HQQError(HQQ_ERR_INVALID_ARG, "gemv expects a contiguous 2-D CUDA fp16/bf16 x")
+    if out is None:
+        out = torch.empty(x.shape[0], rows, dtype=torch.float32, device=x.device)
+    rc = hqq_gemv(q["packed"], q["scale"], q["zero"], q.get("zero_meta"), rows, cols, nbits, group_size, zero_nbits,
+                  x, _DT[x.dtype], x.shape[0], out, stream)
+    if rc != HQQ_OK:
+        raise HQQError(rc, "hqq_gemv")
+    return out
 
 
 def quantize_scale8(q, scale_group=128, stream=None):

@@ -217,6 +217,27 @@ int hqq_quantize_stream(const hqq_host_matrix* mats, int n, int dtype, int nbits
                         float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* device_buffer,
                         size_t device_bytes, void* stream);
 
+/*
+ * hqq_gemv -- fused dequantisation + matrix-vector product of the packed
+ * layout, the step an inference backend runs after quantisation (the
+ * dequantisation rule W_r = (W_q - z) * scale of techreport.ngo, "Weight-only
+ * quantization without the calibration tax", section "Outlier-aware
+ * optimization without gradients"):
+ *   y[b][r] = sum_c W_r[r][c] * x[b][c],  b < batch <= 8.
+ * Groups along the input dimension (axis 1 of an [out, in] = [rows, cols]
+ * weight).  W_q_packed, scale, zero, zero_meta as produced by hqq_quantize
+ * (fp16 scale; fp16 or 8-bit zero).  x: device [batch][cols] fp16/bf16
+ * (x_dtype), 16-byte aligned; y: device fp32 [batch][rows], 4-byte aligned.
+ * Arithmetic in fp32 (per 8-column piece s * (sum q x - z * sum x), the sum of
+ * each row in a fixed order): the same real number as the fp64 product of the
+ * dequantised weights, up to rounding.  Returns HQQ_OK, HQQ_ERR_DTYPE,
+ * HQQ_ERR_SHAPE, HQQ_ERR_INVALID_ARG (batch outside 1..8, bad pointer),
+ * HQQ_ERR_ALIGN or HQQ_ERR_CUDA.  Allocates nothing.
+ */
+int hqq_gemv(const void* W_q_packed, const void* scale, const void* zero, const void* zero_meta, int64_t rows,
+             int64_t cols, int nbits, int group_size, int zero_nbits, const void* x, int x_dtype, int batch, float* y,
+             void* stream);
+
 /* Synchronise `stream` and return the device status word held in `workspace`
  * by the last hqq_quantize on it (HQQ_OK), or HQQ_ERR_CUDA if the
  * synchronisation or copy fails. */
