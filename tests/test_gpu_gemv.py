@@ -4,10 +4,11 @@ against the oracle's fp64 product of the dequantised weights.
 Both sides run on the oracle's own quantisation outputs (uploaded to the GPU),
 so no oracle input comes from the CUDA path.  The GPU computes in fp32, per
 8-column piece s * (sum q x - z * sum x); the bound below is derived from that
-order of operations: with u = 2^-24 and n the longest chain of additions one
-thread performs (cols / 2048 pieces, the 8-term piece sums and the 8-level
-reduction), |y_gpu - y_ref| <= u * (n + 25) * sum_c s (|q| + |z|) |x|, where
-the extra terms cover the oracle's own fp32 rounding of each W_r.
+order of operations: with u = 2^-24 and n the longest chain of roundings one
+thread performs (at most cols / 1024 + 1 piece or chunk additions, an
+in-chunk chain of up to 32 fused multiply-adds, and up to 8 reduction
+levels), |y_gpu - y_ref| <= u * (n + 25) * sum_c s (|q| + |z|) |x|, where the
+extra terms cover the oracle's own fp32 rounding of each W_r.
 """
 import numpy as np
 import pytest
@@ -56,14 +57,15 @@ def _case(hq, rows, cols, nbits, g, zb, batch, xdt, seed):
     y = hq.gemv(dev, X.cuda(), rows, cols, nbits, g, zero_nbits=zb)
     torch.cuda.synchronize()
     got = y.cpu().numpy().astype(np.float64)
-    n = cols // 2048 + 1 + 8 + 8
+    n = cols // 1024 + 1 + 32 + 8
     bound = U * (n + 25) * _magnitude(o, rows, cols, nbits, g, zb, Xn).T
     err = np.abs(got - ref)
     assert np.all(err <= bound), f"max err/bound {np.max(err / np.maximum(bound, 1e-300))}"
     return float(np.max(err / np.maximum(bound, 1e-300)))
 
 
-@pytest.mark.parametrize("nbits,g", [(1, 16), (2, 16), (3, 64), (4, 64), (8, 128), (4, 8), (2, 1024)])
+@pytest.mark.parametrize("nbits,g", [(1, 16), (2, 16), (3, 64), (4, 64), (8, 128), (4, 8), (2, 1024), (3, 16),
+                                     (1, 32), (8, 16)])
 @pytest.mark.parametrize("zb", [16, 8])
 def test_gemv_settings(hq, nbits, g, zb):
     _case(hq, 99, 2048, nbits, g, zb, 1, oracle.F16, seed=nbits * 7 + g)
@@ -75,7 +77,8 @@ def test_gemv_batches_and_dtypes(hq, batch, xdt):
     _case(hq, 130, 1024, 4, 64, 16, batch, xdt, seed=batch)
 
 
-@pytest.mark.parametrize("rows,cols", [(1, 8 * 16), (3, 1024), (4096, 4096), (1024, 8192), (4096, 11008)])
+@pytest.mark.parametrize("rows,cols", [(1, 8 * 16), (3, 1024), (4096, 4096), (1024, 8192), (4096, 11008),
+                                       (40000, 1024)])  # the last: 4 rows per warp
 def test_gemv_shapes(hq, rows, cols):
     _case(hq, rows, cols, 4, 64 if cols % 64 == 0 else 16, 8, 1, oracle.F16, seed=rows + cols)
 
