@@ -18,7 +18,7 @@ constexpr float kScaleCap = 2.0e4f;  // cap on s (and on the 8-bit zero quantise
 //   header      256 B: status word, CTA ticket, kept-zero range, pass counts
 //   zbest       float[G]               kept zeros (8-bit zero path)
 //   group / no stop, per slice of S entries (a warp-tile slot each; S = all
-//   entries unless the workspace is smaller):
+//   entries, at most 2^31, unless the workspace is smaller):
 //                state float4[2][S], state_it int[S], survivor lists u32[2][S]
 //   tensor mode: tparts double[12][kMaxPartials], etot double[kMaxIters],
 //                s f32[G], z0 f32[G], sum w*s f64[G], zeros of every iteration of

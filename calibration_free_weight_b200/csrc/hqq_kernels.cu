@@ -1151,7 +1151,9 @@ WorkspaceLayout workspace_layout(int64_t rows, int64_t cols, int g, int axis, in
         off = up(off + 4 * 2 * slots * Gs);
     } else {
         const int64_t n = group_entries(rows, cols, g, axis);
+        constexpr int64_t kMaxSlice = int64_t{1} << 31;  // survivor lists hold 32-bit entry offsets
         l.slice = (slice > 0 && slice < n) ? slice : n;
+        if (l.slice > kMaxSlice) l.slice = kMaxSlice;
         const size_t S = static_cast<size_t>(l.slice > 0 ? l.slice : 0);
         l.state = off;
         off = up(off + 32 * S);
