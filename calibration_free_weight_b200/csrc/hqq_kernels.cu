@@ -494,10 +494,19 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2) solve_tensor_ker
             const WarpTile w = warp_tile<AXIS>(k, t);
             float x[E], ws[E];
             load_lane<DT, AXIS, E>(k, w, x);
-            float s, z0, lmin, lmax;
-            double sws;
-            init_lane<E, false>(k, w, x, ws, &s, &z0, &sws, &lmin, &lmax);
-            const float z = iters == 0 ? z0 : (w.valid ? Zc[w.j] : 0.0f);
+            float s, z0, z;
+            if (nch > 0) {  // s, z0 and the kept zero-point were stored by the chunks
+                s = w.valid ? k.t_s[w.j] : 1.0f;
+                z0 = w.valid ? k.t_z0[w.j] : 0.0f;
+                z = w.valid ? Zc[w.j] : 0.0f;
+#pragma unroll
+                for (int i = 0; i < E; ++i) ws[i] = __fmul_rn(x[i], s);
+            } else {  // iters == 0: z* = z0 from min/max
+                float lmin, lmax;
+                double sws;
+                init_lane<E, false>(k, w, x, ws, &s, &z0, &sws, &lmin, &lmax);
+                z = z0;
+            }
             store_lane_codes<AXIS, E>(k, w, ws, z);
             float err_mean = 0.0f;
             if (k.dbg_err) {
