@@ -439,7 +439,8 @@ __device__ __forceinline__ double warp_sum_d(double x) {
 // Resident CTAs per SM: 2 for 32 elements per lane (128 registers), 4 below
 // (64 registers; the few spilled bytes cost less than the lost occupancy).
 template <int DT, int AXIS, int E>
-__global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2) solve_tensor_kernel(const KParams k, int chunk) {
+__global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2)
+    solve_tensor_kernel(const KParams k, int chunk, int write_outputs) {
     __shared__ float2 sred[kRegWarps];
     __shared__ double sacc[kChunkMax][kRegThreads];  // per-thread tensor error partials
     __shared__ float saccf[E <= 16 ? 1 : kChunkMax][kRegThreads];  // fp32 running partials (32-element tiles)
@@ -474,7 +475,7 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2) solve_tensor_ker
     const int prev_begin = chunk > 0 ? chunk_begin(chunk - 1, iters, C) : 0;
     bool finalize;
     if (stop_at >= 0) {
-        if (stop_at < prev_begin) return;  // an earlier launch already wrote the outputs
+        if (stop_at < prev_begin || !write_outputs) return;  // outputs written elsewhere
         finalize = true;
     } else {
         finalize = chunk >= nch;
@@ -634,6 +635,85 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2) solve_tensor_ker
         if (lane == 0) k.etot[k0 + q] = v / static_cast<double>(k.n);
     }
     if (threadIdx.x == 0) k.counters[kWordTicket] = 0;
+}
+
+// The outputs of a tensor-stop call, axis 1, no debug outputs: a streaming
+// pass over W after the last chunk, one 8-element piece per thread: the kept
+// iterate (first rise of the stored tensor errors), its stored zero-point and
+// the stored scale give the codes; the first piece of a group writes the
+// group's scale and zero.  Far fewer registers than the chunk kernel, so far
+// more loads in flight.
+constexpr int kOutPieces = 4;  // pieces per thread of tensor_output_kernel, loads issued together
+
+template <int DT, int NBITS>
+__global__ void __launch_bounds__(256) tensor_output_kernel(const KParams k) {
+    __shared__ float2 sred[8];
+    __shared__ double serr[kMaxIters];
+    __shared__ int skb;
+    constexpr float Lf = static_cast<float>((1 << NBITS) - 1);
+    const int iters = k.iters_eff;
+    // kept iterate: the tensor errors loaded in parallel, scanned by one thread
+    for (int it = threadIdx.x; it < iters; it += 256) serr[it] = __ldcg(k.etot + it);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int kb = iters - 1;
+        double best = INFINITY;
+        for (int it = 0; it < iters; ++it) {
+            if (serr[it] < best) {
+                best = serr[it];
+                kb = it;
+            } else {
+                break;
+            }
+        }
+        skb = kb;
+    }
+    __syncthreads();
+    const int kb = skb;
+    const int C = chunk_len(k.E);
+    const int cb = chunk_of(kb, C, iters), b0 = chunk_begin(cb, iters, C);
+    const int64_t slots = chunk_max(C) + 1;
+    const float* Zc = k.t_zs + ((cb & 1) * slots + (kb - b0)) * k.G;
+    int log_ppg = 0;
+    while ((kPiece << log_ppg) < k.g) ++log_ppg;  // pieces per group: g / 8, a power of two
+    float zmin = FLT_MAX, zmax = -FLT_MAX;
+    const int64_t npieces = k.n / kPiece;
+    const int64_t pc0 = static_cast<int64_t>(blockIdx.x) * 256 * kOutPieces + threadIdx.x;
+    uint4 raw[kOutPieces];
+    float sv[kOutPieces], zv[kOutPieces];
+#pragma unroll
+    for (int u = 0; u < kOutPieces; ++u) {
+        const int64_t pc = pc0 + u * 256;
+        if (pc < npieces) {
+            const int64_t j = pc >> log_ppg;
+            raw[u] = __ldg(reinterpret_cast<const uint4*>(k.W) + pc);
+            sv[u] = __ldg(k.t_s + j);
+            zv[u] = __ldcg(Zc + j);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kOutPieces; ++u) {
+        const int64_t pc = pc0 + u * 256;
+        if (pc >= npieces) break;
+        float x[kPiece];
+        unpack8<DT>(raw[u], x);
+        uint32_t code[kPiece];
+#pragma unroll
+        for (int i = 0; i < kPiece; ++i) round_clamp(__fadd_rn(__fmul_rn(x[i], sv[u]), zv[u]), Lf, &code[i]);
+        const uint64_t v = pack8_t<NBITS>(code);
+        uint8_t* dst = k.packed + pc * NBITS;
+        if (NBITS == 8) *reinterpret_cast<uint64_t*>(dst) = v;
+        else if (NBITS == 4) *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(v);
+        else if (NBITS == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(v);
+        else if (NBITS == 1) *dst = static_cast<uint8_t>(v);
+        else {
+            dst[0] = static_cast<uint8_t>(v);
+            dst[1] = static_cast<uint8_t>(v >> 8);
+            dst[2] = static_cast<uint8_t>(v >> 16);
+        }
+        if ((pc & ((int64_t{1} << log_ppg) - 1)) == 0) store_group(k, pc >> log_ppg, sv[u], zv[u], kb, 0.0f, &zmin, &zmax);
+    }
+    if (k.zero_nbits == 8) merge_zero_range<8>(k, zmin, zmax, sred);
 }
 
 // ============================================================= group stop ==
@@ -1091,12 +1171,27 @@ cudaError_t launch_tensor(KParams& k, cudaStream_t stream) {
     cudaError_t err = persistent_grid(kern, kRegThreads, 0, (tiles + kRegWarps - 1) / kRegWarps, &grid);
     if (err != cudaSuccess) return err;
     const int nch = num_chunks(k.iters_eff, chunk_len(E));
-    for (int c = 0; c <= nch; ++c) {  // nch chunks, then the launch that writes the outputs
-        kern<<<grid, kRegThreads, 0, stream>>>(k, c);
+    // axis 1 without debug outputs: the outputs come from a streaming kernel
+    const bool stream_out = AXIS == 1 && nch > 0 && !k.dbg_iter && !k.dbg_err && !k.dbg_zero;
+    for (int c = 0; c < nch; ++c) {
+        kern<<<grid, kRegThreads, 0, stream>>>(k, c, stream_out ? 0 : 1);
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }
-    return cudaSuccess;
+    if (!stream_out) {  // the chunk kernel's own output launch
+        kern<<<grid, kRegThreads, 0, stream>>>(k, nch, 1);
+        return cudaGetLastError();
+    }
+    const int64_t pieces = k.n / kPiece;
+    const unsigned og = static_cast<unsigned>((pieces + 256 * kOutPieces - 1) / (256 * kOutPieces));
+    switch (k.nbits) {
+        case 1: tensor_output_kernel<DT, 1><<<og, 256, 0, stream>>>(k); break;
+        case 2: tensor_output_kernel<DT, 2><<<og, 256, 0, stream>>>(k); break;
+        case 3: tensor_output_kernel<DT, 3><<<og, 256, 0, stream>>>(k); break;
+        case 4: tensor_output_kernel<DT, 4><<<og, 256, 0, stream>>>(k); break;
+        default: tensor_output_kernel<DT, 8><<<og, 256, 0, stream>>>(k); break;
+    }
+    return cudaGetLastError();
 }
 
 template <int DT, int AXIS, int E>

@@ -215,3 +215,21 @@ def test_llama_mlp_tensor_mode(hq, nbits, g):
     W = synth.weight(11008, 4096, seed=4, dtype=torch.bfloat16)
     rep, gpu, orc = _run(hq, W, _params(nbits, g, stop=1), check_recon=(nbits == 2))
     assert np.all(gpu["best_iter"] == orc["best_iter"][0])
+
+
+@pytest.mark.parametrize("nbits,g,zb,iters", [(4, 64, 16, 20), (8, 128, 8, 20), (2, 16, 8, 20), (1, 16, 16, 20),
+                                              (3, 64, 16, 11), (4, 32, 8, 1), (2, 64, 16, 2)])
+def test_tensor_outputs_without_debug(hq, nbits, g, zb, iters):
+    """Tensor stop without debug outputs writes its outputs in a separate
+    streaming pass (axis 1); they must equal the debug run's, which the other
+    tests check against the oracle."""
+    W = synth.weight(1000, 1024, seed=nbits * 31 + g, dtype=torch.bfloat16).cuda()
+    ref = hq.quantize(W, nbits, g, iters=iters, stop_mode=1, zero_nbits=zb, debug=True)
+    got = hq.quantize(W, nbits, g, iters=iters, stop_mode=1, zero_nbits=zb)
+    torch.cuda.synchronize()
+    for k in ("packed", "scale", "zero", "zero_meta"):
+        if ref[k] is None:
+            continue
+        assert torch.equal(ref[k].view(torch.uint8), got[k].view(torch.uint8)), k
+    # and the debug run against the oracle
+    _run(hq, W.cpu(), _params(nbits, g, stop=1, zb=zb, iters=iters), check_recon=False)
