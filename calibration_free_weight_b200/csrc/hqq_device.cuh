@@ -90,20 +90,6 @@ __device__ __forceinline__ bool clamp_free(float wsmin, float wsmax, float z, fl
     return __fadd_rn(wsmin, z) >= -0.5f && __fadd_rn(wsmax, z) < Lf + 0.5f;
 }
 
-// Compensated (TwoSum) fp32 accumulation: every rounding error of the running
-// sum is formed exactly and collected in lo, so hi + lo carries the sum of the
-// fp32 terms to ~n^2 * 2^-48 of it (Kahan's compensation is not enough here: it
-// leaves an error of order 2^-23 of the sum of magnitudes, which can move z by
-// an ulp, flip a code and change the whole trajectory).  No per-term
-// conversion to fp64 (an XU-pipe op on this GPU) is needed.
-__device__ __forceinline__ void two_sum_acc(float& hi, float& lo, float x) {
-    const float s = __fadd_rn(hi, x);
-    const float bp = __fsub_rn(s, hi);
-    const float e = __fadd_rn(__fsub_rn(hi, __fsub_rn(s, bp)), __fsub_rn(x, bp));
-    hi = s;
-    lo = __fadd_rn(lo, e);
-}
-
 // Proximal step of the lp term for one element: d = r/s, W_e = shrink(d).
 __device__ __forceinline__ float shrink_elem(float r, float s, float p, float beta) {
     const float d = __fdiv_rn(r, s);

@@ -263,13 +263,14 @@ __device__ __forceinline__ void init_lane(const KParams& k, const WarpTile& w, c
     const float mx = seg_max(lmx, k.P);
     float s = kScaleCap;
     if (mx > mn) s = fminf(__fdiv_rn(k.Lf, __fsub_rn(mx, mn)), kScaleCap);
-    float hi = 0.0f, lo = 0.0f;
+    // the sum of fp32 w*s in fp64, as the oracle accumulates it (up to the order)
+    double accd = 0.0;
 #pragma unroll
     for (int i = 0; i < E; ++i) {
         ws[i] = __fmul_rn(x[i], s);
-        if (SUM) two_sum_acc(hi, lo, ws[i]);
+        if (SUM) accd += static_cast<double>(ws[i]);
     }
-    const double acc = (SUM && w.valid) ? static_cast<double>(hi) + static_cast<double>(lo) : 0.0;
+    const double acc = (SUM && w.valid) ? accd : 0.0;
     *s_out = s;
     *z0_out = __fmul_rn(-mn, s);
     *sws_out = SUM ? seg_sum_d(acc, k.P) : 0.0;
