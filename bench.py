@@ -343,6 +343,12 @@ LLAMA70B = [("q", 8192, 8192), ("k", 1024, 8192), ("v", 1024, 8192), ("o", 8192,
             ("gate", 28672, 8192), ("up", 28672, 8192), ("down", 8192, 28672)]
 
 
+def rank_layers(layers, world, rank):
+    """Layers a rank streams in the multi-GPU run: every world-th layer from
+    its own index (whole layers per rank, no exchange between ranks)."""
+    return list(range(rank, layers, world))
+
+
 def run_stream(args):
     """Llama-2-70B-shaped model (80 layers x q, k, v, o, gate, up, down; fp16)
     streamed layer by layer from pinned host memory through hqq_quantize_stream
@@ -351,20 +357,26 @@ def run_stream(args):
     those buffers: each layer's copy-in, solve and copy-out is real, only the
     values repeat (137 GB of distinct synthetic weights would take minutes to
     generate).  Reports the end-to-end wall time of the blocking call and, for
-    the same matrices resident on the device, the solver's throughput."""
+    the same matrices resident on the device, the solver's throughput.
+    Under torchrun each rank streams its share of the layers (rank_layers);
+    the end-to-end time is the max over ranks of the blocking call's wall time
+    between barriers."""
     from calibration_free_weight_b200 import hqq
-    torch.cuda.set_device(0)
+    world, rank, local = dist_setup()
     layers = args.layers
+    mine = len(rank_layers(layers, world, rank))
     Ws = [synth.weight(r, c, seed=synth.seed_for(0, n), dtype=torch.float16).pin_memory() for n, r, c in LLAMA70B]
     w_layer = sum(r * c for _, r, c in LLAMA70B)
     res = []
     for nbits, g in ((2, 16), (4, 128)):
         outs = [hqq.host_outputs(r, c, nbits, g, zero_nbits=8) for _, r, c in LLAMA70B]
         buf = hqq.quantize_stream(Ws, outs, nbits, g, zero_nbits=8)  # warm-up: one layer
-        torch.cuda.synchronize()
+        barrier(world)
         t0 = time.perf_counter()
-        hqq.quantize_stream(Ws * layers, outs * layers, nbits, g, zero_nbits=8, device_buffer=buf)
-        wall = time.perf_counter() - t0
+        if mine:
+            hqq.quantize_stream(Ws * mine, outs * mine, nbits, g, zero_nbits=8, device_buffer=buf)
+        wall = max_over_ranks(time.perf_counter() - t0, world)
+        barrier(world)
         del buf
         # the same matrices resident on the device: solver time per layer (CUDA events)
         dev = [w.cuda() for w in Ws]
@@ -391,9 +403,13 @@ def run_stream(args):
                                         "solve_s_all_layers": layer_ms / 1e3 * layers}})
         del dev, q
         torch.cuda.empty_cache()
-    print(json.dumps({"workload": "llama2-70b-stream", "layers": layers, "weights": w_layer * layers,
-                      "dtype_in": "fp16", "zero": "8-bit", "stop_mode": "group", "host": "pinned",
-                      "data": "synthetic; one layer's buffers streamed for every layer", "results": res}))
+    if rank == 0:
+        print(json.dumps({"workload": "llama2-70b-stream", "layers": layers, "weights": w_layer * layers,
+                          "n_gpus": world, "scaling": "layers split across ranks",
+                          "dtype_in": "fp16", "zero": "8-bit", "stop_mode": "group", "host": "pinned",
+                          "data": "synthetic; one layer's buffers streamed for every layer", "results": res}))
+    if world > 1:
+        torch.distributed.destroy_process_group()
 
 
 def run_gemv_case(spec):

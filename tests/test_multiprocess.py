@@ -70,6 +70,16 @@ def test_two_gloo_ranks(tmp_path):
     assert res[1]["ref_out"] == ""                 # rank 1 runs no reference work
 
 
+def test_stream_layers_split_across_ranks():
+    sys.path.insert(0, ROOT)
+    import bench
+    for layers, world in ((80, 1), (80, 8), (80, 3), (5, 8)):
+        parts = [bench.rank_layers(layers, world, r) for r in range(world)]
+        flat = sorted(x for p in parts for x in p)
+        assert flat == list(range(layers))  # every layer once
+        assert max(map(len, parts)) - min(map(len, parts)) <= 1  # balanced
+
+
 def test_throughput_is_whole_job():
     sys.path.insert(0, ROOT)
     import bench
