@@ -46,11 +46,12 @@ SMS = 148
 MUFU_PER_CLK_PER_SM = 16
 KERNEL_SOURCES = ["calibration_free_weight_b200/csrc/hqq_kernels.cu", "calibration_free_weight_b200/csrc/hqq_device.cuh"]
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
-# kernel per hqq_quantize call, averaged over the timed step's tensor-stop calls,
+# kernel family per hqq_quantize call (its chunk launches and its output
+# launch), averaged over the timed step's tensor-stop calls,
 # from the ncu launch list summarised in profiles/ (taken on the kernel sources
 # whose sha256 is recorded here; None until a capture exists).
-TRAFFIC = {"src_sha256": "9a60d8380ce04766634a59571142b28e6f3b5be0eb786da03639d9a971725bb4",
-           "bytes_per_call": 410190592, "summary": "profiles/launches_llama2-7b-mlp-sweep.md"}
+TRAFFIC = {"src_sha256": "4e5d07e06aac7ae4c4a36c786c2548ebaf216fd611d307b8ccc4496b9a2dae9b",
+           "bytes_per_call": 420784265, "summary": "profiles/launches_llama2-7b-mlp-sweep.md"}
 
 
 def kernel_sources_sha():
@@ -627,8 +628,9 @@ def main():
                          "unit": "Gop/s (MUFU lg2+ex2)", "frac": achieved / mufu_peak, "traffic": traffic,
                          "traffic_unit": "bytes per call", "algorithmic_bytes_per_call": bytes_dom,
                          "peak_basis": f"{SMS} SMs x {MUFU_PER_CLK_PER_SM} MUFU/clk x {sm_max:.0f} MHz",
-                         "timed_unit": f"one hqq_quantize call = {solver_launches(dom, 20, 64)} (g >= 32) or "
-                                       f"{solver_launches(dom, 20, 16)} (g <= 16) launches of {dom_name}",
+                         "timed_unit": f"one hqq_quantize call = {solver_launches(dom, 20, 64) - 1} (g >= 32) or "
+                                       f"{solver_launches(dom, 20, 16) - 1} (g <= 16) chunk launches of {dom_name} "
+                                       f"and one tensor_output_kernel",
                          "avg_launch_ms": avg_ms, "hbm_gbs": gb_dom, "hbm_frac": gb_dom / hbm_peak},
             "hbm": {"achieved_gbs_step": hbm_step, "peak_gbs": hbm_peak, "peak_kind": peak_kind,
                     "frac_step": hbm_step / hbm_peak,
