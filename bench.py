@@ -642,7 +642,11 @@ def main():
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, nth, desc, _, _ = oracle_sample_rate(0, budget_s=args.ref_budget)
-        line["cpu_baseline"] = {"value": rate / 1e9, "unit": UNIT, "cores": nth, "kind": "oracle", "sample": desc}
+        # the same sample on one host thread
+        n1, t1 = oracle_pass(make_inputs(0), 16, 1)
+        line["cpu_baseline"] = {"value": rate / 1e9, "unit": UNIT, "cores": nth, "kind": "oracle", "sample": desc,
+                                "single_thread": {"value": n1 / t1 / 1e9, "cores": 1,
+                                                  "sample": oracle_desc(16, n1)}}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

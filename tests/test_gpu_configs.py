@@ -101,3 +101,11 @@ def test_llama2_13b_mixed_tensor_stop(hq, rows, cols, nbits, g):
 def test_llama2_70b_shapes_zero8(hq, rows, cols, nbits, g):
     W = synth.weight(rows, cols, seed=rows // 1024 + cols // 1024, dtype=torch.float16)
     _sampled(hq, W, _params(nbits, g, zb=8))
+
+
+def test_llama2_7b_every_layer_first_matrix(hq):
+    """Full-model configuration, sampled: the first matrix (q) of every one of
+    the 32 layers, each with that layer's seed, 1000 random groups per layer."""
+    for layer in range(32):
+        W = synth.weight(4096, 4096, seed=synth.seed_for(layer, "q"), dtype=torch.float16)
+        _sampled(hq, W, _params(4, 128, zb=8), n=1000, seed=layer)
