@@ -554,10 +554,12 @@ def main():
     with Clocks(local) as clk:
         barrier(world)
         clk.mark_start()
+        torch.cuda.nvtx.range_push("timed steps")
         ev0.record(stream)
         for _ in range(args.steps):
             one_step(rec)
         ev1.record(stream)
+        torch.cuda.nvtx.range_pop()
         barrier(world)
         clk.mark_end()
     for o in outs.values():
