@@ -210,9 +210,10 @@ def oracle_calibrate(ins, pass_s, nth):
         rows *= 4
 
 
-def oracle_desc(rows, n):
+def oracle_desc(rows, n, nthreads=0):
+    par = "one thread" if nthreads == 1 else "OpenMP over groups"
     return (f"first {rows} rows of gate/up (and the same element count of down) at all 10 settings/modes, "
-            f"{n / 1e6:.2f} M weights per pass, bf16, OpenMP over groups")
+            f"{n / 1e6:.2f} M weights per pass, bf16, {par}")
 
 
 def oracle_sample_rate(layer, budget_s=12.0, nthreads=0):
@@ -648,7 +649,7 @@ def main():
         n1, t1 = oracle_pass(make_inputs(0), 16, 1)
         line["cpu_baseline"] = {"value": rate / 1e9, "unit": UNIT, "cores": nth, "kind": "oracle", "sample": desc,
                                 "single_thread": {"value": n1 / t1 / 1e9, "cores": 1,
-                                                  "sample": oracle_desc(16, n1)}}
+                                                  "sample": oracle_desc(16, n1, 1)}}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

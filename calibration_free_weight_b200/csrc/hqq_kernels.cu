@@ -51,11 +51,17 @@ constexpr int kChunkMax = 12;  // most iterations of one tensor-mode launch
 __host__ __device__ constexpr int chunk_len(int E) { return E <= 16 ? 4 : 8; }
 // Longest chunk: with C >= 8 a short last chunk is merged into the one before.
 __host__ __device__ constexpr int chunk_max(int C) { return C >= 8 ? C + C / 2 - 1 : C; }
+// Whether the last chunk writes the outputs of its last iterate when the
+// outputs are streamed (32-element tiles; the smaller tiles have no spare
+// registers for it).
+__host__ __device__ constexpr bool last_chunk_outputs(int E) { return E > 16; }
 
 // Header words of the workspace (uint32 index); word 0 is the status word.
 constexpr int kWordTicket = 1;
 constexpr int kWordZmin = 2;   // ~key(min kept zero), by atomicMax
 constexpr int kWordZmax = 3;   // key(max kept zero), by atomicMax
+constexpr int kWordSpecZmin = 4;  // the same two keys for the zeros of the last tensor-mode iterate
+constexpr int kWordSpecZmax = 5;
 constexpr int kWordPass = 8;   // survivor count of group pass p at kWordPass + p
 constexpr int kMaxPasses = 16;
 
@@ -88,8 +94,10 @@ __device__ __forceinline__ float key_value(uint32_t u) {
 // Block-wide min/max of the kept zeros, merged into the workspace header by
 // two atomics per CTA (exact and order-independent, so launches and slices
 // can all contribute).  The header starts at zero: the neutral element of both.
+// The keys go to header words `word` (min) and `word` + 1 (max).
 template <int NW>
-__device__ __forceinline__ void merge_zero_range(const KParams& k, float zmin, float zmax, float2* sred) {
+__device__ __forceinline__ void merge_zero_range(const KParams& k, float zmin, float zmax, float2* sred,
+                                                 int word = kWordZmin) {
     for (int o = 16; o > 0; o >>= 1) {
         zmin = fminf(zmin, __shfl_xor_sync(kFull, zmin, o));
         zmax = fmaxf(zmax, __shfl_xor_sync(kFull, zmax, o));
@@ -104,8 +112,8 @@ __device__ __forceinline__ void merge_zero_range(const KParams& k, float zmin, f
             r.y = fmaxf(r.y, sred[w].y);
         }
         if (r.x <= r.y) {  // this CTA stored at least one zero
-            atomicMax(k.counters + kWordZmin, ~order_key(r.x));
-            atomicMax(k.counters + kWordZmax, order_key(r.y));
+            atomicMax(k.counters + word, ~order_key(r.x));
+            atomicMax(k.counters + word + 1, order_key(r.y));
         }
     }
 }
@@ -530,6 +538,11 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2)
     const int nk = k1 - k0;
     const float* const Zin = chunk > 0 ? zslot(chunk - 1, k0 - prev_begin) : nullptr;
     float* const Zcur = zslot(chunk, 0);
+    // Streamed outputs: the last chunk also writes the outputs of its last
+    // iterate.  They are the call's outputs whenever no tensor error rose
+    // (the kept iterate is then the last one); otherwise the output kernel
+    // overwrites every one of them.
+    const bool spec = AXIS == 1 && last_chunk_outputs(E) && !write_outputs && k1 == iters;
     // per-thread tensor error partials: registers for small tiles, else shared
     constexpr int CM = chunk_max(C);
     double accr[CM] = {};
@@ -586,6 +599,7 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2)
         // small tiles: unrolled over the chunk's iterations (more independent
         // work in flight); large tiles: a loop, to keep the code cache-resident
         float* const zrow = (w.valid && w.part == 0) ? Zcur + w.j : nullptr;
+        float zl = z;  // zero-point of the last iteration run
         if constexpr (E <= 16) {
 #pragma unroll
             for (int q = 0; q < CM; ++q)
@@ -598,12 +612,20 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2)
 #pragma unroll 1
             for (int q = 0; q < nk; ++q) {
                 if (zrow) zrow[q * G] = z;
+                zl = z;
                 tensor_iteration<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z0, k0 + q, sthr[q], spow, sws2, inv_g,
                                               saccf[q][threadIdx.x], z);
             }
         }
         if (zrow) zrow[nk * G] = z;  // the next chunk's first zero-point
+        if constexpr (AXIS == 1 && last_chunk_outputs(E)) {
+            if (spec) {
+                store_lane_codes<AXIS, E>(k, w, ws, zl);
+                if (w.valid && w.part == 0) store_group(k, w.j, s, zl, iters - 1, 0.0f, &zmin, &zmax);
+            }
+        }
     }
+    if (spec && k.zero_nbits == 8) merge_zero_range<kRegWarps>(k, zmin, zmax, sred, kWordSpecZmin);
     // per-CTA partials (fixed order), then the last CTA sums them in a fixed order
     if constexpr (E <= 16) {
 #pragma unroll
@@ -638,12 +660,13 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2)
     if (threadIdx.x == 0) k.counters[kWordTicket] = 0;
 }
 
-// The outputs of a tensor-stop call, axis 1, no debug outputs: a streaming
-// pass over W after the last chunk, one 8-element piece per thread: the kept
-// iterate (first rise of the stored tensor errors), its stored zero-point and
-// the stored scale give the codes; the first piece of a group writes the
-// group's scale and zero.  Far fewer registers than the chunk kernel, so far
-// more loads in flight.
+// The outputs of a tensor-stop call, axis 1, no debug outputs.  The kept
+// iterate is the first rise of the stored tensor errors.  When no error rose
+// it is the last iterate, whose outputs the last chunk already wrote, and
+// there is nothing left to do.  Otherwise a streaming pass over W (persistent
+// CTAs, 8-element pieces, kOutPieces per thread with their loads issued
+// together): the kept iterate's stored zero-point and the stored scale give
+// the codes; the first piece of a group writes the group's scale and zero.
 constexpr int kOutPieces = 4;  // pieces per thread of tensor_output_kernel, loads issued together
 
 template <int DT, int NBITS>
@@ -671,6 +694,13 @@ __global__ void __launch_bounds__(256) tensor_output_kernel(const KParams k) {
     }
     __syncthreads();
     const int kb = skb;
+    if (kb == iters - 1 && last_chunk_outputs(k.E)) {  // no error rose: the last chunk wrote these outputs
+        if (k.zero_nbits == 8 && blockIdx.x == 0 && threadIdx.x == 0) {
+            k.counters[kWordZmin] = __ldcg(k.counters + kWordSpecZmin);
+            k.counters[kWordZmax] = __ldcg(k.counters + kWordSpecZmax);
+        }
+        return;
+    }
     const int C = chunk_len(k.E);
     const int cb = chunk_of(kb, C, iters), b0 = chunk_begin(cb, iters, C);
     const int64_t slots = chunk_max(C) + 1;
@@ -679,40 +709,44 @@ __global__ void __launch_bounds__(256) tensor_output_kernel(const KParams k) {
     while ((kPiece << log_ppg) < k.g) ++log_ppg;  // pieces per group: g / 8, a power of two
     float zmin = FLT_MAX, zmax = -FLT_MAX;
     const int64_t npieces = k.n / kPiece;
-    const int64_t pc0 = static_cast<int64_t>(blockIdx.x) * 256 * kOutPieces + threadIdx.x;
-    uint4 raw[kOutPieces];
-    float sv[kOutPieces], zv[kOutPieces];
+    const int64_t nblk = (npieces + 256 * kOutPieces - 1) / (256 * kOutPieces);
+    for (int64_t blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
+        const int64_t pc0 = blk * 256 * kOutPieces + threadIdx.x;
+        uint4 raw[kOutPieces];
+        float sv[kOutPieces], zv[kOutPieces];
 #pragma unroll
-    for (int u = 0; u < kOutPieces; ++u) {
-        const int64_t pc = pc0 + u * 256;
-        if (pc < npieces) {
-            const int64_t j = pc >> log_ppg;
-            raw[u] = __ldg(reinterpret_cast<const uint4*>(k.W) + pc);
-            sv[u] = __ldg(k.t_s + j);
-            zv[u] = __ldcg(Zc + j);
+        for (int u = 0; u < kOutPieces; ++u) {
+            const int64_t pc = pc0 + u * 256;
+            if (pc < npieces) {
+                const int64_t j = pc >> log_ppg;
+                raw[u] = __ldg(reinterpret_cast<const uint4*>(k.W) + pc);
+                sv[u] = __ldg(k.t_s + j);
+                zv[u] = __ldcg(Zc + j);
+            }
         }
-    }
 #pragma unroll
-    for (int u = 0; u < kOutPieces; ++u) {
-        const int64_t pc = pc0 + u * 256;
-        if (pc >= npieces) break;
-        float x[kPiece];
-        unpack8<DT>(raw[u], x);
-        uint32_t code[kPiece];
+        for (int u = 0; u < kOutPieces; ++u) {
+            const int64_t pc = pc0 + u * 256;
+            if (pc >= npieces) break;
+            float x[kPiece];
+            unpack8<DT>(raw[u], x);
+            uint32_t code[kPiece];
 #pragma unroll
-        for (int i = 0; i < kPiece; ++i) round_clamp(__fadd_rn(__fmul_rn(x[i], sv[u]), zv[u]), Lf, &code[i]);
-        const uint64_t v = pack8_t<NBITS>(code);
-        uint8_t* dst = k.packed + pc * NBITS;
-        if (NBITS == 8) *reinterpret_cast<uint64_t*>(dst) = v;
-        else if (NBITS == 4) *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(v);
-        else if (NBITS == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(v);
-        else if (NBITS == 1) *dst = static_cast<uint8_t>(v);
-        else {
-            dst[0] = static_cast<uint8_t>(v);
-            dst[1] = static_cast<uint8_t>(v >> 8);
-            dst[2] = static_cast<uint8_t>(v >> 16);
+            for (int i = 0; i < kPiece; ++i) round_clamp(__fadd_rn(__fmul_rn(x[i], sv[u]), zv[u]), Lf, &code[i]);
+            const uint64_t v = pack8_t<NBITS>(code);
+            uint8_t* dst = k.packed + pc * NBITS;
+            if (NBITS == 8) *reinterpret_cast<uint64_t*>(dst) = v;
+            else if (NBITS == 4) *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(v);
+            else if (NBITS == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(v);
+            else if (NBITS == 1) *dst = static_cast<uint8_t>(v);
+            else {
+                dst[0] = static_cast<uint8_t>(v);
+                dst[1] = static_cast<uint8_t>(v >> 8);
+                dst[2] = static_cast<uint8_t>(v >> 16);
+            }
+            if ((pc & ((int64_t{1} << log_ppg) - 1)) == 0)
+                store_group(k, pc >> log_ppg, sv[u], zv[u], kb, 0.0f, &zmin, &zmax);
         }
-        if ((pc & ((int64_t{1} << log_ppg) - 1)) == 0) store_group(k, pc >> log_ppg, sv[u], zv[u], kb, 0.0f, &zmin, &zmax);
     }
     if (k.zero_nbits == 8) merge_zero_range<8>(k, zmin, zmax, sred);
 }
@@ -1184,15 +1218,21 @@ cudaError_t launch_tensor(KParams& k, cudaStream_t stream) {
         return cudaGetLastError();
     }
     const int64_t pieces = k.n / kPiece;
-    const unsigned og = static_cast<unsigned>((pieces + 256 * kOutPieces - 1) / (256 * kOutPieces));
+    const int64_t blocks = (pieces + 256 * kOutPieces - 1) / (256 * kOutPieces);
+    auto launch_out = [&](auto kernel) {
+        int og = 0;
+        cudaError_t e = persistent_grid(kernel, 256, 0, blocks, &og);
+        if (e != cudaSuccess) return e;
+        kernel<<<og, 256, 0, stream>>>(k);
+        return cudaGetLastError();
+    };
     switch (k.nbits) {
-        case 1: tensor_output_kernel<DT, 1><<<og, 256, 0, stream>>>(k); break;
-        case 2: tensor_output_kernel<DT, 2><<<og, 256, 0, stream>>>(k); break;
-        case 3: tensor_output_kernel<DT, 3><<<og, 256, 0, stream>>>(k); break;
-        case 4: tensor_output_kernel<DT, 4><<<og, 256, 0, stream>>>(k); break;
-        default: tensor_output_kernel<DT, 8><<<og, 256, 0, stream>>>(k); break;
+        case 1: return launch_out(tensor_output_kernel<DT, 1>);
+        case 2: return launch_out(tensor_output_kernel<DT, 2>);
+        case 3: return launch_out(tensor_output_kernel<DT, 3>);
+        case 4: return launch_out(tensor_output_kernel<DT, 4>);
+        default: return launch_out(tensor_output_kernel<DT, 8>);
     }
-    return cudaGetLastError();
 }
 
 template <int DT, int AXIS, int E>

@@ -233,3 +233,44 @@ def test_tensor_outputs_without_debug(hq, nbits, g, zb, iters):
         assert torch.equal(ref[k].view(torch.uint8), got[k].view(torch.uint8)), k
     # and the debug run against the oracle
     _run(hq, W.cpu(), _params(nbits, g, stop=1, zb=zb, iters=iters), check_recon=False)
+
+
+def _nodebug_equals_debug(hq, W, nbits, g, zb, iters):
+    ref = hq.quantize(W, nbits, g, iters=iters, stop_mode=1, zero_nbits=zb, debug=True)
+    got = hq.quantize(W, nbits, g, iters=iters, stop_mode=1, zero_nbits=zb)
+    torch.cuda.synchronize()
+    assert hq.hqq_get_status(got["workspace"]) == hq.HQQ_OK
+    for k in ("packed", "scale", "zero", "zero_meta"):
+        if ref[k] is None:
+            continue
+        assert torch.equal(ref[k].view(torch.uint8), got[k].view(torch.uint8)), k
+
+
+@pytest.mark.parametrize("nbits,g,zb", [(4, 64, 16), (2, 64, 8), (1, 32, 16), (8, 128, 8), (3, 256, 16)])
+@pytest.mark.parametrize("place", ["last", "rise_last", "rise_in_last_chunk", "rise_before_last_chunk"])
+def test_tensor_outputs_kept_iterate_placement(hq, nbits, g, zb, place):
+    """Without debug outputs the last chunk writes the outputs of its last
+    iterate, and the output pass rewrites them when a tensor error rose.  The
+    iteration count is set from the oracle's own tensor trajectory (kept
+    iterate kb at 100 iterations, its error rising at kb + 1) so that the
+    rise falls after the last iteration, at it, inside the last chunk, or
+    before the last chunk; the outputs must equal the debug run's, and the
+    debug run must match the oracle."""
+    W_cpu = synth.weight(600, 1024, seed=nbits * 53 + g, dtype=torch.bfloat16)
+    Wo, dt = pc.w_for_oracle(W_cpu)
+    kb = int(oracle.quantize(Wo, nbits, g, 1, 0.7, 1.0, 1.01, 100, 1, zb, dtype=dt)["best_iter"][0])
+    assert 4 <= kb < 90, kb
+    iters = {"last": kb + 1, "rise_last": kb + 2, "rise_in_last_chunk": kb + 4,
+             "rise_before_last_chunk": kb + 30}[place]
+    _nodebug_equals_debug(hq, W_cpu.cuda(), nbits, g, zb, iters)
+    _run(hq, W_cpu, _params(nbits, g, stop=1, zb=zb, iters=iters), check_recon=False)
+
+
+@pytest.mark.parametrize("nbits,g", SWEEP)
+@pytest.mark.parametrize("zb", [16, 8])
+def test_llama_mlp_tensor_mode_outputs_without_debug(hq, nbits, g, zb):
+    """The benchmark's launch configuration (tensor stop, no debug outputs) on
+    the Llama-2-7B gate shape: the same bytes as the debug run, which
+    test_llama_mlp_tensor_mode checks against the oracle."""
+    W = synth.weight(11008, 4096, seed=4, dtype=torch.bfloat16).cuda()
+    _nodebug_equals_debug(hq, W, nbits, g, zb, 20)
