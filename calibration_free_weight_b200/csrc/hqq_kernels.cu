@@ -62,6 +62,8 @@ constexpr int kWordZmin = 2;   // ~key(min kept zero), by atomicMax
 constexpr int kWordZmax = 3;   // key(max kept zero), by atomicMax
 constexpr int kWordSpecZmin = 4;  // the same two keys for the zeros of the last tensor-mode iterate
 constexpr int kWordSpecZmax = 5;
+constexpr int kWordStopAt = 6;  // tensor stop rule over the iterations run so far: first rise + 1 (0: none)
+constexpr int kWordBestIt = 7;  // and the kept iterate + 1 (0: none), written by each chunk's last CTA
 constexpr int kWordPass = 8;   // survivor count of group pass p at kWordPass + p
 constexpr int kMaxPasses = 16;
 
@@ -438,6 +440,69 @@ __device__ __forceinline__ void tensor_iteration(const KParams& k, const WarpTil
     if (w.valid) acc += static_cast<Acc>(err * spow);
 }
 
+// tensor_iteration that also stores the packed codes of the evaluated
+// iterate (axis 1).  On the fast path the codes are the ones the evaluation
+// rounds to (every v is clamp-free, so round-half-even is already in [0, L]),
+// packed as they come: element e of the lane at bit e * NBITS of the lane's
+// E * NBITS / 8 bytes, which start on a multiple of 4 * NBITS bytes (the
+// packed buffer is 16-byte aligned, g >= 32).  Otherwise the codes are
+// recomputed with the clamp after the step.
+template <int DT, int E, int NBITS, typename Acc>
+__device__ __forceinline__ void tensor_iteration_codes(const KParams& k, const WarpTile& w, const float* ws,
+                                                       float lmin, float lmax, float s, float z0, int it, float thr,
+                                                       float spow, F2 sws2, float inv_g, Acc& acc, float& z) {
+    static_assert(E == 32, "one lane holds 32 elements");
+    const bool sp = w.valid && shrink_possible(s, z, z0, thr, k.Lf);
+    if (__all_sync(kFull, !w.valid || (!sp && clamp_free(lmin, lmax, z, k.Lf)))) {
+        float err = 0.0f, sq = 0.0f;
+        uint32_t pk[NBITS] = {};
+        if (w.valid) {
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const ElemEval e = eval_elem_nc(ws[i], z);
+                err += pow_pos(fabsf(e.r), k.p);
+                sq += e.q;
+                const int b = i * NBITS;
+                pk[b / 32] |= e.code << (b % 32);
+                if (b % 32 + NBITS > 32) pk[b / 32 + 1] |= e.code >> (32 - b % 32);
+            }
+            uint8_t* dst = k.packed + (w.j * (k.g / kPiece) + w.part * (E / kPiece)) * NBITS;
+            if (NBITS == 1) {
+                *reinterpret_cast<uint32_t*>(dst) = pk[0];
+            } else if (NBITS == 2) {
+                *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1 % NBITS]);
+            } else if (NBITS == 3) {
+#pragma unroll
+                for (int m = 0; m < NBITS; ++m) reinterpret_cast<uint32_t*>(dst)[m] = pk[m];
+            } else {
+#pragma unroll
+                for (int m = 0; m < NBITS; m += 4)
+                    reinterpret_cast<uint4*>(dst)[m / 4] =
+                        make_uint4(pk[m], pk[(m + 1) % NBITS], pk[(m + 2) % NBITS], pk[(m + 3) % NBITS]);
+            }
+        }
+        sq = seg_sum(sq, k.P);
+        z = zero_from_sums_f2(sq, sws2, inv_g);
+        if (w.valid) acc += static_cast<Acc>(err * spow);
+    } else {
+        const float ze = z;
+        tensor_iteration<DT, 1, E>(k, w, ws, lmin, lmax, s, z0, it, thr, spow, sws2, inv_g, acc, z);
+        if (w.valid) store_lane_codes_t<1, E, NBITS>(k, w, ws, ze);
+    }
+}
+
+// tensor_iteration_codes with the bit width chosen by a warp-uniform switch.
+template <int DT, int E, typename... Args>
+__device__ __forceinline__ void tensor_iteration_codes_n(int nbits, Args&&... args) {
+    switch (nbits) {
+        case 1: tensor_iteration_codes<DT, E, 1>(args...); break;
+        case 2: tensor_iteration_codes<DT, E, 2>(args...); break;
+        case 3: tensor_iteration_codes<DT, E, 3>(args...); break;
+        case 4: tensor_iteration_codes<DT, E, 4>(args...); break;
+        default: tensor_iteration_codes<DT, E, 8>(args...); break;
+    }
+}
+
 __device__ __forceinline__ double warp_sum_d(double x) {
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
     return x;
@@ -465,21 +530,13 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2)
     const int iters = k.iters_eff;
     constexpr int C = chunk_len(E);
     const int nch = num_chunks(iters, C);
-    // Stop rule on the tensor errors of iterations [0, k0) (same decision in every CTA).
+    // Stop rule on the tensor errors of iterations [0, k0) (same decision in
+    // every CTA), as summarised by the last CTA of the last chunk that ran.
     const int k0 = chunk_begin(chunk, iters, C);
     int best_it = -1, stop_at = -1;
-    {
-        double best = INFINITY;
-        for (int it = 0; it < k0; ++it) {
-            const double e = __ldcg(k.etot + it);
-            if (e < best) {
-                best = e;
-                best_it = it;
-            } else {
-                stop_at = it;
-                break;
-            }
-        }
+    if (k0 > 0) {
+        stop_at = static_cast<int>(__ldcg(k.counters + kWordStopAt)) - 1;
+        best_it = static_cast<int>(__ldcg(k.counters + kWordBestIt)) - 1;
     }
     const int prev_begin = chunk > 0 ? chunk_begin(chunk - 1, iters, C) : 0;
     bool finalize;
@@ -599,7 +656,6 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2)
         // small tiles: unrolled over the chunk's iterations (more independent
         // work in flight); large tiles: a loop, to keep the code cache-resident
         float* const zrow = (w.valid && w.part == 0) ? Zcur + w.j : nullptr;
-        float zl = z;  // zero-point of the last iteration run
         if constexpr (E <= 16) {
 #pragma unroll
             for (int q = 0; q < CM; ++q)
@@ -609,21 +665,25 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2)
                                                   accr[q], z);
                 }
         } else {
+            const int nrun = spec ? nk - 1 : nk;  // with streamed outputs the last iteration also stores codes
 #pragma unroll 1
-            for (int q = 0; q < nk; ++q) {
+            for (int q = 0; q < nrun; ++q) {
                 if (zrow) zrow[q * G] = z;
-                zl = z;
                 tensor_iteration<DT, AXIS, E>(k, w, ws, lmin, lmax, s, z0, k0 + q, sthr[q], spow, sws2, inv_g,
                                               saccf[q][threadIdx.x], z);
             }
-        }
-        if (zrow) zrow[nk * G] = z;  // the next chunk's first zero-point
-        if constexpr (AXIS == 1 && last_chunk_outputs(E)) {
-            if (spec) {
-                store_lane_codes<AXIS, E>(k, w, ws, zl);
-                if (w.valid && w.part == 0) store_group(k, w.j, s, zl, iters - 1, 0.0f, &zmin, &zmax);
+            if constexpr (AXIS == 1 && last_chunk_outputs(E)) {
+                if (spec) {
+                    const int q = nk - 1;
+                    const float zl = z;
+                    if (zrow) zrow[q * G] = z;
+                    tensor_iteration_codes_n<DT, E>(k.nbits, k, w, ws, lmin, lmax, s, z0, k0 + q, sthr[q], spow,
+                                                    sws2, inv_g, saccf[q][threadIdx.x], z);
+                    if (w.valid && w.part == 0) store_group(k, w.j, s, zl, iters - 1, 0.0f, &zmin, &zmax);
+                }
             }
         }
+        if (zrow) zrow[nk * G] = z;  // the next chunk's first zero-point
     }
     if (spec && k.zero_nbits == 8) merge_zero_range<kRegWarps>(k, zmin, zmax, sred, kWordSpecZmin);
     // per-CTA partials (fixed order), then the last CTA sums them in a fixed order
@@ -650,18 +710,43 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2)
     __syncthreads();
     if (!sflag) return;
     __threadfence();
+    // the tensor errors of iterations [0, k1): earlier ones from memory, this chunk's from the partials
+    static_assert(kChunkMax * kRegThreads >= kMaxIters, "the error history fits in the partials' buffer");
+    double* const serr = &sacc[0][0];  // free once the partials are written
+    for (int it = threadIdx.x; it < k0; it += kRegThreads) serr[it] = __ldcg(k.etot + it);
     for (int q = warp; q < nk; q += kRegWarps) {
         double v = 0.0;
         for (unsigned b = lane; b < gridDim.x; b += 32)
             v += __ldcg(k.tparts + static_cast<size_t>(q) * kMaxPartials + b);
         v = warp_sum_d(v);
-        if (lane == 0) k.etot[k0 + q] = v / static_cast<double>(k.n);
+        if (lane == 0) {
+            const double e = v / static_cast<double>(k.n);
+            k.etot[k0 + q] = e;
+            serr[k0 + q] = e;
+        }
     }
-    if (threadIdx.x == 0) k.counters[kWordTicket] = 0;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // stop at the first iteration whose error is not below the best so far
+        int bi = -1, sa = -1;
+        double best = INFINITY;
+        for (int it = 0; it < k1; ++it) {
+            if (serr[it] < best) {
+                best = serr[it];
+                bi = it;
+            } else {
+                sa = it;
+                break;
+            }
+        }
+        k.counters[kWordStopAt] = static_cast<uint32_t>(sa + 1);
+        k.counters[kWordBestIt] = static_cast<uint32_t>(bi + 1);
+        k.counters[kWordTicket] = 0;
+    }
 }
 
 // The outputs of a tensor-stop call, axis 1, no debug outputs.  The kept
-// iterate is the first rise of the stored tensor errors.  When no error rose
+// iterate (the stop rule's outcome) is in the workspace header.  When no error rose
 // it is the last iterate, whose outputs the last chunk already wrote, and
 // there is nothing left to do.  Otherwise a streaming pass over W (persistent
 // CTAs, 8-element pieces, kOutPieces per thread with their loads issued
@@ -669,31 +754,41 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2)
 // the codes; the first piece of a group writes the group's scale and zero.
 constexpr int kOutPieces = 4;  // pieces per thread of tensor_output_kernel, loads issued together
 
+// Codes of one 8-element piece at (s, z), packed LSB first.  As in
+// round_clamp, t = fl(clamp(fl(fl(w*s) + z), 0, L) + 1.5*2^23) holds the code
+// in its low mantissa bits: bits(t) = bits(1.5*2^23) + code.  So the packed
+// value is the sum of bits(t_i) << (i * NBITS) less the magic's share of that
+// sum, all mod 2^32 (one multiply-add per element).
+template <int DT, int NBITS>
+__device__ __forceinline__ uint64_t piece_codes(const uint4 raw, float s, float z) {
+    constexpr float Lf = static_cast<float>((1 << NBITS) - 1);
+    constexpr int kPer = NBITS == 8 ? 4 : 8;  // codes per 32-bit word
+    constexpr uint32_t kOnes = NBITS == 8 ? 0x01010101u
+                               : NBITS == 4 ? 0x11111111u
+                               : NBITS == 3 ? 0x00249249u
+                               : NBITS == 2 ? 0x00005555u
+                                            : 0x000000ffu;  // sum of 1 << (i * NBITS) over a word's codes
+    constexpr uint32_t kMagicShare = kMagicBits * kOnes;     // mod 2^32
+    float x[kPiece];
+    unpack8<DT>(raw, x);
+    uint32_t word[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < kPiece; ++i) {
+        const float t = __fadd_rn(fminf(fmaxf(__fadd_rn(__fmul_rn(x[i], s), z), 0.0f), Lf), kMagic);
+        word[i / kPer] += __float_as_uint(t) << ((i % kPer) * NBITS);
+    }
+    if (NBITS == 8)
+        return static_cast<uint64_t>(word[0] - kMagicShare) | (static_cast<uint64_t>(word[1] - kMagicShare) << 32);
+    return word[0] - kMagicShare;
+}
+
 template <int DT, int NBITS>
 __global__ void __launch_bounds__(256) tensor_output_kernel(const KParams k) {
     __shared__ float2 sred[8];
-    __shared__ double serr[kMaxIters];
-    __shared__ int skb;
-    constexpr float Lf = static_cast<float>((1 << NBITS) - 1);
     const int iters = k.iters_eff;
-    // kept iterate: the tensor errors loaded in parallel, scanned by one thread
-    for (int it = threadIdx.x; it < iters; it += 256) serr[it] = __ldcg(k.etot + it);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int kb = iters - 1;
-        double best = INFINITY;
-        for (int it = 0; it < iters; ++it) {
-            if (serr[it] < best) {
-                best = serr[it];
-                kb = it;
-            } else {
-                break;
-            }
-        }
-        skb = kb;
-    }
-    __syncthreads();
-    const int kb = skb;
+    // kept iterate: the stop rule's outcome, written by the last chunk that ran
+    const int bi = static_cast<int>(__ldcg(k.counters + kWordBestIt)) - 1;
+    const int kb = bi < 0 ? 0 : bi;
     if (kb == iters - 1 && last_chunk_outputs(k.E)) {  // no error rose: the last chunk wrote these outputs
         if (k.zero_nbits == 8 && blockIdx.x == 0 && threadIdx.x == 0) {
             k.counters[kWordZmin] = __ldcg(k.counters + kWordSpecZmin);
@@ -728,12 +823,7 @@ __global__ void __launch_bounds__(256) tensor_output_kernel(const KParams k) {
         for (int u = 0; u < kOutPieces; ++u) {
             const int64_t pc = pc0 + u * 256;
             if (pc >= npieces) break;
-            float x[kPiece];
-            unpack8<DT>(raw[u], x);
-            uint32_t code[kPiece];
-#pragma unroll
-            for (int i = 0; i < kPiece; ++i) round_clamp(__fadd_rn(__fmul_rn(x[i], sv[u]), zv[u]), Lf, &code[i]);
-            const uint64_t v = pack8_t<NBITS>(code);
+            const uint64_t v = piece_codes<DT, NBITS>(raw[u], sv[u], zv[u]);
             uint8_t* dst = k.packed + pc * NBITS;
             if (NBITS == 8) *reinterpret_cast<uint64_t*>(dst) = v;
             else if (NBITS == 4) *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(v);
