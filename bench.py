@@ -414,6 +414,72 @@ def run_stream(args):
         torch.distributed.destroy_process_group()
 
 
+LLAMA13B_NAMES = {"q": "self_attn.q_proj", "k": "self_attn.k_proj", "v": "self_attn.v_proj",
+                  "o": "self_attn.o_proj", "gate": "mlp.gate_proj", "up": "mlp.up_proj", "down": "mlp.down_proj"}
+LLAMA13B_CONFIG = dict(base=dict(nbits=4, group_size=64, stop_mode=1),
+                       dynamic={"attn": dict(nbits=4, group_size=64, stop_mode=1),
+                                "mlp": dict(nbits=2, group_size=32, stop_mode=1)})
+
+
+def run_stream_mixed(args):
+    """Llama-2-13B-shaped model (40 layers x q, k, v, o 5120x5120, gate/up
+    13824x5120, down 5120x13824; fp16) with per-layer-type settings
+    (attention b4 g64, MLP b2 g32, tensor stop, fp16 zero) streamed layer by
+    layer from pinned host memory through hqq_quantize_stream_jobs.  As in
+    the 70B workload, one layer of synthetic weights is streamed for every
+    layer.  Under torchrun each rank streams its share of the layers."""
+    from calibration_free_weight_b200 import hqq
+    world, rank, local = dist_setup()
+    model = synth.LLAMA2_13B
+    layers = args.layers if args.layers_given else model.layers
+    mine = len(rank_layers(layers, world, rank))
+    mats = model.matrices()
+    Ws = [synth.weight(r, c, seed=synth.seed_for(0, n), dtype=torch.float16).pin_memory() for n, r, c in mats]
+    sets = [hqq.settings_for(f"model.layers.0.{LLAMA13B_NAMES[n]}", LLAMA13B_CONFIG["base"],
+                             LLAMA13B_CONFIG["dynamic"]) for n, _, _ in mats]
+    outs = [hqq.host_outputs(r, c, st["nbits"], st["group_size"], st["axis"], st["zero_nbits"])
+            for (_, r, c), st in zip(mats, sets)]
+    w_layer = model.weights_per_layer()
+    buf, _ = hqq.quantize_stream_jobs(Ws, sets, outs)  # warm-up: one layer
+    barrier(world)
+    t0 = time.perf_counter()
+    done = 0
+    if mine:
+        _, done = hqq.quantize_stream_jobs(Ws * mine, sets * mine, outs * mine, device_buffer=buf)
+    wall = max_over_ranks(time.perf_counter() - t0, world)
+    barrier(world)
+    del buf
+    # the same matrices resident on the device: solver time per layer (CUDA events)
+    dev = [w.cuda() for w in Ws]
+    q = [hqq.alloc_outputs(r, c, st["nbits"], st["group_size"], 1, st["stop_mode"], 16)
+         for (_, r, c), st in zip(mats, sets)]
+    call = lambda: [hqq.quantize(w, st["nbits"], st["group_size"], stop_mode=st["stop_mode"], out=o)  # noqa: E731
+                    for w, st, o in zip(dev, sets, q)]
+    for _ in range(2):
+        call()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    call()
+    b.record()
+    torch.cuda.synchronize()
+    layer_ms = a.elapsed_time(b)
+    h2d = 2 * w_layer * layers
+    d2h = sum(o["packed"].numel() + o["scale"].numel() * 2 + o["zero"].numel() * 2 for o in outs) * layers
+    if rank == 0:
+        print(json.dumps({"workload": "llama2-13b-stream", "layers": layers, "weights": w_layer * layers,
+                          "n_gpus": world, "scaling": "layers split across ranks", "dtype_in": "fp16",
+                          "settings": {"attn (q, k, v, o)": sets[0], "mlp (gate, up, down)": sets[4]},
+                          "zero": "fp16", "host": "pinned", "matrices_done_rank0": done,
+                          "data": "synthetic; one layer's buffers streamed for every layer",
+                          "e2e_s": wall, "e2e_gweights_s": w_layer * layers / wall / 1e9, "h2d_bytes": h2d,
+                          "d2h_bytes": d2h, "h2d_gbs_effective": h2d / wall / 1e9,
+                          "device_resident": {"ms_per_layer": layer_ms,
+                                              "gweights_s": w_layer / (layer_ms / 1e3) / 1e9,
+                                              "solve_s_all_layers": layer_ms / 1e3 * layers}}))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def run_gemv_case(spec):
     """Time hqq_gemv (fused dequantisation + matrix-vector product) on one
     quantised synthetic fp16 matrix: "gemv,rows,cols,nbits,g[,batch[,reps]]".
@@ -495,11 +561,19 @@ def main():
                     help="single-matrix timing instead of the sweep: stop_mode,rows,cols,nbits,group_size[,reps]; "
                          "or scale8,G[,S[,reps]] for the 8-bit scale quantiser, "
                          "or gemv,rows,cols,nbits,g[,batch[,reps]] for the fused dequantise + matrix-vector product")
-    ap.add_argument("--workload", default="llama2-7b-mlp-sweep", choices=["llama2-7b-mlp-sweep", "llama2-70b-stream"])
-    ap.add_argument("--layers", type=int, default=80, help="layers of the llama2-70b-stream workload")
+    ap.add_argument("--workload", default="llama2-7b-mlp-sweep",
+                    choices=["llama2-7b-mlp-sweep", "llama2-70b-stream", "llama2-13b-stream"])
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers of a streamed-model workload (default: the model's, 80 or 40)")
     args = ap.parse_args()
+    args.layers_given = args.layers is not None
     if args.workload == "llama2-70b-stream":
+        if not args.layers_given:
+            args.layers = 80
         run_stream(args)
+        return
+    if args.workload == "llama2-13b-stream":
+        run_stream_mixed(args)
         return
     if args.case:
         run_case(args.case)

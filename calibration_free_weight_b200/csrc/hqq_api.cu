@@ -51,10 +51,8 @@ bool is_device_ptr(const void* p) {
 
 namespace hqq {
 
-int quantize_entry(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p,
-                   float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* W_q_packed, void* scale,
-                   void* zero, void* zero_meta, void* workspace, size_t workspace_bytes, bool allow_slices,
-                   int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32, void* stream) {
+int check_args(int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p, float beta,
+               float kappa, int iters, int stop_mode, int zero_nbits) {
     if (dtype != HQQ_F16 && dtype != HQQ_BF16) return HQQ_ERR_DTYPE;
     if (!valid_nbits(nbits)) return HQQ_ERR_INVALID_ARG;
     const int sh = check_shape(rows, cols, group_size, axis);
@@ -65,6 +63,15 @@ int quantize_entry(const void* W, int64_t rows, int64_t cols, int dtype, int nbi
     if (iters < 0 || iters > hqq::kMaxIters) return HQQ_ERR_INVALID_ARG;
     if (stop_mode < 0 || stop_mode > 2) return HQQ_ERR_INVALID_ARG;
     if (zero_nbits != 8 && zero_nbits != 16) return HQQ_ERR_INVALID_ARG;
+    return HQQ_OK;
+}
+
+int quantize_entry(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p,
+                   float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* W_q_packed, void* scale,
+                   void* zero, void* zero_meta, void* workspace, size_t workspace_bytes, bool allow_slices,
+                   int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32, void* stream) {
+    const int ck = check_args(rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode, zero_nbits);
+    if (ck != HQQ_OK) return ck;
     const int64_t G = rows * cols / group_size;
     const int64_t slice =
         hqq::fit_slice(rows, cols, group_size, axis, stop_mode, zero_nbits, workspace == nullptr ? 0 : workspace_bytes);

@@ -90,6 +90,11 @@ cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream);
 cudaError_t launch_dequant(const DequantArgs& a, cudaStream_t stream);
 cudaError_t launch_scale8(const uint16_t* scale, int64_t G, int S, uint8_t* codes, float* meta, cudaStream_t stream);
 
+// The host-side argument checks of hqq_quantize (dtype, bit width, shape,
+// solver parameters, modes): HQQ_OK or the status hqq_quantize returns.
+int check_args(int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p, float beta,
+               float kappa, int iters, int stop_mode, int zero_nbits);
+
 // hqq_quantize with an option to cut group-mode work into slices that fit a
 // smaller workspace (used by hqq_quantize_noalloc).
 int quantize_entry(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p,

@@ -1,5 +1,8 @@
-// hqq_stream.cu -- hqq_quantize_stream: quantise a list of matrices held in
-// host memory, streaming them through one GPU.
+// hqq_stream.cu -- hqq_quantize_stream / hqq_quantize_stream_jobs: quantise
+// a list of matrices held in host memory, streaming them through one GPU,
+// with settings per matrix (attention and MLP layers at different bit widths,
+// "HQQ - Half-Quadratic Quantization" (skill4agent.com), section "Mixed
+// precision quantization").
 //
 // The pages quantise a model layer by layer on the GPU and move data only
 // once per layer (techreport.ngo, "Weight-only quantization without the
@@ -12,6 +15,11 @@
 // copied in only after the solver on matrix i has finished reading it, and its
 // outputs are written only after those of matrix i have been copied out.
 //
+// Each job is reported (callback, in order) once its outputs are in host
+// memory; the report of job i-2 is taken just before its slot's copy-out event
+// is reused for job i, by which time the solver on job i has already waited
+// for that copy on the GPU, so reporting costs no overlap.
+//
 // The call blocks until every output has reached host memory.  Host buffers
 // should be pinned (cudaHostAlloc / cudaHostRegister) for the copies to
 // overlap; pageable buffers work but serialise.  Device memory is the
@@ -21,6 +29,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <vector>
 
 #include "../../include/hqq.h"
 #include "hqq_internal.h"
@@ -31,26 +40,45 @@ constexpr size_t kAlign = 256;
 
 size_t up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
-// Largest per-matrix sizes of the list (bytes).
-struct SlotSizes {
+// Buffer sizes of one job (bytes).
+struct JobSizes {
     size_t W = 0, packed = 0, scale = 0, zero = 0, workspace = 0;
-    size_t total() const { return up(W) + up(packed) + up(scale) + up(zero) + up(8) + up(workspace); }
 };
 
-int slot_sizes(const hqq_host_matrix* mats, int n, int nbits, int group_size, int axis, int stop_mode,
-               int zero_nbits, SlotSizes* out) {
+JobSizes job_sizes(const hqq_stream_job& j) {
+    const int64_t rows = j.m.rows, cols = j.m.cols;
+    const int64_t G = hqq_num_groups(rows, cols, j.group_size, j.axis);
+    JobSizes s;
+    s.W = static_cast<size_t>(rows * cols) * 2;
+    s.packed = hqq_packed_bytes(rows, cols, j.nbits, j.group_size, j.axis);
+    s.scale = static_cast<size_t>(G) * 2;
+    s.zero = static_cast<size_t>(G) * (j.zero_nbits == 16 ? 2 : 1);
+    s.workspace = hqq_workspace_bytes(rows, cols, j.group_size, j.axis, j.stop_mode, j.zero_nbits);
+    return s;
+}
+
+// One slot: each buffer kind sized for the largest job of the list.
+struct SlotSizes {
+    JobSizes m;
+    size_t total() const { return up(m.W) + up(m.packed) + up(m.scale) + up(m.zero) + up(8) + up(m.workspace); }
+};
+
+// Settings and shape of every job (the solver parameters of the call
+// included), before anything is copied or launched.
+int check_jobs(const hqq_stream_job* jobs, int n, int dtype, float p, float beta, float kappa, int iters,
+               SlotSizes* out) {
     SlotSizes s;
     for (int i = 0; i < n; ++i) {
-        const int64_t rows = mats[i].rows, cols = mats[i].cols;
-        const int64_t G = hqq_num_groups(rows, cols, group_size, axis);
-        if (G < 0) return HQQ_ERR_SHAPE;
-        const size_t ws = hqq_workspace_bytes(rows, cols, group_size, axis, stop_mode, zero_nbits);
-        if (ws == 0) return HQQ_ERR_INVALID_ARG;
-        s.W = std::max(s.W, static_cast<size_t>(rows * cols) * 2);
-        s.packed = std::max(s.packed, hqq_packed_bytes(rows, cols, nbits, group_size, axis));
-        s.scale = std::max(s.scale, static_cast<size_t>(G) * 2);
-        s.zero = std::max(s.zero, static_cast<size_t>(G) * (zero_nbits == 16 ? 2 : 1));
-        s.workspace = std::max(s.workspace, ws);
+        const hqq_stream_job& j = jobs[i];
+        const int ck = hqq::check_args(j.m.rows, j.m.cols, dtype, j.nbits, j.group_size, j.axis, p, beta, kappa, iters,
+                                       j.stop_mode, j.zero_nbits);
+        if (ck != HQQ_OK) return ck;
+        const JobSizes z = job_sizes(j);
+        s.m.W = std::max(s.m.W, z.W);
+        s.m.packed = std::max(s.m.packed, z.packed);
+        s.m.scale = std::max(s.m.scale, z.scale);
+        s.m.zero = std::max(s.m.zero, z.zero);
+        s.m.workspace = std::max(s.m.workspace, z.workspace);
     }
     *out = s;
     return HQQ_OK;
@@ -64,13 +92,13 @@ Slot carve(uint8_t* base, const SlotSizes& s) {
     Slot t;
     size_t off = 0;
     t.W = base + off;
-    off += up(s.W);
+    off += up(s.m.W);
     t.packed = base + off;
-    off += up(s.packed);
+    off += up(s.m.packed);
     t.scale = base + off;
-    off += up(s.scale);
+    off += up(s.m.scale);
     t.zero = base + off;
-    off += up(s.zero);
+    off += up(s.m.zero);
     t.meta = base + off;
     off += up(8);
     t.ws = base + off;
@@ -103,30 +131,45 @@ struct Resources {
     }
 };
 
+std::vector<hqq_stream_job> uniform_jobs(const hqq_host_matrix* mats, int n, int nbits, int group_size, int axis,
+                                         int stop_mode, int zero_nbits) {
+    std::vector<hqq_stream_job> jobs(static_cast<size_t>(n));
+    for (int i = 0; i < n; ++i) jobs[i] = hqq_stream_job{mats[i], nbits, group_size, axis, stop_mode, zero_nbits};
+    return jobs;
+}
+
 }  // namespace
 
 extern "C" {
 
-size_t hqq_stream_device_bytes(const hqq_host_matrix* mats, int n, int nbits, int group_size, int axis,
-                               int stop_mode, int zero_nbits) {
-    if (mats == nullptr || n < 1) return 0;
+size_t hqq_stream_jobs_device_bytes(const hqq_stream_job* jobs, int n) {
+    if (jobs == nullptr || n < 1) return 0;
     SlotSizes s;
-    if (slot_sizes(mats, n, nbits, group_size, axis, stop_mode, zero_nbits, &s) != HQQ_OK) return 0;
+    // solver parameters that every check accepts: only the jobs' own settings decide
+    if (check_jobs(jobs, n, HQQ_F16, 0.7f, 1.0f, 1.0f, 0, &s) != HQQ_OK) return 0;
     return 2 * s.total();
 }
 
-int hqq_quantize_stream(const hqq_host_matrix* mats, int n, int dtype, int nbits, int group_size, int axis, float p,
-                        float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* device_buffer,
-                        size_t device_bytes, void* stream) {
-    if (mats == nullptr || n < 0) return HQQ_ERR_INVALID_ARG;
+size_t hqq_stream_device_bytes(const hqq_host_matrix* mats, int n, int nbits, int group_size, int axis,
+                               int stop_mode, int zero_nbits) {
+    if (mats == nullptr || n < 1) return 0;
+    const std::vector<hqq_stream_job> jobs = uniform_jobs(mats, n, nbits, group_size, axis, stop_mode, zero_nbits);
+    return hqq_stream_jobs_device_bytes(jobs.data(), n);
+}
+
+int hqq_quantize_stream_jobs(const hqq_stream_job* jobs, int n, int dtype, float p, float beta, float kappa, int iters,
+                             void* device_buffer, size_t device_bytes, hqq_stream_done_fn on_done, void* user,
+                             int* jobs_done, void* stream) {
+    if (jobs_done) *jobs_done = 0;
+    if (jobs == nullptr || n < 0) return HQQ_ERR_INVALID_ARG;
     if (n == 0) return HQQ_OK;
     SlotSizes s;
-    const int rc0 = slot_sizes(mats, n, nbits, group_size, axis, stop_mode, zero_nbits, &s);
+    const int rc0 = check_jobs(jobs, n, dtype, p, beta, kappa, iters, &s);
     if (rc0 != HQQ_OK) return rc0;
     for (int i = 0; i < n; ++i) {
-        const hqq_host_matrix& m = mats[i];
-        if (m.rows * m.cols == 0) continue;
-        if (!m.W || !m.W_q_packed || !m.scale || !m.zero || (zero_nbits == 8 && !m.zero_meta))
+        const hqq_stream_job& j = jobs[i];
+        if (j.m.rows * j.m.cols == 0) continue;
+        if (!j.m.W || !j.m.W_q_packed || !j.m.scale || !j.m.zero || (j.zero_nbits == 8 && !j.m.zero_meta))
             return HQQ_ERR_INVALID_ARG;
     }
     if (device_buffer == nullptr || device_bytes < 2 * s.total()) return HQQ_ERR_WORKSPACE;
@@ -141,40 +184,48 @@ int hqq_quantize_stream(const hqq_host_matrix* mats, int n, int dtype, int nbits
     Slot slot[2] = {carve(static_cast<uint8_t*>(device_buffer), s),
                     carve(static_cast<uint8_t*>(device_buffer) + s.total(), s)};
     int rc = HQQ_OK;
+    int reported = 0;  // jobs 0 .. reported-1 have been reported done
     auto cuda_ok = [&](cudaError_t e) {
         if (e != cudaSuccess && rc == HQQ_OK) rc = HQQ_ERR_CUDA;
         return e == cudaSuccess;
     };
+    // job k is done once its copy-out event (slot k & 1, not yet reused) has completed
+    auto report = [&](int k) {
+        if (!cuda_ok(cudaEventSynchronize(r.out_done[k & 1]))) return false;
+        if (on_done) on_done(k, user);
+        reported = k + 1;
+        return true;
+    };
     for (int i = 0; i < n && rc == HQQ_OK; ++i) {
-        const hqq_host_matrix& m = mats[i];
+        const hqq_stream_job& j = jobs[i];
+        const hqq_host_matrix& m = j.m;
         const Slot& t = slot[i & 1];
-        const int64_t G = m.rows * m.cols / group_size;
-        const size_t wb = static_cast<size_t>(m.rows * m.cols) * 2;
-        const size_t pb = hqq_packed_bytes(m.rows, m.cols, nbits, group_size, axis);
-        const size_t sb = static_cast<size_t>(G) * 2, zb = static_cast<size_t>(G) * (zero_nbits == 16 ? 2 : 1);
-        // copy-in: the solver on matrix i-2 (same slot) must have finished reading W
+        const JobSizes z = job_sizes(j);
+        // copy-in: the solver on job i-2 (same slot) must have finished reading W
         if (i >= 2 && !cuda_ok(cudaStreamWaitEvent(r.cin, r.solved[i & 1], 0))) break;
-        if (wb && !cuda_ok(cudaMemcpyAsync(t.W, m.W, wb, cudaMemcpyHostToDevice, r.cin))) break;
+        if (z.W && !cuda_ok(cudaMemcpyAsync(t.W, m.W, z.W, cudaMemcpyHostToDevice, r.cin))) break;
         if (!cuda_ok(cudaEventRecord(r.in_done[i & 1], r.cin))) break;
-        // solve: W has arrived, and matrix i-2's outputs in this slot have been copied out
+        // solve: W has arrived, and job i-2's outputs in this slot have been copied out
         if (!cuda_ok(cudaStreamWaitEvent(cs, r.in_done[i & 1], 0))) break;
         if (i >= 2 && !cuda_ok(cudaStreamWaitEvent(cs, r.out_done[i & 1], 0))) break;
-        const size_t wsb = hqq_workspace_bytes(m.rows, m.cols, group_size, axis, stop_mode, zero_nbits);
-        const int q = hqq::quantize_entry(t.W, m.rows, m.cols, dtype, nbits, group_size, axis, p, beta, kappa, iters,
-                                          stop_mode, zero_nbits, t.packed, t.scale, t.zero,
-                                          zero_nbits == 8 ? t.meta : nullptr, t.ws, wsb, false, nullptr, nullptr,
-                                          nullptr, cs);
+        const int q = hqq::quantize_entry(t.W, m.rows, m.cols, dtype, j.nbits, j.group_size, j.axis, p, beta, kappa,
+                                          iters, j.stop_mode, j.zero_nbits, t.packed, t.scale, t.zero,
+                                          j.zero_nbits == 8 ? t.meta : nullptr, t.ws, z.workspace, false, nullptr,
+                                          nullptr, nullptr, cs);
         if (q != HQQ_OK) {
             rc = q;
             break;
         }
         if (!cuda_ok(cudaEventRecord(r.solved[i & 1], cs))) break;
+        // job i-2's copy-out event is about to be reused: report it first
+        if (i >= 2 && !report(i - 2)) break;
         // copy-out
         if (!cuda_ok(cudaStreamWaitEvent(r.cout, r.solved[i & 1], 0))) break;
-        if (pb && !cuda_ok(cudaMemcpyAsync(m.W_q_packed, t.packed, pb, cudaMemcpyDeviceToHost, r.cout))) break;
-        if (sb && !cuda_ok(cudaMemcpyAsync(m.scale, t.scale, sb, cudaMemcpyDeviceToHost, r.cout))) break;
-        if (zb && !cuda_ok(cudaMemcpyAsync(m.zero, t.zero, zb, cudaMemcpyDeviceToHost, r.cout))) break;
-        if (zero_nbits == 8 && !cuda_ok(cudaMemcpyAsync(m.zero_meta, t.meta, 8, cudaMemcpyDeviceToHost, r.cout)))
+        if (z.packed && !cuda_ok(cudaMemcpyAsync(m.W_q_packed, t.packed, z.packed, cudaMemcpyDeviceToHost, r.cout)))
+            break;
+        if (z.scale && !cuda_ok(cudaMemcpyAsync(m.scale, t.scale, z.scale, cudaMemcpyDeviceToHost, r.cout))) break;
+        if (z.zero && !cuda_ok(cudaMemcpyAsync(m.zero, t.zero, z.zero, cudaMemcpyDeviceToHost, r.cout))) break;
+        if (j.zero_nbits == 8 && !cuda_ok(cudaMemcpyAsync(m.zero_meta, t.meta, 8, cudaMemcpyDeviceToHost, r.cout)))
             break;
         if (!cuda_ok(cudaEventRecord(r.out_done[i & 1], r.cout))) break;
     }
@@ -183,8 +234,22 @@ int hqq_quantize_stream(const hqq_host_matrix* mats, int n, int dtype, int nbits
     const cudaError_t e2 = cudaStreamSynchronize(r.cout);
     const cudaError_t e3 = cudaStreamSynchronize(r.cin);
     if ((e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) && rc == HQQ_OK) rc = HQQ_ERR_CUDA;
+    if (rc == HQQ_OK)
+        for (int k = reported; k < n; ++k)
+            if (!report(k)) break;
     if (rc != HQQ_OK) cudaGetLastError();
+    if (jobs_done) *jobs_done = rc == HQQ_OK ? n : reported;
     return rc;
+}
+
+int hqq_quantize_stream(const hqq_host_matrix* mats, int n, int dtype, int nbits, int group_size, int axis, float p,
+                        float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* device_buffer,
+                        size_t device_bytes, void* stream) {
+    if (mats == nullptr || n < 0) return HQQ_ERR_INVALID_ARG;
+    if (n == 0) return HQQ_OK;
+    const std::vector<hqq_stream_job> jobs = uniform_jobs(mats, n, nbits, group_size, axis, stop_mode, zero_nbits);
+    return hqq_quantize_stream_jobs(jobs.data(), n, dtype, p, beta, kappa, iters, device_buffer, device_bytes, nullptr,
+                                    nullptr, nullptr, stream);
 }
 
 }  // extern "C"

@@ -19,13 +19,23 @@ HQQ_STOP_GROUP, HQQ_STOP_TENSOR, HQQ_STOP_NONE = 0, 1, 2
 
 EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_quantize", "hqq_dequantize",
             "hqq_get_status", "hqq_status_string", "hqq_quantize_noalloc", "hqq_quantize_scale8",
-            "hqq_dequantize_s8", "hqq_stream_device_bytes", "hqq_quantize_stream", "hqq_gemv")
+            "hqq_dequantize_s8", "hqq_stream_device_bytes", "hqq_quantize_stream", "hqq_gemv",
+            "hqq_stream_jobs_device_bytes", "hqq_quantize_stream_jobs")
 
 
 class hqq_host_matrix(C.Structure):
     """struct hqq_host_matrix of include/hqq.h (host pointers)."""
     _fields_ = [("W", C.c_void_p), ("rows", C.c_int64), ("cols", C.c_int64), ("W_q_packed", C.c_void_p),
                 ("scale", C.c_void_p), ("zero", C.c_void_p), ("zero_meta", C.c_void_p)]
+
+
+class hqq_stream_job(C.Structure):
+    """struct hqq_stream_job of include/hqq.h: a host matrix and its settings."""
+    _fields_ = [("m", hqq_host_matrix), ("nbits", C.c_int), ("group_size", C.c_int), ("axis", C.c_int),
+                ("stop_mode", C.c_int), ("zero_nbits", C.c_int)]
+
+
+hqq_stream_done_fn = C.CFUNCTYPE(None, C.c_int, C.c_void_p)
 HQQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -61,6 +71,12 @@ def _load():
     L.hqq_stream_device_bytes.argtypes = [HM, i32, i32, i32, i32, i32, i32]
     L.hqq_quantize_stream.restype = i32
     L.hqq_quantize_stream.argtypes = [HM, i32, i32, i32, i32, i32, f32, f32, f32, i32, i32, i32, P, sz, P]
+    SJ = C.POINTER(hqq_stream_job)
+    L.hqq_stream_jobs_device_bytes.restype = sz
+    L.hqq_stream_jobs_device_bytes.argtypes = [SJ, i32]
+    L.hqq_quantize_stream_jobs.restype = i32
+    L.hqq_quantize_stream_jobs.argtypes = [SJ, i32, i32, f32, f32, f32, i32, P, sz, hqq_stream_done_fn, P,
+                                           C.POINTER(i32), P]
     L.hqq_quantize_noalloc.restype = i32
     L.hqq_quantize_noalloc.argtypes = [P, i64, i64, i32, i32, i32, i32, f32, f32, f32, i32, i32, i32,
                                        P, P, P, P, P, P, P, P]
@@ -149,6 +165,17 @@ def hqq_quantize_stream(mats, n, dtype, nbits, group_size, axis, p, beta, kappa,
                         device_buffer, device_bytes, stream=None):
     return lib.hqq_quantize_stream(mats, n, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
                                    zero_nbits, _ptr(device_buffer), device_bytes, _stream(stream))
+
+
+def hqq_stream_jobs_device_bytes(jobs, n):
+    return lib.hqq_stream_jobs_device_bytes(jobs, n)
+
+
+def hqq_quantize_stream_jobs(jobs, n, dtype, p, beta, kappa, iters, device_buffer, device_bytes, on_done=None,
+                             user=None, jobs_done=None, stream=None):
+    cb = on_done if on_done is not None else hqq_stream_done_fn()
+    return lib.hqq_quantize_stream_jobs(jobs, n, dtype, p, beta, kappa, iters, _ptr(device_buffer), device_bytes, cb,
+                                        user, jobs_done, _stream(stream))
 
 
 def hqq_gemv(W_q_packed, scale, zero, zero_meta, rows, cols, nbits, group_size, zero_nbits, x, x_dtype, batch, y,
@@ -245,6 +272,73 @@ def quantize_stream(Ws, outs, nbits=4, group_size=64, axis=1, p=0.7, beta=1.0, k
     if rc != HQQ_OK:
         raise HQQError(rc, "hqq_quantize_stream")
     return device_buffer
+
+
+SETTING_KEYS = ("nbits", "group_size", "axis", "stop_mode", "zero_nbits")
+
+
+def settings_for(name, base, dynamic=None):
+    """Settings of the matrix `name` (e.g. "layers.3.self_attn.q_proj"): `base`
+    (a dict of SETTING_KEYS) overridden by the first entry of `dynamic` whose
+    key occurs in the name, as in a per-layer-type config
+    {"attn": {"nbits": 4, "group_size": 64}, "mlp": {"nbits": 2, "group_size": 32}}."""
+    out = {k: base[k] for k in SETTING_KEYS if k in base}
+    for key, over in (dynamic or {}).items():
+        if key in name:
+            unknown = set(over) - set(SETTING_KEYS)
+            if unknown:
+                raise HQQError(HQQ_ERR_INVALID_ARG, f"unknown settings {sorted(unknown)} for {key!r}")
+            out.update(over)
+            break
+    defaults = dict(axis=1, stop_mode=HQQ_STOP_GROUP, zero_nbits=16)
+    return {k: out.get(k, defaults.get(k)) for k in SETTING_KEYS}
+
+
+def quantize_stream_jobs(Ws, settings, outs, p=0.7, beta=1.0, kappa=1.01, iters=20, on_done=None,
+                         device_buffer=None, stream=None):
+    """quantize_stream with settings per matrix: settings[i] is a dict of
+    SETTING_KEYS (see settings_for), outs[i] from host_outputs() with the same
+    settings.  on_done(i) runs on this thread as soon as matrix i's outputs are
+    in host memory, in order (persist them there to make a run resumable: pass
+    only the matrices not yet persisted next time).  Returns (device buffer,
+    number of leading matrices completed)."""
+    n = len(Ws)
+    if n == 0 or len(settings) != n or len(outs) != n:
+        raise HQQError(HQQ_ERR_INVALID_ARG, "quantize_stream_jobs needs one settings dict and one output dict "
+                       "per matrix")
+    dt = Ws[0].dtype
+    if dt not in _DT or any(w.dtype != dt or w.is_cuda or w.dim() != 2 or not w.is_contiguous() for w in Ws):
+        raise HQQError(HQQ_ERR_INVALID_ARG, "quantize_stream_jobs expects contiguous 2-D host tensors of one dtype")
+    arr = (hqq_stream_job * n)()
+    for a, w, st, o in zip(arr, Ws, settings, outs):
+        a.m.W, a.m.rows, a.m.cols = w.data_ptr(), w.shape[0], w.shape[1]
+        a.m.W_q_packed, a.m.scale, a.m.zero = o["packed"].data_ptr(), o["scale"].data_ptr(), o["zero"].data_ptr()
+        a.m.zero_meta = o["zero_meta"].data_ptr() if o.get("zero_meta") is not None else None
+        for k in SETTING_KEYS:
+            setattr(a, k, int(st[k]))
+    need = hqq_stream_jobs_device_bytes(arr, n)
+    if need == 0:
+        raise HQQError(HQQ_ERR_INVALID_ARG, "hqq_stream_jobs_device_bytes")
+    if device_buffer is None or device_buffer.numel() < need:
+        device_buffer = torch.empty(need, dtype=torch.uint8, device="cuda")
+    errors = []
+
+    def report(i, _user):
+        try:
+            if on_done is not None:
+                on_done(i)
+        except BaseException as e:  # a ctypes callback cannot raise into C: keep it for after the call
+            errors.append(e)
+
+    cb = hqq_stream_done_fn(report)
+    done = C.c_int(0)
+    rc = hqq_quantize_stream_jobs(arr, n, _DT[dt], p, beta, kappa, iters, device_buffer, device_buffer.numel(), cb,
+                                  None, C.byref(done), stream)
+    if errors:
+        raise errors[0]
+    if rc != HQQ_OK:
+        raise HQQError(rc, f"hqq_quantize_stream_jobs ({done.value} of {n} matrices completed)")
+    return device_buffer, done.value
 
 
 def gemv(q, x, rows, cols, nbits, group_size, zero_nbits=16, out=None, stream=None):

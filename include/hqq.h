@@ -204,7 +204,8 @@ size_t hqq_stream_device_bytes(const hqq_host_matrix* mats, int n, int nbits, in
                                int stop_mode, int zero_nbits);
 
 /*
- * hqq_quantize_stream -- hqq_quantize on each of the n matrices, with the
+ * hqq_quantize_stream -- hqq_quantize on each of the n matrices (the same
+ * settings for all; hqq_quantize_stream_jobs below takes them per matrix), with the
  * copy of matrix i+1 to the GPU and of matrix i-1's outputs back to the host
  * overlapping the solver on matrix i (two device slots; copies on two
  * streams the call creates; the solver on `stream`).  Solver arguments as in
@@ -216,6 +217,52 @@ size_t hqq_stream_device_bytes(const hqq_host_matrix* mats, int n, int nbits, in
 int hqq_quantize_stream(const hqq_host_matrix* mats, int n, int dtype, int nbits, int group_size, int axis, float p,
                         float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* device_buffer,
                         size_t device_bytes, void* stream);
+
+/*
+ * Per-matrix settings for a streamed model: attention and MLP layers at
+ * different bit widths and group sizes ("HQQ - Half-Quadratic Quantization"
+ * (skill4agent.com), section "Mixed precision quantization": attention 4-bit
+ * g64, MLP 2-bit g32), quantised layer by layer (same page, section "Common
+ * issues", out of memory during quantization).
+ *   m            the matrix and its host outputs, as for hqq_quantize_stream
+ *                (zero_meta needed when zero_nbits == 8).
+ *   nbits, group_size, axis, stop_mode, zero_nbits: as in hqq_quantize, for
+ *                this matrix only.
+ */
+typedef struct hqq_stream_job {
+    hqq_host_matrix m;
+    int nbits, group_size, axis, stop_mode, zero_nbits;
+} hqq_stream_job;
+
+/* Called by hqq_quantize_stream_jobs on the calling thread, once per job and
+ * in job order, as soon as the outputs of job `index` are complete in host
+ * memory (e.g. to write them to disk while later jobs run).  It may not free
+ * or reuse the job's host buffers before the call returns. */
+typedef void (*hqq_stream_done_fn)(int index, void* user);
+
+/* Device bytes hqq_quantize_stream_jobs needs: two slots, each buffer kind
+ * (W, codes, scale, zero, workspace) sized for the largest job.  0 on invalid
+ * arguments (n < 1, a bad job setting or shape). */
+size_t hqq_stream_jobs_device_bytes(const hqq_stream_job* jobs, int n);
+
+/*
+ * hqq_quantize_stream_jobs -- hqq_quantize_stream with settings per matrix,
+ * and completion reporting for resumable runs.  p, beta, kappa, iters and the
+ * input dtype are the same for every job.  Every job's settings and pointers
+ * are checked before anything is copied or launched (an invalid job returns
+ * its hqq_quantize status and touches nothing).  on_done (may be NULL) is
+ * called for each finished job, in order, with `user`.  jobs_done (may be
+ * NULL) receives the number of leading jobs whose outputs are complete in
+ * host memory when the call returns: n on success.  A caller that persists
+ * each job in on_done resumes an interrupted run by passing the jobs not yet
+ * persisted.  device_buffer: device memory of at least
+ * hqq_stream_jobs_device_bytes(jobs, n), 256-byte aligned, caller-owned.
+ * Blocks until every output is in host memory.  Returns HQQ_OK or the first
+ * error (HQQ_ERR_WORKSPACE if device_bytes is too small).
+ */
+int hqq_quantize_stream_jobs(const hqq_stream_job* jobs, int n, int dtype, float p, float beta, float kappa, int iters,
+                             void* device_buffer, size_t device_bytes, hqq_stream_done_fn on_done, void* user,
+                             int* jobs_done, void* stream);
 
 /*
  * hqq_gemv -- fused dequantisation + matrix-vector product of the packed

@@ -131,6 +131,82 @@ def test_stream_size_query_and_rejections(hq):
         hq.HQQ_ERR_INVALID_ARG
 
 
+def _jobs(hq, specs):
+    arr = (hq.hqq_stream_job * len(specs))()
+    for a, (r, c, nb, g, axis, stop, zb) in zip(arr, specs):
+        a.m.rows, a.m.cols = r, c
+        a.nbits, a.group_size, a.axis, a.stop_mode, a.zero_nbits = nb, g, axis, stop, zb
+    return arr
+
+
+def test_stream_jobs_size_query(hq):
+    """Two slots, each buffer kind sized for the largest job (256-byte parts)."""
+    specs = [(5120, 5120, 4, 64, 1, 1, 16), (13824, 5120, 2, 32, 1, 1, 16), (5120, 13824, 2, 32, 1, 1, 16),
+             (1024, 8192, 8, 128, 0, 0, 8)]
+    arr = _jobs(hq, specs)
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    mx = dict(W=0, packed=0, scale=0, zero=0, ws=0)
+    for r, c, nb, g, axis, stop, zb in specs:
+        G = hq.hqq_num_groups(r, c, g, axis)
+        mx["W"] = max(mx["W"], 2 * r * c)
+        mx["packed"] = max(mx["packed"], hq.hqq_packed_bytes(r, c, nb, g, axis))
+        mx["scale"] = max(mx["scale"], 2 * G)
+        mx["zero"] = max(mx["zero"], G * (2 if zb == 16 else 1))
+        mx["ws"] = max(mx["ws"], hq.hqq_workspace_bytes(r, c, g, axis, stop, zb))
+    slot = up(mx["W"]) + up(mx["packed"]) + up(mx["scale"]) + up(mx["zero"]) + up(8) + up(mx["ws"])
+    assert hq.hqq_stream_jobs_device_bytes(arr, 4) == 2 * slot
+    # the uniform-settings query is the same computation
+    mats = (hq.hqq_host_matrix * 1)()
+    mats[0].rows, mats[0].cols = 5120, 5120
+    assert hq.hqq_stream_device_bytes(mats, 1, 4, 64, 1, 1, 16) == hq.hqq_stream_jobs_device_bytes(arr, 1)
+    assert hq.hqq_stream_jobs_device_bytes(arr, 0) == 0
+    assert hq.hqq_stream_jobs_device_bytes(None, 1) == 0
+
+
+@pytest.mark.parametrize("bad,status", [((4096, 1024, 5, 64, 1, 0, 16), "HQQ_ERR_INVALID_ARG"),
+                                        ((4096, 1000, 4, 64, 1, 0, 16), "HQQ_ERR_SHAPE"),
+                                        ((4096, 1024, 4, 48, 1, 0, 16), "HQQ_ERR_SHAPE"),
+                                        ((4096, 1024, 4, 64, 2, 0, 16), "HQQ_ERR_INVALID_ARG"),
+                                        ((4096, 1024, 4, 64, 1, 3, 16), "HQQ_ERR_INVALID_ARG"),
+                                        ((4096, 1024, 4, 64, 1, 0, 4), "HQQ_ERR_INVALID_ARG")])
+def test_stream_jobs_rejects_a_bad_job_before_anything_runs(hq, bad, status):
+    """One bad job anywhere in the list: its hqq_quantize status, no copy,
+    no launch, no callback, zero jobs done (checked on a box with no GPU)."""
+    good = (1024, 1024, 4, 64, 1, 0, 16)
+    arr = _jobs(hq, [good, bad, good])
+    assert hq.hqq_stream_jobs_device_bytes(arr, 3) == 0
+    calls = []
+    cb = hq.hqq_stream_done_fn(lambda i, u: calls.append(i))
+    done = C.c_int(-1)
+    rc = hq.lib.hqq_quantize_stream_jobs(arr, 3, 0, 0.7, 1.0, 1.01, 20, None, 0, cb, None, C.byref(done), None)
+    assert rc == getattr(hq, status) and calls == [] and done.value == 0
+    # the call's own solver parameters are checked the same way
+    arr = _jobs(hq, [good])
+    assert hq.lib.hqq_quantize_stream_jobs(arr, 1, 0, 2.5, 1.0, 1.01, 20, None, 0, cb, None, None, None) == \
+        hq.HQQ_ERR_INVALID_ARG
+    assert hq.lib.hqq_quantize_stream_jobs(arr, 1, 9, 0.7, 1.0, 1.01, 20, None, 0, cb, None, None, None) == \
+        hq.HQQ_ERR_DTYPE
+    # host buffers missing, then no device buffer
+    assert hq.lib.hqq_quantize_stream_jobs(arr, 1, 0, 0.7, 1.0, 1.01, 20, None, 0, cb, None, None, None) == \
+        hq.HQQ_ERR_INVALID_ARG
+    assert hq.lib.hqq_quantize_stream_jobs(arr, 0, 0, 0.7, 1.0, 1.01, 20, None, 0, cb, None, None, None) == \
+        hq.HQQ_OK
+
+
+def test_settings_for_per_layer_types(hq):
+    """A per-layer-type config: attention 4-bit g64, MLP 2-bit g32 tensor stop."""
+    base = dict(nbits=4, group_size=64)
+    dyn = {"attn": dict(nbits=4, group_size=64), "mlp": dict(nbits=2, group_size=32, stop_mode=1)}
+    a = hq.settings_for("model.layers.7.self_attn.o_proj", base, dyn)
+    m = hq.settings_for("model.layers.7.mlp.down_proj", base, dyn)
+    o = hq.settings_for("lm_head", dict(base, zero_nbits=8), dyn)
+    assert a == dict(nbits=4, group_size=64, axis=1, stop_mode=0, zero_nbits=16)
+    assert m == dict(nbits=2, group_size=32, axis=1, stop_mode=1, zero_nbits=16)
+    assert o == dict(nbits=4, group_size=64, axis=1, stop_mode=0, zero_nbits=8)
+    with pytest.raises(hq.HQQError):
+        hq.settings_for("x.mlp", base, {"mlp": dict(bits=2)})
+
+
 def test_status_strings(hq):
     for code in range(9):
         s = hq.hqq_status_string(code)

@@ -65,3 +65,93 @@ def test_stream_rejects_small_buffer(hq):
     assert rc == hq.HQQ_ERR_WORKSPACE
     rc = hq.hqq_quantize_stream(arr, 1, hq.HQQ_F16, 4, 64, 1, 0.7, 1.0, 1.01, 20, 0, 16, buf, need)
     assert rc == hq.HQQ_OK
+
+
+MIXED = [  # (rows, cols, settings): per-layer-type configs, both axes, all stop modes, both zero widths
+    (1024, 1024, dict(nbits=4, group_size=64, axis=1, stop_mode=0, zero_nbits=16)),
+    (2048, 1024, dict(nbits=2, group_size=32, axis=1, stop_mode=1, zero_nbits=16)),
+    (1024, 2048, dict(nbits=2, group_size=32, axis=1, stop_mode=1, zero_nbits=8)),
+    (512, 768, dict(nbits=3, group_size=64, axis=0, stop_mode=0, zero_nbits=8)),
+    (4096, 512, dict(nbits=8, group_size=128, axis=1, stop_mode=2, zero_nbits=16)),
+    (256, 4096, dict(nbits=1, group_size=16, axis=1, stop_mode=1, zero_nbits=8)),
+    (768, 1024, dict(nbits=4, group_size=64, axis=1, stop_mode=0, zero_nbits=16)),
+]
+
+
+def _mixed(hq, dtype=torch.float16, pin=True):
+    Ws = [synth.weight(r, c, seed=31 * i + 5, dtype=dtype) for i, (r, c, _) in enumerate(MIXED)]
+    if pin:
+        Ws = [w.pin_memory() for w in Ws]
+    sets = [st for _, _, st in MIXED]
+    outs = [hq.host_outputs(r, c, st["nbits"], st["group_size"], st["axis"], st["zero_nbits"], pin=pin)
+            for r, c, st in MIXED]
+    return Ws, sets, outs
+
+
+def _expect(hq, w, st):
+    ref = hq.quantize(w.cuda(), st["nbits"], st["group_size"], st["axis"], stop_mode=st["stop_mode"],
+                      zero_nbits=st["zero_nbits"])
+    torch.cuda.synchronize()
+    return ref
+
+
+def _same(o, ref):
+    for k in ("packed", "scale", "zero", "zero_meta"):
+        if o.get(k) is None:
+            continue
+        assert np.array_equal(o[k].numpy().view(np.uint8), ref[k].cpu().numpy().view(np.uint8)), k
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_stream_jobs_per_matrix_settings(hq, dtype):
+    """Every matrix with its own settings: each output equals hqq_quantize
+    with those settings on the device-resident matrix, bit for bit; the done
+    callback comes once per matrix, in order, when that matrix's host outputs
+    are already complete."""
+    Ws, sets, outs = _mixed(hq, dtype)
+    refs = [_expect(hq, w, st) for w, st in zip(Ws, sets)]
+    seen = []
+
+    def on_done(i):
+        _same(outs[i], refs[i])  # complete when reported
+        seen.append(i)
+
+    _, done = hq.quantize_stream_jobs(Ws, sets, outs, on_done=on_done)
+    assert seen == list(range(len(MIXED))) and done == len(MIXED)
+    for o, ref in zip(outs, refs):
+        _same(o, ref)
+
+
+def test_stream_jobs_resume(hq):
+    """A run resumed from the first matrix not yet persisted (a new call with
+    the remaining matrices) gives the same outputs as one uninterrupted run
+    (pageable host memory here)."""
+    Ws, sets, outs = _mixed(hq, torch.bfloat16, pin=False)
+    _, done = hq.quantize_stream_jobs(Ws, sets, outs)
+    assert done == len(MIXED)
+    outs2 = [hq.host_outputs(r, c, st["nbits"], st["group_size"], st["axis"], st["zero_nbits"], pin=False)
+             for r, c, st in MIXED]
+    buf, done = hq.quantize_stream_jobs(Ws[:3], sets[:3], outs2[:3])
+    assert done == 3
+    _, done = hq.quantize_stream_jobs(Ws[3:], sets[3:], outs2[3:], device_buffer=buf)
+    assert done == len(MIXED) - 3
+    for a, b in zip(outs, outs2):
+        _same(a, b)
+
+
+def test_stream_jobs_callback_error_surfaces_after_the_call(hq):
+    """An exception in on_done cannot unwind through the C call: every matrix
+    is still reported and finished, and the first exception is raised after."""
+    Ws, sets, outs = _mixed(hq)
+    seen = []
+
+    def on_done(i):
+        seen.append(i)
+        if i == 2:
+            raise KeyError("persist failed")
+
+    with pytest.raises(KeyError):
+        hq.quantize_stream_jobs(Ws, sets, outs, on_done=on_done)
+    assert seen == list(range(len(MIXED)))
+    for w, st, o in zip(Ws, sets, outs):
+        _same(o, _expect(hq, w, st))
