@@ -43,6 +43,8 @@ def _bind(L):
     L.oracle_dequantize_s8.argtypes = [P, P, P, i32, P, P, i64, i64, i32, i32, i32, i32, i32, P]
     L.oracle_gemv.restype = i32
     L.oracle_gemv.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, i32, i32, P]
+    L.oracle_gemm.restype = i32
+    L.oracle_gemm.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, i32, i32, P, P]
     L.oracle_quantize_scale8.restype = i32
     L.oracle_quantize_scale8.argtypes = [P, i64, i32, P, P]
     L.oracle_trace_group.restype = i32
@@ -157,6 +159,23 @@ def gemv(packed, scale, zero, zero_meta, rows, cols, nbits, group_size, zero_nbi
     if rc != 0:
         raise ValueError(f"oracle_gemv failed with code {rc}")
     return y
+
+
+def gemm(packed, scale, zero, zero_meta, rows, cols, nbits, group_size, zero_nbits, x, x_dtype=F16, L=None):
+    """(y, yabs): y[b] = round16(W_r) @ x[b] in fp64, W_r = (W_q - zero) * scale in
+    fp32 rounded to x's 16-bit type (axis 1); yabs[b][r] = sum |w16 * x|.
+    x: [batch, cols] float16 array (x_dtype F16) or uint16 bf16 bits (BF16)."""
+    L = L or lib()
+    x = np.ascontiguousarray(x)
+    x2 = x.reshape(-1, cols)
+    y = np.zeros((x2.shape[0], rows), np.float64)
+    yabs = np.zeros((x2.shape[0], rows), np.float64)
+    rc = L.oracle_gemm(_p(np.ascontiguousarray(packed)), _p(np.ascontiguousarray(scale)),
+                       _p(np.ascontiguousarray(zero)), _p(zero_meta), rows, cols, nbits, group_size, zero_nbits,
+                       _p(x2.view(np.uint16)), x_dtype, x2.shape[0], _p(y), _p(yabs))
+    if rc != 0:
+        raise ValueError(f"oracle_gemm failed with code {rc}")
+    return y, yabs
 
 
 def shrink(x, p, beta, L=None):

@@ -27,7 +27,7 @@
  * and the solver keeps the best zero-point seen, stopping once the lp error
  * stops falling.
  *
- * Readings of points the pages leave open (each also listed in the design doc):
+ * Readings of points the pages leave open:
  *   R1  s = min(L / (max - min), 2e4) when max > min, else 2e4.
  *   R2  round() is round-half-to-even (nearbyintf, default rounding mode).
  *   R3  the lp error of a zero-point is mean(|W - W_r|^p) with the same p.
@@ -518,6 +518,45 @@ int oracle_gemv(const uint8_t *W_q_packed, const uint16_t *scale, const void *ze
             else z = ((float)((const uint8_t *)zero)[j] - zero_meta[1]) * zero_meta[0];
             const float w = (q - z) * from_f16(scale[j]);
             for (int b = 0; b < batch; ++b) y[b * rows + r] += (double)w * (double)load_elem(x + b * cols, x_dtype, c);
+        }
+    }
+    return 0;
+}
+
+/*
+ * The same product as a tensor-core backend forms it (the consumer of the
+ * packed layout: "HQQ - Half-Quadratic Quantization" (skill4agent.com),
+ * section "Backends"): W_r rebuilt per element exactly as in
+ * oracle_gemv (fp32), then rounded to the activations' 16-bit type (x_dtype;
+ * round to nearest, ties to even) because both operands of a 16-bit
+ * tensor-core product share one type; every product and sum in fp64.
+ * yabs[b][r] receives the sum of |w16 * x| over the row (the scale of a
+ * bound on fp32 accumulation error).  Groups along the input dimension.
+ */
+int oracle_gemm(const uint8_t *W_q_packed, const uint16_t *scale, const void *zero, const float *zero_meta,
+                int64_t rows, int64_t cols, int nbits, int group_size, int zero_nbits, const uint16_t *x,
+                int x_dtype, int batch, double *y, double *yabs)
+{
+    if (!valid_args(rows, cols, x_dtype, nbits, group_size, 1, 0, zero_nbits) || batch < 1) return 1;
+    const int g = group_size;
+    for (int64_t i = 0; i < (int64_t)batch * rows; ++i) {
+        y[i] = 0.0;
+        yabs[i] = 0.0;
+    }
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t c = 0; c < cols; ++c) {
+            const int64_t grp = (r * cols + c) / g;
+            const float q = (float)unpack_elem(W_q_packed, r, c, cols, nbits, 1);
+            float z;
+            if (zero_nbits == 16) z = from_f16(((const uint16_t *)zero)[grp]);
+            else z = ((float)((const uint8_t *)zero)[grp] - zero_meta[1]) * zero_meta[0];
+            const float wr = (q - z) * from_f16(scale[grp]);
+            const double w16 = x_dtype == ORACLE_BF16 ? (double)from_bf16(to_bf16(wr)) : (double)from_f16(to_f16(wr));
+            for (int b = 0; b < batch; ++b) {
+                const double p = w16 * (double)load_elem(x + b * cols, x_dtype, c);
+                y[b * rows + r] += p;
+                yabs[b * rows + r] += fabs(p);
+            }
         }
     }
     return 0;

@@ -50,6 +50,15 @@ MUTANTS = [
     ("gemv-group-index", "const int64_t j = (r * cols + c) / g;", "const int64_t j = (r * cols + c) / (2 * g);", 1),
     ("gemv-skips-last-column", "        for (int64_t c = 0; c < cols; ++c) {\n            const int64_t j = (r * cols + c) / g;",
      "        for (int64_t c = 0; c < cols - 1; ++c) {\n            const int64_t j = (r * cols + c) / g;", 1),
+    ("gemm-no-16-bit-rounding",
+     "const double w16 = x_dtype == ORACLE_BF16 ? (double)from_bf16(to_bf16(wr)) : (double)from_f16(to_f16(wr));",
+     "const double w16 = (double)wr;", 1),
+    ("gemm-rounds-to-the-other-type",
+     "const double w16 = x_dtype == ORACLE_BF16 ? (double)from_bf16(to_bf16(wr)) : (double)from_f16(to_f16(wr));",
+     "const double w16 = x_dtype != ORACLE_BF16 ? (double)from_bf16(to_bf16(wr)) : (double)from_f16(to_f16(wr));", 1),
+    ("gemm-drops-zero", "const float wr = (q - z) * from_f16(scale[grp]);", "const float wr = q * from_f16(scale[grp]);",
+     1),
+    ("gemm-signed-abs-sum", "yabs[b * rows + r] += fabs(p);", "yabs[b * rows + r] += p;", 1),
     ("pack-msb-first", "unsigned v = level << off; /* at most 8 + 7 bits */",
      "unsigned v = (off + b <= 8 ? level << (8 - b - off) : level << off);", 1),
 ]

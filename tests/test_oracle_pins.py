@@ -599,3 +599,81 @@ def test_gemv_is_linear_and_batched(orc):
     assert np.array_equal(Y[0], y1) and np.array_equal(Y[1], y2) and np.array_equal(Y[2], y1)
     xb = (x1.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
     assert np.array_equal(orc.gemv(*args, xb, x_dtype=orc.BF16)[0], y1)
+
+
+# ------------------------------- tensor-core product (16-bit weights) ---
+
+def _golden(name):
+    d = {}
+    for line in open(os.path.join(GOLDEN, name)):
+        if line.startswith("#") or not line.strip():
+            continue
+        k, *v = line.split()
+        d[k] = v
+    return d
+
+
+def _bf16_bits(a):
+    """fp32 values exact in bf16 -> their bf16 bit patterns."""
+    u = np.asarray(a, np.float32).view(np.uint32)
+    assert np.all(u & 0xFFFF == 0)
+    return (u >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("xdt", ["bf16", "f16"])
+def test_gemm_hand_values(orc, xdt):
+    """Hand-worked values, including a tie that rounds to even in bf16."""
+    d = _golden("gemm_hand_values.txt")
+    rows, cols, nb, g = (int(d[k][0]) for k in ("rows", "cols", "nbits", "group"))
+    lv = np.array([int(v) for v in d["levels"]], np.uint8).reshape(rows, cols)
+    packed = np.zeros(rows * cols * nb // 8, np.uint8)
+    orc.lib().oracle_pack_levels(lv.ctypes.data, rows, cols, nb, 1, packed.ctypes.data)
+    sc = np.array([float(v) for v in d["scale"]], np.float16)
+    z = np.array([float(v) for v in d["zero"]], np.float16)
+    xf = np.array([float(v) for v in d["x"]], np.float32)
+    if xdt == "bf16":
+        y, ya = orc.gemm(packed, sc, z, None, rows, cols, nb, g, 16, _bf16_bits(xf), orc.BF16)
+    else:
+        y, ya = orc.gemm(packed, sc, z, None, rows, cols, nb, g, 16, xf.astype(np.float16), orc.F16)
+    assert y[0].tolist() == [float(v) for v in d["y_" + xdt]]
+    assert ya[0].tolist() == [float(v) for v in d["yabs_" + xdt]]
+
+
+@pytest.mark.parametrize("nbits,g,zb", [(4, 64, 16), (2, 16, 8), (3, 32, 16), (8, 128, 8)])
+def test_gemm_unit_vectors_give_dequantised_columns(orc, nbits, g, zb):
+    """x = e_c picks column c of W_r rounded to x's type: the dequantiser's
+    output in that type, for fp16 and bf16."""
+    W = _synth_f16(24, 256, seed=3 * nbits + g)
+    o = orc.quantize(W, nbits, g, 1, 0.7, 1.0, 1.01, 20, orc.STOP_GROUP, zb)
+    cols = [0, 1, g - 1, g, 255]
+    X = np.zeros((len(cols), 256), np.float32)
+    for i, c in enumerate(cols):
+        X[i, c] = 1.0
+    for dt, xs in ((orc.F16, X.astype(np.float16)), (orc.BF16, _bf16_bits(X))):
+        deq = orc.dequantize(o["packed"], o["scale"], o["zero"], o["zero_meta"], 24, 256, nbits, g, 1, zb,
+                             out_dtype=dt)
+        Y, Ya = orc.gemm(o["packed"], o["scale"], o["zero"], o["zero_meta"], 24, 256, nbits, g, zb, xs, dt)
+        for i, c in enumerate(cols):
+            col = deq[:, c].astype(np.float32) if dt == orc.F16 else \
+                (deq[:, c].astype(np.uint32) << 16).view(np.float32)
+            assert np.array_equal(Y[i], col.astype(np.float64))
+            assert np.array_equal(Ya[i], np.abs(col).astype(np.float64))
+
+
+def test_gemm_equals_gemv_when_weights_are_16_bit_exact(orc):
+    """Codes at 2 bit, zero a multiple of 2^-4 below 3, scale a power of two:
+    q - z has at most 6 significant bits, so every W_r is exact in bf16, the
+    rounding is the identity and the product is the fp32-weight product of
+    the matrix-vector oracle."""
+    r = np.random.default_rng(9)
+    rows, cols, nb, g = 16, 128, 2, 32
+    lv = r.integers(0, 4, (rows, cols)).astype(np.uint8)
+    packed = np.zeros(rows * cols * nb // 8, np.uint8)
+    orc.lib().oracle_pack_levels(lv.ctypes.data, rows, cols, nb, 1, packed.ctypes.data)
+    G = rows * cols // g
+    sc = (2.0 ** -r.integers(0, 5, G)).astype(np.float16)
+    z = (r.integers(0, 48, G) / 16).astype(np.float16)
+    x = (r.integers(-64, 64, (3, cols)) / 32).astype(np.float32)
+    y16, _ = orc.gemm(packed, sc, z, None, rows, cols, nb, g, 16, _bf16_bits(x), orc.BF16)
+    y32 = orc.gemv(packed, sc, z, None, rows, cols, nb, g, 16, _bf16_bits(x), orc.BF16)
+    assert np.array_equal(y16, y32)
