@@ -100,6 +100,16 @@ def peaks():
         return 6650.0, 1965.0, "fallback"
 
 
+def _measured_peaks():
+    """The measured peak figures (empty when the file is absent; the recipe's
+    fallback for the dense bf16 figure is 1590 TFLOP/s burst)."""
+    try:
+        with open(PEAKS_FILE) as f:
+            return json.load(f)
+    except Exception:
+        return {"bf16_tflops": 1590.0}
+
+
 def algorithmic_bytes(rows, cols, nbits, g, zero_nbits=16):
     """One read of W (2 B/weight) + packed codes + fp16 scale + zero."""
     n = rows * cols
@@ -518,6 +528,51 @@ def run_gemv_case(spec):
                       "gweights_s": rows * cols / (med / 1e3) / 1e9, "l2": "flushed before every call"}))
 
 
+def run_gemm_case(spec):
+    """Time hqq_gemm (fused dequantisation + tcgen05 matrix product) on one
+    quantised synthetic matrix with bf16 activations:
+    "gemm,rows,cols,nbits,g[,batch[,reps]]".  Reports TFLOP/s (2 rows cols
+    batch per call) against the measured bf16 GEMM peak, and the HBM view
+    (codes b/8 B + fp16 scale and 8-bit zero 3/g B per weight, activations,
+    outputs); L2 flushed before every call."""
+    from calibration_free_weight_b200 import hqq
+    v = [int(x) for x in spec.split(",")[1:]]
+    rows, cols, nbits, g = v[:4]
+    batch = v[4] if len(v) > 4 else 128
+    reps = v[5] if len(v) > 5 else 20
+    torch.cuda.set_device(0)
+    W = synth.weight(rows, cols, seed=7, dtype=torch.bfloat16).cuda()
+    q = hqq.quantize(W, nbits, g, zero_nbits=8)
+    del W
+    x = synth.weight(batch, cols, seed=8, dtype=torch.float32, std=1.0).to(torch.bfloat16).cuda()
+    y = torch.empty(batch, rows, dtype=torch.float32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    hqq.gemm(q, x, rows, cols, nbits, g, zero_nbits=8, out=y)
+    ev = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        hqq.gemm(q, x, rows, cols, nbits, g, zero_nbits=8, out=y)
+        b.record()
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    st = hqq.hqq_gemm_get_status()
+    if st != hqq.HQQ_OK:
+        raise RuntimeError(hqq.hqq_status_string(st))
+    ms = sorted(a.elapsed_time(b) for a, b in ev)
+    med = ms[len(ms) // 2]
+    G = rows * cols // g
+    nbytes = rows * cols * nbits // 8 + 2 * G + G + 8 + batch * cols * 2 + batch * rows * 4
+    flops = 2.0 * rows * cols * batch
+    hbm, _, kind = peaks()
+    tf = _measured_peaks().get("bf16_tflops")
+    print(json.dumps({"case": spec, "ms_median": med, "ms_min": ms[0], "tflops": flops / (med / 1e3) / 1e12,
+                      "bf16_peak_tflops": tf, "tensor_frac": (flops / (med / 1e3) / 1e12 / tf) if tf else None,
+                      "bytes": nbytes, "gbs": nbytes / (med / 1e3) / 1e9, "hbm_peak_gbs": hbm, "peak_kind": kind,
+                      "hbm_frac": nbytes / (med / 1e3) / 1e9 / hbm, "l2": "flushed before every call"}))
+
+
 def run_case(spec):
     """Time hqq_quantize on one synthetic bf16 matrix (used for kernel profiles)."""
     if spec.startswith("scale8"):
@@ -525,6 +580,9 @@ def run_case(spec):
         return
     if spec.startswith("gemv"):
         run_gemv_case(spec)
+        return
+    if spec.startswith("gemm"):
+        run_gemm_case(spec)
         return
     from calibration_free_weight_b200 import hqq
     v = [int(x) for x in spec.split(",")]

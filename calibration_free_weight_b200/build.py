@@ -10,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = [os.path.join(CSRC, f) for f in ("hqq_kernels.cu", "hqq_api.cu", "hqq_noalloc.cu", "hqq_stream.cu",
-                                                "hqq_gemv.cu")]
+                                                "hqq_gemv.cu", "hqq_gemm.cu")]
 HEADERS = [os.path.join(CSRC, "hqq_internal.h"), os.path.join(CSRC, "hqq_device.cuh"),
            os.path.join(os.path.dirname(HERE), "include", "hqq.h")]
 LIB = os.path.join(HERE, "libhqq_b200.so")

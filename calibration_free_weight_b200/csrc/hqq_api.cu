@@ -261,6 +261,46 @@ int hqq_gemv(const void* W_q_packed, const void* scale, const void* zero, const 
     return HQQ_OK;
 }
 
+int hqq_gemm(const void* W_q_packed, const void* scale, const void* zero, const void* zero_meta, int64_t rows,
+             int64_t cols, int nbits, int group_size, int zero_nbits, const void* x, int x_dtype, int batch, float* y,
+             void* stream) {
+    if (x_dtype != HQQ_F16 && x_dtype != HQQ_BF16) return HQQ_ERR_DTYPE;
+    if (!valid_nbits(nbits) || batch < 1 || batch > hqq::kGemmMaxBatch) return HQQ_ERR_INVALID_ARG;
+    const int sh = check_shape(rows, cols, group_size, 1);
+    if (sh != HQQ_OK) return sh;
+    if (cols % 64 != 0) return HQQ_ERR_SHAPE;
+    if (zero_nbits != 8 && zero_nbits != 16) return HQQ_ERR_INVALID_ARG;
+    if (rows * cols == 0) return HQQ_OK;
+    if (!is_device_ptr(W_q_packed) || !is_device_ptr(scale) || !is_device_ptr(zero) || !is_device_ptr(x) ||
+        !is_device_ptr(y))
+        return HQQ_ERR_INVALID_ARG;
+    if (zero_nbits == 8 && !is_device_ptr(zero_meta)) return HQQ_ERR_INVALID_ARG;
+    if (!aligned(W_q_packed, 16) || !aligned(scale, 2) || !aligned(x, 16) || !aligned(y, 4)) return HQQ_ERR_ALIGN;
+    if (zero_nbits == 16 && !aligned(zero, 2)) return HQQ_ERR_ALIGN;
+    if (zero_nbits == 8 && !aligned(zero_meta, 4)) return HQQ_ERR_ALIGN;
+    hqq::GemvArgs a{};
+    a.packed = static_cast<const uint8_t*>(W_q_packed);
+    a.scale = static_cast<const uint16_t*>(scale);
+    a.zero = zero;
+    a.zero_meta = static_cast<const float*>(zero_meta);
+    a.rows = rows;
+    a.cols = cols;
+    a.nbits = nbits;
+    a.g = group_size;
+    a.zero_nbits = zero_nbits;
+    a.x = x;
+    a.x_dtype = x_dtype;
+    a.batch = batch;
+    a.y = y;
+    if (hqq::launch_gemm(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return HQQ_ERR_CUDA;
+    }
+    return HQQ_OK;
+}
+
+int hqq_gemm_get_status(void* stream) { return hqq::gemm_take_status(static_cast<cudaStream_t>(stream)); }
+
 int hqq_quantize_scale8(const void* scale, int64_t num_groups, int scale_group, void* scale_q, void* scale_meta,
                         void* stream) {
     if (num_groups < 0 || scale_group < 1) return HQQ_ERR_INVALID_ARG;
@@ -296,7 +336,7 @@ const char* hqq_status_string(int status) {
         case HQQ_ERR_DTYPE: return "unsupported dtype";
         case HQQ_ERR_ALIGN: return "misaligned buffer";
         case HQQ_ERR_CUDA: return "CUDA runtime error";
-        case HQQ_ERR_TIMEOUT: return "device wait timed out (reserved; not produced)";
+        case HQQ_ERR_TIMEOUT: return "a bounded device wait gave up";
         case HQQ_ERR_COOP_UNSUPPORTED: return "cooperative launch unsupported (reserved; not produced)";
         case HQQ_ERR_WORKSPACE: return "workspace missing or too small";
         default: return "unknown status";

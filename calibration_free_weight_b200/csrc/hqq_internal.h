@@ -11,6 +11,7 @@ namespace hqq {
 constexpr int kPiece = 8;            // elements per 16-byte piece of 16-bit data
 constexpr int kMaxPartials = 4096;   // per-CTA partial slots in the workspace (tensor mode)
 constexpr int64_t kMinSlice = 4096;  // smallest group-mode slice (entries) a workspace may be cut into
+constexpr int kGemmMaxBatch = 65536;  // batch bound of hqq_gemm (argument check)
 constexpr int kMaxIters = 1000;      // upper bound on iters (argument check)
 constexpr float kScaleCap = 2.0e4f;  // cap on s (and on the 8-bit zero quantiser's scale)
 
@@ -84,6 +85,12 @@ struct GemvArgs {
     float* y;       // [batch][rows]
 };
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t stream);
+// The tensor-core product (batch >= 1, cols a multiple of 64, x 16-byte aligned).
+cudaError_t launch_gemm(const GemvArgs& a, cudaStream_t stream);
+// Batch tiles of launch_gemm: ntiles tiles of ntile (a multiple of 16, <= 256) rows.
+void gemm_tiles(int batch, int* ntile, int* ntiles);
+// Synchronises the stream; 0, 6 (a wait of a product gave up; cleared) or 5 (CUDA error).
+int gemm_take_status(cudaStream_t stream);
 
 // Launchers: return cudaSuccess or the launch error.
 cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream);

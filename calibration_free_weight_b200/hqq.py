@@ -20,7 +20,7 @@ HQQ_STOP_GROUP, HQQ_STOP_TENSOR, HQQ_STOP_NONE = 0, 1, 2
 EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_quantize", "hqq_dequantize",
             "hqq_get_status", "hqq_status_string", "hqq_quantize_noalloc", "hqq_quantize_scale8",
             "hqq_dequantize_s8", "hqq_stream_device_bytes", "hqq_quantize_stream", "hqq_gemv",
-            "hqq_stream_jobs_device_bytes", "hqq_quantize_stream_jobs")
+            "hqq_stream_jobs_device_bytes", "hqq_quantize_stream_jobs", "hqq_gemm", "hqq_gemm_get_status")
 
 
 class hqq_host_matrix(C.Structure):
@@ -66,6 +66,10 @@ def _load():
     L.hqq_dequantize_s8.argtypes = [P, P, P, i32, P, P, i64, i64, i32, i32, i32, i32, i32, P, P]
     L.hqq_gemv.restype = i32
     L.hqq_gemv.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, i32, i32, P, P]
+    L.hqq_gemm.restype = i32
+    L.hqq_gemm.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, i32, i32, P, P]
+    L.hqq_gemm_get_status.restype = i32
+    L.hqq_gemm_get_status.argtypes = [P]
     HM = C.POINTER(hqq_host_matrix)
     L.hqq_stream_device_bytes.restype = sz
     L.hqq_stream_device_bytes.argtypes = [HM, i32, i32, i32, i32, i32, i32]
@@ -165,6 +169,16 @@ def hqq_quantize_stream(mats, n, dtype, nbits, group_size, axis, p, beta, kappa,
                         device_buffer, device_bytes, stream=None):
     return lib.hqq_quantize_stream(mats, n, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
                                    zero_nbits, _ptr(device_buffer), device_bytes, _stream(stream))
+
+
+def hqq_gemm(W_q_packed, scale, zero, zero_meta, rows, cols, nbits, group_size, zero_nbits, x, x_dtype, batch, y,
+             stream=None):
+    return lib.hqq_gemm(_ptr(W_q_packed), _ptr(scale), _ptr(zero), _ptr(zero_meta), rows, cols, nbits, group_size,
+                        zero_nbits, _ptr(x), x_dtype, batch, _ptr(y), _stream(stream))
+
+
+def hqq_gemm_get_status(stream=None):
+    return lib.hqq_gemm_get_status(_stream(stream))
 
 
 def hqq_stream_jobs_device_bytes(jobs, n):
@@ -272,6 +286,21 @@ def quantize_stream(Ws, outs, nbits=4, group_size=64, axis=1, p=0.7, beta=1.0, k
     if rc != HQQ_OK:
         raise HQQError(rc, "hqq_quantize_stream")
     return device_buffer
+
+
+def gemm(q, x, rows, cols, nbits, group_size, zero_nbits=16, out=None, stream=None):
+    """y = round16(dequant(W)) @ x.T on the tensor cores for the outputs of
+    quantize() (axis 1, cols a multiple of 64) and a CUDA [batch, cols]
+    fp16/bf16 tensor x; returns fp32 [batch, rows]."""
+    if x.dtype not in _DT or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
+        raise HQQError(HQQ_ERR_INVALID_ARG, "gemm expects a contiguous 2-D CUDA fp16/bf16 x")
+    if out is None:
+        out = torch.empty(x.shape[0], rows, dtype=torch.float32, device=x.device)
+    rc = hqq_gemm(q["packed"], q["scale"], q["zero"], q.get("zero_meta"), rows, cols, nbits, group_size, zero_nbits,
+                  x, _DT[x.dtype], x.shape[0], out, stream)
+    if rc != HQQ_OK:
+        raise HQQError(rc, "hqq_gemm")
+    return out
 
 
 SETTING_KEYS = ("nbits", "group_size", "axis", "stop_mode", "zero_nbits")

@@ -76,7 +76,7 @@ typedef enum {
     HQQ_ERR_DTYPE = 3,            /* dtype not HQQ_F16 / HQQ_BF16 */
     HQQ_ERR_ALIGN = 4,            /* a buffer is not aligned as documented */
     HQQ_ERR_CUDA = 5,             /* a CUDA runtime call failed (launch, attribute query) */
-    HQQ_ERR_TIMEOUT = 6,          /* reserved: no kernel of this library waits on another */
+    HQQ_ERR_TIMEOUT = 6,          /* a bounded wait inside hqq_gemm gave up (hqq_gemm_get_status) */
     HQQ_ERR_COOP_UNSUPPORTED = 7, /* reserved: no cooperative launch is used */
     HQQ_ERR_WORKSPACE = 8         /* workspace missing or smaller than hqq_workspace_bytes() */
 } hqq_status;
@@ -284,6 +284,37 @@ int hqq_quantize_stream_jobs(const hqq_stream_job* jobs, int n, int dtype, float
 int hqq_gemv(const void* W_q_packed, const void* scale, const void* zero, const void* zero_meta, int64_t rows,
              int64_t cols, int nbits, int group_size, int zero_nbits, const void* x, int x_dtype, int batch, float* y,
              void* stream);
+
+/*
+ * hqq_gemm -- fused dequantisation + matrix product on the tensor cores
+ * (tcgen05) for batches of activation vectors, the product a 16-bit
+ * tensor-core backend computes with the packed layout ("HQQ - Half-Quadratic
+ * Quantization" (skill4agent.com), section "Backends"; dequantisation rule
+ * W_r = (W_q - z) * scale of techreport.ngo, "Weight-only quantization
+ * without the calibration tax", section "Outlier-aware optimization without
+ * gradients"):
+ *   y[b][r] = sum_c round16(W_r[r][c]) * x[b][c],  1 <= batch <= 65536,
+ * with W_r formed in fp32 exactly as hqq_dequantize does, then rounded to the
+ * activations' type (x_dtype; round to nearest even: both operands of one
+ * 16-bit tensor-core product share a type), products exact and sums in fp32
+ * (accumulated in tensor memory, order unspecified: |error| <= cols * 2^-23 *
+ * sum_c |round16(W_r) x|).  Groups along the input dimension (axis 1 of an
+ * [out, in] = [rows, cols] weight); cols must be a multiple of 64.
+ * W_q_packed, scale, zero, zero_meta as produced by hqq_quantize.  x: device
+ * [batch][cols] fp16/bf16, 16-byte aligned; y: device fp32 [batch][rows],
+ * 4-byte aligned.  Returns HQQ_OK, HQQ_ERR_DTYPE, HQQ_ERR_SHAPE,
+ * HQQ_ERR_INVALID_ARG (batch out of range, bad pointer), HQQ_ERR_ALIGN or
+ * HQQ_ERR_CUDA.  Allocates nothing.  Every wait inside the kernel is bounded
+ * (about 1 s); a wait that gives up is reported by hqq_gemm_get_status.
+ */
+int hqq_gemm(const void* W_q_packed, const void* scale, const void* zero, const void* zero_meta, int64_t rows,
+             int64_t cols, int nbits, int group_size, int zero_nbits, const void* x, int x_dtype, int batch, float* y,
+             void* stream);
+
+/* Synchronises `stream`; HQQ_OK, or HQQ_ERR_TIMEOUT if a hqq_gemm since the
+ * last call gave up a wait (its y is then incomplete; the flag is cleared),
+ * or HQQ_ERR_CUDA. */
+int hqq_gemm_get_status(void* stream);
 
 /* Synchronise `stream` and return the device status word held in `workspace`
  * by the last hqq_quantize on it (HQQ_OK), or HQQ_ERR_CUDA if the

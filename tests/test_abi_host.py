@@ -207,6 +207,23 @@ def test_settings_for_per_layer_types(hq):
         hq.settings_for("x.mlp", base, {"mlp": dict(bits=2)})
 
 
+def test_gemm_rejections(hq):
+    """hqq_gemm argument checks, all on the host before any launch."""
+    L = hq.lib
+    a = (None, None, None, None)
+    assert L.hqq_gemm(*a, 128, 128, 4, 64, 16, None, 7, 4, None, None) == hq.HQQ_ERR_DTYPE
+    assert L.hqq_gemm(*a, 128, 128, 5, 64, 16, None, 1, 4, None, None) == hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_gemm(*a, 128, 128, 4, 64, 16, None, 1, 0, None, None) == hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_gemm(*a, 128, 128, 4, 64, 16, None, 1, 65537, None, None) == hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_gemm(*a, 128, 96, 4, 32, 16, None, 1, 4, None, None) == hq.HQQ_ERR_SHAPE  # cols % 64
+    assert L.hqq_gemm(*a, 128, 128, 4, 48, 16, None, 1, 4, None, None) == hq.HQQ_ERR_SHAPE
+    assert L.hqq_gemm(*a, 128, 128, 4, 64, 12, None, 1, 4, None, None) == hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_gemm(*a, 0, 128, 4, 64, 16, None, 1, 4, None, None) == hq.HQQ_OK
+    buf = C.create_string_buffer(4096)
+    p = C.cast(buf, C.c_void_p).value
+    assert L.hqq_gemm(p, p, p, None, 128, 128, 4, 64, 16, p, 1, 4, p, None) == hq.HQQ_ERR_INVALID_ARG
+
+
 def test_status_strings(hq):
     for code in range(9):
         s = hq.hqq_status_string(code)
