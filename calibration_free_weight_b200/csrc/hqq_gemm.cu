@@ -12,16 +12,19 @@
 // One CTA computes a 128-row x N tile of y^T (N = the batch tile, a multiple
 // of 16 up to 256): A = W_r[128 rows][K] and B = x[N][K], both K-major, so the
 // weight side fills the MMA's M = 128 and the (small) batch is the MMA's N.
-// K is walked in 64-element tiles through a ring of kStages shared-memory
+// K is walked in 64-element tiles through a ring of S shared-memory
 // stages, each in the canonical 128-byte-swizzled K-major layout (row r of a
 // tile at r * 128 bytes, its 16-byte chunk c at chunk c ^ (r % 8)):
-//   * every thread dequantises 32 weights of the A tile (codes prefetched in
-//     registers one tile ahead) and stores them as 16-bit values;
-//   * the x tile arrives by cp.async, issued one tile ahead (rows past the
-//     batch are zero-filled);
+//   * every thread dequantises 32 weights of the A tile (codes, scales and
+//     zeros prefetched in registers three tiles ahead) and stores them as
+//     16-bit values;
+//   * the x tile arrives by a 2-D tensor copy (TMA, 128-byte swizzle, from
+//     this GPU's own memory, no multicast) issued by thread 0 two tiles ahead
+//     and completing on the stage's "x full" mbarrier; rows past the batch are
+//     zero-filled by the copy;
 //   * thread 0 issues four tcgen05.mma (K = 16 each) into the fp32 accumulator
 //     in tensor memory and commits them to the stage's mbarrier, which frees
-//     the stage for the tile kStages later.
+//     the stage for the tile S later.
 // The epilogue reads the accumulator with tcgen05.ld (warp w reads the 32 rows
 // of its lane quarter w % 4, half of the columns) and stores y.
 //
@@ -29,9 +32,11 @@
 // timeout in a device status word (read by hqq_gemm_get_status) and makes the
 // whole CTA skip to the release of its tensor memory; no wait can hang.
 
+#include <cuda.h>  // CUtensorMap and its enums (the encoder is fetched at run time; no driver library link)
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 
@@ -42,7 +47,8 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kTileM = 128;          // MMA M: weight rows per CTA
 constexpr int kTileK = 64;           // elements per K tile: one 128-byte swizzle row of 16-bit values
-constexpr int kStages = 4;           // shared-memory ring
+constexpr int kMaxStages = 8;        // shared-memory ring: as many stages as fit (4 at N = 256, 8 at N <= 48)
+constexpr size_t kSmemBudget = 227 * 1024;
 constexpr int kStageA = kTileM * 128;  // bytes of one A stage
 constexpr unsigned long long kWaitNs = 1000000000ull;
 
@@ -85,13 +91,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     return true;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+
+// 2-D tiled tensor copy global -> shared (box of the tensor map at {x0, y0}),
+// completing on `bar` by transaction bytes.  x0 * 2 bytes is a multiple of 16.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x0, int y0, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x0), "r"(y0), "r"(bar)
+        : "memory");
 }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -152,6 +162,7 @@ struct GemmParams {
     int g_log;          // log2(group size)
     int batch;
     int ntile;          // MMA N: batch rows per CTA, a multiple of 16 in [16, 256]
+    int stages;         // S, in [3, kMaxStages]
 };
 
 // Inputs of one thread's 32 consecutive weights of one K tile (one row):
@@ -224,12 +235,6 @@ __device__ __forceinline__ uint32_t code_at(const uint32_t* w, int e) {
     return v & mask;
 }
 
-// Exact small integer -> float through the mantissa of 2^23 (integer-to-float
-// conversion issues on the XU pipe).
-__device__ __forceinline__ float small_int_to_float(uint32_t q) {
-    return __fsub_rn(__uint_as_float(0x4B000000u | q), 8388608.0f);
-}
-
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     if (BF16) {
@@ -240,15 +245,46 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// The 8 codes of piece P as the bit patterns of 2^23 + code (an exact float):
+// byte-sized fields are moved into the mantissa by one byte permute each.
+template <int NBITS, int P>
+__device__ __forceinline__ void piece_codes_f(const uint32_t* w, uint32_t* f) {
+    if (NBITS == 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = __byte_perm(w[2 * P + i / 4], 0x4B00u, 0x5440u | (i % 4));
+    } else if (NBITS == 4) {
+        const uint32_t lo = w[P] & 0x0F0F0F0Fu, hi = (w[P] >> 4) & 0x0F0F0F0Fu;  // codes 0,2,4,6 and 1,3,5,7
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __byte_perm(lo, 0x4B00u, 0x5440u | i);
+            f[2 * i + 1] = __byte_perm(hi, 0x4B00u, 0x5440u | i);
+        }
+    } else if (NBITS == 2) {
+        const uint32_t h = w[P / 2] >> (16 * (P % 2));  // 8 codes in 16 bits
+        const uint32_t t0 = h & 0x0303u, t1 = (h >> 2) & 0x0303u, t2 = (h >> 4) & 0x0303u, t3 = (h >> 6) & 0x0303u;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {  // byte i of t_k holds code 4i + k
+            f[4 * i] = __byte_perm(t0, 0x4B00u, 0x5440u | i);
+            f[4 * i + 1] = __byte_perm(t1, 0x4B00u, 0x5440u | i);
+            f[4 * i + 2] = __byte_perm(t2, 0x4B00u, 0x5440u | i);
+            f[4 * i + 3] = __byte_perm(t3, 0x4B00u, 0x5440u | i);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = 0x4B000000u | code_at<NBITS>(w, 8 * P + i);
+    }
+}
+
 template <int NBITS, bool BF16, int P>
 __device__ __forceinline__ void piece_to_smem(const ARaw<NBITS>& a, uint32_t dst) {
-    uint32_t v[4];
+    uint32_t f[8], v[4];
+    piece_codes_f<NBITS, P>(a.w, f);
+    float wr[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float q0 = small_int_to_float(code_at<NBITS>(a.w, 8 * P + 2 * i));
-        const float q1 = small_int_to_float(code_at<NBITS>(a.w, 8 * P + 2 * i + 1));
-        v[i] = pack2<BF16>(__fmul_rn(__fsub_rn(q0, a.z[P]), a.s[P]), __fmul_rn(__fsub_rn(q1, a.z[P]), a.s[P]));
-    }
+    for (int i = 0; i < 8; ++i)
+        wr[i] = __fmul_rn(__fsub_rn(__fsub_rn(__uint_as_float(f[i]), 8388608.0f), a.z[P]), a.s[P]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = pack2<BF16>(wr[2 * i], wr[2 * i + 1]);
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
                  : "memory");
 }
@@ -265,37 +301,34 @@ __device__ __forceinline__ void store_a(const ARaw<NBITS>& a, uint32_t stage, in
     piece_to_smem<NBITS, BF16, 3>(a, row + ((((4 * h) + 3) ^ sw) << 4));
 }
 
-// The x tile [ntile][64] of K tile kt into a B stage, by cp.async (rows past
-// the batch are zero-filled: source size 0).
-__device__ __forceinline__ void issue_b(const GemmParams& p, int64_t n0, int kt, uint32_t stage) {
-    const int chunks = p.ntile * 8;
-    for (int q = threadIdx.x; q < chunks; q += kThreads) {
-        const int n = q >> 3, c = q & 7;
-        const int64_t b = n0 + n;
-        const bool in = b < p.batch;
-        const uint16_t* src = p.x + (in ? b : 0) * p.cols + static_cast<int64_t>(kt) * kTileK + c * 8;
-        cp_async16(stage + static_cast<uint32_t>(n) * 128u + ((c ^ (n & 7)) << 4), src, in ? 16u : 0u);
-    }
-}
-
 __host__ __device__ constexpr uint32_t tmem_columns(int ntile) {
     return ntile <= 32 ? 32u : ntile <= 64 ? 64u : ntile <= 128 ? 128u : 256u;
 }
 
-__host__ __device__ constexpr size_t gemm_smem_bytes(int ntile) {
+__host__ __device__ constexpr size_t gemm_smem_bytes(int ntile, int stages) {
     // 1024 bytes of slack to align the stages to the 1024-byte swizzle period
-    return 1024 + static_cast<size_t>(kStages) * (kStageA + static_cast<size_t>(ntile) * 128) + kStages * 8 + 16;
+    return 1024 + static_cast<size_t>(stages) * (kStageA + static_cast<size_t>(ntile) * 128) + 2 * stages * 8 + 16;
+}
+
+// As many stages as the shared memory holds (the x tiles are then issued
+// S - 2 tiles ahead).
+int gemm_stages(int ntile) {
+    int st = kMaxStages;
+    while (st > 3 && gemm_smem_bytes(ntile, st) > kSmemBudget) --st;
+    return st;
 }
 
 template <int NBITS, bool BF16, int ZB>
-__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p) {
+__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, const __grid_constant__ CUtensorMap xmap) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t* const smem = smem_raw + (base - smem_u32(smem_raw));
-    const uint32_t sA = base;                                      // kStages x 16 KB
-    const uint32_t sB = sA + kStages * kStageA;                    // kStages x ntile x 128 B
-    const uint32_t bars = sB + kStages * static_cast<uint32_t>(p.ntile) * 128u;  // kStages mbarriers
-    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(smem + (bars + kStages * 8 - base));
+    const int S = p.stages;
+    const uint32_t sA = base;                                               // S x 16 KB
+    const uint32_t sB = sA + S * kStageA;                                   // S x ntile x 128 B
+    const uint32_t bars = sB + S * static_cast<uint32_t>(p.ntile) * 128u;  // S "MMAs done" mbarriers
+    const uint32_t xbars = bars + S * 8;                                    // S "x full" mbarriers
+    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(smem + (xbars + S * 8 - base));
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -303,11 +336,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p) {
     const int num_k = static_cast<int>(p.cols / kTileK);
     const uint32_t ncols = tmem_columns(p.ntile);
     auto bar = [&](int s) { return bars + 8u * static_cast<uint32_t>(s); };
+    auto xbar = [&](int s) { return xbars + 8u * static_cast<uint32_t>(s); };
+    const uint32_t xbytes = static_cast<uint32_t>(p.ntile) * 128u;
     auto stage_a = [&](int s) { return sA + static_cast<uint32_t>(s) * kStageA; };
     auto stage_b = [&](int s) { return sB + static_cast<uint32_t>(s) * static_cast<uint32_t>(p.ntile) * 128u; };
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(bar(s), 1);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(bar(s), 1);
+            mbar_init(xbar(s), 1);
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -326,24 +364,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p) {
     // producer role: row r of the A tile, weights [32h, 32h + 32) of each K tile
     const int r = tid >> 1, h = tid & 1;
     const int64_t row = m0 + r;
-    ARaw<NBITS> cur, nxt;
-    load_a<NBITS, ZB>(p, row, 32 * h, cur);
-    issue_b(p, n0, 0, stage_b(0));
-    cp_async_commit();
-    bool ok = true;
-    for (int kt = 0; kt < num_k; ++kt) {
-        const int s = kt % kStages;
-        if (kt + 1 < num_k) {
-            // tile kt+1's stage is free once the MMAs of tile kt+1-kStages are done
-            const int s1 = (kt + 1) % kStages;
-            if (kt + 1 >= kStages && !mbar_wait(bar(s1), static_cast<uint32_t>((kt + 1) / kStages - 1) & 1u))
-                *abort_flag = 1;
-            issue_b(p, n0, kt + 1, stage_b(s1));
-            load_a<NBITS, ZB>(p, row, static_cast<int64_t>(kt + 1) * kTileK + 32 * h, nxt);
+    // codes, scales and zeros of tiles kt+1 .. kt+3 in flight in registers, the
+    // x tiles kt+1 .. kt+kPB by tensor copies (global latency hidden behind
+    // three and kPB tiles of work)
+    const int kPB = S - 2;
+    auto col = [&](int kt) { return static_cast<int64_t>(kt) * kTileK + 32 * h; };
+    ARaw<NBITS> a0, a1, a2;
+    load_a<NBITS, ZB>(p, row, col(0), a0);
+    if (num_k > 1) load_a<NBITS, ZB>(p, row, col(1), a1);
+    if (num_k > 2) load_a<NBITS, ZB>(p, row, col(2), a2);
+    if (tid == 0)
+        for (int d = 0; d < kPB && d < num_k; ++d) {
+            mbar_expect_tx(xbar(d), xbytes);
+            tma_load_2d(stage_b(d), &xmap, d * kTileK, static_cast<int>(n0), xbar(d));
         }
-        cp_async_commit();  // one group per iteration (empty on the last): uniform group accounting
-        store_a<NBITS, BF16>(cur, stage_a(s), r, h);
-        cp_async_wait<1>();  // tile kt's x has landed
+    bool ok = true;
+    int s = 0, ph = 0;             // stage of tile kt and the parity of its use of that stage
+    int sb = kPB, phb = 0;         // the same for tile kb = kt + kPB (kPB < S)
+    int sl = 0, phl = 0;           // ... of the last tile whose MMAs were issued
+    for (int kt = 0; kt < num_k; ++kt) {
+        // x of tile kb = kt+kPB: its stage (and tile kb's A stage) is free once
+        // the MMAs of tile kb-S (the previous use of the stage) are done
+        const int kb = kt + kPB;
+        if (kb < num_k) {
+            if (kb >= S && !mbar_wait(bar(sb), static_cast<uint32_t>(phb ^ 1))) *abort_flag = 1;
+            if (tid == 0) {
+                mbar_expect_tx(xbar(sb), xbytes);
+                tma_load_2d(stage_b(sb), &xmap, kb * kTileK, static_cast<int>(n0), xbar(sb));
+            }
+        }
+        ARaw<NBITS> a3;
+        if (kt + 3 < num_k) load_a<NBITS, ZB>(p, row, col(kt + 3), a3);
+        store_a<NBITS, BF16>(a0, stage_a(s), r, h);
         fence_async_smem();  // generic-proxy shared-memory writes -> visible to the tensor core
         __syncthreads();
         if (*abort_flag) {
@@ -351,19 +403,34 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p) {
             break;
         }
         if (tid == 0) {
-            tc_fence_after();
+            // tile kt's x has landed
+            if (mbar_wait(xbar(s), static_cast<uint32_t>(ph))) {
+                tc_fence_after();
 #pragma unroll
-            for (int j = 0; j < kTileK / 16; ++j)
-                mma_f16(tmem, smem_desc(stage_a(s) + 32u * j), smem_desc(stage_b(s) + 32u * j), idesc,
-                        (kt | j) != 0 ? 1u : 0u);
-            mma_commit(bar(s));
+                for (int j = 0; j < kTileK / 16; ++j)
+                    mma_f16(tmem, smem_desc(stage_a(s) + 32u * j), smem_desc(stage_b(s) + 32u * j), idesc,
+                            (kt | j) != 0 ? 1u : 0u);
+                mma_commit(bar(s));
+            } else {
+                *abort_flag = 1;  // the next barrier sends every thread out of the loop
+            }
         }
-        cur = nxt;
+        sl = s;
+        phl = ph;
+        if (++s == S) {
+            s = 0;
+            ph ^= 1;
+        }
+        if (++sb == S) {
+            sb = 0;
+            phb ^= 1;
+        }
+        a0 = a1;
+        a1 = a2;
+        a2 = a3;
     }
-    cp_async_wait<0>();
     if (ok) {  // the last commit covers every MMA of this CTA
-        const int kl = num_k - 1;
-        if (!mbar_wait(bar(kl % kStages), static_cast<uint32_t>(kl / kStages) & 1u)) *abort_flag = 1;
+        if (!mbar_wait(bar(sl), static_cast<uint32_t>(phl))) *abort_flag = 1;
     }
     __syncthreads();
     ok = ok && !*abort_flag;
@@ -394,20 +461,53 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p) {
 }
 
 template <int NBITS, bool BF16, int ZB>
-cudaError_t launch_t(const GemmParams& p, dim3 grid, size_t smem, cudaStream_t stream) {
+cudaError_t launch_t(const GemmParams& p, const CUtensorMap& xmap, dim3 grid, size_t smem, cudaStream_t stream) {
     auto kern = gemm_kernel<NBITS, BF16, ZB>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, stream>>>(p);
+    kern<<<grid, kThreads, smem, stream>>>(p, xmap);
     return cudaGetLastError();
 }
 
 template <int NBITS>
-cudaError_t launch_n(const GemmParams& p, bool bf16, int zb, dim3 grid, size_t smem, cudaStream_t stream) {
-    if (bf16) return zb == 8 ? launch_t<NBITS, true, 8>(p, grid, smem, stream)
-                             : launch_t<NBITS, true, 16>(p, grid, smem, stream);
-    return zb == 8 ? launch_t<NBITS, false, 8>(p, grid, smem, stream)
-                   : launch_t<NBITS, false, 16>(p, grid, smem, stream);
+cudaError_t launch_n(const GemmParams& p, const CUtensorMap& xmap, bool bf16, int zb, dim3 grid, size_t smem,
+                     cudaStream_t stream) {
+    if (bf16) return zb == 8 ? launch_t<NBITS, true, 8>(p, xmap, grid, smem, stream)
+                             : launch_t<NBITS, true, 16>(p, xmap, grid, smem, stream);
+    return zb == 8 ? launch_t<NBITS, false, 8>(p, xmap, grid, smem, stream)
+                   : launch_t<NBITS, false, 16>(p, xmap, grid, smem, stream);
+}
+
+// The driver's tensor-map encoder, fetched once through the runtime (the
+// library links no driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            f = nullptr;
+        }
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
+}
+
+// x [batch][cols] as a 2-D tensor (cols innermost), boxes of 64 x ntile in
+// the 128-byte swizzle; reads past the batch fill zeros.
+bool encode_x_map(CUtensorMap* map, const void* x, int bf16, int64_t batch, int64_t cols, int ntile) {
+    const auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(batch)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(ntile)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                           const_cast<void*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -437,15 +537,18 @@ cudaError_t launch_gemm(const GemvArgs& a, cudaStream_t stream) {
     p.batch = a.batch;
     int ntiles = 1;
     gemm_tiles(a.batch, &p.ntile, &ntiles);
+    p.stages = gemm_stages(p.ntile);
     const dim3 grid(static_cast<unsigned>((a.rows + kTileM - 1) / kTileM), static_cast<unsigned>(ntiles));
-    const size_t smem = gemm_smem_bytes(p.ntile);
+    const size_t smem = gemm_smem_bytes(p.ntile, p.stages);
     const bool bf16 = a.x_dtype == 1;
+    alignas(64) CUtensorMap xmap;
+    if (!encode_x_map(&xmap, a.x, bf16 ? 1 : 0, a.batch, a.cols, p.ntile)) return cudaErrorInvalidValue;
     switch (a.nbits) {
-        case 1: return launch_n<1>(p, bf16, a.zero_nbits, grid, smem, stream);
-        case 2: return launch_n<2>(p, bf16, a.zero_nbits, grid, smem, stream);
-        case 3: return launch_n<3>(p, bf16, a.zero_nbits, grid, smem, stream);
-        case 4: return launch_n<4>(p, bf16, a.zero_nbits, grid, smem, stream);
-        default: return launch_n<8>(p, bf16, a.zero_nbits, grid, smem, stream);
+        case 1: return launch_n<1>(p, xmap, bf16, a.zero_nbits, grid, smem, stream);
+        case 2: return launch_n<2>(p, xmap, bf16, a.zero_nbits, grid, smem, stream);
+        case 3: return launch_n<3>(p, xmap, bf16, a.zero_nbits, grid, smem, stream);
+        case 4: return launch_n<4>(p, xmap, bf16, a.zero_nbits, grid, smem, stream);
+        default: return launch_n<8>(p, xmap, bf16, a.zero_nbits, grid, smem, stream);
     }
 }
 
