@@ -44,7 +44,8 @@
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kProducers = 256;               // 8 warps: dequantisation
+constexpr int kThreads = kProducers + 32;     // + 1 warp: tensor copies and MMA issue
 constexpr int kTileM = 128;          // MMA M: weight rows per CTA
 constexpr int kTileK = 64;           // elements per K tile: one 128-byte swizzle row of 16-bit values
 constexpr int kMaxStages = 8;        // shared-memory ring: as many stages as fit (4 at N = 256, 8 at N <= 48)
@@ -82,13 +83,24 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 
-// Completion of the phase with this parity, or false after kWaitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Completion of the phase with this parity; false once the CTA's abort flag
+// is set or after kWaitNs (which sets the flag, so the other roles give up
+// their waits too).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
     if (mbar_test(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
-    while (!mbar_test(bar, parity))
-        if (global_ns() - t0 > kWaitNs) return false;
+    while (!mbar_test(bar, parity)) {
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitNs) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
     return true;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
@@ -307,7 +319,7 @@ __host__ __device__ constexpr uint32_t tmem_columns(int ntile) {
 
 __host__ __device__ constexpr size_t gemm_smem_bytes(int ntile, int stages) {
     // 1024 bytes of slack to align the stages to the 1024-byte swizzle period
-    return 1024 + static_cast<size_t>(stages) * (kStageA + static_cast<size_t>(ntile) * 128) + 2 * stages * 8 + 16;
+    return 1024 + static_cast<size_t>(stages) * (kStageA + static_cast<size_t>(ntile) * 128) + 3 * stages * 8 + 16;
 }
 
 // As many stages as the shared memory holds (the x tiles are then issued
@@ -326,9 +338,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
     const int S = p.stages;
     const uint32_t sA = base;                                               // S x 16 KB
     const uint32_t sB = sA + S * kStageA;                                   // S x ntile x 128 B
-    const uint32_t bars = sB + S * static_cast<uint32_t>(p.ntile) * 128u;  // S "MMAs done" mbarriers
-    const uint32_t xbars = bars + S * 8;                                    // S "x full" mbarriers
-    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(smem + (xbars + S * 8 - base));
+    const uint32_t bars = sB + S * static_cast<uint32_t>(p.ntile) * 128u;  // S "stage empty" (MMAs done)
+    const uint32_t xbars = bars + S * 8;                                    // S "x full" (tensor copy landed)
+    const uint32_t abars = xbars + S * 8;                                   // S "A full" (producers done)
+    uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(smem + (abars + S * 8 - base));
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -337,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
     const uint32_t ncols = tmem_columns(p.ntile);
     auto bar = [&](int s) { return bars + 8u * static_cast<uint32_t>(s); };
     auto xbar = [&](int s) { return xbars + 8u * static_cast<uint32_t>(s); };
+    auto abar = [&](int s) { return abars + 8u * static_cast<uint32_t>(s); };
     const uint32_t xbytes = static_cast<uint32_t>(p.ntile) * 128u;
     auto stage_a = [&](int s) { return sA + static_cast<uint32_t>(s) * kStageA; };
     auto stage_b = [&](int s) { return sB + static_cast<uint32_t>(s) * static_cast<uint32_t>(p.ntile) * 128u; };
@@ -345,6 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
         for (int s = 0; s < S; ++s) {
             mbar_init(bar(s), 1);
             mbar_init(xbar(s), 1);
+            mbar_init(abar(s), kProducers);
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -361,80 +376,85 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
     const uint32_t tmem = *tmem_slot;
     const uint32_t idesc = instr_desc(p.ntile, BF16 ? 1 : 0);
 
-    // producer role: row r of the A tile, weights [32h, 32h + 32) of each K tile
-    const int r = tid >> 1, h = tid & 1;
-    const int64_t row = m0 + r;
-    // codes, scales and zeros of tiles kt+1 .. kt+3 in flight in registers, the
-    // x tiles kt+1 .. kt+kPB by tensor copies (global latency hidden behind
-    // three and kPB tiles of work)
-    const int kPB = S - 2;
-    auto col = [&](int kt) { return static_cast<int64_t>(kt) * kTileK + 32 * h; };
-    ARaw<NBITS> a0, a1, a2;
-    load_a<NBITS, ZB>(p, row, col(0), a0);
-    if (num_k > 1) load_a<NBITS, ZB>(p, row, col(1), a1);
-    if (num_k > 2) load_a<NBITS, ZB>(p, row, col(2), a2);
-    if (tid == 0)
+    bool ok = true;
+    if (warp < kProducers / 32) {
+        // producers: row r of the A tile, weights [32h, 32h + 32) of each K
+        // tile; codes, scales and zeros of tiles kt+1 .. kt+3 in flight in
+        // registers (global latency hidden behind three tiles of work)
+        const int r = tid >> 1, h = tid & 1;
+        const int64_t row = m0 + r;
+        auto col = [&](int kt) { return static_cast<int64_t>(kt) * kTileK + 32 * h; };
+        ARaw<NBITS> a0, a1, a2;
+        load_a<NBITS, ZB>(p, row, col(0), a0);
+        if (num_k > 1) load_a<NBITS, ZB>(p, row, col(1), a1);
+        if (num_k > 2) load_a<NBITS, ZB>(p, row, col(2), a2);
+        int s = 0, ph = 0;  // stage of tile kt and the parity of its use of that stage
+        for (int kt = 0; kt < num_k; ++kt) {
+            ARaw<NBITS> a3;
+            if (kt + 3 < num_k) load_a<NBITS, ZB>(p, row, col(kt + 3), a3);
+            // the stage is free once the MMAs of its previous use (tile kt-S) are done
+            if (kt >= S && !mbar_wait(bar(s), static_cast<uint32_t>(ph ^ 1), abort_flag)) {
+                ok = false;
+                break;
+            }
+            store_a<NBITS, BF16>(a0, stage_a(s), r, h);
+            fence_async_smem();  // generic-proxy shared-memory writes -> visible to the tensor core
+            mbar_arrive(abar(s));
+            if (++s == S) {
+                s = 0;
+                ph ^= 1;
+            }
+            a0 = a1;
+            a1 = a2;
+            a2 = a3;
+        }
+    } else if (lane == 0) {
+        // tensor copies of x (kPB = S - 2 tiles ahead) and the MMAs
+        const int kPB = S - 2;
         for (int d = 0; d < kPB && d < num_k; ++d) {
             mbar_expect_tx(xbar(d), xbytes);
             tma_load_2d(stage_b(d), &xmap, d * kTileK, static_cast<int>(n0), xbar(d));
         }
-    bool ok = true;
-    int s = 0, ph = 0;             // stage of tile kt and the parity of its use of that stage
-    int sb = kPB, phb = 0;         // the same for tile kb = kt + kPB (kPB < S)
-    int sl = 0, phl = 0;           // ... of the last tile whose MMAs were issued
-    for (int kt = 0; kt < num_k; ++kt) {
-        // x of tile kb = kt+kPB: its stage (and tile kb's A stage) is free once
-        // the MMAs of tile kb-S (the previous use of the stage) are done
-        const int kb = kt + kPB;
-        if (kb < num_k) {
-            if (kb >= S && !mbar_wait(bar(sb), static_cast<uint32_t>(phb ^ 1))) *abort_flag = 1;
-            if (tid == 0) {
+        int s = 0, ph = 0, sb = kPB, phb = 0, sl = 0, phl = 0;
+        for (int kt = 0; kt < num_k && ok; ++kt) {
+            const int kb = kt + kPB;  // its stage is free once the MMAs of tile kb-S (issued two tiles ago) are done
+            if (kb < num_k) {
+                if (kb >= S && !mbar_wait(bar(sb), static_cast<uint32_t>(phb ^ 1), abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 mbar_expect_tx(xbar(sb), xbytes);
                 tma_load_2d(stage_b(sb), &xmap, kb * kTileK, static_cast<int>(n0), xbar(sb));
             }
-        }
-        ARaw<NBITS> a3;
-        if (kt + 3 < num_k) load_a<NBITS, ZB>(p, row, col(kt + 3), a3);
-        store_a<NBITS, BF16>(a0, stage_a(s), r, h);
-        fence_async_smem();  // generic-proxy shared-memory writes -> visible to the tensor core
-        __syncthreads();
-        if (*abort_flag) {
-            ok = false;
-            break;
-        }
-        if (tid == 0) {
-            // tile kt's x has landed
-            if (mbar_wait(xbar(s), static_cast<uint32_t>(ph))) {
-                tc_fence_after();
+            if (!mbar_wait(abar(s), static_cast<uint32_t>(ph), abort_flag) ||
+                !mbar_wait(xbar(s), static_cast<uint32_t>(ph), abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
 #pragma unroll
-                for (int j = 0; j < kTileK / 16; ++j)
-                    mma_f16(tmem, smem_desc(stage_a(s) + 32u * j), smem_desc(stage_b(s) + 32u * j), idesc,
-                            (kt | j) != 0 ? 1u : 0u);
-                mma_commit(bar(s));
-            } else {
-                *abort_flag = 1;  // the next barrier sends every thread out of the loop
+            for (int j = 0; j < kTileK / 16; ++j)
+                mma_f16(tmem, smem_desc(stage_a(s) + 32u * j), smem_desc(stage_b(s) + 32u * j), idesc,
+                        (kt | j) != 0 ? 1u : 0u);
+            mma_commit(bar(s));
+            sl = s;
+            phl = ph;
+            if (++s == S) {
+                s = 0;
+                ph ^= 1;
+            }
+            if (++sb == S) {
+                sb = 0;
+                phb ^= 1;
             }
         }
-        sl = s;
-        phl = ph;
-        if (++s == S) {
-            s = 0;
-            ph ^= 1;
-        }
-        if (++sb == S) {
-            sb = 0;
-            phb ^= 1;
-        }
-        a0 = a1;
-        a1 = a2;
-        a2 = a3;
+        // the last commit covers every MMA of this CTA
+        if (ok && !mbar_wait(bar(sl), static_cast<uint32_t>(phl), abort_flag)) ok = false;
     }
-    if (ok) {  // the last commit covers every MMA of this CTA
-        if (!mbar_wait(bar(sl), static_cast<uint32_t>(phl))) *abort_flag = 1;
-    }
-    __syncthreads();
-    ok = ok && !*abort_flag;
-    if (ok) {
+    if (!ok) *abort_flag = 1;
+    __syncthreads();  // the MMA thread has seen its last commit complete (or someone gave up)
+    ok = !*abort_flag;
+    if (ok && warp < kProducers / 32) {
         tc_fence_after();
         const int q = warp & 3, half = warp >> 2, nh = p.ntile / 2;
         const int64_t orow = m0 + 32 * q + lane;
