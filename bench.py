@@ -567,7 +567,19 @@ def run_gemm_case(spec):
     flops = 2.0 * rows * cols * batch
     hbm, _, kind = peaks()
     tf = _measured_peaks().get("bf16_tflops")
+    # the oracle's product (fp64, one host thread) on a sample of rows, beside the kernel
+    import oracle
+    qc = {k: (v.cpu().numpy() if v is not None else None) for k, v in q.items() if k in
+          ("packed", "scale", "zero", "zero_meta")}
+    xo = x.cpu().view(torch.int16).numpy().view(np.uint16)
+    sr = 8
+    t0 = time.perf_counter()
+    oracle.gemm(qc["packed"][:sr * cols * nbits // 8], qc["scale"][:sr * cols // g], qc["zero"][:sr * cols // g],
+                qc["zero_meta"], sr, cols, nbits, g, 8, xo, oracle.BF16)
+    ot = time.perf_counter() - t0
     print(json.dumps({"case": spec, "ms_median": med, "ms_min": ms[0], "tflops": flops / (med / 1e3) / 1e12,
+                      "cpu_baseline": {"value": 2.0 * sr * cols * batch / ot / 1e12, "unit": "TFLOP/s", "cores": 1,
+                                       "kind": "oracle", "sample": f"first {sr} rows, all columns, batch {batch}"},
                       "bf16_peak_tflops": tf, "tensor_frac": (flops / (med / 1e3) / 1e12 / tf) if tf else None,
                       "bytes": nbytes, "gbs": nbytes / (med / 1e3) / 1e9, "hbm_peak_gbs": hbm, "peak_kind": kind,
                       "hbm_frac": nbytes / (med / 1e3) / 1e9 / hbm, "l2": "flushed before every call"}))
