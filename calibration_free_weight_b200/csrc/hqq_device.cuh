@@ -84,6 +84,62 @@ __device__ __forceinline__ ElemEval eval_elem_nc(float ws, float z) {
     return e;
 }
 
+// ---- packed fp32 pairs (add/sub/mul .rn.f32x2: two IEEE fp32 operations,
+// each rounded exactly as the scalar one, in one instruction) ----
+
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// The fast-path sums of one evaluation over a lane's E elements (E even, every
+// v clamp-free): sum |r|^p and sum W_q, with v, t, q, r, p*lg2|r| formed
+// pairwise by packed fp32 operations -- the same values as eval_elem_nc.  The
+// error is accumulated one element at a time in element order (the stop
+// decisions compare these sums, so their rounding is kept as the scalar loop
+// forms it); sum W_q is exact in any order (integers), so it is kept pairwise.
+template <int E>
+__device__ __forceinline__ void fast_sums(const float* ws, float z, float p, float* err_out, float* sq_out) {
+    const uint64_t z2 = f2_pack(z, z), m2 = f2_pack(kMagic, kMagic), p2 = f2_pack(p, p);
+    uint64_t sq2 = f2_pack(0.0f, 0.0f);
+    float err = 0.0f;
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+        const uint64_t v = f2_add(f2_pack(ws[i], ws[i + 1]), z2);
+        const uint64_t q = f2_sub(f2_add(v, m2), m2);  // round half to even: fl(fl(v + M) - M)
+        const uint64_t r = f2_sub(v, q);
+        float r0, r1;
+        f2_unpack(r, r0, r1);
+        float l0, l1;
+        f2_unpack(f2_mul(f2_pack(lg2_approx(fabsf(r0)), lg2_approx(fabsf(r1))), p2), l0, l1);
+        err = __fadd_rn(__fadd_rn(err, ex2_approx(l0)), ex2_approx(l1));
+        sq2 = f2_add(sq2, q);
+    }
+    float s0, s1;
+    f2_unpack(sq2, s0, s1);
+    *err_out = err;
+    *sq_out = __fadd_rn(s0, s1);
+}
+
 // True when no v = fl(ws + z) of a set with ws in [wsmin, wsmax] needs the
 // clamp (fl(. + z) is monotone, so the extremes decide).
 __device__ __forceinline__ bool clamp_free(float wsmin, float wsmax, float z, float Lf) {

@@ -377,14 +377,7 @@ __device__ __forceinline__ void eval_lane_reload(const KParams& k, const WarpTil
     float err = 0.0f, sq = 0.0f;
     double swe = 0.0;
     if (fast) {
-        if (w.valid) {
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                const ElemEval e = eval_elem_nc(ws[i], z);
-                err += pow_pos(fabsf(e.r), k.p);
-                sq += e.q;
-            }
-        }
+        if (w.valid) fast_sums<E>(ws, z, k.p, &err, &sq);
     } else if (w.valid) {
         const float3 r = eval_lane_slow<DT, AXIS, E>(k, w, s, z, it, sp, &swe);
         err = r.x;
@@ -416,14 +409,7 @@ __device__ __forceinline__ void tensor_iteration(const KParams& k, const WarpTil
     const bool sp = w.valid && shrink_possible(s, z, z0, thr, k.Lf);
     float err = 0.0f, sq = 0.0f;
     if (__all_sync(kFull, !w.valid || (!sp && clamp_free(lmin, lmax, z, k.Lf)))) {
-        if (w.valid) {
-#pragma unroll
-            for (int i = 0; i < E; ++i) {
-                const ElemEval e = eval_elem_nc(ws[i], z);
-                err += pow_pos(fabsf(e.r), k.p);
-                sq += e.q;
-            }
-        }
+        if (w.valid) fast_sums<E>(ws, z, k.p, &err, &sq);
         sq = seg_sum(sq, k.P);
         z = zero_from_sums_f2(sq, sws2, inv_g);
     } else {
