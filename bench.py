@@ -50,8 +50,8 @@ KERNEL_SOURCES = ["calibration_free_weight_b200/csrc/hqq_kernels.cu", "calibrati
 # launch), averaged over the timed step's tensor-stop calls,
 # from the ncu launch list summarised in profiles/ (taken on the kernel sources
 # whose sha256 is recorded here; None until a capture exists).
-TRAFFIC = {"src_sha256": "51ad6fc66440f5caf9c4a5d955037d91c206a9f8f57755c3553d344a7ec5ed5b",
-           "bytes_per_call": 381090492, "summary": "profiles/launches_llama2-7b-mlp-sweep.md"}
+TRAFFIC = {"src_sha256": "46f27c58d4c01e2788eb81495396900f6a1351042cc803321971036b3d7b0eed",
+           "bytes_per_call": 381103462, "summary": "profiles/launches_llama2-7b-mlp-sweep.md"}
 
 
 def kernel_sources_sha():
