@@ -15,18 +15,19 @@
 // K is walked in 64-element tiles through a ring of S shared-memory
 // stages, each in the canonical 128-byte-swizzled K-major layout (row r of a
 // tile at r * 128 bytes, its 16-byte chunk c at chunk c ^ (r % 8)):
-//   * every thread dequantises 32 weights of the A tile (codes, scales and
-//     zeros prefetched in registers three tiles ahead) and stores them as
-//     16-bit values;
-//   * the x tile arrives by a 2-D tensor copy (TMA, 128-byte swizzle, from
-//     this GPU's own memory, no multicast) issued by thread 0 two tiles ahead
-//     and completing on the stage's "x full" mbarrier; rows past the batch are
-//     zero-filled by the copy;
-//   * thread 0 issues four tcgen05.mma (K = 16 each) into the fp32 accumulator
-//     in tensor memory and commits them to the stage's mbarrier, which frees
-//     the stage for the tile S later.
-// The epilogue reads the accumulator with tcgen05.ld (warp w reads the 32 rows
-// of its lane quarter w % 4, half of the columns) and stores y.
+//   * 16 producer warps dequantise, 16 weights of the A tile per thread
+//     (codes, scales and zeros prefetched in registers three tiles ahead),
+//     store them as 16-bit values and arrive on the stage's "A full" mbarrier;
+//   * one thread of a 17th warp issues the x tile's 2-D tensor copy (TMA,
+//     128-byte swizzle, from this GPU's own memory, no multicast) S - 2 tiles
+//     ahead, completing on the stage's "x full" mbarrier (rows past the batch
+//     are zero-filled by the copy), and, once both halves of a stage are full,
+//     four tcgen05.mma (K = 16 each) into the fp32 accumulator in tensor
+//     memory, committed to the stage's "empty" mbarrier, which frees the
+//     stage for the tile S later.
+// The epilogue reads the accumulator with tcgen05.ld (producer warp w reads
+// the 32 rows of its lane quarter w % 4, every fourth 8-column chunk) and
+// stores y.
 //
 // Waits: every mbarrier wait gives up after ~1 s of global time, records a
 // timeout in a device status word (read by hqq_gemm_get_status) and makes the
@@ -44,7 +45,9 @@
 
 namespace {
 
-constexpr int kProducers = 256;               // 8 warps: dequantisation
+constexpr int kWpt = 16;                      // weights per producer thread per K tile (two 8-weight pieces)
+constexpr int kPieces = kWpt / 8;
+constexpr int kProducers = 128 * 64 / kWpt;   // 512 threads, 16 warps: dequantisation
 constexpr int kThreads = kProducers + 32;     // + 1 warp: tensor copies and MMA issue
 constexpr int kTileM = 128;          // MMA M: weight rows per CTA
 constexpr int kTileK = 64;           // elements per K tile: one 128-byte swizzle row of 16-bit values
@@ -177,13 +180,14 @@ struct GemmParams {
     int stages;         // S, in [3, kMaxStages]
 };
 
-// Inputs of one thread's 32 consecutive weights of one K tile (one row):
+// Inputs of one thread's kWpt consecutive weights of one K tile (one row):
 // the codes as a little-endian bit stream (weight e at bit e * NBITS) and the
-// scale and zero of each 8-weight piece.  Loaded one tile ahead.
+// scale and zero of each 8-weight piece.  Loaded ahead of use.
 template <int NBITS>
 struct ARaw {
-    uint32_t w[NBITS];
-    float s[4], z[4];
+    static constexpr int kWords = (kWpt * NBITS + 31) / 32;
+    uint32_t w[kWords];
+    float s[kPieces], z[kPieces];
 };
 
 __device__ __forceinline__ float half_to_float(uint16_t h) { return __half2float(__ushort_as_half(h)); }
@@ -192,34 +196,36 @@ template <int NBITS, int ZB>
 __device__ __forceinline__ void load_a(const GemmParams& p, int64_t row, int64_t c0, ARaw<NBITS>& a) {
     if (row >= p.rows) {  // rows past the matrix: W_r = (0 - 0) * 0
 #pragma unroll
-        for (int i = 0; i < NBITS; ++i) a.w[i] = 0u;
+        for (int i = 0; i < ARaw<NBITS>::kWords; ++i) a.w[i] = 0u;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) a.s[i] = a.z[i] = 0.0f;
+        for (int i = 0; i < kPieces; ++i) a.s[i] = a.z[i] = 0.0f;
         return;
     }
-    const int64_t e0 = row * p.cols + c0;  // first weight; a multiple of 32, so its codes start on 4 * NBITS bytes
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(p.packed + (e0 / 32) * (4 * NBITS));
-    if (NBITS == 4 || NBITS == 8) {
-#pragma unroll
-        for (int i = 0; i < NBITS; i += 4) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(src) + i / 4);
-            a.w[i] = v.x;
-            a.w[(i + 1) % NBITS] = v.y;
-            a.w[(i + 2) % NBITS] = v.z;
-            a.w[(i + 3) % NBITS] = v.w;
-        }
-    } else if (NBITS == 2) {
+    const int64_t e0 = row * p.cols + c0;  // first weight, a multiple of 16: its codes start on 2 * NBITS bytes
+    const uint8_t* src = p.packed + (e0 / 16) * (2 * NBITS);
+    if (NBITS == 8) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src));
+        a.w[0] = v.x;
+        a.w[1 % ARaw<NBITS>::kWords] = v.y;
+        a.w[2 % ARaw<NBITS>::kWords] = v.z;
+        a.w[3 % ARaw<NBITS>::kWords] = v.w;
+    } else if (NBITS == 4) {
         const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
         a.w[0] = v.x;
-        a.w[1 % NBITS] = v.y;
-    } else {
-#pragma unroll
-        for (int i = 0; i < NBITS; ++i) a.w[i] = __ldg(src + i);
+        a.w[1 % ARaw<NBITS>::kWords] = v.y;
+    } else if (NBITS == 2) {
+        a.w[0] = __ldg(reinterpret_cast<const uint32_t*>(src));
+    } else if (NBITS == 1) {
+        a.w[0] = __ldg(reinterpret_cast<const uint16_t*>(src));
+    } else {  // 3 bits: 6 bytes on a 2-byte boundary
+        const uint16_t* h = reinterpret_cast<const uint16_t*>(src);
+        a.w[0] = static_cast<uint32_t>(__ldg(h)) | (static_cast<uint32_t>(__ldg(h + 1)) << 16);
+        a.w[1 % ARaw<NBITS>::kWords] = __ldg(h + 2);
     }
-    // one group for all 32 weights when g >= 32, else one per piece
-    const int npc = p.g_log >= 5 ? 1 : 4;
+    // one group for both pieces when g >= 16, else one per piece
+    const int npc = p.g_log >= 4 ? 1 : kPieces;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < kPieces; ++q) {
         if (q < npc) {
             const int64_t j = (e0 + 8 * q) >> p.g_log;
             a.s[q] = half_to_float(__ldg(p.scale + j));
@@ -243,7 +249,7 @@ __device__ __forceinline__ uint32_t code_at(const uint32_t* w, int e) {
     const int b = e * NBITS, word = b / 32, off = b % 32;
     constexpr uint32_t mask = (1u << NBITS) - 1u;
     uint32_t v = w[word] >> off;
-    if (off + NBITS > 32) v |= w[(word + 1) % NBITS] << (32 - off);
+    if (off + NBITS > 32) v |= w[(word + 1) % ARaw<NBITS>::kWords] << (32 - off);
     return v & mask;
 }
 
@@ -301,16 +307,16 @@ __device__ __forceinline__ void piece_to_smem(const ARaw<NBITS>& a, uint32_t dst
                  : "memory");
 }
 
-// W_r of this thread's 32 weights, rounded to 16 bits, into row r, chunks
-// 4h .. 4h+3 of an A stage (128-byte swizzle: chunk c of row r at c ^ (r % 8)).
+// W_r of this thread's kWpt weights, rounded to 16 bits, into row r, chunks
+// kPieces*h .. kPieces*h + kPieces-1 of an A stage (128-byte swizzle: chunk c of
+// row r at c ^ (r % 8)).
 template <int NBITS, bool BF16>
 __device__ __forceinline__ void store_a(const ARaw<NBITS>& a, uint32_t stage, int r, int h) {
+    static_assert(kPieces == 2, "two pieces per thread");
     const uint32_t row = stage + static_cast<uint32_t>(r) * 128u;
     const int sw = r & 7;
-    piece_to_smem<NBITS, BF16, 0>(a, row + ((((4 * h) + 0) ^ sw) << 4));
-    piece_to_smem<NBITS, BF16, 1>(a, row + ((((4 * h) + 1) ^ sw) << 4));
-    piece_to_smem<NBITS, BF16, 2>(a, row + ((((4 * h) + 2) ^ sw) << 4));
-    piece_to_smem<NBITS, BF16, 3>(a, row + ((((4 * h) + 3) ^ sw) << 4));
+    piece_to_smem<NBITS, BF16, 0>(a, row + ((((kPieces * h) + 0) ^ sw) << 4));
+    piece_to_smem<NBITS, BF16, 1>(a, row + ((((kPieces * h) + 1) ^ sw) << 4));
 }
 
 __host__ __device__ constexpr uint32_t tmem_columns(int ntile) {
@@ -378,12 +384,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
 
     bool ok = true;
     if (warp < kProducers / 32) {
-        // producers: row r of the A tile, weights [32h, 32h + 32) of each K
+        // producers: row r of the A tile, weights [16h, 16h + 16) of each K
         // tile; codes, scales and zeros of tiles kt+1 .. kt+3 in flight in
         // registers (global latency hidden behind three tiles of work)
-        const int r = tid >> 1, h = tid & 1;
+        const int r = tid >> 2, h = tid & 3;
         const int64_t row = m0 + r;
-        auto col = [&](int kt) { return static_cast<int64_t>(kt) * kTileK + 32 * h; };
+        auto col = [&](int kt) { return static_cast<int64_t>(kt) * kTileK + kWpt * h; };
         ARaw<NBITS> a0, a1, a2;
         load_a<NBITS, ZB>(p, row, col(0), a0);
         if (num_k > 1) load_a<NBITS, ZB>(p, row, col(1), a1);
@@ -456,9 +462,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
     ok = !*abort_flag;
     if (ok && warp < kProducers / 32) {
         tc_fence_after();
-        const int q = warp & 3, half = warp >> 2, nh = p.ntile / 2;
+        // warp w reads lane quarter w % 4 (rows 32q .. 32q+31), every
+        // (kProducers/128)-th 8-column chunk from chunk w / 4
+        constexpr int kColWarps = kProducers / 128;
+        const int q = warp & 3;
         const int64_t orow = m0 + 32 * q + lane;
-        for (int c0 = half * nh; c0 < (half + 1) * nh; c0 += 8) {
+        for (int c0 = 8 * (warp >> 2); c0 < p.ntile; c0 += 8 * kColWarps) {
             float v[8];
             tmem_ld8(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0), v);
             if (orow < p.rows) {
