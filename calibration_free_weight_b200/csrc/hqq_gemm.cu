@@ -293,16 +293,40 @@ __device__ __forceinline__ void piece_codes_f(const uint32_t* w, uint32_t* f) {
     }
 }
 
+// Packed fp32 pairs: two IEEE fp32 operations, each rounded as the scalar
+// one, per instruction.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 template <int NBITS, bool BF16, int P>
 __device__ __forceinline__ void piece_to_smem(const ARaw<NBITS>& a, uint32_t dst) {
     uint32_t f[8], v[4];
     piece_codes_f<NBITS, P>(a.w, f);
-    float wr[8];
+    const uint64_t two23 = f2_pack(8388608.0f, 8388608.0f), z2 = f2_pack(a.z[P], a.z[P]),
+                   s2 = f2_pack(a.s[P], a.s[P]);
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-        wr[i] = __fmul_rn(__fsub_rn(__fsub_rn(__uint_as_float(f[i]), 8388608.0f), a.z[P]), a.s[P]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = pack2<BF16>(wr[2 * i], wr[2 * i + 1]);
+    for (int i = 0; i < 4; ++i) {  // (q - z) * s for a pair of weights, q = (2^23 + q) - 2^23 exactly
+        const uint64_t q = f2_sub(f2_pack(__uint_as_float(f[2 * i]), __uint_as_float(f[2 * i + 1])), two23);
+        float w0, w1;
+        f2_unpack(f2_mul(f2_sub(q, z2), s2), w0, w1);
+        v[i] = pack2<BF16>(w0, w1);
+    }
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
                  : "memory");
 }
