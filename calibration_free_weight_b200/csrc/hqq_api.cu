@@ -301,6 +301,16 @@ int hqq_gemm(const void* W_q_packed, const void* scale, const void* zero, const 
 
 int hqq_gemm_get_status(void* stream) { return hqq::gemm_take_status(static_cast<cudaStream_t>(stream)); }
 
+int hqq_gemm_wait_selftest(int64_t limit_us, void* stream) {
+    if (limit_us < 1 || limit_us > 1000000) return HQQ_ERR_INVALID_ARG;
+    if (hqq::launch_gemm_wait_selftest(static_cast<unsigned long long>(limit_us) * 1000ull,
+                                       static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return HQQ_ERR_CUDA;
+    }
+    return HQQ_OK;
+}
+
 int hqq_quantize_scale8(const void* scale, int64_t num_groups, int scale_group, void* scale_q, void* scale_meta,
                         void* stream) {
     if (num_groups < 0 || scale_group < 1) return HQQ_ERR_INVALID_ARG;

@@ -87,14 +87,15 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 // Completion of the phase with this parity; false once the CTA's abort flag
-// is set or after kWaitNs (which sets the flag, so the other roles give up
+// is set or after limit_ns (which sets the flag, so the other roles give up
 // their waits too).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns = kWaitNs) {
     if (mbar_test(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (!mbar_test(bar, parity)) {
         if (*abort_flag) return false;
-        if (global_ns() - t0 > kWaitNs) {
+        if (global_ns() - t0 > limit_ns) {
             *abort_flag = 1;
             return false;
         }
@@ -513,6 +514,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
     }
 }
 
+// Diagnostic: the product's bounded wait on an mbarrier that nothing arrives
+// on, with a short limit; it gives up and records the timeout exactly as the
+// product does.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x != 0) return;
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (!mbar_wait(smem_u32(&bar), 0u, &abort_flag, limit_ns)) atomicExch(&g_gemm_status, 1u);
+}
+
 template <int NBITS, bool BF16, int ZB>
 cudaError_t launch_t(const GemmParams& p, const CUtensorMap& xmap, dim3 grid, size_t smem, cudaStream_t stream) {
     auto kern = gemm_kernel<NBITS, BF16, ZB>;
@@ -603,6 +617,11 @@ cudaError_t launch_gemm(const GemvArgs& a, cudaStream_t stream) {
         case 4: return launch_n<4>(p, xmap, bf16, a.zero_nbits, grid, smem, stream);
         default: return launch_n<8>(p, xmap, bf16, a.zero_nbits, grid, smem, stream);
     }
+}
+
+cudaError_t launch_gemm_wait_selftest(unsigned long long limit_ns, cudaStream_t stream) {
+    wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+    return cudaGetLastError();
 }
 
 // HQQ_OK, or HQQ_ERR_TIMEOUT if a product since the last call gave up a wait

@@ -89,6 +89,8 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t stream);
 cudaError_t launch_gemm(const GemvArgs& a, cudaStream_t stream);
 // Batch tiles of launch_gemm: ntiles tiles of ntile (a multiple of 16, <= 256) rows.
 void gemm_tiles(int batch, int* ntile, int* ntiles);
+// One bounded wait, as the product's, on a barrier nothing arrives on (diagnostic).
+cudaError_t launch_gemm_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
 // Synchronises the stream; 0, 6 (a wait of a product gave up; cleared) or 5 (CUDA error).
 int gemm_take_status(cudaStream_t stream);
 

@@ -20,7 +20,8 @@ HQQ_STOP_GROUP, HQQ_STOP_TENSOR, HQQ_STOP_NONE = 0, 1, 2
 EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_quantize", "hqq_dequantize",
             "hqq_get_status", "hqq_status_string", "hqq_quantize_noalloc", "hqq_quantize_scale8",
             "hqq_dequantize_s8", "hqq_stream_device_bytes", "hqq_quantize_stream", "hqq_gemv",
-            "hqq_stream_jobs_device_bytes", "hqq_quantize_stream_jobs", "hqq_gemm", "hqq_gemm_get_status")
+            "hqq_stream_jobs_device_bytes", "hqq_quantize_stream_jobs", "hqq_gemm", "hqq_gemm_get_status",
+            "hqq_gemm_wait_selftest")
 
 
 class hqq_host_matrix(C.Structure):
@@ -70,6 +71,8 @@ def _load():
     L.hqq_gemm.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, i32, i32, P, P]
     L.hqq_gemm_get_status.restype = i32
     L.hqq_gemm_get_status.argtypes = [P]
+    L.hqq_gemm_wait_selftest.restype = i32
+    L.hqq_gemm_wait_selftest.argtypes = [i64, P]
     HM = C.POINTER(hqq_host_matrix)
     L.hqq_stream_device_bytes.restype = sz
     L.hqq_stream_device_bytes.argtypes = [HM, i32, i32, i32, i32, i32, i32]
@@ -179,6 +182,10 @@ def hqq_gemm(W_q_packed, scale, zero, zero_meta, rows, cols, nbits, group_size, 
 
 def hqq_gemm_get_status(stream=None):
     return lib.hqq_gemm_get_status(_stream(stream))
+
+
+def hqq_gemm_wait_selftest(limit_us, stream=None):
+    return lib.hqq_gemm_wait_selftest(limit_us, _stream(stream))
 
 
 def hqq_stream_jobs_device_bytes(jobs, n):

@@ -316,6 +316,14 @@ int hqq_gemm(const void* W_q_packed, const void* scale, const void* zero, const 
  * or HQQ_ERR_CUDA. */
 int hqq_gemm_get_status(void* stream);
 
+/* Diagnostic of the bounded waits: one thread runs hqq_gemm's mbarrier wait,
+ * with a limit of limit_us microseconds (1 .. 1e6), on a barrier that nothing
+ * arrives on; it gives up and records the timeout as hqq_gemm does, so the
+ * next hqq_gemm_get_status returns HQQ_ERR_TIMEOUT (and the one after that
+ * HQQ_OK).  Asynchronous on `stream`; returns HQQ_OK, HQQ_ERR_INVALID_ARG or
+ * HQQ_ERR_CUDA. */
+int hqq_gemm_wait_selftest(int64_t limit_us, void* stream);
+
 /* Synchronise `stream` and return the device status word held in `workspace`
  * by the last hqq_quantize on it (HQQ_OK), or HQQ_ERR_CUDA if the
  * synchronisation or copy fails. */

@@ -224,6 +224,11 @@ def test_gemm_rejections(hq):
     assert L.hqq_gemm(p, p, p, None, 128, 128, 4, 64, 16, p, 1, 4, p, None) == hq.HQQ_ERR_INVALID_ARG
 
 
+def test_gemm_wait_selftest_rejects_bad_limits(hq):
+    assert hq.lib.hqq_gemm_wait_selftest(0, None) == hq.HQQ_ERR_INVALID_ARG
+    assert hq.lib.hqq_gemm_wait_selftest(1000001, None) == hq.HQQ_ERR_INVALID_ARG
+
+
 def test_status_strings(hq):
     for code in range(9):
         s = hq.hqq_status_string(code)

@@ -136,3 +136,19 @@ def test_gemm_repeated_calls_are_deterministic(hq):
     a = run(hq, q, x, rows, cols, nbits, g, zb)
     b = run(hq, q, x, rows, cols, nbits, g, zb)
     assert np.array_equal(a, b)
+
+
+def test_gemm_bounded_wait_gives_up_and_reports(hq):
+    """The product's mbarrier wait, run on a barrier nothing arrives on with a
+    5 ms limit, gives up, the status reads HQQ_ERR_TIMEOUT once (then it is
+    cleared), and the context stays usable: a product right after is correct."""
+    assert hq.hqq_gemm_get_status() == hq.HQQ_OK
+    assert hq.hqq_gemm_wait_selftest(5000) == hq.HQQ_OK
+    assert hq.hqq_gemm_get_status() == hq.HQQ_ERR_TIMEOUT
+    assert hq.hqq_gemm_get_status() == hq.HQQ_OK
+    rows, cols, nbits, g, zb = 256, 512, 4, 64, 16
+    q = make_q(rows, cols, nbits, g, zb, seed=11)
+    x, xo, xdt = make_x(16, cols, torch.bfloat16, seed=11)
+    y = run(hq, q, x, rows, cols, nbits, g, zb)
+    yo, ya = oracle.gemm(q["packed"], q["scale"], q["zero"], q["zero_meta"], rows, cols, nbits, g, zb, xo, xdt)
+    check(y, yo, ya, cols)
