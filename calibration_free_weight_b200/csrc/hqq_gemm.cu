@@ -19,7 +19,7 @@
 //     (codes, scales and zeros prefetched in registers three tiles ahead),
 //     store them as 16-bit values and arrive on the stage's "A full" mbarrier;
 //   * one thread of a 17th warp issues the x tile's 2-D tensor copy (TMA,
-//     128-byte swizzle, from this GPU's own memory, no multicast) S - 2 tiles
+//     128-byte swizzle, from this GPU's own memory, into this CTA only) S - 2 tiles
 //     ahead, completing on the stage's "x full" mbarrier (rows past the batch
 //     are zero-filled by the copy), and, once both halves of a stage are full,
 //     four tcgen05.mma (K = 16 each) into the fp32 accumulator in tensor
