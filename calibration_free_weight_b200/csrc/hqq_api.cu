@@ -261,9 +261,15 @@ int hqq_gemv(const void* W_q_packed, const void* scale, const void* zero, const 
     return HQQ_OK;
 }
 
+size_t hqq_gemm_workspace_bytes(int64_t rows, int64_t cols, int batch) {
+    if (rows < 1 || cols < 64 || cols % 64 != 0 || batch < 1 || batch > hqq::kGemmMaxBatch) return 0;
+    if (cols > 0 && rows > (INT64_MAX / 16) / cols) return 0;
+    return hqq::gemm_workspace_bytes(rows, cols, batch);
+}
+
 int hqq_gemm(const void* W_q_packed, const void* scale, const void* zero, const void* zero_meta, int64_t rows,
              int64_t cols, int nbits, int group_size, int zero_nbits, const void* x, int x_dtype, int batch, float* y,
-             void* stream) {
+             void* workspace, size_t workspace_bytes, void* stream) {
     if (x_dtype != HQQ_F16 && x_dtype != HQQ_BF16) return HQQ_ERR_DTYPE;
     if (!valid_nbits(nbits) || batch < 1 || batch > hqq::kGemmMaxBatch) return HQQ_ERR_INVALID_ARG;
     const int sh = check_shape(rows, cols, group_size, 1);
@@ -278,6 +284,7 @@ int hqq_gemm(const void* W_q_packed, const void* scale, const void* zero, const 
     if (!aligned(W_q_packed, 16) || !aligned(scale, 2) || !aligned(x, 16) || !aligned(y, 4)) return HQQ_ERR_ALIGN;
     if (zero_nbits == 16 && !aligned(zero, 2)) return HQQ_ERR_ALIGN;
     if (zero_nbits == 8 && !aligned(zero_meta, 4)) return HQQ_ERR_ALIGN;
+    if (workspace != nullptr && (!is_device_ptr(workspace) || !aligned(workspace, 256))) return HQQ_ERR_INVALID_ARG;
     hqq::GemvArgs a{};
     a.packed = static_cast<const uint8_t*>(W_q_packed);
     a.scale = static_cast<const uint16_t*>(scale);
@@ -292,6 +299,8 @@ int hqq_gemm(const void* W_q_packed, const void* scale, const void* zero, const 
     a.x_dtype = x_dtype;
     a.batch = batch;
     a.y = y;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace ? workspace_bytes : 0;
     if (hqq::launch_gemm(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
         cudaGetLastError();
         return HQQ_ERR_CUDA;

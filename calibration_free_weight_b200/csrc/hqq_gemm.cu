@@ -179,6 +179,10 @@ struct GemmParams {
     int batch;
     int ntile;          // MMA N: batch rows per CTA, a multiple of 16 in [16, 256]
     int stages;         // S, in [3, kMaxStages]
+    int splits;         // K splits (grid z); 1: each CTA writes y directly
+    int kps;            // K tiles per split
+    float* part;        // splits > 1: [tile][split][ntile][128] fp32 partial tiles
+    uint32_t* tickets;  // splits > 1: [tile] arrival counts, zero at launch
 };
 
 // Inputs of one thread's kWpt consecutive weights of one K tile (one row):
@@ -377,7 +381,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kTileM, n0 = static_cast<int64_t>(blockIdx.y) * p.ntile;
-    const int num_k = static_cast<int>(p.cols / kTileK);
+    // this CTA's K tiles: [kbase, kbase + num_k) of the split blockIdx.z
+    const int kbase = static_cast<int>(blockIdx.z) * p.kps;
+    const int ktot = static_cast<int>(p.cols / kTileK);
+    const int num_k = min(p.kps, ktot - kbase);
     const uint32_t ncols = tmem_columns(p.ntile);
     auto bar = [&](int s) { return bars + 8u * static_cast<uint32_t>(s); };
     auto xbar = [&](int s) { return xbars + 8u * static_cast<uint32_t>(s); };
@@ -414,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
         // registers (global latency hidden behind three tiles of work)
         const int r = tid >> 2, h = tid & 3;
         const int64_t row = m0 + r;
-        auto col = [&](int kt) { return static_cast<int64_t>(kt) * kTileK + kWpt * h; };
+        auto col = [&](int kt) { return static_cast<int64_t>(kbase + kt) * kTileK + kWpt * h; };
         ARaw<NBITS> a0, a1, a2;
         load_a<NBITS, ZB>(p, row, col(0), a0);
         if (num_k > 1) load_a<NBITS, ZB>(p, row, col(1), a1);
@@ -444,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
         const int kPB = S - 2;
         for (int d = 0; d < kPB && d < num_k; ++d) {
             mbar_expect_tx(xbar(d), xbytes);
-            tma_load_2d(stage_b(d), &xmap, d * kTileK, static_cast<int>(n0), xbar(d));
+            tma_load_2d(stage_b(d), &xmap, (kbase + d) * kTileK, static_cast<int>(n0), xbar(d));
         }
         int s = 0, ph = 0, sb = kPB, phb = 0, sl = 0, phl = 0;
         for (int kt = 0; kt < num_k && ok; ++kt) {
@@ -455,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
                     break;
                 }
                 mbar_expect_tx(xbar(sb), xbytes);
-                tma_load_2d(stage_b(sb), &xmap, kb * kTileK, static_cast<int>(n0), xbar(sb));
+                tma_load_2d(stage_b(sb), &xmap, (kbase + kb) * kTileK, static_cast<int>(n0), xbar(sb));
             }
             if (!mbar_wait(abar(s), static_cast<uint32_t>(ph), abort_flag) ||
                 !mbar_wait(xbar(s), static_cast<uint32_t>(ph), abort_flag)) {
@@ -492,10 +499,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
         constexpr int kColWarps = kProducers / 128;
         const int q = warp & 3;
         const int64_t orow = m0 + 32 * q + lane;
+        const int64_t tile = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+        float* const mine = p.splits > 1 ? p.part + (tile * p.splits + blockIdx.z) * p.ntile * kTileM : nullptr;
         for (int c0 = 8 * (warp >> 2); c0 < p.ntile; c0 += 8 * kColWarps) {
             float v[8];
             tmem_ld8(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(c0), v);
-            if (orow < p.rows) {
+            if (mine) {  // this split's partial tile, column-major, rows contiguous
+#pragma unroll
+                for (int i = 0; i < 8; ++i) __stcg(mine + (c0 + i) * kTileM + 32 * q + lane, v[i]);
+            } else if (orow < p.rows) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int64_t b = n0 + c0 + i;
@@ -505,6 +517,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
         }
     } else if (tid == 0) {
         atomicExch(&g_gemm_status, 1u);
+    }
+    if (p.splits > 1) {
+        // the last split of this tile to arrive sums the partials in split order (deterministic)
+        __shared__ int last;
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            const int64_t tile = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+            last = atomicAdd(p.tickets + tile, 1u) == static_cast<uint32_t>(p.splits - 1);
+        }
+        __syncthreads();
+        if (last && !*abort_flag) {
+            __threadfence();
+            const int64_t tile = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+            const float* const base = p.part + tile * p.splits * p.ntile * kTileM;
+            for (int e = tid; e < p.ntile * kTileM; e += kThreads) {
+                const int c = e / kTileM, rr = e % kTileM;
+                const int64_t orow = m0 + rr, b = n0 + c;
+                float acc = 0.0f;
+                for (int z = 0; z < p.splits; ++z) acc = __fadd_rn(acc, __ldcg(base + z * p.ntile * kTileM + e));
+                if (orow < p.rows && b < p.batch) p.y[b * p.rows + orow] = acc;
+            }
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -581,6 +616,53 @@ bool encode_x_map(CUtensorMap* map, const void* x, int bf16, int64_t batch, int6
 
 namespace hqq {
 
+int sm_count() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return 148;  // no device here: the B200's count
+    }
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 148;
+        }
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+// K splits for grids too small to fill the GPU: about one CTA per SM, each
+// split long enough to amortise its pipeline fill and partial-tile traffic
+// (at least 8 K tiles, 40 for batch tiles of 128 and more).  Measured on
+// 4096-row matrices: 4096x11008 batch 256 (4 splits of 43 tiles) 0.132 ->
+// 0.080 ms, 4096x4096 batch 16 (4 of 16) 0.046 -> 0.025 ms; 4096x4096 batch
+// 256 stays unsplit (0.055 ms; 4 splits of 16 tiles 0.059, 2 of 32 0.070).
+int gemm_splits(int64_t rows, int64_t cols, int batch) {
+    int ntile = 0, ntiles = 0;
+    gemm_tiles(batch, &ntile, &ntiles);
+    const int64_t ctas = ((rows + kTileM - 1) / kTileM) * ntiles;
+    const int sms = sm_count();
+    const int64_t ktot = cols / kTileK, min_kps = ntile >= 128 ? 40 : 8;
+    int64_t sp = ctas >= (sms * 3) / 4 ? 1 : sms / ctas;
+    if (sp > ktot / min_kps) sp = ktot / min_kps;
+    return sp < 1 ? 1 : static_cast<int>(sp);
+}
+
+// Workspace of a split product: tickets [tiles] (rounded to 256 bytes), then
+// the fp32 partial tiles; 0 when the product runs unsplit.
+size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int batch) {
+    const int sp = gemm_splits(rows, cols, batch);
+    if (sp <= 1) return 0;
+    int ntile = 0, ntiles = 0;
+    gemm_tiles(batch, &ntile, &ntiles);
+    const int64_t ktot = cols / kTileK, kps = (ktot + sp - 1) / sp, splits = (ktot + kps - 1) / kps;
+    const int64_t tiles = ((rows + kTileM - 1) / kTileM) * ntiles;
+    return static_cast<size_t>(((tiles * 4 + 255) / 256) * 256 + tiles * splits * ntile * kTileM * 4);
+}
+
 // Batch tiles: as few as possible (N <= 256 each), of equal size rounded up to 16.
 void gemm_tiles(int batch, int* ntile, int* ntiles) {
     const int nt = (batch + 255) / 256;
@@ -605,7 +687,21 @@ cudaError_t launch_gemm(const GemvArgs& a, cudaStream_t stream) {
     int ntiles = 1;
     gemm_tiles(a.batch, &p.ntile, &ntiles);
     p.stages = gemm_stages(p.ntile);
-    const dim3 grid(static_cast<unsigned>((a.rows + kTileM - 1) / kTileM), static_cast<unsigned>(ntiles));
+    const int ktot = static_cast<int>(a.cols / kTileK);
+    p.splits = gemm_splits(a.rows, a.cols, a.batch);
+    if (p.splits > 1 && (a.workspace == nullptr || a.workspace_bytes < gemm_workspace_bytes(a.rows, a.cols, a.batch)))
+        p.splits = 1;  // no room for the partials: run unsplit
+    p.kps = (ktot + p.splits - 1) / p.splits;
+    p.splits = (ktot + p.kps - 1) / p.kps;
+    if (p.splits > 1) {
+        const int64_t tiles = ((a.rows + kTileM - 1) / kTileM) * ((a.batch + p.ntile - 1) / p.ntile);
+        p.tickets = static_cast<uint32_t*>(a.workspace);
+        p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + ((tiles * 4 + 255) / 256) * 256);
+        const cudaError_t e = cudaMemsetAsync(p.tickets, 0, static_cast<size_t>(tiles) * 4, stream);
+        if (e != cudaSuccess) return e;
+    }
+    const dim3 grid(static_cast<unsigned>((a.rows + kTileM - 1) / kTileM), static_cast<unsigned>(ntiles),
+                    static_cast<unsigned>(p.splits));
     const size_t smem = gemm_smem_bytes(p.ntile, p.stages);
     const bool bf16 = a.x_dtype == 1;
     alignas(64) CUtensorMap xmap;

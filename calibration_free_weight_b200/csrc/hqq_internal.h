@@ -83,12 +83,18 @@ struct GemvArgs {
     const void* x;  // [batch][cols] fp16/bf16
     int x_dtype, batch;
     float* y;       // [batch][rows]
+    void* workspace = nullptr;  // split tensor-core products: tickets and partial tiles
+    size_t workspace_bytes = 0;
 };
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t stream);
 // The tensor-core product (batch >= 1, cols a multiple of 64, x 16-byte aligned).
 cudaError_t launch_gemm(const GemvArgs& a, cudaStream_t stream);
 // Batch tiles of launch_gemm: ntiles tiles of ntile (a multiple of 16, <= 256) rows.
 void gemm_tiles(int batch, int* ntile, int* ntiles);
+// K splits launch_gemm uses when its workspace allows, and the bytes that needs (0: unsplit).
+int gemm_splits(int64_t rows, int64_t cols, int batch);
+size_t gemm_workspace_bytes(int64_t rows, int64_t cols, int batch);
+int sm_count();
 // One bounded wait, as the product's, on a barrier nothing arrives on (diagnostic).
 cudaError_t launch_gemm_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
 // Synchronises the stream; 0, 6 (a wait of a product gave up; cleared) or 5 (CUDA error).

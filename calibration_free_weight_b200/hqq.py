@@ -21,7 +21,7 @@ EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_qu
             "hqq_get_status", "hqq_status_string", "hqq_quantize_noalloc", "hqq_quantize_scale8",
             "hqq_dequantize_s8", "hqq_stream_device_bytes", "hqq_quantize_stream", "hqq_gemv",
             "hqq_stream_jobs_device_bytes", "hqq_quantize_stream_jobs", "hqq_gemm", "hqq_gemm_get_status",
-            "hqq_gemm_wait_selftest")
+            "hqq_gemm_wait_selftest", "hqq_gemm_workspace_bytes")
 
 
 class hqq_host_matrix(C.Structure):
@@ -68,7 +68,9 @@ def _load():
     L.hqq_gemv.restype = i32
     L.hqq_gemv.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, i32, i32, P, P]
     L.hqq_gemm.restype = i32
-    L.hqq_gemm.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, i32, i32, P, P]
+    L.hqq_gemm.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, P, i32, i32, P, P, sz, P]
+    L.hqq_gemm_workspace_bytes.restype = sz
+    L.hqq_gemm_workspace_bytes.argtypes = [i64, i64, i32]
     L.hqq_gemm_get_status.restype = i32
     L.hqq_gemm_get_status.argtypes = [P]
     L.hqq_gemm_wait_selftest.restype = i32
@@ -175,9 +177,14 @@ def hqq_quantize_stream(mats, n, dtype, nbits, group_size, axis, p, beta, kappa,
 
 
 def hqq_gemm(W_q_packed, scale, zero, zero_meta, rows, cols, nbits, group_size, zero_nbits, x, x_dtype, batch, y,
-             stream=None):
+             workspace=None, workspace_bytes=0, stream=None):
     return lib.hqq_gemm(_ptr(W_q_packed), _ptr(scale), _ptr(zero), _ptr(zero_meta), rows, cols, nbits, group_size,
-                        zero_nbits, _ptr(x), x_dtype, batch, _ptr(y), _stream(stream))
+                        zero_nbits, _ptr(x), x_dtype, batch, _ptr(y), _ptr(workspace), workspace_bytes,
+                        _stream(stream))
+
+
+def hqq_gemm_workspace_bytes(rows, cols, batch):
+    return lib.hqq_gemm_workspace_bytes(rows, cols, batch)
 
 
 def hqq_gemm_get_status(stream=None):
@@ -295,16 +302,24 @@ def quantize_stream(Ws, outs, nbits=4, group_size=64, axis=1, p=0.7, beta=1.0, k
     return device_buffer
 
 
-def gemm(q, x, rows, cols, nbits, group_size, zero_nbits=16, out=None, stream=None):
+def gemm(q, x, rows, cols, nbits, group_size, zero_nbits=16, out=None, workspace=None, split=True, stream=None):
     """y = round16(dequant(W)) @ x.T on the tensor cores for the outputs of
     quantize() (axis 1, cols a multiple of 64) and a CUDA [batch, cols]
-    fp16/bf16 tensor x; returns fp32 [batch, rows]."""
+    fp16/bf16 tensor x; returns fp32 [batch, rows].  With split (default) a
+    workspace is allocated when the shape is split along K (or the one given
+    is used)."""
     if x.dtype not in _DT or not x.is_cuda or x.dim() != 2 or not x.is_contiguous():
         raise HQQError(HQQ_ERR_INVALID_ARG, "gemm expects a contiguous 2-D CUDA fp16/bf16 x")
     if out is None:
         out = torch.empty(x.shape[0], rows, dtype=torch.float32, device=x.device)
+    need = hqq_gemm_workspace_bytes(rows, cols, x.shape[0]) if split else 0
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    if not need:
+        workspace = None
     rc = hqq_gemm(q["packed"], q["scale"], q["zero"], q.get("zero_meta"), rows, cols, nbits, group_size, zero_nbits,
-                  x, _DT[x.dtype], x.shape[0], out, stream)
+                  x, _DT[x.dtype], x.shape[0], out, workspace, workspace.numel() if workspace is not None else 0,
+                  stream)
     if rc != HQQ_OK:
         raise HQQError(rc, "hqq_gemm")
     return out

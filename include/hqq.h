@@ -302,14 +302,25 @@ int hqq_gemv(const void* W_q_packed, const void* scale, const void* zero, const 
  * [out, in] = [rows, cols] weight); cols must be a multiple of 64.
  * W_q_packed, scale, zero, zero_meta as produced by hqq_quantize.  x: device
  * [batch][cols] fp16/bf16, 16-byte aligned; y: device fp32 [batch][rows],
- * 4-byte aligned.  Returns HQQ_OK, HQQ_ERR_DTYPE, HQQ_ERR_SHAPE,
- * HQQ_ERR_INVALID_ARG (batch out of range, bad pointer), HQQ_ERR_ALIGN or
- * HQQ_ERR_CUDA.  Allocates nothing.  Every wait inside the kernel is bounded
- * (about 1 s); a wait that gives up is reported by hqq_gemm_get_status.
+ * 4-byte aligned.  workspace (may be NULL): device memory of at least
+ * hqq_gemm_workspace_bytes(rows, cols, batch), 256-byte aligned, caller-owned;
+ * with it, a product whose 128-row x batch tiles are too few to fill the GPU
+ * splits K across CTAs and the last split of each tile sums the partial tiles
+ * in split order (the result is deterministic, but its fp32 summation order,
+ * within the bound above, differs from the unsplit product's); without it, or
+ * when it is smaller, the product runs unsplit.  Returns HQQ_OK,
+ * HQQ_ERR_DTYPE, HQQ_ERR_SHAPE, HQQ_ERR_INVALID_ARG (batch out of range, bad
+ * pointer), HQQ_ERR_ALIGN or HQQ_ERR_CUDA.  Allocates nothing.  Every wait
+ * inside the kernel is bounded (about 1 s); a wait that gives up is reported
+ * by hqq_gemm_get_status.
  */
 int hqq_gemm(const void* W_q_packed, const void* scale, const void* zero, const void* zero_meta, int64_t rows,
              int64_t cols, int nbits, int group_size, int zero_nbits, const void* x, int x_dtype, int batch, float* y,
-             void* stream);
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes hqq_gemm uses to split K for this shape on the current
+ * device (0: the product runs unsplit; also 0 on invalid sizes). */
+size_t hqq_gemm_workspace_bytes(int64_t rows, int64_t cols, int batch);
 
 /* Synchronises `stream`; HQQ_OK, or HQQ_ERR_TIMEOUT if a hqq_gemm since the
  * last call gave up a wait (its y is then incomplete; the flag is cleared),

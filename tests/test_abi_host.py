@@ -211,17 +211,29 @@ def test_gemm_rejections(hq):
     """hqq_gemm argument checks, all on the host before any launch."""
     L = hq.lib
     a = (None, None, None, None)
-    assert L.hqq_gemm(*a, 128, 128, 4, 64, 16, None, 7, 4, None, None) == hq.HQQ_ERR_DTYPE
-    assert L.hqq_gemm(*a, 128, 128, 5, 64, 16, None, 1, 4, None, None) == hq.HQQ_ERR_INVALID_ARG
-    assert L.hqq_gemm(*a, 128, 128, 4, 64, 16, None, 1, 0, None, None) == hq.HQQ_ERR_INVALID_ARG
-    assert L.hqq_gemm(*a, 128, 128, 4, 64, 16, None, 1, 65537, None, None) == hq.HQQ_ERR_INVALID_ARG
-    assert L.hqq_gemm(*a, 128, 96, 4, 32, 16, None, 1, 4, None, None) == hq.HQQ_ERR_SHAPE  # cols % 64
-    assert L.hqq_gemm(*a, 128, 128, 4, 48, 16, None, 1, 4, None, None) == hq.HQQ_ERR_SHAPE
-    assert L.hqq_gemm(*a, 128, 128, 4, 64, 12, None, 1, 4, None, None) == hq.HQQ_ERR_INVALID_ARG
-    assert L.hqq_gemm(*a, 0, 128, 4, 64, 16, None, 1, 4, None, None) == hq.HQQ_OK
+    assert L.hqq_gemm(*a, 128, 128, 4, 64, 16, None, 7, 4, None, None, 0, None) == hq.HQQ_ERR_DTYPE
+    assert L.hqq_gemm(*a, 128, 128, 5, 64, 16, None, 1, 4, None, None, 0, None) == hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_gemm(*a, 128, 128, 4, 64, 16, None, 1, 0, None, None, 0, None) == hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_gemm(*a, 128, 128, 4, 64, 16, None, 1, 65537, None, None, 0, None) == hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_gemm(*a, 128, 96, 4, 32, 16, None, 1, 4, None, None, 0, None) == hq.HQQ_ERR_SHAPE  # cols % 64
+    assert L.hqq_gemm(*a, 128, 128, 4, 48, 16, None, 1, 4, None, None, 0, None) == hq.HQQ_ERR_SHAPE
+    assert L.hqq_gemm(*a, 128, 128, 4, 64, 12, None, 1, 4, None, None, 0, None) == hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_gemm(*a, 0, 128, 4, 64, 16, None, 1, 4, None, None, 0, None) == hq.HQQ_OK
     buf = C.create_string_buffer(4096)
     p = C.cast(buf, C.c_void_p).value
-    assert L.hqq_gemm(p, p, p, None, 128, 128, 4, 64, 16, p, 1, 4, p, None) == hq.HQQ_ERR_INVALID_ARG
+    assert L.hqq_gemm(p, p, p, None, 128, 128, 4, 64, 16, p, 1, 4, p, None, 0, None) == hq.HQQ_ERR_INVALID_ARG
+
+
+def test_gemm_workspace_query(hq):
+    """Split products need tickets and partial tiles; the query is 0 for
+    shapes whose tiles already fill the GPU and for invalid sizes."""
+    assert hq.hqq_gemm_workspace_bytes(28672, 8192, 256) == 0  # 224 tiles
+    w = hq.hqq_gemm_workspace_bytes(4096, 11008, 256)          # 32 tiles, 172 K tiles: split
+    assert w > 0 and w >= 4096 * 256 * 4 * 2
+    assert hq.hqq_gemm_workspace_bytes(4096, 4096, 256) == 0   # 64 K tiles: too short to split
+    assert hq.hqq_gemm_workspace_bytes(4096, 4096, 16) > 0     # narrow batch tile: split
+    assert hq.hqq_gemm_workspace_bytes(4096, 100, 16) == 0     # cols not a multiple of 64
+    assert hq.hqq_gemm_workspace_bytes(4096, 4096, 0) == 0
 
 
 def test_gemm_wait_selftest_rejects_bad_limits(hq):

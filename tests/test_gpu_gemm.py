@@ -152,3 +152,31 @@ def test_gemm_bounded_wait_gives_up_and_reports(hq):
     y = run(hq, q, x, rows, cols, nbits, g, zb)
     yo, ya = oracle.gemm(q["packed"], q["scale"], q["zero"], q["zero_meta"], rows, cols, nbits, g, zb, xo, xdt)
     check(y, yo, ya, cols)
+
+
+@pytest.mark.parametrize("rows,cols,batch", [(512, 4096, 16), (4096, 11008, 256), (1000, 8192, 40), (4096, 4096, 16)])
+def test_gemm_split_k(hq, rows, cols, batch):
+    """Grids too small for the GPU split K across CTAs; the last split of each
+    tile sums the partials in split order: within the bound of the oracle,
+    within twice the bound of the unsplit product, and bit-identical on
+    repeated calls."""
+    nbits, g, zb = 4, 64, 8
+    assert hq.hqq_gemm_workspace_bytes(rows, cols, batch) > 0
+    q = make_q(rows, cols, nbits, g, zb, seed=rows + batch)
+    x, xo, xdt = make_x(batch, cols, torch.bfloat16, seed=batch)
+    d = {k: (torch.from_numpy(v).cuda() if v is not None else None) for k, v in q.items()}
+    xc = x.cuda()
+    ys = hq.gemm(d, xc, rows, cols, nbits, g, zb)
+    ys2 = hq.gemm(d, xc, rows, cols, nbits, g, zb)
+    yu = hq.gemm(d, xc, rows, cols, nbits, g, zb, split=False)
+    assert hq.hqq_gemm_get_status() == hq.HQQ_OK
+    assert torch.equal(ys, ys2)
+    ys, yu = ys.cpu().numpy().astype(np.float64), yu.cpu().numpy().astype(np.float64)
+    sample = np.unique(np.r_[0, rows - 1, np.random.default_rng(2).choice(rows, 24, replace=False)])
+    bpr, gpr = cols * nbits // 8, cols // g
+    for r0 in sample:
+        yo, ya = oracle.gemm(q["packed"][r0 * bpr:(r0 + 1) * bpr], q["scale"][r0 * gpr:(r0 + 1) * gpr],
+                             q["zero"][r0 * gpr:(r0 + 1) * gpr], q["zero_meta"], 1, cols, nbits, g, zb, xo, xdt)
+        check(ys[:, r0:r0 + 1], yo, ya, cols)
+        check(yu[:, r0:r0 + 1], yo, ya, cols)
+        assert np.all(np.abs(ys[:, r0:r0 + 1] - yu[:, r0:r0 + 1]) <= 2 * cols * 2.0 ** -23 * ya + 1e-30)
