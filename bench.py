@@ -50,16 +50,22 @@ KERNEL_SOURCES = ["calibration_free_weight_b200/csrc/hqq_kernels.cu", "calibrati
 # launch), averaged over the timed step's tensor-stop calls,
 # from the ncu launch list summarised in profiles/ (taken on the kernel sources
 # whose sha256 is recorded here; None until a capture exists).
-TRAFFIC = {"src_sha256": "46f27c58d4c01e2788eb81495396900f6a1351042cc803321971036b3d7b0eed",
+TRAFFIC = {"src_sha256": "2a27860d0d38b7224791bf0cb5d250c7aed7d1f9553c0ac9e65c4dc2b05037f5",
            "bytes_per_call": 381103462, "summary": "profiles/launches_llama2-7b-mlp-sweep.md"}
 
 
 def kernel_sources_sha():
+    """sha256 of the solver's kernel sources with comments and blank lines
+    removed: a change of code, not of commentary, invalidates the stored
+    DRAM-traffic counters."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f)) as fh:
+            src = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+        lines = (re.sub(r"//.*", "", ln).rstrip() for ln in src.splitlines())
+        h.update("\n".join(ln for ln in lines if ln).encode())
     return h.hexdigest()
 
 

@@ -9,8 +9,9 @@
 // the per-element evaluation is in hqq_device.cuh.
 //
 // The path has no dense contraction: no tensor cores.  Each element and
-// evaluation costs ~7 FP32-pipe instructions and two MUFU ops (|r|^p through
-// lg2/ex2), so the MUFU pipe, not HBM, bounds the solver.
+// evaluation costs 7 fp32 operations, six of them issued as packed pairs
+// (add/sub/mul.rn.f32x2), and two MUFU ops (|r|^p through lg2/ex2), so the
+// MUFU pipe, not HBM, bounds the solver.
 //
 // Both solver kernels hold a warp tile of 32/P groups in registers, E = g/P
 // elements per lane (E = min(g, 32)), and re-read W from HBM rather than keep
@@ -27,11 +28,15 @@
 //   lanes of a warp stay busy: a tile only runs as long as its slowest group
 //   within one pass.
 // solve_tensor_kernel (tensor stop): runs iterations [k0, k1) of every group,
-//   accumulates the per-iteration tensor error in fp64 per CTA, and the last
-//   CTA to finish (atomic ticket) sums the partials in a fixed order.  The next
-//   launch reads those sums, applies the stop rule, and either runs the next
-//   chunk or writes the final codes with the kept iterate (recomputed from the
-//   stored chunk-start zero with the cheap part of the iteration).
+//   stores the zero-point of each of them, accumulates the per-iteration tensor
+//   error per CTA, and the last CTA to finish (atomic ticket) sums the partials
+//   in a fixed order, applies the stop rule to the errors so far and leaves
+//   its outcome (first rise, kept iterate) in two workspace header words.  The
+//   next launch reads those words and either runs the next chunk or returns.
+//   The outputs: without debug outputs (axis 1) the last chunk writes those of
+//   its last iterate (g >= 32), and tensor_output_kernel rewrites them from the
+//   kept iterate's stored zero-point only when a tensor error rose; otherwise
+//   the chunk kernel's own output launch writes them.
 
 #include "hqq_device.cuh"
 
