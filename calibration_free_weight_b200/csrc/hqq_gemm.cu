@@ -427,6 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
         if (num_k > 1) load_a<NBITS, ZB>(p, row, col(1), a1);
         if (num_k > 2) load_a<NBITS, ZB>(p, row, col(2), a2);
         int s = 0, ph = 0;  // stage of tile kt and the parity of its use of that stage
+#pragma unroll 4
         for (int kt = 0; kt < num_k; ++kt) {
             ARaw<NBITS> a3;
             if (kt + 3 < num_k) load_a<NBITS, ZB>(p, row, col(kt + 3), a3);
