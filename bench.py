@@ -54,14 +54,22 @@ TRAFFIC = {"src_sha256": "2a27860d0d38b7224791bf0cb5d250c7aed7d1f9553c0ac9e65c4d
            "bytes_per_call": 381103462, "summary": "profiles/launches_llama2-7b-mlp-sweep.md"}
 
 
-def kernel_sources_sha():
-    """sha256 of the solver's kernel sources with comments and blank lines
-    removed: a change of code, not of commentary, invalidates the stored
-    DRAM-traffic counters."""
+# DRAM traffic of one hqq_gemm call in the profiled case (ncu, same command as
+# the summary), valid while hqq_gemm.cu hashes to the profiled source.
+GEMM_SOURCES = ["calibration_free_weight_b200/csrc/hqq_gemm.cu"]
+GEMM_TRAFFIC = {"src_sha256": "6047c8fb4337f86155429e2a54e5e1946effb14b71f0514dd011fdf3db4ae611",
+                "case": "gemm,28672,8192,4,64,256", "bytes_per_call": 141282304,
+                "summary": "profiles/gemm_kernel_28672x8192_b4g64_batch256.md"}
+
+
+def kernel_sources_sha(files=None):
+    """sha256 of kernel sources (default: the solver's) with comments and
+    blank lines removed: a change of code, not of commentary, invalidates the
+    stored DRAM-traffic counters."""
     import hashlib
     import re
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in files or KERNEL_SOURCES:
         with open(os.path.join(ROOT, f)) as fh:
             src = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
         lines = (re.sub(r"//.*", "", ln).rstrip() for ln in src.splitlines())
@@ -583,7 +591,15 @@ def run_gemm_case(spec):
     oracle.gemm(qc["packed"][:sr * cols * nbits // 8], qc["scale"][:sr * cols // g], qc["zero"][:sr * cols // g],
                 qc["zero_meta"], sr, cols, nbits, g, 8, xo, oracle.BF16)
     ot = time.perf_counter() - t0
-    print(json.dumps({"case": spec, "ms_median": med, "ms_min": ms[0], "tflops": flops / (med / 1e3) / 1e12,
+    achieved = flops / (med / 1e3) / 1e12
+    same = ",".join(spec.split(",")[:6]) == GEMM_TRAFFIC["case"] and \
+        kernel_sources_sha(GEMM_SOURCES) == GEMM_TRAFFIC["src_sha256"]
+    print(json.dumps({"case": spec, "ms_median": med, "ms_min": ms[0], "tflops": achieved,
+                      "roofline": {"bound": "tensor", "kernel": "gemm_kernel", "achieved": achieved, "peak": tf,
+                                   "unit": "TFLOP/s", "frac": achieved / tf if tf else None,
+                                   "peak_basis": "measured bf16 GEMM (burst)",
+                                   "traffic": GEMM_TRAFFIC["bytes_per_call"] if same else None,
+                                   "traffic_unit": "bytes per call", "algorithmic_bytes_per_call": nbytes},
                       "cpu_baseline": {"value": 2.0 * sr * cols * batch / ot / 1e12, "unit": "TFLOP/s", "cores": 1,
                                        "kind": "oracle", "sample": f"first {sr} rows, all columns, batch {batch}"},
                       "bf16_peak_tflops": tf, "tensor_frac": (flops / (med / 1e3) / 1e12 / tf) if tf else None,
