@@ -250,6 +250,26 @@ def oracle_sample_rate(layer, budget_s=12.0, nthreads=0):
     return n / dt, nth, oracle_desc(rows, n), n, dt
 
 
+def oracle_model_rate(Ws, settings, weights_total, rows=64, nthreads=0):
+    """The CPU oracle, as it stands, on a deterministic sample of a streamed
+    model: the first `rows` rows of each of one layer's matrices (host fp16
+    tensors) with that matrix's settings; the whole model's oracle time is
+    extrapolated from the sample's weights/s.  Returns a cpu_baseline dict."""
+    import oracle
+    nth = nthreads or (os.cpu_count() or 1)
+    n, t0 = 0, time.perf_counter()
+    for W, st in zip(Ws, settings):
+        w = W[:rows].contiguous().numpy()
+        oracle.quantize(w, st["nbits"], st["group_size"], 1, 0.7, 1.0, 1.01, 20, st["stop_mode"], st["zero_nbits"],
+                        dtype=oracle.F16, nthreads=nth)
+        n += w.size
+    dt = time.perf_counter() - t0
+    rate = n / dt
+    return {"value": rate / 1e9, "unit": "Gweights/s", "cores": nth, "kind": "oracle",
+            "sample": f"first {rows} rows of each matrix of one layer, {n / 1e6:.2f} M weights, "
+                      f"fp16, OpenMP over groups", "extrapolated_model_s": weights_total / rate}
+
+
 # ------------------------------------------------------------------- main ---
 
 def dist_setup(backend="nccl"):
@@ -421,7 +441,12 @@ def run_stream(args):
         hbm, _, kind = peaks()
         h2d = 2 * w_layer * layers
         d2h = sum(o["packed"].numel() + o["scale"].numel() * 2 + o["zero"].numel() + 8 for o in outs) * layers
+        cpu = None
+        if rank == 0:
+            sets = [dict(nbits=nbits, group_size=g, stop_mode=0, zero_nbits=8)] * len(Ws)
+            cpu = oracle_model_rate(Ws, sets, w_layer * layers)
         res.append({"nbits": nbits, "group_size": g, "e2e_s": wall, "e2e_gweights_s": w_layer * layers / wall / 1e9,
+                    "cpu_baseline": cpu,
                     "h2d_bytes": h2d, "d2h_bytes": d2h, "h2d_gbs_effective": h2d / wall / 1e9,
                     "device_resident": {"ms_per_layer": layer_ms, "gweights_s": w_layer / (layer_ms / 1e3) / 1e9,
                                         "algorithmic_gbs": alg / (layer_ms / 1e3) / 1e9,
@@ -490,7 +515,8 @@ def run_stream_mixed(args):
     h2d = 2 * w_layer * layers
     d2h = sum(o["packed"].numel() + o["scale"].numel() * 2 + o["zero"].numel() * 2 for o in outs) * layers
     if rank == 0:
-        print(json.dumps({"workload": "llama2-13b-stream", "layers": layers, "weights": w_layer * layers,
+        cpu = oracle_model_rate(Ws, sets, w_layer * layers)
+        print(json.dumps({"workload": "llama2-13b-stream", "cpu_baseline": cpu, "layers": layers, "weights": w_layer * layers,
                           "n_gpus": world, "scaling": "layers split across ranks", "dtype_in": "fp16",
                           "settings": {"attn (q, k, v, o)": sets[0], "mlp (gate, up, down)": sets[4]},
                           "zero": "fp16", "host": "pinned", "matrices_done_rank0": done,

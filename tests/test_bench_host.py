@@ -8,6 +8,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
+import torch  # noqa: E402
+from calibration_free_weight_b200 import synth  # noqa: E402
 
 
 def test_solver_launches_follow_the_schedules():
@@ -48,3 +50,16 @@ def test_plan_and_bytes():
     assert bench.algorithmic_bytes(4096, 4096, 4, 64) == 4096 * 4096 * 2.5625
     # consecutive calls never reuse the previous call's matrix
     assert all(a[0] != b[0] for a, b in zip(calls, calls[1:]))
+
+
+def test_oracle_model_rate_extrapolates_from_its_sample():
+    """The streamed workloads' CPU baseline: the oracle on the first rows of one
+    layer's matrices, with each matrix's settings, extrapolated to the model."""
+    import bench
+    Ws = [synth.weight(32, 256, seed=1, dtype=torch.float16), synth.weight(32, 512, seed=2, dtype=torch.float16)]
+    sets = [dict(nbits=4, group_size=64, stop_mode=1, zero_nbits=16),
+            dict(nbits=2, group_size=32, stop_mode=0, zero_nbits=8)]
+    cb = bench.oracle_model_rate(Ws, sets, 1e9, rows=16, nthreads=1)
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] > 0
+    assert abs(cb["extrapolated_model_s"] - 1e9 / (cb["value"] * 1e9)) < 1e-6 * cb["extrapolated_model_s"]
+    assert "first 16 rows" in cb["sample"]
