@@ -236,6 +236,34 @@ def test_gemm_workspace_query(hq):
     assert hq.hqq_gemm_workspace_bytes(4096, 4096, 0) == 0
 
 
+def _gemm_ws_expected(rows, cols, batch, sms=148):
+    """The split policy and workspace size of hqq_gemm, restated: batch tiles
+    of at most 256 rows (equal, multiples of 16); a grid under 3/4 of the SMs
+    splits K into sms // ctas parts, each at least 8 K tiles (40 for batch
+    tiles >= 128); tickets (rounded to 256 bytes) then fp32 partial tiles."""
+    nt = (batch + 255) // 256
+    ntile = ((batch + nt - 1) // nt + 15) // 16 * 16
+    ctas = ((rows + 127) // 128) * nt
+    ktot = cols // 64
+    sp = 1 if ctas >= sms * 3 // 4 else sms // ctas
+    sp = min(sp, ktot // (40 if ntile >= 128 else 8))
+    if sp <= 1:
+        return 0
+    kps = (ktot + sp - 1) // sp
+    splits = (ktot + kps - 1) // kps
+    tiles = ((rows + 127) // 128) * nt
+    return (tiles * 4 + 255) // 256 * 256 + tiles * splits * ntile * 128 * 4
+
+
+@pytest.mark.parametrize("rows,cols,batch", [(4096, 11008, 256), (4096, 4096, 16), (512, 4096, 16), (1000, 8192, 40),
+                                             (4096, 4096, 256), (11008, 4096, 256), (256, 1024, 1), (128, 64, 1),
+                                             (4096, 28672, 512), (8192, 8192, 300)])
+def test_gemm_split_policy(hq, rows, cols, batch):
+    """With no GPU the library assumes the B200's 148 SMs, so the policy is
+    checked here against its restatement."""
+    assert hq.hqq_gemm_workspace_bytes(rows, cols, batch) == _gemm_ws_expected(rows, cols, batch)
+
+
 def test_gemm_wait_selftest_rejects_bad_limits(hq):
     assert hq.lib.hqq_gemm_wait_selftest(0, None) == hq.HQQ_ERR_INVALID_ARG
     assert hq.lib.hqq_gemm_wait_selftest(1000001, None) == hq.HQQ_ERR_INVALID_ARG
