@@ -53,7 +53,9 @@
  *
  * Conventions for every call:
  *   - All buffers are caller-owned device memory (cudaMalloc, torch, ...).
- *     The library never allocates or frees.
+ *     The library allocates and frees no device memory (hqq_quantize_noalloc
+ *     uses a static device array of the library; the stream executors create
+ *     and destroy their own copy streams and events within the call).
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL = legacy default stream).  Argument errors are detected on the host
  *     and returned before anything is launched; no output is touched then.
