@@ -59,6 +59,10 @@ MUTANTS = [
     ("gemm-drops-zero", "const float wr = (q - z) * from_f16(scale[grp]);", "const float wr = q * from_f16(scale[grp]);",
      1),
     ("gemm-signed-abs-sum", "yabs[b * rows + r] += fabs(p);", "yabs[b * rows + r] += p;", 1),
+    ("groups-axis0-index", "int64_t j = group_ids[k];\n            for (int i = 0; i < g; ++i) w[i] = load_elem(W, dtype, elem_index(j, i, cols, g, axis));",
+     "int64_t j = group_ids[k];\n            for (int i = 0; i < g; ++i) w[i] = load_elem(W, dtype, elem_index(j, i, cols, g, 1));", 1),
+    ("groups-levels-reversed", "levels[k * g + i] = (uint8_t)quantize_elem(w[i], res.s, res.zbest, L);",
+     "levels[k * g + (g - 1 - i)] = (uint8_t)quantize_elem(w[i], res.s, res.zbest, L);", 1),
     ("pack-msb-first", "unsigned v = level << off; /* at most 8 + 7 bits */",
      "unsigned v = (off + b <= 8 ? level << (8 - b - off) : level << off);", 1),
 ]

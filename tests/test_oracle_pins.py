@@ -677,3 +677,34 @@ def test_gemm_equals_gemv_when_weights_are_16_bit_exact(orc):
     y16, _ = orc.gemm(packed, sc, z, None, rows, cols, nb, g, 16, _bf16_bits(x), orc.BF16)
     y32 = orc.gemv(packed, sc, z, None, rows, cols, nb, g, 16, _bf16_bits(x), orc.BF16)
     assert np.array_equal(y16, y32)
+
+
+# ------------------------------------------------- sampled-group solver ----
+
+@pytest.mark.parametrize("axis", [0, 1])
+@pytest.mark.parametrize("g,nbits", [(8, 4), (1024, 2)])
+@pytest.mark.parametrize("mode", [0, 2])
+def test_quantize_groups_equals_whole_tensor(orc, axis, g, nbits, mode):
+    """oracle_quantize_groups (the checker of every sampled full-size GPU case)
+    returns, for each listed group, exactly what the whole-tensor oracle
+    returns for it: codes, scale, kept zero, kept iterate and its error.  The
+    list holds the first and last group, is unsorted and repeats ids."""
+    long_, short = (2048, 6) if g == 1024 else (40, 24)
+    rows, cols = (short, long_) if axis == 1 else (long_, short)
+    W = _synth_f16(rows, cols, seed=70 + g + axis + mode)
+    full = orc.quantize(W, nbits, g, axis=axis, stop_mode=mode)
+    G = rows * cols // g
+    ids = np.array([G - 1, 0, 5, 5, 3, G - 1, 1, G // 2], np.int64)
+    part = orc.quantize_groups(W, ids, nbits, g, axis=axis, stop_mode=mode)
+    levels = orc.unpack_levels(full["packed"], rows, cols, nbits, axis)
+    for k, j in enumerate(ids):
+        if axis == 1:
+            want = levels.reshape(-1)[j * g:(j + 1) * g]
+        else:
+            rb, c = divmod(int(j), cols)
+            want = levels[rb * g:(rb + 1) * g, c]
+        assert np.array_equal(part["levels"][k], want), f"codes of group {j}"
+        assert np.float16(1.0 / part["s"][k]) == full["scale"][j], f"scale of group {j}"
+        assert part["zbest"][k] == full["zero_f32"][j]
+        assert part["best_iter"][k] == full["best_iter"][j]
+        assert part["best_err"][k] == full["best_err"][j]
