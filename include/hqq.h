@@ -87,16 +87,26 @@ typedef enum { HQQ_F16 = 0, HQQ_BF16 = 1 } hqq_dtype;
 
 typedef enum { HQQ_STOP_GROUP = 0, HQQ_STOP_TENSOR = 1, HQQ_STOP_NONE = 2 } hqq_stop_mode;
 
-/* Bytes of the packed code buffer: rows*cols*nbits/8.  0 for invalid args. */
+/* Bytes of the packed code buffer: rows*cols*nbits/8.  0 for invalid args.
+ * The bit widths are those of "HQQ - Half-Quadratic Quantization"
+ * (skill4agent.com), section "Core concepts" (nbits 1-8, of which the pages
+ * use 8/4/3/2/1); the pages print no storage layout, so the bit stream above
+ * is this library's own. */
 size_t hqq_packed_bytes(int64_t rows, int64_t cols, int nbits, int group_size, int axis);
 
-/* Number of groups G = rows*cols/group_size.  -1 for invalid args. */
+/* Number of groups G = rows*cols/group_size (one scale and one zero each).
+ * -1 for invalid args.  Groups of group_size consecutive weights along `axis`
+ * ("HQQ - Half-Quadratic Quantization" (skill4agent.com), section "Core
+ * concepts": BaseQuantizeConfig(nbits, group_size, axis)). */
 int64_t hqq_num_groups(int64_t rows, int64_t cols, int group_size, int axis);
 
 /* Bytes of device workspace hqq_quantize needs for this problem (always > 0;
- * holds the status word, the work counter, per-CTA partials, the fp32 zeros
- * of the 8-bit zero path and, for the tensor stop, the per-group state and
- * per-iteration errors).  0 for invalid args. */
+ * holds the status word, the work counters, the fp32 kept zeros of the 8-bit
+ * zero path (4 bytes per group, hence zero_nbits), the running state of
+ * groups between passes and, for the tensor stop, the per-group state,
+ * per-CTA partials and per-iteration errors).  0 for invalid args.  The pages
+ * have no counterpart: their solver runs as whole-tensor operations that
+ * allocate as they go; here the caller owns every byte. */
 size_t hqq_workspace_bytes(int64_t rows, int64_t cols, int group_size, int axis, int stop_mode, int zero_nbits);
 
 /*
@@ -135,7 +145,11 @@ int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits
                  void* stream);
 
 /*
- * Dequantise for inspection: W_out = (W_q - zero) * scale computed in fp32 and
+ * Dequantise for inspection ("HQQ - Half-Quadratic Quantization"
+ * (skill4agent.com), section "Core concepts": HQQLinear's dequantize(); the
+ * rule W_r = (W_q - z) / s of techreport.ngo, "Weight-only quantization
+ * without the calibration tax", section "Outlier-aware optimization without
+ * gradients", with scale = 1/s): W_out = (W_q - zero) * scale computed in fp32 and
  * rounded (to nearest even) to out_dtype; with zero_nbits == 8 the zero is
  * first rebuilt as (zq - zz) * (1/sz) from zero_meta.  Buffers as in
  * hqq_quantize; W_out is device out_dtype [rows, cols], 16-byte aligned.
@@ -339,10 +353,11 @@ int hqq_gemm_wait_selftest(int64_t limit_us, void* stream);
 
 /* Synchronise `stream` and return the device status word held in `workspace`
  * by the last hqq_quantize on it (HQQ_OK), or HQQ_ERR_CUDA if the
- * synchronisation or copy fails. */
+ * synchronisation or copy fails.  No counterpart on the pages: the channel for
+ * errors found on the device after an asynchronous call returned. */
 int hqq_get_status(const void* workspace, void* stream);
 
-/* Static English description of a status code. */
+/* Static English description of a status code (no counterpart on the pages). */
 const char* hqq_status_string(int status);
 
 /* Size of the library-owned scratch buffer used by hqq_quantize_noalloc. */
