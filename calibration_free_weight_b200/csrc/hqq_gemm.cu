@@ -520,24 +520,34 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const GemmParams p, c
         atomicExch(&g_gemm_status, 1u);
     }
     if (p.splits > 1) {
-        // the last split of this tile to arrive sums the partials in split order (deterministic)
-        __shared__ int last;
+        // The last split of this tile to arrive sums the partials in split
+        // order (deterministic).  The ticket counts arrivals in its low 16 bits
+        // and splits that gave up a wait in its high bits; if any did, a
+        // partial is missing and the tile of y is filled with NaN instead.
+        __shared__ int last, torn;
         __threadfence();
         __syncthreads();
         if (tid == 0) {
             const int64_t tile = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
-            last = atomicAdd(p.tickets + tile, 1u) == static_cast<uint32_t>(p.splits - 1);
+            const uint32_t inc = *abort_flag ? (1u << 16) + 1u : 1u;
+            const uint32_t old = atomicAdd(p.tickets + tile, inc);
+            last = (old & 0xffffu) == static_cast<uint32_t>(p.splits - 1);
+            torn = (old >> 16) != 0u || *abort_flag;
         }
         __syncthreads();
-        if (last && !*abort_flag) {
+        if (last) {
             __threadfence();
             const int64_t tile = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
             const float* const base = p.part + tile * p.splits * p.ntile * kTileM;
             for (int e = tid; e < p.ntile * kTileM; e += kThreads) {
                 const int c = e / kTileM, rr = e % kTileM;
                 const int64_t orow = m0 + rr, b = n0 + c;
-                float acc = 0.0f;
-                for (int z = 0; z < p.splits; ++z) acc = __fadd_rn(acc, __ldcg(base + z * p.ntile * kTileM + e));
+                float acc = __int_as_float(0x7fc00000);  // NaN
+                if (!torn) {
+                    acc = 0.0f;
+                    for (int z = 0; z < p.splits; ++z)
+                        acc = __fadd_rn(acc, __ldcg(base + z * p.ntile * kTileM + e));
+                }
                 if (orow < p.rows && b < p.batch) p.y[b * p.rows + orow] = acc;
             }
         }

@@ -1400,9 +1400,10 @@ int64_t fit_slice(int64_t rows, int64_t cols, int g, int axis, int stop_mode, in
     if (stop_mode == 1) return 0;
     const WorkspaceLayout base = workspace_layout(rows, cols, g, axis, stop_mode, zero_nbits, 1);
     const size_t fixed = base.state;  // header and kept zeros
-    const size_t per = 44, pad = 4 * 256;
-    if (bytes < fixed + pad) return 0;
-    int64_t s = static_cast<int64_t>((bytes - fixed - pad) / per) & ~static_cast<int64_t>(31);
+    const size_t per = 44;            // bytes per entry of a slice, before each part's rounding to 256
+    if (bytes < fixed) return 0;
+    // the largest multiple of 32 entries whose parts, each rounded up to 256 bytes, fit
+    int64_t s = static_cast<int64_t>((bytes - fixed) / per) & ~static_cast<int64_t>(31);
     while (s >= kMinSlice && workspace_layout(rows, cols, g, axis, stop_mode, zero_nbits, s).total > bytes) s -= 32;
     return s >= kMinSlice ? s : 0;
 }

@@ -339,8 +339,10 @@ int hqq_gemm(const void* W_q_packed, const void* scale, const void* zero, const 
 size_t hqq_gemm_workspace_bytes(int64_t rows, int64_t cols, int batch);
 
 /* Synchronises `stream`; HQQ_OK, or HQQ_ERR_TIMEOUT if a hqq_gemm since the
- * last call gave up a wait (its y is then incomplete; the flag is cleared),
- * or HQQ_ERR_CUDA. */
+ * last call gave up a wait (the flag is then cleared), or HQQ_ERR_CUDA.
+ * After HQQ_ERR_TIMEOUT the y of that product is undefined: a tile whose CTA
+ * gave up keeps whatever y held before, and a tile of a split product that
+ * lost one of its partials is filled with NaN. */
 int hqq_gemm_get_status(void* stream);
 
 /* Diagnostic of the bounded waits: one thread runs hqq_gemm's mbarrier wait,
@@ -377,11 +379,14 @@ const char* hqq_status_string(int status);
  * Scratch: one buffer of HQQ_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory per
  * GPU, held by the library from load until the process exits.  A problem whose
  * hqq_workspace_bytes() exceeds it runs in slices of groups, one after another
- * on `stream` (same results); each slice needs 44 bytes per group and at least
- * 4,096 groups.  With zero_nbits = 8 the kept zeros of all groups (4 bytes each)
- * must fit beside one slice: more than 4,149,184 groups (4 bytes per group plus
- * 180,480 fixed bytes) returns HQQ_ERR_WORKSPACE before anything is launched.
- * With zero_nbits = 16 every size fits.
+ * on `stream` (same results); each slice needs 44 bytes per entry and at least
+ * 4,096 entries (an entry is a group; with axis = 0 the columns of each block
+ * of group_size rows are counted up to whole warp tiles of 32/P groups, P =
+ * group_size/32 for group_size >= 32, else 1).  With zero_nbits = 8 the kept
+ * zeros of all groups (4 bytes each, the array rounded up to 256 bytes) must
+ * fit beside one slice and a 256-byte header: 4,149,184 groups fit exactly,
+ * more return HQQ_ERR_WORKSPACE before anything is launched.  With
+ * zero_nbits = 16 every size fits.
  * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
  * routine).  The first call on each device looks up the buffer's device
  * address (cudaGetSymbolAddress) with that device current; make that first call
