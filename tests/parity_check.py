@@ -237,3 +237,104 @@ def check_zero8(gpu, orc):
     zg = (gz - gm[1]) * gm[0]
     zo = (oz - om[1]) * om[0]
     assert np.all(np.abs(zg - zo) <= Z_TOL * np.maximum(np.abs(zo), 1.0) + gm[0] * 1.0001)
+
+
+def check_stored(W_cpu, params, out, orc=None, sample=None):
+    """Compare stored outputs only -- codes, scale, zero and zero_meta, what a
+    streamed run returns (numpy dict, no debug outputs) -- with the oracle.
+
+    Bars as in check(): scale within 1e-3 relative; a 16-bit zero within
+    1e-3 * max(|z*|, 1) plus half its fp16 step; an 8-bit zero, dequantised with
+    the stored pair, within half a quantiser step (plus 1e-3) of the oracle's
+    z*; codes identical except <= 1e-4 of elements, each within one level.  A
+    group that misses these bars is accepted only as a near tie: some iterate
+    k that the oracle's own error trajectory allows (near ties, TIE_TOL) must
+    reproduce its codes and zero; such groups stay <= 1e-4 of groups (+1).
+    With sample= (group / no stop) only those groups are solved by the oracle.
+    Returns a report dict; raises AssertionError."""
+    nb, g, axis = params["nbits"], params["group_size"], params["axis"]
+    p, beta, kappa, iters = params["p"], params["beta"], params["kappa"], params["iters"]
+    mode, zb = params["stop_mode"], params["zero_nbits"]
+    rows, cols = W_cpu.shape
+    G = rows * cols // g
+    Wo, dt = w_for_oracle(W_cpu)
+    Wf = w_float(W_cpu)
+    gl = oracle.unpack_levels(out["packed"], rows, cols, nb, axis)
+    if sample is not None:
+        assert mode != oracle.STOP_TENSOR
+        ids = np.asarray(sample, np.int64)
+        o = oracle.quantize_groups(Wo, ids, nb, g, axis, p, beta, kappa, iters, mode, dtype=dt)
+        o_levels, o_z, o_bi = o["levels"], o["zbest"], o["best_iter"]
+        o_scale = (1.0 / o["s"]).astype(np.float16)
+    else:
+        if orc is None:
+            orc = oracle.quantize(Wo, nb, g, axis, p, beta, kappa, iters, mode, zb, dtype=dt)
+        ids = np.arange(G)
+        o_levels = all_groups(oracle.unpack_levels(orc["packed"], rows, cols, nb, axis), g, axis)
+        o_z, o_bi, o_scale = orc["zero_f32"], orc["best_iter"], orc["scale"]
+    g_levels = all_groups(gl, g, axis)[ids]
+
+    gs, os_ = out["scale"][ids].astype(np.float64), o_scale.astype(np.float64)
+    assert np.all(np.abs(gs - os_) <= 1e-3 * np.abs(os_)), "scale mismatch"
+
+    if zb == 16:
+        gz = out["zero"][ids].astype(np.float64)
+        ztol = Z_TOL * np.maximum(np.abs(o_z), 1.0) + np.abs(o_z) * 2.0 ** -11
+
+        def zero_ok(zg, zo):
+            return np.abs(zg - zo) <= Z_TOL * max(abs(zo), 1.0) + abs(zo) * 2.0 ** -11
+    else:
+        meta = out["zero_meta"].astype(np.float64)
+        gz = (out["zero"][ids].astype(np.float64) - meta[1]) * meta[0]
+        ztol = 0.5 * meta[0] * (1 + 1e-6) + Z_TOL * np.maximum(np.abs(o_z), 1.0)
+
+        def zero_ok(zg, zo):
+            return np.abs(zg - zo) <= 0.5 * meta[0] * (1 + 1e-6) + Z_TOL * max(abs(zo), 1.0)
+    zbad = np.abs(gz - o_z.astype(np.float64)) > ztol
+    diff = g_levels.astype(np.int32) - o_levels.astype(np.int32)
+    bad = zbad | (np.abs(diff) > 1).any(axis=1)
+    nbad = np.nonzero(bad)[0]
+    rep = {"groups": int(len(ids))}
+
+    def explain(t, allowed):
+        """An iterate k allowed by the trajectory's near ties that reproduces group t."""
+        j = ids[t]
+        w = group_values(Wf, j, g, axis)
+        s, zt, et, _ = oracle.trace_group(w, nb, p, beta, kappa, max(iters, 1))
+        for k in allowed(et):
+            lv = oracle.group_codes(w, nb, s, zt[k]).astype(np.int32)
+            if zero_ok(gz[t], zt[k]) and np.all(np.abs(lv - g_levels[t]) <= 1) and \
+                    np.count_nonzero(lv - g_levels[t]) <= max(1, CODE_FRAC * g):
+                return True
+        return False
+
+    if mode == oracle.STOP_TENSOR and len(nbad) > CODE_FRAC * len(ids) + 1:
+        # the tensor-wide decision itself went the other way: every group at one other iterate
+        traces = [oracle.trace_group(group_values(Wf, j, g, axis), nb, p, beta, kappa, max(iters, 1)) for j in ids]
+        E = np.mean([t[2] for t in traces], axis=0)
+        ko = int(o_bi[0])
+        ks = [k for k in range(max(iters, 1)) if _path_ok(E, k, ko, iters, mode)]
+        ok = False
+        for k in ks:
+            lv = np.stack([oracle.group_codes(group_values(Wf, j, g, axis), nb, t[0], t[1][k])
+                           for j, t in zip(ids, traces)]).astype(np.int32)
+            zk = np.array([t[1][k] for t in traces], np.float64)
+            d = lv - g_levels.astype(np.int32)
+            if np.all(np.abs(d) <= 1) and np.count_nonzero(d) <= CODE_FRAC * d.size + 1 and \
+                    np.all(np.abs(gz - zk) <= ztol):
+                ok = True
+                rep["tensor_tie"] = (k, ko)
+                break
+        assert ok, f"tensor stop: {len(nbad)} groups differ and no near-tie iterate explains them ({ks})"
+        return rep
+    for t in nbad:
+        allowed = (lambda et, t=t: [k for k in range(max(iters, 1)) if _path_ok(et, k, int(o_bi[t]), iters, mode)])
+        assert explain(t, allowed), f"group {ids[t]}: outputs differ from the oracle's and no near tie explains it"
+    assert len(nbad) <= CODE_FRAC * len(ids) + 1, f"{len(nbad)} tie groups of {len(ids)}"
+    good = np.ones(len(ids), bool)
+    good[nbad] = False
+    nd = int(np.count_nonzero(diff[good]))
+    assert nd <= CODE_FRAC * diff[good].size + 1, f"{nd} differing codes of {diff[good].size}"
+    rep["tie_groups"] = int(len(nbad))
+    rep["code_mismatch"] = nd
+    return rep

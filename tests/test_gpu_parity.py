@@ -267,6 +267,18 @@ def test_tensor_outputs_kept_iterate_placement(hq, nbits, g, zb, place):
 
 
 @pytest.mark.parametrize("nbits,g", SWEEP)
+def test_llama_mlp_down_tensor_mode(hq, nbits, g):
+    """Llama-2-7B down shape (4096x11008, bf16, the layer's seed), tensor
+    stop, every setting of the sweep: full tensor against the full oracle, and
+    the launch configuration without debug outputs gives the same bytes."""
+    W = synth.weight(4096, 11008, seed=6, dtype=torch.bfloat16)
+    rep, gpu, orc = _run(hq, W, _params(nbits, g, stop=1), check_recon=(nbits == 3))
+    if "tensor_tie" not in rep:
+        assert np.all(gpu["best_iter"] == orc["best_iter"][0])
+    _nodebug_equals_debug(hq, W.cuda(), nbits, g, 16, 20)
+
+
+@pytest.mark.parametrize("nbits,g", SWEEP)
 @pytest.mark.parametrize("zb", [16, 8])
 def test_llama_mlp_tensor_mode_outputs_without_debug(hq, nbits, g, zb):
     """The benchmark's launch configuration (tensor stop, no debug outputs) on

@@ -155,3 +155,64 @@ def test_stream_jobs_callback_error_surfaces_after_the_call(hq):
     assert seen == list(range(len(MIXED)))
     for w, st, o in zip(Ws, sets, outs):
         _same(o, _expect(hq, w, st))
+
+
+# ------------------------------------------------- against the oracle ------
+
+from . import parity_check as pc  # noqa: E402
+
+
+def _np(o):
+    return {k: (v.numpy() if v is not None else None) for k, v in o.items() if k in ("packed", "scale", "zero",
+                                                                                     "zero_meta")}
+
+
+def _prm(st):
+    return dict(st, p=0.7, beta=1.0, kappa=1.01, iters=20)
+
+
+def test_stream_jobs_outputs_against_oracle(hq):
+    """Per-matrix settings (both axes, every stop rule, both zero widths)
+    streamed from host memory: each matrix's stored outputs against the full
+    oracle run with that matrix's settings."""
+    Ws, sets, outs = _mixed(hq)
+    hq.quantize_stream_jobs(Ws, sets, outs)
+    for w, st, o in zip(Ws, sets, outs):
+        pc.check_stored(w, _prm(st), _np(o))
+
+
+def test_stream_llama2_13b_mixed_layer_against_oracle(hq):
+    """One Llama-2-13B-shaped layer with per-layer-type settings (attention b4
+    g64, MLP b2 g32, tensor stop, fp16 zero) streamed through
+    quantize_stream_jobs, as the 13B streamed workload runs it: q, gate and
+    down against the full oracle (the stop is tensor-wide)."""
+    base = dict(nbits=4, group_size=64, stop_mode=1)
+    dyn = {"attn": dict(nbits=4, group_size=64, stop_mode=1), "mlp": dict(nbits=2, group_size=32, stop_mode=1)}
+    names = {"q": "self_attn.q_proj", "gate": "mlp.gate_proj", "down": "mlp.down_proj"}
+    mats = [(n, r, c) for n, r, c in synth.LLAMA2_13B.matrices() if n in names]
+    Ws = [synth.weight(r, c, seed=synth.seed_for(3, n), dtype=torch.float16).pin_memory() for n, r, c in mats]
+    sets = [hq.settings_for(f"model.layers.3.{names[n]}", base, dyn) for n, _, _ in mats]
+    outs = [hq.host_outputs(r, c, st["nbits"], st["group_size"], st["axis"], st["zero_nbits"])
+            for (_, r, c), st in zip(mats, sets)]
+    _, done = hq.quantize_stream_jobs(Ws, sets, outs)
+    assert done == len(mats)
+    for w, st, o in zip(Ws, sets, outs):
+        pc.check_stored(w, _prm(st), _np(o))
+
+
+@pytest.mark.parametrize("nbits,g", [(2, 16), (4, 128)])
+def test_stream_llama2_70b_shapes_against_oracle(hq, nbits, g):
+    """The Llama-2-70B settings (8-bit zero, group stop) streamed from host
+    memory on the model's four matrix shapes (q 8192x8192, k 1024x8192, gate
+    28672x8192, down 8192x28672; layer 5's seeds): sampled groups of each
+    against the oracle."""
+    mats = [("q", 8192, 8192), ("k", 1024, 8192), ("gate", 28672, 8192), ("down", 8192, 28672)]
+    Ws = [synth.weight(r, c, seed=synth.seed_for(5, n), dtype=torch.float16).pin_memory() for n, r, c in mats]
+    st = dict(nbits=nbits, group_size=g, axis=1, stop_mode=0, zero_nbits=8)
+    outs = [hq.host_outputs(r, c, nbits, g, zero_nbits=8) for _, r, c in mats]
+    _, done = hq.quantize_stream_jobs(Ws, [st] * len(mats), outs)
+    assert done == len(mats)
+    for i, (w, o) in enumerate(zip(Ws, outs)):
+        G = w.numel() // g
+        ids = np.unique(np.concatenate([[0, G - 1], np.random.default_rng(i).choice(G, 3000, replace=False)]))
+        pc.check_stored(w, _prm(st), _np(o), sample=ids)
