@@ -57,6 +57,13 @@ def _bind(L):
     L.oracle_group_codes.argtypes = [P, i32, i32, f32, f32, P]
     L.oracle_update_zero.restype = f32
     L.oracle_update_zero.argtypes = [P, P, P, i32, f32, f32, f32]
+    L.oracle_quantize_half.restype = i32
+    L.oracle_quantize_half.argtypes = [P, i64, i64, i32, i32, i32, i32, f32, f32, f32, i32, i32, i32,
+                                       P, P, P, P, P, P, P, i32]
+    L.oracle_trace_group_half.restype = i32
+    L.oracle_trace_group_half.argtypes = [P, i32, i32, f32, f32, f32, i32, P, P, P, P]
+    L.oracle_group_codes_half.restype = None
+    L.oracle_group_codes_half.argtypes = [P, i32, i32, f32, f32, P]
     L.oracle_quantize_groups.restype = i32
     L.oracle_quantize_groups.argtypes = [P, i64, i64, i32, i32, i32, i32, f32, f32, f32, i32, i32,
                                          P, i64, P, P, P, P, P, i32]
@@ -251,3 +258,50 @@ def quantize_groups(W, group_ids, nbits, group_size, axis=1, p=0.7, beta=1.0, ka
     if rc != 0:
         raise ValueError("oracle_quantize_groups failed")
     return dict(levels=levels.reshape(n, group_size), s=s, zbest=zb, best_iter=bi, best_err=be)
+
+
+# ---------------------------------------------- half-precision variant ----
+
+def quantize_half(W, nbits, group_size, axis=1, p=0.7, beta=1.0, kappa=1.01, iters=20, stop_mode=STOP_GROUP,
+                  zero_nbits=16, nthreads=0, L=None):
+    """The half-precision solver variant (reading H) on a float16 array; the
+    same output dict as quantize() (zero_f32 holds the fp16 zero-points)."""
+    L = L or lib()
+    bits, dtype = _bits16(W)
+    rows, cols = bits.shape
+    G = num_groups(rows, cols, group_size)
+    packed = np.zeros(rows * cols * nbits // 8, np.uint8)
+    scale = np.zeros(G, np.float16)
+    zero = np.zeros(G, np.float16 if zero_nbits == 16 else np.uint8)
+    meta = np.zeros(2, np.float32) if zero_nbits == 8 else None
+    bi = np.zeros(G, np.int32)
+    be = np.zeros(G, np.float32)
+    zf = np.zeros(G, np.float32)
+    rc = L.oracle_quantize_half(_p(bits), rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters,
+                                stop_mode, zero_nbits, _p(packed), _p(scale), _p(zero), _p(meta), _p(bi), _p(be),
+                                _p(zf), nthreads)
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_half failed with code {rc}")
+    return dict(packed=packed, scale=scale, zero=zero, zero_meta=meta, best_iter=bi, best_err=be, zero_f32=zf)
+
+
+def trace_group_half(w, nbits, p=0.7, beta=1.0, kappa=1.01, iters=20, L=None):
+    """One fp16 group (values as float32) through `iters` iterations of the
+    half-precision variant without early stop: (s, z[iters], e[iters], beta[iters])."""
+    L = L or lib()
+    w = np.ascontiguousarray(w, np.float32)
+    s = np.zeros(1, np.float32)
+    z = np.zeros(iters, np.float32)
+    e = np.zeros(iters, np.float64)
+    b = np.zeros(iters, np.float32)
+    if L.oracle_trace_group_half(_p(w), w.size, nbits, p, beta, kappa, iters, _p(s), _p(z), _p(e), _p(b)) != 0:
+        raise ValueError("oracle_trace_group_half failed")
+    return float(s[0]), z, e, b
+
+
+def group_codes_half(w, nbits, s, z, L=None):
+    L = L or lib()
+    w = np.ascontiguousarray(w, np.float32)
+    out = np.zeros(w.size, np.uint8)
+    L.oracle_group_codes_half(_p(w), w.size, nbits, float(s), float(z), _p(out))
+    return out

@@ -672,3 +672,227 @@ int oracle_quantize_groups(const uint16_t *W, int64_t rows, int64_t cols, int dt
     }
     return 0;
 }
+
+/* ==== the half-precision solver variant ====================================
+ *
+ * The pages run the solver on the GPU in half precision ("Speed: from hours
+ * to minutes"), with the steps of "Outlier-aware optimization without
+ * gradients".  Reading H (this library's restatement of "half precision" for
+ * the steps of the solver above; h(x) rounds x to fp16, to nearest, ties to
+ * even):
+ *   H1 input fp16 only.
+ *   H2 s = h(min(L/(max - min), 2e4)) from the fp32 quotient (R1);
+ *      z0 = h(-min * s).
+ *   H3 ws = h(w*s); v = h(ws + z); W_q = clamp(round_half_even(v), 0, L);
+ *      r = h(v - W_q).
+ *   H4 the lp error of z is s^-p/g times the exact sum of the terms
+ *      h(|r|^p); the stop rule (R4) compares these sums within the group.
+ *   H5 proximal step: d = h(fl32(r / s)), W_e = h(shrink(d)) with the shrink
+ *      in fp32 (oracle_shrink); z' = h((sum W_q - sum h(h(w - W_e) * s)) / g),
+ *      both sums exact.
+ *   H6 beta, the stop modes group and none, the kept iterate and the 8-bit
+ *      zero (R7, from the fp16 zero-points): as the fp32 solver.  Outputs:
+ *      codes clamp(round(h(h(w*s) + z*)), 0, L), scale h(fl32(1/s)), zero z*.
+ * Every product of two fp16 values and every sum of two is exact in fp64, so
+ * each h() below rounds an exact value once.
+ */
+
+static float h16(double x) { return (float)(_Float16)x; }
+
+/* H6: the stored zero-points -- fp16, or R7's 8-bit quantiser over the tensor. */
+static void store_zero_half(const float *zb, int64_t G, int zero_nbits, void *zero, float *zero_meta)
+{
+    if (zero_nbits == 16) {
+        uint16_t *z16 = (uint16_t *)zero;
+        for (int64_t j = 0; j < G; ++j) z16[j] = to_f16(zb[j]);
+        return;
+    }
+    uint8_t *z8 = (uint8_t *)zero;
+    float zmn = G ? zb[0] : 0.0f, zmx = zmn;
+    for (int64_t j = 1; j < G; ++j) {
+        if (zb[j] < zmn) zmn = zb[j];
+        if (zb[j] > zmx) zmx = zb[j];
+    }
+    float sz = ORACLE_S_CAP;
+    if (zmx > zmn) {
+        sz = 255.0f / (zmx - zmn);
+        if (sz > ORACLE_S_CAP) sz = ORACLE_S_CAP;
+    }
+    float zz = -zmn * sz;
+    for (int64_t j = 0; j < G; ++j) z8[j] = (uint8_t)quantize_elem(zb[j], sz, zz, 255);
+    zero_meta[0] = 1.0f / sz;
+    zero_meta[1] = zz;
+}
+
+static void init_half(const float *w, int g, int L, float *s_out, float *z_out)
+{
+    float mn = w[0], mx = w[0];
+    for (int i = 1; i < g; ++i) {
+        if (w[i] < mn) mn = w[i];
+        if (w[i] > mx) mx = w[i];
+    }
+    float s = ORACLE_S_CAP;
+    if (mx > mn) {
+        s = (float)L / (mx - mn);
+        if (s > ORACLE_S_CAP) s = ORACLE_S_CAP;
+    }
+    s = h16(s);
+    *s_out = s;
+    *z_out = h16(-(double)mn * (double)s);
+}
+
+/* H3: the code of one element at zero-point z. */
+static float quantize_half(float w, float s, float z, int L)
+{
+    float ws = h16((double)w * (double)s);
+    float v = h16((double)ws + (double)z);
+    float q = nearbyintf(v);
+    if (q < 0.0f) q = 0.0f;
+    if (q > (float)L) q = (float)L;
+    return q;
+}
+
+/* H3, H4: codes, residuals and the exact sum of the rounded terms |r|^p. */
+static double evaluate_half(const float *w, int g, int L, float s, float z, float p, float *q, float *r)
+{
+    double acc = 0.0;
+    for (int i = 0; i < g; ++i) {
+        float ws = h16((double)w[i] * (double)s);
+        float v = h16((double)ws + (double)z);
+        float qi = nearbyintf(v);
+        if (qi < 0.0f) qi = 0.0f;
+        if (qi > (float)L) qi = (float)L;
+        q[i] = qi;
+        r[i] = h16((double)v - (double)qi);
+        acc += (double)h16(pow(fabs((double)r[i]), (double)p));
+    }
+    return acc;
+}
+
+/* H5: the z update from the codes and residuals. */
+static float update_zero_half(const float *w, const float *q, const float *r, int g, float s, float p, float beta)
+{
+    double sq = 0.0, sws = 0.0;
+    for (int i = 0; i < g; ++i) {
+        float d = h16((double)(r[i] / s));
+        float we = h16((double)oracle_shrink(d, p, beta));
+        float ws = h16((double)h16((double)w[i] - (double)we) * (double)s);
+        sq += (double)q[i];
+        sws += (double)ws;
+    }
+    return h16((sq - sws) / (double)g);
+}
+
+static void solve_one_group_half(const float *w, int g, int L, float p, float beta0, float kappa, int iters,
+                                 int stop_mode, float *q, float *r, group_result *res)
+{
+    float s, z;
+    init_half(w, g, L, &s, &z);
+    double best = INFINITY;
+    float zbest = z;
+    int best_iter = 0;
+    float beta = beta0;
+    for (int it = 0; it < iters; ++it) {
+        double e = evaluate_half(w, g, L, s, z, p, q, r);
+        if (e < best) {
+            best = e;
+            zbest = z;
+            best_iter = it;
+        } else if (stop_mode == ORACLE_STOP_GROUP) {
+            break;
+        }
+        z = update_zero_half(w, q, r, g, s, p, beta);
+        beta = beta * kappa;
+    }
+    if (iters == 0) best = evaluate_half(w, g, L, s, z, p, q, r);
+    res->s = s;
+    res->zbest = zbest;
+    res->best_err = best * pow((double)s, -(double)p) / (double)g;
+    res->best_iter = best_iter;
+}
+
+/*
+ * The half-precision variant of oracle_quantize: fp16 input (dtype must be
+ * ORACLE_F16), group or no stop, either axis; outputs as oracle_quantize
+ * (zero_f32 receives the fp16 zero-points).  Returns 0, or 1 on an invalid
+ * argument, 2 on an allocation failure.
+ */
+int oracle_quantize_half(const uint16_t *W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size,
+                         int axis, float p, float beta, float kappa, int iters, int stop_mode, int zero_nbits,
+                         uint8_t *W_q_packed, uint16_t *scale, void *zero, float *zero_meta, int32_t *best_iter,
+                         float *best_err, float *zero_f32, int nthreads)
+{
+    if (!valid_args(rows, cols, dtype, nbits, group_size, axis, stop_mode, zero_nbits) || iters < 0) return 1;
+    if (dtype != ORACLE_F16 || stop_mode == ORACLE_STOP_TENSOR) return 1;
+    const int g = group_size, L = (1 << nbits) - 1;
+    const int64_t G = rows * cols / g;
+    const int nth = thread_count(nthreads);
+    float *s_all = (float *)malloc(sizeof(float) * (size_t)(G ? G : 1));
+    float *zb_all = (float *)malloc(sizeof(float) * (size_t)(G ? G : 1));
+    if (!s_all || !zb_all) { free(s_all); free(zb_all); return 2; }
+    memset(W_q_packed, 0, (size_t)(rows * cols * nbits / 8));
+#pragma omp parallel num_threads(nth)
+    {
+        float *w = (float *)malloc(sizeof(float) * (size_t)g * 3);
+        float *q = w + g, *r = w + 2 * g;
+#pragma omp for schedule(dynamic, 256)
+        for (int64_t j = 0; j < G; ++j) {
+            for (int i = 0; i < g; ++i) w[i] = load_elem(W, dtype, elem_index(j, i, cols, g, axis));
+            group_result res;
+            solve_one_group_half(w, g, L, p, beta, kappa, iters, stop_mode, q, r, &res);
+            s_all[j] = res.s;
+            zb_all[j] = res.zbest;
+            if (best_iter) best_iter[j] = res.best_iter;
+            if (best_err) best_err[j] = (float)res.best_err;
+        }
+        free(w);
+    }
+    float *w = (float *)malloc(sizeof(float) * (size_t)g);
+    for (int64_t j = 0; j < G; ++j) {
+        for (int i = 0; i < g; ++i) w[i] = load_elem(W, dtype, elem_index(j, i, cols, g, axis));
+        for (int i = 0; i < g; ++i) {
+            int64_t e = elem_index(j, i, cols, g, axis);
+            pack_elem(W_q_packed, e / cols, e % cols, cols, nbits, axis,
+                      (unsigned)quantize_half(w[i], s_all[j], zb_all[j], L));
+        }
+        scale[j] = to_f16(1.0f / s_all[j]);
+        if (zero_f32) zero_f32[j] = zb_all[j];
+    }
+    free(w);
+    store_zero_half(zb_all, G, zero_nbits, zero, zero_meta);
+    free(s_all);
+    free(zb_all);
+    return 0;
+}
+
+/* Trace one fp16 group (values as floats) through `iters` iterations of the
+ * half-precision variant without early stop: z_k, the error of z_k (H4, mean
+ * form) and beta_k, as oracle_trace_group. */
+int oracle_trace_group_half(const float *w, int g, int nbits, float p, float beta0, float kappa, int iters,
+                            float *s_out, float *z_traj, double *e_traj, float *beta_traj)
+{
+    if (g < 1 || iters < 0) return 1;
+    const int L = (1 << nbits) - 1;
+    float *q = (float *)malloc(sizeof(float) * (size_t)g * 2);
+    float *r = q + g;
+    float s, z;
+    init_half(w, g, L, &s, &z);
+    float beta = beta0;
+    for (int it = 0; it < iters; ++it) {
+        z_traj[it] = z;
+        e_traj[it] = evaluate_half(w, g, L, s, z, p, q, r) * pow((double)s, -(double)p) / (double)g;
+        beta_traj[it] = beta;
+        z = update_zero_half(w, q, r, g, s, p, beta);
+        beta = beta * kappa;
+    }
+    *s_out = s;
+    free(q);
+    return 0;
+}
+
+/* Codes of one group of the half-precision variant for a given zero-point. */
+void oracle_group_codes_half(const float *w, int g, int nbits, float s, float z, uint8_t *levels)
+{
+    const int L = (1 << nbits) - 1;
+    for (int i = 0; i < g; ++i) levels[i] = (uint8_t)quantize_half(w[i], s, z, L);
+}

@@ -17,7 +17,8 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "hqq_oracle.c")
 
-# (name, text in the source, replacement, expected number of occurrences)
+# (name, text in the source, replacement, expected number of occurrences; a
+# line the fp32 solver shares with the half-precision variant is mutated in both)
 MUTANTS = [
     ("z-update-sign", "return (float)((sq - sws) / (double)g);", "return (float)((sq + sws) / (double)g);", 1),
     ("z-update-drops-We", "float ws = (w[i] - we) * s;", "float ws = (w[i] - 0.0f * we) * s;", 1),
@@ -26,16 +27,16 @@ MUTANTS = [
     ("residual-sign", "float r = v - qi;", "float r = qi - v + 2.0f * (qi - v) * (qi > 0.0f);", 1),
     ("residual-unscaled", "d[i] = r / s;", "d[i] = r;", 1),
     ("l1-instead-of-lp", "acc += (double)powf(fabsf(d[i]), p);", "acc += (double)fabsf(d[i]);", 1),
-    ("tie-continues", "        if (e < best) {\n            best = e;\n            zbest = z;",
-     "        if (e <= best) {\n            best = e;\n            zbest = z;", 1),
-    ("keeps-last-z", "    res->zbest = zbest;", "    res->zbest = z;", 1),
-    ("beta-divides", "beta = beta * kappa;", "beta = beta / kappa;", 2),
+    ("tie-continues", "        double e = evaluate(w, g, L, s, z, p, q, d) / (double)g;\n        if (e < best) {",
+     "        double e = evaluate(w, g, L, s, z, p, q, d) / (double)g;\n        if (e <= best) {", 1),
+    ("keeps-last-z", "    res->zbest = zbest;", "    res->zbest = z;", 2),
+    ("beta-divides", "beta = beta * kappa;", "beta = beta / kappa;", 4),
     ("z0-from-max", "*z_out = -mn * s;", "*z_out = -mx * s;", 1),
-    ("scale-uses-2^b", "s = (float)L / (mx - mn);", "s = (float)(L + 1) / (mx - mn);", 1),
-    ("floor-instead-of-round", "float q = nearbyintf(v);", "float q = floorf(v);", 1),
+    ("scale-uses-2^b", "s = (float)L / (mx - mn);", "s = (float)(L + 1) / (mx - mn);", 2),
+    ("floor-instead-of-round", "float q = nearbyintf(v);", "float q = floorf(v);", 2),
     ("tensor-stop-first-group", "double e = G ? total / (double)(G * g) : 0.0;",
      "double e = G ? gerr[0] / (double)g : 0.0;", 1),
-    ("zero8-scale", "sz = 255.0f / (zmx - zmn);", "sz = 254.0f / (zmx - zmn);", 1),
+    ("zero8-scale", "sz = 255.0f / (zmx - zmn);", "sz = 254.0f / (zmx - zmn);", 2),
     ("dequant-sign", "float v = (q - z) * sc;", "float v = (q + z) * sc;", 1),
     ("scale8-zc-sign", "const float zc = -mn * sc;", "const float zc = mn * sc;", 1),
     ("scale8-254-levels", "? 255.0f / (mx - mn) : 1.0f;", "? 254.0f / (mx - mn) : 1.0f;", 1),
@@ -63,6 +64,13 @@ MUTANTS = [
      "int64_t j = group_ids[k];\n            for (int i = 0; i < g; ++i) w[i] = load_elem(W, dtype, elem_index(j, i, cols, g, 1));", 1),
     ("groups-levels-reversed", "levels[k * g + i] = (uint8_t)quantize_elem(w[i], res.s, res.zbest, L);",
      "levels[k * g + (g - 1 - i)] = (uint8_t)quantize_elem(w[i], res.s, res.zbest, L);", 1),
+    ("half-ws-unrounded", "        float ws = h16((double)w[i] * (double)s);\n        float v = h16((double)ws + (double)z);",
+     "        float ws = (float)((double)w[i] * (double)s);\n        float v = h16((double)ws + (double)z);", 1),
+    ("half-z-unrounded", "    return h16((sq - sws) / (double)g);", "    return (float)((sq - sws) / (double)g);", 1),
+    ("half-s-unrounded", "    s = h16(s);\n", "", 1),
+    ("half-tie-continues", "        double e = evaluate_half(w, g, L, s, z, p, q, r);\n        if (e < best) {",
+     "        double e = evaluate_half(w, g, L, s, z, p, q, r);\n        if (e <= best) {", 1),
+    ("half-codes-in-fp32", "    float ws = h16((double)w * (double)s);", "    float ws = w * s;", 1),
     ("pack-msb-first", "unsigned v = level << off; /* at most 8 + 7 bits */",
      "unsigned v = (off + b <= 8 ? level << (8 - b - off) : level << off);", 1),
 ]

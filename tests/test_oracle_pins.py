@@ -708,3 +708,95 @@ def test_quantize_groups_equals_whole_tensor(orc, axis, g, nbits, mode):
         assert part["zbest"][k] == full["zero_f32"][j]
         assert part["best_iter"][k] == full["best_iter"][j]
         assert part["best_err"][k] == full["best_err"][j]
+
+
+# --------------------------------------------- half-precision variant ------
+
+def _half_rows():
+    rows = []
+    with open(os.path.join(GOLDEN, "half_worked_groups.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            head, w = line.split(";")
+            name, nb, s, z0, z1, codes = head.split()
+            rows.append((name, int(nb), float(s), float(z0), float(z1), [int(c) for c in codes.split(",")],
+                         np.array([float(x) for x in w.split()], np.float32)))
+    return rows
+
+
+@pytest.mark.parametrize("name,nbits,s,z0,z1,codes,w", _half_rows())
+def test_half_worked_groups(orc, name, nbits, s, z0, z1, codes, w):
+    """Hand-worked fp16 steps (tests/golden/half_worked_groups.txt): the scale,
+    z0, the codes at z0 (group B has a code that the fp16 rounding of w*s
+    decides) and z1 (group A's mean is not an fp16 number)."""
+    assert np.array_equal(w.astype(np.float16).astype(np.float32), w)
+    ss, zt, et, _ = orc.trace_group_half(w, nbits, iters=2)
+    assert ss == s and zt[0] == z0 and zt[1] == z1
+    assert list(orc.group_codes_half(w, nbits, ss, zt[0])) == codes
+
+
+@pytest.mark.parametrize("nbits", NBITS)
+def test_half_values_are_fp16(orc, nbits):
+    """Every scale and zero-point of the variant is an fp16 number, and so are
+    the stored zeros; the kept error is the lowest of the trajectory."""
+    rng = _rng(200 + nbits)
+    for g in (8, 16, 64):
+        for _ in range(20):
+            w = (rng.standard_normal(g) * rng.choice([0.02, 0.3, 3.0])).astype(np.float16).astype(np.float32)
+            s, zt, et, _ = orc.trace_group_half(w, nbits, iters=12)
+            assert np.float32(np.float16(s)) == s
+            assert np.array_equal(zt.astype(np.float16).astype(np.float32), zt)
+            assert np.all(np.isfinite(et)) and np.all(et >= 0)
+    W = _synth_f16(32, 256, seed=nbits)
+    out = orc.quantize_half(W, nbits, 32, stop_mode=2)
+    zf = out["zero_f32"]
+    assert np.array_equal(zf.astype(np.float16).astype(np.float32), zf)
+    assert np.array_equal(out["zero"].astype(np.float32), zf)
+
+
+@pytest.mark.parametrize("nbits", [1, 2, 3, 4])
+def test_half_trajectory_equals_fp32_when_exact(orc, nbits):
+    """On groups whose every intermediate value is exact in fp16 (values m/256,
+    range (2^b - 1)/16 so that s = 16, g = 8), no fp16 rounding happens: the
+    variant's zero-points and codes follow the fp32 oracle's exactly, and its
+    errors agree within the fp16 rounding of the terms (2^-11 relative each)."""
+    rng = _rng(300 + nbits)
+    L = (1 << nbits) - 1
+    for _ in range(30):
+        lo = int(rng.integers(-64, 64))
+        m = rng.integers(lo, lo + 16 * L + 1, size=8)
+        m[0], m[1] = lo, lo + 16 * L
+        w = (m / 256.0).astype(np.float32)
+        assert np.array_equal(w.astype(np.float16).astype(np.float32), w)
+        s16, zh, eh, _ = orc.trace_group_half(w, nbits, iters=6)
+        s32, z32, e32, _ = orc.trace_group(w, nbits, iters=6)
+        assert s16 == s32 == 16.0
+        if np.all(np.abs(z32) < 16):
+            assert np.array_equal(zh, z32), (zh, z32)
+            for z in zh:
+                assert np.array_equal(orc.group_codes_half(w, nbits, s16, z), orc.group_codes(w, nbits, s32, z))
+            assert np.all(np.abs(eh - e32) <= 2.0 ** -10 * e32 + 1e-30)
+
+
+def test_half_quantize_matches_its_trace(orc):
+    """The whole-tensor variant keeps, per group, the first iterate of lowest
+    error along its own trace (group stop: up to the first rise) and stores
+    fp16(1/s) and the codes of that iterate."""
+    W = _synth_f16(16, 512, seed=9)
+    for stop in (0, 2):
+        out = orc.quantize_half(W, 4, 64, stop_mode=stop, iters=20)
+        levels = orc.unpack_levels(out["packed"], 16, 512, 4, 1).reshape(-1, 64)
+        for j in range(0, 16 * 512 // 64, 7):
+            w = W.reshape(-1, 64)[j].astype(np.float32)
+            s, zt, et, _ = orc.trace_group_half(w, 4, iters=20)
+            if stop == 0:
+                k = 0
+                while k + 1 < 20 and et[k + 1] < et[k]:
+                    k += 1
+            else:
+                k = int(np.argmin(et))
+            assert out["best_iter"][j] == k and out["zero_f32"][j] == zt[k]
+            assert out["scale"][j] == np.float16(np.float32(1.0) / np.float32(s))
+            assert np.array_equal(levels[j], orc.group_codes_half(w, 4, s, zt[k]))
