@@ -1,24 +1,28 @@
-"""Benchmark: HQQ quantisation throughput on Llama-2-7B MLP shapes.
+"""Benchmark: HQQ quantisation throughput on a Llama-2-70B-shaped weight set.
 
-One step = the whole quantiser over one batch: the MLP weights of one decoder
-layer (gate/up 11008x4096, down 4096x11008, bf16, synthetic Llama-2 weight
-statistics) quantised at every (nbits, group_size) of the sweep
-(8/128, 4/64, 3/64, 2/16, 1/16), each with stop_mode=group and
-stop_mode=tensor: 30 hqq_quantize calls, 1.353 G weights.
+Default workload (`llama2-70b`): 80 decoder layers x (q, o 8192x8192; k, v
+1024x8192; gate, up 28672x8192; down 8192x28672), fp16 synthetic weights with
+the Llama-2 weight statistics (0.02*N(0,1), 0.1% outliers x10), per-layer
+seeds; quantised whole at nbits/group 2/16 and at 4/128, 8-bit zero, group
+stop.  One step = 1120 hqq_quantize calls, 136.9 G weights.
 
-value     = weights quantised / device time (CUDA events), inputs resident in HBM.
-e2e       = the same through the C ABI with host buffers: every step copies the
-            step's inputs from pinned host memory and reads all outputs back.
-roofline  = the dominant kernel family (solve_tensor_kernel: the tensor-stop
-            calls), bound by the MUFU pipe that evaluates |r|^p (two ops per
-            element and evaluated iterate); timed per hqq_quantize call (its
-            launch sequence) with CUDA events on the launching stream.
-            traffic = DRAM bytes per call from the ncu launch list in
-            profiles/, reported only while the kernel sources are unchanged.
+value     = weights quantised / device time (CUDA events), every layer resident
+            in HBM (drawn on the GPU before the timed region; 137 GB).
+e2e       = the same weight set end to end through hqq_quantize_stream_jobs
+            (C ABI) with pinned host buffers: each step copies every weight in
+            and every output out (PCIe-bound).
+roofline  = the group-stop solver (solve_group_onepass_kernel), bound by the MUFU pipe
+            that evaluates |r|^p (two ops per element and evaluated iterate),
+            timed per hqq_quantize call with CUDA events on the launching
+            stream; the HBM fraction of the same calls beside it.
 cpu_baseline / --impl reference = the CPU oracle on a bounded sample.
 
-Multi-GPU (torchrun): each rank quantises its own layer's MLP (weak scaling,
-no data-path collective); time = max over ranks.
+Multi-GPU (torchrun): the layers are split across ranks (strong scaling, no
+data-path collective); time = max over ranks.
+
+Other workloads: `llama2-7b-mlp-sweep` (the Llama-2-7B MLP shapes at five
+settings and two stop rules), `llama2-70b-stream` and `llama2-13b-stream`
+(streamed models), and `--case` lines for single kernels.
 """
 import argparse
 import json
@@ -62,6 +66,13 @@ GEMM_TRAFFIC = {"src_sha256": "6047c8fb4337f86155429e2a54e5e1946effb14b71f0514dd
                 "summary": "profiles/gemm_kernel_28672x8192_b4g64_batch256.md"}
 
 
+# DRAM traffic of the group-stop solver on the 70B-shaped workload, as a ratio
+# to the algorithmic bytes of the captured calls (ncu, one call per setting on
+# the gate shape 28672x8192; see profiles/), valid while the kernel sources
+# hash to the captured ones.
+TRAFFIC70 = {"src_sha256": None, "bytes_per_alg_byte": None, "summary": None}
+
+
 def kernel_sources_sha(files=None):
     """sha256 of kernel sources (default: the solver's) with comments and
     blank lines removed: a change of code, not of commentary, invalidates the
@@ -77,11 +88,12 @@ def kernel_sources_sha(files=None):
     return h.hexdigest()
 
 
-def solver_launches(mode, iters=20, g=64):
+def solver_launches(mode, iters=20, g=64, axis=1):
     """Kernel launches of one hqq_quantize call (fp16 zero), as the library
-    schedules them: group stop runs passes of 2 and 3 evaluations and then the
-    rest (no stop: one pass); tensor stop runs chunks of iterations [0,2) and
-    then C at a time (C = 8 for g >= 32, with a last chunk shorter than 4
+    schedules them: group and no stop on axis 1 run one launch of the one-pass
+    kernel; on axis 0 group stop runs passes of 2 and 3 evaluations and then
+    the rest (no stop: one pass); tensor stop runs chunks of iterations [0,2)
+    and then C at a time (C = 8 for g >= 32, with a last chunk shorter than 4
     merged into the one before; C = 4 for g <= 16), and one launch that writes
     the outputs."""
     if mode == 1:
@@ -95,7 +107,7 @@ def solver_launches(mode, iters=20, g=64):
             if C >= 8 and n > 2 and (iters - 2) - (n - 2) * C < C // 2:
                 n -= 1
         return n + 1
-    if mode == 2 or iters <= 2:
+    if axis == 1 or mode == 2 or iters <= 2:
         return 1
     n, done = 0, 0
     for v in (2, 3):
@@ -342,6 +354,53 @@ def run_reference(args, world, rank):
     print(json.dumps(line))
 
 
+def run_reference70(args, world, rank):
+    """The reference arm of the llama2-70b workload: the CPU oracle, as it
+    stands, on the machine's host cores; each step is a bounded sample of the
+    workload (the first rows of every matrix of one layer at both settings,
+    about --ref-step seconds; layer = step index, its seeds drawn on the host
+    with the CPU generator).  Rank 0 only; the other ranks exit without work."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.lib()
+    nth = os.cpu_count() or 1
+    mats = synth.LLAMA2_70B.matrices()
+    probe = [synth.weight(64, c, seed=synth.seed_for(0, n), dtype=torch.float16) for n, r, c in mats]
+    rows = oracle_rows_for_budget(probe, SETTINGS70B, args.ref_step, nth, rows0=8,
+                                  rows_cap=min(r for _, r, _ in mats))
+    per = []
+    for i in range(args.warmup + args.steps):
+        Ws = [synth.weight(rows, c, seed=synth.seed_for(i % args.layers, n), dtype=torch.float16)
+              for n, r, c in mats]
+        n_w, dt, _ = _oracle_fixed_rows(Ws, rows, nth)
+        if i >= args.warmup:
+            per.append((n_w, dt))
+    n_w = sum(a for a, _ in per)
+    t = sum(b for _, b in per)
+    value = n_w / t / 1e9
+    desc = (f"first {rows} rows of each of one layer's 7 matrices (layer = step index) at both settings, "
+            f"{per[0][0] / 1e6:.2f} M weight-solves per step, fp16, OpenMP over groups")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": config70(world, args.layers),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nth, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def _oracle_fixed_rows(Ws, rows, nth):
+    import oracle
+    n, t0 = 0, time.perf_counter()
+    for nb, g in SETTINGS70B:
+        for W in Ws:
+            w = W[:rows].contiguous().numpy()
+            oracle.quantize(w, nb, g, 1, 0.7, 1.0, 1.01, 20, 0, 8, dtype=oracle.F16, nthreads=nth)
+            n += w.size
+    return n, time.perf_counter() - t0, rows
+
+
 def config_dict(world):
     return {"workload": "llama2-7b-mlp-sweep", "model": "Llama-2-7B MLP shapes (synthetic weights)",
             "matrices": "gate 11008x4096, up 11008x4096, down 4096x11008 (out x in), bf16",
@@ -461,6 +520,282 @@ def run_stream(args):
                           "data": "synthetic; one layer's buffers streamed for every layer", "results": res}))
     if world > 1:
         torch.distributed.destroy_process_group()
+
+
+SETTINGS70B = [(2, 16), (4, 128)]
+
+
+def model70_calls(layers):
+    """The hqq_quantize calls of one step of the Llama-2-70B-shaped workload on
+    the given layers: the whole weight set at b2 g16, then at b4 g128."""
+    mats = synth.LLAMA2_70B.matrices()
+    return [(l, n, r, c, nb, g) for nb, g in SETTINGS70B for l in layers for n, r, c in mats]
+
+
+def host_bytes_available():
+    try:
+        import psutil
+        return int(psutil.virtual_memory().available)
+    except Exception:
+        return 0
+
+
+def oracle_rows_for_budget(Ws, settings, budget_s, nth, rows0=16, rows_cap=None):
+    """Rows per matrix so that the oracle over the first rows of every matrix
+    at every setting takes about budget_s seconds (calibrated on rows0 rows;
+    at most rows_cap, default the smallest matrix's row count)."""
+    import oracle
+    t0 = time.perf_counter()
+    for W, (nb, g) in ((W, st) for st in settings for W in Ws):
+        oracle.quantize(W[:rows0].contiguous().numpy(), nb, g, 1, 0.7, 1.0, 1.01, 20, 0, 8, dtype=oracle.F16,
+                        nthreads=nth)
+    dt = time.perf_counter() - t0
+    rows = int(rows0 * budget_s / max(dt, 1e-3))
+    return max(rows0, min(rows, rows_cap or min(W.shape[0] for W in Ws)))
+
+
+def oracle_70b_sample(Ws, budget_s, nth):
+    """The oracle, as it stands, on the first rows of each of one layer's
+    matrices (host fp16) at both settings; returns (weights, seconds, rows)."""
+    rows = oracle_rows_for_budget(Ws, SETTINGS70B, budget_s, nth)
+    return _oracle_fixed_rows(Ws, rows, nth)
+
+
+def config70(world, layers_total):
+    mats = synth.LLAMA2_70B.matrices()
+    w_layer = synth.LLAMA2_70B.weights_per_layer()
+    return {"workload": "llama2-70b", "model": "Llama-2-70B shapes, synthetic weights",
+            "layers": layers_total,
+            "matrices": ", ".join(f"{n} {r}x{c}" for n, r, c in mats) + " (out x in), fp16",
+            "settings": "nbits/group 2/16 and 4/128 (the whole weight set at each), axis 1, zero 8-bit, group stop, "
+                        "p 0.7, beta 1, kappa 1.01, 20 iters",
+            "calls_per_step": len(mats) * layers_total * len(SETTINGS70B),
+            "weights_per_step": w_layer * layers_total * len(SETTINGS70B),
+            "inputs": "per-layer seeds (1000*layer + matrix index), drawn on the GPU before the timed region, all "
+                      "layers resident in HBM",
+            "global_batch": world, "seq_len": None, "parallelism": f"layers split over {world} GPU(s)",
+            "l2": "each step reads 137 GB of distinct weights, far above the 126 MB L2"}
+
+
+def run_llama70(args):
+    """The default workload: a Llama-2-70B-shaped weight set (80 layers x q, o
+    8192x8192; k, v 1024x8192; gate, up 28672x8192; down 8192x28672; fp16,
+    per-layer seeds) quantised whole at b2 g16 and at b4 g128, 8-bit zero, group
+    stop.  One step = 1120 hqq_quantize calls over 136.9 G weights.
+
+    value = weights / device time (CUDA events on the launching stream), every
+            layer resident in HBM (drawn on the GPU before the timed region).
+    e2e   = the same weight set end to end through hqq_quantize_stream_jobs with
+            host buffers (pinned): every step copies all weights in and all
+            outputs out; timed with CUDA events around the blocking call.
+    Under torchrun the layers are split across ranks (rank_layers); each rank
+    holds and quantises its own layers; time = max over ranks."""
+    from calibration_free_weight_b200 import hqq
+    world, rank, local = dist_setup()
+    total_layers = args.layers
+    layers = rank_layers(total_layers, world, rank)
+    mats = synth.LLAMA2_70B.matrices()
+    w_layer = synth.LLAMA2_70B.weights_per_layer()
+    hbm_peak, sm_max, peak_kind = peaks()
+    stream = torch.cuda.current_stream()
+
+    t0 = time.perf_counter()
+    Wd = {(l, n): synth.weight_device(r, c, synth.seed_for(l, n)) for l in layers for n, r, c in mats}
+    torch.cuda.synchronize()
+    gen_s = time.perf_counter() - t0
+
+    outs, ws_bytes, g_max = {}, 0, 0
+    for nb, g in SETTINGS70B:
+        for n, r, c in mats:
+            G = r * c // g
+            outs[(n, nb, g)] = dict(packed=torch.empty(r * c * nb // 8, dtype=torch.uint8, device="cuda"),
+                                    scale=torch.empty(G, dtype=torch.float16, device="cuda"),
+                                    zero=torch.empty(G, dtype=torch.uint8, device="cuda"),
+                                    zero_meta=torch.empty(2, dtype=torch.float32, device="cuda"))
+            ws_bytes = max(ws_bytes, hqq.hqq_workspace_bytes(r, c, g, 1, 0, 8))
+            g_max = max(g_max, G)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    calls = model70_calls(layers)
+
+    def call(l, n, r, c, nb, g, dbg=None):
+        o = outs[(n, nb, g)]
+        rc = hqq.hqq_quantize(Wd[(l, n)], r, c, hqq.HQQ_F16, nb, g, 1, 0.7, 1.0, 1.01, 20, 0, 8, o["packed"],
+                              o["scale"], o["zero"], o["zero_meta"], ws, ws.numel(), dbg)
+        if rc != hqq.HQQ_OK:
+            raise RuntimeError(hqq.hqq_status_string(rc))
+
+    # algorithmic element-evaluations from the kept iterates (an untimed pass):
+    # the stop rule needs e_0 .. e_{k*+1}, i.e. k* + 2 evaluations, at most iters
+    bi_buf = torch.empty(g_max, dtype=torch.int32, device="cuda")
+    ev_dev = torch.zeros((), dtype=torch.int64, device="cuda")
+    for l, n, r, c, nb, g in calls:
+        G = r * c // g
+        call(l, n, r, c, nb, g, bi_buf[:G])
+        ev_dev += (bi_buf[:G].to(torch.int64) + 2).clamp_(max=20).sum() * g
+    evals = int(ev_dev.item())
+    del bi_buf
+
+    def one_step(rec=None):
+        for cl in calls:
+            if rec is not None:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+            call(*cl)
+            if rec is not None:
+                b.record(stream)
+                rec.append((a, b))
+
+    for _ in range(args.warmup):
+        one_step()
+    barrier(world)
+    rec = []
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        barrier(world)
+        clk.mark_start()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            one_step(rec)
+        ev1.record(stream)
+        barrier(world)
+        clk.mark_end()
+    if hqq.hqq_get_status(ws) != hqq.HQQ_OK:
+        raise RuntimeError("device status")
+    dev_ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    w_rank_step = w_layer * len(layers) * len(SETTINGS70B)
+    value = total_layers * w_layer * len(SETTINGS70B) * args.steps / (dev_ms / 1e3) / 1e9
+
+    call_ms = sum(a.elapsed_time(b) for a, b in rec)
+    n_calls = len(rec)
+    avg_ms = call_ms / max(1, n_calls)
+    mufu_ops = 2.0 * evals * args.steps  # over the timed calls
+    mufu_peak = SMS * MUFU_PER_CLK_PER_SM * sm_max * 1e6 / 1e9
+    achieved = mufu_ops / (call_ms / 1e3) / 1e9 if call_ms > 0 else 0.0
+    alg_step = sum(algorithmic_bytes(r, c, nb, g, 8) for _, _, r, c, nb, g in calls)
+    gbs = alg_step * args.steps / (call_ms / 1e3) / 1e9 if call_ms > 0 else 0.0
+    traffic = None
+    if TRAFFIC70["src_sha256"] == kernel_sources_sha() and TRAFFIC70["bytes_per_alg_byte"]:
+        traffic = TRAFFIC70["bytes_per_alg_byte"] * alg_step / len(calls)
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dev_ms / args.steps, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (Llama-2-70B shapes, weight statistics 0.02*N(0,1) with 0.1% outliers x10)",
+            "config": config70(world, total_layers),
+            "roofline": {"bound": "alu", "kernel": "solve_group_onepass_kernel", "achieved": achieved, "peak": mufu_peak,
+                         "unit": "Gop/s (MUFU lg2+ex2)", "frac": achieved / mufu_peak, "traffic": traffic,
+                         "traffic_unit": "DRAM bytes per call", "peak_kind": "nominal",
+                         "peak_basis": f"{SMS} SMs x {MUFU_PER_CLK_PER_SM} MUFU ops/clk x {sm_max:.0f} MHz "
+                                       f"(16/clk/SM confirmed by a microbenchmark of independent lg2/ex2 chains; "
+                                       f"not driver-measured)",
+                         "achieved_basis": "2 MUFU ops x (k*+2, at most 20) evaluations x group size, summed over "
+                                           "the timed calls, / the sum of their CUDA-event durations",
+                         "timed_unit": "one hqq_quantize call (its solver launches and the 8-bit zero launch)",
+                         "avg_call_ms": avg_ms, "evals_per_weight": evals / max(1, w_rank_step),
+                         "algorithmic_bytes_per_call": alg_step / len(calls),
+                         "hbm_gbs": gbs, "hbm_peak_gbs": hbm_peak, "hbm_peak_kind": peak_kind,
+                         "hbm_frac": gbs / hbm_peak},
+            "gpu_launches": None, "clocks": clk.summary(), "input_generation_s": gen_s}
+    line["gpu_launches"] = launches_per_call70(hqq) * len(calls) * args.steps
+
+    # end to end through the C ABI with host buffers
+    line["e2e"] = e2e70(args, hqq, world, rank, Wd, layers, mats, stream)
+    del Wd, outs, ws
+    torch.cuda.empty_cache()
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nth = os.cpu_count() or 1
+        Ws = [synth.weight_device(r, c, synth.seed_for(0, n)).cpu() for n, r, c in mats]
+        n, dt, rows = oracle_70b_sample(Ws, args.ref_budget, nth)
+        rate = n / dt
+        line["cpu_baseline"] = {
+            "value": rate / 1e9, "unit": UNIT, "cores": nth, "kind": "oracle",
+            "sample": f"first {rows} rows of each of layer 0's 7 matrices at both settings, {n / 1e6:.1f} M "
+                      f"weight-solves, fp16, OpenMP over groups",
+            "extrapolated_model_s": w_layer * total_layers * len(SETTINGS70B) / rate}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def launches_per_call70(hqq):
+    """Kernel launches of one group-stop hqq_quantize call with an 8-bit zero:
+    the solver's passes and the 8-bit zero quantiser."""
+    return solver_launches(0, 20, 16) + 1
+
+
+def host_plan70(avail, w_layer_bytes, out_layer_bytes, nlayers):
+    """How the end-to-end leg holds the weight set in host memory: (ring,
+    outs_per_job).  Every layer's weights get their own pinned buffers when
+    they fit (ring = nlayers), else a ring of as many layers as fit (at least
+    one); outputs get a buffer set per job when those fit too, else one set
+    per matrix and setting."""
+    if avail >= (w_layer_bytes + out_layer_bytes) * nlayers:
+        return nlayers, True
+    if avail >= w_layer_bytes * nlayers + out_layer_bytes:
+        return nlayers, False
+    ring = int((avail - out_layer_bytes) // w_layer_bytes) if avail > out_layer_bytes else 1
+    return max(1, min(ring, nlayers)), False
+
+
+def e2e70(args, hqq, world, rank, Wd, layers, mats, stream):
+    """The weight set through hqq_quantize_stream_jobs with host buffers.  The
+    device-resident weights are copied into pinned host memory (one distinct
+    buffer per matrix and layer when the host has room, else a ring of as many
+    layers as fit, reused in layer order); host outputs per job when they fit,
+    else per matrix and setting.  One untimed warm-up call on one layer, then
+    e2e_steps timed calls over the whole set (each one copies every weight in
+    and every output out)."""
+    nset = len(SETTINGS70B)
+    w_layer = sum(r * c for _, r, c in mats)
+    out_layer = {(nb, g): sum(r * c * nb // 8 + 3 * (r * c // g) + 8 for _, r, c in mats) for nb, g in SETTINGS70B}
+    ring, outs_per_job = host_plan70(host_bytes_available() - (16 << 30), 2 * w_layer, sum(out_layer.values()),
+                                     len(layers))
+    Wh = {}
+    for i, l in enumerate(layers[:ring]):
+        for n, r, c in mats:
+            h = torch.empty(r, c, dtype=torch.float16, pin_memory=True)
+            h.copy_(Wd[(l, n)])
+            Wh[(i, n)] = h
+    torch.cuda.synchronize()
+    host_o = {}
+
+    def host_out(key, r, c, nb, g):
+        if key not in host_o:
+            host_o[key] = hqq.host_outputs(r, c, nb, g, zero_nbits=8)
+        return host_o[key]
+
+    jobs_W, jobs_set, jobs_out = [], [], []
+    for nb, g in SETTINGS70B:
+        for i, l in enumerate(layers):
+            for n, r, c in mats:
+                jobs_W.append(Wh[(i % ring, n)])
+                jobs_set.append(dict(nbits=nb, group_size=g, axis=1, stop_mode=0, zero_nbits=8))
+                key = (l, n, nb, g) if outs_per_job else (n, nb, g)
+                jobs_out.append(host_out(key, r, c, nb, g))
+    k = len(mats)
+    buf, _ = hqq.quantize_stream_jobs(jobs_W[:k], jobs_set[:k], jobs_out[:k])  # warm-up: one layer
+    steps = max(1, min(args.steps, args.e2e_steps))
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        _, done = hqq.quantize_stream_jobs(jobs_W, jobs_set, jobs_out, device_buffer=buf)
+        if done != len(jobs_W):
+            raise RuntimeError("streamed run incomplete")
+    e1.record(stream)
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = 2 * w_layer * len(layers) * nset
+    d2h = sum(out_layer.values()) * len(layers)
+    del buf
+    return {"value": args.layers * w_layer * nset * steps / (ms / 1e3) / 1e9, "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "s_per_step": ms / 1e3 / steps, "api": "hqq_quantize_stream_jobs (C ABI), host buffers pinned",
+            "host_weights": ("one buffer per matrix and layer" if ring == len(layers) else
+                             f"a ring of {ring} layers' buffers reused in layer order (host memory)"),
+            "host_outputs": "one set per job" if outs_per_job else "one set per matrix and setting, reused"}
 
 
 LLAMA13B_NAMES = {"q": "self_attn.q_proj", "k": "self_attn.k_proj", "v": "self_attn.v_proj",
@@ -672,19 +1007,29 @@ def main():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--ref-budget", type=float, default=8.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-step", type=float, default=1.0, help="seconds of oracle work per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
                     help="single-matrix timing instead of the sweep: stop_mode,rows,cols,nbits,group_size[,reps]; "
                          "or scale8,G[,S[,reps]] for the 8-bit scale quantiser, "
                          "or gemv,rows,cols,nbits,g[,batch[,reps]] for the fused dequantise + matrix-vector product")
-    ap.add_argument("--workload", default="llama2-7b-mlp-sweep",
-                    choices=["llama2-7b-mlp-sweep", "llama2-70b-stream", "llama2-13b-stream"])
+    ap.add_argument("--workload", default="llama2-70b",
+                    choices=["llama2-70b", "llama2-7b-mlp-sweep", "llama2-70b-stream", "llama2-13b-stream"])
     ap.add_argument("--layers", type=int, default=None,
-                    help="layers of a streamed-model workload (default: the model's, 80 or 40)")
+                    help="layers of a model workload (default: the model's, 80 or 40)")
+    ap.add_argument("--e2e-steps", type=int, default=2,
+                    help="timed steps of the end-to-end leg of the llama2-70b workload (at most --steps)")
     args = ap.parse_args()
     args.layers_given = args.layers is not None
+    if args.workload == "llama2-70b" and not args.case:
+        if not args.layers_given:
+            args.layers = 80
+        if args.impl == "reference":
+            run_reference70(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        else:
+            run_llama70(args)
+        return
     if args.workload == "llama2-70b-stream":
         if not args.layers_given:
             args.layers = 80
@@ -770,7 +1115,7 @@ def main():
         fam[mode].append((a.elapsed_time(b), key))
     tot = {m: sum(t for t, _ in v) for m, v in fam.items()}
     dom = max(tot, key=tot.get)
-    dom_name = "solve_tensor_kernel" if dom == 1 else "solve_group_kernel"
+    dom_name = "solve_tensor_kernel" if dom == 1 else "solve_group_onepass_kernel"
     n_l = len(fam[dom])
     avg_ms = tot[dom] / n_l
     mufu_ops = sum(2 * evals[key] for _, key in fam[dom]) / n_l  # per call

@@ -111,16 +111,21 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     return d;
 }
 
-// The fast-path sums of one evaluation over a lane's E elements (E even, every
-// v clamp-free): sum |r|^p and sum W_q, with v, t, q, r, p*lg2|r| formed
-// pairwise by packed fp32 operations -- the same values as eval_elem_nc.  The
-// error is accumulated one element at a time in element order (the stop
-// decisions compare these sums, so their rounding is kept as the scalar loop
-// forms it); sum W_q is exact in any order (integers), so it is kept pairwise.
+// The fast-path sums of one evaluation over a lane's E elements (E a multiple
+// of 4, every v clamp-free): sum |r|^p and sum W_q, with v, t, q, r, p*lg2|r|
+// formed pairwise by packed fp32 operations -- the same values as
+// eval_elem_nc.  The error is accumulated one element at a time in element
+// order: the stop decisions compare these sums, and this order agrees with
+// the oracle's decisions at near ties more often than reordered partial sums
+// do (measured: with four interleaved partial sums, 7 of 4,800 groups kept
+// another iterate than the oracle in a 20-iteration no-stop run, against at
+// most 1 in element order).  Sum W_q is exact in any order (integers), so it
+// runs in two packed partial sums.
 template <int E>
 __device__ __forceinline__ void fast_sums(const float* ws, float z, float p, float* err_out, float* sq_out) {
+    static_assert(E % 4 == 0, "two packed partial sums");
     const uint64_t z2 = f2_pack(z, z), m2 = f2_pack(kMagic, kMagic), p2 = f2_pack(p, p);
-    uint64_t sq2 = f2_pack(0.0f, 0.0f);
+    uint64_t sq[2] = {f2_pack(0.0f, 0.0f), f2_pack(0.0f, 0.0f)};
     float err = 0.0f;
 #pragma unroll
     for (int i = 0; i < E; i += 2) {
@@ -132,10 +137,10 @@ __device__ __forceinline__ void fast_sums(const float* ws, float z, float p, flo
         float l0, l1;
         f2_unpack(f2_mul(f2_pack(lg2_approx(fabsf(r0)), lg2_approx(fabsf(r1))), p2), l0, l1);
         err = __fadd_rn(__fadd_rn(err, ex2_approx(l0)), ex2_approx(l1));
-        sq2 = f2_add(sq2, q);
+        sq[(i >> 1) & 1] = f2_add(sq[(i >> 1) & 1], q);
     }
     float s0, s1;
-    f2_unpack(sq2, s0, s1);
+    f2_unpack(f2_add(sq[0], sq[1]), s0, s1);
     *err_out = err;
     *sq_out = __fadd_rn(s0, s1);
 }

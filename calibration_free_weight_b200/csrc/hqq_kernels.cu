@@ -13,11 +13,13 @@
 // (add/sub/mul.rn.f32x2), and two MUFU ops (|r|^p through lg2/ex2), so the
 // MUFU pipe, not HBM, bounds the solver.
 //
-// Both solver kernels hold a warp tile of 32/P groups in registers, E = g/P
-// elements per lane (E = min(g, 32)), and re-read W from HBM rather than keep
-// a second copy on chip; no CTA ever waits for another.
+// The solver kernels hold a warp tile of 32/P groups in registers, E = g/P
+// elements per lane (E = min(g, 32)); no CTA ever waits for another.
 //
-// solve_group_kernel (group / no stop, both axes): a sequence of passes.  Pass
+// solve_group_onepass_kernel (group / no stop, axis 1): reads W once; groups
+//   that run past their first two evaluations wait in a per-warp pool in
+//   shared memory (see the kernel's own comment).
+// solve_group_kernel (group / no stop, axis 0): a sequence of passes.  Pass
 //   0 initialises every group (min/max -> s, z0; fp32 w*s; sum of w*s) and runs
 //   up to m_0 evaluations; a group that stops is packed and stored at once, a
 //   group still running leaves its state (z, best error, kept zero, s, z0,
@@ -71,6 +73,7 @@ constexpr int kWordStopAt = 6;  // tensor stop rule over the iterations run so f
 constexpr int kWordBestIt = 7;  // and the kept iterate + 1 (0: none), written by each chunk's last CTA
 constexpr int kWordPass = 8;   // survivor count of group pass p at kWordPass + p
 constexpr int kMaxPasses = 16;
+constexpr int kWordChunk = 24;  // words 24-25: next chunk of the one-pass group solver (64-bit counter)
 
 // ------------------------------------------------------- group outputs ----
 
@@ -980,6 +983,410 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 3) solve_group_kern
     if (k.zero_nbits == 8) merge_zero_range<kRegWarps>(k, zmin, zmax, sred);
 }
 
+// ====================================================== one-pass group stop ==
+//
+// solve_group_onepass_kernel (axis 1, group or no stop): every group is read
+// from HBM once and stays on chip from its first evaluation to its packed
+// codes.  A warp owns S = 32/P group slots (a slot is the P lanes of one
+// group) and works in rounds:
+//   fresh round: the next chunk of S consecutive groups (32*E contiguous
+//     16-bit elements, staged in shared memory by cp.async, the chunk after it
+//     already in flight) fills every slot; each is initialised and evaluated
+//     twice -- most groups stop there (group stop needs at least two
+//     evaluations) -- or, without early stopping, to the end;
+//   survivor round: when the warp's pool of running groups in shared memory
+//     holds S of them (or nothing else is left), S of them are restored to the
+//     slots and evaluated until fewer than S/2 still run (or, at the end, all
+//     have stopped).
+// After a round the stopped groups are packed and stored, and the running
+// ones go to the pool (raw values, scale, state: the codes of a group are
+// never recomputed from a second read of W).  Slots run at different
+// iteration indices; beta only matters on the rare proximal path, which takes
+// each slot's own.
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Packed min/max of eight 16-bit values held in a uint4 (fp16 or bf16; the
+// order of 16-bit values equals the order of their fp32 conversions).
+template <int DT>
+__device__ __forceinline__ void minmax8(const uint4 u, uint32_t& mn2, uint32_t& mx2) {
+    const uint32_t x[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (DT == 0) {
+            asm("min.f16x2 %0, %0, %1;" : "+r"(mn2) : "r"(x[i]));
+            asm("max.f16x2 %0, %0, %1;" : "+r"(mx2) : "r"(x[i]));
+        } else {
+            asm("min.bf16x2 %0, %0, %1;" : "+r"(mn2) : "r"(x[i]));
+            asm("max.bf16x2 %0, %0, %1;" : "+r"(mx2) : "r"(x[i]));
+        }
+    }
+}
+
+// Error-free sum of two floats (Knuth's TwoSum): s + e == a + b exactly.
+__device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
+    s = __fadd_rn(a, b);
+    const float bp = __fsub_rn(s, a);
+    e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bp)), __fsub_rn(b, bp));
+}
+
+// A fresh group for this lane's slot (fresh) from its raw 16-bit values:
+// min/max -> s, z0; fp32 w*s into ws; the sum of w*s as an unevaluated pair
+// hi + lo (hi = fl(hi + lo)) over the group's P lanes, accumulated by pairwise
+// TwoSum (no fp64 conversions: those issue on the pipe the solver is bound
+// by); and this lane's range of w*s.  Executed by every lane of the warp
+// (shuffles); lanes without a fresh group keep ws and the outputs unchanged.
+template <int DT, int E>
+__device__ __forceinline__ void init_fresh(const KParams& k, bool fresh, const uint4* raw, float* ws, float& s,
+                                           float& z0, F2& sws2, float& lmin, float& lmax) {
+    uint32_t mn2 = raw[0].x, mx2 = raw[0].x;
+#pragma unroll
+    for (int t = 0; t < E / kPiece; ++t) minmax8<DT>(raw[t], mn2, mx2);
+    const float lmn = fminf(bits_to_float<DT>(mn2 & 0xffffu), bits_to_float<DT>(mn2 >> 16));
+    const float lmx = fmaxf(bits_to_float<DT>(mx2 & 0xffffu), bits_to_float<DT>(mx2 >> 16));
+    const float mn = seg_min(lmn, k.P), mx = seg_max(lmx, k.P);
+    float sn = kScaleCap;
+    if (mx > mn) sn = fminf(__fdiv_rn(k.Lf, __fsub_rn(mx, mn)), kScaleCap);
+    float hi = 0.0f, lo = 0.0f;
+    if (fresh) {
+        s = sn;
+        z0 = __fmul_rn(-mn, sn);
+        lmin = __fmul_rn(lmn, sn);
+        lmax = __fmul_rn(lmx, sn);
+        const uint64_t s2 = f2_pack(sn, sn);
+        uint64_t acc[2] = {f2_pack(0.0f, 0.0f), f2_pack(0.0f, 0.0f)};
+        uint64_t cmp[2] = {f2_pack(0.0f, 0.0f), f2_pack(0.0f, 0.0f)};
+#pragma unroll
+        for (int t = 0; t < E / kPiece; ++t) {
+            float x[kPiece];
+            unpack8<DT>(raw[t], x);
+#pragma unroll
+            for (int i = 0; i < kPiece; i += 2) {
+                const int c = (i >> 1) & 1;  // two independent chains of packed pairs
+                const uint64_t w2 = f2_mul(f2_pack(x[i], x[i + 1]), s2);
+                f2_unpack(w2, ws[t * kPiece + i], ws[t * kPiece + i + 1]);
+                // TwoSum of the running pair and the two new products
+                const uint64_t sum = f2_add(acc[c], w2);
+                const uint64_t bp = f2_sub(sum, acc[c]);
+                cmp[c] = f2_add(cmp[c], f2_add(f2_sub(acc[c], f2_sub(sum, bp)), f2_sub(w2, bp)));
+                acc[c] = sum;
+            }
+        }
+        float a0, a1, a2, a3, c0, c1, h0, h1, e0, e1, a, e2;
+        f2_unpack(acc[0], a0, a1);
+        f2_unpack(acc[1], a2, a3);
+        f2_unpack(f2_add(cmp[0], cmp[1]), c0, c1);
+        two_sum(a0, a1, h0, e0);
+        two_sum(a2, a3, h1, e1);
+        two_sum(h0, h1, a, e2);
+        const float c = __fadd_rn(__fadd_rn(c0, c1), __fadd_rn(__fadd_rn(e0, e1), e2));
+        hi = __fadd_rn(a, c);  // Fast2Sum (|a| >= |c|)
+        lo = __fsub_rn(c, __fsub_rn(hi, a));
+    }
+    for (int o = 1; o < k.P; o <<= 1) {
+        const float h2 = __shfl_xor_sync(kFull, hi, o), l2 = __shfl_xor_sync(kFull, lo, o);
+        float h, e;
+        two_sum(hi, h2, h, e);
+        const float l = __fadd_rn(__fadd_rn(lo, l2), e);
+        hi = __fadd_rn(h, l);
+        lo = __fsub_rn(l, __fsub_rn(hi, h));
+    }
+    if (fresh) sws2 = F2{hi, lo};
+}
+
+// Packed codes of this lane's E elements at zero-point z (axis 1); cf: every
+// v = fl(fl(w*s) + z) of the lane is clamp-free, so the code is read from the
+// rounding sum's low mantissa bits without the clamp.
+template <int E, int NBITS>
+__device__ __forceinline__ void store_codes_lane(const KParams& k, int64_t j, int part, const float* ws, float z,
+                                                 bool cf) {
+    constexpr float Lf = static_cast<float>((1 << NBITS) - 1);
+    constexpr int kWords = (E * NBITS + 31) / 32;
+    uint32_t wd[kWords];
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) wd[w] = 0u;
+    const uint64_t z2 = f2_pack(z, z), m2 = f2_pack(kMagic, kMagic);
+    if (cf && NBITS != 3) {
+        // t = fl(fl(w*s + z) + 1.5*2^23) holds its code in the low mantissa bits,
+        // bits(t) = bits(1.5*2^23) + code: a word is the sum of bits(t_i) << (i*NBITS)
+        // less the magic's share (mod 2^32) -- one shifted add per code
+#pragma unroll
+        for (int i = 0; i < E; i += 2) {
+            float t0, t1;
+            f2_unpack(f2_add(f2_add(f2_pack(ws[i], ws[i + 1]), z2), m2), t0, t1);
+            wd[(i * NBITS) / 32] += __float_as_uint(t0) << ((i * NBITS) % 32);
+            wd[((i + 1) * NBITS) / 32] += __float_as_uint(t1) << (((i + 1) * NBITS) % 32);
+        }
+        constexpr uint32_t kOnes = NBITS == 8 ? 0x01010101u
+                                   : NBITS == 4 ? 0x11111111u
+                                   : NBITS == 2 ? 0x55555555u
+                                                : 0xffffffffu;  // sum of 1 << (i*NBITS % 32) over a full word
+        constexpr int kPerWord = 32 / NBITS;
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) {
+            const int n_in = E - w * kPerWord < kPerWord ? E - w * kPerWord : kPerWord;  // codes in this word
+            const uint32_t ones = n_in == kPerWord ? kOnes : (kOnes & ((1u << (n_in * NBITS)) - 1u));
+            wd[w] -= kMagicBits * ones;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < E; i += 2) {
+            uint32_t c2[2];
+            if (cf) {
+                float t0, t1;
+                f2_unpack(f2_add(f2_add(f2_pack(ws[i], ws[i + 1]), z2), m2), t0, t1);
+                c2[0] = __float_as_uint(t0) - kMagicBits;
+                c2[1] = __float_as_uint(t1) - kMagicBits;
+            } else {
+                round_clamp(__fadd_rn(ws[i], z), Lf, &c2[0]);
+                round_clamp(__fadd_rn(ws[i + 1], z), Lf, &c2[1]);
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int b = (i + h) * NBITS;
+                wd[b / 32] |= c2[h] << (b % 32);
+                if (b % 32 + NBITS > 32) wd[b / 32 + 1] |= c2[h] >> (32 - b % 32);
+            }
+        }
+    }
+    constexpr int kBytes = E * NBITS / 8;
+    uint8_t* dst = k.packed + (j * (k.g / E) + part) * kBytes;
+    if (kBytes % 16 == 0) {
+#pragma unroll
+        for (int q = 0; q < kBytes / 16; ++q)
+            reinterpret_cast<uint4*>(dst)[q] = make_uint4(wd[4 * q], wd[4 * q + 1], wd[4 * q + 2], wd[4 * q + 3]);
+    } else if (kBytes == 8) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(wd[0], wd[kWords > 1 ? 1 : 0]);
+    } else if (kBytes == 4) {
+        *reinterpret_cast<uint32_t*>(dst) = wd[0];
+    } else if (kBytes == 2) {
+        *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(wd[0]);
+    } else if (kBytes == 1) {
+        *dst = static_cast<uint8_t>(wd[0]);
+    } else if (kBytes == 12) {  // 3-bit, E = 32: 4-byte aligned
+#pragma unroll
+        for (int q = 0; q < 3; ++q) reinterpret_cast<uint32_t*>(dst)[q] = wd[q];
+    } else if (kBytes == 6) {  // 3-bit, E = 16: 2-byte aligned
+#pragma unroll
+        for (int q = 0; q < 3; ++q) reinterpret_cast<uint16_t*>(dst)[q] = static_cast<uint16_t>(wd[q / 2] >> (16 * (q & 1)));
+    } else {  // 3-bit, E = 8: 3 bytes
+#pragma unroll
+        for (int q = 0; q < kBytes; ++q) dst[q] = static_cast<uint8_t>(wd[0] >> (8 * q));
+    }
+}
+
+template <int E>
+__device__ __forceinline__ void store_codes_lane_n(const KParams& k, int64_t j, int part, const float* ws, float z,
+                                                   bool cf) {
+    switch (k.nbits) {
+        case 1: store_codes_lane<E, 1>(k, j, part, ws, z, cf); break;
+        case 2: store_codes_lane<E, 2>(k, j, part, ws, z, cf); break;
+        case 3: store_codes_lane<E, 3>(k, j, part, ws, z, cf); break;
+        case 4: store_codes_lane<E, 4>(k, j, part, ws, z, cf); break;
+        default: store_codes_lane<E, 8>(k, j, part, ws, z, cf); break;
+    }
+}
+
+// Shared memory of one warp of the one-pass kernel, in uint4 units: two chunk
+// buffers of 32*E 16-bit values, and a pool of 2S running groups stored as 64
+// lane records (a group's P lanes), structure of arrays: record field f of
+// record r at pool[f * 64 + r], fields 0 .. E/8-1 the lane's raw values, then
+// (s, z, z0, best error), (kept zero, sum hi, sum lo, lane min w*s),
+// (lane max w*s, kept iterate, iteration, group lo), (group hi, -, -, -).
+__host__ __device__ constexpr int onepass_fields(int E) { return E / kPiece + 4; }
+__host__ __device__ constexpr int onepass_warp_uint4(int E) { return 8 * E + 64 * onepass_fields(E); }
+constexpr int kPoolRecords = 64;
+__host__ __device__ constexpr int onepass_ctas(int E) { return E >= 32 ? 2 : (E == 16 ? 3 : 4); }
+
+template <int DT, int E>
+__global__ void __launch_bounds__(kRegThreads, onepass_ctas(E))
+    solve_group_onepass_kernel(const KParams k, int64_t nchunks) {
+    extern __shared__ uint4 dyn_smem[];
+    __shared__ float2 sred[kRegWarps];
+    constexpr int F = onepass_fields(E);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint4* const cbuf = dyn_smem + warp * onepass_warp_uint4(E);  // [2][4E]
+    uint4* const pool = cbuf + 8 * E;                              // [F][64]
+    const int logP = k.logP;
+    const int part = lane & (k.P - 1);
+    const int slot = lane >> logP;
+    const int S = 32 >> logP;  // group slots per warp
+    const bool stop_group = k.stop_mode == 0;
+    const int m_fresh = stop_group ? 2 : k.iters_eff;  // evaluations of a fresh round
+    const float inv_g = 1.0f / static_cast<float>(k.g);
+    const float thr = shrink_threshold(k.beta_last, k.p);  // smallest threshold of the run: a conservative gate
+    unsigned long long* const counter = reinterpret_cast<unsigned long long*>(k.counters + kWordChunk);
+    const unsigned leader = lane & ~(k.P - 1);  // first lane of this lane's slot
+    const unsigned below = (1u << leader) - 1u;
+    float zmin = FLT_MAX, zmax = -FLT_MAX;
+
+    // take the next chunk and start copying it into buffer b; returns its group count
+    auto fetch = [&](int b, int64_t& c_out) -> int {
+        unsigned long long c = 0;
+        if (lane == 0) c = atomicAdd(counter, 1ull);
+        c = __shfl_sync(kFull, c, 0);
+        int cnt = 0;
+        if (static_cast<int64_t>(c) < nchunks) {
+            const int64_t g0 = static_cast<int64_t>(c) * S;
+            cnt = static_cast<int>(k.G - g0 < S ? k.G - g0 : S);
+            if (lane * E < cnt * k.g) {
+                const uint4* src = reinterpret_cast<const uint4*>(k.W + g0 * k.g + lane * E);
+#pragma unroll
+                for (int t = 0; t < E / kPiece; ++t) cp_async16(cbuf + b * 4 * E + lane * (E / kPiece) + t, src + t);
+            }
+        }
+        cp_async_commit();
+        c_out = static_cast<int64_t>(c);
+        return cnt;
+    };
+
+    int cur = 0;
+    int64_t cur_c, nxt_c;
+    int cur_cnt = fetch(0, cur_c);
+    int nxt_cnt = fetch(1, nxt_c);
+    int pool_n = 0;  // running groups in the pool
+
+    float ws[E];
+    float s = 1.0f, z = 0.0f, z0 = 0.0f, be = INFINITY, zb = 0.0f, lmin = 0.0f, lmax = 0.0f;
+    F2 sws2{0.0f, 0.0f};
+    int bi = 0, it = 0;
+    int64_t j = 0;
+
+    for (;;) {
+        const bool survivor = pool_n >= S || (cur_cnt == 0 && pool_n > 0);
+        if (!survivor && cur_cnt == 0) break;  // nothing left
+        bool has = false;  // this slot holds a group this round
+        uint4 raw[E / kPiece];
+        if (survivor) {
+            const int n = pool_n < S ? pool_n : S;
+            has = slot < n;
+            if (has) {
+                const int r = (pool_n - n + slot) * k.P + part;
+#pragma unroll
+                for (int t = 0; t < E / kPiece; ++t) raw[t] = pool[t * kPoolRecords + r];
+                const uint4 f0 = pool[(E / kPiece) * kPoolRecords + r];
+                const uint4 f1 = pool[(E / kPiece + 1) * kPoolRecords + r];
+                const uint4 f2 = pool[(E / kPiece + 2) * kPoolRecords + r];
+                const uint4 f3 = pool[(E / kPiece + 3) * kPoolRecords + r];
+                s = __uint_as_float(f0.x);
+                z = __uint_as_float(f0.y);
+                z0 = __uint_as_float(f0.z);
+                be = __uint_as_float(f0.w);
+                zb = __uint_as_float(f1.x);
+                sws2 = F2{__uint_as_float(f1.y), __uint_as_float(f1.z)};
+                lmin = __uint_as_float(f1.w);
+                lmax = __uint_as_float(f2.x);
+                bi = static_cast<int>(f2.y);
+                it = static_cast<int>(f2.z);
+                j = static_cast<int64_t>((static_cast<uint64_t>(f3.x) << 32) | f2.w);
+                const uint64_t s2 = f2_pack(s, s);
+#pragma unroll
+                for (int t = 0; t < E / kPiece; ++t) {  // fl(w*s), as at initialisation
+                    float x[kPiece];
+                    unpack8<DT>(raw[t], x);
+#pragma unroll
+                    for (int i = 0; i < kPiece; i += 2)
+                        f2_unpack(f2_mul(f2_pack(x[i], x[i + 1]), s2), ws[t * kPiece + i], ws[t * kPiece + i + 1]);
+                }
+            }
+            pool_n -= n;
+            __syncwarp();  // every lane has read its record before records are rewritten at the end of the round
+        } else {
+            cp_async_wait<1>();
+            __syncwarp();  // this chunk has landed in every lane's copy
+            has = slot < cur_cnt;
+            const uint4* src = cbuf + cur * 4 * E + lane * (E / kPiece);
+#pragma unroll
+            for (int t = 0; t < E / kPiece; ++t) raw[t] = has ? src[t] : make_uint4(0, 0, 0, 0);
+            j = cur_c * S + slot;
+            __syncwarp();  // every lane has read the buffer: refill it with the chunk after next
+            int64_t c_new;
+            const int cnt_new = fetch(cur, c_new);
+            cur ^= 1;
+            cur_c = nxt_c;
+            cur_cnt = nxt_cnt;
+            nxt_c = c_new;
+            nxt_cnt = cnt_new;
+            init_fresh<DT, E>(k, has, raw, ws, s, z0, sws2, lmin, lmax);
+            if (has) {
+                z = zb = z0;
+                be = INFINITY;
+                bi = 0;
+                it = 0;
+            }
+        }
+        bool alive = has && it < k.iters_eff;
+        // ---------------------------------------------- evaluations -------
+        const bool more = pool_n > 0 || cur_cnt > 0;  // work beyond this round
+        for (int e = 0;; ++e) {
+            const int n_alive = __popc(__ballot_sync(kFull, part == 0 && alive));
+            if (n_alive == 0) break;
+            if (!survivor && e >= m_fresh) break;
+            if (survivor && more && 2 * n_alive < S) break;
+            WarpTile wt;
+            wt.valid = alive;
+            wt.j = j;
+            wt.part = part;
+            float err, sq;
+            bool sp;
+            double swe;
+            eval_lane_reload<DT, 1, E>(k, wt, ws, lmin, lmax, s, z, z0, it, thr, &err, &sq, &sp, &swe);
+            if (alive) {
+                const bool improved = err < be;
+                if (improved) {
+                    be = err;
+                    zb = z;
+                    bi = it;
+                }
+                bool stop = (stop_group && !improved) || it >= k.iters_eff - 1;
+                if (!stop) {
+                    const float zn = sp ? zero_from_sums(sq, swe, k.g) : zero_from_sums_f2(sq, sws2, inv_g);
+                    if (stop_group && zn == z) stop = true;  // fixed point: the next error equals this one
+                    else z = zn;
+                }
+                if (stop) alive = false;
+                else ++it;
+            }
+        }
+        // ------------------------------------------ stopped: outputs -------
+        if (has && !alive) {
+            store_codes_lane_n<E>(k, j, part, ws, zb, clamp_free(lmin, lmax, zb, k.Lf));
+            if (part == 0) {
+                const float err_mean = k.dbg_err ? be * pow_pos(s, -k.p) * inv_g : 0.0f;
+                store_group(k, j, s, zb, bi, err_mean, &zmin, &zmax);
+            }
+        }
+        // ------------------------------------------ running: to the pool ---
+        const unsigned run = __ballot_sync(kFull, part == 0 && alive);
+        if (alive) {
+            const int r = (pool_n + __popc(run & below)) * k.P + part;
+#pragma unroll
+            for (int t = 0; t < E / kPiece; ++t) pool[t * kPoolRecords + r] = raw[t];
+            pool[(E / kPiece) * kPoolRecords + r] =
+                make_uint4(__float_as_uint(s), __float_as_uint(z), __float_as_uint(z0), __float_as_uint(be));
+            pool[(E / kPiece + 1) * kPoolRecords + r] = make_uint4(__float_as_uint(zb), __float_as_uint(sws2.hi),
+                                                                   __float_as_uint(sws2.lo), __float_as_uint(lmin));
+            pool[(E / kPiece + 2) * kPoolRecords + r] =
+                make_uint4(__float_as_uint(lmax), static_cast<uint32_t>(bi), static_cast<uint32_t>(it),
+                           static_cast<uint32_t>(static_cast<uint64_t>(j)));
+            pool[(E / kPiece + 3) * kPoolRecords + r] =
+                make_uint4(static_cast<uint32_t>(static_cast<uint64_t>(j) >> 32), 0u, 0u, 0u);
+        }
+        pool_n += __popc(run);
+        __syncwarp();  // pool writes visible to the whole warp before the next round reads them
+    }
+    cp_async_wait<0>();
+    if (k.zero_nbits == 8) merge_zero_range<kRegWarps>(k, zmin, zmax, sred);
+}
+
 // ------------------------------------------------------- 8-bit zero ------
 
 // One RTN quantiser for all kept zeros of the tensor, from their min/max
@@ -1205,7 +1612,7 @@ DevInfo device_info() {
 
 template <typename K>
 cudaError_t persistent_grid(K kernel, int threads, size_t smem, int64_t work_units, int* grid) {
-    if (smem > 48 * 1024) {
+    if (smem > 47 * 1024) {  // with the kernel's static shared memory, beyond the default 48 KB
         const cudaError_t e =
             cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
@@ -1278,6 +1685,19 @@ cudaError_t launch_group(KParams& k, const WorkspaceLayout& L, uint8_t* ws, cuda
     return cudaSuccess;
 }
 
+template <int DT, int E>
+cudaError_t launch_group_onepass(KParams& k, cudaStream_t stream) {
+    auto kern = solve_group_onepass_kernel<DT, E>;
+    const int S = 32 >> k.logP;
+    const int64_t nchunks = (k.G + S - 1) / S;
+    const size_t smem = sizeof(uint4) * static_cast<size_t>(onepass_warp_uint4(E)) * kRegWarps;
+    int grid = 0;
+    cudaError_t err = persistent_grid(kern, kRegThreads, smem, (nchunks + kRegWarps - 1) / kRegWarps, &grid);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, kRegThreads, smem, stream>>>(k, nchunks);
+    return cudaGetLastError();
+}
+
 template <int DT, int AXIS, int E>
 cudaError_t launch_tensor(KParams& k, cudaStream_t stream) {
     const int gpw = 32 >> k.logP;
@@ -1319,6 +1739,7 @@ cudaError_t launch_tensor(KParams& k, cudaStream_t stream) {
 template <int DT, int AXIS, int E>
 cudaError_t launch_solver(KParams& k, const WorkspaceLayout& L, uint8_t* ws, cudaStream_t stream) {
     if (k.stop_mode == 1) return launch_tensor<DT, AXIS, E>(k, stream);
+    if (AXIS == 1) return launch_group_onepass<DT, E>(k, stream);
     return launch_group<DT, AXIS, E>(k, L, ws, stream);
 }
 
@@ -1375,6 +1796,8 @@ WorkspaceLayout workspace_layout(int64_t rows, int64_t cols, int g, int axis, in
         l.t_zs = off;  // z of every iteration of two chunks
         const size_t slots = static_cast<size_t>(chunk_max(chunk_len(g < 32 ? g : 32)) + 1);
         off = up(off + 4 * 2 * slots * Gs);
+    } else if (axis == 1) {
+        l.slice = group_entries(rows, cols, g, axis);  // one pass over every group: no per-group state
     } else {
         const int64_t n = group_entries(rows, cols, g, axis);
         constexpr int64_t kMaxSlice = int64_t{1} << 31;  // survivor lists hold 32-bit entry offsets
@@ -1397,7 +1820,7 @@ WorkspaceLayout workspace_layout(int64_t rows, int64_t cols, int g, int axis, in
 int64_t fit_slice(int64_t rows, int64_t cols, int g, int axis, int stop_mode, int zero_nbits, size_t bytes) {
     const WorkspaceLayout full = workspace_layout(rows, cols, g, axis, stop_mode, zero_nbits, 0);
     if (full.total <= bytes) return full.slice > 0 ? full.slice : 1;
-    if (stop_mode == 1) return 0;
+    if (stop_mode == 1 || axis == 1) return 0;  // nothing to cut into slices
     const WorkspaceLayout base = workspace_layout(rows, cols, g, axis, stop_mode, zero_nbits, 1);
     const size_t fixed = base.state;  // header and kept zeros
     const size_t per = 44;            // bytes per entry of a slice, before each part's rounding to 256

@@ -9,6 +9,8 @@ picks outliers, which are multiplied by 10; the result is cast to the stated
 dtype.  Both draws come from one CPU ``torch.Generator`` seeded with ``seed``,
 ``randn`` first and ``rand`` second.  Model weight sets use
 seed = 1000 * layer + matrix index (q=0, k=1, v=2, o=3, gate=4, up=5, down=6).
+weight_device() draws the same recipe on the GPU (for the 70B-shaped set,
+137 GB of fp16 weights).
 """
 from dataclasses import dataclass
 
@@ -28,6 +30,20 @@ def weight(rows: int, cols: int, seed: int, dtype=torch.float16, std: float = ST
     w = torch.randn(rows, cols, generator=g, dtype=torch.float32) * std
     mask = torch.rand(rows, cols, generator=g) < outlier_frac
     w = torch.where(mask, w * outlier_scale, w)
+    return w.to(dtype)
+
+
+def weight_device(rows: int, cols: int, seed: int, dtype=torch.float16, device="cuda", std: float = STD,
+                  outlier_frac: float = OUTLIER_FRAC, outlier_scale: float = OUTLIER_SCALE) -> torch.Tensor:
+    """The same recipe drawn on the GPU (one CUDA ``torch.Generator`` seeded
+    with ``seed``, ``randn`` then ``rand``), for weight sets too large to draw
+    on the host in reasonable time.  The values differ from weight()'s for the
+    same seed (another generator); the distribution is the same."""
+    g = torch.Generator(device).manual_seed(int(seed))
+    w = torch.randn(rows, cols, generator=g, device=device, dtype=torch.float32).mul_(std)
+    mask = torch.rand(rows, cols, generator=g, device=device) < outlier_frac
+    w = torch.where(mask, w * outlier_scale, w)
+    del mask
     return w.to(dtype)
 
 

@@ -102,9 +102,9 @@ int64_t hqq_num_groups(int64_t rows, int64_t cols, int group_size, int axis);
 
 /* Bytes of device workspace hqq_quantize needs for this problem (always > 0;
  * holds the status word, the work counters, the fp32 kept zeros of the 8-bit
- * zero path (4 bytes per group, hence zero_nbits), the running state of
- * groups between passes and, for the tensor stop, the per-group state,
- * per-CTA partials and per-iteration errors).  0 for invalid args.  The pages
+ * zero path (4 bytes per group, hence zero_nbits), for axis 0 the running
+ * state of groups between passes and, for the tensor stop, the per-group
+ * state, per-CTA partials and per-iteration errors).  0 for invalid args.  The pages
  * have no counterpart: their solver runs as whole-tensor operations that
  * allocate as they go; here the caller owns every byte. */
 size_t hqq_workspace_bytes(int64_t rows, int64_t cols, int group_size, int axis, int stop_mode, int zero_nbits);
@@ -377,16 +377,18 @@ const char* hqq_status_string(int status);
  * be HQQ_STOP_GROUP or HQQ_STOP_NONE; HQQ_STOP_TENSOR returns
  * HQQ_ERR_INVALID_ARG (use hqq_quantize for it).
  * Scratch: one buffer of HQQ_NOALLOC_SCRATCH_BYTES (16 MiB) of device memory per
- * GPU, held by the library from load until the process exits.  A problem whose
- * hqq_workspace_bytes() exceeds it runs in slices of groups, one after another
- * on `stream` (same results); each slice needs 44 bytes per entry and at least
- * 4,096 entries (an entry is a group; with axis = 0 the columns of each block
- * of group_size rows are counted up to whole warp tiles of 32/P groups, P =
- * group_size/32 for group_size >= 32, else 1).  With zero_nbits = 8 the kept
- * zeros of all groups (4 bytes each, the array rounded up to 256 bytes) must
- * fit beside one slice and a 256-byte header: 4,149,184 groups fit exactly,
- * more return HQQ_ERR_WORKSPACE before anything is launched.  With
- * zero_nbits = 16 every size fits.
+ * GPU, held by the library from load until the process exits.  Axis 1 needs a
+ * 256-byte header and, with zero_nbits = 8, the kept zeros of all groups (4
+ * bytes each): 4,194,240 groups fit exactly.  Axis 0 keeps running state per
+ * group; a problem whose hqq_workspace_bytes() exceeds the scratch runs in
+ * slices of groups, one after another on `stream` (same results); each slice
+ * needs 44 bytes per entry and at least 4,096 entries (an entry is a group;
+ * the columns of each block of group_size rows are counted up to whole warp
+ * tiles of 32/P groups, P = group_size/32 for group_size >= 32, else 1), and
+ * with zero_nbits = 8 the kept zeros (the array rounded up to 256 bytes) must
+ * fit beside one slice and the header: 4,149,184 groups fit exactly.  More
+ * return HQQ_ERR_WORKSPACE before anything is launched.  With zero_nbits = 16
+ * every size fits.
  * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
  * routine).  The first call on each device looks up the buffer's device
  * address (cudaGetSymbolAddress) with that device current; make that first call

@@ -290,17 +290,21 @@ def test_binding_fails_loudly_without_library(tmp_path):
 
 @pytest.mark.parametrize("axis", [1, 0])
 def test_noalloc_zero8_limit_is_exact(hq, axis):
-    """hqq_quantize_noalloc with an 8-bit zero: 4,149,184 groups (the kept
-    zeros, 4 bytes each, plus a 256-byte header and one 4,096-entry slice fill
-    the 16 MiB scratch exactly) are accepted by the size check; one group more
-    is refused with HQQ_ERR_WORKSPACE before anything else happens.  The
-    accepted call then fails on its missing buffers (or, with no GPU, on the
-    device query), never on the size."""
+    """hqq_quantize_noalloc with an 8-bit zero.  Axis 1 needs only the kept
+    zeros (4 bytes each) beside a 256-byte header: 4,194,240 groups fill the
+    16 MiB scratch.  Axis 0 also needs one slice of 4,096 entries of running
+    state: 4,149,184 groups fill it.  At the limit the size check passes;
+    one group more is refused with HQQ_ERR_WORKSPACE before anything else
+    happens.  The accepted call then fails on its missing buffers (or, with
+    no GPU, on the device query), never on the size."""
     def call(rows, cols):
-        if axis == 0:
-            rows, cols = cols, rows
         return hq.lib.hqq_quantize_noalloc(None, rows, cols, hq.HQQ_F16, 2, 16, axis, 0.7, 1.0, 1.01, 20,
                                            hq.HQQ_STOP_GROUP, 8, None, None, None, None, None, None, None, None)
-    assert 64831 * 1024 // 16 == 4_149_184 and 829837 * 80 // 16 == 4_149_185
-    assert call(64831, 1024) not in (hq.HQQ_ERR_WORKSPACE, hq.HQQ_OK)
-    assert call(829837, 80) == hq.HQQ_ERR_WORKSPACE
+    if axis == 1:
+        fit, over = (4_194_240, 16), (4_194_241, 16)
+    else:
+        fit, over = (1024, 64831), (80, 829837)
+    assert fit[0] * fit[1] // 16 == (4_194_240 if axis == 1 else 4_149_184)
+    assert over[0] * over[1] // 16 == fit[0] * fit[1] // 16 + 1
+    assert call(*fit) not in (hq.HQQ_ERR_WORKSPACE, hq.HQQ_OK)
+    assert call(*over) == hq.HQQ_ERR_WORKSPACE

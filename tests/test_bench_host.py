@@ -13,10 +13,12 @@ from calibration_free_weight_b200 import synth  # noqa: E402
 
 
 def test_solver_launches_follow_the_schedules():
-    # group stop: passes of 2 and 3 evaluations, then the rest
-    assert bench.solver_launches(0, 20) == 3
-    assert bench.solver_launches(0, 5) == 2 and bench.solver_launches(0, 6) == 3
-    assert bench.solver_launches(0, 2) == 1 and bench.solver_launches(0, 1) == 1
+    # group stop, axis 1: one launch of the one-pass kernel
+    assert bench.solver_launches(0, 20) == 1 and bench.solver_launches(0, 20, 16) == 1
+    # axis 0: passes of 2 and 3 evaluations, then the rest
+    assert bench.solver_launches(0, 20, axis=0) == 3
+    assert bench.solver_launches(0, 5, axis=0) == 2 and bench.solver_launches(0, 6, axis=0) == 3
+    assert bench.solver_launches(0, 2, axis=0) == 1 and bench.solver_launches(0, 1, axis=0) == 1
     # no stop: one pass
     assert bench.solver_launches(2, 20) == 1
     # tensor stop, g <= 16: chunks [0,2) [2,6) [6,10) [10,14) [14,18) [18,20) + the writing launch
@@ -63,3 +65,28 @@ def test_oracle_model_rate_extrapolates_from_its_sample():
     assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] > 0
     assert abs(cb["extrapolated_model_s"] - 1e9 / (cb["value"] * 1e9)) < 1e-6 * cb["extrapolated_model_s"]
     assert "first 16 rows" in cb["sample"]
+
+
+def test_llama70_plan():
+    """The default workload: 80 layers x 7 matrices at two settings = 1120
+    calls and 136.9 G weights per step; layers split across ranks cover every
+    layer exactly once."""
+    calls = bench.model70_calls(range(80))
+    assert len(calls) == 1120
+    assert sum(r * c for _, _, r, c, _, _ in calls) == 2 * 80 * synth.LLAMA2_70B.weights_per_layer()
+    assert 2 * 80 * synth.LLAMA2_70B.weights_per_layer() == 136_902_082_560
+    assert {(nb, g) for *_, nb, g in calls} == {(2, 16), (4, 128)}
+    for world in (1, 2, 4, 8):
+        got = sorted(l for r in range(world) for l in bench.rank_layers(80, world, r))
+        assert got == list(range(80))
+    cfg = bench.config70(1, 80)
+    assert cfg["workload"] == "llama2-70b" and cfg["calls_per_step"] == 1120
+    assert cfg["weights_per_step"] == 136_902_082_560
+
+
+def test_llama70_host_plan():
+    GB = 1 << 30
+    assert bench.host_plan70(400 * GB, 2 * GB, 1 * GB, 80) == (80, True)
+    assert bench.host_plan70(170 * GB, 2 * GB, 1 * GB, 80) == (80, False)
+    assert bench.host_plan70(41 * GB, 2 * GB, 1 * GB, 80) == (20, False)
+    assert bench.host_plan70(0, 2 * GB, 1 * GB, 80) == (1, False)
