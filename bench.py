@@ -968,6 +968,32 @@ def run_gemm_case(spec):
                       "hbm_frac": nbytes / (med / 1e3) / 1e9 / hbm, "l2": "flushed before every call"}))
 
 
+def run_half_case(spec):
+    """Time the half-precision solver variant beside hqq_quantize on one
+    synthetic fp16 matrix: "half,rows,cols,nbits,g[,reps]" (group stop, 8-bit
+    zero); L2 holds none of a large matrix between calls."""
+    from calibration_free_weight_b200 import hqq
+    v = [int(x) for x in spec.split(",")[1:]]
+    rows, cols, nbits, g = v[:4]
+    reps = v[4] if len(v) > 4 else 5
+    torch.cuda.set_device(0)
+    W = synth.weight(rows, cols, seed=4, dtype=torch.float16).cuda()
+    res = {}
+    for name, fn in (("fp32", hqq.quantize), ("half", hqq.quantize_half)):
+        out = fn(W, nbits, g, zero_nbits=8)
+        ev = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn(W, nbits, g, zero_nbits=8, out=out)
+            b.record()
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        ms = min(a.elapsed_time(b) for a, b in ev)
+        res[name] = {"ms": ms, "gweights_s": rows * cols / (ms / 1e3) / 1e9}
+    print(json.dumps({"case": spec, **res, "half_over_fp32": res["fp32"]["ms"] / res["half"]["ms"]}))
+
+
 def run_case(spec):
     """Time hqq_quantize on one synthetic bf16 matrix (used for kernel profiles)."""
     if spec.startswith("scale8"):
@@ -978,6 +1004,9 @@ def run_case(spec):
         return
     if spec.startswith("gemm"):
         run_gemm_case(spec)
+        return
+    if spec.startswith("half"):
+        run_half_case(spec)
         return
     from calibration_free_weight_b200 import hqq
     v = [int(x) for x in spec.split(",")]
@@ -1013,7 +1042,8 @@ def main():
     ap.add_argument("--case", default=None,
                     help="single-matrix timing instead of the sweep: stop_mode,rows,cols,nbits,group_size[,reps]; "
                          "or scale8,G[,S[,reps]] for the 8-bit scale quantiser, "
-                         "or gemv,rows,cols,nbits,g[,batch[,reps]] for the fused dequantise + matrix-vector product")
+                         "or gemv,rows,cols,nbits,g[,batch[,reps]] for the fused dequantise + matrix-vector product, "
+                         "or half,rows,cols,nbits,g[,reps] for the half-precision solver variant beside the fp32 one")
     ap.add_argument("--workload", default="llama2-70b",
                     choices=["llama2-70b", "llama2-7b-mlp-sweep", "llama2-70b-stream", "llama2-13b-stream"])
     ap.add_argument("--layers", type=int, default=None,

@@ -69,9 +69,14 @@ int check_args(int64_t rows, int64_t cols, int dtype, int nbits, int group_size,
 int quantize_entry(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p,
                    float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* W_q_packed, void* scale,
                    void* zero, void* zero_meta, void* workspace, size_t workspace_bytes, bool allow_slices,
-                   int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32, void* stream) {
+                   int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32, void* stream,
+                   bool half) {
     const int ck = check_args(rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode, zero_nbits);
     if (ck != HQQ_OK) return ck;
+    if (half) {
+        if (dtype != HQQ_F16) return HQQ_ERR_DTYPE;
+        if (axis != 1 || stop_mode == HQQ_STOP_TENSOR) return HQQ_ERR_INVALID_ARG;
+    }
     const int64_t G = rows * cols / group_size;
     const int64_t slice =
         hqq::fit_slice(rows, cols, group_size, axis, stop_mode, zero_nbits, workspace == nullptr ? 0 : workspace_bytes);
@@ -120,6 +125,7 @@ int quantize_entry(const void* W, int64_t rows, int64_t cols, int dtype, int nbi
     a.dbg_iter = debug_best_iter;
     a.dbg_err = debug_best_err;
     a.dbg_zero = debug_zero_f32;
+    a.half = half;
     const cudaError_t err = hqq::launch_solve(a, static_cast<cudaStream_t>(stream));
     if (err != cudaSuccess) {
         cudaGetLastError();
@@ -155,6 +161,15 @@ int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits
     return hqq::quantize_entry(W, rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
                                zero_nbits, W_q_packed, scale, zero, zero_meta, workspace, workspace_bytes, false,
                                debug_best_iter, debug_best_err, debug_zero_f32, stream);
+}
+
+int hqq_quantize_half(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis,
+                      float p, float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* W_q_packed,
+                      void* scale, void* zero, void* zero_meta, void* workspace, size_t workspace_bytes,
+                      int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32, void* stream) {
+    return hqq::quantize_entry(W, rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
+                               zero_nbits, W_q_packed, scale, zero, zero_meta, workspace, workspace_bytes, false,
+                               debug_best_iter, debug_best_err, debug_zero_f32, stream, true);
 }
 
 }  // extern "C"

@@ -58,6 +58,7 @@ struct SolveArgs {
     int32_t* dbg_iter;
     float* dbg_err;
     float* dbg_zero;
+    bool half = false;  // the half-precision solver variant (fp16 input, axis 1, group or no stop)
 };
 
 struct DequantArgs {
@@ -115,6 +116,7 @@ int check_args(int64_t rows, int64_t cols, int dtype, int nbits, int group_size,
 int quantize_entry(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis, float p,
                    float beta, float kappa, int iters, int stop_mode, int zero_nbits, void* W_q_packed, void* scale,
                    void* zero, void* zero_meta, void* workspace, size_t workspace_bytes, bool allow_slices,
-                   int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32, void* stream);
+                   int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32, void* stream,
+                   bool half = false);
 
 }  // namespace hqq

@@ -1387,6 +1387,209 @@ __global__ void __launch_bounds__(kRegThreads, onepass_ctas(E))
     if (k.zero_nbits == 8) merge_zero_range<kRegWarps>(k, zmin, zmax, sred);
 }
 
+// ============================================= half-precision variant ==
+//
+// solve_half_kernel (group / no stop, axis 1, fp16 input): the solver in half
+// precision, as the pages run it on the GPU ("Speed: from hours to minutes"),
+// with the steps of "Outlier-aware optimization without gradients".  Reading
+// H: every element-wise value is rounded to fp16 (to nearest, ties to even):
+// s = h(min(L/(max-min), 2e4)), z0 = h(-min*s), ws = h(w*s), v = h(ws + z)
+// (add.rn.f16x2), W_q = clamp(round(v), 0, L), r = h(v - W_q); the error of z
+// is the sum of h(|r|^p) (|r|^p through the hardware base-2 log and
+// exponential in fp32, then rounded to fp16); each z update rounds an exact
+// mean to fp16 once; the rare proximal step rounds d = h(fl32(r/s)),
+// W_e = h(shrink(d)) and h(h(w - W_e)*s).  A warp holds a tile of 32/P groups
+// in registers (ws as packed f16x2 pairs) and runs it until every group has
+// stopped; W is read once (again only on the rare proximal path).
+__device__ __forceinline__ uint32_t h2_add(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ float h_lo(uint32_t x) { return __half2float(__ushort_as_half(static_cast<unsigned short>(x))); }
+__device__ __forceinline__ float h_hi(uint32_t x) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(x >> 16)));
+}
+__device__ __forceinline__ float h_round(float x) { return __half2float(__float2half_rn(x)); }
+__device__ __forceinline__ uint32_t h2_splat(float x) {
+    const uint32_t b = __half_as_ushort(__float2half_rn(x));
+    return b | (b << 16);
+}
+constexpr uint32_t kHalfMagic2 = 0x66006600u;  // 1536 in both halves: adding it rounds |v| < 512 to an integer
+
+// Slow path of one evaluation for one lane (a clamp is needed or the proximal
+// step may be non-zero): W re-read one 16-byte piece at a time; err, sq and
+// (sp) the exact sum of h(h(w - W_e)*s) accumulate.
+template <int E>
+__device__ __forceinline__ void half_eval_slow(const KParams& k, int64_t j, int part, float s, float z, float beta,
+                                               bool sp, float* err, float* sq, double* swe) {
+    const __half zh = __float2half_rn(z);
+    const uint4* src = reinterpret_cast<const uint4*>(k.W + j * k.g + part * E);
+#pragma unroll 1
+    for (int t = 0; t < E / kPiece; ++t) {
+        float x[kPiece];
+        unpack8<0>(__ldg(src + t), x);
+#pragma unroll
+        for (int i = 0; i < kPiece; ++i) {
+            const float wsv = h_round(__fmul_rn(x[i], s));  // the fp16 product is exact in fp32: one rounding
+            const float v = __half2float(__hadd(__float2half_rn(wsv), zh));
+            const float q = fminf(fmaxf(rintf(v), 0.0f), k.Lf);
+            const float r = h_round(__fsub_rn(v, q));  // v - q is exact in fp32
+            *err = __fadd_rn(*err, h_round(pow_pos(fabsf(r), k.p)));
+            *sq = __fadd_rn(*sq, q);
+            if (sp) {
+                const float d = h_round(__fdiv_rn(r, s));
+                const float we = h_round(shrink_elem(d, 1.0f, k.p, beta));
+                const float a = __half2float(__double2half(static_cast<double>(x[i]) - static_cast<double>(we)));
+                *swe += static_cast<double>(h_round(__fmul_rn(a, s)));
+            }
+        }
+    }
+}
+
+// Packed codes of this lane's E elements at zero-point z: clamp(round(h(ws + z))).
+template <int E, int NBITS>
+__device__ __forceinline__ void store_codes_half(const KParams& k, int64_t j, int part, const uint32_t* ws2,
+                                                 float z) {
+    constexpr float Lf = static_cast<float>((1 << NBITS) - 1);
+    constexpr int kWords = (E * NBITS + 31) / 32;
+    uint32_t wd[kWords];
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) wd[w] = 0u;
+    const uint32_t z2 = h2_splat(z);
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+        const uint32_t v = h2_add(ws2[i / 2], z2);
+        const uint32_t c2[2] = {static_cast<uint32_t>(fminf(fmaxf(rintf(h_lo(v)), 0.0f), Lf)),
+                                static_cast<uint32_t>(fminf(fmaxf(rintf(h_hi(v)), 0.0f), Lf))};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int b = (i + h) * NBITS;
+            wd[b / 32] |= c2[h] << (b % 32);
+            if (b % 32 + NBITS > 32) wd[b / 32 + 1] |= c2[h] >> (32 - b % 32);
+        }
+    }
+    constexpr int kBytes = E * NBITS / 8;
+    uint8_t* dst = k.packed + (j * (k.g / E) + part) * kBytes;
+#pragma unroll
+    for (int q = 0; q < kBytes; ++q) dst[q] = static_cast<uint8_t>(wd[q / 4] >> (8 * (q % 4)));
+}
+
+template <int E>
+__device__ __forceinline__ void store_codes_half_n(const KParams& k, int64_t j, int part, const uint32_t* ws2,
+                                                   float z) {
+    switch (k.nbits) {
+        case 1: store_codes_half<E, 1>(k, j, part, ws2, z); break;
+        case 2: store_codes_half<E, 2>(k, j, part, ws2, z); break;
+        case 3: store_codes_half<E, 3>(k, j, part, ws2, z); break;
+        case 4: store_codes_half<E, 4>(k, j, part, ws2, z); break;
+        default: store_codes_half<E, 8>(k, j, part, ws2, z); break;
+    }
+}
+
+template <int E>
+__global__ void __launch_bounds__(kRegThreads, 3) solve_half_kernel(const KParams k) {
+    __shared__ float2 sred[kRegWarps];
+    const int warp = threadIdx.x >> 5;
+    const bool stop_group = k.stop_mode == 0;
+    const float thr = shrink_threshold(k.beta_last, k.p);  // smallest threshold of the run: a conservative gate
+    const int64_t ntiles = num_warp_tiles<1>(k);
+    float zmin = FLT_MAX, zmax = -FLT_MAX;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kRegWarps + warp; t < ntiles;
+         t += static_cast<int64_t>(gridDim.x) * kRegWarps) {
+        const WarpTile w = warp_tile<1>(k, t);
+        uint4 raw[E / kPiece];
+        const uint4* src = reinterpret_cast<const uint4*>(k.W + w.j * k.g + w.part * E);
+#pragma unroll
+        for (int q = 0; q < E / kPiece; ++q) raw[q] = w.valid ? __ldg(src + q) : make_uint4(0, 0, 0, 0);
+        // initialisation: s, z0, ws = h(w*s) as f16x2 pairs, the exact sum of ws, this lane's ws range
+        uint32_t mn2 = raw[0].x, mx2 = raw[0].x;
+#pragma unroll
+        for (int q = 0; q < E / kPiece; ++q) minmax8<0>(raw[q], mn2, mx2);
+        const float lmn = fminf(h_lo(mn2), h_hi(mn2)), lmx = fmaxf(h_lo(mx2), h_hi(mx2));
+        const float mn = seg_min(lmn, k.P), mx = seg_max(lmx, k.P);
+        float s = kScaleCap;
+        if (mx > mn) s = fminf(__fdiv_rn(k.Lf, __fsub_rn(mx, mn)), kScaleCap);
+        s = h_round(s);
+        const float z0 = h_round(__fmul_rn(-mn, s));
+        uint32_t ws2[E / 2];
+        double acc = 0.0;
+#pragma unroll
+        for (int q = 0; q < E / kPiece; ++q) {
+            float x[kPiece];
+            unpack8<0>(raw[q], x);
+#pragma unroll
+            for (int i = 0; i < kPiece; i += 2) {
+                const __half2 h2 = __floats2half2_rn(__fmul_rn(x[i], s), __fmul_rn(x[i + 1], s));
+                ws2[(q * kPiece + i) / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                acc += static_cast<double>(__low2float(h2)) + static_cast<double>(__high2float(h2));
+            }
+        }
+        const double sws = seg_sum_d(w.valid ? acc : 0.0, k.P);
+        const float wsmin = h_round(__fmul_rn(lmn, s)), wsmax = h_round(__fmul_rn(lmx, s));
+        float z = z0, zb = z0, be = INFINITY;
+        int bi = 0;
+        bool active = w.valid && k.iters_eff > 0;
+        for (int it = 0; __any_sync(kFull, active); ++it) {
+            const float beta = beta_at(k, it);
+            const bool sp = active && shrink_possible(s, z, z0, thr, k.Lf);
+            const __half zh = __float2half_rn(z);
+            const bool cf = __half2float(__hadd(__float2half_rn(wsmin), zh)) >= -0.5f &&
+                            __half2float(__hadd(__float2half_rn(wsmax), zh)) < k.Lf + 0.5f;
+            float err = 0.0f, sq = 0.0f;
+            double swe = 0.0;
+            if (__all_sync(kFull, !active || (!sp && cf))) {
+                if (active) {
+                    const uint32_t z2 = h2_splat(z);
+#pragma unroll
+                    for (int i = 0; i < E / 2; ++i) {
+                        const uint32_t v = h2_add(ws2[i], z2);
+                        const uint32_t qv = h2_sub(h2_add(v, kHalfMagic2), kHalfMagic2);
+                        const uint32_t r = h2_sub(v, qv) & 0x7fff7fffu;  // |r|, exact
+                        err = __fadd_rn(err, h_round(pow_pos(h_lo(r), k.p)));
+                        err = __fadd_rn(err, h_round(pow_pos(h_hi(r), k.p)));
+                        sq = __fadd_rn(sq, __fadd_rn(h_lo(qv), h_hi(qv)));
+                    }
+                }
+            } else if (active) {
+                half_eval_slow<E>(k, w.j, w.part, s, z, beta, sp, &err, &sq, &swe);
+            }
+            err = seg_sum(err, k.P);
+            sq = seg_sum(sq, k.P);
+            if (__any_sync(kFull, sp)) swe = seg_sum_d(swe, k.P);
+            if (active) {
+                const bool improved = err < be;
+                if (improved) {
+                    be = err;
+                    zb = z;
+                    bi = it;
+                }
+                bool stop = (stop_group && !improved) || it >= k.iters_eff - 1;
+                if (!stop) {
+                    const double m = (static_cast<double>(sq) - (sp ? swe : sws)) / static_cast<double>(k.g);
+                    const float zn = __half2float(__double2half(m));
+                    if (stop_group && zn == z) stop = true;  // fixed point: the next error equals this one
+                    else z = zn;
+                }
+                if (stop) active = false;
+            }
+        }
+        if (w.valid) {
+            store_codes_half_n<E>(k, w.j, w.part, ws2, zb);
+            if (w.part == 0) {
+                const float err_mean = k.dbg_err ? be * pow_pos(s, -k.p) / static_cast<float>(k.g) : 0.0f;
+                store_group(k, w.j, s, zb, bi, err_mean, &zmin, &zmax);
+            }
+        }
+    }
+    if (k.zero_nbits == 8) merge_zero_range<kRegWarps>(k, zmin, zmax, sred);
+}
+
 // ------------------------------------------------------- 8-bit zero ------
 
 // One RTN quantiser for all kept zeros of the tensor, from their min/max
@@ -1743,6 +1946,18 @@ cudaError_t launch_solver(KParams& k, const WorkspaceLayout& L, uint8_t* ws, cud
     return launch_group<DT, AXIS, E>(k, L, ws, stream);
 }
 
+template <int E>
+cudaError_t launch_half(KParams& k, cudaStream_t stream) {
+    auto kern = solve_half_kernel<E>;
+    int grid = 0;
+    const int gpw = 32 >> k.logP;
+    const int64_t tiles = (k.G + gpw - 1) / gpw;
+    cudaError_t err = persistent_grid(kern, kRegThreads, 0, (tiles + kRegWarps - 1) / kRegWarps, &grid);
+    if (err != cudaSuccess) return err;
+    kern<<<grid, kRegThreads, 0, stream>>>(k);
+    return cudaGetLastError();
+}
+
 template <int DT, int AXIS>
 cudaError_t launch_solver_e(KParams& k, const WorkspaceLayout& L, uint8_t* ws, cudaStream_t stream) {
     if (k.E == 8) return launch_solver<DT, AXIS, 8>(k, L, ws, stream);
@@ -1876,7 +2091,12 @@ cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream) {
 
     cudaError_t err = cudaMemsetAsync(a.ws + L.header, 0, 256, stream);
     if (err != cudaSuccess) return err;
-    if (a.G > 0) {
+    if (a.G > 0 && a.half) {  // the half-precision variant: fp16 input, axis 1, group or no stop
+        if (k.E == 8) err = launch_half<8>(k, stream);
+        else if (k.E == 16) err = launch_half<16>(k, stream);
+        else err = launch_half<32>(k, stream);
+        if (err != cudaSuccess) return err;
+    } else if (a.G > 0) {
         if (a.dtype == 0 && a.axis == 1) err = launch_solver_e<0, 1>(k, L, a.ws, stream);
         else if (a.dtype == 0) err = launch_solver_e<0, 0>(k, L, a.ws, stream);
         else if (a.axis == 1) err = launch_solver_e<1, 1>(k, L, a.ws, stream);

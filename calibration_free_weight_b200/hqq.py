@@ -21,7 +21,7 @@ EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_qu
             "hqq_get_status", "hqq_status_string", "hqq_quantize_noalloc", "hqq_quantize_scale8",
             "hqq_dequantize_s8", "hqq_stream_device_bytes", "hqq_quantize_stream", "hqq_gemv",
             "hqq_stream_jobs_device_bytes", "hqq_quantize_stream_jobs", "hqq_gemm", "hqq_gemm_get_status",
-            "hqq_gemm_wait_selftest", "hqq_gemm_workspace_bytes")
+            "hqq_gemm_wait_selftest", "hqq_gemm_workspace_bytes", "hqq_quantize_half")
 
 
 class hqq_host_matrix(C.Structure):
@@ -55,6 +55,8 @@ def _load():
     L.hqq_quantize.restype = i32
     L.hqq_quantize.argtypes = [P, i64, i64, i32, i32, i32, i32, f32, f32, f32, i32, i32, i32,
                                P, P, P, P, P, sz, P, P, P, P]
+    L.hqq_quantize_half.restype = i32
+    L.hqq_quantize_half.argtypes = L.hqq_quantize.argtypes
     L.hqq_dequantize.restype = i32
     L.hqq_dequantize.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, i32, i32, P, P]
     L.hqq_get_status.restype = i32
@@ -135,6 +137,16 @@ def hqq_quantize(W, rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, 
                             zero_nbits, _ptr(W_q_packed), _ptr(scale), _ptr(zero), _ptr(zero_meta), _ptr(workspace),
                             workspace_bytes, _ptr(debug_best_iter), _ptr(debug_best_err), _ptr(debug_zero_f32),
                             _stream(stream))
+
+
+def hqq_quantize_half(W, rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode, zero_nbits,
+                      W_q_packed, scale, zero, zero_meta, workspace, workspace_bytes, debug_best_iter=None,
+                      debug_best_err=None, debug_zero_f32=None, stream=None):
+    """Raw call of the half-precision solver variant; returns the status code."""
+    return lib.hqq_quantize_half(_ptr(W), rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters,
+                                 stop_mode, zero_nbits, _ptr(W_q_packed), _ptr(scale), _ptr(zero), _ptr(zero_meta),
+                                 _ptr(workspace), workspace_bytes, _ptr(debug_best_iter), _ptr(debug_best_err),
+                                 _ptr(debug_zero_f32), _stream(stream))
 
 
 def hqq_quantize_noalloc(W, rows, cols, dtype, nbits, group_size, axis, p, beta, kappa, iters, stop_mode,
@@ -262,6 +274,24 @@ def quantize(W, nbits=4, group_size=64, axis=1, p=0.7, beta=1.0, kappa=1.01, ite
                       stream)
     if rc != HQQ_OK:
         raise HQQError(rc, "hqq_quantize")
+    return out
+
+
+def quantize_half(W, nbits=4, group_size=64, p=0.7, beta=1.0, kappa=1.01, iters=20, stop_mode=HQQ_STOP_GROUP,
+                  zero_nbits=16, debug=False, out=None, stream=None):
+    """The half-precision solver variant on a CUDA fp16 [rows, cols] tensor
+    (axis 1, group or no stop); returns the output dict."""
+    if W.dtype != torch.float16 or not W.is_cuda or W.dim() != 2 or not W.is_contiguous():
+        raise HQQError(HQQ_ERR_INVALID_ARG, "quantize_half expects a contiguous 2-D CUDA fp16 tensor")
+    rows, cols = W.shape
+    if out is None:
+        out = alloc_outputs(rows, cols, nbits, group_size, 1, stop_mode, zero_nbits, debug, W.device)
+    rc = hqq_quantize_half(W, rows, cols, HQQ_F16, nbits, group_size, 1, p, beta, kappa, iters, stop_mode,
+                           zero_nbits, out["packed"], out["scale"], out["zero"], out["zero_meta"], out["workspace"],
+                           out["workspace"].numel(), out.get("best_iter"), out.get("best_err"), out.get("zero_f32"),
+                           stream)
+    if rc != HQQ_OK:
+        raise HQQError(rc, "hqq_quantize_half")
     return out
 
 

@@ -145,6 +145,33 @@ int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits
                  void* stream);
 
 /*
+ * hqq_quantize_half -- the solver in half precision, the variant the pages run
+ * on the GPU (techreport.ngo, "Weight-only quantization without the
+ * calibration tax", section "Speed: from hours to minutes"; the steps of
+ * section "Outlier-aware optimization without gradients").  This library's
+ * reading of half precision: every element-wise value is rounded to fp16 (to
+ * nearest, ties to even) -- s = h(min(L/(max w - min w), 2e4)), z0 = h(-min w
+ * * s), w*s, v = h(h(w*s) + z), W_q = clamp(round(v), 0, L), r = h(v - W_q),
+ * the error terms h(|r|^p) (their sum exact); each z update rounds an exact
+ * mean to fp16 once; the proximal step rounds d = h(fl32(r/s)), W_e =
+ * h(shrink(d)) and h(h(w - W_e)*s).  The stop rules group and none, beta and
+ * the 8-bit zero are as in hqq_quantize; scale = h(fl32(1/s)), zero = the fp16
+ * z*.  |r|^p is evaluated with the hardware base-2 log and exponential in fp32
+ * and then rounded to fp16, so a term can sit one fp16 step from the exactly
+ * rounded value and a stop decision whose two sums differ by less than about
+ * 2^-9 relative may go the other way.
+ * Arguments as hqq_quantize, with: dtype must be HQQ_F16 (else HQQ_ERR_DTYPE);
+ * axis must be 1 and stop_mode HQQ_STOP_GROUP or HQQ_STOP_NONE (else
+ * HQQ_ERR_INVALID_ARG); workspace as for hqq_quantize with the same arguments.
+ */
+int hqq_quantize_half(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis,
+                      float p, float beta, float kappa, int iters, int stop_mode, int zero_nbits,
+                      void* W_q_packed, void* scale, void* zero, void* zero_meta,
+                      void* workspace, size_t workspace_bytes,
+                      int32_t* debug_best_iter, float* debug_best_err, float* debug_zero_f32,
+                      void* stream);
+
+/*
  * Dequantise for inspection ("HQQ - Half-Quadratic Quantization"
  * (skill4agent.com), section "Core concepts": HQQLinear's dequantize(); the
  * rule W_r = (W_q - z) / s of techreport.ngo, "Weight-only quantization

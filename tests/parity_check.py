@@ -338,3 +338,60 @@ def check_stored(W_cpu, params, out, orc=None, sample=None):
     rep["tie_groups"] = int(len(nbad))
     rep["code_mismatch"] = nd
     return rep
+
+
+# ------------------------------------------- half-precision variant -------
+
+# The variant's error terms are |r|^p rounded to fp16; the GPU forms |r|^p
+# with the hardware base-2 log and exponential in fp32 before that rounding,
+# so a term can land one fp16 step (at most 2^-10 relative) from the oracle's
+# exactly rounded one, and a sum of such terms can move by up to 2^-10
+# relative.  A decision can therefore flip when the oracle's two sums differ
+# by less than twice that.
+TIE_TOL_HALF = 2.0 ** -9
+
+
+def _path_ok_tol(e, k_gpu, k_orc, iters, mode, tol):
+    if mode == oracle.STOP_NONE:
+        return e[k_gpu] <= e[k_orc] * (1 + tol) + 1e-30
+    for i in range(1, k_gpu + 1):
+        if not e[i] < e[i - 1] and (e[i] - e[i - 1]) > tol * e[i - 1]:
+            return False
+    if k_gpu + 1 < iters:
+        nxt = k_gpu + 1
+        if e[nxt] < e[k_gpu] and (e[k_gpu] - e[nxt]) > tol * e[k_gpu]:
+            return False
+    return True
+
+
+def check_half(W_cpu, params, gpu, orc):
+    """The half-precision variant (GPU outputs with debug, numpy) against its
+    oracle.  The arithmetic is the same on both sides except the error terms,
+    so every group whose kept iterate matches has bit-identical scale, kept
+    zero and codes; a group whose kept iterate differs must be explained by
+    decisions within TIE_TOL_HALF on the oracle's own trajectory and must then
+    match the oracle's iterate at the GPU's index exactly.  Returns a report."""
+    nb, g = params["nbits"], params["group_size"]
+    p, beta, kappa, iters, mode = params["p"], params["beta"], params["kappa"], params["iters"], params["stop_mode"]
+    rows, cols = W_cpu.shape
+    G = rows * cols // g
+    Wf = W_cpu.float().numpy()
+    assert np.array_equal(gpu["scale"].view(np.uint16), orc["scale"].view(np.uint16)), "scale"
+    gl = all_groups(oracle.unpack_levels(gpu["packed"], rows, cols, nb, 1), g, 1)
+    ol = all_groups(oracle.unpack_levels(orc["packed"], rows, cols, nb, 1), g, 1)
+    differ = np.nonzero(gpu["best_iter"] != orc["best_iter"])[0]
+    same = np.ones(G, bool)
+    same[differ] = False
+    assert np.array_equal(gpu["zero_f32"][same], orc["zero_f32"][same]), "kept zero"
+    assert np.array_equal(gl[same], ol[same]), "codes"
+    for j in differ:
+        w = group_values(Wf, j, g, 1)
+        s, zt, et, _ = oracle.trace_group_half(w, nb, p, beta, kappa, max(iters, 1))
+        kg = int(gpu["best_iter"][j])
+        assert _path_ok_tol(et, kg, int(orc["best_iter"][j]), iters, mode, TIE_TOL_HALF), (
+            f"group {j}: kept iterate {kg} vs oracle {orc['best_iter'][j]} is not a near tie: {et[:kg + 3]}")
+        assert gpu["zero_f32"][j] == zt[kg], (j, gpu["zero_f32"][j], zt[kg])
+        assert np.array_equal(gl[j], oracle.group_codes_half(w, nb, s, zt[kg])), j
+    if params["zero_nbits"] == 16:
+        assert np.array_equal(gpu["zero"].astype(np.float32), gpu["zero_f32"])
+    return {"groups": G, "tie_groups": int(len(differ)), "tie_frac": float(len(differ)) / max(G, 1)}

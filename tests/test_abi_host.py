@@ -308,3 +308,15 @@ def test_noalloc_zero8_limit_is_exact(hq, axis):
     assert over[0] * over[1] // 16 == fit[0] * fit[1] // 16 + 1
     assert call(*fit) not in (hq.HQQ_ERR_WORKSPACE, hq.HQQ_OK)
     assert call(*over) == hq.HQQ_ERR_WORKSPACE
+
+
+def test_half_variant_rejects_on_host(hq):
+    """hqq_quantize_half takes fp16 input, axis 1, group or no stop; the other
+    cases are refused before anything is touched."""
+    def call(dtype=0, axis=1, stop=0):
+        return hq.lib.hqq_quantize_half(None, 64, 64, dtype, 4, 64, axis, 0.7, 1.0, 1.01, 20, stop, 16, None, None,
+                                        None, None, None, 0, None, None, None, None)
+    assert call(dtype=1) == 3
+    assert call(axis=0) == 1
+    assert call(stop=1) == 1
+    assert call() == 8  # every argument valid: only the missing workspace is left
