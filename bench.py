@@ -70,7 +70,9 @@ GEMM_TRAFFIC = {"src_sha256": "6047c8fb4337f86155429e2a54e5e1946effb14b71f0514dd
 # to the algorithmic bytes of the captured calls (ncu, one call per setting on
 # the gate shape 28672x8192; see profiles/), valid while the kernel sources
 # hash to the captured ones.
-TRAFFIC70 = {"src_sha256": None, "bytes_per_alg_byte": None, "summary": None}
+TRAFFIC70 = {"src_sha256": "c605bf6a126d5cd41ac5be48777e4723afdb29b4b59adade8d184376fdfc2f8f",
+             "bytes_per_alg_byte": {(2, 16): 623.33 / 572.52, (4, 128): 579.18 / 592.68},
+             "summary": "profiles/solve_group_onepass_kernel_28672x8192_b2g16.md, ..._b4g128.md"}
 
 
 def kernel_sources_sha(files=None):
@@ -674,8 +676,11 @@ def run_llama70(args):
     alg_step = sum(algorithmic_bytes(r, c, nb, g, 8) for _, _, r, c, nb, g in calls)
     gbs = alg_step * args.steps / (call_ms / 1e3) / 1e9 if call_ms > 0 else 0.0
     traffic = None
-    if TRAFFIC70["src_sha256"] == kernel_sources_sha() and TRAFFIC70["bytes_per_alg_byte"]:
-        traffic = TRAFFIC70["bytes_per_alg_byte"] * alg_step / len(calls)
+    if TRAFFIC70["src_sha256"] == kernel_sources_sha():
+        # DRAM bytes per algorithmic byte of the captured gate-shape calls, per setting,
+        # applied to the benched calls' algorithmic bytes
+        traffic = sum(TRAFFIC70["bytes_per_alg_byte"][(nb, g)] * algorithmic_bytes(r, c, nb, g, 8)
+                      for _, _, r, c, nb, g in calls) / len(calls)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dev_ms / args.steps, "higher_is_better": True,
@@ -684,7 +689,9 @@ def run_llama70(args):
             "config": config70(world, total_layers),
             "roofline": {"bound": "alu", "kernel": "solve_group_onepass_kernel", "achieved": achieved, "peak": mufu_peak,
                          "unit": "Gop/s (MUFU lg2+ex2)", "frac": achieved / mufu_peak, "traffic": traffic,
-                         "traffic_unit": "DRAM bytes per call", "peak_kind": "nominal",
+                         "traffic_unit": "DRAM bytes per call", "traffic_basis": TRAFFIC70["summary"] +
+                         " (ratio to algorithmic bytes per setting, scaled to the benched calls)",
+                         "peak_kind": "nominal",
                          "peak_basis": f"{SMS} SMs x {MUFU_PER_CLK_PER_SM} MUFU ops/clk x {sm_max:.0f} MHz "
                                        f"(16/clk/SM confirmed by a microbenchmark of independent lg2/ex2 chains; "
                                        f"not driver-measured)",
@@ -767,14 +774,14 @@ def e2e70(args, hqq, world, rank, Wd, layers, mats, stream):
         return host_o[key]
 
     jobs_W, jobs_set, jobs_out = [], [], []
-    for nb, g in SETTINGS70B:
-        for i, l in enumerate(layers):
-            for n, r, c in mats:
+    for i, l in enumerate(layers):
+        for n, r, c in mats:
+            for nb, g in SETTINGS70B:  # consecutive jobs on one matrix share its device copy
                 jobs_W.append(Wh[(i % ring, n)])
                 jobs_set.append(dict(nbits=nb, group_size=g, axis=1, stop_mode=0, zero_nbits=8))
                 key = (l, n, nb, g) if outs_per_job else (n, nb, g)
                 jobs_out.append(host_out(key, r, c, nb, g))
-    k = len(mats)
+    k = len(mats) * nset
     buf, _ = hqq.quantize_stream_jobs(jobs_W[:k], jobs_set[:k], jobs_out[:k])  # warm-up: one layer
     steps = max(1, min(args.steps, args.e2e_steps))
     barrier(world)
@@ -787,12 +794,13 @@ def e2e70(args, hqq, world, rank, Wd, layers, mats, stream):
     e1.record(stream)
     barrier(world)
     ms = max_over_ranks(e0.elapsed_time(e1), world)
-    h2d = 2 * w_layer * len(layers) * nset
+    h2d = 2 * w_layer * len(layers)  # each matrix crosses once for both settings
     d2h = sum(out_layer.values()) * len(layers)
     del buf
     return {"value": args.layers * w_layer * nset * steps / (ms / 1e3) / 1e9, "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "s_per_step": ms / 1e3 / steps, "api": "hqq_quantize_stream_jobs (C ABI), host buffers pinned",
+            "s_per_step": ms / 1e3 / steps, "api": "hqq_quantize_stream_jobs (C ABI), host buffers pinned, "
+                                                   "the two settings of a matrix as consecutive jobs on one copy",
             "host_weights": ("one buffer per matrix and layer" if ring == len(layers) else
                              f"a ring of {ring} layers' buffers reused in layer order (host memory)"),
             "host_outputs": "one set per job" if outs_per_job else "one set per matrix and setting, reused"}
@@ -995,7 +1003,7 @@ def run_half_case(spec):
 
 
 def run_case(spec):
-    """Time hqq_quantize on one synthetic bf16 matrix (used for kernel profiles)."""
+    """Time hqq_quantize on one synthetic matrix (used for kernel profiles)."""
     if spec.startswith("scale8"):
         run_scale8_case(spec)
         return
@@ -1009,17 +1017,19 @@ def run_case(spec):
         run_half_case(spec)
         return
     from calibration_free_weight_b200 import hqq
-    v = [int(x) for x in spec.split(",")]
-    mode, rows, cols, nbits, g = v[:5]
-    reps = v[5] if len(v) > 5 else 3
+    f = spec.split(",")
+    mode, rows, cols, nbits, g = (int(x) for x in f[:5])
+    reps = int(f[5]) if len(f) > 5 else 3
+    dtype = torch.float16 if len(f) > 6 and f[6] == "f16" else torch.bfloat16
+    zb = int(f[7]) if len(f) > 7 else 16
     torch.cuda.set_device(0)
-    W = synth.weight(rows, cols, seed=4, dtype=torch.bfloat16).cuda()
-    out = hqq.alloc_outputs(rows, cols, nbits, g, 1, mode, 16)
+    W = synth.weight(rows, cols, seed=4, dtype=dtype).cuda()
+    out = hqq.alloc_outputs(rows, cols, nbits, g, 1, mode, zb)
     ev = []
     for _ in range(reps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        hqq.quantize(W, nbits, g, stop_mode=mode, out=out)
+        hqq.quantize(W, nbits, g, stop_mode=mode, zero_nbits=zb, out=out)
         b.record()
         ev.append((a, b))
     torch.cuda.synchronize()
@@ -1040,7 +1050,8 @@ def main():
     ap.add_argument("--ref-step", type=float, default=1.0, help="seconds of oracle work per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
-                    help="single-matrix timing instead of the sweep: stop_mode,rows,cols,nbits,group_size[,reps]; "
+                    help="single-matrix timing: stop_mode,rows,cols,nbits,group_size[,reps[,f16|bf16[,zero_nbits]]] "
+                         "(seed-4 synthetic weights, bf16 and fp16 zero by default); "
                          "or scale8,G[,S[,reps]] for the 8-bit scale quantiser, "
                          "or gemv,rows,cols,nbits,g[,batch[,reps]] for the fused dequantise + matrix-vector product, "
                          "or half,rows,cols,nbits,g[,reps] for the half-precision solver variant beside the fp32 one")
