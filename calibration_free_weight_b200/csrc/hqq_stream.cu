@@ -15,6 +15,11 @@
 // copied in only after the solver on matrix i has finished reading it, and its
 // outputs are written only after those of matrix i have been copied out.
 //
+// A job whose matrix is the previous job's (the same host buffer and shape,
+// e.g. one weight quantised at two settings) reuses the device copy of it:
+// the weights cross PCIe once.  The W buffers alternate between the two slots
+// on copies only, and a copy into one waits for every solver that read it.
+//
 // Each job is reported (callback, in order) once its outputs are in host
 // memory; the report of job i-2 is taken just before its slot's copy-out event
 // is reused for job i, by which time the solver on job i has already waited
@@ -23,7 +28,7 @@
 // The call blocks until every output has reached host memory.  Host buffers
 // should be pinned (cudaHostAlloc / cudaHostRegister) for the copies to
 // overlap; pageable buffers work but serialise.  Device memory is the
-// caller's buffer; the executor creates two streams and six events per call
+// caller's buffer; the executor creates two streams and eight events per call
 // and destroys them before returning.
 
 #include <cuda_runtime.h>
@@ -108,13 +113,16 @@ Slot carve(uint8_t* base, const SlotSizes& s) {
 // Streams and events of one call, released on every exit path.
 struct Resources {
     cudaStream_t cin = nullptr, cout = nullptr;
-    cudaEvent_t in_done[2] = {}, solved[2] = {}, out_done[2] = {};
+    // in_done / w_read: per W buffer (copied in; last read by a solver),
+    // solved / out_done: per output slot (solved; copied out)
+    cudaEvent_t in_done[2] = {}, w_read[2] = {}, solved[2] = {}, out_done[2] = {};
     bool ok = true;
     Resources() {
         ok = cudaStreamCreateWithFlags(&cin, cudaStreamNonBlocking) == cudaSuccess &&
              cudaStreamCreateWithFlags(&cout, cudaStreamNonBlocking) == cudaSuccess;
         for (int k = 0; k < 2 && ok; ++k)
             ok = cudaEventCreateWithFlags(&in_done[k], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&w_read[k], cudaEventDisableTiming) == cudaSuccess &&
                  cudaEventCreateWithFlags(&solved[k], cudaEventDisableTiming) == cudaSuccess &&
                  cudaEventCreateWithFlags(&out_done[k], cudaEventDisableTiming) == cudaSuccess;
     }
@@ -123,6 +131,7 @@ struct Resources {
         if (cout) cudaStreamSynchronize(cout);
         for (int k = 0; k < 2; ++k) {
             if (in_done[k]) cudaEventDestroy(in_done[k]);
+            if (w_read[k]) cudaEventDestroy(w_read[k]);
             if (solved[k]) cudaEventDestroy(solved[k]);
             if (out_done[k]) cudaEventDestroy(out_done[k]);
         }
@@ -196,26 +205,34 @@ int hqq_quantize_stream_jobs(const hqq_stream_job* jobs, int n, int dtype, float
         reported = k + 1;
         return true;
     };
+    int copies = 0, wb = 0;  // W buffers filled so far; the one holding the current job's matrix
     for (int i = 0; i < n && rc == HQQ_OK; ++i) {
         const hqq_stream_job& j = jobs[i];
         const hqq_host_matrix& m = j.m;
         const Slot& t = slot[i & 1];
         const JobSizes z = job_sizes(j);
-        // copy-in: the solver on job i-2 (same slot) must have finished reading W
-        if (i >= 2 && !cuda_ok(cudaStreamWaitEvent(r.cin, r.solved[i & 1], 0))) break;
-        if (z.W && !cuda_ok(cudaMemcpyAsync(t.W, m.W, z.W, cudaMemcpyHostToDevice, r.cin))) break;
-        if (!cuda_ok(cudaEventRecord(r.in_done[i & 1], r.cin))) break;
+        const bool reuse = i >= 1 && z.W && m.W == jobs[i - 1].m.W && m.rows == jobs[i - 1].m.rows &&
+                           m.cols == jobs[i - 1].m.cols;
+        if (!reuse) {
+            // copy-in: every solver that read this W buffer must be done with it
+            wb = copies & 1;
+            ++copies;
+            if (copies > 2 && !cuda_ok(cudaStreamWaitEvent(r.cin, r.w_read[wb], 0))) break;
+            if (z.W && !cuda_ok(cudaMemcpyAsync(slot[wb].W, m.W, z.W, cudaMemcpyHostToDevice, r.cin))) break;
+            if (!cuda_ok(cudaEventRecord(r.in_done[wb], r.cin))) break;
+        }
         // solve: W has arrived, and job i-2's outputs in this slot have been copied out
-        if (!cuda_ok(cudaStreamWaitEvent(cs, r.in_done[i & 1], 0))) break;
+        if (!cuda_ok(cudaStreamWaitEvent(cs, r.in_done[wb], 0))) break;
         if (i >= 2 && !cuda_ok(cudaStreamWaitEvent(cs, r.out_done[i & 1], 0))) break;
-        const int q = hqq::quantize_entry(t.W, m.rows, m.cols, dtype, j.nbits, j.group_size, j.axis, p, beta, kappa,
-                                          iters, j.stop_mode, j.zero_nbits, t.packed, t.scale, t.zero,
+        const int q = hqq::quantize_entry(slot[wb].W, m.rows, m.cols, dtype, j.nbits, j.group_size, j.axis, p, beta,
+                                          kappa, iters, j.stop_mode, j.zero_nbits, t.packed, t.scale, t.zero,
                                           j.zero_nbits == 8 ? t.meta : nullptr, t.ws, z.workspace, false, nullptr,
                                           nullptr, nullptr, cs);
         if (q != HQQ_OK) {
             rc = q;
             break;
         }
+        if (!cuda_ok(cudaEventRecord(r.w_read[wb], cs))) break;
         if (!cuda_ok(cudaEventRecord(r.solved[i & 1], cs))) break;
         // job i-2's copy-out event is about to be reused: report it first
         if (i >= 2 && !report(i - 2)) break;

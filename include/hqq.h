@@ -298,8 +298,11 @@ size_t hqq_stream_jobs_device_bytes(const hqq_stream_job* jobs, int n);
  * NULL) receives the number of leading jobs whose outputs are complete in
  * host memory when the call returns: n on success.  A caller that persists
  * each job in on_done resumes an interrupted run by passing the jobs not yet
- * persisted.  device_buffer: device memory of at least
- * hqq_stream_jobs_device_bytes(jobs, n), 256-byte aligned, caller-owned.
+ * persisted.  A job whose matrix is the previous job's (the same host W
+ * pointer and shape, e.g. one weight quantised at two settings) reuses the
+ * device copy: the matrix crosses PCIe once.  device_buffer: device memory
+ * of at least hqq_stream_jobs_device_bytes(jobs, n), 256-byte aligned,
+ * caller-owned.
  * Blocks until every output is in host memory.  Returns HQQ_OK or the first
  * error (HQQ_ERR_WORKSPACE if device_bytes is too small).
  */

@@ -216,3 +216,24 @@ def test_stream_llama2_70b_shapes_against_oracle(hq, nbits, g):
         G = w.numel() // g
         ids = np.unique(np.concatenate([[0, G - 1], np.random.default_rng(i).choice(G, 3000, replace=False)]))
         pc.check_stored(w, _prm(st), _np(o), sample=ids)
+
+
+def test_stream_jobs_reuse_a_repeated_matrix(hq):
+    """Consecutive jobs on the same host matrix (one weight at several
+    settings) share one device copy of it; every output still equals the
+    per-matrix call with that job's settings, whatever the interleaving."""
+    A = synth.weight(2048, 1024, seed=71, dtype=torch.float16).pin_memory()
+    B = synth.weight(1024, 2048, seed=72, dtype=torch.float16).pin_memory()
+    C = synth.weight(512, 512, seed=73, dtype=torch.float16).pin_memory()
+    s1 = dict(nbits=2, group_size=16, axis=1, stop_mode=0, zero_nbits=8)
+    s2 = dict(nbits=4, group_size=128, axis=1, stop_mode=0, zero_nbits=8)
+    s3 = dict(nbits=3, group_size=64, axis=1, stop_mode=1, zero_nbits=16)
+    s4 = dict(nbits=4, group_size=64, axis=0, stop_mode=2, zero_nbits=16)
+    order = [(A, s1), (A, s2), (B, s1), (B, s2), (B, s3), (C, s4), (A, s3), (A, s4), (C, s1)]
+    Ws = [w for w, _ in order]
+    sets = [st for _, st in order]
+    outs = [hq.host_outputs(*w.shape, st["nbits"], st["group_size"], st["axis"], st["zero_nbits"]) for w, st in order]
+    _, done = hq.quantize_stream_jobs(Ws, sets, outs)
+    assert done == len(order)
+    for w, st, o in zip(Ws, sets, outs):
+        _same(o, _expect(hq, w, st))
