@@ -996,8 +996,8 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 3) solve_group_kern
 //     evaluations) -- or, without early stopping, to the end;
 //   survivor round: when the warp's pool of running groups in shared memory
 //     holds S of them (or nothing else is left), S of them are restored to the
-//     slots and evaluated until fewer than S/2 still run (or, at the end, all
-//     have stopped).
+//     slots and evaluated until fewer than S/2 (3S/4 for 32 elements per lane)
+//     still run (or, at the end, all have stopped).
 // After a round the stopped groups are packed and stored, and the running
 // ones go to the pool (raw values, scale, state: the codes of a group are
 // never recomputed from a second read of W).  Slots run at different
@@ -1330,7 +1330,9 @@ __global__ void __launch_bounds__(kRegThreads, onepass_ctas(E))
             const int n_alive = __popc(__ballot_sync(kFull, part == 0 && alive));
             if (n_alive == 0) break;
             if (!survivor && e >= m_fresh) break;
-            if (survivor && more && 2 * n_alive < S) break;
+            // a survivor round ends when too few of its slots still run (tiles of 32 elements per
+            // lane return them to the pool sooner: measured 2.5% faster at g128, 2% slower at g16)
+            if (survivor && more && (E >= 32 ? 4 * n_alive < 3 * S : 2 * n_alive < S)) break;
             WarpTile wt;
             wt.valid = alive;
             wt.j = j;
