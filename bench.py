@@ -1002,6 +1002,55 @@ def run_half_case(spec):
     print(json.dumps({"case": spec, **res, "half_over_fp32": res["fp32"]["ms"] / res["half"]["ms"]}))
 
 
+def run_tensor_case(spec):
+    """Tensor stop on one synthetic matrix, the resident launch (wherever it
+    fits) beside the chunked launches:
+    "tensor,rows,cols,nbits,g[,reps[,f16|bf16[,zero_nbits]]]" (seed-4 weights,
+    20 iterations); "default_path" is the library's own choice.  Reports each path's best call time and
+    its MUFU rate counted on the algorithmic evaluations (k* + 2 per group, at
+    most 20; k* from a debug call) against the nominal MUFU peak."""
+    from calibration_free_weight_b200 import hqq
+    f = spec.split(",")[1:]
+    rows, cols, nbits, g = (int(x) for x in f[:4])
+    reps = int(f[4]) if len(f) > 4 else 5
+    dtype = torch.float16 if len(f) > 5 and f[5] == "f16" else torch.bfloat16
+    zb = int(f[6]) if len(f) > 6 else 16
+    torch.cuda.set_device(0)
+    W = synth.weight(rows, cols, seed=4, dtype=dtype).cuda()
+    dbg = hqq.quantize(W, nbits, g, stop_mode=1, zero_nbits=zb, debug=True)
+    kb = int(dbg["best_iter"][0].item())
+    evals = min(kb + 2, 20)
+    _, sm_max, _ = peaks()
+    mufu_peak = SMS * MUFU_PER_CLK_PER_SM * sm_max * 1e6 / 1e9
+    res = {}
+    default = hqq.hqq_tensor_resident(rows, cols, 0 if dtype == torch.float16 else 1, g, 1, 20) == 1
+    for name, on in (("resident", 2), ("chunked", 0)):
+        prev = hqq.hqq_set_tensor_resident(on)
+        try:
+            used = hqq.hqq_tensor_resident(rows, cols, 0 if dtype == torch.float16 else 1, g, 1, 20) == 1
+            out = hqq.quantize(W, nbits, g, stop_mode=1, zero_nbits=zb)
+            ev = []
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                hqq.quantize(W, nbits, g, stop_mode=1, zero_nbits=zb, out=out)
+                b.record()
+                ev.append((a, b))
+            torch.cuda.synchronize()
+            st = hqq.hqq_get_status(out["workspace"])
+            if st != hqq.HQQ_OK:
+                raise RuntimeError(hqq.hqq_status_string(st))
+        finally:
+            hqq.hqq_set_tensor_resident(prev)
+        ms = min(a.elapsed_time(b) for a, b in ev)
+        gops = 2.0 * rows * cols * evals / (ms / 1e3) / 1e9
+        res[name] = {"path": "resident" if used else "chunked", "ms": ms,
+                     "gweights_s": rows * cols / (ms / 1e3) / 1e9, "mufu_gops": gops, "mufu_frac": gops / mufu_peak}
+    print(json.dumps({"case": spec, "kept_iterate": kb, "evals_per_weight": evals, "mufu_peak_gops": mufu_peak,
+                      "default_path": "resident" if default else "chunked",
+                      **res, "chunked_over_resident": res["chunked"]["ms"] / res["resident"]["ms"]}))
+
+
 def run_case(spec):
     """Time hqq_quantize on one synthetic matrix (used for kernel profiles)."""
     if spec.startswith("scale8"):
@@ -1015,6 +1064,9 @@ def run_case(spec):
         return
     if spec.startswith("half"):
         run_half_case(spec)
+        return
+    if spec.startswith("tensor"):
+        run_tensor_case(spec)
         return
     from calibration_free_weight_b200 import hqq
     f = spec.split(",")
@@ -1054,7 +1106,9 @@ def main():
                          "(seed-4 synthetic weights, bf16 and fp16 zero by default); "
                          "or scale8,G[,S[,reps]] for the 8-bit scale quantiser, "
                          "or gemv,rows,cols,nbits,g[,batch[,reps]] for the fused dequantise + matrix-vector product, "
-                         "or half,rows,cols,nbits,g[,reps] for the half-precision solver variant beside the fp32 one")
+                         "or half,rows,cols,nbits,g[,reps] for the half-precision solver variant beside the fp32 one, "
+                         "or tensor,rows,cols,nbits,g[,reps[,f16|bf16[,zero_nbits]]] for tensor stop on its "
+                         "resident launch beside its chunked launches")
     ap.add_argument("--workload", default="llama2-70b",
                     choices=["llama2-70b", "llama2-7b-mlp-sweep", "llama2-70b-stream", "llama2-13b-stream"])
     ap.add_argument("--layers", type=int, default=None,

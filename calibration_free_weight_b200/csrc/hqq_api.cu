@@ -335,6 +335,31 @@ int hqq_gemm_wait_selftest(int64_t limit_us, void* stream) {
     return HQQ_OK;
 }
 
+int hqq_set_tensor_resident(int mode) {
+    if (mode < 0 || mode > 2) return -1;
+    const int prev = hqq::tensor_resident();
+    hqq::set_tensor_resident(mode);
+    return prev;
+}
+
+int hqq_tensor_resident(int64_t rows, int64_t cols, int dtype, int group_size, int axis, int iters) {
+    if (hqq::check_args(rows, cols, dtype, 4, group_size, axis, 0.7f, 1.0f, 1.0f, iters, HQQ_STOP_TENSOR, 16) !=
+        HQQ_OK)
+        return 0;
+    return hqq::tensor_uses_resident(rows, cols, dtype, group_size, axis, iters) ? 1 : 0;
+}
+
+int hqq_quantize_wait_selftest(void* workspace, size_t workspace_bytes, int64_t limit_us, void* stream) {
+    if (limit_us < 1 || limit_us > 1000000 || workspace_bytes < 256) return HQQ_ERR_INVALID_ARG;
+    if (!is_device_ptr(workspace) || !aligned(workspace, 256)) return HQQ_ERR_INVALID_ARG;
+    if (hqq::launch_tensor_wait_selftest(static_cast<uint8_t*>(workspace), static_cast<unsigned long long>(limit_us) * 1000ull,
+                                         static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return HQQ_ERR_CUDA;
+    }
+    return HQQ_OK;
+}
+
 int hqq_quantize_scale8(const void* scale, int64_t num_groups, int scale_group, void* scale_q, void* scale_meta,
                         void* stream) {
     if (num_groups < 0 || scale_group < 1) return HQQ_ERR_INVALID_ARG;
@@ -371,7 +396,7 @@ const char* hqq_status_string(int status) {
         case HQQ_ERR_ALIGN: return "misaligned buffer";
         case HQQ_ERR_CUDA: return "CUDA runtime error";
         case HQQ_ERR_TIMEOUT: return "a bounded device wait gave up";
-        case HQQ_ERR_COOP_UNSUPPORTED: return "cooperative launch unsupported (reserved; not produced)";
+        case HQQ_ERR_COOP_UNSUPPORTED: return "cooperative launch unsupported (reserved; not returned)";
         case HQQ_ERR_WORKSPACE: return "workspace missing or too small";
         default: return "unknown status";
     }

@@ -14,6 +14,7 @@ constexpr int64_t kMinSlice = 4096;  // smallest group-mode slice (entries) a wo
 constexpr int kGemmMaxBatch = 65536;  // batch bound of hqq_gemm (argument check)
 constexpr int kMaxIters = 1000;      // upper bound on iters (argument check)
 constexpr float kScaleCap = 2.0e4f;  // cap on s (and on the 8-bit zero quantiser's scale)
+constexpr uint32_t kStatusTimeout = 6;  // HQQ_ERR_TIMEOUT, as the device writes it to the status word
 
 // Workspace layout (offsets 256-byte aligned):
 //   header      256 B: status word, CTA ticket, kept-zero range, pass counts
@@ -100,6 +101,17 @@ int sm_count();
 cudaError_t launch_gemm_wait_selftest(unsigned long long limit_ns, cudaStream_t stream);
 // Synchronises the stream; 0, 6 (a wait of a product gave up; cleared) or 5 (CUDA error).
 int gemm_take_status(cudaStream_t stream);
+
+// Tensor stop on one cooperative launch with W kept on chip, or the chunked
+// launches: mode 0 never the former, 1 (default) for g >= 32 where it fits, 2
+// wherever it fits.
+void set_tensor_resident(int mode);
+int tensor_resident();
+// Whether a tensor-stop call of this shape takes the resident kernel on the current device.
+bool tensor_uses_resident(int64_t rows, int64_t cols, int dtype, int g, int axis, int iters);
+// The resident kernel's bounded wait on a decision nothing publishes (diagnostic):
+// zeroes the workspace header, then records HQQ_ERR_TIMEOUT in its status word.
+cudaError_t launch_tensor_wait_selftest(uint8_t* ws, unsigned long long limit_ns, cudaStream_t stream);
 
 // Launchers: return cudaSuccess or the launch error.
 cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream);

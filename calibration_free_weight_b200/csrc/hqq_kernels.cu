@@ -40,6 +40,9 @@
 //   kept iterate's stored zero-point only when a tensor error rose; otherwise
 //   the chunk kernel's own output launch writes them.
 
+#include <atomic>
+#include <type_traits>
+
 #include "hqq_device.cuh"
 
 namespace hqq {
@@ -74,6 +77,9 @@ constexpr int kWordBestIt = 7;  // and the kept iterate + 1 (0: none), written b
 constexpr int kWordPass = 8;   // survivor count of group pass p at kWordPass + p
 constexpr int kMaxPasses = 16;
 constexpr int kWordChunk = 24;  // words 24-25: next chunk of the one-pass group solver (64-bit counter)
+constexpr int kWordArrive = 26;  // words 26-29: warps of the resident tensor solver that posted the error
+                                 // partial of an iteration, by iteration mod 4 (cumulative over the call)
+constexpr int kWordDec = 32;     // words 32-63: its published stop decisions, 4 entries of 8 words
 
 // ------------------------------------------------------- group outputs ----
 
@@ -835,6 +841,427 @@ __global__ void __launch_bounds__(256) tensor_output_kernel(const KParams k) {
     if (k.zero_nbits == 8) merge_zero_range<8>(k, zmin, zmax, sred);
 }
 
+// 16-byte copies global -> shared that bypass the registers (and L1).
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ============================================ tensor stop, W kept on chip ==
+//
+// solve_tensor_resident_kernel (tensor stop, axis 1): one cooperative launch
+// runs every iteration of every group.  Each warp owns a fixed run of T warp
+// tiles.  The iterations go in rounds of C: in a round the warp visits
+// each of its tiles once, copies its raw values from W (cp.async, two buffers
+// per warp), forms fl(w*s) once and runs the round's iterations on it in
+// registers.  The launcher only takes this path when W fits in half the L2, so
+// after the first round those copies are L2 hits, and when each group's state
+// between rounds -- float4 (s, z0, the group's largest w*s, s^-p), float2 (the
+// sum of w*s split into two floats) and the zero-point to continue from --
+// fits in the warp's shared memory.  The zero-point of every iteration goes to
+// a ring of 2*C + 2 slots per group in the workspace, from which the kept one
+// is read at the end.
+//
+// The tensor error of iteration m is the sum over all groups: one grid-wide
+// reduction per iteration, and no grid barrier.  At the end of a round every
+// warp adds its fp64 partials to its CTA's shared memory; the CTA's last warp
+// to arrive sums the CTA's eight in warp order and posts them to the workspace
+// with a global arrival counter; the warp that brings the counter to the grid
+// size sums all CTAs' partials of each of the round's iterations in CTA order
+// (the same on every run with the same grid), applies the stop rule to the
+// state published for the previous round, and publishes (best error so far,
+// first rise) for the round.  A warp starts round r only after round r-2 is
+// published, so the wait is normally already satisfied, and leaves the loop
+// when a rise is reported: the kept iterate, the one before the first rise,
+// then lies in the last 2*C + 1 iterations run, all still in the ring.
+// Iterations past the rise run speculatively and are discarded.  Every wait
+// is bounded by the global timer: after the limit the warp records
+// HQQ_ERR_TIMEOUT in the workspace's status word, the other warps see it in
+// their next wait and give up too, and no outputs are written.
+// Iterations per round: 8 for tiles of 32 elements per lane, 4 below (the
+// workspace's zero-point slots, 24 and 10, hold the ring of 2*C + 2).
+__host__ __device__ constexpr int res_c(int E) { return E >= 32 ? 8 : 4; }
+__host__ __device__ constexpr int res_slots(int E) { return 2 * res_c(E) + 2; }
+constexpr unsigned long long kResWaitNs = 1000000000ull;
+
+__device__ __forceinline__ unsigned long long res_now_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Published decision of round r: words kWordDec + 8*(r mod 4) + (0-1: tensor
+// error of the round's last iteration, 2-3: best error so far, 4: first rise
+// + 1 or 0, 5: r + 1 once published).
+__device__ __forceinline__ uint32_t* res_dec(const KParams& k, int r) { return k.counters + kWordDec + 8 * (r & 3); }
+
+// Lane-0 wait until round r is published; false after the limit (recording
+// the timeout) or when another warp already gave up.
+__device__ __forceinline__ bool res_wait_dec(const KParams& k, int r, unsigned long long limit_ns) {
+    volatile uint32_t* tag = res_dec(k, r) + 5;
+    volatile uint32_t* status = k.counters;
+    if (*tag == static_cast<uint32_t>(r + 1)) {
+        __threadfence();
+        return true;
+    }
+    const unsigned long long t0 = res_now_ns();
+    while (*tag != static_cast<uint32_t>(r + 1)) {
+        if (*status != 0u) return false;
+        if (res_now_ns() - t0 > limit_ns) {
+            atomicCAS(k.counters, 0u, kStatusTimeout);
+            return false;
+        }
+        __nanosleep(128);
+    }
+    __threadfence();
+    return true;
+}
+
+// Lane-0 wait of a warp for the first rise (or -1) reported by round r,
+// through its CTA's copy in shared memory: the CTA knows the rounds < *pub, the
+// rises in rise[r mod 4]; one warp at a time (*poll) reads the workspace for
+// the CTA and copies what was published, the others wait on shared memory, so
+// the published words see one reader per CTA.  False after the limit
+// (recording the timeout) or when another warp already gave up.
+__device__ __forceinline__ bool res_cta_dec(const KParams& k, int r, volatile int* pub, volatile int* rise,
+                                            int* poll, unsigned long long limit_ns, int* rise_out) {
+    volatile uint32_t* status = k.counters;
+    unsigned long long t0 = 0;
+    unsigned spins = 0;
+    for (;;) {
+        if (*pub > r) {
+            *rise_out = rise[r & 3];
+            return true;
+        }
+        if (t0 == 0) t0 = res_now_ns();
+        if (atomicCAS(poll, 0, 1) == 0) {  // this warp reads the workspace for the CTA
+            bool ok = true;
+            while (*pub <= r) {
+                const int rr = *pub;
+                const uint32_t* d = res_dec(k, rr);
+                if (*reinterpret_cast<volatile const uint32_t*>(d + 5) == static_cast<uint32_t>(rr + 1)) {
+                    __threadfence();
+                    rise[rr & 3] = static_cast<int>(__ldcg(d + 4)) - 1;
+                    __threadfence_block();
+                    *pub = rr + 1;
+                    continue;
+                }
+                if ((++spins & 15u) == 0u && *status != 0u) {
+                    ok = false;
+                    break;
+                }
+                if (res_now_ns() - t0 > limit_ns) {
+                    atomicCAS(k.counters, 0u, kStatusTimeout);
+                    ok = false;
+                    break;
+                }
+                __nanosleep(128);
+            }
+            atomicExch(poll, 0);
+            if (!ok) return false;
+            continue;
+        }
+        if ((++spins & 63u) == 0u && *status != 0u) return false;
+        if (res_now_ns() - t0 > limit_ns) {
+            atomicCAS(k.counters, 0u, kStatusTimeout);
+            return false;
+        }
+        __nanosleep(64);
+    }
+}
+
+__device__ __forceinline__ double res_load_d(const uint32_t* w) {
+    const uint32_t lo = __ldcg(w), hi = __ldcg(w + 1);
+    return __hiloint2double(static_cast<int>(hi), static_cast<int>(lo));
+}
+
+// Called by the whole warp after its CTA posted the partials of round r
+// (iterations k0 .. k0+nk-1, row c of `parts` for iteration k0+c) as the last
+// of nc CTAs: sum each iteration's partials in CTA order (a lane's loads for
+// the nk iterations are issued together), apply the stop rule in iteration
+// order, publish.
+template <int C>
+__device__ __forceinline__ bool res_publish(const KParams& k, int r, int k0, int nk, const double* parts, int nc,
+                                            unsigned long long limit_ns) {
+    const int lane = threadIdx.x & 31;
+    double v[C] = {};
+    for (int b = lane; b < nc; b += 32) {
+        double t[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) t[c] = c < nk ? __ldcg(parts + static_cast<size_t>(c) * nc + b) : 0.0;
+#pragma unroll
+        for (int c = 0; c < C; ++c) v[c] += t[c];
+    }
+#pragma unroll
+    for (int c = 0; c < C; ++c) v[c] = warp_sum_d(v[c]);
+    bool ok = true;
+    if (lane == 0) {
+        double best = INFINITY, e = 0.0;
+        int rise = -1;
+        if (r > 0) {
+            ok = res_wait_dec(k, r - 1, limit_ns);
+            if (ok) {
+                const uint32_t* d = res_dec(k, r - 1);
+                best = res_load_d(d + 2);
+                rise = static_cast<int>(__ldcg(d + 4)) - 1;
+            }
+        }
+        if (ok) {
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                if (c >= nk) break;
+                e = v[c] / static_cast<double>(k.n);
+                if (rise < 0) {  // first iteration whose error is not below the best so far
+                    if (e < best) best = e;
+                    else rise = k0 + c;
+                }
+            }
+            uint32_t* d = res_dec(k, r);
+            d[0] = static_cast<uint32_t>(__double2loint(e));
+            d[1] = static_cast<uint32_t>(__double2hiint(e));
+            d[2] = static_cast<uint32_t>(__double2loint(best));
+            d[3] = static_cast<uint32_t>(__double2hiint(best));
+            d[4] = static_cast<uint32_t>(rise + 1);
+            __threadfence();
+            atomicExch(d + 5, static_cast<uint32_t>(r + 1));
+        }
+    }
+    return __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+}
+
+// Shared memory of one warp, in bytes: two copy buffers of a tile (64*E bytes
+// each), then per group of its T tiles a float4, a float2 and a float (the
+// state between rounds); rounded up to 16 bytes so that every warp's region
+// starts 16-byte aligned.
+__host__ __device__ constexpr size_t res_warp_bytes(int E, int T, int gpw) {
+    return (static_cast<size_t>(128 * E) + static_cast<size_t>(T) * gpw * (16 + 8 + 4) + 15) & ~static_cast<size_t>(15);
+}
+
+template <int DT, int E>
+__global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 2)
+    solve_tensor_resident_kernel(const KParams k, int T, unsigned long long limit_ns) {
+    constexpr int C = res_c(E);
+    constexpr int kSlots = res_slots(E);
+    extern __shared__ uint4 dyn_smem[];
+    __shared__ float2 sred[kRegWarps];
+    __shared__ double sacc[C][kRegThreads];      // this round's error partial of each thread
+    __shared__ double cpart[4][C][kRegWarps];    // warps' partials, by round mod 4
+    __shared__ unsigned ccount[4];                   // warps that posted them (cumulative)
+    __shared__ int dpub, dpoll, drise[4];            // the CTA's copy of the published rounds
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x < 4) ccount[threadIdx.x] = 0u;
+    if (threadIdx.x == 0) dpub = dpoll = 0;
+    __syncthreads();
+    const int gpw = 32 >> k.logP;
+    const int slot = lane >> k.logP;
+    const int nst = T * gpw;  // state entries of this warp
+    unsigned char* const base = reinterpret_cast<unsigned char*>(dyn_smem) + res_warp_bytes(E, T, gpw) * warp;
+    uint4* const buf = reinterpret_cast<uint4*>(base);              // [2][E/8][32]
+    float4* const stA = reinterpret_cast<float4*>(base + 128 * E);  // [nst]
+    float2* const stB = reinterpret_cast<float2*>(stA + nst);       // [nst]
+    float* const stZ = reinterpret_cast<float*>(stB + nst);         // [nst]
+    const int nc = static_cast<int>(gridDim.x);
+    const int gw = static_cast<int>(blockIdx.x) * kRegWarps + warp;
+    const int64_t ntiles = num_warp_tiles<1>(k);
+    const int64_t t0 = static_cast<int64_t>(gw) * T;
+    const int nt = t0 >= ntiles ? 0 : static_cast<int>(ntiles - t0 < T ? ntiles - t0 : T);
+    const float inv_g = 1.0f / static_cast<float>(k.g);
+    const int iters = k.iters_eff;
+    const int64_t G = k.G;
+    float zmin = FLT_MAX, zmax = -FLT_MAX;
+
+    // The copies of this warp's tiles form one cyclic stream (tile q of copy
+    // number c = q + nt * round).  Copy c goes to buffer c mod 2, as the
+    // tile's 16-byte pieces in order, piece p of the tile by lane p mod 32 (so
+    // each instruction copies 512 contiguous bytes), stored where its owner
+    // lane reads it: piece p belongs to lane p / (E/8), as that lane's piece
+    // p mod (E/8), at buf[(c&1)][p mod (E/8)][p / (E/8)].
+    int issued = 0, qi = 0, used = 0;
+    auto issue = [&]() {
+        if (nt > 0) {
+            const int64_t e0 = (t0 + qi) * 32 * E;  // first element of the tile
+            const int64_t n_el = k.n - e0;          // elements left in W (the last tile may be partial)
+#pragma unroll
+            for (int u = 0; u < E / kPiece; ++u) {
+                const int p = u * 32 + lane;
+                if (static_cast<int64_t>(p) * kPiece < n_el)
+                    cp_async16(buf + ((issued & 1) * (E / kPiece) + p % (E / kPiece)) * 32 + p / (E / kPiece),
+                               k.W + e0 + static_cast<int64_t>(p) * kPiece);
+            }
+            if (++qi == nt) qi = 0;
+        }
+        cp_async_commit();
+        ++issued;
+    };
+    // the next tile of the stream as fp32 (zeros for lanes past the last group)
+    auto next_tile = [&](int q, float* x, WarpTile& w) {
+        __syncwarp();  // every lane has read the buffer the next copy overwrites
+        issue();
+        cp_async_wait<1>();
+        __syncwarp();  // every lane's share of this copy has landed
+        w = warp_tile<1>(k, t0 + q);
+        if (w.valid) {
+#pragma unroll
+            for (int u = 0; u < E / kPiece; ++u) unpack8<DT>(buf[((used & 1) * (E / kPiece) + u) * 32 + lane], x + u * kPiece);
+        } else {
+#pragma unroll
+            for (int i = 0; i < E; ++i) x[i] = 0.0f;
+        }
+        ++used;
+    };
+
+    issue();
+    bool ok = true;
+    int kept = -1;  // kept iterate once a rise is known
+    float beta = k.beta;  // beta of the round's first iteration (sequential fp32 products)
+    const int nrounds = (iters + C - 1) / C;
+    int r = 0;
+    for (; r < nrounds; ++r) {
+        const int k0 = r * C;
+        const int nk = iters - k0 < C ? iters - k0 : C;
+        if (r >= 2) {
+            int rise = -1;
+            if (lane == 0) ok = res_cta_dec(k, r - 2, &dpub, drise, &dpoll, limit_ns, &rise);
+            ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+            rise = __shfl_sync(kFull, rise, 0);
+            if (!ok) break;
+            if (rise >= 0) {
+                kept = rise > 0 ? rise - 1 : 0;
+                break;
+            }
+        }
+        float thr[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            thr[c] = shrink_threshold(beta, k.p);
+            if (c < nk) beta = __fmul_rn(beta, k.kappa);
+        }
+#pragma unroll
+        for (int c = 0; c < C; ++c) sacc[c][threadIdx.x] = 0.0;
+        for (int q = 0; q < nt; ++q) {
+            float x[E], ws[E];
+            WarpTile w;
+            next_tile(q, x, w);
+            const int i = q * gpw + slot;
+            const bool writer = w.valid && w.part == 0;
+            float s, z0, z, lmin, lmax, spow;
+            F2 sws2;
+            if (r == 0) {
+                double sws;
+                init_lane<E>(k, w, x, ws, &s, &z0, &sws, &lmin, &lmax);
+                spow = pow_pos(s, -k.p);
+                sws2 = split_f2(sws);
+                z = z0;
+                const float gmax = seg_max(lmax, k.P);
+                if (writer) {
+                    stA[i] = make_float4(s, z0, gmax, spow);
+                    stB[i] = make_float2(sws2.hi, sws2.lo);
+                }
+            } else {
+                const float4 a = w.valid ? stA[i] : make_float4(1.0f, 0.0f, 0.0f, 1.0f);
+                const float2 b = w.valid ? stB[i] : make_float2(0.0f, 0.0f);
+                s = a.x;
+                z0 = a.y;
+                lmin = -z0;  // fl(min w * s), exactly: rounding is symmetric
+                lmax = a.z;  // the group's; the warp-wide clamp test is the same as with the lanes' own
+                spow = a.w;
+                sws2 = F2{b.x, b.y};
+                z = w.valid ? stZ[i] : 0.0f;
+                const uint64_t s2 = f2_pack(s, s);
+#pragma unroll
+                for (int e = 0; e < E; e += 2) f2_unpack(f2_mul(f2_pack(x[e], x[e + 1]), s2), ws[e], ws[e + 1]);
+            }
+            float* const zring = writer ? k.t_zs + w.j : nullptr;
+#pragma unroll 1
+            for (int c = 0; c < nk; ++c) {
+                if (zring) zring[static_cast<int64_t>((k0 + c) % kSlots) * G] = z;
+                tensor_iteration<DT, 1, E>(k, w, ws, lmin, lmax, s, z0, k0 + c, thr[c], spow, sws2, inv_g,
+                                           sacc[c][threadIdx.x], z);
+            }
+            if (writer) stZ[i] = z;
+        }
+        // post this warp's partials; the CTA's last warp posts the CTA's, and
+        // the grid's last CTA publishes the round
+        double v[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) v[c] = warp_sum_d(sacc[c][threadIdx.x]);
+        double* const parts = k.tparts + static_cast<size_t>(r & 3) * C * nc;
+        unsigned last = 0;
+        if (lane == 0) {
+#pragma unroll
+            for (int c = 0; c < C; ++c) cpart[r & 3][c][warp] = v[c];
+            __threadfence_block();
+            const unsigned ctarget = static_cast<unsigned>(r / 4 + 1) * kRegWarps;
+            if (atomicAdd(&ccount[r & 3], 1u) + 1u == ctarget) {
+                __threadfence_block();
+                for (int c = 0; c < nk; ++c) {
+                    double cv = 0.0;
+                    for (int w = 0; w < kRegWarps; ++w) cv += cpart[r & 3][c][w];
+                    parts[static_cast<size_t>(c) * nc + blockIdx.x] = cv;
+                }
+                __threadfence();
+                const uint32_t target = static_cast<uint32_t>(r / 4 + 1) * static_cast<uint32_t>(nc);
+                last = atomicAdd(k.counters + kWordArrive + (r & 3), 1u) + 1u == target;
+                if (last) __threadfence();
+            }
+        }
+        if (__shfl_sync(kFull, last, 0)) {
+            ok = res_publish<C>(k, r, k0, nk, parts, nc, limit_ns);
+            if (!ok) break;
+        }
+    }
+    if (ok && kept < 0) {  // every round ran: the rule over all of them
+        int rise = -1;
+        if (lane == 0) ok = res_cta_dec(k, nrounds - 1, &dpub, drise, &dpoll, limit_ns, &rise);
+        ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+        rise = __shfl_sync(kFull, rise, 0);
+        kept = rise >= 0 ? (rise > 0 ? rise - 1 : 0) : iters - 1;
+    }
+    if (ok) {  // outputs of the kept iterate
+        __threadfence();  // the ring's zero-points, written by this warp's lanes, are read back below
+        __syncwarp();
+        const float* const zk = k.t_zs + static_cast<int64_t>(kept % kSlots) * G;
+        float bk = k.beta;
+        for (int i = 0; i < kept; ++i) bk = __fmul_rn(bk, k.kappa);
+        for (int q = 0; q < nt; ++q) {
+            float x[E], ws[E];
+            WarpTile w;
+            next_tile(q, x, w);
+            const int i = q * gpw + slot;
+            const float4 a = w.valid ? stA[i] : make_float4(1.0f, 0.0f, 0.0f, 1.0f);
+            const float s = a.x, z0 = a.y;
+            const float z = w.valid ? __ldcg(zk + w.j) : 0.0f;
+            const uint64_t s2 = f2_pack(s, s);
+#pragma unroll
+            for (int e = 0; e < E; e += 2) f2_unpack(f2_mul(f2_pack(x[e], x[e + 1]), s2), ws[e], ws[e + 1]);
+            store_lane_codes<1, E>(k, w, ws, z);
+            float err_mean = 0.0f;
+            if (k.dbg_err) {
+                float err, sq;
+                bool sp;
+                double swe;
+                eval_lane<E>(k, w.valid, x, ws, s, z, z0, bk, shrink_threshold(bk, k.p), &err, &sq, &sp, &swe);
+                err_mean = err * a.w * inv_g;
+            }
+            if (w.valid && w.part == 0) store_group(k, w.j, s, z, kept, err_mean, &zmin, &zmax);
+        }
+    }
+    cp_async_wait<0>();
+    if (k.zero_nbits == 8) merge_zero_range<kRegWarps>(k, zmin, zmax, sred);
+}
+
+// Diagnostic: the resident solver's bounded wait on a decision that nothing
+// publishes, with a short limit; it gives up and records the timeout in the
+// workspace's status word exactly as the solver does.
+__global__ void res_wait_selftest_kernel(KParams k, unsigned long long limit_ns) {
+    if (threadIdx.x == 0) res_wait_dec(k, 0, limit_ns);
+}
+
 // ============================================================= group stop ==
 
 // One pass of the group-stop solver (see the file comment).  Entries are warp
@@ -1003,16 +1430,6 @@ __global__ void __launch_bounds__(kRegThreads, E <= 16 ? 4 : 3) solve_group_kern
 // never recomputed from a second read of W).  Slots run at different
 // iteration indices; beta only matters on the rare proximal path, which takes
 // each slot's own.
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-    const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // Packed min/max of eight 16-bit values held in a uint4 (fp16 or bf16; the
 // order of 16-bit values equals the order of their fp32 conversions).
@@ -1798,6 +2215,9 @@ __global__ void __launch_bounds__(256) dequant_kernel(const DqParams d) {
 
 struct DevInfo {
     int sms = 0;
+    int l2_bytes = 0;
+    int coop = 0;        // cooperative launches supported
+    int smem_optin = 0;  // largest dynamic shared memory per CTA after opting in
 };
 
 DevInfo device_info() {
@@ -1807,13 +2227,19 @@ DevInfo device_info() {
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
     if (!have[dev]) {
-        int sms = 0;
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cache[dev].sms = sms > 0 ? sms : 1;
+        DevInfo d;
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&d.l2_bytes, cudaDevAttrL2CacheSize, dev);
+        cudaDeviceGetAttribute(&d.coop, cudaDevAttrCooperativeLaunch, dev);
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (d.sms < 1) d.sms = 1;
+        cache[dev] = d;
         have[dev] = true;
     }
     return cache[dev];
 }
+
+std::atomic<int> g_tensor_resident{1};
 
 template <typename K>
 cudaError_t persistent_grid(K kernel, int threads, size_t smem, int64_t work_units, int* grid) {
@@ -1903,8 +2329,68 @@ cudaError_t launch_group_onepass(KParams& k, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+// Launch shape of the resident tensor-stop kernel, or false when this problem
+// does not take it: the mode allows it (0 never; 1, the default, for tiles of
+// 32 elements per lane, g >= 32; 2 for every g); axis 1 and at least one
+// iteration; a device with
+// cooperative launches; W within half the L2 (so its copies at every
+// iteration hit); the per-group state of every warp's tiles within the shared
+// memory of the CTAs one SM holds.  Two (32-element tiles) or four CTAs per
+// SM, fewer when the state needs more shared memory per CTA.
+template <int DT, int E>
+bool plan_resident(const KParams& k, int* grid_out, int* T_out, size_t* smem_out) {
+    if (!g_tensor_resident.load() || k.axis != 1 || k.iters_eff < 1) return false;
+    if (E < 32 && g_tensor_resident.load() != 2) return false;  // measured slower than the chunks below g = 32
+                                                                  // (mode 2 takes it wherever it fits)
+    const DevInfo d = device_info();
+    if (!d.coop || static_cast<double>(k.n) * 2.0 > 0.5 * static_cast<double>(d.l2_bytes)) return false;
+    auto kern = solve_tensor_resident_kernel<DT, E>;
+    const int gpw = 32 >> k.logP;
+    const int64_t ntiles = (k.G + gpw - 1) / gpw;
+    static_assert(res_slots(E) <= 2 * (chunk_max(chunk_len(E)) + 1), "the zero-point ring fits the workspace's slots");
+    for (int cps = E <= 16 ? 4 : 2; cps >= 2; --cps) {  // at least 16 warps per SM
+        int64_t grid = static_cast<int64_t>(d.sms) * cps;
+        const int64_t enough = (ntiles + kRegWarps - 1) / kRegWarps;  // a tile per warp
+        if (grid > enough) grid = enough;
+        const int64_t nw = grid * kRegWarps;
+        if (4 * res_c(E) * grid > static_cast<int64_t>(kChunkMax) * kMaxPartials) continue;  // partial rows
+        const int64_t T = (ntiles + nw - 1) / nw;
+        const size_t smem = res_warp_bytes(E, static_cast<int>(T), gpw) * kRegWarps;
+        if (smem + 20 * 1024 > static_cast<size_t>(d.smem_optin)) continue;  // with the kernel's static shared memory
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRegThreads, smem) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        if (per_sm < cps) continue;
+        *grid_out = static_cast<int>(grid);
+        *T_out = static_cast<int>(T);
+        *smem_out = smem;
+        return true;
+    }
+    return false;
+}
+
+template <int DT, int E>
+cudaError_t launch_resident(KParams& k, int grid, int T, size_t smem, cudaStream_t stream) {
+    unsigned long long limit = kResWaitNs;
+    void* args[] = {&k, &T, &limit};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(solve_tensor_resident_kernel<DT, E>), dim3(grid),
+                                       dim3(kRegThreads), args, smem, stream);
+}
+
 template <int DT, int AXIS, int E>
 cudaError_t launch_tensor(KParams& k, cudaStream_t stream) {
+    if constexpr (AXIS == 1) {
+        int rg = 0, rt = 0;
+        size_t rs = 0;
+        if (plan_resident<DT, E>(k, &rg, &rt, &rs)) return launch_resident<DT, E>(k, rg, rt, rs, stream);
+    }
     const int gpw = 32 >> k.logP;
     const int64_t tiles = AXIS == 1 ? (k.G + gpw - 1) / gpw : (k.rows / k.g) * ((k.cols + gpw - 1) / gpw);
     auto kern = solve_tensor_kernel<DT, AXIS, E>;
@@ -2115,6 +2601,43 @@ cudaError_t launch_solve(const SolveArgs& a, cudaStream_t stream) {
         err = cudaGetLastError();
     }
     return err;
+}
+
+void set_tensor_resident(int mode) { g_tensor_resident.store(mode < 0 ? 0 : (mode > 2 ? 2 : mode)); }
+int tensor_resident() { return g_tensor_resident.load(); }
+
+bool tensor_uses_resident(int64_t rows, int64_t cols, int dtype, int g, int axis, int iters) {
+    if (axis != 1 || iters < 1 || rows * cols <= 0) return false;
+    const Geometry geo = make_geometry(g);
+    KParams k{};
+    k.rows = rows;
+    k.cols = cols;
+    k.n = rows * cols;
+    k.G = k.n / g;
+    k.g = g;
+    k.E = geo.E;
+    k.P = geo.P;
+    k.logP = geo.logP;
+    k.axis = axis;
+    k.iters_eff = iters;
+    int grid = 0, T = 0;
+    size_t smem = 0;
+    auto plan = [&](auto dt) {
+        constexpr int DT = decltype(dt)::value;
+        if (k.E == 8) return plan_resident<DT, 8>(k, &grid, &T, &smem);
+        if (k.E == 16) return plan_resident<DT, 16>(k, &grid, &T, &smem);
+        return plan_resident<DT, 32>(k, &grid, &T, &smem);
+    };
+    return dtype == 0 ? plan(std::integral_constant<int, 0>{}) : plan(std::integral_constant<int, 1>{});
+}
+
+cudaError_t launch_tensor_wait_selftest(uint8_t* ws, unsigned long long limit_ns, cudaStream_t stream) {
+    cudaError_t err = cudaMemsetAsync(ws, 0, 256, stream);
+    if (err != cudaSuccess) return err;
+    KParams k{};
+    k.counters = reinterpret_cast<uint32_t*>(ws);
+    res_wait_selftest_kernel<<<1, 32, 0, stream>>>(k, limit_ns);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_scale8(const uint16_t* scale, int64_t G, int S, uint8_t* codes, float* meta,

@@ -21,7 +21,8 @@ EXPORTED = ("hqq_packed_bytes", "hqq_num_groups", "hqq_workspace_bytes", "hqq_qu
             "hqq_get_status", "hqq_status_string", "hqq_quantize_noalloc", "hqq_quantize_scale8",
             "hqq_dequantize_s8", "hqq_stream_device_bytes", "hqq_quantize_stream", "hqq_gemv",
             "hqq_stream_jobs_device_bytes", "hqq_quantize_stream_jobs", "hqq_gemm", "hqq_gemm_get_status",
-            "hqq_gemm_wait_selftest", "hqq_gemm_workspace_bytes", "hqq_quantize_half")
+            "hqq_gemm_wait_selftest", "hqq_gemm_workspace_bytes", "hqq_quantize_half", "hqq_tensor_resident",
+            "hqq_set_tensor_resident", "hqq_quantize_wait_selftest")
 
 
 class hqq_host_matrix(C.Structure):
@@ -77,6 +78,12 @@ def _load():
     L.hqq_gemm_get_status.argtypes = [P]
     L.hqq_gemm_wait_selftest.restype = i32
     L.hqq_gemm_wait_selftest.argtypes = [i64, P]
+    L.hqq_tensor_resident.restype = i32
+    L.hqq_tensor_resident.argtypes = [i64, i64, i32, i32, i32, i32]
+    L.hqq_set_tensor_resident.restype = i32
+    L.hqq_set_tensor_resident.argtypes = [i32]
+    L.hqq_quantize_wait_selftest.restype = i32
+    L.hqq_quantize_wait_selftest.argtypes = [P, sz, i64, P]
     HM = C.POINTER(hqq_host_matrix)
     L.hqq_stream_device_bytes.restype = sz
     L.hqq_stream_device_bytes.argtypes = [HM, i32, i32, i32, i32, i32, i32]
@@ -205,6 +212,18 @@ def hqq_gemm_get_status(stream=None):
 
 def hqq_gemm_wait_selftest(limit_us, stream=None):
     return lib.hqq_gemm_wait_selftest(limit_us, _stream(stream))
+
+
+def hqq_tensor_resident(rows, cols, dtype, group_size, axis=1, iters=20):
+    return lib.hqq_tensor_resident(rows, cols, dtype, group_size, axis, iters)
+
+
+def hqq_set_tensor_resident(mode):
+    return lib.hqq_set_tensor_resident(int(mode))
+
+
+def hqq_quantize_wait_selftest(workspace, workspace_bytes, limit_us, stream=None):
+    return lib.hqq_quantize_wait_selftest(_ptr(workspace), workspace_bytes, limit_us, _stream(stream))
 
 
 def hqq_stream_jobs_device_bytes(jobs, n):

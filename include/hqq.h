@@ -78,8 +78,10 @@ typedef enum {
     HQQ_ERR_DTYPE = 3,            /* dtype not HQQ_F16 / HQQ_BF16 */
     HQQ_ERR_ALIGN = 4,            /* a buffer is not aligned as documented */
     HQQ_ERR_CUDA = 5,             /* a CUDA runtime call failed (launch, attribute query) */
-    HQQ_ERR_TIMEOUT = 6,          /* a bounded wait inside hqq_gemm gave up (hqq_gemm_get_status) */
-    HQQ_ERR_COOP_UNSUPPORTED = 7, /* reserved: no cooperative launch is used */
+    HQQ_ERR_TIMEOUT = 6,          /* a bounded device wait gave up: the tensor-stop solver's (hqq_get_status)
+                                     or hqq_gemm's (hqq_gemm_get_status) */
+    HQQ_ERR_COOP_UNSUPPORTED = 7, /* reserved, not returned: without cooperative launches the tensor-stop
+                                     solver takes its chunked launches instead */
     HQQ_ERR_WORKSPACE = 8         /* workspace missing or smaller than hqq_workspace_bytes() */
 } hqq_status;
 
@@ -132,10 +134,13 @@ size_t hqq_workspace_bytes(int64_t rows, int64_t cols, int group_size, int axis,
  *                    zero-point (lg2/ex2 hardware approximations, ~1e-6 rel).
  *   debug_zero_f32   optional device fp32[G]: z* before storage.
  *   stream       cudaStream_t as void*.
- * Returns HQQ_OK or an error code.  No kernel waits on another CTA, so there
- * is no device-side failure to report; hqq_get_status reads the (zeroed)
- * status word for callers that check it.  Calls that share a workspace must
- * not run concurrently.
+ * Returns HQQ_OK or an error code.  Tensor stop on axis 1 runs, when the
+ * problem fits (hqq_tensor_resident), as one cooperative launch whose warps
+ * wait for the tensor error of earlier iterations; each such wait gives up
+ * after about 1 s, and then the call's outputs are undefined and the
+ * workspace's status word holds HQQ_ERR_TIMEOUT (hqq_get_status).  No other
+ * path waits on another CTA.  Calls that share a workspace must not run
+ * concurrently.
  */
 int hqq_quantize(const void* W, int64_t rows, int64_t cols, int dtype, int nbits, int group_size, int axis,
                  float p, float beta, float kappa, int iters, int stop_mode, int zero_nbits,
@@ -384,10 +389,41 @@ int hqq_gemm_get_status(void* stream);
 int hqq_gemm_wait_selftest(int64_t limit_us, void* stream);
 
 /* Synchronise `stream` and return the device status word held in `workspace`
- * by the last hqq_quantize on it (HQQ_OK), or HQQ_ERR_CUDA if the
- * synchronisation or copy fails.  No counterpart on the pages: the channel for
- * errors found on the device after an asynchronous call returned. */
+ * by the last hqq_quantize on it: HQQ_OK, or HQQ_ERR_TIMEOUT when a wait of the
+ * resident tensor-stop solver gave up; HQQ_ERR_CUDA if the synchronisation or
+ * copy fails.  No counterpart on the pages: the channel for errors found on
+ * the device after an asynchronous call returned (the hot-path table's
+ * "grid barrier with a bounded spin"). */
 int hqq_get_status(const void* workspace, void* stream);
+
+/* Tensor stop (techreport.ngo, "Weight-only quantization without the
+ * calibration tax", section "Outlier-aware optimization without gradients":
+ * the mean error over the whole tensor decides the stop) keeps W on chip
+ * where it fits: one cooperative launch runs every iteration, the per-group
+ * state stays in shared memory and W (within half the L2) is read from L2 at
+ * each iteration; one grid-wide fp64 reduction per iteration, no grid
+ * barrier.  Otherwise the iterations run in chunks of launches that re-read W.
+ * Both give the outputs the stop rule defines; their tensor errors are summed
+ * in different orders, so a near-tied decision may differ.
+ * hqq_tensor_resident: 1 if hqq_quantize with stop_mode HQQ_STOP_TENSOR and
+ * these arguments (iters >= 1) takes the resident launch on the current
+ * device, else 0 (also for invalid arguments).
+ * hqq_set_tensor_resident: for the whole process, mode 0 never takes the
+ * resident launch, 1 (the default) takes it for group sizes >= 32 where it
+ * fits (below that it measured slower than the chunks), 2 wherever it fits;
+ * returns the previous mode, or -1 (nothing changed) for another value.  Not
+ * synchronised with calls in flight on other threads. */
+int hqq_tensor_resident(int64_t rows, int64_t cols, int dtype, int group_size, int axis, int iters);
+int hqq_set_tensor_resident(int mode);
+
+/* Diagnostic of the resident tensor-stop solver's bounded wait: zeroes the
+ * first 256 bytes of `workspace` (device, 256-byte aligned, workspace_bytes >=
+ * 256), then one thread runs the solver's wait, with a limit of limit_us
+ * microseconds (1 .. 1e6), on a decision that nothing publishes; it gives up
+ * and records the timeout as the solver does, so hqq_get_status(workspace)
+ * then returns HQQ_ERR_TIMEOUT.  Asynchronous on `stream`; returns HQQ_OK,
+ * HQQ_ERR_INVALID_ARG or HQQ_ERR_CUDA. */
+int hqq_quantize_wait_selftest(void* workspace, size_t workspace_bytes, int64_t limit_us, void* stream);
 
 /* Static English description of a status code (no counterpart on the pages). */
 const char* hqq_status_string(int status);

@@ -7,6 +7,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -320,3 +321,23 @@ def test_half_variant_rejects_on_host(hq):
     assert call(axis=0) == 1
     assert call(stop=1) == 1
     assert call() == 8  # every argument valid: only the missing workspace is left
+
+
+def test_tensor_resident_switch_and_query(hq):
+    """The process-wide switch returns the previous setting; the query answers 0
+    for invalid arguments and, without a device, for any problem; the wait
+    self-test rejects bad limits and host memory before launching."""
+    assert hq.lib.hqq_set_tensor_resident(0) == 1
+    assert hq.lib.hqq_set_tensor_resident(2) == 0
+    assert hq.lib.hqq_set_tensor_resident(3) == -1 and hq.lib.hqq_set_tensor_resident(-1) == -1
+    assert hq.lib.hqq_set_tensor_resident(1) == 2
+    assert hq.lib.hqq_set_tensor_resident(1) == 1
+    assert hq.lib.hqq_tensor_resident(4096, 4096, 0, 48, 1, 20) == 0
+    assert hq.lib.hqq_tensor_resident(4096, 4096, 5, 64, 1, 20) == 0
+    assert hq.lib.hqq_tensor_resident(4096, 4096, 0, 64, 1, -1) == 0
+    if not torch.cuda.is_available():
+        assert hq.lib.hqq_tensor_resident(4096, 4096, 0, 64, 1, 20) == 0
+    buf = (C.c_uint8 * 512)()
+    assert hq.lib.hqq_quantize_wait_selftest(C.cast(buf, C.c_void_p), 512, 0, None) == hq.HQQ_ERR_INVALID_ARG
+    assert hq.lib.hqq_quantize_wait_selftest(C.cast(buf, C.c_void_p), 512, 1000001, None) == hq.HQQ_ERR_INVALID_ARG
+    assert hq.lib.hqq_quantize_wait_selftest(C.cast(buf, C.c_void_p), 512, 1000, None) == hq.HQQ_ERR_INVALID_ARG
