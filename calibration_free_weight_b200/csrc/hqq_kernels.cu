@@ -14,7 +14,8 @@
 // MUFU pipe, not HBM, bounds the solver.
 //
 // The solver kernels hold a warp tile of 32/P groups in registers, E = g/P
-// elements per lane (E = min(g, 32)); no CTA ever waits for another.
+// elements per lane (E = min(g, 32)).  Only solve_tensor_resident_kernel has
+// CTAs that wait for others (bounded waits, in a cooperative launch).
 //
 // solve_group_onepass_kernel (group / no stop, axis 1): reads W once; groups
 //   that run past their first two evaluations wait in a per-warp pool in
@@ -29,7 +30,12 @@
 //   of iterations, so the iteration index and beta are warp-uniform, and the
 //   lanes of a warp stay busy: a tile only runs as long as its slowest group
 //   within one pass.
-// solve_tensor_kernel (tensor stop): runs iterations [k0, k1) of every group,
+// solve_tensor_resident_kernel (tensor stop, axis 1, W within half the L2 and
+//   the groups' state within shared memory): one cooperative launch runs every
+//   iteration; W stays in L2, the state between rounds in shared memory, and
+//   the tensor error of each iteration is reduced and the stop decided on the
+//   device (see the kernel's own comment).
+// solve_tensor_kernel (tensor stop, otherwise): runs iterations [k0, k1) of every group,
 //   stores the zero-point of each of them, accumulates the per-iteration tensor
 //   error per CTA, and the last CTA to finish (atomic ticket) sums the partials
 //   in a fixed order, applies the stop rule to the errors so far and leaves
