@@ -715,11 +715,16 @@ def run_llama70(args):
         Ws = [synth.weight_device(r, c, synth.seed_for(0, n)).cpu() for n, r, c in mats]
         n, dt, rows = oracle_70b_sample(Ws, args.ref_budget, nth)
         rate = n / dt
+        # the same oracle on one host thread, on a 32 times smaller sample (about the same seconds)
+        n1, dt1, rows1 = _oracle_fixed_rows(Ws, max(8, rows // 32), 1)
         line["cpu_baseline"] = {
             "value": rate / 1e9, "unit": UNIT, "cores": nth, "kind": "oracle",
             "sample": f"first {rows} rows of each of layer 0's 7 matrices at both settings, {n / 1e6:.1f} M "
                       f"weight-solves, fp16, OpenMP over groups",
-            "extrapolated_model_s": w_layer * total_layers * len(SETTINGS70B) / rate}
+            "extrapolated_model_s": w_layer * total_layers * len(SETTINGS70B) / rate,
+            "single_thread": {"value": n1 / dt1 / 1e9, "cores": 1,
+                              "sample": f"first {rows1} rows of each of layer 0's 7 matrices at both settings, "
+                                        f"{n1 / 1e6:.2f} M weight-solves"}}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
