@@ -70,8 +70,8 @@ GEMM_TRAFFIC = {"src_sha256": "6047c8fb4337f86155429e2a54e5e1946effb14b71f0514dd
 # to the algorithmic bytes of the captured calls (ncu, one call per setting on
 # the gate shape 28672x8192; see profiles/), valid while the kernel sources
 # hash to the captured ones.
-TRAFFIC70 = {"src_sha256": "c605bf6a126d5cd41ac5be48777e4723afdb29b4b59adade8d184376fdfc2f8f",
-             "bytes_per_alg_byte": {(2, 16): 623.33 / 572.52, (4, 128): 579.18 / 592.68},
+TRAFFIC70 = {"src_sha256": "f5aadf1fc1af577e001a946de7f45320460cfe58a6237f887b62898f050c85aa",
+             "bytes_per_alg_byte": {(2, 16): 623.31 / 572.52, (4, 128): 579.74 / 592.68},
              "summary": "profiles/solve_group_onepass_kernel_28672x8192_b2g16.md, ..._b4g128.md"}
 
 
