@@ -51,18 +51,19 @@ MUFU_PER_CLK_PER_SM = 16
 KERNEL_SOURCES = ["calibration_free_weight_b200/csrc/hqq_kernels.cu", "calibration_free_weight_b200/csrc/hqq_device.cuh"]
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
 # kernel family per hqq_quantize call (its chunk launches and its output
-# launch), averaged over the timed step's tensor-stop calls,
-# from the ncu launch list summarised in profiles/ (taken on the kernel sources
-# whose sha256 is recorded here; None until a capture exists).
-TRAFFIC = {"src_sha256": "2a27860d0d38b7224791bf0cb5d250c7aed7d1f9553c0ac9e65c4dc2b05037f5",
-           "bytes_per_call": 381103462, "summary": "profiles/launches_llama2-7b-mlp-sweep.md"}
+# launch), averaged over the sweep's tensor-stop calls: one call per setting
+# on the gate shape captured launch by launch (ncu, two DRAM metrics), the
+# mean of the five (every setting has three calls of the same size); valid
+# while the kernel sources hash to the captured ones.
+TRAFFIC = {"src_sha256": "f5aadf1fc1af577e001a946de7f45320460cfe58a6237f887b62898f050c85aa",
+           "bytes_per_call": 390389000, "summary": "profiles/solve_tensor_kernel_11008x4096_b4g64.md"}
 
 
 # DRAM traffic of one hqq_gemm call in the profiled case (ncu, same command as
 # the summary), valid while hqq_gemm.cu hashes to the profiled source.
 GEMM_SOURCES = ["calibration_free_weight_b200/csrc/hqq_gemm.cu"]
-GEMM_TRAFFIC = {"src_sha256": "6047c8fb4337f86155429e2a54e5e1946effb14b71f0514dd011fdf3db4ae611",
-                "case": "gemm,28672,8192,4,64,256", "bytes_per_call": 141282304,
+GEMM_TRAFFIC = {"src_sha256": "9ad1e18a87f9cdd83180be975fcb89b1f8c7da0978ccec10b870f0a5289f7093",
+                "case": "gemm,28672,8192,4,64,256", "bytes_per_call": 145337088,
                 "summary": "profiles/gemm_kernel_28672x8192_b4g64_batch256.md"}
 
 
