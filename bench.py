@@ -55,8 +55,8 @@ KERNEL_SOURCES = ["calibration_free_weight_b200/csrc/hqq_kernels.cu", "calibrati
 # on the gate shape captured launch by launch (ncu, two DRAM metrics), the
 # mean of the five (every setting has three calls of the same size); valid
 # while the kernel sources hash to the captured ones.
-TRAFFIC = {"src_sha256": "f5aadf1fc1af577e001a946de7f45320460cfe58a6237f887b62898f050c85aa",
-           "bytes_per_call": 390389000, "summary": "profiles/solve_tensor_kernel_11008x4096_b4g64.md"}
+TRAFFIC = {"src_sha256": "0c7c40747e8a1b6988d047afac0ab5f97f721b67ebefdc0dfa0e3c7c0079741d",
+           "bytes_per_call": 390480000, "summary": "profiles/solve_tensor_kernel_11008x4096_b4g64.md"}
 
 
 # DRAM traffic of one hqq_gemm call in the profiled case (ncu, same command as
@@ -71,8 +71,8 @@ GEMM_TRAFFIC = {"src_sha256": "9ad1e18a87f9cdd83180be975fcb89b1f8c7da0978ccec10b
 # to the algorithmic bytes of the captured calls (ncu, one call per setting on
 # the gate shape 28672x8192; see profiles/), valid while the kernel sources
 # hash to the captured ones.
-TRAFFIC70 = {"src_sha256": "f5aadf1fc1af577e001a946de7f45320460cfe58a6237f887b62898f050c85aa",
-             "bytes_per_alg_byte": {(2, 16): 623.31 / 572.52, (4, 128): 579.74 / 592.68},
+TRAFFIC70 = {"src_sha256": "0c7c40747e8a1b6988d047afac0ab5f97f721b67ebefdc0dfa0e3c7c0079741d",
+             "bytes_per_alg_byte": {(2, 16): 625.87 / 572.52, (4, 128): 579.53 / 592.68},
              "summary": "profiles/solve_group_onepass_kernel_28672x8192_b2g16.md, ..._b4g128.md"}
 
 
