@@ -82,7 +82,7 @@ def test_fast_path_gate(orc, nbits, p):
             for beta in betas[::3]:
                 thr = np.float64(beta) ** (-1.0 / (2.0 - p))
                 # the kernel's threshold is a hardware approximation: a relative
-                # error of 1e-5 either way must not change the verdict
+                # error of 1e-5 either way must not change the decision
                 for t in (thr * (1 - 1e-5), thr * (1 + 1e-5)):
                     if bound >= 0.99 * t * s:
                         continue  # gate open: the full proximal step runs
@@ -91,7 +91,7 @@ def test_fast_path_gate(orc, nbits, p):
                     for x in d:
                         n_checked += 1
                         assert orc.shrink(float(x), p, float(beta)) == 0.0, (nbits, p, float(x), float(beta))
-    # some closed verdicts sit within 10 % of the gate's edge
+    # some closed decisions sit within 10 % of the gate's edge
     assert n_closed > 0 and n_checked > 0 and n_near > 0, (n_closed, n_near)
 
 
