@@ -178,6 +178,25 @@ def test_constant_and_zero_groups(hq):
     _run(hq, W, _params(2, 16, zb=8))
 
 
+@pytest.mark.parametrize("p,beta,kappa,nbits,g", [(1.9, 20.0, 1.0, 2, 128), (1.0, 20.0, 1.05, 2, 64)])
+@pytest.mark.parametrize("mode", [2, 0])
+def test_long_runs(hq, p, beta, kappa, nbits, g, mode):
+    """Tensor errors that keep falling for hundreds of iterations (p near 2 or
+    1, a large beta; the oracle keeps iterates 543 and 321 of 1000): the
+    resident launch's rounds wrap its decision ring, its zero-point ring and
+    its arrival counters many times, and the chunked launches (mode 0) run
+    over a hundred chunks against their fixed error history; outputs against
+    the oracle."""
+    W = synth.weight(256, 1024, seed=17, dtype=torch.float16)
+    prev = hq.hqq_set_tensor_resident(mode)
+    try:
+        assert _resident(hq, W, g, iters=1000) == (mode == 2)
+        rep, gpu, orc = _run(hq, W, _params(nbits, g, p=p, beta=beta, kappa=kappa, iters=1000))
+    finally:
+        hq.hqq_set_tensor_resident(prev)
+    assert int(orc["best_iter"][0]) > 300
+
+
 def test_llama2_7b_attention_b4_g64(hq):
     """The Llama-2-7B attention shape (4096x4096, fp16, seed 0) with tensor
     stop: every group against the full oracle, and the launch without debug
