@@ -30,7 +30,7 @@ def _params(nbits, g, axis=1, p=0.7, beta=1.0, kappa=1.01, iters=20, stop=0, zb=
                 zero_nbits=zb)
 
 
-def _run(hq, W_cpu, prm, check_recon=True):
+def _run(hq, W_cpu, prm, check_recon=True, tie_cap=None):
     W = W_cpu.cuda()
     out = hq.quantize(W, prm["nbits"], prm["group_size"], prm["axis"], prm["p"], prm["beta"], prm["kappa"],
                       prm["iters"], prm["stop_mode"], prm["zero_nbits"], debug=True)
@@ -41,7 +41,7 @@ def _run(hq, W_cpu, prm, check_recon=True):
     Wo, dt = pc.w_for_oracle(W_cpu)
     orc = oracle.quantize(Wo, prm["nbits"], prm["group_size"], prm["axis"], prm["p"], prm["beta"], prm["kappa"],
                           prm["iters"], prm["stop_mode"], prm["zero_nbits"], dtype=dt)
-    rep = pc.check(W_cpu, prm, gpu, orc)
+    rep = pc.check(W_cpu, prm, gpu, orc, tie_cap=tie_cap)
     if prm["zero_nbits"] == 8:
         pc.check_zero8(gpu, orc)
     if check_recon:
@@ -86,6 +86,26 @@ def test_axis0(hq, rows, cols, g, nbits):
 def test_iteration_counts_and_modes(hq, iters, stop):
     W = synth.weight(300, 512, seed=iters * 3 + stop, dtype=torch.float16)
     _run(hq, W, _params(2, 32, iters=iters, stop=stop))
+
+
+@pytest.mark.parametrize("nbits,g,stop", [(2, 128, 0), (2, 16, 0), (4, 32, 0), (2, 128, 2)])
+def test_long_group_runs(hq, nbits, g, stop):
+    """Groups that keep improving for hundreds of iterations (p = 1.9, beta 20,
+    no annealing; on the oracle the kept iterates average 116, 74 and 63 at
+    g128, g16 and g32, up to 543): the one-pass solver's groups pass through
+    many survivor rounds of its shared-memory pool; group stop and no stop,
+    1000 iterations, against the oracle.  Here a group's error flattens for
+    hundreds of iterations, so successive errors differ by less than the tie
+    margin (reading T1: the hardware lg2/ex2 and the summation order move a
+    sum by up to ~5e-6 relative) and nearly every group's stop is a near tie
+    (2,007 of 2,048 at g128): the cap of 1e-4 of the groups, made for the
+    benchmark's regime, is lifted, and every group whose kept iterate differs
+    must still be explained by near ties on the oracle's own trajectory and
+    match the oracle's iterate at the GPU's index (zero and codes), which is
+    what a corrupted pool record would fail."""
+    W = synth.weight(256, 1024, seed=17, dtype=torch.float16)
+    _run(hq, W, _params(nbits, g, p=1.9, beta=20.0, kappa=1.0, iters=1000, stop=stop), check_recon=False,
+         tie_cap=256 * 1024 // g)
 
 
 @pytest.mark.parametrize("p,beta,kappa", [(0.5, 1.0, 1.01), (1.2, 1.0, 1.01), (0.7, 10.0, 1.05), (0.7, 1.0, 1.0)])
