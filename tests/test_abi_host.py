@@ -341,3 +341,19 @@ def test_tensor_resident_switch_and_query(hq):
     assert hq.lib.hqq_quantize_wait_selftest(C.cast(buf, C.c_void_p), 512, 0, None) == hq.HQQ_ERR_INVALID_ARG
     assert hq.lib.hqq_quantize_wait_selftest(C.cast(buf, C.c_void_p), 512, 1000001, None) == hq.HQQ_ERR_INVALID_ARG
     assert hq.lib.hqq_quantize_wait_selftest(C.cast(buf, C.c_void_p), 512, 1000, None) == hq.HQQ_ERR_INVALID_ARG
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/hqq.h is a C header: a C99 translation unit that includes it and
+    names every declared entry point compiles with -pedantic -Werror."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    header = open(os.path.join(root, "include", "hqq.h")).read()
+    names = sorted(set(re.findall(r"^(?:int|size_t|int64_t|const char\*)\s+(hqq_\w+)\(", header, re.M)))
+    assert len(names) >= 20
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "hqq.h"\nint hqq_header_declares = (int)(' + " + ".join(f"sizeof(&{n})" for n in names)
+                   + ");\n")
+    r = subprocess.run(["gcc", "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                        "-I", os.path.join(root, "include"), "-c", str(src), "-o", str(tmp_path / "u.o")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
